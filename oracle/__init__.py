@@ -1,0 +1,148 @@
+"""fp64 CPU oracle of the Mamba-2 SSD layer core (TEST INFRASTRUCTURE ONLY).
+
+Only the tests, the package smoke check and the benchmark's CPU-baseline /
+reference legs may import this package.  The product path (the CUDA library
+and its Python binding) never does.
+
+The arithmetic lives in ``ssd_oracle.c`` (plain C, double precision, the
+token-by-token recurrence); this file compiles it with gcc on first use and
+passes numpy float64 arrays to it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssd_oracle.c")
+_LIB = os.path.join(_HERE, "libssd_oracle.so")
+_lib = None
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_long), ("seqlen", ctypes.c_long), ("nheads", ctypes.c_int),
+                ("headdim", ctypes.c_int), ("d_state", ctypes.c_int), ("ngroups", ctypes.c_int)]
+
+
+def build(force: bool = False) -> str:
+    """Compile ssd_oracle.c into libssd_oracle.so next to it (plain gcc -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-shared", "-fPIC", "-pthread", "-o", tmp, _SRC,
+                               "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(lib):
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_conv_silu.argtypes = [ctypes.c_long, dp, ctypes.c_long, dp, dp, ctypes.c_double, dp]
+    lib.oracle_prefill.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 12 + [ctypes.c_void_p] + [dp] * 3 + [
+        ctypes.c_int]
+    lib.oracle_decode_step.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 12 + [ctypes.c_void_p, dp]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def use_library(path: str | None):
+    """Point the wrappers at another compiled copy of ssd_oracle.c (None = the
+    default one).  Used by the test that plants mistakes in the oracle to check
+    that its pins catch them."""
+    global _lib
+    _lib = None if path is None else _bind(ctypes.CDLL(path))
+
+
+def _f64(a):
+    """Widen an array (numpy or torch, any float dtype) to a contiguous float64 numpy array (exact)."""
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _dims(batch, seqlen, nheads, headdim, d_state, ngroups):
+    return _Dims(int(batch), int(seqlen), int(nheads), int(headdim), int(d_state), int(ngroups))
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def conv_silu(seq, hist, w, b):
+    """silu(b + sum_k w[k] * seq[t-3+k]) for one channel; hist = tokens -3..-1 or None."""
+    seq = _f64(seq)
+    hist = _f64(hist)
+    w = _f64(w)
+    out = np.empty(seq.shape[0], dtype=np.float64)
+    _load().oracle_conv_silu(seq.shape[0], _ptr(seq), 1, _ptr(hist), _ptr(w), float(b), _ptr(out))
+    return out
+
+
+def prefill(inp: dict, unit_mask=None, nthreads: int | None = None):
+    """Token-by-token fp64 prefill.  ``inp`` holds x, dt, B, C, z, A, D, dt_bias,
+    conv_w, conv_b, init_state (or None), init_conv_state (or None) with the
+    layouts x/z [Bt, L, H*P], dt [Bt, L, H], B/C [Bt, L, G, N].
+
+    ``unit_mask`` (bool [Bt, H]) restricts the work to some (b, h) pairs; the
+    other entries of y and final_state come back as NaN.
+    Returns (y [Bt, L, H*P], final_state [Bt, H, P, N], conv_state [Bt, conv_dim, 3]).
+    """
+    x = _f64(inp["x"])
+    Bt, L, HP = x.shape
+    Bm = _f64(inp["B"])
+    G, N = Bm.shape[2], Bm.shape[3]
+    H = inp["A"].shape[0]
+    P = HP // H
+    d = _dims(Bt, L, H, P, N, G)
+    arrs = [x, _f64(inp["dt"]), Bm, _f64(inp["C"]), _f64(inp["z"]), _f64(inp["A"]), _f64(inp["D"]),
+            _f64(inp["dt_bias"]), _f64(inp["conv_w"]), _f64(inp["conv_b"]), _f64(inp.get("init_state")),
+            _f64(inp.get("init_conv_state"))]
+    mask = None
+    if unit_mask is not None:
+        mask = np.ascontiguousarray(np.asarray(unit_mask, dtype=np.uint8).reshape(Bt * H))
+    y = np.full((Bt, L, HP), np.nan)
+    fs = np.full((Bt, H, P, N), np.nan)
+    cs = np.empty((Bt, HP + 2 * G * N, 3))
+    _load().oracle_prefill(ctypes.byref(d), *[_ptr(a) for a in arrs],
+                           None if mask is None else mask.ctypes.data_as(ctypes.c_void_p),
+                           _ptr(y), _ptr(fs), _ptr(cs), int(nthreads or default_threads()))
+    return y, fs, cs
+
+
+def decode_step(step: dict, params: dict, conv_state, ssm_state, unit_mask=None):
+    """One fp64 decode step.  ``conv_state`` and ``ssm_state`` must be float64
+    numpy arrays; they are updated in place.  Returns y [Bt, H*P]."""
+    assert conv_state.dtype == np.float64 and conv_state.flags.c_contiguous
+    assert ssm_state.dtype == np.float64 and ssm_state.flags.c_contiguous
+    x = _f64(step["x"])
+    Bt, HP = x.shape
+    Bm = _f64(step["B"])
+    G, N = Bm.shape[1], Bm.shape[2]
+    H = params["A"].shape[0]
+    P = HP // H
+    d = _dims(Bt, 1, H, P, N, G)
+    arrs = [x, _f64(step["dt"]), Bm, _f64(step["C"]), _f64(step["z"]), _f64(params["A"]), _f64(params["D"]),
+            _f64(params["dt_bias"]), _f64(params["conv_w"]), _f64(params["conv_b"]), conv_state, ssm_state]
+    mask = None
+    if unit_mask is not None:
+        mask = np.ascontiguousarray(np.asarray(unit_mask, dtype=np.uint8).reshape(Bt * H))
+    y = np.full((Bt, HP), np.nan)
+    _load().oracle_decode_step(ctypes.byref(d), *[_ptr(a) for a in arrs],
+                               None if mask is None else mask.ctypes.data_as(ctypes.c_void_p), _ptr(y))
+    return y

@@ -1,0 +1,87 @@
+"""The oracle's pins are strong enough: each plausible mistake planted in a copy
+of the oracle's C source (a dropped term, a wrong sign or index, swapped
+operands) makes at least one pin fail.  CPU only; the mistakes are planted in
+temporary copies, never in the committed oracle.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ssd_oracle.c")
+
+MUTANTS = {
+    "transition sign": ("const double a = exp(dt * j->A[h]);", "const double a = exp(-dt * j->A[h]);"),
+    "dropped D skip": ("const double yv = acc + j->D[h] * xt[p];", "const double yv = acc;"),
+    "reversed conv taps": ("acc += w[k] * v;", "acc += w[3 - k] * v;"),
+    "reversed conv history": ("else v = hist ? hist[s + 3] : 0.0;", "else v = hist ? hist[-s - 1] : 0.0;"),
+    "wrong head->group map": ("const int g = h / (H / G);\n    const long cx",
+                              "const int g = h % G;\n    const long cx"),
+    "B and C swapped": ("Sp[n] = a * Sp[n] + dt * xt[p] * Bt[n];\n                acc += Sp[n] * Ct[n];",
+                        "Sp[n] = a * Sp[n] + dt * xt[p] * Ct[n];\n                acc += Sp[n] * Bt[n];"),
+    "read-out before update": ("Sp[n] = a * Sp[n] + dt * xt[p] * Bt[n];\n                acc += Sp[n] * Ct[n];",
+                               "acc += Sp[n] * Ct[n];\n                Sp[n] = a * Sp[n] + dt * xt[p] * Bt[n];"),
+    "missing dt bias": ("j->dt_raw[((size_t)b * L + t) * H + h] + j->dt_bias[h]",
+                        "j->dt_raw[((size_t)b * L + t) * H + h]"),
+    "input not scaled by dt": ("Sp[n] = a * Sp[n] + dt * xt[p] * Bt[n];", "Sp[n] = a * Sp[n] + xt[p] * Bt[n];"),
+    "ungated output": ("= yv * o_silu(zv);", "= yv * zv;"),
+    "conv bias dropped": ("double acc = b;", "double acc = 0.0;"),
+    "decode roll stale": ("cs[0] = win[1];", "cs[0] = win[0];"),
+    "decode missing D": ("const double yv = acc + D[h] * xt[p];", "const double yv = acc;"),
+    "decode wrong B group": ("const double* Bt = u + HP + (size_t)g * N;", "const double* Bt = u + HP;"),
+    "softplus branch wrong": ("if (v > 30.0) return v + log1p(exp(-v));", "if (v > 0.0) return v;"),
+}
+
+PINS = [
+    lambda: pins.test_conv_silu_matches_library_fir(True),
+    lambda: pins.test_prefill_matches_quadratic_form(1, True),
+    lambda: pins.test_prefill_quadratic_form_bf16_inputs_groups_of_three(),
+    lambda: pins.test_closed_form_constant_inputs(-1.2, -2.5),
+    lambda: pins.test_closed_form_constant_inputs(0.8, -0.6),
+    lambda: pins.test_closed_form_constant_inputs(35.0, -0.01),
+    lambda: pins.test_decode_steps_reproduce_prefill(True),
+]
+
+
+def _compile(src_text, out_dir, name):
+    c = os.path.join(out_dir, name + ".c")
+    so = os.path.join(out_dir, name + ".so")
+    with open(c, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["gcc", "-O1", "-shared", "-fPIC", "-pthread", "-o", so, c, "-lm"])
+    return so
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    src = open(SRC).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for '{name}' not unique"
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _compile(src.replace(old, new), tmp, "mutant")
+        oracle.use_library(so)
+        try:
+            failed = 0
+            for pin in PINS:
+                try:
+                    pin()
+                except AssertionError:
+                    failed += 1
+            assert failed > 0, f"no pin caught the planted mistake '{name}'"
+        finally:
+            oracle.use_library(None)
+
+
+def test_unmutated_copy_passes_every_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _compile(open(SRC).read(), tmp, "clean")
+        oracle.use_library(so)
+        try:
+            for pin in PINS:
+                pin()
+        finally:
+            oracle.use_library(None)
