@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-2 SSD layer core on B200.
+
+Headline (`value`): SSD prefill throughput in tokens/s for one Mamba-2 layer
+of the Nemotron-H 8B shape (batch 1, seqlen 4096, 128 heads x 64, d_state
+128, 8 groups, chunk 128, bf16 activations, fp32 state), inputs resident in
+HBM, L2 flushed between timed steps.  Also reported on the same line:
+  decode      GB/s of one decode step for 256 sequences of the same layer
+              shape (64 consecutive steps), fraction of measured HBM peak;
+  roofline    the dominant prefill kernel's algorithmic bytes per launch over
+              its own CUDA-event duration, against measured HBM bandwidth;
+  e2e         the same prefill through the public API from pinned HOST
+              tensors, host<->device copies inside the timed region;
+  cpu_baseline the fp64 oracle timed on this host's cores on a sample of the
+              same workload;
+  clocks      SM clocks and throttle reasons sampled while timing.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU (weak scaling, no data-path collective: every rank runs its own
+sequences): python -m torch.distributed.run --nproc-per-node N bench.py --gpus N
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from selective_state_space_43_b200.synth import (Dims, WORKLOADS, make_decode_inputs,  # noqa: E402
+                                                 make_prefill_inputs, seed_of)
+
+METRIC = "SSD prefill tokens/s per layer (% bf16 TC peak); decode GB/s (% of HBM peak)"
+PREFILL_WORKLOAD = "nemotron_h_8b"
+DECODE_WORKLOAD = "decode_nemotron_h_8b"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------------------------------------
+# algorithmic work (what the layer must read, write and compute, independent of the implementation)
+
+def prefill_bytes(d: Dims, act_bytes: int, init_state: bool) -> int:
+    tok = d.batch * d.seqlen
+    inputs = tok * (2 * d.d_inner + d.nheads + 2 * d.ngroups * d.d_state) * act_bytes   # x, z, dt, B, C
+    out = tok * d.d_inner * act_bytes                                                 # y
+    state = d.batch * d.nheads * d.headdim * d.d_state * 4 * (2 if init_state else 1)
+    conv = d.batch * d.conv_dim * 3 * act_bytes
+    return inputs + out + state + conv
+
+
+def prefill_flops(d: Dims) -> int:
+    # per token: C.B^T once per group (2QN per group), then per head the masked
+    # Q x Q times X (2QP), the chunk state B^T X (2NP) and C times the state (2NP)
+    per_tok = 2 * d.chunk * d.d_state * d.ngroups + d.nheads * (2 * d.chunk * d.headdim + 4 * d.d_state * d.headdim)
+    return d.batch * d.seqlen * per_tok
+
+
+def decode_bytes(d: Dims, act_bytes: int) -> tuple[int, int]:
+    """(bytes of the whole step, bytes of the state-stream kernel alone)."""
+    B = d.batch
+    state = 2 * B * d.nheads * d.headdim * d.d_state * 4
+    conv = 2 * B * d.conv_dim * 3 * act_bytes
+    inputs = B * (2 * d.d_inner + d.nheads + 2 * d.ngroups * d.d_state) * act_bytes
+    y = B * d.d_inner * act_bytes
+    roll = B * 2 * d.ngroups * d.d_state * (3 + 3) * act_bytes     # B/C conv window rewritten by the roll kernel
+    total = state + conv + inputs + y
+    return total, total - roll
+
+
+# ---------------------------------------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None if
+    the summary is missing or the kernel's source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        t = json.load(f).get(kernel)
+    if not t:
+        return None
+    src = os.path.join(ROOT, t["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != t["source_sha256_16"]:
+        return None
+    return t["dram_bytes_per_launch"]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event (throttle) reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
+        self._load = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.ok = True
+        except Exception as e:  # no NVML: report that, never guess
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            if self._load.is_set():
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self._reasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def load(self, on: bool):
+        (self._load.set if on else self._load.clear)()
+
+    def stop(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "error": self.err}
+        self._stop.set()
+        self.t.join()
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = sorted(name for b, name in self.REASONS.items() if bits & b)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "source": "NVML, sampled every 5 ms during the timed regions"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------------------------
+# CPU oracle baseline
+
+def oracle_inputs_f64(inp):
+    return {k: (None if v is None else np.ascontiguousarray(v.double().numpy())) for k, v in inp.items()}
+
+
+def oracle_sample(inp64, d: Dims, first_unit: int, n_units: int, threads: int):
+    """Run the oracle on n_units (b, h) pairs starting at first_unit; returns seconds."""
+    import oracle
+    mask = np.zeros(d.batch * d.nheads, dtype=bool)
+    idx = [(first_unit + i) % (d.batch * d.nheads) for i in range(n_units)]
+    mask[idx] = True
+    t0 = time.perf_counter()
+    oracle.prefill(inp64, unit_mask=mask.reshape(d.batch, d.nheads), nthreads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(inp, d: Dims, budget_s: float):
+    import oracle
+    threads = oracle.default_threads()
+    inp64 = oracle_inputs_f64(inp)
+    done, elapsed, u = 0, 0.0, 0
+    while elapsed < budget_s and done < d.batch * d.nheads:
+        n = min(threads, d.batch * d.nheads - done)
+        elapsed += oracle_sample(inp64, d, u, n, threads)
+        done += n
+        u += n
+    tokens_equiv = done * d.seqlen / d.nheads      # each (b, h) pair is one head's share of L tokens
+    return {"value": tokens_equiv / elapsed, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of the {d.batch * d.nheads} (sequence, head) pairs of the {PREFILL_WORKLOAD} "
+                      f"workload ({d.seqlen} tokens each), fp64 token-by-token recurrence, {elapsed:.1f} s; "
+                      f"tokens/s = pairs x L / H / seconds"}
+
+
+# ---------------------------------------------------------------------------------------------------------
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle as it stands, on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = WORKLOADS[PREFILL_WORKLOAD]
+    d = w["dims"]
+    inp = make_prefill_inputs(d, dtype=w["dtype"], seed=seed_of(PREFILL_WORKLOAD), init_state=w["init_state"])
+    inp64 = oracle_inputs_f64(inp)
+    threads = oracle.default_threads()
+    n = threads
+    for i in range(args.warmup):
+        oracle_sample(inp64, d, i * n, n, threads)
+    times = [oracle_sample(inp64, d, (args.warmup + k) * n, n, threads) for k in range(args.steps)]
+    sec = sum(times) / len(times)
+    value = n * d.seqlen / d.nheads / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w["desc"], "sample_per_step": f"{n} (sequence, head) pairs of {d.seqlen} tokens"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} (sequence, head) pairs per step, {args.steps} steps"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from selective_state_space_43_b200 import ops
+    ops.lib()   # fail loudly here if the CUDA library is missing
+
+    peaks, peak_src = load_peaks()
+    w = WORKLOADS[PREFILL_WORKLOAD]
+    d = w["dims"]
+    act = w["dtype"]
+    inp = make_prefill_inputs(d, dtype=act, seed=seed_of(PREFILL_WORKLOAD) + 1000 * rank, init_state=w["init_state"])
+    g = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    dims = ops.make_dims(d.batch, d.seqlen, d.nheads, d.headdim, d.d_state, d.ngroups, d.chunk)
+    path = ops.prefill_path(dims, act)
+    ws_bytes = ops.prefill_workspace_bytes(dims, act)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    y = torch.empty_like(g["x"])
+    fs = torch.empty((d.batch, d.nheads, d.headdim, d.d_state), dtype=torch.float32, device=dev)
+    cs = torch.empty((d.batch, d.conv_dim, 3), dtype=act, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def prefill_once():
+        ops.prefill(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], g["conv_w"], g["conv_b"],
+                    g["init_state"], None, chunk=d.chunk, workspace=ws, y=y, final_state=fs, conv_state=cs)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+
+    # ---- prefill, device-resident inputs --------------------------------------------------------------
+    for _ in range(args.warmup):
+        flush.zero_()
+        prefill_once()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.load(True)
+    for k in range(K):
+        flush.zero_()                      # L2 flush, outside the step's events
+        ops.set_timing_events(ks[k], ke[k])
+        st[k].record()
+        prefill_once()
+        en[k].record()
+    torch.cuda.synchronize(dev)
+    sampler.load(False)
+    barrier(world)
+    ops.set_timing_events(None, None)
+    step_ms = sum(s.elapsed_time(e) for s, e in zip(st, en)) / K
+    kern_ms = sum(s.elapsed_time(e) for s, e in zip(ks, ke)) / K
+    step_ms_max = max_over_ranks(step_ms, world, dev)
+    tokens_per_rank = d.batch * d.seqlen
+    value = tokens_per_rank * world / (step_ms_max * 1e-3)
+
+    act_bytes = 2 if act == torch.bfloat16 else 4
+    pbytes = prefill_bytes(d, act_bytes, w["init_state"])
+    pflops = prefill_flops(d)
+    kernel_name = "ssd_chunk_scan_tc" if path == 1 else "prefill_simt_kernel"
+    kernel_src = ("selective_state_space_43_b200/csrc/ssd_prefill_tc.cu" if path == 1 else
+                  "selective_state_space_43_b200/csrc/ssd_prefill_simt.cu")
+    achieved_gbs = pbytes / (kern_ms * 1e-3) / 1e9
+    traffic = kernel_traffic(kernel_name)
+    roofline = {"bound": "hbm", "kernel": kernel_name, "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                "algorithmic_bytes_per_launch": pbytes, "kernel_ms": kern_ms,
+                "peak_source": f"{peak_src} (copy bandwidth)"}
+    tflops = pflops / (step_ms * 1e-3) / 1e12
+    tc = {"algorithmic_tflops": tflops, "frac_bf16_peak": tflops / peaks["bf16_tflops"],
+          "frac_bf16_sustained": tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+          "algorithmic_flops_per_step": pflops, "peak_source": peak_src}
+
+    # ---- e2e through the public API from pinned host memory ------------------------------------------------
+    e2e = None
+    if not args.no_e2e:
+        host = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
+        for _ in range(3):
+            ops.prefill_host(host, chunk=d.chunk, device=dev)
+        torch.cuda.synchronize(dev)
+        KE = max(3, min(K, 20))
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+        barrier(world)
+        sampler.load(True)
+        for k in range(KE):
+            es[k].record()
+            _, h2d, d2h = ops.prefill_host(host, chunk=d.chunk, device=dev)
+            ee[k].record()
+        torch.cuda.synchronize(dev)
+        sampler.load(False)
+        barrier(world)
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(es, ee)) / KE, world, dev)
+        e2e = {"value": tokens_per_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": KE,
+               "how": "ops.prefill_host: pinned host inputs -> device, ssd_prefill, outputs -> pinned host; "
+                      "CUDA events on the stream around all three"}
+        del host
+
+    # ---- decode -------------------------------------------------------------------------------------------
+    decode = None
+    if not args.no_decode:
+        del g, y, ws
+        wd = WORKLOADS[DECODE_WORKLOAD]
+        dd = wd["dims"]
+        data = make_decode_inputs(dd, steps=args.decode_steps, dtype=wd["dtype"], seed=seed_of(DECODE_WORKLOAD))
+        p = {k: v.to(dev) for k, v in data["params"].items()}
+        conv = data["conv_state"].to(dev)
+        ssm = data["ssm_state"].to(dev)
+        steps = [{k: v.to(dev) for k, v in s.items()} for s in data["steps"]]
+        del data
+
+        def dstep(s):
+            ops.decode_step(s["x"], s["dt"], s["B"], s["C"], s["z"], p["A"], p["D"], p["dt_bias"], p["conv_w"],
+                            p["conv_b"], conv, ssm)
+        for i in range(3):
+            dstep(steps[i % len(steps)])
+        torch.cuda.synchronize(dev)
+        KD = len(steps)
+        ds = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+        de = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+        dks = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+        dke = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+        barrier(world)
+        sampler.load(True)
+        for k in range(KD):
+            ops.set_timing_events(dks[k], dke[k])
+            ds[k].record()
+            dstep(steps[k])
+            de[k].record()
+        torch.cuda.synchronize(dev)
+        sampler.load(False)
+        barrier(world)
+        ops.set_timing_events(None, None)
+        dms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(ds, de)) / KD, world, dev)
+        dkms = sum(a.elapsed_time(b) for a, b in zip(dks, dke)) / KD
+        tot_b, kern_b = decode_bytes(dd, 2 if wd["dtype"] == torch.bfloat16 else 4)
+        gbs = tot_b * world / (dms * 1e-3) / 1e9
+        kgbs = kern_b / (dkms * 1e-3) / 1e9
+        decode = {"value": gbs, "unit": "GB/s", "ms_per_step": dms, "steps": KD, "workload": wd["desc"],
+                  "frac_hbm_peak": gbs / world / peaks["hbm_gbs"], "frac_8tbs_spec": gbs / world / 8000.0,
+                  "algorithmic_bytes_per_step": tot_b,
+                  "roofline": {"bound": "hbm", "kernel": "decode_state_kernel", "achieved": kgbs,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kgbs / peaks["hbm_gbs"],
+                               "traffic": kernel_traffic("decode_state_kernel"),
+                               "algorithmic_bytes_per_launch": kern_b, "kernel_ms": dkms},
+                  "l2": "state (1.07 GB) larger than L2; no flush"}
+
+    clocks = sampler.stop()
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(inp, d, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if act == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded recipe: x,z,dt~N(0,1), B,C~N(0,1)/sqrt(N), A=-exp(U[0,ln16]))",
+            "config": {"workload": w["desc"], "batch_per_gpu": d.batch, "seqlen": d.seqlen, "nheads": d.nheads,
+                       "headdim": d.headdim, "d_state": d.d_state, "ngroups": d.ngroups, "chunk": d.chunk,
+                       "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+                       "l2": "flushed between timed steps (256 MB write outside the step events)",
+                       "kernel_path": "tcgen05 tensor-core" if path == 1 else "CUDA-core"},
+            "tensor": tc, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+            "gpu_launches": K * (2 if path == 1 else 1), "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

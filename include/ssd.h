@@ -1,0 +1,165 @@
+/*
+ * ssd.h -- C ABI of the B200 (sm_100a) Mamba-2 selective-SSM layer core.
+ *
+ * Two operations, both from the Mamba-2 layer used by the hybrid models on
+ * the pages ("Nemotron-H 스타일 Hybrid Mamba-Transformer 3B 모델 구현 타당성
+ * 분석", §1.4 Mamba-2 구성 and §3.2 접근법 A):
+ *
+ *   ssd_prefill      the chunked state-space-duality (SSD) scan over a whole
+ *                    sequence ("EP6. 트랜스포머 대체 신경망 연구" §7, §8:
+ *                    Mamba-2's SSD is exactly a masked, attention-like form);
+ *   ssd_decode_step  one token of the recurrence for a batch of sequences,
+ *                    streaming the fixed-size state once ("Mamba-3: 추론을
+ *                    우선한 상태 공간 모델", opening section: with a scalar
+ *                    transition the decode step is memory-bandwidth bound).
+ *
+ * Per token t, head h (group g = h / (H/G)), with u = SiLU(causal conv4(.)+b)
+ * applied to the channels [x | B | C]:
+ *     dt  = softplus(dt_raw[t,h] + dt_bias[h])
+ *     S_h = exp(dt * A[h]) * S_h + dt * u_x[t,h,:] (outer) u_B[t,g,:]   (P x N)
+ *     y   = (S_h . u_C[t,g,:] + D[h] * u_x[t,h,:]) * SiLU(z[t,h,:])
+ *
+ * Conventions shared by every entry point
+ *  - Pointers: all tensor pointers are DEVICE pointers, row-major and
+ *    contiguous, owned by the caller.  The library allocates no memory and
+ *    keeps no pointer after it returns.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  Calls are asynchronous: a returned SSD_OK means the
+ *    work was enqueued; faults during execution surface on the stream.
+ *  - Validation happens before any launch; a failing check returns its status
+ *    and writes nothing.
+ *  - Activation dtype (`dtype`): applies to x, dt, B, C, z, y, conv_state and
+ *    init_conv_state (y is fp32 under SSD_BF16_YF32).  Parameters and SSM
+ *    states are always fp32.
+ *  - Shapes: headdim P = 64; d_state N in {16, 32, 64, 128}; nheads % ngroups
+ *    == 0; d_conv = 4; chunk Q in {64, 128}.  conv_dim = H*P + 2*G*N.
+ *  - Alignment: every tensor pointer 16-byte aligned.
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_NULL = 1,        /* a required pointer is NULL                              */
+    SSD_ERR_SHAPE = 2,       /* a size is out of range or inconsistent                  */
+    SSD_ERR_DTYPE = 3,       /* unknown activation dtype                                */
+    SSD_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned                        */
+    SSD_ERR_UNSUPPORTED = 5, /* valid but not implemented (e.g. aliasing outputs)      */
+    SSD_ERR_CUDA = 6,        /* a CUDA runtime call failed (launch or query)            */
+    SSD_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than ssd_prefill_workspace_bytes */
+    SSD_ERR_TIMEOUT = 8      /* a bounded device-side wait gave up                      */
+} ssd_status;
+
+/* Activation dtype.  SSD_BF16_YF32 reads bf16 activations (and keeps the conv
+ * state in bf16) but writes y in fp32: the same arithmetic as SSD_BF16, whose y
+ * is exactly the round-to-nearest-even bf16 of this fp32 y. */
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1, SSD_BF16_YF32 = 2 } ssd_dtype;
+
+typedef struct {
+    int64_t batch;   /* sequences                                       */
+    int64_t seqlen;  /* tokens per sequence (ignored by decode)          */
+    int32_t nheads;  /* H                                                */
+    int32_t headdim; /* P (must be 64)                                   */
+    int32_t d_state; /* N                                                */
+    int32_t ngroups; /* G; heads h*G/H .. share one B/C group            */
+    int32_t chunk;   /* Q, the SSD chunk length (64 or 128)              */
+    int32_t d_conv;  /* conv taps (must be 4)                            */
+} ssd_dims;
+
+/* Layer parameters, fp32 device pointers. */
+typedef struct {
+    const float* A;       /* [H]  per-head transition rate, A < 0                   */
+    const float* D;       /* [H]  skip weight                                       */
+    const float* dt_bias; /* [H]  added to dt_raw before softplus                   */
+    const float* conv_w;  /* [conv_dim][4] depthwise taps, tap 3 = current token   */
+    const float* conv_b;  /* [conv_dim]                                            */
+} ssd_params;
+
+/* Human-readable name of a status code (static storage). */
+SSD_API const char* ssd_status_string(ssd_status s);
+
+/* Library build identification (static storage). */
+SSD_API const char* ssd_version(void);
+
+/*
+ * Bytes of device workspace ssd_prefill needs for these sizes (0 if none).
+ * The workspace holds the post-conv, post-SiLU B and C channels of every
+ * token ([batch][seqlen][2][G][N] in the activation dtype) on the tensor-core
+ * path.  Returns 0 for invalid sizes.
+ */
+SSD_API size_t ssd_prefill_workspace_bytes(const ssd_dims* dims, ssd_dtype dtype);
+
+/*
+ * Which kernel path ssd_prefill takes for these sizes:
+ *   1 = tcgen05 tensor-core chunk scan (bf16 activations, P=64, Q=128, N in {64,128});
+ *   2 = CUDA-core chunk scan (every other supported shape, and fp32);
+ *  <0 = -(ssd_status) for invalid sizes.
+ */
+SSD_API int ssd_prefill_path(const ssd_dims* dims, ssd_dtype dtype);
+
+/*
+ * Chunked SSD prefill over batch x seqlen tokens.
+ *   x, z        [batch][seqlen][H*P]     dtype
+ *   dt          [batch][seqlen][H]       dtype (dt_raw, before bias and softplus)
+ *   B, C        [batch][seqlen][G][N]    dtype (pre-conv)
+ *   init_state  [batch][H][P][N] fp32, or NULL for zeros; may equal final_state
+ *   init_conv_state [batch][conv_dim][3] dtype, tokens -3..-1 of the conv
+ *               history, or NULL for zeros; must not alias conv_state
+ *   y           [batch][seqlen][H*P]     dtype, fp32 for SSD_BF16_YF32 (out);
+ *               must not alias x or z
+ *   final_state [batch][H][P][N] fp32 (out): the state after the last token
+ *   conv_state  [batch][conv_dim][3] dtype (out): pre-conv inputs of tokens
+ *               seqlen-3 .. seqlen-1 (history-filled when seqlen < 3)
+ *   workspace   device scratch of at least ssd_prefill_workspace_bytes()
+ *               bytes (may be NULL when that is 0)
+ * seqlen == 0 is valid: final_state = init_state (or zeros), conv_state =
+ * the history, y untouched.
+ */
+SSD_API ssd_status ssd_prefill(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
+                       const void* x, const void* dt, const void* B, const void* C, const void* z,
+                       const float* init_state, const void* init_conv_state,
+                       void* y, float* final_state, void* conv_state,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One decode token for each of `batch` sequences (dims->seqlen is ignored).
+ *   x, z        [batch][H*P]   dtype
+ *   dt          [batch][H]     dtype
+ *   B, C        [batch][G][N]  dtype (pre-conv)
+ *   conv_state  [batch][conv_dim][3] dtype, in/out: rolled by one token
+ *   ssm_state   [batch][H][P][N] fp32, in/out, updated in place
+ *   y           [batch][H*P]   dtype, fp32 for SSD_BF16_YF32 (out)
+ * Two launches: the state stream (all heads) and the roll of the shared B/C
+ * conv channels, which must follow every head's read of them.
+ */
+SSD_API ssd_status ssd_decode_step(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
+                           const void* x, const void* dt, const void* B, const void* C, const void* z,
+                           void* conv_state, float* ssm_state, void* y, void* stream);
+
+/*
+ * Optional timing hook for benchmarks.  When both are non-NULL, the next
+ * ssd_prefill / ssd_decode_step calls on this host thread record
+ * `before_main` (a cudaEvent_t) on their stream immediately before the
+ * dominant kernel launch and `after_main` immediately after it.  Pass NULLs
+ * to switch it off.  Thread-local; never synchronises.
+ */
+SSD_API ssd_status ssd_set_timing_events(void* before_main, void* after_main);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_H */

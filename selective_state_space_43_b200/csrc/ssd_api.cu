@@ -1,0 +1,142 @@
+// ssd_api.cu -- the extern "C" entry points declared in include/ssd.h:
+// argument validation (before any launch), kernel-path choice, launches.
+#include <stdint.h>
+
+#include "ssd.h"
+#include "ssd_common.cuh"
+#include "ssd_internal.h"
+
+namespace {
+
+thread_local ssd::TimingHook g_hook;
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ssd_status check_dims(const ssd_dims* d, ssd_dtype dtype, bool prefill) {
+    if (!d) return SSD_ERR_NULL;
+    if (dtype != SSD_F32 && dtype != SSD_BF16 && dtype != SSD_BF16_YF32) return SSD_ERR_DTYPE;
+    if (d->batch < 0 || (prefill && d->seqlen < 0)) return SSD_ERR_SHAPE;
+    if (d->nheads <= 0 || d->ngroups <= 0 || d->nheads % d->ngroups != 0) return SSD_ERR_SHAPE;
+    if (d->headdim != 64) return SSD_ERR_SHAPE;
+    if (!(d->d_state == 16 || d->d_state == 32 || d->d_state == 64 || d->d_state == 128)) return SSD_ERR_SHAPE;
+    if (d->d_conv != 4) return SSD_ERR_SHAPE;
+    if (prefill && !(d->chunk == 64 || d->chunk == 128)) return SSD_ERR_SHAPE;
+    // index arithmetic inside the kernels uses 32-bit per-token offsets
+    const int64_t conv_dim = (int64_t)d->nheads * d->headdim + 2LL * d->ngroups * d->d_state;
+    if (conv_dim > (1LL << 24)) return SSD_ERR_SHAPE;
+    if (d->batch * (int64_t)d->nheads > (1LL << 31) - 1) return SSD_ERR_SHAPE;
+    return SSD_OK;
+}
+
+ssd_status check_params(const ssd_params* p) {
+    if (!p || !p->A || !p->D || !p->dt_bias || !p->conv_w || !p->conv_b) return SSD_ERR_NULL;
+    if (!aligned16(p->A) || !aligned16(p->D) || !aligned16(p->dt_bias) || !aligned16(p->conv_w) ||
+        !aligned16(p->conv_b))
+        return SSD_ERR_ALIGN;
+    return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(ssd_status s) {
+    switch (s) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_NULL: return "a required pointer is NULL";
+        case SSD_ERR_SHAPE: return "unsupported or inconsistent sizes";
+        case SSD_ERR_DTYPE: return "unknown activation dtype";
+        case SSD_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case SSD_ERR_UNSUPPORTED: return "valid but unsupported arguments (aliasing outputs)";
+        case SSD_ERR_CUDA: return "a CUDA runtime call failed";
+        case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSD_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    }
+    return "unknown status";
+}
+
+const char* ssd_version(void) { return "ssd_b200 1.0 (sm_100a)"; }
+
+int ssd_prefill_path(const ssd_dims* d, ssd_dtype dtype) {
+    const ssd_status st = check_dims(d, dtype, true);
+    if (st != SSD_OK) return -(int)st;
+    return ssd::prefill_tc_supported(d->headdim, d->d_state, d->chunk, dtype != SSD_F32) ? 1 : 2;
+}
+
+size_t ssd_prefill_workspace_bytes(const ssd_dims* d, ssd_dtype dtype) {
+    if (ssd_prefill_path(d, dtype) != 1) return 0;
+    return ssd::prefill_tc_workspace_bytes(d->batch, d->seqlen, d->ngroups, d->d_state);
+}
+
+ssd_status ssd_prefill(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params, const void* x,
+                       const void* dt, const void* B, const void* C, const void* z, const float* init_state,
+                       const void* init_conv_state, void* y, float* final_state, void* conv_state,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    ssd_status st = check_dims(d, dtype, true);
+    if (st != SSD_OK) return st;
+    if ((st = check_params(params)) != SSD_OK) return st;
+    if (!x || !dt || !B || !C || !z || !y || !final_state || !conv_state) return SSD_ERR_NULL;
+    const void* ptrs[] = {x, dt, B, C, z, init_state, init_conv_state, y, final_state, conv_state, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return SSD_ERR_ALIGN;
+    if (y == x || y == z || (init_conv_state && init_conv_state == conv_state)) return SSD_ERR_UNSUPPORTED;
+    const int path = ssd_prefill_path(d, dtype);
+    const size_t need = path == 1 ? ssd::prefill_tc_workspace_bytes(d->batch, d->seqlen, d->ngroups, d->d_state) : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
+    if (d->batch == 0) return SSD_OK;
+
+    const ssd::Shape s = ssd::make_shape(*d);
+    ssd::PrefillArgs a;
+    a.batch = s.batch;
+    a.L = s.seqlen;
+    a.nchunks = s.nchunks;
+    a.H = s.H; a.P = s.P; a.N = s.N; a.G = s.G; a.Q = s.Q;
+    a.HP = s.HP; a.GN = s.GN; a.conv_dim = s.conv_dim; a.hpg = s.heads_per_group;
+    a.A = params->A; a.D = params->D; a.dt_bias = params->dt_bias;
+    a.conv_w = params->conv_w; a.conv_b = params->conv_b;
+    a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z;
+    a.init_state = init_state; a.init_conv_state = init_conv_state;
+    a.y = y; a.final_state = final_state; a.conv_state = conv_state;
+    a.workspace = workspace;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
+                                                                                        : ssd::ActKind::BF16_YF32);
+    cudaError_t e = path == 1 ? ssd::launch_prefill_tc(a, kind, cs, g_hook)
+                              : ssd::launch_prefill_simt(a, kind, cs, g_hook);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_decode_step(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params, const void* x,
+                           const void* dt, const void* B, const void* C, const void* z, void* conv_state,
+                           float* ssm_state, void* y, void* stream) {
+    ssd_status st = check_dims(d, dtype, false);
+    if (st != SSD_OK) return st;
+    if ((st = check_params(params)) != SSD_OK) return st;
+    if (!x || !dt || !B || !C || !z || !conv_state || !ssm_state || !y) return SSD_ERR_NULL;
+    const void* ptrs[] = {x, dt, B, C, z, conv_state, ssm_state, y};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return SSD_ERR_ALIGN;
+    if (y == x || y == z) return SSD_ERR_UNSUPPORTED;
+    if (d->batch == 0) return SSD_OK;
+    const ssd::Shape s = ssd::make_shape(*d);
+    ssd::DecodeArgs a;
+    a.H = s.H; a.P = s.P; a.N = s.N; a.G = s.G; a.HP = s.HP; a.GN = s.GN;
+    a.conv_dim = s.conv_dim; a.hpg = s.heads_per_group;
+    a.A = params->A; a.D = params->D; a.dt_bias = params->dt_bias;
+    a.conv_w = params->conv_w; a.conv_b = params->conv_b;
+    a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z;
+    a.conv_state = conv_state; a.ssm_state = ssm_state; a.y = y;
+    const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
+                                                                                        : ssd::ActKind::BF16_YF32);
+    cudaError_t e = ssd::launch_decode(a, s.batch, kind, static_cast<cudaStream_t>(stream), g_hook);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_set_timing_events(void* before_main, void* after_main) {
+    if ((before_main == nullptr) != (after_main == nullptr)) return SSD_ERR_NULL;
+    g_hook.ev_before = static_cast<cudaEvent_t>(before_main);
+    g_hook.ev_after = static_cast<cudaEvent_t>(after_main);
+    return SSD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// ssd_internal.h -- launch arguments and launcher entry points shared by the
+// C-ABI layer (ssd_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// Activation / output types: fp32 in and out; bf16 in and out; bf16 in, fp32 y.
+enum class ActKind { F32, BF16, BF16_YF32 };
+
+// Records the caller's events around the dominant kernel (benchmark hook).
+struct TimingHook {
+    cudaEvent_t ev_before = nullptr, ev_after = nullptr;
+    void before(cudaStream_t s) const {
+        if (ev_before) cudaEventRecord(ev_before, s);
+    }
+    void after(cudaStream_t s) const {
+        if (ev_after) cudaEventRecord(ev_after, s);
+    }
+};
+
+struct DecodeArgs {
+    int H, P, N, G, HP, GN, conv_dim, hpg;
+    const float *A, *D, *dt_bias, *conv_w, *conv_b;
+    const void *x, *dt, *B, *C, *z;
+    void* conv_state;
+    float* ssm_state;
+    void* y;
+};
+
+struct PrefillArgs {
+    int64_t batch, L, nchunks;
+    int H, P, N, G, Q, HP, GN, conv_dim, hpg;
+    const float *A, *D, *dt_bias, *conv_w, *conv_b;
+    const void *x, *dt, *B, *C, *z;
+    const float* init_state;
+    const void* init_conv_state;
+    void* y;
+    float* final_state;
+    void* conv_state;
+    void* workspace;  // tensor-core path: post-conv B and C, [batch*L][2][G][N] bf16
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, int64_t batch, ActKind kind, cudaStream_t st, const TimingHook& hook);
+
+// CUDA-core chunked SSD (any supported shape, fp32 or bf16 activations).
+cudaError_t launch_prefill_simt(const PrefillArgs& a, ActKind kind, cudaStream_t st, const TimingHook& hook);
+
+// tcgen05 tensor-core chunked SSD (bf16 activations, P = 64, Q = 128, N in {64, 128}).
+bool prefill_tc_supported(int P, int N, int Q, bool bf16);
+size_t prefill_tc_workspace_bytes(int64_t batch, int64_t L, int G, int N);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t st, const TimingHook& hook);
+
+}  // namespace ssd

@@ -1,0 +1,234 @@
+"""Thin ctypes binding of the C ABI in include/ssd.h.
+
+Argument marshalling only: every step of the layer runs in the CUDA library
+(libssd_b200.so).  Tensors are checked for device, dtype, shape and
+contiguity, then their data pointers and torch's current CUDA stream are
+passed through.  There is no CPU fallback: if the library is missing or the
+tensors are not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssd_b200.so")
+
+SSD_F32, SSD_BF16, SSD_BF16_YF32 = 0, 1, 2
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE", 4: "SSD_ERR_ALIGN",
+          5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_WORKSPACE", 8: "SSD_ERR_TIMEOUT"}
+
+
+class SsdDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int32),
+                ("headdim", ctypes.c_int32), ("d_state", ctypes.c_int32), ("ngroups", ctypes.c_int32),
+                ("chunk", ctypes.c_int32), ("d_conv", ctypes.c_int32)]
+
+
+class SsdParams(ctypes.Structure):
+    _fields_ = [("A", ctypes.c_void_p), ("D", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p)]
+
+
+class SsdError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({lib().ssd_status_string(status).decode()})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; "
+                               "g.build()'` (needs nvcc); there is no CPU fallback")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        dimp, parp = ctypes.POINTER(SsdDims), ctypes.POINTER(SsdParams)
+        L.ssd_status_string.restype = ctypes.c_char_p
+        L.ssd_status_string.argtypes = [ctypes.c_int]
+        L.ssd_version.restype = ctypes.c_char_p
+        L.ssd_version.argtypes = []
+        L.ssd_prefill_workspace_bytes.restype = sz
+        L.ssd_prefill_workspace_bytes.argtypes = [dimp, ctypes.c_int]
+        L.ssd_prefill_path.restype = ctypes.c_int
+        L.ssd_prefill_path.argtypes = [dimp, ctypes.c_int]
+        L.ssd_prefill.restype = ctypes.c_int
+        L.ssd_prefill.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 11 + [sz, vp]
+        L.ssd_decode_step.restype = ctypes.c_int
+        L.ssd_decode_step.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 8 + [vp]
+        L.ssd_set_timing_events.restype = ctypes.c_int
+        L.ssd_set_timing_events.argtypes = [vp, vp]
+        _lib = L
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor, y_dtype: torch.dtype) -> int:
+    if t.dtype == torch.bfloat16:
+        if y_dtype == torch.bfloat16:
+            return SSD_BF16
+        if y_dtype == torch.float32:
+            return SSD_BF16_YF32
+    elif t.dtype == torch.float32 and y_dtype == torch.float32:
+        return SSD_F32
+    raise TypeError(f"unsupported activation / output dtypes {t.dtype} / {y_dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, name, shape, dtype, device):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_ptr(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def make_dims(batch, seqlen, nheads, headdim, d_state, ngroups, chunk=128) -> SsdDims:
+    return SsdDims(int(batch), int(seqlen), int(nheads), int(headdim), int(d_state), int(ngroups), int(chunk), 4)
+
+
+def prefill_workspace_bytes(dims: SsdDims, dtype: torch.dtype) -> int:
+    return int(lib().ssd_prefill_workspace_bytes(ctypes.byref(dims), SSD_BF16 if dtype == torch.bfloat16 else
+                                                  SSD_F32))
+
+
+def prefill_path(dims: SsdDims, dtype: torch.dtype) -> int:
+    """1 = tcgen05 tensor-core path, 2 = CUDA-core path, <0 = invalid sizes."""
+    return int(lib().ssd_prefill_path(ctypes.byref(dims), SSD_BF16 if dtype == torch.bfloat16 else SSD_F32))
+
+
+def _params(A, D, dt_bias, conv_w, conv_b, H, conv_dim, device):
+    for name, t, shp in (("A", A, (H,)), ("D", D, (H,)), ("dt_bias", dt_bias, (H,)),
+                         ("conv_w", conv_w, (conv_dim, 4)), ("conv_b", conv_b, (conv_dim,))):
+        _check(t, name, shp, torch.float32, device)
+    return SsdParams(A.data_ptr(), D.data_ptr(), dt_bias.data_ptr(), conv_w.data_ptr(), conv_b.data_ptr())
+
+
+def prefill(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=None, init_conv_state=None, chunk=128,
+            workspace=None, y=None, final_state=None, conv_state=None, y_dtype=None):
+    """Chunked SSD prefill on the GPU.
+
+    x, z [Bt, L, H*P]; dt [Bt, L, H]; B, C [Bt, L, G, N] (bf16 or fp32, one dtype);
+    A, D, dt_bias [H], conv_w [conv_dim, 4], conv_b [conv_dim] fp32;
+    init_state [Bt, H, P, N] fp32 or None; init_conv_state [Bt, conv_dim, 3] or None.
+    y_dtype: the dtype of y (default: the activation dtype; float32 with bf16
+    activations gives the unrounded fp32 y of the same computation).
+    Returns (y, final_state, conv_state).
+    """
+    dev = x.device
+    Bt, L, HP = x.shape
+    H = A.shape[0]
+    P = HP // H
+    G, N = B.shape[2], B.shape[3]
+    act = x.dtype
+    conv_dim = HP + 2 * G * N
+    for name, t, shp in (("x", x, (Bt, L, HP)), ("z", z, (Bt, L, HP)), ("dt", dt, (Bt, L, H)),
+                         ("B", B, (Bt, L, G, N)), ("C", C, (Bt, L, G, N))):
+        _check(t, name, shp, act, dev)
+    if init_state is not None:
+        _check(init_state, "init_state", (Bt, H, P, N), torch.float32, dev)
+    if init_conv_state is not None:
+        _check(init_conv_state, "init_conv_state", (Bt, conv_dim, 3), act, dev)
+    params = _params(A, D, dt_bias, conv_w, conv_b, H, conv_dim, dev)
+    dims = make_dims(Bt, L, H, P, N, G, chunk)
+    ydt = y_dtype or (y.dtype if y is not None else act)
+    code = _dtype_code(x, ydt)
+    if y is None:
+        y = torch.empty((Bt, L, HP), dtype=ydt, device=dev)
+    if final_state is None:
+        final_state = torch.empty((Bt, H, P, N), dtype=torch.float32, device=dev)
+    if conv_state is None:
+        conv_state = torch.empty((Bt, conv_dim, 3), dtype=act, device=dev)
+    _check(y, "y", (Bt, L, HP), ydt, dev)
+    _check(final_state, "final_state", (Bt, H, P, N), torch.float32, dev)
+    _check(conv_state, "conv_state", (Bt, conv_dim, 3), act, dev)
+    need = prefill_workspace_bytes(dims, act)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().ssd_prefill(ctypes.byref(dims), code, ctypes.byref(params), _ptr(x), _ptr(dt), _ptr(B),
+                           _ptr(C), _ptr(z), _ptr(init_state), _ptr(init_conv_state), _ptr(y), _ptr(final_state),
+                           _ptr(conv_state), _ptr(workspace), ws_bytes, _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_prefill")
+    return y, final_state, conv_state
+
+
+def decode_step(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, conv_state, ssm_state, y=None, y_dtype=None):
+    """One decode token for Bt sequences; conv_state and ssm_state update in place.
+
+    x, z [Bt, H*P]; dt [Bt, H]; B, C [Bt, G, N]; conv_state [Bt, conv_dim, 3];
+    ssm_state [Bt, H, P, N] fp32.  Returns y [Bt, H*P].
+    """
+    dev = x.device
+    Bt, HP = x.shape
+    H = A.shape[0]
+    P = HP // H
+    G, N = B.shape[1], B.shape[2]
+    act = x.dtype
+    conv_dim = HP + 2 * G * N
+    for name, t, shp in (("x", x, (Bt, HP)), ("z", z, (Bt, HP)), ("dt", dt, (Bt, H)), ("B", B, (Bt, G, N)),
+                         ("C", C, (Bt, G, N)), ("conv_state", conv_state, (Bt, conv_dim, 3))):
+        _check(t, name, shp, act, dev)
+    _check(ssm_state, "ssm_state", (Bt, H, P, N), torch.float32, dev)
+    params = _params(A, D, dt_bias, conv_w, conv_b, H, conv_dim, dev)
+    ydt = y_dtype or (y.dtype if y is not None else act)
+    code = _dtype_code(x, ydt)
+    if y is None:
+        y = torch.empty((Bt, HP), dtype=ydt, device=dev)
+    _check(y, "y", (Bt, HP), ydt, dev)
+    dims = make_dims(Bt, 1, H, P, N, G)
+    st = lib().ssd_decode_step(ctypes.byref(dims), code, ctypes.byref(params), _ptr(x), _ptr(dt), _ptr(B),
+                               _ptr(C), _ptr(z), _ptr(conv_state), _ptr(ssm_state), _ptr(y), _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_decode_step")
+    return y
+
+
+def set_timing_events(before, after):
+    """Record two torch.cuda.Event objects around the dominant kernel of the next calls (None, None = off)."""
+    if before is None:
+        st = lib().ssd_set_timing_events(None, None)
+    else:
+        for ev in (before, after):
+            if not ev.cuda_event:   # torch creates the CUDA event lazily, on its first record
+                ev.record()
+        st = lib().ssd_set_timing_events(ctypes.c_void_p(before.cuda_event), ctypes.c_void_p(after.cuda_event))
+    if st != 0:
+        raise SsdError(st, "ssd_set_timing_events")
+
+
+def prefill_host(inputs: dict, chunk=128, device="cuda", stream=None):
+    """End-to-end prefill from HOST tensors: copies the inputs to the device
+    (pinned memory -> HBM, asynchronous), runs ssd_prefill and copies y,
+    final_state and conv_state back into pinned host tensors.  Returns the
+    host outputs and the number of bytes moved each way."""
+    dev = torch.device(device)
+    names = ("x", "dt", "B", "C", "z", "A", "D", "dt_bias", "conv_w", "conv_b", "init_state", "init_conv_state")
+    d = {k: (None if inputs.get(k) is None else inputs[k].to(dev, non_blocking=True)) for k in names}
+    y, fs, cs = prefill(d["x"], d["dt"], d["B"], d["C"], d["z"], d["A"], d["D"], d["dt_bias"], d["conv_w"],
+                        d["conv_b"], d["init_state"], d["init_conv_state"], chunk=chunk)
+    outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (y, fs, cs)]
+    for o, t in zip(outs, (y, fs, cs)):
+        o.copy_(t, non_blocking=True)
+    h2d = sum(t.numel() * t.element_size() for t in inputs.values() if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    return outs, h2d, d2h

@@ -1,0 +1,130 @@
+"""The C-ABI library loads, exports every function include/ssd.h declares,
+and rejects bad arguments before touching the device (CPU only: no call here
+reaches a kernel launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_43_b200 import build as build_mod
+from selective_state_space_43_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_mod.build()
+    return ops.lib()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names.update(re.findall(r"SSD_API\s+[\w\s\*]+?\b(ssd_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("ssd_prefill", "ssd_decode_step", "ssd_prefill_workspace_bytes", "ssd_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings_and_version(L):
+    for code in range(0, 9):
+        assert L.ssd_status_string(code)
+    assert b"sm_100a" in L.ssd_version()
+
+
+def dims(**kw):
+    base = dict(batch=1, seqlen=4096, nheads=128, headdim=64, d_state=128, ngroups=8, chunk=128)
+    base.update(kw)
+    return ops.make_dims(**base)
+
+
+def test_path_and_workspace_queries(L):
+    import torch
+    d = dims()
+    path = ops.prefill_path(d, torch.bfloat16)
+    assert path in (1, 2)
+    ws = ops.prefill_workspace_bytes(d, torch.bfloat16)
+    if path == 1:
+        assert ws == 1 * 4096 * 2 * 8 * 128 * 2
+    else:
+        assert ws == 0
+    assert ops.prefill_path(dims(headdim=32), torch.bfloat16) == -2
+    assert ops.prefill_path(dims(nheads=12, ngroups=8), torch.bfloat16) == -2
+    assert ops.prefill_path(dims(chunk=96), torch.bfloat16) == -2
+    assert ops.prefill_path(dims(d_state=48), torch.bfloat16) == -2
+    # fp32 activations and small shapes always take the CUDA-core path
+    assert ops.prefill_path(dims(d_state=32, chunk=64, nheads=4, ngroups=1), torch.float32) == 2
+    assert ops.prefill_workspace_bytes(dims(headdim=32), torch.bfloat16) == 0
+
+
+def _fake_params():
+    # 16-byte aligned fake addresses: every call below fails validation first
+    return ops.SsdParams(0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
+
+
+def _call_prefill(L, d, dtype=1, params=None, ptrs=None, ws=None, ws_bytes=0):
+    p = ptrs or dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, init=None, init_conv=None,
+                     y=0x60000, fs=0x70000, cs=0x80000)
+    prm = params if params is not None else _fake_params()
+    return L.ssd_prefill(ctypes.byref(d), dtype, ctypes.byref(prm) if prm is not False else None,
+                         p["x"], p["dt"], p["B"], p["C"], p["z"], p["init"], p["init_conv"], p["y"], p["fs"],
+                         p["cs"], ws, ws_bytes, None)
+
+
+def test_prefill_rejects_bad_arguments_before_launch(L):
+    assert L.ssd_prefill(None, 1, None, *([None] * 11), 0, None) == 1
+    assert _call_prefill(L, dims(headdim=32)) == 2
+    assert _call_prefill(L, dims(d_conv=3) if False else ops.SsdDims(1, 16, 4, 64, 32, 1, 64, 3)) == 2
+    assert _call_prefill(L, dims(), dtype=7) == 3
+    assert _call_prefill(L, dims(), params=False) == 1
+    assert _call_prefill(L, dims(), params=ops.SsdParams(0x1000, 0, 0x3000, 0x4000, 0x5000)) == 1
+    assert _call_prefill(L, dims(), params=ops.SsdParams(0x1004, 0x2000, 0x3000, 0x4000, 0x5000)) == 4
+    base = dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, init=None, init_conv=None,
+                y=0x60000, fs=0x70000, cs=0x80000)
+    assert _call_prefill(L, dims(), ptrs={**base, "x": None}) == 1
+    assert _call_prefill(L, dims(), ptrs={**base, "fs": None}) == 1
+    assert _call_prefill(L, dims(), ptrs={**base, "B": 0x30008}) == 4
+    assert _call_prefill(L, dims(), ptrs={**base, "y": base["x"]}) == 5
+    assert _call_prefill(L, dims(), ptrs={**base, "init_conv": 0x80000}) == 5
+    assert _call_prefill(L, dims(batch=-1)) == 2
+    import torch
+    if ops.prefill_path(dims(), torch.bfloat16) == 1:
+        assert _call_prefill(L, dims()) == 7                       # no workspace
+        assert _call_prefill(L, dims(), ws=0x90000, ws_bytes=16) == 7
+
+
+def test_decode_rejects_bad_arguments_before_launch(L):
+    d = dims(seqlen=1, batch=256)
+    prm = _fake_params()
+    ok = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000, 0x80000]
+    assert L.ssd_decode_step(None, 1, ctypes.byref(prm), *ok, None) == 1
+    for i in range(8):
+        args = list(ok)
+        args[i] = None
+        assert L.ssd_decode_step(ctypes.byref(d), 1, ctypes.byref(prm), *args, None) == 1
+    args = list(ok)
+    args[6] = 0x70004
+    assert L.ssd_decode_step(ctypes.byref(d), 1, ctypes.byref(prm), *args, None) == 4
+    args = list(ok)
+    args[7] = args[0]
+    assert L.ssd_decode_step(ctypes.byref(d), 1, ctypes.byref(prm), *args, None) == 5
+    bad = dims(nheads=10, ngroups=4)
+    assert L.ssd_decode_step(ctypes.byref(bad), 1, ctypes.byref(prm), *ok, None) == 2
+
+
+def test_timing_hook_requires_both_or_neither(L):
+    assert L.ssd_set_timing_events(ctypes.c_void_p(0x10), None) == 1
+    assert L.ssd_set_timing_events(None, None) == 0
