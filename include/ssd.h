@@ -126,7 +126,7 @@ SSD_API int ssd_prefill_path(const ssd_dims* dims, ssd_dtype dtype);
  *   workspace   device scratch of at least ssd_prefill_workspace_bytes()
  *               bytes (may be NULL when that is 0)
  * seqlen == 0 is valid: final_state = init_state (or zeros), conv_state =
- * the history, y untouched.
+ * the history, y untouched; x, dt, B, C, z and y may then be NULL.
  */
 SSD_API ssd_status ssd_prefill(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
                        const void* x, const void* dt, const void* B, const void* C, const void* z,

@@ -75,11 +75,15 @@ ssd_status ssd_prefill(const ssd_dims* d, ssd_dtype dtype, const ssd_params* par
     ssd_status st = check_dims(d, dtype, true);
     if (st != SSD_OK) return st;
     if ((st = check_params(params)) != SSD_OK) return st;
-    if (!x || !dt || !B || !C || !z || !y || !final_state || !conv_state) return SSD_ERR_NULL;
+    // with no tokens the activations and y are never touched and may be NULL
+    const bool tokens = d->batch > 0 && d->seqlen > 0;
+    if (tokens && (!x || !dt || !B || !C || !z || !y)) return SSD_ERR_NULL;
+    if (d->batch > 0 && (!final_state || !conv_state)) return SSD_ERR_NULL;
     const void* ptrs[] = {x, dt, B, C, z, init_state, init_conv_state, y, final_state, conv_state, workspace};
     for (const void* p : ptrs)
         if (!aligned16(p)) return SSD_ERR_ALIGN;
-    if (y == x || y == z || (init_conv_state && init_conv_state == conv_state)) return SSD_ERR_UNSUPPORTED;
+    if ((tokens && (y == x || y == z)) || (init_conv_state && init_conv_state == conv_state))
+        return SSD_ERR_UNSUPPORTED;
     const int path = ssd_prefill_path(d, dtype);
     const size_t need = path == 1 ? ssd::prefill_tc_workspace_bytes(d->batch, d->seqlen, d->ngroups, d->d_state) : 0;
     if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;

@@ -100,6 +100,10 @@ def test_prefill_rejects_bad_arguments_before_launch(L):
     assert _call_prefill(L, dims(), ptrs={**base, "y": base["x"]}) == 5
     assert _call_prefill(L, dims(), ptrs={**base, "init_conv": 0x80000}) == 5
     assert _call_prefill(L, dims(batch=-1)) == 2
+    # zero tokens: activations may be NULL, the states may not
+    empty = {**base, "x": None, "dt": None, "B": None, "C": None, "z": None, "y": None}
+    assert _call_prefill(L, dims(seqlen=0), ptrs={**empty, "fs": None}) == 1
+    assert _call_prefill(L, dims(seqlen=0), ptrs={**empty, "cs": None}) == 1
     import torch
     if ops.prefill_path(dims(), torch.bfloat16) == 1:
         assert _call_prefill(L, dims()) == 7                       # no workspace
