@@ -104,7 +104,7 @@ SSD_API size_t ssd_prefill_workspace_bytes(const ssd_dims* dims, ssd_dtype dtype
 
 /*
  * Which kernel path ssd_prefill takes for these sizes:
- *   1 = tcgen05 tensor-core chunk scan (bf16 activations, P=64, Q=128, N in {64,128});
+ *   1 = tcgen05 tensor-core chunk scan (bf16 activations, P=64, Q=128, N=128);
  *   2 = CUDA-core chunk scan (every other supported shape, and fp32);
  *  <0 = -(ssd_status) for invalid sizes.
  */
@@ -148,6 +148,15 @@ SSD_API ssd_status ssd_prefill(const ssd_dims* dims, ssd_dtype dtype, const ssd_
 SSD_API ssd_status ssd_decode_step(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
                            const void* x, const void* dt, const void* B, const void* C, const void* z,
                            void* conv_state, float* ssm_state, void* y, void* stream);
+
+/*
+ * Synchronises `stream` and reports whether a kernel launched by this library
+ * gave up on a bounded device-side wait since the last call (SSD_ERR_TIMEOUT;
+ * its outputs are then incomplete), or whether the stream holds a CUDA error
+ * (SSD_ERR_CUDA).  Clears the flag.  Every wait inside the kernels is bounded
+ * (about 2 s), so a kernel can never hang the device.
+ */
+SSD_API ssd_status ssd_device_status(void* stream);
 
 /*
  * Optional timing hook for benchmarks.  When both are non-NULL, the next

@@ -136,6 +136,12 @@ ssd_status ssd_decode_step(const ssd_dims* d, ssd_dtype dtype, const ssd_params*
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
+ssd_status ssd_device_status(void* stream) {
+    int flag = 0;
+    if (ssd::read_and_clear_tc_error(&flag, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSD_ERR_CUDA;
+    return flag ? SSD_ERR_TIMEOUT : SSD_OK;
+}
+
 ssd_status ssd_set_timing_events(void* before_main, void* after_main) {
     if ((before_main == nullptr) != (after_main == nullptr)) return SSD_ERR_NULL;
     g_hook.ev_before = static_cast<cudaEvent_t>(before_main);

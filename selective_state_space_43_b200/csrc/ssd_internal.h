@@ -52,5 +52,7 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, ActKind kind, cudaStream_t
 bool prefill_tc_supported(int P, int N, int Q, bool bf16);
 size_t prefill_tc_workspace_bytes(int64_t batch, int64_t L, int G, int N);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t st, const TimingHook& hook);
+// Synchronises `st`, then reads and clears the tensor-core kernel's timeout flag.
+cudaError_t read_and_clear_tc_error(int* flag, cudaStream_t st);
 
 }  // namespace ssd

@@ -47,16 +47,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Waits for the phase of `parity` to complete.  Gives up after `timeout_ns`
-// (or as soon as *abort is set by another role) and returns false.
+// Waits for the phase of `parity` to complete.  Returns false without waiting
+// once *abort is set (abort may be nullptr), or after `timeout_ns`.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns = 2000000000ull) {
+    if (abort && *abort) return false;
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0u) {
-            if (*abort) return false;
+            if (abort && *abort) return false;
             if (globaltimer_ns() - t0 > timeout_ns) return false;
         }
     }

@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 11 + [sz, vp]
         L.ssd_decode_step.restype = ctypes.c_int
         L.ssd_decode_step.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 8 + [vp]
+        L.ssd_device_status.restype = ctypes.c_int
+        L.ssd_device_status.argtypes = [vp]
         L.ssd_set_timing_events.restype = ctypes.c_int
         L.ssd_set_timing_events.argtypes = [vp, vp]
         _lib = L
@@ -201,6 +203,13 @@ def decode_step(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, conv_state, ssm_s
     if st != 0:
         raise SsdError(st, "ssd_decode_step")
     return y
+
+
+def device_status(device="cuda"):
+    """Synchronise the current stream and raise if a kernel gave up on a bounded device-side wait."""
+    st = lib().ssd_device_status(_stream_ptr(torch.device(device)))
+    if st != 0:
+        raise SsdError(st, "ssd_device_status")
 
 
 def set_timing_events(before, after):

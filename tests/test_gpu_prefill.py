@@ -26,7 +26,7 @@ def run_both(dev, chunk):
 def _check_full(inp, chunk, tag):
     dev = dev_inputs(inp)
     y32, _, fs, cs = run_both(dev, chunk)
-    torch.cuda.synchronize()
+    ops.device_status()
     yo, fo, co = oracle.prefill(inp)
     r1 = assert_close(np64(y32), yo, f"{tag} y")
     r2 = assert_close(np64(fs), fo, f"{tag} final_state")
@@ -148,7 +148,7 @@ def test_prefill_full_size_sampled(name):
     d, dt, inp = workload(name)
     dev = dev_inputs(inp)
     y, _, fs, cs = run_both(dev, d.chunk)
-    torch.cuda.synchronize()
+    ops.device_status()
     assert torch.isfinite(y).all() and torch.isfinite(fs).all()
     mask = np.zeros((d.batch, d.nheads), dtype=bool)
     hpg = d.nheads // d.ngroups
@@ -162,3 +162,11 @@ def test_prefill_full_size_sampled(name):
         assert_close(yg[b, :, h * P:(h + 1) * P], yo[b, :, h * P:(h + 1) * P], f"{name} y (b={b}, h={h})")
         assert_close(fg[b, h], fo[b, h], f"{name} final_state (b={b}, h={h})")
     assert np.array_equal(np64(cs), co)
+
+
+def test_layer_shapes_take_the_tensor_core_path():
+    from selective_state_space_43_b200.synth import WORKLOADS
+    for name in ("nemotron_h_8b", "nemotron3_nano", "hybrid_3b"):
+        d = WORKLOADS[name]["dims"]
+        dims = ops.make_dims(d.batch, d.seqlen, d.nheads, d.headdim, d.d_state, d.ngroups, d.chunk)
+        assert ops.prefill_path(dims, torch.bfloat16) == 1, name
