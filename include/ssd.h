@@ -150,6 +150,35 @@ SSD_API ssd_status ssd_decode_step(const ssd_dims* dims, ssd_dtype dtype, const 
                            void* conv_state, float* ssm_state, void* y, void* stream);
 
 /*
+ * Size of the built-in scratch array used by ssd_prefill_noalloc: 16 MiB,
+ * enough for batch * seqlen * 2 * ngroups * d_state * 2 bytes, e.g. 4096
+ * tokens of a layer with 8 groups of d_state 128.
+ */
+#define SSD_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * ssd_prefill without a workspace argument, for callers that cannot allocate
+ * device memory themselves (no access to an allocator, or an allocation would
+ * synchronise or break a pre-reserved memory budget).  No counterpart in the
+ * pages: this is a packaging of ssd_prefill, not another step of the method.
+ * Arguments, layouts and results are exactly those of ssd_prefill; the
+ * scratch lives in a fixed SSD_NOALLOC_SCRATCH_BYTES array inside the
+ * library, held on every GPU that loads it until the process exits.
+ *  - Returns SSD_ERR_WORKSPACE, launching nothing, when the sizes need more
+ *    scratch than that (ssd_prefill_workspace_bytes() > SSD_NOALLOC_SCRATCH_BYTES).
+ *  - Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's address there; make it before any stream capture.
+ *  - All calls share the array: calls whose kernels overlap on the GPU race.
+ *    Each call rewrites every scratch element it reads, so no clearing is
+ *    needed between calls.
+ */
+SSD_API ssd_status ssd_prefill_noalloc(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
+                               const void* x, const void* dt, const void* B, const void* C, const void* z,
+                               const float* init_state, const void* init_conv_state,
+                               void* y, float* final_state, void* conv_state, void* stream);
+
+/*
  * Synchronises `stream` and reports whether a kernel launched by this library
  * gave up on a bounded device-side wait since the last call (SSD_ERR_TIMEOUT;
  * its outputs are then incomplete), or whether the stream holds a CUDA error

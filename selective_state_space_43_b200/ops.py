@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 11 + [sz, vp]
         L.ssd_decode_step.restype = ctypes.c_int
         L.ssd_decode_step.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 8 + [vp]
+        L.ssd_prefill_noalloc.restype = ctypes.c_int
+        L.ssd_prefill_noalloc.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 10 + [vp]
         L.ssd_device_status.restype = ctypes.c_int
         L.ssd_device_status.argtypes = [vp]
         L.ssd_set_timing_events.restype = ctypes.c_int
@@ -203,6 +205,50 @@ def decode_step(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, conv_state, ssm_s
     if st != 0:
         raise SsdError(st, "ssd_decode_step")
     return y
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def prefill_noalloc(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=None, init_conv_state=None,
+                    chunk=128, y=None, final_state=None, conv_state=None, y_dtype=None):
+    """ssd_prefill_noalloc: the same prefill with the library's built-in scratch
+    (for callers that cannot allocate a workspace).  Outputs must be passed in
+    if the caller cannot allocate them either.  Raises SsdError
+    (SSD_ERR_WORKSPACE) when the sizes need more than 16 MiB of scratch."""
+    dev = x.device
+    Bt, L, HP = x.shape
+    H = A.shape[0]
+    P = HP // H
+    G, N = B.shape[2], B.shape[3]
+    act = x.dtype
+    conv_dim = HP + 2 * G * N
+    for name, t, shp in (("x", x, (Bt, L, HP)), ("z", z, (Bt, L, HP)), ("dt", dt, (Bt, L, H)),
+                         ("B", B, (Bt, L, G, N)), ("C", C, (Bt, L, G, N))):
+        _check(t, name, shp, act, dev)
+    if init_state is not None:
+        _check(init_state, "init_state", (Bt, H, P, N), torch.float32, dev)
+    if init_conv_state is not None:
+        _check(init_conv_state, "init_conv_state", (Bt, conv_dim, 3), act, dev)
+    params = _params(A, D, dt_bias, conv_w, conv_b, H, conv_dim, dev)
+    ydt = y_dtype or (y.dtype if y is not None else act)
+    code = _dtype_code(x, ydt)
+    if y is None:
+        y = torch.empty((Bt, L, HP), dtype=ydt, device=dev)
+    if final_state is None:
+        final_state = torch.empty((Bt, H, P, N), dtype=torch.float32, device=dev)
+    if conv_state is None:
+        conv_state = torch.empty((Bt, conv_dim, 3), dtype=act, device=dev)
+    _check(y, "y", (Bt, L, HP), ydt, dev)
+    _check(final_state, "final_state", (Bt, H, P, N), torch.float32, dev)
+    _check(conv_state, "conv_state", (Bt, conv_dim, 3), act, dev)
+    dims = make_dims(Bt, L, H, P, N, G, chunk)
+    st = lib().ssd_prefill_noalloc(ctypes.byref(dims), code, ctypes.byref(params), _ptr(x), _ptr(dt), _ptr(B),
+                                   _ptr(C), _ptr(z), _ptr(init_state), _ptr(init_conv_state), _ptr(y),
+                                   _ptr(final_state), _ptr(conv_state), _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_prefill_noalloc")
+    return y, final_state, conv_state
 
 
 def device_status(device="cuda"):
