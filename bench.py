@@ -444,7 +444,7 @@ def main():
                        "l2": "flushed between timed steps (256 MB write outside the step events)",
                        "kernel_path": "tcgen05 tensor-core" if path == 1 else "CUDA-core"},
             "tensor": tc, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
-            "gpu_launches": K * (2 if path == 1 else 1), "clocks": clocks,
+            "gpu_launches": K * (3 if path == 1 else 1), "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

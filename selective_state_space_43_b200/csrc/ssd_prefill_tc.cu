@@ -15,19 +15,32 @@
 //   y      = (Y + exp(cs_i) Y2 + D x) SiLU(z)
 //   S_prev <- exp(cs_last) S_prev + S_c
 //
-// Two kernels:
+// Three kernels:
 //   bc_prologue  SiLU(conv4) of the B and C channels of every token, written
 //                once per group to the workspace in bf16 (the 16 heads of a
-//                group then read it from L2 instead of recomputing it), and
-//                the conv_state tail of all channels.
+//                group then read it from L2 instead of recomputing it);
+//   conv_tail    the conv_state output (last 3 pre-conv tokens, all channels);
 //   chunk_scan   one CTA per (sequence b, head h) walks the chunks in order;
 //                all accumulators live in TMEM; 7 warps:
-//                  warp 0  TMA producer: raw x and z tiles (2-stage ring)
+//                  warp 0  TMA producer: raw x tiles (2-stage ring)
 //                  warp 1  TMEM allocator + single-thread tcgen05.mma issuer
-//                  warp 2  TMA producer: post-conv B and C tiles
-//                  warps 3-6  128 compute threads, thread i <-> token row i
-//                           <-> TMEM lane i: x conv, decay mask, state pass,
-//                           epilogue (D skip, z gate, y store).
+//                  warp 2  TMA producer: post-conv B and C tiles; the whole
+//                           warp also computes each chunk's dt, cumsum of dt*A
+//                           and mask factors one chunk ahead (double-buffered)
+//                  warps 3-18 512 compute threads.  The x conv runs channel-
+//                           major (warp = 8 tokens, lane = 2 channels, taps in
+//                           registers); the TMEM phases run row-major, four
+//                           threads per token row i (= TMEM lane i), each owning
+//                           16 columns and one of the 4 decay-mask column blocks:
+//                           decay mask, state pass, epilogue (D skip from the
+//                           fp32 conv output, z gate loaded straight from
+//                           global memory, y store).  Elementwise math uses
+//                           the packed fp32x2 FMA / MUL of sm_100.
+// The decay mask exp(cs_i - cs_j) is formed per 32-column block: exactly
+// (one exp per element) on the diagonal block, and as the product of a row
+// factor exp(cs_i - cs_r) and a column factor exp(cs_r - cs_j) dt_j, with r the
+// block's last column, below it.  Both factors are <= 1, so neither overflows,
+// and either underflows only where the true product is below ~1e-38.
 // Every mbarrier wait is bounded; a wait that gives up raises a device error
 // flag (read back by ssd_device_status) and the CTA drains and exits.
 #include <cuda.h>
@@ -45,9 +58,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kQ = 128, kP = 64, kN = 128;
-constexpr int kThreads = 224;
+constexpr int kThreads = 608;
 constexpr int kWarpRaw = 0, kWarpMma = 1, kWarpBc = 2, kFirstCompute = 3;
-constexpr int kComputeThreads = 128;
+constexpr int kComputeThreads = 512;  // 16 warps: four per TMEM lane quadrant
 
 // shared memory map (bytes from a 1024-byte aligned base)
 constexpr uint32_t OFF_C = 0;          // u_C tile: two boxes [128 tok][64 n] bf16, 128B swizzle
@@ -57,17 +70,16 @@ constexpr uint32_t OFF_XP = 81920;     // X' [j][p] bf16
 constexpr uint32_t OFF_M = 98304;      // M  [i][j] bf16, two K blocks of 64 (K-major A operand)
 constexpr uint32_t OFF_S = 131072;     // S_prev [n][p] bf16 (MN-major B operand)
 constexpr uint32_t OFF_RAWX = 147456;  // 2 x raw x tile [tok][p] bf16 (TMA, 128B swizzle)
-constexpr uint32_t OFF_RAWZ = 180224;  // 2 x raw z tile
+constexpr uint32_t OFF_U = 180224;     // post-conv x [tok][p] fp32 for the D skip (256-byte rows, swizzled)
 constexpr uint32_t OFF_SMALL = 212992;
 // small region
-constexpr uint32_t OFF_W = OFF_SMALL;              // conv taps of the head's x channels  [64] float4
-constexpr uint32_t OFF_CB = OFF_W + 64 * 16;       // conv bias [64] float
-constexpr uint32_t OFF_HALO = OFF_CB + 64 * 4;     // [2][3][64] bf16 raw x history
-constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;  // cs [128] float
-constexpr uint32_t OFF_DT = OFF_CS + 128 * 4;      // dt [128] float
-constexpr uint32_t OFF_WTOT = OFF_DT + 128 * 4;    // warp totals of the dA scan [4] float
-constexpr uint32_t OFF_BAR = OFF_WTOT + 16;        // mbarriers (8 B each)
-constexpr int NBAR = 13;
+constexpr uint32_t OFF_HALO = OFF_SMALL;           // [2][3][64] bf16 raw x history
+constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;  // cs [2][128] float (double-buffered by chunk parity)
+constexpr uint32_t OFF_DT = OFF_CS + 2 * 128 * 4;      // dt [2][128]
+constexpr uint32_t OFF_COLF = OFF_DT + 2 * 128 * 4;    // column factors of the decay mask [2][128]
+constexpr uint32_t OFF_WX = OFF_COLF + 2 * 128 * 4;    // weight of x_j in the chunk state [2][128]
+constexpr uint32_t OFF_BAR = OFF_WX + 2 * 128 * 4;     // mbarriers (8 B each)
+constexpr int NBAR = 16;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;  // TMEM base address
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
@@ -75,23 +87,22 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 enum Bar { FULL_RAW0 = 0, FULL_RAW1, EMPTY_RAW0, EMPTY_RAW1, FULL_BC, EMPTY_BC, XREADY, MREADY, G_FULL, SC_FULL,
-           Y_FULL, MMA_DONE, COMPUTE_SYNC };
+           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1 };
 
 // TMEM columns (fp32 accumulators, 128 lanes)
 constexpr uint32_t COL_G = 0, COL_Y = 128, COL_Y2 = 192, COL_SC = 256, COL_SRUN = 320, TMEM_COLS = 512;
 
 struct TcParams {
     PrefillArgs a;
-    CUtensorMap tm_x, tm_z, tm_bc;
+    CUtensorMap tm_x, tm_bc;
 };
 
-// Barrier among the 128 compute threads, on an mbarrier so that it is bounded
-// like every other wait (a named barrier could not give up).
-__device__ __forceinline__ bool compute_sync(uint64_t* bar, uint32_t& phase, volatile int* abort_flag) {
-    mbar_arrive(bar);
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase, abort_flag));
-    phase ^= 1u;
-    return ok;
+// Byte offset of the float2 `pair` (0..31) of row `row` in the fp32 [128][64]
+// conv-output tile: 256-byte rows, 16-byte chunks XOR-swizzled by the row so that
+// a warp reading 32 consecutive rows at one column, or writing one row, is conflict-free.
+__device__ __forceinline__ uint32_t u_off(uint32_t row, uint32_t pair) {
+    const uint32_t chunk = pair >> 1;  // 16-byte chunk (0..15)
+    return row * 256u + (((chunk ^ (row & 15u)) << 4) | ((pair & 1u) << 3));
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -107,6 +118,28 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
+// SiLU(v) = v sigmoid(v) with sigmoid(v) = (1 + tanh(v/2)) / 2: one MUFU
+// operation (the hardware tanh approximation, relative error ~2^-11) instead
+// of an exponential and a reciprocal.
+__device__ __forceinline__ float tanh_approx(float v) {
+    float r;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ float silu_fast(float v) {
+    const float hv = 0.5f * v;
+    return fmaf(hv, tanh_approx(hv), hv);
+}
+
+// softplus(v) = log(1 + e^v) with the fast exp / log (absolute error ~1e-7
+// for the small dt this layer uses); above 20 the correction is below 2.1e-9.
+__device__ __forceinline__ float softplus_fast(float v) { return v > 20.f ? v : __logf(1.f + __expf(v)); }
+
+__device__ __forceinline__ float2 silu2(float2 v) {
+    const float2 hv = __fmul2_rn(v, make_float2(0.5f, 0.5f));
+    return __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+}
+
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
     *abort_flag = 1;
     atomicExch(&g_tc_error, 1);
@@ -120,6 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
+    float* s_cs = reinterpret_cast<float*>(sm + OFF_CS);      // [2][128] per chunk parity
+    float* s_dt = reinterpret_cast<float*>(sm + OFF_DT);
+    float* s_colf = reinterpret_cast<float*>(sm + OFF_COLF);
+    float* s_wx = reinterpret_cast<float*>(sm + OFF_WX);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
@@ -139,7 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         mbar_init(&bars[SC_FULL], 1);
         mbar_init(&bars[Y_FULL], 1);
         mbar_init(&bars[MMA_DONE], 1);
-        mbar_init(&bars[COMPUTE_SYNC], kComputeThreads);
+        mbar_init(&bars[CS_READY0], 32);
+        mbar_init(&bars[CS_READY1], 32);
+        mbar_init(&bars[CS_FREE0], kComputeThreads);
+        mbar_init(&bars[CS_FREE1], kComputeThreads);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -150,10 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     if (warp >= kFirstCompute) {
         const int i = threadIdx.x - kFirstCompute * 32;
         if (i < kP) {
-            const int ch = h * kP + i;
-            reinterpret_cast<float4*>(sm + OFF_W)[i] = *reinterpret_cast<const float4*>(a.conv_w + (size_t)ch * 4);
-            reinterpret_cast<float*>(sm + OFF_CB)[i] = a.conv_b[ch];
             // conv history of token 0: the initial conv state (tokens -3..-1) or zeros
+            const int ch = h * kP + i;
             __nv_bfloat16* halo = reinterpret_cast<__nv_bfloat16*>(sm + OFF_HALO);
             for (int k = 0; k < 3; ++k) {
                 __nv_bfloat16 v = __float2bfloat16_rn(0.f);
@@ -168,10 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     const uint32_t tmem = *tmem_holder;
 
     if (warp == kWarpRaw) {
-        // ---------------- raw x / z producer ----------------
+        // ---------------- raw x producer ----------------
         if (lane == 0) {
             prefetch_tmap(&prm.tm_x);
-            prefetch_tmap(&prm.tm_z);
             int issued[2] = {-1, -1};
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
@@ -179,9 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     raise_abort(abort_flag);
                     break;
                 }
-                mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 2 * 16384);
+                mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384);
                 tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, c * kQ, b);
-                tma_load_3d(sm + OFF_RAWZ + s * 16384, &prm.tm_z, &bars[FULL_RAW0 + s], h * kP, c * kQ, b);
                 issued[s] = c;
             }
             if (*abort_flag) {  // let copies still in flight land before the CTA exits
@@ -190,25 +226,75 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
         }
     } else if (warp == kWarpBc) {
-        // ---------------- post-conv B / C producer ----------------
-        if (lane == 0) {
-            prefetch_tmap(&prm.tm_bc);
-            int last = -1;
-            for (int c = 0; c < nc; ++c) {
-                if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) {
-                    raise_abort(abort_flag);
-                    break;
-                }
-                mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
-                const int xc = a.GN + g * kN, xb = g * kN;
-                tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, c * kQ, b);
-                tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, c * kQ, b);
-                tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, c * kQ, b);
-                tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, c * kQ, b);
-                last = c;
+        // ---------------- post-conv B / C producer + the chunk's dt / cumsum ----------------
+        const float A = a.A[h], dtb = a.dt_bias[h];
+        const __nv_bfloat16* dtp = static_cast<const __nv_bfloat16*>(a.dt);
+        float dt_next[4];
+        auto load_dt = [&](int cc) {  // dt of rows 4*lane .. 4*lane+3 of chunk cc
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int64_t t = (int64_t)cc * kQ + 4 * lane + k;
+                dt_next[k] = t < a.L ? __bfloat162float(dtp[((size_t)b * a.L + t) * a.H + h]) : 0.f;
             }
-            if (*abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
+        };
+        load_dt(0);
+        if (lane == 0) prefetch_tmap(&prm.tm_bc);
+        int last = -1;
+        for (int c = 0; c < nc; ++c) {
+            int okc = 1;
+            if (lane == 0) {
+                if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) {
+                    okc = 0;
+                } else {
+                    mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
+                    const int xc = a.GN + g * kN, xb = g * kN;
+                    tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, c * kQ, b);
+                    tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, c * kQ, b);
+                    tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, c * kQ, b);
+                    tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, c * kQ, b);
+                    last = c;
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, okc, 0)) { raise_abort(abort_flag); break; }
+            // dt = softplus(dt_raw + bias) and the inclusive cumsum of dt*A over the chunk's 128 rows,
+            // into the buffer of this chunk's parity once every compute thread is done with it
+            const int buf = c & 1;
+            if (c >= 2 && !warp_wait(&bars[CS_FREE0 + buf], ((c >> 1) + 1) & 1, abort_flag)) {
+                raise_abort(abort_flag);
+                break;
+            }
+            const int Qc = (int)(a.L - (int64_t)c * kQ < kQ ? a.L - (int64_t)c * kQ : kQ);
+            float dr[4] = {dt_next[0], dt_next[1], dt_next[2], dt_next[3]};
+            if (c + 1 < nc) load_dt(c + 1);
+            float dtv[4], cs[4];
+            float run = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                dtv[k] = (4 * lane + k < Qc) ? softplus_fast(dr[k] + dtb) : 0.f;
+                run += dtv[k] * A;
+                cs[k] = run;
+            }
+            float incl = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float up = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += up;
+            }
+            const float excl = incl - run;
+            const float cs_last = __shfl_sync(0xffffffffu, incl, 31);
+            const float cs_blk = __shfl_sync(0xffffffffu, incl, lane | 7);  // cs at the last row of the 32-row block
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = 4 * lane + k;
+                const float csr = cs[k] + excl;
+                s_cs[buf * 128 + r] = csr;
+                s_dt[buf * 128 + r] = dtv[k];
+                s_colf[buf * 128 + r] = __expf(cs_blk - csr) * dtv[k];
+                s_wx[buf * 128 + r] = __expf(cs_last - csr) * dtv[k];
+            }
+            mbar_arrive(&bars[CS_READY0 + buf]);
         }
+        if (lane == 0 && *abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
     } else if (warp == kWarpMma) {
         // ---------------- tcgen05.mma issuer ----------------
         if (lane == 0) {
@@ -261,147 +347,135 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         }
     } else {
         // ---------------- compute warps ----------------
-        const int q = warp & 3;                       // TMEM lane quadrant of this warp
-        const int i = q * 32 + lane;                  // token row / TMEM lane / state row n
+        const int wc = warp - kFirstCompute;               // 0..15
+        const int q = warp & 3;                            // TMEM lane quadrant of this warp
+        const int quarter = wc >> 2;                       // row-major phases: columns 16*quarter .. +15
+        const int i = q * 32 + lane;                       // row-major phases: token row / TMEM lane
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float A = a.A[h], Dh = a.D[h], dtb = a.dt_bias[h];
-        const __nv_bfloat16* dtp = static_cast<const __nv_bfloat16*>(a.dt);
-        float* s_cs = reinterpret_cast<float*>(sm + OFF_CS);
-        float* s_dt = reinterpret_cast<float*>(sm + OFF_DT);
-        float* s_wtot = reinterpret_cast<float*>(sm + OFF_WTOT);
-        const float4* s_w = reinterpret_cast<const float4*>(sm + OFF_W);
-        const float* s_cb = reinterpret_cast<const float*>(sm + OFF_CB);
+        const float Dh = a.D[h];
         uint8_t* sX = sm + OFF_X;
         uint8_t* sXp = sm + OFF_XP;
         uint8_t* sMm = sm + OFF_M;
         uint8_t* sS = sm + OFF_S;
+        uint8_t* sU = sm + OFF_U;
 
-        // initial state: S_run (TMEM, fp32) and its bf16 copy (smem) for the first chunk's C S^T
+        // conv taps of this lane's channel pair (channel-major conv), constant over the sequence
+        const int ch0 = h * kP + 2 * lane;
+        const float4 wa = *reinterpret_cast<const float4*>(a.conv_w + (size_t)ch0 * 4);
+        const float4 wb = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(ch0 + 1) * 4);
+        const float2 tap0 = make_float2(wa.x, wb.x), tap1 = make_float2(wa.y, wb.y);
+        const float2 tap2 = make_float2(wa.z, wb.z), tap3 = make_float2(wa.w, wb.w);
+        const float2 cbias = make_float2(a.conv_b[ch0], a.conv_b[ch0 + 1]);
+
+        // initial state (this thread's 16 columns): S_run in TMEM, bf16 copy in smem
         {
             const float* init = a.init_state ? a.init_state + ((size_t)b * a.H + h) * kP * kN : nullptr;
+            float v[16];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
+            for (int k = 0; k < 16; ++k) v[k] = init ? init[(size_t)(quarter * 16 + k) * kN + i] : 0.f;
+            tmem_st16(tmem + lane_base + COL_SRUN + quarter * 16, v);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) v[k] = init ? init[(size_t)(half * 32 + k) * kN + i] : 0.f;
-                tmem_st32(tmem + lane_base + COL_SRUN + half * 32, v);
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    uint4 w;
-                    w.x = pack_bf2(v[k4 * 8 + 0], v[k4 * 8 + 1]);
-                    w.y = pack_bf2(v[k4 * 8 + 2], v[k4 * 8 + 3]);
-                    w.z = pack_bf2(v[k4 * 8 + 4], v[k4 * 8 + 5]);
-                    w.w = pack_bf2(v[k4 * 8 + 6], v[k4 * 8 + 7]);
-                    *reinterpret_cast<uint4*>(sS + sw128_off(i, half * 4 + k4)) = w;
-                }
+            for (int k2 = 0; k2 < 2; ++k2) {
+                uint4 w;
+                w.x = pack_bf2(v[k2 * 8 + 0], v[k2 * 8 + 1]);
+                w.y = pack_bf2(v[k2 * 8 + 2], v[k2 * 8 + 3]);
+                w.z = pack_bf2(v[k2 * 8 + 4], v[k2 * 8 + 5]);
+                w.w = pack_bf2(v[k2 * 8 + 6], v[k2 * 8 + 7]);
+                *reinterpret_cast<uint4*>(sS + sw128_off(i, quarter * 2 + k2)) = w;
             }
             tmem_wait_st();
         }
 
-        float u[kP];  // post-conv x of row i, kept for the D skip
-        bool ok = true;
-        uint32_t sync_phase = 0;
-        for (int c = 0; c < nc && ok; ++c) {
-            const int s = c & 1;
+        for (int c = 0; c < nc; ++c) {
+            const int s = c & 1, buf = c & 1;
             const int64_t t0 = (int64_t)c * kQ;
             const int Qc = (int)(a.L - t0 < kQ ? a.L - t0 : kQ);
-            const bool valid = i < Qc;
+            const float* cs_b = s_cs + buf * 128;
 
-            // (b) dt, in-chunk inclusive cumsum of dt*A
-            float dtv = 0.f, dA = 0.f;
-            if (valid) {
-                dtv = softplus_f(__bfloat162float(dtp[((size_t)b * a.L + t0 + i) * a.H + h]) + dtb);
-                dA = dtv * A;
-            }
-            float inc = dA;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float up = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += up;
-            }
-            if (lane == 31) s_wtot[q] = inc;
-            if (!compute_sync(&bars[COMPUTE_SYNC], sync_phase, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
-            float off = 0.f;
-            for (int k = 0; k < q; ++k) off += s_wtot[k];
-            const float cs_i = inc + off;
-            const float cs_last = s_wtot[0] + s_wtot[1] + s_wtot[2] + s_wtot[3];
-            s_cs[i] = cs_i;
-            s_dt[i] = dtv;
-            const float wx = valid ? __expf(cs_last - cs_i) * dtv : 0.f;  // weight of x_i in the chunk state
-            const float ecs = __expf(cs_i);                               // decay of S_prev up to row i
+            if (!warp_wait(&bars[CS_READY0 + buf], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            const float cs_i = cs_b[i];
+            const float cs_last = cs_b[kQ - 1];
+            const float ecs = __expf(cs_i);  // decay of S_prev up to row i
 
-            // (c) raw x tile -> conv + SiLU -> X, X'
-            if (!warp_wait(&bars[FULL_RAW0 + s], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
-            const uint8_t* rx = sm + OFF_RAWX + s * 16384;
-            const __nv_bfloat16* halo_in = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_HALO) + (c & 1) * 192;
+            // (c) conv + SiLU, channel-major: rows 8*wc .. 8*wc+7, channels 2*lane, 2*lane+1
+            if (!warp_wait(&bars[FULL_RAW0 + s], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            {
+                const uint8_t* rx = sm + OFF_RAWX + s * 16384;
+                const uint32_t* halo_in = reinterpret_cast<const uint32_t*>(sm + OFF_HALO) + (c & 1) * 96;
+                const float* wx_b = s_wx + buf * 128;
+                const int r0 = 8 * wc;
+                const uint32_t lane_byte = (uint32_t)(lane & 3) * 4;
+                uint32_t raw[11];
 #pragma unroll
-            for (int k8 = 0; k8 < 8; ++k8) {  // 8 channels (16 bytes) at a time
-                float acc[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = s_cb[k8 * 8 + e];
-#pragma unroll
-                for (int tap = 0; tap < 4; ++tap) {
-                    const int r = i - 3 + tap;
-                    uint4 w;
-                    if (r >= 0) {
-                        w = *reinterpret_cast<const uint4*>(rx + sw128_off(r, k8));
-                    } else {
-                        w = *reinterpret_cast<const uint4*>(halo_in + (r + 3) * 64 + k8 * 8);
-                    }
-                    const float xv[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
-                                         bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float4 wt = s_w[k8 * 8 + e];
-                        const float tw = tap == 0 ? wt.x : (tap == 1 ? wt.y : (tap == 2 ? wt.z : wt.w));
-                        acc[e] = fmaf(tw, xv[e], acc[e]);
-                    }
+                for (int k = 0; k < 11; ++k) {
+                    const int r = r0 - 3 + k;
+                    raw[k] = r >= 0 ? *reinterpret_cast<const uint32_t*>(rx + sw128_off(r, lane >> 2) + lane_byte)
+                                    : halo_in[(r + 3) * 32 + lane];
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) u[k8 * 8 + e] = valid ? silu_f(acc[e]) : 0.f;
-                uint4 o1, o2;
-                o1.x = pack_bf2(u[k8 * 8 + 0], u[k8 * 8 + 1]);
-                o1.y = pack_bf2(u[k8 * 8 + 2], u[k8 * 8 + 3]);
-                o1.z = pack_bf2(u[k8 * 8 + 4], u[k8 * 8 + 5]);
-                o1.w = pack_bf2(u[k8 * 8 + 6], u[k8 * 8 + 7]);
-                o2.x = pack_bf2(u[k8 * 8 + 0] * wx, u[k8 * 8 + 1] * wx);
-                o2.y = pack_bf2(u[k8 * 8 + 2] * wx, u[k8 * 8 + 3] * wx);
-                o2.z = pack_bf2(u[k8 * 8 + 4] * wx, u[k8 * 8 + 5] * wx);
-                o2.w = pack_bf2(u[k8 * 8 + 6] * wx, u[k8 * 8 + 7] * wx);
-                *reinterpret_cast<uint4*>(sX + sw128_off(i, k8)) = o1;
-                *reinterpret_cast<uint4*>(sXp + sw128_off(i, k8)) = o2;
-            }
-            if (i >= kQ - 3) {  // raw history of the next chunk
-                __nv_bfloat16* halo_out = reinterpret_cast<__nv_bfloat16*>(sm + OFF_HALO) + ((c + 1) & 1) * 192;
-#pragma unroll
-                for (int k8 = 0; k8 < 8; ++k8)
-                    *reinterpret_cast<uint4*>(halo_out + (i - (kQ - 3)) * 64 + k8 * 8) =
-                        *reinterpret_cast<const uint4*>(rx + sw128_off(i, k8));
+                for (int k = 0; k < 8; ++k) {
+                    const int r = r0 + k;
+                    uint32_t xo = 0u, xpo = 0u;
+                    float2 uv = make_float2(0.f, 0.f);
+                    if (r < Qc) {  // warp-uniform
+                        float2 acc = cbias;
+                        acc = __ffma2_rn(tap0, make_float2(bf_lo(raw[k + 0]), bf_hi(raw[k + 0])), acc);
+                        acc = __ffma2_rn(tap1, make_float2(bf_lo(raw[k + 1]), bf_hi(raw[k + 1])), acc);
+                        acc = __ffma2_rn(tap2, make_float2(bf_lo(raw[k + 2]), bf_hi(raw[k + 2])), acc);
+                        acc = __ffma2_rn(tap3, make_float2(bf_lo(raw[k + 3]), bf_hi(raw[k + 3])), acc);
+                        uv = silu2(acc);
+                        const float wxr = wx_b[r];
+                        xo = pack_bf2(uv.x, uv.y);
+                        const float2 up = __fmul2_rn(uv, make_float2(wxr, wxr));
+                        xpo = pack_bf2(up.x, up.y);
+                    }
+                    const uint32_t off = sw128_off(r, lane >> 2) + lane_byte;
+                    *reinterpret_cast<uint32_t*>(sX + off) = xo;
+                    *reinterpret_cast<uint32_t*>(sXp + off) = xpo;
+                    *reinterpret_cast<float2*>(sU + u_off(r, lane)) = uv;
+                }
+                if (wc == 15) {  // raw history (rows 125..127) of the next chunk
+                    uint32_t* halo_out = reinterpret_cast<uint32_t*>(sm + OFF_HALO) + ((c + 1) & 1) * 96;
+                    halo_out[0 * 32 + lane] = raw[8];
+                    halo_out[1 * 32 + lane] = raw[9];
+                    halo_out[2 * 32 + lane] = raw[10];
+                }
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[XREADY]);
-            // s_cs / s_dt of this chunk visible to every compute thread
-            if (!compute_sync(&bars[COMPUTE_SYNC], sync_phase, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
 
-            // (e) decay mask: M[i, j] = G[i, j] exp(cs_i - cs_j) dt_j for j <= i
-            if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
+            // (e) decay mask, column block kb = quarter of row i
+            if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {  // 32 columns j at a time
+            {
+                const int kb = quarter;
                 uint32_t packed[16];
-                if (kb <= q) {  // warp-uniform: blocks right of the diagonal are all zero
+                if (kb < q) {  // strictly below the diagonal: row factor x column factor
+                    const float rowf = __expf(cs_i - cs_b[kb * 32 + 31]);
+                    const float2 rf = make_float2(rowf, rowf);
+                    float gv[32];
+                    tmem_ld32(tmem + lane_base + COL_G + kb * 32, gv);
+                    tmem_wait_ld();
+                    const float2* colf = reinterpret_cast<const float2*>(s_colf + buf * 128 + kb * 32);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float2 m = __fmul2_rn(__fmul2_rn(make_float2(gv[e], gv[e + 1]), colf[e >> 1]), rf);
+                        packed[e >> 1] = pack_bf2(m.x, m.y);
+                    }
+                } else if (kb == q) {  // diagonal block: exact decay for j <= i
+                    const float* dt_b = s_dt + buf * 128;
                     float gv[32];
                     tmem_ld32(tmem + lane_base + COL_G + kb * 32, gv);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int j = kb * 32 + e;
-                        const float m0 = j <= i ? gv[e] * __expf(cs_i - s_cs[j]) * s_dt[j] : 0.f;
-                        const float m1 = j + 1 <= i ? gv[e + 1] * __expf(cs_i - s_cs[j + 1]) * s_dt[j + 1] : 0.f;
+                        const float m0 = e <= lane ? gv[e] * __expf(cs_i - cs_b[j]) * dt_b[j] : 0.f;
+                        const float m1 = e + 1 <= lane ? gv[e + 1] * __expf(cs_i - cs_b[j + 1]) * dt_b[j + 1] : 0.f;
                         packed[e >> 1] = pack_bf2(m0, m1);
                     }
-                } else {
+                } else {  // above the diagonal: zero
 #pragma unroll
                     for (int e = 0; e < 16; ++e) packed[e] = 0u;
                 }
@@ -416,77 +490,89 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[MREADY]);
+            mbar_arrive(&bars[CS_FREE0 + buf]);  // this chunk's dt / cumsum buffer is no longer read
 
-            // (f) state passing: S_run <- exp(cs_last) S_run + S_c  (lane i = state row n)
-            if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
+            // z of row i (this thread's 16 columns) for the epilogue, loaded now to hide the latency
+            uint4 zw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            if (i < Qc) {
+                const uint4* zrow = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.z) +
+                                                                   ((size_t)b * a.L + t0 + i) * a.HP +
+                                                                   (size_t)h * kP + quarter * 16);
+                zw[0] = __ldg(zrow);
+                zw[1] = __ldg(zrow + 1);
+            }
+
+            // (f) state passing: S_run <- exp(cs_last) S_run + S_c  (lane i = state row n; 16 columns p)
+            if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
             {
                 const float dl = __expf(cs_last);
-                const bool last = c == nc - 1;
+                const float2 dl2 = make_float2(dl, dl);
+                float sc[16], sr[16];
+                tmem_ld16(tmem + lane_base + COL_SC + quarter * 16, sc);
+                tmem_ld16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float sc[32], sr[32];
-                    tmem_ld32(tmem + lane_base + COL_SC + half * 32, sc);
-                    tmem_ld32(tmem + lane_base + COL_SRUN + half * 32, sr);
-                    tmem_wait_ld();
+                for (int k = 0; k < 16; k += 2) {
+                    const float2 v = __ffma2_rn(dl2, make_float2(sr[k], sr[k + 1]), make_float2(sc[k], sc[k + 1]));
+                    sr[k] = v.x;
+                    sr[k + 1] = v.y;
+                }
+                tmem_st16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) sr[k] = fmaf(dl, sr[k], sc[k]);
-                    tmem_st32(tmem + lane_base + COL_SRUN + half * 32, sr);
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    uint4 w;
+                    w.x = pack_bf2(sr[k2 * 8 + 0], sr[k2 * 8 + 1]);
+                    w.y = pack_bf2(sr[k2 * 8 + 2], sr[k2 * 8 + 3]);
+                    w.z = pack_bf2(sr[k2 * 8 + 4], sr[k2 * 8 + 5]);
+                    w.w = pack_bf2(sr[k2 * 8 + 6], sr[k2 * 8 + 7]);
+                    *reinterpret_cast<uint4*>(sS + sw128_off(i, quarter * 2 + k2)) = w;
+                }
+                if (c == nc - 1) {
+                    float* fs = a.final_state + ((size_t)b * a.H + h) * kP * kN;
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        uint4 w;
-                        w.x = pack_bf2(sr[k4 * 8 + 0], sr[k4 * 8 + 1]);
-                        w.y = pack_bf2(sr[k4 * 8 + 2], sr[k4 * 8 + 3]);
-                        w.z = pack_bf2(sr[k4 * 8 + 4], sr[k4 * 8 + 5]);
-                        w.w = pack_bf2(sr[k4 * 8 + 6], sr[k4 * 8 + 7]);
-                        *reinterpret_cast<uint4*>(sS + sw128_off(i, half * 4 + k4)) = w;
-                    }
-                    if (last) {
-                        float* fs = a.final_state + ((size_t)b * a.H + h) * kP * kN;
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) fs[(size_t)(half * 32 + k) * kN + i] = sr[k];
-                    }
+                    for (int k = 0; k < 16; ++k) fs[(size_t)(quarter * 16 + k) * kN + i] = sr[k];
                 }
                 tmem_wait_st();
             }
 
-            // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z)
-            if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
+            // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 16*quarter .. +15
+            if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
             {
-                const uint8_t* rz = sm + OFF_RAWZ + s * 16384;
-                TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP;
+                TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
+                float y1[16], y2[16];
+                tmem_ld16(tmem + lane_base + COL_Y + quarter * 16, y1);
+                tmem_ld16(tmem + lane_base + COL_Y2 + quarter * 16, y2);
+                tmem_wait_ld();
+                const float2 e2 = make_float2(ecs, ecs), d2 = make_float2(Dh, Dh);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float y1[32], y2[32];
-                    tmem_ld32(tmem + lane_base + COL_Y + half * 32, y1);
-                    tmem_ld32(tmem + lane_base + COL_Y2 + half * 32, y2);
-                    tmem_wait_ld();
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const uint32_t zr[4] = {zw[k2].x, zw[k2].y, zw[k2].z, zw[k2].w};
+                    float o[8];
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint4 zw = *reinterpret_cast<const uint4*>(rz + sw128_off(i, half * 4 + k4));
-                        const float zv[8] = {bf_lo(zw.x), bf_hi(zw.x), bf_lo(zw.y), bf_hi(zw.y),
-                                             bf_lo(zw.z), bf_hi(zw.z), bf_lo(zw.w), bf_hi(zw.w)};
-                        float o[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int k = k4 * 8 + e;
-                            const float yv = fmaf(ecs, y2[k], y1[k]) + Dh * u[half * 32 + k];
-                            o[e] = yv * silu_f(zv[e]);
-                        }
-                        if (valid) {
-                            if constexpr (sizeof(TY) == 2) {
-                                uint4 w;
-                                w.x = pack_bf2(o[0], o[1]);
-                                w.y = pack_bf2(o[2], o[3]);
-                                w.z = pack_bf2(o[4], o[5]);
-                                w.w = pack_bf2(o[6], o[7]);
-                                *reinterpret_cast<uint4*>(yrow + half * 32 + k4 * 8) = w;
-                            } else {
-                                float4* dst = reinterpret_cast<float4*>(yrow + half * 32 + k4 * 8);
-                                dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-                                dst[1] = make_float4(o[4], o[5], o[6], o[7]);
-                            }
+                    for (int e = 0; e < 8; e += 2) {
+                        const int k = k2 * 8 + e;
+                        const float2 uv = *reinterpret_cast<const float2*>(sU + u_off(i, quarter * 8 + (k >> 1)));
+                        float2 yv = __ffma2_rn(e2, make_float2(y2[k], y2[k + 1]), make_float2(y1[k], y1[k + 1]));
+                        yv = __ffma2_rn(d2, uv, yv);
+                        const float2 gz = silu2(make_float2(bf_lo(zr[e >> 1]), bf_hi(zr[e >> 1])));
+                        const float2 ov = __fmul2_rn(yv, gz);
+                        o[e] = ov.x;
+                        o[e + 1] = ov.y;
+                    }
+                    if (i < Qc) {
+                        if constexpr (sizeof(TY) == 2) {
+                            uint4 w;
+                            w.x = pack_bf2(o[0], o[1]);
+                            w.y = pack_bf2(o[2], o[3]);
+                            w.z = pack_bf2(o[4], o[5]);
+                            w.w = pack_bf2(o[6], o[7]);
+                            *reinterpret_cast<uint4*>(yrow + k2 * 8) = w;
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
+                            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
                         }
                     }
                 }
@@ -503,72 +589,81 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     }
 }
 
-// SiLU(conv4) of the B and C channels into the workspace [b][t][2][G*N] (bf16),
-// plus the conv_state tail of every channel.  Block: 256 threads = 256 channel
-// pairs of one token block; each thread slides a 4-tap window along 64 tokens.
-constexpr int kProTok = 64;
+// SiLU(conv4) of the B and C channels into the workspace [b][t][2][G*N] (bf16).
+// Block: 256 threads = 256 channel
+// pairs (bf16x2) over kProTok tokens; a thread issues all kProTok + 3 loads of
+// its window before the first FMA, so the block's loads are all in flight at once.
+constexpr int kProTok = 16;
 
 __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a) {
     const int64_t b = blockIdx.y;
     const int64_t t0 = (int64_t)blockIdx.x * kProTok;
-    const int pairs = a.GN;  // (2 arrays x GN channels) / 2 per pair
-    const int pair = blockIdx.z * 256 + threadIdx.x;
+    const int half_gn = a.GN / 2;                    // channel pairs per array
+    const int pair = blockIdx.z * 256 + threadIdx.x;  // 0 .. GN-1 over both arrays
     const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.init_conv_state);
-    if (pair < pairs) {
-        const int sel = pair >= a.GN / 2;                      // 0 = B, 1 = C
-        const int ch0 = (pair - sel * (a.GN / 2)) * 2;         // channel within the array
-        const int cglob = a.HP + sel * a.GN + ch0;             // conv channel index
-        const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B);
-        uint32_t* dst = static_cast<uint32_t*>(a.workspace);
+    if (pair < a.GN) {
+        const int sel = pair >= half_gn;                // 0 = B, 1 = C
+        const int cp = pair - sel * half_gn;            // pair index within the array
+        const int cglob = a.HP + sel * a.GN + 2 * cp;   // conv channel of the pair's first element
+        const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B) + (size_t)b * a.L * half_gn + cp;
+        uint32_t* dst = static_cast<uint32_t*>(a.workspace) + ((size_t)b * a.L * 2 + sel) * half_gn + cp;
         const float4 w0 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cglob * 4);
         const float4 w1 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(cglob + 1) * 4);
         const float b0 = a.conv_b[cglob], b1 = a.conv_b[cglob + 1];
-        float h0[3], h1[3];  // window: tokens t-3, t-2, t-1
+        float v0[kProTok + 3], v1[kProTok + 3];  // tokens t0-3 .. t0+kProTok-1
+        uint32_t raw[kProTok + 3];
+#pragma unroll
+        for (int k = 0; k < kProTok + 3; ++k) {
+            const int64_t t = t0 - 3 + k;
+            raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * half_gn] : 0u;
+        }
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int64_t t = t0 - 3 + k;
-            if (t >= 0) {
-                const uint32_t v = src[((size_t)b * a.L + t) * (a.GN / 2) + ch0 / 2];
-                h0[k] = bf_lo(v);
-                h1[k] = bf_hi(v);
-            } else if (hist) {
-                h0[k] = __bfloat162float(hist[((size_t)b * a.conv_dim + cglob) * 3 + (t + 3)]);
-                h1[k] = __bfloat162float(hist[((size_t)b * a.conv_dim + cglob + 1) * 3 + (t + 3)]);
+            if (t < 0 && hist) {
+                v0[k] = __bfloat162float(hist[((size_t)b * a.conv_dim + cglob) * 3 + (t + 3)]);
+                v1[k] = __bfloat162float(hist[((size_t)b * a.conv_dim + cglob + 1) * 3 + (t + 3)]);
             } else {
-                h0[k] = h1[k] = 0.f;
+                v0[k] = bf_lo(raw[k]);
+                v1[k] = bf_hi(raw[k]);
             }
         }
-        const int64_t tend = t0 + kProTok < a.L ? t0 + kProTok : a.L;
-        for (int64_t t = t0; t < tend; ++t) {
-            const uint32_t v = src[((size_t)b * a.L + t) * (a.GN / 2) + ch0 / 2];
-            const float x0 = bf_lo(v), x1 = bf_hi(v);
-            const float p0 = b0 + w0.x * h0[0] + w0.y * h0[1] + w0.z * h0[2] + w0.w * x0;
-            const float p1 = b1 + w1.x * h1[0] + w1.y * h1[1] + w1.z * h1[2] + w1.w * x1;
-            dst[(((size_t)b * a.L + t) * 2 + sel) * (a.GN / 2) + ch0 / 2] = pack_bf2(silu_f(p0), silu_f(p1));
-            h0[0] = h0[1]; h0[1] = h0[2]; h0[2] = x0;
-            h1[0] = h1[1]; h1[1] = h1[2]; h1[2] = x1;
+#pragma unroll
+        for (int k = 3; k < kProTok + 3; ++k) {
+            v0[k] = bf_lo(raw[k]);
+            v1[k] = bf_hi(raw[k]);
         }
-    }
-    // conv_state tail (pre-conv inputs of tokens L-3..L-1) for every channel, by the last token block
-    if (blockIdx.x == gridDim.x - 1 && blockIdx.z == 0) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.conv_state);
-        for (int c = threadIdx.x; c < a.conv_dim; c += 256) {
-            for (int k = 0; k < 3; ++k) {
-                const int64_t t = a.L - 3 + k;
-                __nv_bfloat16 v;
-                if (t >= 0) {
-                    if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[((size_t)b * a.L + t) * a.HP + c];
-                    else if (c < a.HP + a.GN)
-                        v = static_cast<const __nv_bfloat16*>(a.B)[((size_t)b * a.L + t) * a.GN + (c - a.HP)];
-                    else
-                        v = static_cast<const __nv_bfloat16*>(a.C)[((size_t)b * a.L + t) * a.GN + (c - a.HP - a.GN)];
-                } else {
-                    v = hist ? hist[((size_t)b * a.conv_dim + c) * 3 + (t + 3)] : __float2bfloat16_rn(0.f);
-                }
-                out[((size_t)b * a.conv_dim + c) * 3 + k] = v;
+#pragma unroll
+        for (int k = 0; k < kProTok; ++k) {
+            const int64_t t = t0 + k;
+            if (t < a.L) {
+                const float p0 = b0 + w0.x * v0[k] + w0.y * v0[k + 1] + w0.z * v0[k + 2] + w0.w * v0[k + 3];
+                const float p1 = b1 + w1.x * v1[k] + w1.y * v1[k + 1] + w1.z * v1[k + 2] + w1.w * v1[k + 3];
+                dst[(size_t)t * 2 * half_gn] = pack_bf2(silu_f(p0), silu_f(p1));
             }
         }
     }
+}
+
+// conv_state tail: the pre-conv inputs of tokens L-3..L-1 (history-filled when
+// L < 3) of every channel, one element per thread.
+__global__ void __launch_bounds__(256) conv_tail_kernel(PrefillArgs a) {
+    const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    if (e >= a.batch * a.conv_dim * 3) return;
+    const int k = (int)(e % 3);
+    const int c = (int)((e / 3) % a.conv_dim);
+    const int64_t b = e / (3 * (int64_t)a.conv_dim);
+    const int64_t t = a.L - 3 + k;
+    const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.init_conv_state);
+    __nv_bfloat16 v;
+    if (t >= 0) {
+        if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[((size_t)b * a.L + t) * a.HP + c];
+        else if (c < a.HP + a.GN) v = static_cast<const __nv_bfloat16*>(a.B)[((size_t)b * a.L + t) * a.GN + (c - a.HP)];
+        else v = static_cast<const __nv_bfloat16*>(a.C)[((size_t)b * a.L + t) * a.GN + (c - a.HP - a.GN)];
+    } else {
+        v = hist ? hist[((size_t)b * a.conv_dim + c) * 3 + (t + 3)] : __float2bfloat16_rn(0.f);
+    }
+    static_cast<__nv_bfloat16*>(a.conv_state)[e] = v;
 }
 
 // ---- host side ------------------------------------------------------------------------------------------
@@ -614,11 +709,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     if (a.L == 0) return launch_prefill_simt(a, kind, st, hook);  // nothing to scan: states pass through
     TcParams prm;
     prm.a = a;
-    if (!make_map(&prm.tm_x, a.x, a.HP, a.L, a.batch) || !make_map(&prm.tm_z, a.z, a.HP, a.L, a.batch) ||
+    if (!make_map(&prm.tm_x, a.x, a.HP, a.L, a.batch) ||
         !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, a.batch))
         return cudaErrorInvalidValue;
     const dim3 pgrid((unsigned)((a.L + kProTok - 1) / kProTok), (unsigned)a.batch, (unsigned)((a.GN + 255) / 256));
     bc_prologue_kernel<<<pgrid, 256, 0, st>>>(a);
+    const int64_t tail = a.batch * (int64_t)a.conv_dim * 3;
+    conv_tail_kernel<<<(unsigned)((tail + 255) / 256), 256, 0, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     auto kern = kind == ActKind::BF16_YF32 ? chunk_scan_kernel<float> : chunk_scan_kernel<__nv_bfloat16>;
