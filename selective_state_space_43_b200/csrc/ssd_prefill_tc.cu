@@ -22,7 +22,9 @@
 //   conv_tail    the conv_state output (last 3 pre-conv tokens, all channels);
 //   chunk_scan   one CTA per (sequence b, head h) walks the chunks in order;
 //                all accumulators live in TMEM; 7 warps:
-//                  warp 0  TMA producer: raw x tiles (2-stage ring)
+//                  warp 0  TMA producer: raw x tiles (2-stage ring); once a
+//                           chunk's conv has consumed its stage, z of the same
+//                           chunk is loaded into it for the epilogue
 //                  warp 1  TMEM allocator + single-thread tcgen05.mma issuer
 //                  warp 2  TMA producer: post-conv B and C tiles; the whole
 //                           warp also computes each chunk's dt, cumsum of dt*A
@@ -31,16 +33,17 @@
 //                           major (warp = 8 tokens, lane = 2 channels, taps in
 //                           registers); the TMEM phases run row-major, four
 //                           threads per token row i (= TMEM lane i), each owning
-//                           16 columns and one of the 4 decay-mask column blocks:
+//                           16 state / output columns and one 8-column group of
+//                           each of the 4 decay-mask column blocks:
 //                           decay mask, state pass, epilogue (D skip from the
-//                           fp32 conv output, z gate loaded straight from
-//                           global memory, y store).  Elementwise math uses
+//                           fp32 conv output, z gate, y store).  Elementwise math uses
 //                           the packed fp32x2 FMA / MUL of sm_100.
-// The decay mask exp(cs_i - cs_j) is formed per 32-column block: exactly
-// (one exp per element) on the diagonal block, and as the product of a row
+// The decay mask exp(cs_i - cs_j) is formed per 8-column group: exactly (one
+// exp per element) for the rows inside the group, and as the product of a row
 // factor exp(cs_i - cs_r) and a column factor exp(cs_r - cs_j) dt_j, with r the
-// block's last column, below it.  Both factors are <= 1, so neither overflows,
-// and either underflows only where the true product is below ~1e-38.
+// group's last column, for the rows below it.  Both factors are <= 1, so
+// neither overflows, and either underflows only where the true product is
+// below ~1e-38.
 // Every mbarrier wait is bounded; a wait that gives up raises a device error
 // flag (read back by ssd_device_status) and the CTA drains and exits.
 #include <cuda.h>
@@ -69,17 +72,17 @@ constexpr uint32_t OFF_X = 65536;      // X  [j][p] bf16 (MN-major B operand)
 constexpr uint32_t OFF_XP = 81920;     // X' [j][p] bf16
 constexpr uint32_t OFF_M = 98304;      // M  [i][j] bf16, two K blocks of 64 (K-major A operand)
 constexpr uint32_t OFF_S = 131072;     // S_prev [n][p] bf16 (MN-major B operand)
-constexpr uint32_t OFF_RAWX = 147456;  // 2 x raw x tile [tok][p] bf16 (TMA, 128B swizzle)
+constexpr uint32_t OFF_RAWX = 147456;  // 2 stages [tok][p] bf16 (TMA, 128B swizzle): a chunk's raw x, then its z
 constexpr uint32_t OFF_U = 180224;     // post-conv x [tok][p] fp32 for the D skip (256-byte rows, swizzled)
 constexpr uint32_t OFF_SMALL = 212992;
 // small region
 constexpr uint32_t OFF_HALO = OFF_SMALL;           // [2][3][64] bf16 raw x history
 constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;  // cs [2][128] float (double-buffered by chunk parity)
 constexpr uint32_t OFF_DT = OFF_CS + 2 * 128 * 4;      // dt [2][128]
-constexpr uint32_t OFF_COLF = OFF_DT + 2 * 128 * 4;    // column factors of the decay mask [2][128]
+constexpr uint32_t OFF_COLF = OFF_DT + 2 * 128 * 4;    // column factors of the decay mask [2][128] (8-col groups)
 constexpr uint32_t OFF_WX = OFF_COLF + 2 * 128 * 4;    // weight of x_j in the chunk state [2][128]
 constexpr uint32_t OFF_BAR = OFF_WX + 2 * 128 * 4;     // mbarriers (8 B each)
-constexpr int NBAR = 16;
+constexpr int NBAR = 18;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;  // TMEM base address
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
@@ -87,22 +90,22 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 enum Bar { FULL_RAW0 = 0, FULL_RAW1, EMPTY_RAW0, EMPTY_RAW1, FULL_BC, EMPTY_BC, XREADY, MREADY, G_FULL, SC_FULL,
-           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1 };
+           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, FULL_Z0, FULL_Z1 };
 
 // TMEM columns (fp32 accumulators, 128 lanes)
 constexpr uint32_t COL_G = 0, COL_Y = 128, COL_Y2 = 192, COL_SC = 256, COL_SRUN = 320, TMEM_COLS = 512;
 
 struct TcParams {
     PrefillArgs a;
-    CUtensorMap tm_x, tm_bc;
+    CUtensorMap tm_x, tm_z, tm_bc;
 };
 
 // Byte offset of the float2 `pair` (0..31) of row `row` in the fp32 [128][64]
-// conv-output tile: 256-byte rows, 16-byte chunks XOR-swizzled by the row so that
-// a warp reading 32 consecutive rows at one column, or writing one row, is conflict-free.
+// conv-output tile: 256-byte rows whose 8-byte slots are XOR-swizzled by the row,
+// so that a warp reading one column of 32 consecutive rows, or writing one row,
+// touches every bank exactly twice (the minimum for 256 bytes).
 __device__ __forceinline__ uint32_t u_off(uint32_t row, uint32_t pair) {
-    const uint32_t chunk = pair >> 1;  // 16-byte chunk (0..15)
-    return row * 256u + (((chunk ^ (row & 15u)) << 4) | ((pair & 1u) << 3));
+    return row * 256u + ((pair ^ (row & 31u)) << 3);
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -180,6 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         mbar_init(&bars[CS_READY1], 32);
         mbar_init(&bars[CS_FREE0], kComputeThreads);
         mbar_init(&bars[CS_FREE1], kComputeThreads);
+        mbar_init(&bars[FULL_Z0], 1);
+        mbar_init(&bars[FULL_Z1], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -206,23 +211,38 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     const uint32_t tmem = *tmem_holder;
 
     if (warp == kWarpRaw) {
-        // ---------------- raw x producer ----------------
+        // ---------------- raw x / z producer ----------------
         if (lane == 0) {
             prefetch_tmap(&prm.tm_x);
-            int issued[2] = {-1, -1};
-            for (int c = 0; c < nc; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !mbar_wait(&bars[EMPTY_RAW0 + s], ((c >> 1) + 1) & 1, abort_flag)) {
-                    raise_abort(abort_flag);
-                    break;
+            prefetch_tmap(&prm.tm_z);
+            int issued_x[2] = {-1, -1}, issued_z[2] = {-1, -1};
+            for (int c = 0; c <= nc; ++c) {
+                if (c < nc) {  // x of chunk c into stage c & 1, once chunk c-2 (its z) is fully consumed
+                    const int s = c & 1;
+                    if (c >= 2 && !mbar_wait(&bars[EMPTY_RAW0 + s], ((c >> 1) + 1) & 1, abort_flag)) {
+                        raise_abort(abort_flag);
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384);
+                    tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, c * kQ, b);
+                    issued_x[s] = c;
                 }
-                mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384);
-                tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, c * kQ, b);
-                issued[s] = c;
+                if (c >= 1) {  // z of chunk c-1 into its stage, once that chunk's conv has read the x there
+                    const int cz = c - 1, s = cz & 1;
+                    if (!mbar_wait(&bars[XREADY], cz & 1, abort_flag)) {
+                        raise_abort(abort_flag);
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars[FULL_Z0 + s], 16384);
+                    tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_z, &bars[FULL_Z0 + s], h * kP, cz * kQ, b);
+                    issued_z[s] = cz;
+                }
             }
             if (*abort_flag) {  // let copies still in flight land before the CTA exits
-                for (int s = 0; s < 2; ++s)
-                    if (issued[s] >= 0) mbar_wait(&bars[FULL_RAW0 + s], (issued[s] >> 1) & 1, nullptr, 100000000ull);
+                for (int s = 0; s < 2; ++s) {
+                    if (issued_x[s] >= 0) mbar_wait(&bars[FULL_RAW0 + s], (issued_x[s] >> 1) & 1, nullptr, 100000000ull);
+                    if (issued_z[s] >= 0) mbar_wait(&bars[FULL_Z0 + s], (issued_z[s] >> 1) & 1, nullptr, 100000000ull);
+                }
             }
         }
     } else if (warp == kWarpBc) {
@@ -241,21 +261,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         if (lane == 0) prefetch_tmap(&prm.tm_bc);
         int last = -1;
         for (int c = 0; c < nc; ++c) {
-            int okc = 1;
-            if (lane == 0) {
-                if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) {
-                    okc = 0;
-                } else {
-                    mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
-                    const int xc = a.GN + g * kN, xb = g * kN;
-                    tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, c * kQ, b);
-                    tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, c * kQ, b);
-                    tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, c * kQ, b);
-                    tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, c * kQ, b);
-                    last = c;
-                }
-            }
-            if (!__shfl_sync(0xffffffffu, okc, 0)) { raise_abort(abort_flag); break; }
             // dt = softplus(dt_raw + bias) and the inclusive cumsum of dt*A over the chunk's 128 rows,
             // into the buffer of this chunk's parity once every compute thread is done with it
             const int buf = c & 1;
@@ -282,17 +287,33 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
             const float excl = incl - run;
             const float cs_last = __shfl_sync(0xffffffffu, incl, 31);
-            const float cs_blk = __shfl_sync(0xffffffffu, incl, lane | 7);  // cs at the last row of the 32-row block
+            // cs at the last row of the 8-row group (rows 8m .. 8m+7 live on lanes 2m, 2m+1)
+            const float cs_g8 = __shfl_sync(0xffffffffu, incl, lane | 1);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int r = 4 * lane + k;
                 const float csr = cs[k] + excl;
                 s_cs[buf * 128 + r] = csr;
                 s_dt[buf * 128 + r] = dtv[k];
-                s_colf[buf * 128 + r] = __expf(cs_blk - csr) * dtv[k];
+                s_colf[buf * 128 + r] = __expf(cs_g8 - csr) * dtv[k];
                 s_wx[buf * 128 + r] = __expf(cs_last - csr) * dtv[k];
             }
             mbar_arrive(&bars[CS_READY0 + buf]);
+            int okc = 1;
+            if (lane == 0) {
+                if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) {
+                    okc = 0;
+                } else {
+                    mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
+                    const int xc = a.GN + g * kN, xb = g * kN;
+                    tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, c * kQ, b);
+                    tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, c * kQ, b);
+                    tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, c * kQ, b);
+                    tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, c * kQ, b);
+                    last = c;
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, okc, 0)) { raise_abort(abort_flag); break; }
         }
         if (lane == 0 && *abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
     } else if (warp == kWarpMma) {
@@ -412,6 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     raw[k] = r >= 0 ? *reinterpret_cast<const uint32_t*>(rx + sw128_off(r, lane >> 2) + lane_byte)
                                     : halo_in[(r + 3) * 32 + lane];
                 }
+                float2 xv[11];
+#pragma unroll
+                for (int k = 0; k < 11; ++k) xv[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
+                float2 uvs[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int r = r0 + k;
@@ -419,10 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     float2 uv = make_float2(0.f, 0.f);
                     if (r < Qc) {  // warp-uniform
                         float2 acc = cbias;
-                        acc = __ffma2_rn(tap0, make_float2(bf_lo(raw[k + 0]), bf_hi(raw[k + 0])), acc);
-                        acc = __ffma2_rn(tap1, make_float2(bf_lo(raw[k + 1]), bf_hi(raw[k + 1])), acc);
-                        acc = __ffma2_rn(tap2, make_float2(bf_lo(raw[k + 2]), bf_hi(raw[k + 2])), acc);
-                        acc = __ffma2_rn(tap3, make_float2(bf_lo(raw[k + 3]), bf_hi(raw[k + 3])), acc);
+                        acc = __ffma2_rn(tap0, xv[k + 0], acc);
+                        acc = __ffma2_rn(tap1, xv[k + 1], acc);
+                        acc = __ffma2_rn(tap2, xv[k + 2], acc);
+                        acc = __ffma2_rn(tap3, xv[k + 3], acc);
                         uv = silu2(acc);
                         const float wxr = wx_b[r];
                         xo = pack_bf2(uv.x, uv.y);
@@ -432,8 +457,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     const uint32_t off = sw128_off(r, lane >> 2) + lane_byte;
                     *reinterpret_cast<uint32_t*>(sX + off) = xo;
                     *reinterpret_cast<uint32_t*>(sXp + off) = xpo;
-                    *reinterpret_cast<float2*>(sU + u_off(r, lane)) = uv;
+                    uvs[k] = uv;
                 }
+                // the fp32 tile is still read by the previous chunk's epilogue in other warps:
+                // overwrite it only once every compute thread has finished that epilogue
+                if (c >= 1 && !warp_wait(&bars[EMPTY_RAW0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag)) {
+                    raise_abort(abort_flag);
+                    break;
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) *reinterpret_cast<float2*>(sU + u_off(r0 + k, lane)) = uvs[k];
                 if (wc == 15) {  // raw history (rows 125..127) of the next chunk
                     uint32_t* halo_out = reinterpret_cast<uint32_t*>(sm + OFF_HALO) + ((c + 1) & 1) * 96;
                     halo_out[0 * 32 + lane] = raw[8];
@@ -445,62 +478,57 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             tc_fence_before();
             mbar_arrive(&bars[XREADY]);
 
-            // (e) decay mask, column block kb = quarter of row i
+            // (e) decay mask of row i, columns 8*quarter .. +7 of each 32-column block
             if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
             {
-                const int kb = quarter;
-                uint32_t packed[16];
-                if (kb < q) {  // strictly below the diagonal: row factor x column factor
-                    const float rowf = __expf(cs_i - cs_b[kb * 32 + 31]);
-                    const float2 rf = make_float2(rowf, rowf);
-                    float gv[32];
-                    tmem_ld32(tmem + lane_base + COL_G + kb * 32, gv);
-                    tmem_wait_ld();
-                    const float2* colf = reinterpret_cast<const float2*>(s_colf + buf * 128 + kb * 32);
+                const float* dt_b = s_dt + buf * 128;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float2 m = __fmul2_rn(__fmul2_rn(make_float2(gv[e], gv[e + 1]), colf[e >> 1]), rf);
-                        packed[e >> 1] = pack_bf2(m.x, m.y);
-                    }
-                } else if (kb == q) {  // diagonal block: exact decay for j <= i
-                    const float* dt_b = s_dt + buf * 128;
-                    float gv[32];
-                    tmem_ld32(tmem + lane_base + COL_G + kb * 32, gv);
+                for (int kp = 0; kp < 4; kp += 2) {  // two 8-column groups per TMEM round trip
+                    float gv[2][8];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)  // warp-uniform: groups right of the diagonal block are zero
+                        if (kp + t <= q) tmem_ld8(tmem + lane_base + COL_G + (kp + t) * 32 + quarter * 8, gv[t]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int j = kb * 32 + e;
-                        const float m0 = e <= lane ? gv[e] * __expf(cs_i - cs_b[j]) * dt_b[j] : 0.f;
-                        const float m1 = e + 1 <= lane ? gv[e + 1] * __expf(cs_i - cs_b[j + 1]) * dt_b[j + 1] : 0.f;
-                        packed[e >> 1] = pack_bf2(m0, m1);
+                    for (int t = 0; t < 2; ++t) {
+                        const int kb = kp + t;
+                        const int j0 = kb * 32 + quarter * 8;  // first column of this 8-column group
+                        uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+                        if (kb <= q) {
+                            float m[8];
+                            if (i > j0 + 7) {
+                                // below the group: exp(cs_i - cs_j) = exp(cs_i - cs_r) exp(cs_r - cs_j), r = j0 + 7
+                                const float rowf = __expf(cs_i - cs_b[j0 + 7]);
+                                const float2 rf = make_float2(rowf, rowf);
+                                const float2* colf = reinterpret_cast<const float2*>(s_colf + buf * 128 + j0);
+#pragma unroll
+                                for (int e = 0; e < 8; e += 2) {
+                                    const float2 v =
+                                        __fmul2_rn(__fmul2_rn(make_float2(gv[t][e], gv[t][e + 1]), colf[e >> 1]), rf);
+                                    m[e] = v.x;
+                                    m[e + 1] = v.y;
+                                }
+                            } else {
+                                // the group holds the diagonal (or lies right of it): exact decay for j <= i
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    const int j = j0 + e;
+                                    m[e] = j <= i ? gv[t][e] * __expf(cs_i - cs_b[j]) * dt_b[j] : 0.f;
+                                }
+                            }
+                            packed = make_uint4(pack_bf2(m[0], m[1]), pack_bf2(m[2], m[3]), pack_bf2(m[4], m[5]),
+                                                pack_bf2(m[6], m[7]));
+                        }
+                        *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 + sw128_off(i, (kb & 1) * 4 + quarter)) =
+                            packed;
                     }
-                } else {  // above the diagonal: zero
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) packed[e] = 0u;
-                }
-                uint8_t* mrow = sMm + (kb >> 1) * 16384;
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const int chunk = (kb & 1) * 4 + k4;
-                    *reinterpret_cast<uint4*>(mrow + sw128_off(i, chunk)) =
-                        make_uint4(packed[k4 * 4 + 0], packed[k4 * 4 + 1], packed[k4 * 4 + 2], packed[k4 * 4 + 3]);
                 }
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[MREADY]);
             mbar_arrive(&bars[CS_FREE0 + buf]);  // this chunk's dt / cumsum buffer is no longer read
-
-            // z of row i (this thread's 16 columns) for the epilogue, loaded now to hide the latency
-            uint4 zw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-            if (i < Qc) {
-                const uint4* zrow = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.z) +
-                                                                   ((size_t)b * a.L + t0 + i) * a.HP +
-                                                                   (size_t)h * kP + quarter * 16);
-                zw[0] = __ldg(zrow);
-                zw[1] = __ldg(zrow + 1);
-            }
 
             // (f) state passing: S_run <- exp(cs_last) S_run + S_c  (lane i = state row n; 16 columns p)
             if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
@@ -537,9 +565,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
 
             // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 16*quarter .. +15
+            if (!warp_wait(&bars[FULL_Z0 + s], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
             if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
             {
+                const uint8_t* rz = sm + OFF_RAWX + s * 16384;
+                const uint4 zw[2] = {*reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2)),
+                                     *reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2 + 1))};
                 TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
                 float y1[16], y2[16];
                 tmem_ld16(tmem + lane_base + COL_Y + quarter * 16, y1);
@@ -709,7 +741,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     if (a.L == 0) return launch_prefill_simt(a, kind, st, hook);  // nothing to scan: states pass through
     TcParams prm;
     prm.a = a;
-    if (!make_map(&prm.tm_x, a.x, a.HP, a.L, a.batch) ||
+    if (!make_map(&prm.tm_x, a.x, a.HP, a.L, a.batch) || !make_map(&prm.tm_z, a.z, a.HP, a.L, a.batch) ||
         !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, a.batch))
         return cudaErrorInvalidValue;
     const dim3 pgrid((unsigned)((a.L + kProTok - 1) / kProTok), (unsigned)a.batch, (unsigned)((a.GN + 255) / 256));
