@@ -185,6 +185,13 @@ def barrier(world):
         dist.barrier()
 
 
+def weak_scaling_value(tokens_per_rank: int, ms_per_rank: float, world: int, device) -> tuple[float, float]:
+    """Whole-job tokens/s for independent per-rank work: all ranks' tokens over the
+    slowest rank's step time.  Returns (tokens/s, max ms)."""
+    ms = max_over_ranks(ms_per_rank, world, device)
+    return tokens_per_rank * world / (ms * 1e-3), ms
+
+
 def max_over_ranks(value: float, world: int, device) -> float:
     if world == 1:
         return value
@@ -329,9 +336,8 @@ def main():
     ops.set_timing_events(None, None)
     step_ms = sum(s.elapsed_time(e) for s, e in zip(st, en)) / K
     kern_ms = sum(s.elapsed_time(e) for s, e in zip(ks, ke)) / K
-    step_ms_max = max_over_ranks(step_ms, world, dev)
     tokens_per_rank = d.batch * d.seqlen
-    value = tokens_per_rank * world / (step_ms_max * 1e-3)
+    value, step_ms_max = weak_scaling_value(tokens_per_rank, step_ms, world, dev)
 
     act_bytes = 2 if act == torch.bfloat16 else 4
     pbytes = prefill_bytes(d, act_bytes, w["init_state"])

@@ -1,0 +1,63 @@
+"""Host-side logic of the multi-GPU bench (one process per GPU, independent
+sequences per rank, max-over-ranks timing), exercised with 2 gloo ranks on CPU."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank(rank, world, port, out):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port))
+    w, r, local = bench.dist_setup()
+    assert (w, r, local) == (world, rank, rank)
+    bench.barrier(w)
+    # rank 1 is the slower one: the job's step time is the max, tokens add up over ranks
+    value, ms = bench.weak_scaling_value(4096, 1.0 + rank, w, torch.device("cpu"))
+    out[rank] = (value, ms)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_rank_weak_scaling_aggregation():
+    if not torch.distributed.is_gloo_available():
+        pytest.skip("gloo backend not available")
+    world, port = 2, _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
+    for r in range(world):
+        value, ms = out[r]
+        assert ms == pytest.approx(2.0)
+        assert value == pytest.approx(2 * 4096 / 2.0e-3)
+
+
+def test_single_rank_needs_no_process_group():
+    os.environ.pop("WORLD_SIZE", None)
+    w, r, local = bench.dist_setup()
+    assert (w, r) == (1, 0)
+    value, ms = bench.weak_scaling_value(4096, 0.5, 1, torch.device("cpu"))
+    assert ms == 0.5 and value == pytest.approx(4096 / 0.5e-3)
+
+
+def test_algorithmic_byte_and_flop_counts_match_the_survey_figures():
+    from selective_state_space_43_b200.synth import WORKLOADS
+    d = WORKLOADS["nemotron_h_8b"]["dims"]
+    # 53,504 B per token of activations plus the 4.19 MB final state and the conv tail
+    assert bench.prefill_bytes(d, 2, False) == 4096 * 53504 + 128 * 64 * 128 * 4 + 10240 * 3 * 2
+    assert bench.prefill_flops(d) == 4096 * 6553600
+    dd = WORKLOADS["decode_nemotron_h_8b"]["dims"]
+    total, _ = bench.decode_bytes(dd, 2)
+    assert abs(total / 1e6 - 2192.6) < 0.1
