@@ -68,15 +68,16 @@ constexpr int kComputeThreads = 512;  // 16 warps: four per TMEM lane quadrant
 // shared memory map (bytes from a 1024-byte aligned base)
 constexpr uint32_t OFF_C = 0;          // u_C tile: two boxes [128 tok][64 n] bf16, 128B swizzle
 constexpr uint32_t OFF_B = 32768;      // u_B tile
-constexpr uint32_t OFF_X = 65536;      // X  [j][p] bf16 (MN-major B operand)
-constexpr uint32_t OFF_XP = 81920;     // X' [j][p] bf16
-constexpr uint32_t OFF_M = 98304;      // M  [i][j] bf16, two K blocks of 64 (K-major A operand)
-constexpr uint32_t OFF_S = 131072;     // S_prev [n][p] bf16 (MN-major B operand)
-constexpr uint32_t OFF_RAWX = 147456;  // 2 stages [tok][p] bf16 (TMA, 128B swizzle): a chunk's raw x, then its z
-constexpr uint32_t OFF_U = 180224;     // post-conv x [tok][p] fp32 for the D skip (256-byte rows, swizzled)
+constexpr uint32_t OFF_X = 65536;      // 2 x X [j][p] bf16 (MN-major B operand), by chunk parity
+constexpr uint32_t OFF_XP = 98304;     // X' [j][p] bf16
+constexpr uint32_t OFF_M = 114688;     // M  [i][j] bf16, two K blocks of 64 (K-major A operand)
+constexpr uint32_t OFF_S = 147456;     // 2 x S_prev [n][p] bf16 (MN-major B operand), by chunk parity
+constexpr uint32_t OFF_RAWX = 180224;  // 2 stages [tok][p] bf16 (TMA, 128B swizzle): a chunk's x, then its z, then its y
 constexpr uint32_t OFF_SMALL = 212992;
 // small region
-constexpr uint32_t OFF_HALO = OFF_SMALL;           // [2][3][64] bf16 raw x history
+constexpr uint32_t OFF_WT = OFF_SMALL;                 // conv taps of the head's x channels [4][64] float
+constexpr uint32_t OFF_CB = OFF_WT + 4 * 64 * 4;       // conv bias [64] float
+constexpr uint32_t OFF_HALO = OFF_CB + 64 * 4;         // [2][3][64] bf16 raw x history
 constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;  // cs [2][128] float (double-buffered by chunk parity)
 constexpr uint32_t OFF_DT = OFF_CS + 2 * 128 * 4;      // dt [2][128]
 constexpr uint32_t OFF_COLF = OFF_DT + 2 * 128 * 4;    // column factors of the decay mask [2][128] (8-col groups)
@@ -92,21 +93,14 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 enum Bar { FULL_RAW0 = 0, FULL_RAW1, EMPTY_RAW0, EMPTY_RAW1, FULL_BC, EMPTY_BC, XREADY, MREADY, G_FULL, SC_FULL,
            Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, FULL_Z0, FULL_Z1 };
 
-// TMEM columns (fp32 accumulators, 128 lanes)
-constexpr uint32_t COL_G = 0, COL_Y = 128, COL_Y2 = 192, COL_SC = 256, COL_SRUN = 320, TMEM_COLS = 512;
+// TMEM columns (fp32, 128 lanes): G = C B^T, Y = M X, Y2 = C S^T, S_c, the running state, and the
+// post-conv x of two chunks (for the D skip)
+constexpr uint32_t COL_G = 0, COL_Y = 128, COL_Y2 = 192, COL_SC = 256, COL_SRUN = 320, COL_U = 384, TMEM_COLS = 512;
 
 struct TcParams {
     PrefillArgs a;
-    CUtensorMap tm_x, tm_z, tm_bc;
+    CUtensorMap tm_x, tm_z, tm_y, tm_bc;
 };
-
-// Byte offset of the float2 `pair` (0..31) of row `row` in the fp32 [128][64]
-// conv-output tile: 256-byte rows whose 8-byte slots are XOR-swizzled by the row,
-// so that a warp reading one column of 32 consecutive rows, or writing one row,
-// touches every bank exactly twice (the minimum for 256 bytes).
-__device__ __forceinline__ uint32_t u_off(uint32_t row, uint32_t pair) {
-    return row * 256u + ((pair ^ (row & 31u)) << 3);
-}
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -143,9 +137,89 @@ __device__ __forceinline__ float2 silu2(float2 v) {
     return __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
 }
 
+__device__ __forceinline__ float s_wx_at(const uint8_t* sm, int buf, int row) {
+    return reinterpret_cast<const float*>(sm + OFF_WX)[buf * 128 + row];
+}
+
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
     *abort_flag = 1;
     atomicExch(&g_tc_error, 1);
+}
+
+// Row-major x conv of chunk cc for the calling thread: token row i, channels 16*quarter .. +15.
+// Writes X and X' (bf16, smem operands) and the fp32 conv output into TMEM (for the D skip), and the
+// raw history of the next chunk.  Returns false if a wait gave up.
+__device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, uint64_t* bars, volatile int* abort_flag,
+                                           uint32_t tmem, uint32_t lane_base, int cc, int nc, int i, int quarter) {
+    const int buf = cc & 1;
+    if (!warp_wait(&bars[CS_READY0 + buf], (cc >> 1) & 1, abort_flag)) return false;
+    if (!warp_wait(&bars[FULL_RAW0 + buf], (cc >> 1) & 1, abort_flag)) return false;
+    // the raw history rows were written by other threads in the previous chunk's conv
+    if (cc >= 1 && !warp_wait(&bars[XREADY], (cc - 1) & 1, abort_flag)) return false;
+    const int64_t t0 = (int64_t)cc * kQ;
+    const int Qc = (int)(a.L - t0 < kQ ? a.L - t0 : kQ);
+    const bool valid = i < Qc;
+    const uint8_t* rx = sm + OFF_RAWX + buf * 16384;
+    const uint4* halo_in = reinterpret_cast<const uint4*>(sm + OFF_HALO + (cc & 1) * 384);
+    const float4* wt = reinterpret_cast<const float4*>(sm + OFF_WT);   // [tap][64 channels]
+    const float4* cb = reinterpret_cast<const float4*>(sm + OFF_CB);
+    float2 acc[8];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float4 bv = cb[quarter * 4 + m];
+        acc[2 * m] = make_float2(bv.x, bv.y);
+        acc[2 * m + 1] = make_float2(bv.z, bv.w);
+    }
+#pragma unroll
+    for (int tap = 0; tap < 4; ++tap) {
+        const int r = i - 3 + tap;
+        uint4 w[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            w[k] = r >= 0 ? *reinterpret_cast<const uint4*>(rx + sw128_off(r, quarter * 2 + k))
+                          : halo_in[(r + 3) * 8 + quarter * 2 + k];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float4 tv = wt[tap * 16 + quarter * 4 + m];
+            const uint32_t lo = (m & 1) ? w[m >> 1].z : w[m >> 1].x;
+            const uint32_t hi = (m & 1) ? w[m >> 1].w : w[m >> 1].y;
+            acc[2 * m] = __ffma2_rn(make_float2(tv.x, tv.y), make_float2(bf_lo(lo), bf_hi(lo)), acc[2 * m]);
+            acc[2 * m + 1] = __ffma2_rn(make_float2(tv.z, tv.w), make_float2(bf_lo(hi), bf_hi(hi)), acc[2 * m + 1]);
+        }
+    }
+    const float wxr = s_wx_at(sm, buf, i);
+    float u[16];
+    uint32_t xo[8], xpo[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float2 uv = valid ? silu2(acc[k]) : make_float2(0.f, 0.f);
+        u[2 * k] = uv.x;
+        u[2 * k + 1] = uv.y;
+        xo[k] = pack_bf2(uv.x, uv.y);
+        const float2 up = __fmul2_rn(uv, make_float2(wxr, wxr));
+        xpo[k] = pack_bf2(up.x, up.y);
+    }
+    tmem_st16(tmem + lane_base + COL_U + buf * 64 + quarter * 16, u);
+    uint8_t* sX = sm + OFF_X + buf * 16384;
+    uint8_t* sXp = sm + OFF_XP;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        *reinterpret_cast<uint4*>(sX + sw128_off(i, quarter * 2 + k)) =
+            make_uint4(xo[4 * k], xo[4 * k + 1], xo[4 * k + 2], xo[4 * k + 3]);
+        *reinterpret_cast<uint4*>(sXp + sw128_off(i, quarter * 2 + k)) =
+            make_uint4(xpo[4 * k], xpo[4 * k + 1], xpo[4 * k + 2], xpo[4 * k + 3]);
+    }
+    if (i >= kQ - 3 && cc + 1 < nc) {  // raw history (rows 125..127) of the next chunk
+        uint4* halo_out = reinterpret_cast<uint4*>(sm + OFF_HALO + ((cc + 1) & 1) * 384);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            halo_out[(i - (kQ - 3)) * 8 + quarter * 2 + k] = *reinterpret_cast<const uint4*>(rx + sw128_off(i, quarter * 2 + k));
+    }
+    tmem_wait_st();
+    fence_async_smem();
+    tc_fence_before();
+    mbar_arrive(&bars[XREADY]);
+    return true;
 }
 
 template <typename TY>
@@ -160,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     float* s_dt = reinterpret_cast<float*>(sm + OFF_DT);
     float* s_colf = reinterpret_cast<float*>(sm + OFF_COLF);
     float* s_wx = reinterpret_cast<float*>(sm + OFF_WX);
+    constexpr bool kTmaStoreY = sizeof(TY) == 2;  // bf16 y goes out through TMA from the stage it was written in
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
@@ -167,24 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     const int nc = (int)a.nchunks;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[FULL_RAW0], 1);
-        mbar_init(&bars[FULL_RAW1], 1);
-        mbar_init(&bars[EMPTY_RAW0], kComputeThreads);
-        mbar_init(&bars[EMPTY_RAW1], kComputeThreads);
-        mbar_init(&bars[FULL_BC], 1);
-        mbar_init(&bars[EMPTY_BC], 1);
-        mbar_init(&bars[XREADY], kComputeThreads);
-        mbar_init(&bars[MREADY], kComputeThreads);
-        mbar_init(&bars[G_FULL], 1);
-        mbar_init(&bars[SC_FULL], 1);
-        mbar_init(&bars[Y_FULL], 1);
-        mbar_init(&bars[MMA_DONE], 1);
-        mbar_init(&bars[CS_READY0], 32);
-        mbar_init(&bars[CS_READY1], 32);
-        mbar_init(&bars[CS_FREE0], kComputeThreads);
-        mbar_init(&bars[CS_FREE1], kComputeThreads);
-        mbar_init(&bars[FULL_Z0], 1);
-        mbar_init(&bars[FULL_Z1], 1);
+        for (int k = 0; k < NBAR; ++k) {
+            uint32_t cnt = 1;
+            if (k == EMPTY_RAW0 || k == EMPTY_RAW1 || k == XREADY || k == MREADY || k == CS_FREE0 || k == CS_FREE1)
+                cnt = kComputeThreads;
+            if (k == CS_READY0 || k == CS_READY1) cnt = 32;
+            mbar_init(&bars[k], cnt);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -195,8 +259,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     if (warp >= kFirstCompute) {
         const int i = threadIdx.x - kFirstCompute * 32;
         if (i < kP) {
-            // conv history of token 0: the initial conv state (tokens -3..-1) or zeros
             const int ch = h * kP + i;
+            // conv taps [tap][channel], bias, and the history of token 0 (initial conv state or zeros)
+            const float4 w4 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)ch * 4);
+            float* wt = reinterpret_cast<float*>(sm + OFF_WT);
+            wt[0 * 64 + i] = w4.x;
+            wt[1 * 64 + i] = w4.y;
+            wt[2 * 64 + i] = w4.z;
+            wt[3 * 64 + i] = w4.w;
+            reinterpret_cast<float*>(sm + OFF_CB)[i] = a.conv_b[ch];
             __nv_bfloat16* halo = reinterpret_cast<__nv_bfloat16*>(sm + OFF_HALO);
             for (int k = 0; k < 3; ++k) {
                 __nv_bfloat16 v = __float2bfloat16_rn(0.f);
@@ -211,33 +282,39 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     const uint32_t tmem = *tmem_holder;
 
     if (warp == kWarpRaw) {
-        // ---------------- raw x / z producer ----------------
+        // ---------------- raw x / z producer, y store ----------------
+        // Stage c&1 holds x(c) until chunk c's conv has read it, then z(c) until chunk c's
+        // epilogue has read it (and written y(c) over it), then y(c) until it is stored.
         if (lane == 0) {
             prefetch_tmap(&prm.tm_x);
             prefetch_tmap(&prm.tm_z);
             int issued_x[2] = {-1, -1}, issued_z[2] = {-1, -1};
-            for (int c = 0; c <= nc; ++c) {
-                if (c < nc) {  // x of chunk c into stage c & 1, once chunk c-2 (its z) is fully consumed
-                    const int s = c & 1;
-                    if (c >= 2 && !mbar_wait(&bars[EMPTY_RAW0 + s], ((c >> 1) + 1) & 1, abort_flag)) {
-                        raise_abort(abort_flag);
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384);
-                    tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, c * kQ, b);
-                    issued_x[s] = c;
-                }
-                if (c >= 1) {  // z of chunk c-1 into its stage, once that chunk's conv has read the x there
-                    const int cz = c - 1, s = cz & 1;
-                    if (!mbar_wait(&bars[XREADY], cz & 1, abort_flag)) {
-                        raise_abort(abort_flag);
-                        break;
-                    }
+            bool ok = true;
+            for (int it = 0; it <= nc + 1 && ok; ++it) {
+                if (it >= 1 && it <= nc) {  // z(it-1), once its conv has consumed x(it-1)
+                    const int cz = it - 1, s = cz & 1;
+                    if (!mbar_wait(&bars[XREADY], cz & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
                     mbar_arrive_expect_tx(&bars[FULL_Z0 + s], 16384);
                     tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_z, &bars[FULL_Z0 + s], h * kP, cz * kQ, b);
                     issued_z[s] = cz;
                 }
+                if (it >= 2) {  // y(it-2) out of its stage, once its epilogue is complete
+                    const int cy = it - 2, s = cy & 1;
+                    if (!mbar_wait(&bars[EMPTY_RAW0 + s], (cy >> 1) & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
+                    if constexpr (kTmaStoreY) {
+                        tma_store_3d(&prm.tm_y, sm + OFF_RAWX + s * 16384, h * kP, cy * kQ, b);
+                        bulk_commit();
+                        bulk_wait_read_all();  // the stage may be refilled once the store has read it
+                    }
+                }
+                if (it < nc) {  // x(it) into its stage
+                    const int s = it & 1;
+                    mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384);
+                    tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, it * kQ, b);
+                    issued_x[s] = it;
+                }
             }
+            if constexpr (kTmaStoreY) bulk_wait_all();
             if (*abort_flag) {  // let copies still in flight land before the CTA exits
                 for (int s = 0; s < 2; ++s) {
                     if (issued_x[s] >= 0) mbar_wait(&bars[FULL_RAW0 + s], (issued_x[s] >> 1) & 1, nullptr, 100000000ull);
@@ -246,18 +323,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
         }
     } else if (warp == kWarpBc) {
-        // ---------------- post-conv B / C producer + the chunk's dt / cumsum ----------------
+        // ---------------- chunk dt / cumsum (whole warp) + post-conv B / C producer (lane 0) ----------------
         const float A = a.A[h], dtb = a.dt_bias[h];
         const __nv_bfloat16* dtp = static_cast<const __nv_bfloat16*>(a.dt);
-        float dt_next[4];
-        auto load_dt = [&](int cc) {  // dt of rows 4*lane .. 4*lane+3 of chunk cc
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int64_t t = (int64_t)cc * kQ + 4 * lane + k;
-                dt_next[k] = t < a.L ? __bfloat162float(dtp[((size_t)b * a.L + t) * a.H + h]) : 0.f;
-            }
-        };
-        load_dt(0);
+        // dt of rows 4*lane .. 4*lane+3, loaded one chunk ahead
+        float dn0, dn1, dn2, dn3;
+#define SSD_LOAD_DT(CC)                                                                                  \
+    do {                                                                                                 \
+        const int64_t tb = (int64_t)(CC) * kQ + 4 * lane;                                               \
+        const __nv_bfloat16* p = dtp + ((size_t)b * a.L + tb) * a.H + h;                                \
+        dn0 = tb + 0 < a.L ? __bfloat162float(p[0]) : 0.f;                                               \
+        dn1 = tb + 1 < a.L ? __bfloat162float(p[a.H]) : 0.f;                                             \
+        dn2 = tb + 2 < a.L ? __bfloat162float(p[2 * a.H]) : 0.f;                                         \
+        dn3 = tb + 3 < a.L ? __bfloat162float(p[3 * a.H]) : 0.f;                                         \
+    } while (0)
+        SSD_LOAD_DT(0);
         if (lane == 0) prefetch_tmap(&prm.tm_bc);
         int last = -1;
         for (int c = 0; c < nc; ++c) {
@@ -269,8 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 break;
             }
             const int Qc = (int)(a.L - (int64_t)c * kQ < kQ ? a.L - (int64_t)c * kQ : kQ);
-            float dr[4] = {dt_next[0], dt_next[1], dt_next[2], dt_next[3]};
-            if (c + 1 < nc) load_dt(c + 1);
+            const float dr[4] = {dn0, dn1, dn2, dn3};
+            if (c + 1 < nc) SSD_LOAD_DT(c + 1);
             float dtv[4], cs[4];
             float run = 0.f;
 #pragma unroll
@@ -315,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
             if (!__shfl_sync(0xffffffffu, okc, 0)) { raise_abort(abort_flag); break; }
         }
+#undef SSD_LOAD_DT
         if (lane == 0 && *abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
     } else if (warp == kWarpMma) {
         // ---------------- tcgen05.mma issuer ----------------
@@ -324,9 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             constexpr uint32_t ID_Y2 = idesc_bf16_f32(128, 64, false, true);    // C (K-major) x S (MN-major)
             constexpr uint32_t ID_SC = idesc_bf16_f32(128, 64, true, true);     // B^T (MN-major) x X' (MN-major)
             const uint32_t sC = smem_u32(sm + OFF_C), sB = smem_u32(sm + OFF_B);
-            const uint32_t sX = smem_u32(sm + OFF_X), sXp = smem_u32(sm + OFF_XP);
+            const uint32_t sXp = smem_u32(sm + OFF_XP);
             const uint32_t sM = smem_u32(sm + OFF_M), sS = smem_u32(sm + OFF_S);
             for (int c = 0; c < nc; ++c) {
+                const uint32_t sX = smem_u32(sm + OFF_X + (c & 1) * 16384);
                 if (!mbar_wait(&bars[FULL_BC], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 if (c >= 1 && !mbar_wait(&bars[MREADY], (c - 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 tc_fence_after();
@@ -337,21 +419,29 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                              kk > 0);
                 }
                 mma_commit(&bars[G_FULL]);
+                // chunk state S_c = B^T X'  (needs this chunk's conv)
                 if (!mbar_wait(&bars[XREADY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tmem + COL_Y2, sw128_desc(sC + koff, 16, 1024), sw128_desc(sS + kk * 2048, 16384, 1024),
-                             ID_Y2, kk > 0);
-                }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     mma_bf16(tmem + COL_SC, sw128_desc(sB + kk * 2048, 16384, 1024),
                              sw128_desc(sXp + kk * 2048, 16384, 1024), ID_SC, kk > 0);
                 }
                 mma_commit(&bars[SC_FULL]);
+                // Y2 = C S_prev^T, once the previous chunk's epilogue has read the previous Y2
+                if (c >= 1 && !mbar_wait(&bars[EMPTY_RAW0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag)) {
+                    raise_abort(abort_flag);
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_bf16(tmem + COL_Y2, sw128_desc(sC + koff, 16, 1024),
+                             sw128_desc(sS + (c & 1) * 16384 + kk * 2048, 16384, 1024), ID_Y2, kk > 0);
+                }
                 mma_commit(&bars[EMPTY_BC]);
+                // Y = M X, once every row's decay mask is written
                 if (!mbar_wait(&bars[MREADY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 tc_fence_after();
 #pragma unroll
@@ -368,25 +458,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         }
     } else {
         // ---------------- compute warps ----------------
+        // Per chunk c: decay mask (c), state pass (c), x conv (c+1), epilogue (c), so that the next
+        // chunk's conv and its S_c / Y2 tensor-core work overlap this chunk's Y = M X and epilogue.
         const int wc = warp - kFirstCompute;               // 0..15
         const int q = warp & 3;                            // TMEM lane quadrant of this warp
-        const int quarter = wc >> 2;                       // row-major phases: columns 16*quarter .. +15
-        const int i = q * 32 + lane;                       // row-major phases: token row / TMEM lane
+        const int quarter = wc >> 2;                       // columns 16*quarter .. +15 (mask: 8-column groups)
+        const int i = q * 32 + lane;                       // token row / TMEM lane / state row n
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float Dh = a.D[h];
-        uint8_t* sX = sm + OFF_X;
         uint8_t* sXp = sm + OFF_XP;
         uint8_t* sMm = sm + OFF_M;
         uint8_t* sS = sm + OFF_S;
-        uint8_t* sU = sm + OFF_U;
-
-        // conv taps of this lane's channel pair (channel-major conv), constant over the sequence
-        const int ch0 = h * kP + 2 * lane;
-        const float4 wa = *reinterpret_cast<const float4*>(a.conv_w + (size_t)ch0 * 4);
-        const float4 wb = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(ch0 + 1) * 4);
-        const float2 tap0 = make_float2(wa.x, wb.x), tap1 = make_float2(wa.y, wb.y);
-        const float2 tap2 = make_float2(wa.z, wb.z), tap3 = make_float2(wa.w, wb.w);
-        const float2 cbias = make_float2(a.conv_b[ch0], a.conv_b[ch0 + 1]);
+        (void)sXp;
 
         // initial state (this thread's 16 columns): S_run in TMEM, bf16 copy in smem
         {
@@ -407,76 +490,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             tmem_wait_st();
         }
 
-        for (int c = 0; c < nc; ++c) {
+        bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, i, quarter);
+        if (!ok) raise_abort(abort_flag);
+        for (int c = 0; c < nc && ok; ++c) {
             const int s = c & 1, buf = c & 1;
             const int64_t t0 = (int64_t)c * kQ;
             const int Qc = (int)(a.L - t0 < kQ ? a.L - t0 : kQ);
             const float* cs_b = s_cs + buf * 128;
-
-            if (!warp_wait(&bars[CS_READY0 + buf], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
             const float cs_i = cs_b[i];
             const float cs_last = cs_b[kQ - 1];
             const float ecs = __expf(cs_i);  // decay of S_prev up to row i
-
-            // (c) conv + SiLU, channel-major: rows 8*wc .. 8*wc+7, channels 2*lane, 2*lane+1
-            if (!warp_wait(&bars[FULL_RAW0 + s], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
-            {
-                const uint8_t* rx = sm + OFF_RAWX + s * 16384;
-                const uint32_t* halo_in = reinterpret_cast<const uint32_t*>(sm + OFF_HALO) + (c & 1) * 96;
-                const float* wx_b = s_wx + buf * 128;
-                const int r0 = 8 * wc;
-                const uint32_t lane_byte = (uint32_t)(lane & 3) * 4;
-                uint32_t raw[11];
-#pragma unroll
-                for (int k = 0; k < 11; ++k) {
-                    const int r = r0 - 3 + k;
-                    raw[k] = r >= 0 ? *reinterpret_cast<const uint32_t*>(rx + sw128_off(r, lane >> 2) + lane_byte)
-                                    : halo_in[(r + 3) * 32 + lane];
-                }
-                float2 xv[11];
-#pragma unroll
-                for (int k = 0; k < 11; ++k) xv[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
-                float2 uvs[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int r = r0 + k;
-                    uint32_t xo = 0u, xpo = 0u;
-                    float2 uv = make_float2(0.f, 0.f);
-                    if (r < Qc) {  // warp-uniform
-                        float2 acc = cbias;
-                        acc = __ffma2_rn(tap0, xv[k + 0], acc);
-                        acc = __ffma2_rn(tap1, xv[k + 1], acc);
-                        acc = __ffma2_rn(tap2, xv[k + 2], acc);
-                        acc = __ffma2_rn(tap3, xv[k + 3], acc);
-                        uv = silu2(acc);
-                        const float wxr = wx_b[r];
-                        xo = pack_bf2(uv.x, uv.y);
-                        const float2 up = __fmul2_rn(uv, make_float2(wxr, wxr));
-                        xpo = pack_bf2(up.x, up.y);
-                    }
-                    const uint32_t off = sw128_off(r, lane >> 2) + lane_byte;
-                    *reinterpret_cast<uint32_t*>(sX + off) = xo;
-                    *reinterpret_cast<uint32_t*>(sXp + off) = xpo;
-                    uvs[k] = uv;
-                }
-                // the fp32 tile is still read by the previous chunk's epilogue in other warps:
-                // overwrite it only once every compute thread has finished that epilogue
-                if (c >= 1 && !warp_wait(&bars[EMPTY_RAW0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag)) {
-                    raise_abort(abort_flag);
-                    break;
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) *reinterpret_cast<float2*>(sU + u_off(r0 + k, lane)) = uvs[k];
-                if (wc == 15) {  // raw history (rows 125..127) of the next chunk
-                    uint32_t* halo_out = reinterpret_cast<uint32_t*>(sm + OFF_HALO) + ((c + 1) & 1) * 96;
-                    halo_out[0 * 32 + lane] = raw[8];
-                    halo_out[1 * 32 + lane] = raw[9];
-                    halo_out[2 * 32 + lane] = raw[10];
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[XREADY]);
 
             // (e) decay mask of row i, columns 8*quarter .. +7 of each 32-column block
             if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
@@ -554,7 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     w.y = pack_bf2(sr[k2 * 8 + 2], sr[k2 * 8 + 3]);
                     w.z = pack_bf2(sr[k2 * 8 + 4], sr[k2 * 8 + 5]);
                     w.w = pack_bf2(sr[k2 * 8 + 6], sr[k2 * 8 + 7]);
-                    *reinterpret_cast<uint4*>(sS + sw128_off(i, quarter * 2 + k2)) = w;
+                    // the state entering chunk c+1, into the buffer of that chunk's parity (Y2 of chunk c may
+                    // still be reading the other one)
+                    *reinterpret_cast<uint4*>(sS + ((c + 1) & 1) * 16384 + sw128_off(i, quarter * 2 + k2)) = w;
                 }
                 if (c == nc - 1) {
                     float* fs = a.final_state + ((size_t)b * a.H + h) * kP * kN;
@@ -564,51 +589,51 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 tmem_wait_st();
             }
 
+            // (c) the next chunk's x conv (its S_c then overlaps this chunk's Y = M X and epilogue)
+            if (c + 1 < nc && !conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, c + 1, nc, i, quarter)) {
+                raise_abort(abort_flag);
+                break;
+            }
+
             // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 16*quarter .. +15
             if (!warp_wait(&bars[FULL_Z0 + s], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
             if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
             {
-                const uint8_t* rz = sm + OFF_RAWX + s * 16384;
-                const uint4 zw[2] = {*reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2)),
-                                     *reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2 + 1))};
+                uint8_t* rz = sm + OFF_RAWX + s * 16384;  // z in, y out (same positions, this thread's only)
                 TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
-                float y1[16], y2[16];
-                tmem_ld16(tmem + lane_base + COL_Y + quarter * 16, y1);
-                tmem_ld16(tmem + lane_base + COL_Y2 + quarter * 16, y2);
-                tmem_wait_ld();
                 const float2 e2 = make_float2(ecs, ecs), d2 = make_float2(Dh, Dh);
 #pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                    const uint32_t zr[4] = {zw[k2].x, zw[k2].y, zw[k2].z, zw[k2].w};
+                for (int k2 = 0; k2 < 2; ++k2) {  // 8 columns per TMEM round trip
+                    float y1[8], y2[8], uu[8];
+                    tmem_ld8(tmem + lane_base + COL_Y + quarter * 16 + k2 * 8, y1);
+                    tmem_ld8(tmem + lane_base + COL_Y2 + quarter * 16 + k2 * 8, y2);
+                    tmem_ld8(tmem + lane_base + COL_U + buf * 64 + quarter * 16 + k2 * 8, uu);
+                    const uint4 zw = *reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2 + k2));
+                    tmem_wait_ld();
+                    const uint32_t zr[4] = {zw.x, zw.y, zw.z, zw.w};
                     float o[8];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
-                        const int k = k2 * 8 + e;
-                        const float2 uv = *reinterpret_cast<const float2*>(sU + u_off(i, quarter * 8 + (k >> 1)));
-                        float2 yv = __ffma2_rn(e2, make_float2(y2[k], y2[k + 1]), make_float2(y1[k], y1[k + 1]));
-                        yv = __ffma2_rn(d2, uv, yv);
+                        float2 yv = __ffma2_rn(e2, make_float2(y2[e], y2[e + 1]), make_float2(y1[e], y1[e + 1]));
+                        yv = __ffma2_rn(d2, make_float2(uu[e], uu[e + 1]), yv);
                         const float2 gz = silu2(make_float2(bf_lo(zr[e >> 1]), bf_hi(zr[e >> 1])));
                         const float2 ov = __fmul2_rn(yv, gz);
                         o[e] = ov.x;
                         o[e + 1] = ov.y;
                     }
-                    if (i < Qc) {
-                        if constexpr (sizeof(TY) == 2) {
-                            uint4 w;
-                            w.x = pack_bf2(o[0], o[1]);
-                            w.y = pack_bf2(o[2], o[3]);
-                            w.z = pack_bf2(o[4], o[5]);
-                            w.w = pack_bf2(o[6], o[7]);
-                            *reinterpret_cast<uint4*>(yrow + k2 * 8) = w;
-                        } else {
-                            float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
-                            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-                            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
-                        }
+                    if constexpr (kTmaStoreY) {
+                        *reinterpret_cast<uint4*>(rz + sw128_off(i, quarter * 2 + k2)) =
+                            make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]),
+                                       pack_bf2(o[6], o[7]));
+                    } else if (i < Qc) {
+                        float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
+                        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
                     }
                 }
             }
+            fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[EMPTY_RAW0 + s]);
         }
@@ -742,6 +767,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     TcParams prm;
     prm.a = a;
     if (!make_map(&prm.tm_x, a.x, a.HP, a.L, a.batch) || !make_map(&prm.tm_z, a.z, a.HP, a.L, a.batch) ||
+        (kind == ActKind::BF16 && !make_map(&prm.tm_y, a.y, a.HP, a.L, a.batch)) ||
         !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, a.batch))
         return cudaErrorInvalidValue;
     const dim3 pgrid((unsigned)((a.L + kProTok - 1) / kProTok), (unsigned)a.batch, (unsigned)((a.GN + 255) / 256));
