@@ -319,22 +319,28 @@ def main():
     K = args.steps
     st = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     en = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ks = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize(dev)
     sampler.load(True)
     for k in range(K):
         flush.zero_()                      # L2 flush, outside the step's events
-        ops.set_timing_events(ks[k], ke[k])
         st[k].record()
         prefill_once()
         en[k].record()
     torch.cuda.synchronize(dev)
     sampler.load(False)
     barrier(world)
-    ops.set_timing_events(None, None)
     step_ms = sum(s.elapsed_time(e) for s, e in zip(st, en)) / K
+    # the dominant kernel alone, in a second pass: events recorded between the two launches of a
+    # step would also serialise them, so they are kept out of the pass that gives `value`
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for k in range(K):
+        flush.zero_()
+        ops.set_timing_events(ks[k], ke[k])
+        prefill_once()
+    torch.cuda.synchronize(dev)
+    ops.set_timing_events(None, None)
     kern_ms = sum(s.elapsed_time(e) for s, e in zip(ks, ke)) / K
     tokens_per_rank = d.batch * d.seqlen
     value, step_ms_max = weak_scaling_value(tokens_per_rank, step_ms, world, dev)
@@ -450,7 +456,7 @@ def main():
                        "l2": "flushed between timed steps (256 MB write outside the step events)",
                        "kernel_path": "tcgen05 tensor-core" if path == 1 else "CUDA-core"},
             "tensor": tc, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
-            "gpu_launches": K * (3 if path == 1 else 1), "clocks": clocks,
+            "gpu_launches": K * (2 if path == 1 else 1), "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

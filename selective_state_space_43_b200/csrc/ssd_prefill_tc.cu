@@ -15,11 +15,12 @@
 //   y      = (Y + exp(cs_i) Y2 + D x) SiLU(z)
 //   S_prev <- exp(cs_last) S_prev + S_c
 //
-// Three kernels:
+// Two kernels (the second launched with programmatic dependent launch):
 //   bc_prologue  SiLU(conv4) of the B and C channels of every token, written
 //                once per group to the workspace in bf16 (the 16 heads of a
 //                group then read it from L2 instead of recomputing it);
-//   conv_tail    the conv_state output (last 3 pre-conv tokens, all channels);
+//                The same launch writes the conv_state output (last 3 pre-conv
+//                tokens of every channel).
 //   chunk_scan   one CTA per (sequence b, head h) walks the chunks in order;
 //                all accumulators live in TMEM; 7 warps:
 //                  warp 0  TMA producer: raw x tiles (2-stage ring); once a
@@ -215,7 +216,6 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
         for (int k = 0; k < 2; ++k)
             halo_out[(i - (kQ - 3)) * 8 + quarter * 2 + k] = *reinterpret_cast<const uint4*>(rx + sw128_off(i, quarter * 2 + k));
     }
-    tmem_wait_st();
     fence_async_smem();
     tc_fence_before();
     mbar_arrive(&bars[XREADY]);
@@ -339,6 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     } while (0)
         SSD_LOAD_DT(0);
         if (lane == 0) prefetch_tmap(&prm.tm_bc);
+        // the post-conv B/C come from the prologue kernel launched just before this one
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         int last = -1;
         for (int c = 0; c < nc; ++c) {
             // dt = softplus(dt_raw + bias) and the inclusive cumsum of dt*A over the chunk's 128 rows,
@@ -586,7 +588,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
 #pragma unroll
                     for (int k = 0; k < 16; ++k) fs[(size_t)(quarter * 16 + k) * kN + i] = sr[k];
                 }
-                tmem_wait_st();
             }
 
             // (c) the next chunk's x conv (its S_c then overlaps this chunk's Y = M X and epilogue)
@@ -599,6 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             if (!warp_wait(&bars[FULL_Z0 + s], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
             if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
+            tmem_wait_st();  // this thread's TMEM stores (the conv output read below, the running state) are done
             {
                 uint8_t* rz = sm + OFF_RAWX + s * 16384;  // z in, y out (same positions, this thread's only)
                 TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
@@ -646,81 +648,79 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     }
 }
 
-// SiLU(conv4) of the B and C channels into the workspace [b][t][2][G*N] (bf16).
-// Block: 256 threads = 256 channel
-// pairs (bf16x2) over kProTok tokens; a thread issues all kProTok + 3 loads of
-// its window before the first FMA, so the block's loads are all in flight at once.
+// SiLU(conv4) of the B and C channels into the workspace [b][t][2][G*N] (bf16),
+// and the conv_state output (pre-conv inputs of the last 3 tokens of every channel).
+// Blocks with blockIdx.x < ntok: 256 channel pairs (bf16x2) over kProTok tokens each; a
+// thread issues all kProTok + 3 loads of its window before the first FMA.  Blocks with
+// blockIdx.x >= ntok (and blockIdx.z == 0): the conv_state tail, one element per thread.
 constexpr int kProTok = 16;
 
-__global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int ntok) {
+    // the chunk scan may start its launch now; it waits for this grid before reading the workspace
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.init_conv_state);
+    if ((int)blockIdx.x >= ntok) {
+        if (blockIdx.z != 0) return;
+        const int64_t e = ((int64_t)(blockIdx.x - ntok) * gridDim.y + blockIdx.y) * 256 + threadIdx.x;
+        if (e >= a.batch * a.conv_dim * 3) return;
+        const int k = (int)(e % 3);
+        const int c = (int)((e / 3) % a.conv_dim);
+        const int64_t b = e / (3 * (int64_t)a.conv_dim);
+        const int64_t t = a.L - 3 + k;
+        __nv_bfloat16 v;
+        if (t >= 0) {
+            if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[((size_t)b * a.L + t) * a.HP + c];
+            else if (c < a.HP + a.GN)
+                v = static_cast<const __nv_bfloat16*>(a.B)[((size_t)b * a.L + t) * a.GN + (c - a.HP)];
+            else v = static_cast<const __nv_bfloat16*>(a.C)[((size_t)b * a.L + t) * a.GN + (c - a.HP - a.GN)];
+        } else {
+            v = hist ? hist[((size_t)b * a.conv_dim + c) * 3 + (t + 3)] : __float2bfloat16_rn(0.f);
+        }
+        static_cast<__nv_bfloat16*>(a.conv_state)[e] = v;
+        return;
+    }
     const int64_t b = blockIdx.y;
     const int64_t t0 = (int64_t)blockIdx.x * kProTok;
     const int half_gn = a.GN / 2;                    // channel pairs per array
     const int pair = blockIdx.z * 256 + threadIdx.x;  // 0 .. GN-1 over both arrays
-    const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.init_conv_state);
-    if (pair < a.GN) {
-        const int sel = pair >= half_gn;                // 0 = B, 1 = C
-        const int cp = pair - sel * half_gn;            // pair index within the array
-        const int cglob = a.HP + sel * a.GN + 2 * cp;   // conv channel of the pair's first element
-        const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B) + (size_t)b * a.L * half_gn + cp;
-        uint32_t* dst = static_cast<uint32_t*>(a.workspace) + ((size_t)b * a.L * 2 + sel) * half_gn + cp;
-        const float4 w0 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cglob * 4);
-        const float4 w1 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(cglob + 1) * 4);
-        const float b0 = a.conv_b[cglob], b1 = a.conv_b[cglob + 1];
-        float v0[kProTok + 3], v1[kProTok + 3];  // tokens t0-3 .. t0+kProTok-1
-        uint32_t raw[kProTok + 3];
+    if (pair >= a.GN) return;
+    const int sel = pair >= half_gn;                // 0 = B, 1 = C
+    const int cp = pair - sel * half_gn;            // pair index within the array
+    const int cglob = a.HP + sel * a.GN + 2 * cp;   // conv channel of the pair's first element
+    const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B) + (size_t)b * a.L * half_gn + cp;
+    uint32_t* dst = static_cast<uint32_t*>(a.workspace) + ((size_t)b * a.L * 2 + sel) * half_gn + cp;
+    const float4 w0 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cglob * 4);
+    const float4 w1 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(cglob + 1) * 4);
+    const float2 bias = make_float2(a.conv_b[cglob], a.conv_b[cglob + 1]);
+    float2 v[kProTok + 3];  // tokens t0-3 .. t0+kProTok-1, channels (2cp, 2cp+1)
+    uint32_t raw[kProTok + 3];
 #pragma unroll
-        for (int k = 0; k < kProTok + 3; ++k) {
-            const int64_t t = t0 - 3 + k;
-            raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * half_gn] : 0u;
-        }
+    for (int k = 0; k < kProTok + 3; ++k) {
+        const int64_t t = t0 - 3 + k;
+        raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * half_gn] : 0u;
+    }
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int64_t t = t0 - 3 + k;
-            if (t < 0 && hist) {
-                v0[k] = __bfloat162float(hist[((size_t)b * a.conv_dim + cglob) * 3 + (t + 3)]);
-                v1[k] = __bfloat162float(hist[((size_t)b * a.conv_dim + cglob + 1) * 3 + (t + 3)]);
-            } else {
-                v0[k] = bf_lo(raw[k]);
-                v1[k] = bf_hi(raw[k]);
-            }
-        }
+    for (int k = 0; k < kProTok + 3; ++k) {
+        const int64_t t = t0 - 3 + k;
+        if (t < 0 && hist)
+            v[k] = make_float2(__bfloat162float(hist[((size_t)b * a.conv_dim + cglob) * 3 + (t + 3)]),
+                               __bfloat162float(hist[((size_t)b * a.conv_dim + cglob + 1) * 3 + (t + 3)]));
+        else
+            v[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
+    }
 #pragma unroll
-        for (int k = 3; k < kProTok + 3; ++k) {
-            v0[k] = bf_lo(raw[k]);
-            v1[k] = bf_hi(raw[k]);
-        }
-#pragma unroll
-        for (int k = 0; k < kProTok; ++k) {
-            const int64_t t = t0 + k;
-            if (t < a.L) {
-                const float p0 = b0 + w0.x * v0[k] + w0.y * v0[k + 1] + w0.z * v0[k + 2] + w0.w * v0[k + 3];
-                const float p1 = b1 + w1.x * v1[k] + w1.y * v1[k + 1] + w1.z * v1[k + 2] + w1.w * v1[k + 3];
-                dst[(size_t)t * 2 * half_gn] = pack_bf2(silu_f(p0), silu_f(p1));
-            }
+    for (int k = 0; k < kProTok; ++k) {
+        const int64_t t = t0 + k;
+        if (t < a.L) {
+            float2 p = bias;
+            p = __ffma2_rn(make_float2(w0.x, w1.x), v[k], p);
+            p = __ffma2_rn(make_float2(w0.y, w1.y), v[k + 1], p);
+            p = __ffma2_rn(make_float2(w0.z, w1.z), v[k + 2], p);
+            p = __ffma2_rn(make_float2(w0.w, w1.w), v[k + 3], p);
+            const float2 u = silu2(p);
+            dst[(size_t)t * 2 * half_gn] = pack_bf2(u.x, u.y);
         }
     }
-}
-
-// conv_state tail: the pre-conv inputs of tokens L-3..L-1 (history-filled when
-// L < 3) of every channel, one element per thread.
-__global__ void __launch_bounds__(256) conv_tail_kernel(PrefillArgs a) {
-    const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    if (e >= a.batch * a.conv_dim * 3) return;
-    const int k = (int)(e % 3);
-    const int c = (int)((e / 3) % a.conv_dim);
-    const int64_t b = e / (3 * (int64_t)a.conv_dim);
-    const int64_t t = a.L - 3 + k;
-    const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.init_conv_state);
-    __nv_bfloat16 v;
-    if (t >= 0) {
-        if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[((size_t)b * a.L + t) * a.HP + c];
-        else if (c < a.HP + a.GN) v = static_cast<const __nv_bfloat16*>(a.B)[((size_t)b * a.L + t) * a.GN + (c - a.HP)];
-        else v = static_cast<const __nv_bfloat16*>(a.C)[((size_t)b * a.L + t) * a.GN + (c - a.HP - a.GN)];
-    } else {
-        v = hist ? hist[((size_t)b * a.conv_dim + c) * 3 + (t + 3)] : __float2bfloat16_rn(0.f);
-    }
-    static_cast<__nv_bfloat16*>(a.conv_state)[e] = v;
 }
 
 // ---- host side ------------------------------------------------------------------------------------------
@@ -770,17 +770,31 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
         (kind == ActKind::BF16 && !make_map(&prm.tm_y, a.y, a.HP, a.L, a.batch)) ||
         !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, a.batch))
         return cudaErrorInvalidValue;
-    const dim3 pgrid((unsigned)((a.L + kProTok - 1) / kProTok), (unsigned)a.batch, (unsigned)((a.GN + 255) / 256));
-    bc_prologue_kernel<<<pgrid, 256, 0, st>>>(a);
+    const int ntok = (int)((a.L + kProTok - 1) / kProTok);
     const int64_t tail = a.batch * (int64_t)a.conv_dim * 3;
-    conv_tail_kernel<<<(unsigned)((tail + 255) / 256), 256, 0, st>>>(a);
+    const int tail_blocks = (int)((tail + 256 * a.batch - 1) / (256 * a.batch));
+    const dim3 pgrid((unsigned)(ntok + tail_blocks), (unsigned)a.batch, (unsigned)((a.GN + 255) / 256));
+    bc_prologue_kernel<<<pgrid, 256, 0, st>>>(a, ntok);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     auto kern = kind == ActKind::BF16_YF32 ? chunk_scan_kernel<float> : chunk_scan_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    // programmatic dependent launch: the scan's set-up (TMEM, barriers, state, first x conv)
+    // overlaps the prologue; only its B/C loads wait for the prologue grid to complete
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.batch * a.H));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     hook.before(st);
-    kern<<<(unsigned)(a.batch * a.H), kThreads, SMEM_BYTES, st>>>(prm);
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    if (e != cudaSuccess) return e;
     hook.after(st);
     return cudaGetLastError();
 }
