@@ -104,7 +104,8 @@ SSD_API size_t ssd_prefill_workspace_bytes(const ssd_dims* dims, ssd_dtype dtype
 
 /*
  * Which kernel path ssd_prefill takes for these sizes:
- *   1 = tcgen05 tensor-core chunk scan (bf16 activations, P=64, Q=128, N=128);
+ *   1 = tcgen05 tensor-core chunk scan (bf16 activations, P=64, Q=128, N=128,
+ *       nheads a multiple of 8);
  *   2 = CUDA-core chunk scan (every other supported shape, and fp32);
  *  <0 = -(ssd_status) for invalid sizes.
  */

@@ -60,7 +60,7 @@ const char* ssd_version(void) { return "ssd_b200 1.0 (sm_100a)"; }
 int ssd_prefill_path(const ssd_dims* d, ssd_dtype dtype) {
     const ssd_status st = check_dims(d, dtype, true);
     if (st != SSD_OK) return -(int)st;
-    return ssd::prefill_tc_supported(d->headdim, d->d_state, d->chunk, dtype != SSD_F32) ? 1 : 2;
+    return ssd::prefill_tc_supported(d->headdim, d->d_state, d->chunk, d->nheads, dtype != SSD_F32) ? 1 : 2;
 }
 
 size_t ssd_prefill_workspace_bytes(const ssd_dims* d, ssd_dtype dtype) {

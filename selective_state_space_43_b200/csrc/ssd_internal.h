@@ -49,7 +49,7 @@ cudaError_t launch_decode(const DecodeArgs& a, int64_t batch, ActKind kind, cuda
 cudaError_t launch_prefill_simt(const PrefillArgs& a, ActKind kind, cudaStream_t st, const TimingHook& hook);
 
 // tcgen05 tensor-core chunked SSD (bf16 activations, P = 64, Q = 128, N in {64, 128}).
-bool prefill_tc_supported(int P, int N, int Q, bool bf16);
+bool prefill_tc_supported(int P, int N, int Q, int H, bool bf16);
 size_t prefill_tc_workspace_bytes(int64_t batch, int64_t L, int G, int N);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t st, const TimingHook& hook);
 // Synchronises `st`, then reads and clears the tensor-core kernel's timeout flag.

@@ -22,23 +22,22 @@
 //                The same launch writes the conv_state output (last 3 pre-conv
 //                tokens of every channel).
 //   chunk_scan   one CTA per (sequence b, head h) walks the chunks in order;
-//                all accumulators live in TMEM; 7 warps:
-//                  warp 0  TMA producer: raw x tiles (2-stage ring); once a
-//                           chunk's conv has consumed its stage, z of the same
-//                           chunk is loaded into it for the epilogue
+//                all accumulators live in TMEM; 20 warps:
+//                  warp 0  TMA producer: raw x tiles two chunks ahead (2-stage
+//                           ring), z of the current chunk (one buffer, which
+//                           the epilogue overwrites with y for the TMA store)
 //                  warp 1  TMEM allocator + single-thread tcgen05.mma issuer
-//                  warp 2  TMA producer: post-conv B and C tiles; the whole
-//                           warp also computes each chunk's dt, cumsum of dt*A
-//                           and mask factors one chunk ahead (double-buffered)
-//                  warps 3-18 512 compute threads.  The x conv runs channel-
-//                           major (warp = 8 tokens, lane = 2 channels, taps in
-//                           registers); the TMEM phases run row-major, four
-//                           threads per token row i (= TMEM lane i), each owning
-//                           16 state / output columns and one 8-column group of
-//                           each of the 4 decay-mask column blocks:
-//                           decay mask, state pass, epilogue (D skip from the
-//                           fp32 conv output, z gate, y store).  Elementwise math uses
-//                           the packed fp32x2 FMA / MUL of sm_100.
+//                  warp 2  each chunk's dt, cumsum of dt*A and mask factors,
+//                           one chunk ahead (double-buffered), from a raw dt
+//                           tile that warp 0 loads with the chunk's raw x
+//                  warp 3  TMA producer: post-conv B and C tiles
+//                  warps 4-19 512 compute threads, four per token row i (= TMEM
+//                           lane i), each owning 16 channels / state / output
+//                           columns and one 8-column group of each of the 4
+//                           decay-mask column blocks: x conv (fp32 output kept
+//                           in TMEM for the D skip), decay mask, state pass,
+//                           epilogue (D skip, z gate, y store).  Elementwise
+//                           math uses the packed fp32x2 FMA / MUL of sm_100.
 // The decay mask exp(cs_i - cs_j) is formed per 8-column group: exactly (one
 // exp per element) for the rows inside the group, and as the product of a row
 // factor exp(cs_i - cs_r) and a column factor exp(cs_r - cs_j) dt_j, with r the
@@ -62,8 +61,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kQ = 128, kP = 64, kN = 128;
-constexpr int kThreads = 608;
-constexpr int kWarpRaw = 0, kWarpMma = 1, kWarpBc = 2, kFirstCompute = 3;
+constexpr int kThreads = 640;
+constexpr int kWarpRaw = 0, kWarpMma = 1, kWarpCs = 2, kWarpBc = 3, kFirstCompute = 4;
 constexpr int kComputeThreads = 512;  // 16 warps: four per TMEM lane quadrant
 
 // shared memory map (bytes from a 1024-byte aligned base)
@@ -72,11 +71,13 @@ constexpr uint32_t OFF_B = 32768;      // u_B tile
 constexpr uint32_t OFF_X = 65536;      // 2 x X [j][p] bf16 (MN-major B operand), by chunk parity
 constexpr uint32_t OFF_XP = 98304;     // X' [j][p] bf16
 constexpr uint32_t OFF_M = 114688;     // M  [i][j] bf16, two K blocks of 64 (K-major A operand)
-constexpr uint32_t OFF_S = 147456;     // 2 x S_prev [n][p] bf16 (MN-major B operand), by chunk parity
-constexpr uint32_t OFF_RAWX = 180224;  // 2 stages [tok][p] bf16 (TMA, 128B swizzle): a chunk's x, then its z, then its y
+constexpr uint32_t OFF_S = 147456;     // S_prev [n][p] bf16 (MN-major B operand)
+constexpr uint32_t OFF_RAWX = 163840;  // 2 stages [tok][p] bf16 (TMA, 128B swizzle): raw x of chunks c, c+1
+constexpr uint32_t OFF_Z = 196608;     // [tok][p] bf16 (TMA, 128B swizzle): a chunk's z, then its y
 constexpr uint32_t OFF_SMALL = 212992;
 // small region
-constexpr uint32_t OFF_WT = OFF_SMALL;                 // conv taps of the head's x channels [4][64] float
+constexpr uint32_t OFF_DTRAW = OFF_SMALL;              // 2 stages [128 tok][8 heads] bf16 raw dt (TMA, with x)
+constexpr uint32_t OFF_WT = OFF_DTRAW + 2 * 2048;      // conv taps of the head's x channels [4][64] float
 constexpr uint32_t OFF_CB = OFF_WT + 4 * 64 * 4;       // conv bias [64] float
 constexpr uint32_t OFF_HALO = OFF_CB + 64 * 4;         // [2][3][64] bf16 raw x history
 constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;  // cs [2][128] float (double-buffered by chunk parity)
@@ -84,15 +85,17 @@ constexpr uint32_t OFF_DT = OFF_CS + 2 * 128 * 4;      // dt [2][128]
 constexpr uint32_t OFF_COLF = OFF_DT + 2 * 128 * 4;    // column factors of the decay mask [2][128] (8-col groups)
 constexpr uint32_t OFF_WX = OFF_COLF + 2 * 128 * 4;    // weight of x_j in the chunk state [2][128]
 constexpr uint32_t OFF_BAR = OFF_WX + 2 * 128 * 4;     // mbarriers (8 B each)
-constexpr int NBAR = 18;
+constexpr int NBAR = 17;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;  // TMEM base address
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-enum Bar { FULL_RAW0 = 0, FULL_RAW1, EMPTY_RAW0, EMPTY_RAW1, FULL_BC, EMPTY_BC, XREADY, MREADY, G_FULL, SC_FULL,
-           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, FULL_Z0, FULL_Z1 };
+// FULL_RAW / XREADY / CS_* come in pairs by chunk parity; EPI_DONE = a chunk's epilogue is complete
+// (its Y / Y2 / z read, its y written); EMPTY_BC = the chunk's last B / C reader (Y2) is complete.
+enum Bar { FULL_RAW0 = 0, FULL_RAW1, XREADY0, XREADY1, FULL_Z, EPI_DONE, FULL_BC, EMPTY_BC, MREADY, G_FULL, SC_FULL,
+           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1 };
 
 // TMEM columns (fp32, 128 lanes): G = C B^T, Y = M X, Y2 = C S^T, S_c, the running state, and the
 // post-conv x of two chunks (for the D skip)
@@ -100,7 +103,7 @@ constexpr uint32_t COL_G = 0, COL_Y = 128, COL_Y2 = 192, COL_SC = 256, COL_SRUN 
 
 struct TcParams {
     PrefillArgs a;
-    CUtensorMap tm_x, tm_z, tm_y, tm_bc;
+    CUtensorMap tm_x, tm_z, tm_y, tm_bc, tm_dt;
 };
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -142,6 +145,17 @@ __device__ __forceinline__ float s_wx_at(const uint8_t* sm, int buf, int row) {
     return reinterpret_cast<const float*>(sm + OFF_WX)[buf * 128 + row];
 }
 
+// D (+)= A B over K = 128 in eight K = 16 steps, from base descriptors (see sw128_desc); a descriptor's
+// start address field holds the byte address / 16, so a step adds its byte offset / 16.
+template <bool a_mn, bool b_mn>
+__device__ __forceinline__ void mma_k128(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
+#pragma unroll
+    for (uint32_t kk = 0; kk < 8; ++kk) {
+        const uint32_t kmaj = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, mnmaj = (kk * 2048) >> 4;
+        mma_bf16(d_tmem, a0 + (a_mn ? mnmaj : kmaj), b0 + (b_mn ? mnmaj : kmaj), idesc, kk > 0);
+    }
+}
+
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
     *abort_flag = 1;
     atomicExch(&g_tc_error, 1);
@@ -156,7 +170,7 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
     if (!warp_wait(&bars[CS_READY0 + buf], (cc >> 1) & 1, abort_flag)) return false;
     if (!warp_wait(&bars[FULL_RAW0 + buf], (cc >> 1) & 1, abort_flag)) return false;
     // the raw history rows were written by other threads in the previous chunk's conv
-    if (cc >= 1 && !warp_wait(&bars[XREADY], (cc - 1) & 1, abort_flag)) return false;
+    if (cc >= 1 && !warp_wait(&bars[XREADY0 + ((cc - 1) & 1)], ((cc - 1) >> 1) & 1, abort_flag)) return false;
     const int64_t t0 = (int64_t)cc * kQ;
     const int Qc = (int)(a.L - t0 < kQ ? a.L - t0 : kQ);
     const bool valid = i < Qc;
@@ -218,7 +232,7 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
     }
     fence_async_smem();
     tc_fence_before();
-    mbar_arrive(&bars[XREADY]);
+    mbar_arrive(&bars[XREADY0 + buf]);
     return true;
 }
 
@@ -226,7 +240,9 @@ template <typename TY>
 __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_constant__ TcParams prm) {
     const PrefillArgs& a = prm.a;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, formed as an offset from the shared array so that every access through it
+    // stays a shared-window access (32-bit addresses) rather than a generic one
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
@@ -244,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int k = 0; k < NBAR; ++k) {
             uint32_t cnt = 1;
-            if (k == EMPTY_RAW0 || k == EMPTY_RAW1 || k == XREADY || k == MREADY || k == CS_FREE0 || k == CS_FREE1)
+            if (k == XREADY0 || k == XREADY1 || k == EPI_DONE || k == MREADY || k == CS_FREE0 || k == CS_FREE1)
                 cnt = kComputeThreads;
             if (k == CS_READY0 || k == CS_READY1) cnt = 32;
             mbar_init(&bars[k], cnt);
@@ -283,81 +299,92 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
 
     if (warp == kWarpRaw) {
         // ---------------- raw x / z producer, y store ----------------
-        // Stage c&1 holds x(c) until chunk c's conv has read it, then z(c) until chunk c's
-        // epilogue has read it (and written y(c) over it), then y(c) until it is stored.
+        // Raw x runs two chunks ahead: stage c&1 is refilled with x(c+2) as soon as chunk c's conv
+        // has read it.  The z buffer holds z(c) until chunk c's epilogue has read it and written
+        // y(c) over it; y(c) is then stored and z(c+1) loaded.  The waits follow the order in which
+        // the compute threads complete the two events (conv(c+1) before epilogue(c)).
         if (lane == 0) {
             prefetch_tmap(&prm.tm_x);
             prefetch_tmap(&prm.tm_z);
-            int issued_x[2] = {-1, -1}, issued_z[2] = {-1, -1};
-            bool ok = true;
-            for (int it = 0; it <= nc + 1 && ok; ++it) {
-                if (it >= 1 && it <= nc) {  // z(it-1), once its conv has consumed x(it-1)
-                    const int cz = it - 1, s = cz & 1;
-                    if (!mbar_wait(&bars[XREADY], cz & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
-                    mbar_arrive_expect_tx(&bars[FULL_Z0 + s], 16384);
-                    tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_z, &bars[FULL_Z0 + s], h * kP, cz * kQ, b);
-                    issued_z[s] = cz;
+            prefetch_tmap(&prm.tm_dt);
+            int issued_x0 = -1, issued_x1 = -1, issued_z = -1;  // last chunk loaded into each buffer
+            auto load_x = [&](int c) {  // raw x of chunk c and its dt (the 8-head column block holding h)
+                const int s = c & 1;
+                mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384 + 2048);
+                tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, c * kQ, b);
+                tma_load_3d(sm + OFF_DTRAW + s * 2048, &prm.tm_dt, &bars[FULL_RAW0 + s], h & ~7, c * kQ, b);
+                if (s) issued_x1 = c;
+                else issued_x0 = c;
+            };
+            auto load_z = [&](int c) {
+                mbar_arrive_expect_tx(&bars[FULL_Z], 16384);
+                tma_load_3d(sm + OFF_Z, &prm.tm_z, &bars[FULL_Z], h * kP, c * kQ, b);
+                issued_z = c;
+            };
+            for (int c = 0; c < nc && c < 2; ++c) load_x(c);
+            load_z(0);
+            for (int c = 0; c < nc; ++c) {
+                if (c + 2 < nc) {  // x(c+2), once chunk c's conv has consumed x(c)
+                    if (!mbar_wait(&bars[XREADY0 + (c & 1)], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+                    load_x(c + 2);
                 }
-                if (it >= 2) {  // y(it-2) out of its stage, once its epilogue is complete
-                    const int cy = it - 2, s = cy & 1;
-                    if (!mbar_wait(&bars[EMPTY_RAW0 + s], (cy >> 1) & 1, abort_flag)) { raise_abort(abort_flag); ok = false; break; }
-                    if constexpr (kTmaStoreY) {
-                        tma_store_3d(&prm.tm_y, sm + OFF_RAWX + s * 16384, h * kP, cy * kQ, b);
-                        bulk_commit();
-                        bulk_wait_read_all();  // the stage may be refilled once the store has read it
-                    }
+                // y(c) out of the z buffer once chunk c's epilogue is complete, then z(c+1) in
+                if (!mbar_wait(&bars[EPI_DONE], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
+                if constexpr (kTmaStoreY) {
+                    tma_store_3d(&prm.tm_y, sm + OFF_Z, h * kP, c * kQ, b);
+                    bulk_commit();
+                    bulk_wait_read_all();  // the buffer may be refilled once the store has read it
                 }
-                if (it < nc) {  // x(it) into its stage
-                    const int s = it & 1;
-                    mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384);
-                    tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, it * kQ, b);
-                    issued_x[s] = it;
-                }
+                if (c + 1 < nc) load_z(c + 1);
             }
             if constexpr (kTmaStoreY) bulk_wait_all();
             if (*abort_flag) {  // let copies still in flight land before the CTA exits
-                for (int s = 0; s < 2; ++s) {
-                    if (issued_x[s] >= 0) mbar_wait(&bars[FULL_RAW0 + s], (issued_x[s] >> 1) & 1, nullptr, 100000000ull);
-                    if (issued_z[s] >= 0) mbar_wait(&bars[FULL_Z0 + s], (issued_z[s] >> 1) & 1, nullptr, 100000000ull);
-                }
+                if (issued_x0 >= 0) mbar_wait(&bars[FULL_RAW0], (issued_x0 >> 1) & 1, nullptr, 100000000ull);
+                if (issued_x1 >= 0) mbar_wait(&bars[FULL_RAW1], (issued_x1 >> 1) & 1, nullptr, 100000000ull);
+                if (issued_z >= 0) mbar_wait(&bars[FULL_Z], issued_z & 1, nullptr, 100000000ull);
             }
         }
     } else if (warp == kWarpBc) {
-        // ---------------- chunk dt / cumsum (whole warp) + post-conv B / C producer (lane 0) ----------------
+        // ---------------- post-conv B / C producer ----------------
+        if (lane == 0) {
+            prefetch_tmap(&prm.tm_bc);
+            // the post-conv B/C come from the prologue kernel launched just before this one
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            int last = -1;
+            for (int c = 0; c < nc; ++c) {
+                // B / C of chunk c, once chunk c-1's last reader of the tiles (Y2) is complete
+                if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+                mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
+                const int xc = a.GN + g * kN, xb = g * kN;
+                tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, c * kQ, b);
+                tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, c * kQ, b);
+                tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, c * kQ, b);
+                tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, c * kQ, b);
+                last = c;
+            }
+            if (*abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
+        }
+    } else if (warp == kWarpCs) {
+        // ---------------- chunk dt / cumsum (whole warp; lane l owns rows 4l .. 4l+3) ----------------
         const float A = a.A[h], dtb = a.dt_bias[h];
-        const __nv_bfloat16* dtp = static_cast<const __nv_bfloat16*>(a.dt);
-        // dt of rows 4*lane .. 4*lane+3, loaded one chunk ahead
-        float dn0, dn1, dn2, dn3;
-#define SSD_LOAD_DT(CC)                                                                                  \
-    do {                                                                                                 \
-        const int64_t tb = (int64_t)(CC) * kQ + 4 * lane;                                               \
-        const __nv_bfloat16* p = dtp + ((size_t)b * a.L + tb) * a.H + h;                                \
-        dn0 = tb + 0 < a.L ? __bfloat162float(p[0]) : 0.f;                                               \
-        dn1 = tb + 1 < a.L ? __bfloat162float(p[a.H]) : 0.f;                                             \
-        dn2 = tb + 2 < a.L ? __bfloat162float(p[2 * a.H]) : 0.f;                                         \
-        dn3 = tb + 3 < a.L ? __bfloat162float(p[3 * a.H]) : 0.f;                                         \
-    } while (0)
-        SSD_LOAD_DT(0);
-        if (lane == 0) prefetch_tmap(&prm.tm_bc);
-        // the post-conv B/C come from the prologue kernel launched just before this one
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        int last = -1;
         for (int c = 0; c < nc; ++c) {
             // dt = softplus(dt_raw + bias) and the inclusive cumsum of dt*A over the chunk's 128 rows,
-            // into the buffer of this chunk's parity once every compute thread is done with it
+            // into the buffer of this chunk's parity once every compute thread is done with it; the raw
+            // dt tile arrives with the chunk's raw x
             const int buf = c & 1;
             if (c >= 2 && !warp_wait(&bars[CS_FREE0 + buf], ((c >> 1) + 1) & 1, abort_flag)) {
                 raise_abort(abort_flag);
                 break;
             }
+            if (!warp_wait(&bars[FULL_RAW0 + buf], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
             const int Qc = (int)(a.L - (int64_t)c * kQ < kQ ? a.L - (int64_t)c * kQ : kQ);
-            const float dr[4] = {dn0, dn1, dn2, dn3};
-            if (c + 1 < nc) SSD_LOAD_DT(c + 1);
+            const __nv_bfloat16* dtr = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_DTRAW + buf * 2048) + (h & 7);
             float dtv[4], cs[4];
             float run = 0.f;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                dtv[k] = (4 * lane + k < Qc) ? softplus_fast(dr[k] + dtb) : 0.f;
+                const int r = 4 * lane + k;
+                dtv[k] = r < Qc ? softplus_fast(__bfloat162float(dtr[r * 8]) + dtb) : 0.f;
                 run += dtv[k] * A;
                 cs[k] = run;
             }
@@ -371,34 +398,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             const float cs_last = __shfl_sync(0xffffffffu, incl, 31);
             // cs at the last row of the 8-row group (rows 8m .. 8m+7 live on lanes 2m, 2m+1)
             const float cs_g8 = __shfl_sync(0xffffffffu, incl, lane | 1);
+            float csr[4], cf[4], wx[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int r = 4 * lane + k;
-                const float csr = cs[k] + excl;
-                s_cs[buf * 128 + r] = csr;
-                s_dt[buf * 128 + r] = dtv[k];
-                s_colf[buf * 128 + r] = __expf(cs_g8 - csr) * dtv[k];
-                s_wx[buf * 128 + r] = __expf(cs_last - csr) * dtv[k];
+                csr[k] = cs[k] + excl;
+                cf[k] = __expf(cs_g8 - csr[k]) * dtv[k];
+                wx[k] = __expf(cs_last - csr[k]) * dtv[k];
             }
+            reinterpret_cast<float4*>(s_cs + buf * 128)[lane] = make_float4(csr[0], csr[1], csr[2], csr[3]);
+            reinterpret_cast<float4*>(s_dt + buf * 128)[lane] = make_float4(dtv[0], dtv[1], dtv[2], dtv[3]);
+            reinterpret_cast<float4*>(s_colf + buf * 128)[lane] = make_float4(cf[0], cf[1], cf[2], cf[3]);
+            reinterpret_cast<float4*>(s_wx + buf * 128)[lane] = make_float4(wx[0], wx[1], wx[2], wx[3]);
             mbar_arrive(&bars[CS_READY0 + buf]);
-            int okc = 1;
-            if (lane == 0) {
-                if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) {
-                    okc = 0;
-                } else {
-                    mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
-                    const int xc = a.GN + g * kN, xb = g * kN;
-                    tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, c * kQ, b);
-                    tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, c * kQ, b);
-                    tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, c * kQ, b);
-                    tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, c * kQ, b);
-                    last = c;
-                }
-            }
-            if (!__shfl_sync(0xffffffffu, okc, 0)) { raise_abort(abort_flag); break; }
         }
-#undef SSD_LOAD_DT
-        if (lane == 0 && *abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
     } else if (warp == kWarpMma) {
         // ---------------- tcgen05.mma issuer ----------------
         if (lane == 0) {
@@ -406,52 +418,39 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             constexpr uint32_t ID_Y = idesc_bf16_f32(128, 64, false, true);     // M (K-major) x X (MN-major)
             constexpr uint32_t ID_Y2 = idesc_bf16_f32(128, 64, false, true);    // C (K-major) x S (MN-major)
             constexpr uint32_t ID_SC = idesc_bf16_f32(128, 64, true, true);     // B^T (MN-major) x X' (MN-major)
-            const uint32_t sC = smem_u32(sm + OFF_C), sB = smem_u32(sm + OFF_B);
-            const uint32_t sXp = smem_u32(sm + OFF_XP);
-            const uint32_t sM = smem_u32(sm + OFF_M), sS = smem_u32(sm + OFF_S);
+            // base descriptors; a K step of 16 advances a K-major operand by 32 bytes inside its 64-wide
+            // swizzle atom (and to the second atom after four steps), an MN-major one by 16 rows (2048 bytes)
+            const uint64_t dC = sw128_desc(smem_u32(sm + OFF_C), 16, 1024);
+            const uint64_t dB = sw128_desc(smem_u32(sm + OFF_B), 16, 1024);
+            const uint64_t dBt = sw128_desc(smem_u32(sm + OFF_B), 16384, 1024);
+            const uint64_t dXp = sw128_desc(smem_u32(sm + OFF_XP), 16384, 1024);
+            const uint64_t dM = sw128_desc(smem_u32(sm + OFF_M), 16, 1024);
+            const uint64_t dS = sw128_desc(smem_u32(sm + OFF_S), 16384, 1024);
+            const uint64_t dX0 = sw128_desc(smem_u32(sm + OFF_X), 16384, 1024);
             for (int c = 0; c < nc; ++c) {
-                const uint32_t sX = smem_u32(sm + OFF_X + (c & 1) * 16384);
+                const uint64_t dX = dX0 + (uint64_t)((c & 1) * (16384 >> 4));
                 if (!mbar_wait(&bars[FULL_BC], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 if (c >= 1 && !mbar_wait(&bars[MREADY], (c - 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tmem + COL_G, sw128_desc(sC + koff, 16, 1024), sw128_desc(sB + koff, 16, 1024), ID_G,
-                             kk > 0);
-                }
+                mma_k128<false, false>(tmem + COL_G, dC, dB, ID_G);
                 mma_commit(&bars[G_FULL]);
                 // chunk state S_c = B^T X'  (needs this chunk's conv)
-                if (!mbar_wait(&bars[XREADY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
+                if (!mbar_wait(&bars[XREADY0 + (c & 1)], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_bf16(tmem + COL_SC, sw128_desc(sB + kk * 2048, 16384, 1024),
-                             sw128_desc(sXp + kk * 2048, 16384, 1024), ID_SC, kk > 0);
-                }
+                mma_k128<true, true>(tmem + COL_SC, dBt, dXp, ID_SC);
                 mma_commit(&bars[SC_FULL]);
                 // Y2 = C S_prev^T, once the previous chunk's epilogue has read the previous Y2
-                if (c >= 1 && !mbar_wait(&bars[EMPTY_RAW0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag)) {
+                if (c >= 1 && !mbar_wait(&bars[EPI_DONE], (c - 1) & 1, abort_flag)) {
                     raise_abort(abort_flag);
                     break;
                 }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tmem + COL_Y2, sw128_desc(sC + koff, 16, 1024),
-                             sw128_desc(sS + (c & 1) * 16384 + kk * 2048, 16384, 1024), ID_Y2, kk > 0);
-                }
-                mma_commit(&bars[EMPTY_BC]);
+                mma_k128<false, true>(tmem + COL_Y2, dC, dS, ID_Y2);
+                mma_commit(&bars[EMPTY_BC]);  // B / C tiles and S_prev free
                 // Y = M X, once every row's decay mask is written
                 if (!mbar_wait(&bars[MREADY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tmem + COL_Y, sw128_desc(sM + koff, 16, 1024), sw128_desc(sX + kk * 2048, 16384, 1024),
-                             ID_Y, kk > 0);
-                }
+                mma_k128<false, true>(tmem + COL_Y, dM, dX, ID_Y);
                 mma_commit(&bars[Y_FULL]);
             }
             // nothing may still be running on the tensor cores when TMEM is released
@@ -495,65 +494,66 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, i, quarter);
         if (!ok) raise_abort(abort_flag);
         for (int c = 0; c < nc && ok; ++c) {
-            const int s = c & 1, buf = c & 1;
+            const int buf = c & 1;
             const int64_t t0 = (int64_t)c * kQ;
             const int Qc = (int)(a.L - t0 < kQ ? a.L - t0 : kQ);
             const float* cs_b = s_cs + buf * 128;
             const float cs_i = cs_b[i];
             const float cs_last = cs_b[kQ - 1];
-            const float ecs = __expf(cs_i);  // decay of S_prev up to row i
 
             // (e) decay mask of row i, columns 8*quarter .. +7 of each 32-column block
             if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
             {
                 const float* dt_b = s_dt + buf * 128;
+                float gv[4][8];
 #pragma unroll
-                for (int kp = 0; kp < 4; kp += 2) {  // two 8-column groups per TMEM round trip
-                    float gv[2][8];
+                for (int kb = 0; kb < 4; ++kb)  // warp-uniform: groups right of the diagonal block are zero
+                    if (kb <= q) tmem_ld8(tmem + lane_base + COL_G + kb * 32 + quarter * 8, gv[kb]);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int t = 0; t < 2; ++t)  // warp-uniform: groups right of the diagonal block are zero
-                        if (kp + t <= q) tmem_ld8(tmem + lane_base + COL_G + (kp + t) * 32 + quarter * 8, gv[t]);
-                    tmem_wait_ld();
+                for (int kb = 0; kb < 4; ++kb) {
+                    const int j0 = kb * 32 + quarter * 8;  // first column of this 8-column group
+                    uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+                    if (kb <= q && i >= j0) {
+                        float m[8];
+                        if (i > j0 + 7) {
+                            // below the group: exp(cs_i - cs_j) = exp(cs_i - cs_r) exp(cs_r - cs_j), r = j0 + 7
+                            const float rowf = __expf(cs_i - cs_b[j0 + 7]);
+                            const float2 rf = make_float2(rowf, rowf);
+                            const float4* colf = reinterpret_cast<const float4*>(s_colf + buf * 128 + j0);
 #pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const int kb = kp + t;
-                        const int j0 = kb * 32 + quarter * 8;  // first column of this 8-column group
-                        uint4 packed = make_uint4(0u, 0u, 0u, 0u);
-                        if (kb <= q) {
-                            float m[8];
-                            if (i > j0 + 7) {
-                                // below the group: exp(cs_i - cs_j) = exp(cs_i - cs_r) exp(cs_r - cs_j), r = j0 + 7
-                                const float rowf = __expf(cs_i - cs_b[j0 + 7]);
-                                const float2 rf = make_float2(rowf, rowf);
-                                const float2* colf = reinterpret_cast<const float2*>(s_colf + buf * 128 + j0);
-#pragma unroll
-                                for (int e = 0; e < 8; e += 2) {
-                                    const float2 v =
-                                        __fmul2_rn(__fmul2_rn(make_float2(gv[t][e], gv[t][e + 1]), colf[e >> 1]), rf);
-                                    m[e] = v.x;
-                                    m[e + 1] = v.y;
-                                }
-                            } else {
-                                // the group holds the diagonal (or lies right of it): exact decay for j <= i
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    const int j = j0 + e;
-                                    m[e] = j <= i ? gv[t][e] * __expf(cs_i - cs_b[j]) * dt_b[j] : 0.f;
-                                }
+                            for (int e = 0; e < 8; e += 4) {
+                                const float4 cf = colf[e >> 2];
+                                const float2 v0 = __fmul2_rn(__fmul2_rn(make_float2(gv[kb][e], gv[kb][e + 1]),
+                                                                        make_float2(cf.x, cf.y)), rf);
+                                const float2 v1 = __fmul2_rn(__fmul2_rn(make_float2(gv[kb][e + 2], gv[kb][e + 3]),
+                                                                        make_float2(cf.z, cf.w)), rf);
+                                m[e] = v0.x;
+                                m[e + 1] = v0.y;
+                                m[e + 2] = v1.x;
+                                m[e + 3] = v1.y;
                             }
-                            packed = make_uint4(pack_bf2(m[0], m[1]), pack_bf2(m[2], m[3]), pack_bf2(m[4], m[5]),
-                                                pack_bf2(m[6], m[7]));
+                        } else {
+                            // the row lies inside the group: exact decay for j <= i
+                            const float4* c4 = reinterpret_cast<const float4*>(cs_b + j0);
+                            const float4* d4 = reinterpret_cast<const float4*>(dt_b + j0);
+                            const float4 ca = c4[0], cb = c4[1], da = d4[0], db = d4[1];
+                            const float cj[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                            const float dj[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                m[e] = j0 + e <= i ? gv[kb][e] * __expf(cs_i - cj[e]) * dj[e] : 0.f;
                         }
-                        *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 + sw128_off(i, (kb & 1) * 4 + quarter)) =
-                            packed;
+                        packed = make_uint4(pack_bf2(m[0], m[1]), pack_bf2(m[2], m[3]), pack_bf2(m[4], m[5]),
+                                            pack_bf2(m[6], m[7]));
                     }
+                    *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 + sw128_off(i, (kb & 1) * 4 + quarter)) = packed;
                 }
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[MREADY]);
-            mbar_arrive(&bars[CS_FREE0 + buf]);  // this chunk's dt / cumsum buffer is no longer read
 
             // (f) state passing: S_run <- exp(cs_last) S_run + S_c  (lane i = state row n; 16 columns p)
             if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
@@ -572,6 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     sr[k + 1] = v.y;
                 }
                 tmem_st16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
+                // S_prev is overwritten once Y2 = C S_prev^T of this chunk has read it
+                if (!warp_wait(&bars[EMPTY_BC], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
 #pragma unroll
                 for (int k2 = 0; k2 < 2; ++k2) {
                     uint4 w;
@@ -579,14 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     w.y = pack_bf2(sr[k2 * 8 + 2], sr[k2 * 8 + 3]);
                     w.z = pack_bf2(sr[k2 * 8 + 4], sr[k2 * 8 + 5]);
                     w.w = pack_bf2(sr[k2 * 8 + 6], sr[k2 * 8 + 7]);
-                    // the state entering chunk c+1, into the buffer of that chunk's parity (Y2 of chunk c may
-                    // still be reading the other one)
-                    *reinterpret_cast<uint4*>(sS + ((c + 1) & 1) * 16384 + sw128_off(i, quarter * 2 + k2)) = w;
-                }
-                if (c == nc - 1) {
-                    float* fs = a.final_state + ((size_t)b * a.H + h) * kP * kN;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) fs[(size_t)(quarter * 16 + k) * kN + i] = sr[k];
+                    // the state entering chunk c+1
+                    *reinterpret_cast<uint4*>(sS + sw128_off(i, quarter * 2 + k2)) = w;
                 }
             }
 
@@ -597,30 +593,36 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
 
             // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 16*quarter .. +15
-            if (!warp_wait(&bars[FULL_Z0 + s], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            if (!warp_wait(&bars[FULL_Z], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
             tmem_wait_st();  // this thread's TMEM stores (the conv output read below, the running state) are done
             {
-                uint8_t* rz = sm + OFF_RAWX + s * 16384;  // z in, y out (same positions, this thread's only)
-                TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
+                uint8_t* rz = sm + OFF_Z;  // z in, y out (same positions, this thread's only)
+                const float ecs = __expf(cs_b[i]);  // decay of S_prev up to row i
                 const float2 e2 = make_float2(ecs, ecs), d2 = make_float2(Dh, Dh);
+                // the gate SiLU(z) of this thread's 16 columns
+                float2 gz[8];
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const uint4 zw = *reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2 + k2));
+                    const uint32_t zr[4] = {zw.x, zw.y, zw.z, zw.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) gz[k2 * 4 + e] = silu2(make_float2(bf_lo(zr[e]), bf_hi(zr[e])));
+                }
 #pragma unroll
                 for (int k2 = 0; k2 < 2; ++k2) {  // 8 columns per TMEM round trip
                     float y1[8], y2[8], uu[8];
                     tmem_ld8(tmem + lane_base + COL_Y + quarter * 16 + k2 * 8, y1);
                     tmem_ld8(tmem + lane_base + COL_Y2 + quarter * 16 + k2 * 8, y2);
                     tmem_ld8(tmem + lane_base + COL_U + buf * 64 + quarter * 16 + k2 * 8, uu);
-                    const uint4 zw = *reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2 + k2));
                     tmem_wait_ld();
-                    const uint32_t zr[4] = {zw.x, zw.y, zw.z, zw.w};
                     float o[8];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         float2 yv = __ffma2_rn(e2, make_float2(y2[e], y2[e + 1]), make_float2(y1[e], y1[e + 1]));
                         yv = __ffma2_rn(d2, make_float2(uu[e], uu[e + 1]), yv);
-                        const float2 gz = silu2(make_float2(bf_lo(zr[e >> 1]), bf_hi(zr[e >> 1])));
-                        const float2 ov = __fmul2_rn(yv, gz);
+                        const float2 ov = __fmul2_rn(yv, gz[k2 * 4 + (e >> 1)]);
                         o[e] = ov.x;
                         o[e + 1] = ov.y;
                     }
@@ -629,6 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                             make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]),
                                        pack_bf2(o[6], o[7]));
                     } else if (i < Qc) {
+                        TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
                         float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
                         dst[0] = make_float4(o[0], o[1], o[2], o[3]);
                         dst[1] = make_float4(o[4], o[5], o[6], o[7]);
@@ -637,7 +640,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars[EMPTY_RAW0 + s]);
+            mbar_arrive(&bars[EPI_DONE]);
+            mbar_arrive(&bars[CS_FREE0 + buf]);  // this chunk's dt / cumsum buffer is no longer read
+        }
+        // final state: the running state after the last chunk (this thread's 16 columns p of row n = i)
+        if (nc > 0 && !*abort_flag) {
+            float sr[16];
+            tmem_ld16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
+            tmem_wait_ld();
+            float* fs = a.final_state + ((size_t)b * a.H + h) * kP * kN;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) fs[(size_t)(quarter * 16 + k) * kN + i] = sr[k];
         }
     }
 
@@ -754,9 +767,24 @@ bool make_map(CUtensorMap* m, const void* base, int64_t width, int64_t L, int64_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over dt [batch][L][H] with a [1][128][8] box (8 heads x 128 tokens, no swizzle); needs H % 8 == 0.
+bool make_dt_map(CUtensorMap* m, const void* base, int64_t H, int64_t L, int64_t batch) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || H % 8 != 0) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)H * 2, (cuuint64_t)(H * L * 2)};
+    const cuuint32_t box[3] = {8, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
-bool prefill_tc_supported(int P, int N, int Q, bool bf16) { return bf16 && P == kP && N == kN && Q == kQ; }
+bool prefill_tc_supported(int P, int N, int Q, int H, bool bf16) {
+    return bf16 && P == kP && N == kN && Q == kQ && H % 8 == 0;  // dt tiles are loaded 8 heads wide
+}
 
 size_t prefill_tc_workspace_bytes(int64_t batch, int64_t L, int G, int N) {
     return (size_t)batch * (size_t)L * 2 * (size_t)G * (size_t)N * 2;
@@ -768,7 +796,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     prm.a = a;
     if (!make_map(&prm.tm_x, a.x, a.HP, a.L, a.batch) || !make_map(&prm.tm_z, a.z, a.HP, a.L, a.batch) ||
         (kind == ActKind::BF16 && !make_map(&prm.tm_y, a.y, a.HP, a.L, a.batch)) ||
-        !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, a.batch))
+        !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, a.batch) ||
+        !make_dt_map(&prm.tm_dt, a.dt, a.H, a.L, a.batch))
         return cudaErrorInvalidValue;
     const int ntok = (int)((a.L + kProTok - 1) / kProTok);
     const int64_t tail = a.batch * (int64_t)a.conv_dim * 3;
