@@ -180,6 +180,33 @@ SSD_API ssd_status ssd_prefill_noalloc(const ssd_dims* dims, ssd_dtype dtype, co
                                void* y, float* final_state, void* conv_state, void* stream);
 
 /*
+ * Packed variable-length prefill (continuous batching).  dims->batch = nseq
+ * sequences of different lengths are laid back to back along the token axis;
+ * dims->seqlen = T, their total.  Sequence s is rows cu_seqlens[s] ..
+ * cu_seqlens[s+1]-1; each is scanned on its own, from its own initial states,
+ * exactly as ssd_prefill scans one sequence of a batch (chunked prefill with
+ * per-sequence states, the serving-stack gap the "EP6" survey's vLLM section
+ * names).
+ *   cu_seqlens  DEVICE array of nseq+1 int64 (8-byte aligned): 0 = cu[0] <= cu[1]
+ *               <= ... <= cu[nseq] = T; empty sequences are allowed.  The kernels
+ *               read it; a sequence whose offsets are out of order or outside
+ *               [0, T] is treated as empty and ssd_device_status() then reports
+ *               SSD_ERR_SHAPE.
+ *   x, z        [T][H*P]     dtype;  dt [T][H];  B, C [T][G][N];  y [T][H*P] (out)
+ *   init_state  [nseq][H][P][N] fp32 or NULL;  init_conv_state [nseq][conv_dim][3] or NULL
+ *   final_state [nseq][H][P][N] fp32 (out);   conv_state [nseq][conv_dim][3] (out)
+ *   workspace   at least ssd_prefill_varlen_workspace_bytes() bytes (the
+ *               post-conv B/C of all T rows on the tensor-core path, else 0)
+ * Same kernel paths, argument rules and error codes as ssd_prefill.
+ */
+SSD_API size_t ssd_prefill_varlen_workspace_bytes(const ssd_dims* dims, ssd_dtype dtype);
+SSD_API ssd_status ssd_prefill_varlen(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
+                                      const int64_t* cu_seqlens, const void* x, const void* dt, const void* B,
+                                      const void* C, const void* z, const float* init_state,
+                                      const void* init_conv_state, void* y, float* final_state,
+                                      void* conv_state, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream` and reports whether a kernel launched by this library
  * gave up on a bounded device-side wait since the last call (SSD_ERR_TIMEOUT;
  * its outputs are then incomplete), or whether the stream holds a CUDA error

@@ -125,6 +125,39 @@ def prefill(inp: dict, unit_mask=None, nthreads: int | None = None):
     return y, fs, cs
 
 
+def prefill_varlen(inp: dict, cu_seqlens, nthreads: int | None = None):
+    """Packed variable-length prefill: x/z [T, H*P], dt [T, H], B/C [T, G, N], init_state
+    [nseq, H, P, N] or None, init_conv_state [nseq, conv_dim, 3] or None; sequence s is rows
+    cu_seqlens[s] .. cu_seqlens[s+1]-1.  Each sequence is an independent prefill from its own
+    initial states (the per-sequence chunked prefill of serving stacks, "EP6" survey, vLLM
+    section), so this is ``prefill`` run on each slice.
+    Returns (y [T, H*P], final_state [nseq, H, P, N], conv_state [nseq, conv_dim, 3]).
+    """
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    x = _f64(inp["x"])
+    T, HP = x.shape
+    G, N = inp["B"].shape[1], inp["B"].shape[2]
+    H = inp["A"].shape[0]
+    P = HP // H
+    nseq = len(cu) - 1
+    y = np.empty((T, HP))
+    fs = np.empty((nseq, H, P, N))
+    cs = np.empty((nseq, HP + 2 * G * N, 3))
+    params = {k: inp[k] for k in ("A", "D", "dt_bias", "conv_w", "conv_b")}
+    for s in range(nseq):
+        r0, r1 = cu[s], cu[s + 1]
+        one = dict(params)
+        for k in ("x", "dt", "B", "C", "z"):
+            one[k] = _f64(inp[k])[r0:r1][None]
+        for k in ("init_state", "init_conv_state"):
+            one[k] = None if inp.get(k) is None else _f64(inp[k])[s:s + 1]
+        ys, fss, css = prefill(one, nthreads=nthreads)
+        y[r0:r1] = ys[0]
+        fs[s] = fss[0]
+        cs[s] = css[0]
+    return y, fs, cs
+
+
 def decode_step(step: dict, params: dict, conv_state, ssm_state, unit_mask=None):
     """One fp64 decode step.  ``conv_state`` and ``ssm_state`` must be float64
     numpy arrays; they are updated in place.  Returns y [Bt, H*P]."""

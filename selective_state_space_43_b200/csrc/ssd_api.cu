@@ -110,6 +110,60 @@ ssd_status ssd_prefill(const ssd_dims* d, ssd_dtype dtype, const ssd_params* par
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
+size_t ssd_prefill_varlen_workspace_bytes(const ssd_dims* d, ssd_dtype dtype) {
+    if (ssd_prefill_path(d, dtype) != 1) return 0;
+    return ssd::prefill_tc_workspace_bytes(1, d->seqlen, d->ngroups, d->d_state);  // post-conv B/C of all rows
+}
+
+ssd_status ssd_prefill_varlen(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params,
+                              const int64_t* cu_seqlens, const void* x, const void* dt, const void* B,
+                              const void* C, const void* z, const float* init_state, const void* init_conv_state,
+                              void* y, float* final_state, void* conv_state, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    ssd_status st = check_dims(d, dtype, true);
+    if (st != SSD_OK) return st;
+    if ((st = check_params(params)) != SSD_OK) return st;
+    if (d->seqlen > (1LL << 31) - 256) return SSD_ERR_SHAPE;  // tensor-map row coordinates are 32-bit
+    if (!cu_seqlens && d->batch > 0) return SSD_ERR_NULL;
+    const bool tokens = d->seqlen > 0;
+    if (tokens && (!x || !dt || !B || !C || !z || !y)) return SSD_ERR_NULL;
+    if (d->batch > 0 && (!final_state || !conv_state)) return SSD_ERR_NULL;
+    const void* ptrs[] = {x, dt, B, C, z, init_state, init_conv_state, y, final_state, conv_state, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return SSD_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(cu_seqlens) & 7u) return SSD_ERR_ALIGN;
+    if ((tokens && (y == x || y == z)) || (init_conv_state && init_conv_state == conv_state))
+        return SSD_ERR_UNSUPPORTED;
+    const int path = ssd_prefill_path(d, dtype);
+    const size_t need = ssd_prefill_varlen_workspace_bytes(d, dtype);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
+    if (d->batch == 0) return SSD_OK;
+    int* err = ssd::device_error_flag();
+    if (!err) return SSD_ERR_CUDA;
+
+    const ssd::Shape s = ssd::make_shape(*d);
+    ssd::PrefillArgs a;
+    a.batch = s.batch;
+    a.L = s.seqlen;  // all rows
+    a.nchunks = s.nchunks;
+    a.H = s.H; a.P = s.P; a.N = s.N; a.G = s.G; a.Q = s.Q;
+    a.HP = s.HP; a.GN = s.GN; a.conv_dim = s.conv_dim; a.hpg = s.heads_per_group;
+    a.A = params->A; a.D = params->D; a.dt_bias = params->dt_bias;
+    a.conv_w = params->conv_w; a.conv_b = params->conv_b;
+    a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z;
+    a.init_state = init_state; a.init_conv_state = init_conv_state;
+    a.y = y; a.final_state = final_state; a.conv_state = conv_state;
+    a.workspace = workspace;
+    a.cu = cu_seqlens;
+    a.err = err;
+    const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
+                                                                                        : ssd::ActKind::BF16_YF32);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = path == 1 ? ssd::launch_prefill_tc(a, kind, cs, g_hook)
+                              : ssd::launch_prefill_simt(a, kind, cs, g_hook);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
 ssd_status ssd_decode_step(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params, const void* x,
                            const void* dt, const void* B, const void* C, const void* z, void* conv_state,
                            float* ssm_state, void* y, void* stream) {
@@ -139,7 +193,8 @@ ssd_status ssd_decode_step(const ssd_dims* d, ssd_dtype dtype, const ssd_params*
 ssd_status ssd_device_status(void* stream) {
     int flag = 0;
     if (ssd::read_and_clear_tc_error(&flag, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSD_ERR_CUDA;
-    return flag ? SSD_ERR_TIMEOUT : SSD_OK;
+    if (flag & ssd::kErrTimeout) return SSD_ERR_TIMEOUT;
+    return flag & ssd::kErrBadSeqlens ? SSD_ERR_SHAPE : SSD_OK;
 }
 
 ssd_status ssd_set_timing_events(void* before_main, void* after_main) {

@@ -41,7 +41,30 @@ struct PrefillArgs {
     float* final_state;
     void* conv_state;
     void* workspace;  // tensor-core path: post-conv B and C, [batch*L][2][G][N] bf16
+    // Packed variable-length batch: device array of batch+1 row offsets (cu[0] = 0, cu[batch] = L);
+    // sequence b is rows cu[b] .. cu[b+1]-1 of [L][...] activations.  nullptr: batch x L layout.
+    const int64_t* cu = nullptr;
+    int* err = nullptr;  // device error word (bit 1: a sequence's offsets were invalid)
 };
+
+// Device error word bits, read back by ssd_device_status.
+constexpr int kErrTimeout = 1, kErrBadSeqlens = 2;
+
+// Rows of sequence b: the first row in the [rows][...] activation arrays, the length, and whether its
+// offsets were valid (0 <= cu[b] <= cu[b+1] <= L); an invalid sequence is treated as empty.
+struct SeqSpan {
+    int64_t row0, len;
+    bool ok;
+};
+__device__ inline SeqSpan seq_span(const PrefillArgs& a, int64_t b) {
+    if (!a.cu) return SeqSpan{b * a.L, a.L, true};
+    const int64_t r0 = a.cu[b], r1 = a.cu[b + 1];
+    if (r0 < 0 || r1 < r0 || r1 > a.L) return SeqSpan{0, 0, false};
+    return SeqSpan{r0, r1 - r0, true};
+}
+
+// The device error word of the current device (nullptr if it cannot be found).
+int* device_error_flag();
 
 cudaError_t launch_decode(const DecodeArgs& a, int64_t batch, ActKind kind, cudaStream_t st, const TimingHook& hook);
 

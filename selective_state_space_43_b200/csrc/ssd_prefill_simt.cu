@@ -38,15 +38,16 @@ struct SimtSmem {
 };
 
 template <typename T>
-__device__ __forceinline__ float raw_at(const PrefillArgs& a, int64_t b, int64_t s, int c) {
-    // pre-conv value of channel c at token s of sequence b; s < 0 reads the history
+__device__ __forceinline__ float raw_at(const PrefillArgs& a, int64_t b, int64_t row0, int64_t s, int c) {
+    // pre-conv value of channel c at token s of sequence b (whose rows start at row0); s < 0 reads the history
     if (s < 0) {
         if (!a.init_conv_state) return 0.f;
         return to_f32(static_cast<const T*>(a.init_conv_state)[((size_t)b * a.conv_dim + c) * 3 + (s + 3)]);
     }
-    if (c < a.HP) return to_f32(static_cast<const T*>(a.x)[((size_t)b * a.L + s) * a.HP + c]);
-    if (c < a.HP + a.GN) return to_f32(static_cast<const T*>(a.B)[((size_t)b * a.L + s) * a.GN + (c - a.HP)]);
-    return to_f32(static_cast<const T*>(a.C)[((size_t)b * a.L + s) * a.GN + (c - a.HP - a.GN)]);
+    const size_t row = (size_t)(row0 + s);
+    if (c < a.HP) return to_f32(static_cast<const T*>(a.x)[row * a.HP + c]);
+    if (c < a.HP + a.GN) return to_f32(static_cast<const T*>(a.B)[row * a.GN + (c - a.HP)]);
+    return to_f32(static_cast<const T*>(a.C)[row * a.GN + (c - a.HP - a.GN)]);
 }
 
 template <typename T, typename TY, int N, int Q>
@@ -65,6 +66,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
 
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
     const int g = h / a.hpg;
+    const SeqSpan span = seq_span(a, b);  // rows of sequence b and its length
+    if (!span.ok && threadIdx.x == 0 && a.err) atomicOr(a.err, kErrBadSeqlens);
+    const int64_t Ls = span.len, nchunks = (Ls + Q - 1) / Q;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const float A = a.A[h], Dh = a.D[h], dtb = a.dt_bias[h];
     const int cx = h * kP, cb = a.HP + g * N, cc = a.HP + a.GN + g * N;
@@ -74,9 +78,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
         sS[p * NB + n] = a.init_state ? a.init_state[((size_t)b * a.H + h) * kP * N + i] : 0.f;
     }
 
-    for (int64_t c = 0; c < a.nchunks; ++c) {
+    for (int64_t c = 0; c < nchunks; ++c) {
         const int64_t t0 = c * Q;
-        const int Qc = (int)(a.L - t0 < Q ? a.L - t0 : Q);
+        const int Qc = (int)(Ls - t0 < Q ? Ls - t0 : Q);
         __syncthreads();  // previous chunk fully consumed
 
         // 1. conv + SiLU of the head's channels, dt and the in-chunk cumsum.
@@ -88,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
             const float* w = a.conv_w + (size_t)ch * 4;
             float acc = a.conv_b[ch];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc += w[k] * raw_at<T>(a, b, t0 + t - 3 + k, ch);
+            for (int k = 0; k < 4; ++k) acc += w[k] * raw_at<T>(a, b, span.row0, t0 + t - 3 + k, ch);
             const float u = silu_f(acc);
             if (j < kP) sX[t * kP + j] = u;
             else if (j < kP + N) sB[t * NB + (j - kP)] = u;
@@ -103,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
                 const int t = lane * PER + k;
                 float dA = 0.f;
                 if (t < Qc) {
-                    const float dtv = softplus_f(to_f32(static_cast<const T*>(a.dt)[((size_t)b * a.L + t0 + t) * a.H + h]) + dtb);
+                    const float dtv = softplus_f(to_f32(static_cast<const T*>(a.dt)[((size_t)span.row0 + t0 + t) * a.H + h]) + dtb);
                     sDt[t] = dtv;
                     dA = dtv * A;
                 } else {
@@ -148,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
 #pragma unroll 8
                 for (int n = 0; n < N; ++n) off += sC[t * N + n] * sS[p * NB + n];
                 const float yv = acc + dec * off + Dh * sX[t * kP + p];
-                const size_t o = ((size_t)b * a.L + t0 + t) * a.HP + cx + p;
+                const size_t o = ((size_t)span.row0 + t0 + t) * a.HP + cx + p;
                 const float zv = to_f32(static_cast<const T*>(a.z)[o]);
                 static_cast<TY*>(a.y)[o] = from_f32<TY>(yv * silu_f(zv));
             }
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
     for (int i = tid; i < nch * 3; i += kThreads) {
         const int j = i / 3, k = i % 3;
         const int ch = j < kP ? cx + j : (j < kP + N ? cb + (j - kP) : cc + (j - kP - N));
-        const float v = raw_at<T>(a, b, a.L - 3 + k, ch);
+        const float v = raw_at<T>(a, b, span.row0, Ls - 3 + k, ch);
         static_cast<T*>(a.conv_state)[((size_t)b * a.conv_dim + ch) * 3 + k] = from_f32<T>(v);
     }
 }

@@ -54,7 +54,7 @@
 
 namespace ssd {
 
-__device__ int g_tc_error = 0;  // set by a chunk_scan CTA whose bounded wait gave up
+__device__ int g_tc_error = 0;  // device error word: kErrTimeout | kErrBadSeqlens
 
 namespace {
 
@@ -127,10 +127,6 @@ __device__ __forceinline__ float tanh_approx(float v) {
     asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
     return r;
 }
-__device__ __forceinline__ float silu_fast(float v) {
-    const float hv = 0.5f * v;
-    return fmaf(hv, tanh_approx(hv), hv);
-}
 
 // softplus(v) = log(1 + e^v) with the fast exp / log (absolute error ~1e-7
 // for the small dt this layer uses); above 20 the correction is below 2.1e-9.
@@ -156,23 +152,32 @@ __device__ __forceinline__ void mma_k128(uint32_t d_tmem, uint64_t a0, uint64_t 
     }
 }
 
+// Whether bf16 y of chunk c leaves through the TMA store of its smem tile.  The store clips rows beyond
+// the tensor map (the end of a [batch][L] row), but in a packed batch the rows past a sequence's end
+// belong to the next sequence, so a partial last chunk there is stored from registers instead.
+template <bool kVarlen>
+__device__ __forceinline__ bool tma_y_chunk(int64_t Ls, int c) {
+    return !kVarlen || Ls - (int64_t)c * kQ >= kQ;
+}
+
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
     *abort_flag = 1;
-    atomicExch(&g_tc_error, 1);
+    atomicOr(&g_tc_error, kErrTimeout);
 }
 
 // Row-major x conv of chunk cc for the calling thread: token row i, channels 16*quarter .. +15.
 // Writes X and X' (bf16, smem operands) and the fp32 conv output into TMEM (for the D skip), and the
 // raw history of the next chunk.  Returns false if a wait gave up.
 __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, uint64_t* bars, volatile int* abort_flag,
-                                           uint32_t tmem, uint32_t lane_base, int cc, int nc, int i, int quarter) {
+                                           uint32_t tmem, uint32_t lane_base, int cc, int nc, int64_t Ls, int i,
+                                           int quarter) {
     const int buf = cc & 1;
     if (!warp_wait(&bars[CS_READY0 + buf], (cc >> 1) & 1, abort_flag)) return false;
     if (!warp_wait(&bars[FULL_RAW0 + buf], (cc >> 1) & 1, abort_flag)) return false;
     // the raw history rows were written by other threads in the previous chunk's conv
     if (cc >= 1 && !warp_wait(&bars[XREADY0 + ((cc - 1) & 1)], ((cc - 1) >> 1) & 1, abort_flag)) return false;
     const int64_t t0 = (int64_t)cc * kQ;
-    const int Qc = (int)(a.L - t0 < kQ ? a.L - t0 : kQ);
+    const int Qc = (int)(Ls - t0 < kQ ? Ls - t0 : kQ);
     const bool valid = i < Qc;
     const uint8_t* rx = sm + OFF_RAWX + buf * 16384;
     const uint4* halo_in = reinterpret_cast<const uint4*>(sm + OFF_HALO + (cc & 1) * 384);
@@ -236,7 +241,8 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
     return true;
 }
 
-template <typename TY>
+// kVarlen: a packed variable-length batch (a.cu set); the batch x L layout otherwise.
+template <typename TY, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_constant__ TcParams prm) {
     const PrefillArgs& a = prm.a;
     extern __shared__ uint8_t smem_raw[];
@@ -255,7 +261,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
     const int g = h / a.hpg;
-    const int nc = (int)a.nchunks;
+    // sequence b: its rows in the activation arrays, its length and chunk count; the tensor maps are
+    // [batch][L][width] (coordinates: token c*Q, batch b) or, for a packed batch, [1][rows][width]
+    // (coordinates: token row0 + c*Q, batch 0)
+    const SeqSpan span = kVarlen ? seq_span(a, b) : SeqSpan{(int64_t)b * a.L, a.L, true};
+    if (!span.ok && threadIdx.x == 0) atomicOr(&g_tc_error, kErrBadSeqlens);
+    const int64_t Ls = span.len;
+    const int nc = (int)((Ls + kQ - 1) / kQ);
+    const int tok0 = kVarlen ? (int)span.row0 : 0;
+    const int mb = kVarlen ? 0 : b;
 
     if (threadIdx.x == 0) {
         for (int k = 0; k < NBAR; ++k) {
@@ -311,18 +325,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             auto load_x = [&](int c) {  // raw x of chunk c and its dt (the 8-head column block holding h)
                 const int s = c & 1;
                 mbar_arrive_expect_tx(&bars[FULL_RAW0 + s], 16384 + 2048);
-                tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, c * kQ, b);
-                tma_load_3d(sm + OFF_DTRAW + s * 2048, &prm.tm_dt, &bars[FULL_RAW0 + s], h & ~7, c * kQ, b);
+                tma_load_3d(sm + OFF_RAWX + s * 16384, &prm.tm_x, &bars[FULL_RAW0 + s], h * kP, tok0 + c * kQ, mb);
+                tma_load_3d(sm + OFF_DTRAW + s * 2048, &prm.tm_dt, &bars[FULL_RAW0 + s], h & ~7, tok0 + c * kQ, mb);
                 if (s) issued_x1 = c;
                 else issued_x0 = c;
             };
             auto load_z = [&](int c) {
                 mbar_arrive_expect_tx(&bars[FULL_Z], 16384);
-                tma_load_3d(sm + OFF_Z, &prm.tm_z, &bars[FULL_Z], h * kP, c * kQ, b);
+                tma_load_3d(sm + OFF_Z, &prm.tm_z, &bars[FULL_Z], h * kP, tok0 + c * kQ, mb);
                 issued_z = c;
             };
             for (int c = 0; c < nc && c < 2; ++c) load_x(c);
-            load_z(0);
+            if (nc > 0) load_z(0);
             for (int c = 0; c < nc; ++c) {
                 if (c + 2 < nc) {  // x(c+2), once chunk c's conv has consumed x(c)
                     if (!mbar_wait(&bars[XREADY0 + (c & 1)], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
@@ -330,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 }
                 // y(c) out of the z buffer once chunk c's epilogue is complete, then z(c+1) in
                 if (!mbar_wait(&bars[EPI_DONE], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
-                if constexpr (kTmaStoreY) {
-                    tma_store_3d(&prm.tm_y, sm + OFF_Z, h * kP, c * kQ, b);
+                if (kTmaStoreY && tma_y_chunk<kVarlen>(Ls, c)) {
+                    tma_store_3d(&prm.tm_y, sm + OFF_Z, h * kP, tok0 + c * kQ, mb);
                     bulk_commit();
                     bulk_wait_read_all();  // the buffer may be refilled once the store has read it
                 }
@@ -356,10 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
                 const int xc = a.GN + g * kN, xb = g * kN;
-                tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, c * kQ, b);
-                tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, c * kQ, b);
-                tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, c * kQ, b);
-                tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, c * kQ, b);
+                tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, tok0 + c * kQ, mb);
+                tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, tok0 + c * kQ, mb);
+                tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, tok0 + c * kQ, mb);
+                tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, tok0 + c * kQ, mb);
                 last = c;
             }
             if (*abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
@@ -377,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 break;
             }
             if (!warp_wait(&bars[FULL_RAW0 + buf], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
-            const int Qc = (int)(a.L - (int64_t)c * kQ < kQ ? a.L - (int64_t)c * kQ : kQ);
+            const int Qc = (int)(Ls - (int64_t)c * kQ < kQ ? Ls - (int64_t)c * kQ : kQ);
             const __nv_bfloat16* dtr = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_DTRAW + buf * 2048) + (h & 7);
             float dtv[4], cs[4];
             float run = 0.f;
@@ -491,12 +505,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             tmem_wait_st();
         }
 
-        bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, i, quarter);
+        bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, Ls, i, quarter);
         if (!ok) raise_abort(abort_flag);
         for (int c = 0; c < nc && ok; ++c) {
             const int buf = c & 1;
             const int64_t t0 = (int64_t)c * kQ;
-            const int Qc = (int)(a.L - t0 < kQ ? a.L - t0 : kQ);
+            const int Qc = (int)(Ls - t0 < kQ ? Ls - t0 : kQ);
+            const bool tma_y = kTmaStoreY && tma_y_chunk<kVarlen>(Ls, c);  // else y is stored from registers
             const float* cs_b = s_cs + buf * 128;
             const float cs_i = cs_b[i];
             const float cs_last = cs_b[kQ - 1];
@@ -587,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             }
 
             // (c) the next chunk's x conv (its S_c then overlaps this chunk's Y = M X and epilogue)
-            if (c + 1 < nc && !conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, c + 1, nc, i, quarter)) {
+            if (c + 1 < nc && !conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, c + 1, nc, Ls, i, quarter)) {
                 raise_abort(abort_flag);
                 break;
             }
@@ -626,15 +641,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                         o[e] = ov.x;
                         o[e + 1] = ov.y;
                     }
-                    if constexpr (kTmaStoreY) {
+                    if (tma_y) {
                         *reinterpret_cast<uint4*>(rz + sw128_off(i, quarter * 2 + k2)) =
                             make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]),
                                        pack_bf2(o[6], o[7]));
                     } else if (i < Qc) {
-                        TY* yrow = static_cast<TY*>(a.y) + ((size_t)b * a.L + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
-                        float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
-                        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-                        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+                        TY* yrow = static_cast<TY*>(a.y) + ((size_t)span.row0 + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
+                        if constexpr (sizeof(TY) == 2) {
+                            *reinterpret_cast<uint4*>(yrow + k2 * 8) =
+                                make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]),
+                                           pack_bf2(o[6], o[7]));
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
+                            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+                        }
                     }
                 }
             }
@@ -644,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             mbar_arrive(&bars[CS_FREE0 + buf]);  // this chunk's dt / cumsum buffer is no longer read
         }
         // final state: the running state after the last chunk (this thread's 16 columns p of row n = i)
-        if (nc > 0 && !*abort_flag) {
+        if (!*abort_flag) {  // (an empty sequence passes its initial state through)
             float sr[16];
             tmem_ld16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
             tmem_wait_ld();
@@ -661,17 +682,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     }
 }
 
-// SiLU(conv4) of the B and C channels into the workspace [b][t][2][G*N] (bf16),
+// SiLU(conv4) of the B and C channels into the workspace [row][2][G*N] (bf16),
 // and the conv_state output (pre-conv inputs of the last 3 tokens of every channel).
-// Blocks with blockIdx.x < ntok: 256 channel pairs (bf16x2) over kProTok tokens each; a
+// Blocks with blockIdx.x < ntok: 256 channel pairs (bf16x2) over kProTok rows each; a
 // thread issues all kProTok + 3 loads of its window before the first FMA.  Blocks with
 // blockIdx.x >= ntok (and blockIdx.z == 0): the conv_state tail, one element per thread.
+// In a packed batch (a.cu) the window runs over all rows; taps that reach before the
+// start of a row's sequence take that sequence's initial conv state (or zero) instead.
 constexpr int kProTok = 16;
 
+// Pre-conv value of channel c at position t (< 3 tokens before the start) of sequence b's history.
+__device__ __forceinline__ __nv_bfloat16 conv_history(const PrefillArgs& a, int64_t b, int c, int64_t t) {
+    const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.init_conv_state);
+    return hist ? hist[((size_t)b * a.conv_dim + c) * 3 + (t + 3)] : __float2bfloat16_rn(0.f);
+}
+
+template <bool kVarlen>
 __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int ntok) {
     // the chunk scan may start its launch now; it waits for this grid before reading the workspace
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.init_conv_state);
     if ((int)blockIdx.x >= ntok) {
         if (blockIdx.z != 0) return;
         const int64_t e = ((int64_t)(blockIdx.x - ntok) * gridDim.y + blockIdx.y) * 256 + threadIdx.x;
@@ -679,21 +708,22 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
         const int k = (int)(e % 3);
         const int c = (int)((e / 3) % a.conv_dim);
         const int64_t b = e / (3 * (int64_t)a.conv_dim);
-        const int64_t t = a.L - 3 + k;
+        const SeqSpan sp = kVarlen ? seq_span(a, b) : SeqSpan{b * a.L, a.L, true};
+        const int64_t t = sp.len - 3 + k;  // position in the sequence
         __nv_bfloat16 v;
         if (t >= 0) {
-            if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[((size_t)b * a.L + t) * a.HP + c];
-            else if (c < a.HP + a.GN)
-                v = static_cast<const __nv_bfloat16*>(a.B)[((size_t)b * a.L + t) * a.GN + (c - a.HP)];
-            else v = static_cast<const __nv_bfloat16*>(a.C)[((size_t)b * a.L + t) * a.GN + (c - a.HP - a.GN)];
+            const size_t row = (size_t)(sp.row0 + t);
+            if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[row * a.HP + c];
+            else if (c < a.HP + a.GN) v = static_cast<const __nv_bfloat16*>(a.B)[row * a.GN + (c - a.HP)];
+            else v = static_cast<const __nv_bfloat16*>(a.C)[row * a.GN + (c - a.HP - a.GN)];
         } else {
-            v = hist ? hist[((size_t)b * a.conv_dim + c) * 3 + (t + 3)] : __float2bfloat16_rn(0.f);
+            v = conv_history(a, b, c, t);
         }
         static_cast<__nv_bfloat16*>(a.conv_state)[e] = v;
         return;
     }
-    const int64_t b = blockIdx.y;
-    const int64_t t0 = (int64_t)blockIdx.x * kProTok;
+    const int64_t b = blockIdx.y;  // 0 for a packed batch
+    const int64_t t0 = (int64_t)blockIdx.x * kProTok;  // first row of the window within [0, L)
     const int half_gn = a.GN / 2;                    // channel pairs per array
     const int pair = blockIdx.z * 256 + threadIdx.x;  // 0 .. GN-1 over both arrays
     if (pair >= a.GN) return;
@@ -705,7 +735,7 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
     const float4 w0 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cglob * 4);
     const float4 w1 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(cglob + 1) * 4);
     const float2 bias = make_float2(a.conv_b[cglob], a.conv_b[cglob + 1]);
-    float2 v[kProTok + 3];  // tokens t0-3 .. t0+kProTok-1, channels (2cp, 2cp+1)
+    float2 v[kProTok + 3];  // rows t0-3 .. t0+kProTok-1, channels (2cp, 2cp+1)
     uint32_t raw[kProTok + 3];
 #pragma unroll
     for (int k = 0; k < kProTok + 3; ++k) {
@@ -715,21 +745,51 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
 #pragma unroll
     for (int k = 0; k < kProTok + 3; ++k) {
         const int64_t t = t0 - 3 + k;
-        if (t < 0 && hist)
-            v[k] = make_float2(__bfloat162float(hist[((size_t)b * a.conv_dim + cglob) * 3 + (t + 3)]),
-                               __bfloat162float(hist[((size_t)b * a.conv_dim + cglob + 1) * 3 + (t + 3)]));
+        if (!kVarlen && t < 0)
+            v[k] = make_float2(__bfloat162float(conv_history(a, b, cglob, t)),
+                               __bfloat162float(conv_history(a, b, cglob + 1, t)));
         else
             v[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
+    }
+    // packed batch: the sequence of row t0 and where the next one starts
+    int64_t seq = 0, start = 0, next = a.L;
+    if constexpr (kVarlen) {
+        int64_t lo = 0, hi = a.batch;  // largest seq with cu[seq] <= t0 (empty sequences skipped)
+        while (hi - lo > 1) {
+            const int64_t mid = (lo + hi) >> 1;
+            if (a.cu[mid] <= t0) lo = mid;
+            else hi = mid;
+        }
+        seq = lo;
+        start = a.cu[seq];
+        next = a.cu[seq + 1];
     }
 #pragma unroll
     for (int k = 0; k < kProTok; ++k) {
         const int64_t t = t0 + k;
         if (t < a.L) {
+            float2 x4[4] = {v[k], v[k + 1], v[k + 2], v[k + 3]};
+            if constexpr (kVarlen) {
+                while (t >= next && seq + 1 < a.batch) {  // row t opens a later sequence
+                    ++seq;
+                    start = next;
+                    next = a.cu[seq + 1];
+                }
+                if (start <= t && t - 3 < start) {  // within 3 rows of its sequence's start: taps before it are history
+#pragma unroll
+                    for (int j = 0; j < 3; ++j) {
+                        const int64_t tt = t - 3 + j;
+                        if (tt < start)
+                            x4[j] = make_float2(__bfloat162float(conv_history(a, seq, cglob, tt - start)),
+                                                __bfloat162float(conv_history(a, seq, cglob + 1, tt - start)));
+                    }
+                }
+            }
             float2 p = bias;
-            p = __ffma2_rn(make_float2(w0.x, w1.x), v[k], p);
-            p = __ffma2_rn(make_float2(w0.y, w1.y), v[k + 1], p);
-            p = __ffma2_rn(make_float2(w0.z, w1.z), v[k + 2], p);
-            p = __ffma2_rn(make_float2(w0.w, w1.w), v[k + 3], p);
+            p = __ffma2_rn(make_float2(w0.x, w1.x), x4[0], p);
+            p = __ffma2_rn(make_float2(w0.y, w1.y), x4[1], p);
+            p = __ffma2_rn(make_float2(w0.z, w1.z), x4[2], p);
+            p = __ffma2_rn(make_float2(w0.w, w1.w), x4[3], p);
             const float2 u = silu2(p);
             dst[(size_t)t * 2 * half_gn] = pack_bf2(u.x, u.y);
         }
@@ -794,19 +854,23 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     if (a.L == 0) return launch_prefill_simt(a, kind, st, hook);  // nothing to scan: states pass through
     TcParams prm;
     prm.a = a;
-    if (!make_map(&prm.tm_x, a.x, a.HP, a.L, a.batch) || !make_map(&prm.tm_z, a.z, a.HP, a.L, a.batch) ||
-        (kind == ActKind::BF16 && !make_map(&prm.tm_y, a.y, a.HP, a.L, a.batch)) ||
-        !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, a.batch) ||
-        !make_dt_map(&prm.tm_dt, a.dt, a.H, a.L, a.batch))
+    const int64_t mbatch = a.cu ? 1 : a.batch;  // a packed batch is one [L] row of the maps
+    if (!make_map(&prm.tm_x, a.x, a.HP, a.L, mbatch) || !make_map(&prm.tm_z, a.z, a.HP, a.L, mbatch) ||
+        (kind == ActKind::BF16 && !make_map(&prm.tm_y, a.y, a.HP, a.L, mbatch)) ||
+        !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, mbatch) ||
+        !make_dt_map(&prm.tm_dt, a.dt, a.H, a.L, mbatch))
         return cudaErrorInvalidValue;
     const int ntok = (int)((a.L + kProTok - 1) / kProTok);
     const int64_t tail = a.batch * (int64_t)a.conv_dim * 3;
-    const int tail_blocks = (int)((tail + 256 * a.batch - 1) / (256 * a.batch));
-    const dim3 pgrid((unsigned)(ntok + tail_blocks), (unsigned)a.batch, (unsigned)((a.GN + 255) / 256));
-    bc_prologue_kernel<<<pgrid, 256, 0, st>>>(a, ntok);
+    const int tail_blocks = (int)((tail + 256 * mbatch - 1) / (256 * mbatch));
+    const dim3 pgrid((unsigned)(ntok + tail_blocks), (unsigned)mbatch, (unsigned)((a.GN + 255) / 256));
+    if (a.cu) bc_prologue_kernel<true><<<pgrid, 256, 0, st>>>(a, ntok);
+    else bc_prologue_kernel<false><<<pgrid, 256, 0, st>>>(a, ntok);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    auto kern = kind == ActKind::BF16_YF32 ? chunk_scan_kernel<float> : chunk_scan_kernel<__nv_bfloat16>;
+    auto kern = kind == ActKind::BF16_YF32 ? (a.cu ? chunk_scan_kernel<float, true> : chunk_scan_kernel<float, false>)
+                                           : (a.cu ? chunk_scan_kernel<__nv_bfloat16, true>
+                                                   : chunk_scan_kernel<__nv_bfloat16, false>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the scan's set-up (TMEM, barriers, state, first x conv)
@@ -826,6 +890,18 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     if (e != cudaSuccess) return e;
     hook.after(st);
     return cudaGetLastError();
+}
+
+int* device_error_flag() {
+    static int* ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_tc_error) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int*>(p);
+    }
+    return ptrs[dev];
 }
 
 cudaError_t read_and_clear_tc_error(int* flag, cudaStream_t st) {

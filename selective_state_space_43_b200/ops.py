@@ -63,6 +63,10 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 11 + [sz, vp]
         L.ssd_decode_step.restype = ctypes.c_int
         L.ssd_decode_step.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 8 + [vp]
+        L.ssd_prefill_varlen_workspace_bytes.restype = sz
+        L.ssd_prefill_varlen_workspace_bytes.argtypes = [dimp, ctypes.c_int]
+        L.ssd_prefill_varlen.restype = ctypes.c_int
+        L.ssd_prefill_varlen.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 12 + [sz, vp]
         L.ssd_prefill_noalloc.restype = ctypes.c_int
         L.ssd_prefill_noalloc.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 10 + [vp]
         L.ssd_device_status.restype = ctypes.c_int
@@ -176,6 +180,68 @@ def prefill(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=None, init
     return y, final_state, conv_state
 
 
+def prefill_varlen_workspace_bytes(dims: SsdDims, dtype: torch.dtype) -> int:
+    code = SSD_F32 if dtype == torch.float32 else SSD_BF16
+    return int(lib().ssd_prefill_varlen_workspace_bytes(ctypes.byref(dims), code))
+
+
+def prefill_varlen(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, cu_seqlens, init_state=None,
+                   init_conv_state=None, chunk=128, workspace=None, y=None, final_state=None, conv_state=None,
+                   y_dtype=None):
+    """Packed variable-length prefill: sequence s is rows cu_seqlens[s] .. cu_seqlens[s+1]-1.
+
+    x, z [T, H*P]; dt [T, H]; B, C [T, G, N]; cu_seqlens: nseq+1 non-decreasing offsets from 0 to T,
+    an int64 tensor on the device (a list or CPU tensor is copied there first); init_state
+    [nseq, H, P, N] fp32 or None; init_conv_state [nseq, conv_dim, 3] or None.
+    Returns (y [T, H*P], final_state [nseq, H, P, N], conv_state [nseq, conv_dim, 3]).
+    Offsets that are out of order or out of range are reported by device_status().
+    """
+    dev = x.device
+    T, HP = x.shape
+    H = A.shape[0]
+    P = HP // H
+    G, N = B.shape[1], B.shape[2]
+    act = x.dtype
+    conv_dim = HP + 2 * G * N
+    if not torch.is_tensor(cu_seqlens) or cu_seqlens.device != dev:
+        cu_seqlens = torch.as_tensor(cu_seqlens, dtype=torch.int64).to(dev)
+    if cu_seqlens.dtype != torch.int64 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous 1-D int64 tensor")
+    nseq = cu_seqlens.numel() - 1
+    if nseq < 0:
+        raise ValueError("cu_seqlens needs at least one entry")
+    for name, t, shp in (("x", x, (T, HP)), ("z", z, (T, HP)), ("dt", dt, (T, H)), ("B", B, (T, G, N)),
+                         ("C", C, (T, G, N))):
+        _check(t, name, shp, act, dev)
+    if init_state is not None:
+        _check(init_state, "init_state", (nseq, H, P, N), torch.float32, dev)
+    if init_conv_state is not None:
+        _check(init_conv_state, "init_conv_state", (nseq, conv_dim, 3), act, dev)
+    params = _params(A, D, dt_bias, conv_w, conv_b, H, conv_dim, dev)
+    dims = make_dims(nseq, T, H, P, N, G, chunk)
+    ydt = y_dtype or (y.dtype if y is not None else act)
+    code = _dtype_code(x, ydt)
+    if y is None:
+        y = torch.empty((T, HP), dtype=ydt, device=dev)
+    if final_state is None:
+        final_state = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+    if conv_state is None:
+        conv_state = torch.empty((nseq, conv_dim, 3), dtype=act, device=dev)
+    _check(y, "y", (T, HP), ydt, dev)
+    _check(final_state, "final_state", (nseq, H, P, N), torch.float32, dev)
+    _check(conv_state, "conv_state", (nseq, conv_dim, 3), act, dev)
+    need = prefill_varlen_workspace_bytes(dims, act)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().ssd_prefill_varlen(ctypes.byref(dims), code, ctypes.byref(params), _ptr(cu_seqlens), _ptr(x), _ptr(dt),
+                                  _ptr(B), _ptr(C), _ptr(z), _ptr(init_state), _ptr(init_conv_state), _ptr(y),
+                                  _ptr(final_state), _ptr(conv_state), _ptr(workspace), ws_bytes, _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_prefill_varlen")
+    return y, final_state, conv_state
+
+
 def decode_step(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, conv_state, ssm_state, y=None, y_dtype=None):
     """One decode token for Bt sequences; conv_state and ssm_state update in place.
 
@@ -252,7 +318,8 @@ def prefill_noalloc(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=No
 
 
 def device_status(device="cuda"):
-    """Synchronise the current stream and raise if a kernel gave up on a bounded device-side wait."""
+    """Synchronise the current stream; raise if a kernel gave up on a bounded device-side wait
+    (SSD_ERR_TIMEOUT) or met invalid packed-sequence offsets (SSD_ERR_SHAPE)."""
     st = lib().ssd_device_status(_stream_ptr(torch.device(device)))
     if st != 0:
         raise SsdError(st, "ssd_device_status")

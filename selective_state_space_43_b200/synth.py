@@ -110,6 +110,34 @@ def make_prefill_inputs(dims: Dims, dtype=torch.bfloat16, seed: int = 43, init_s
     return out
 
 
+def varlen_lengths(nseq: int, lo: int, hi: int, seed: int) -> list:
+    """``nseq`` sequence lengths drawn log-uniformly from [lo, hi] (a continuous-batching mix)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    u = torch.rand(nseq, generator=g, dtype=torch.float64)
+    return [int(round(math.exp(math.log(lo) + float(v) * (math.log(hi) - math.log(lo))))) for v in u]
+
+
+def make_varlen_inputs(dims: Dims, lengths, dtype=torch.bfloat16, seed: int = 43, init_state: bool = False,
+                       init_conv_state: bool = False) -> tuple:
+    """Inputs of one packed variable-length prefill: the sequences of ``lengths`` back to back
+    (x/z [T, H*P], dt [T, H], B/C [T, G, N]; per-sequence initial states [nseq, ...]), drawn by
+    the same recipe as ``make_prefill_inputs``; ``dims.batch`` / ``dims.seqlen`` are ignored.
+    Returns (inputs, cu_seqlens as a list of nseq+1 offsets)."""
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    T, nseq = cu[-1], len(lengths)
+    packed = make_prefill_inputs(Dims(1, T, dims.nheads, dims.headdim, dims.d_state, dims.ngroups, dims.chunk),
+                                 dtype=dtype, seed=seed)
+    out = {k: (v[0] if k in ("x", "z", "dt", "B", "C") else v) for k, v in packed.items()}
+    g = torch.Generator(device="cpu").manual_seed(seed + 1000)
+    out["init_state"] = (torch.randn((nseq, dims.nheads, dims.headdim, dims.d_state), generator=g) * 0.1
+                         if init_state else None)
+    out["init_conv_state"] = (torch.randn((nseq, dims.conv_dim, 3), generator=g).to(dtype)
+                              if init_conv_state else None)
+    return out, cu
+
+
 def make_decode_inputs(dims: Dims, steps: int, dtype=torch.bfloat16, seed: int = 47,
                        random_D: bool = False) -> dict:
     """Initial states and ``steps`` rounds of fresh one-token inputs for decode."""

@@ -132,3 +132,32 @@ def test_decode_rejects_bad_arguments_before_launch(L):
 def test_timing_hook_requires_both_or_neither(L):
     assert L.ssd_set_timing_events(ctypes.c_void_p(0x10), None) == 1
     assert L.ssd_set_timing_events(None, None) == 0
+
+
+def _call_varlen(L, d, cu=0x98000, ptrs=None, ws=None, ws_bytes=0, params=None):
+    p = ptrs or dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, init=None, init_conv=None,
+                     y=0x60000, fs=0x70000, cs=0x80000)
+    prm = params if params is not None else _fake_params()
+    return L.ssd_prefill_varlen(ctypes.byref(d), 1, ctypes.byref(prm), cu, p["x"], p["dt"], p["B"], p["C"],
+                                p["z"], p["init"], p["init_conv"], p["y"], p["fs"], p["cs"], ws, ws_bytes, None)
+
+
+def test_varlen_rejects_bad_arguments_before_launch(L):
+    import torch
+    d = dims(batch=32, seqlen=30000)
+    assert _call_varlen(L, d, cu=None) == 1                       # offsets required
+    assert _call_varlen(L, d, cu=0x98004) == 4                    # int64 offsets: 8-byte aligned
+    assert _call_varlen(L, dims(batch=32, seqlen=30000, headdim=32)) == 2
+    assert _call_varlen(L, dims(batch=32, seqlen=1 << 31)) == 2   # rows beyond 32-bit tensor-map coordinates
+    base = dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, init=None, init_conv=None,
+                y=0x60000, fs=0x70000, cs=0x80000)
+    assert _call_varlen(L, d, ptrs={**base, "z": None}) == 1
+    assert _call_varlen(L, d, ptrs={**base, "y": base["z"]}) == 5
+    assert _call_varlen(L, d, ptrs={**base, "cs": 0x80008}) == 4
+    if ops.prefill_path(d, torch.bfloat16) == 1:
+        need = ops.prefill_varlen_workspace_bytes(d, torch.bfloat16)
+        assert need == 30000 * 2 * 8 * 128 * 2                    # post-conv B/C of every row
+        assert _call_varlen(L, d) == 7
+        assert _call_varlen(L, d, ws=0x90000, ws_bytes=need - 16) == 7
+    # fp32 activations take the CUDA-core path, which needs no workspace
+    assert ops.prefill_varlen_workspace_bytes(dims(d_state=32, chunk=64, nheads=4, ngroups=1), torch.float32) == 0
