@@ -39,12 +39,16 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from selective_state_space_43_b200.synth import (Dims, WORKLOADS, make_decode_inputs,  # noqa: E402
-                                                 make_prefill_inputs, seed_of)
+                                                 make_prefill_inputs, make_varlen_inputs, seed_of,
+                                                 varlen_lengths)
 
 METRIC = "SSD prefill tokens/s per layer (% bf16 TC peak); decode GB/s (% of HBM peak)"
 PREFILL_WORKLOAD = "nemotron_h_8b"
 DECODE_WORKLOAD = "decode_nemotron_h_8b"
 L2_FLUSH_BYTES = 256 << 20
+# continuous-batching mix for the packed variable-length prefill: this many sequences of the prefill
+# workload's layer, lengths log-uniform in [VARLEN_MIN, VARLEN_MAX], each with its own initial state
+VARLEN_NSEQ, VARLEN_MIN, VARLEN_MAX = 32, 64, 4096
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -57,6 +61,15 @@ def prefill_bytes(d: Dims, act_bytes: int, init_state: bool) -> int:
     out = tok * d.d_inner * act_bytes                                                 # y
     state = d.batch * d.nheads * d.headdim * d.d_state * 4 * (2 if init_state else 1)
     conv = d.batch * d.conv_dim * 3 * act_bytes
+    return inputs + out + state + conv
+
+
+def varlen_bytes(d: Dims, T: int, nseq: int, act_bytes: int) -> int:
+    """Algorithmic bytes of one packed prefill: T rows of inputs and y, per-sequence states in and out."""
+    inputs = T * (2 * d.d_inner + d.nheads + 2 * d.ngroups * d.d_state) * act_bytes
+    out = T * d.d_inner * act_bytes
+    state = nseq * d.nheads * d.headdim * d.d_state * 4 * 2
+    conv = nseq * d.conv_dim * 3 * act_bytes
     return inputs + out + state + conv
 
 
@@ -278,6 +291,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a CUDA graph replay")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed variable-length prefill line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -457,6 +471,64 @@ def main():
                                "algorithmic_bytes_per_launch": kern_b, "kernel_ms": dkms},
                   "l2": "state (1.07 GB) larger than L2; no flush"}
 
+    # ---- packed variable-length prefill (a continuous-batching mix of lengths) -----------------------
+    varlen = None
+    if not args.no_varlen:
+        wv = WORKLOADS[PREFILL_WORKLOAD]
+        dv = wv["dims"]
+        lengths = varlen_lengths(VARLEN_NSEQ, VARLEN_MIN, VARLEN_MAX, seed=seed_of(PREFILL_WORKLOAD) + 100)
+        vin, cu = make_varlen_inputs(dv, lengths, dtype=wv["dtype"], seed=seed_of(PREFILL_WORKLOAD) + 101,
+                                     init_state=True, init_conv_state=True)
+        gv = {k: (None if t is None else t.to(dev)) for k, t in vin.items()}
+        cu_dev = torch.tensor(cu, dtype=torch.int64, device=dev)
+        T = cu[-1]
+        vdims = ops.make_dims(len(lengths), T, dv.nheads, dv.headdim, dv.d_state, dv.ngroups, dv.chunk)
+        vws = torch.empty(max(ops.prefill_varlen_workspace_bytes(vdims, wv["dtype"]), 16), dtype=torch.uint8,
+                          device=dev)
+        vy = torch.empty_like(gv["x"])
+        vfs = torch.empty((len(lengths), dv.nheads, dv.headdim, dv.d_state), dtype=torch.float32, device=dev)
+        vcs = torch.empty((len(lengths), dv.conv_dim, 3), dtype=wv["dtype"], device=dev)
+
+        def vstep_eager():
+            ops.prefill_varlen(gv["x"], gv["dt"], gv["B"], gv["C"], gv["z"], gv["A"], gv["D"], gv["dt_bias"],
+                               gv["conv_w"], gv["conv_b"], cu_dev, gv["init_state"], gv["init_conv_state"],
+                               chunk=dv.chunk, workspace=vws, y=vy, final_state=vfs, conv_state=vcs)
+        for _ in range(args.warmup):
+            flush.zero_()
+            vstep_eager()
+        torch.cuda.synchronize(dev)
+        vstep = vstep_eager
+        if launch != "eager":
+            vgraph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(vgraph):
+                vstep_eager()
+            vstep = vgraph.replay
+        KV = max(3, min(K, 20))
+        vs = [torch.cuda.Event(enable_timing=True) for _ in range(KV)]
+        ve = [torch.cuda.Event(enable_timing=True) for _ in range(KV)]
+        barrier(world)
+        sampler.load(True)
+        for k in range(KV):
+            flush.zero_()
+            vs[k].record()
+            vstep()
+            ve[k].record()
+        torch.cuda.synchronize(dev)
+        sampler.load(False)
+        barrier(world)
+        ops.device_status(dev)
+        vms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(vs, ve)) / KV, world, dev)
+        vbytes = varlen_bytes(dv, T, len(lengths), 2 if wv["dtype"] == torch.bfloat16 else 4)
+        vgbs = vbytes / (vms * 1e-3) / 1e9
+        varlen = {"value": T * world / (vms * 1e-3), "unit": "tokens/s", "ms_per_step": vms, "steps": KV,
+                  "workload": f"{len(lengths)} packed sequences of the {PREFILL_WORKLOAD} layer, lengths "
+                              f"log-uniform in [{VARLEN_MIN}, {VARLEN_MAX}] ({T} tokens; min {min(lengths)}, "
+                              f"max {max(lengths)}), per-sequence initial states",
+                  "algorithmic_bytes_per_step": vbytes, "achieved_gbs": vgbs,
+                  "frac_hbm_peak": vgbs / peaks["hbm_gbs"], "launch": launch,
+                  "l2": "flushed between timed steps (256 MB write outside the step events)"}
+        del gv, vy, vws
+
     clocks = sampler.stop()
 
     # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------------------------------------
@@ -476,6 +548,7 @@ def main():
                        "l2": "flushed between timed steps (256 MB write outside the step events)",
                        "kernel_path": "tcgen05 tensor-core" if path == 1 else "CUDA-core", "launch": launch},
             "tensor": tc, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+            "varlen": varlen,
             "gpu_launches": K * (2 if path == 1 else 1), "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

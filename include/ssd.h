@@ -136,6 +136,29 @@ SSD_API ssd_status ssd_prefill(const ssd_dims* dims, ssd_dtype dtype, const ssd_
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Elements between consecutive tokens (rows) of each prefill input.  Lets
+ * x, z, dt, B and C be views into one wider per-token array -- the in_proj
+ * output [batch][seqlen][z | x | B | C | dt] of a Mamba-2 block -- read in
+ * place instead of being copied out first.  Batch b starts at row b*seqlen.
+ * Each stride must be at least its row width (H*P, H*P, H, G*N, G*N) and a
+ * multiple of 16 bytes (SSD_ERR_SHAPE / SSD_ERR_ALIGN otherwise).
+ */
+typedef struct {
+    int64_t x, z, dt, B, C;
+} ssd_row_strides;
+
+/*
+ * ssd_prefill on strided inputs (row_strides NULL = contiguous rows, the same
+ * as ssd_prefill).  y, the states and the workspace are laid out as for
+ * ssd_prefill; y must not overlap any input.
+ */
+SSD_API ssd_status ssd_prefill_strided(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
+                                       const ssd_row_strides* row_strides, const void* x, const void* dt,
+                                       const void* B, const void* C, const void* z, const float* init_state,
+                                       const void* init_conv_state, void* y, float* final_state, void* conv_state,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * One decode token for each of `batch` sequences (dims->seqlen is ignored).
  *   x, z        [batch][H*P]   dtype
  *   dt          [batch][H]     dtype

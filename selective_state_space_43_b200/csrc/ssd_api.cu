@@ -28,6 +28,17 @@ ssd_status check_dims(const ssd_dims* d, ssd_dtype dtype, bool prefill) {
     return SSD_OK;
 }
 
+// Each input row stride must cover its row and keep rows 16-byte aligned (tensor maps, vector loads).
+ssd_status check_strides(const ssd_row_strides& r, const ssd::Shape& s, ssd_dtype dtype) {
+    const int64_t esz = dtype == SSD_F32 ? 4 : 2;
+    const int64_t st[5] = {r.x, r.z, r.dt, r.B, r.C}, w[5] = {s.HP, s.HP, s.H, s.GN, s.GN};
+    for (int k = 0; k < 5; ++k) {
+        if (st[k] < w[k]) return SSD_ERR_SHAPE;
+        if ((st[k] * esz) % 16 != 0) return SSD_ERR_ALIGN;
+    }
+    return SSD_OK;
+}
+
 ssd_status check_params(const ssd_params* p) {
     if (!p || !p->A || !p->D || !p->dt_bias || !p->conv_w || !p->conv_b) return SSD_ERR_NULL;
     if (!aligned16(p->A) || !aligned16(p->D) || !aligned16(p->dt_bias) || !aligned16(p->conv_w) ||
@@ -68,10 +79,12 @@ size_t ssd_prefill_workspace_bytes(const ssd_dims* d, ssd_dtype dtype) {
     return ssd::prefill_tc_workspace_bytes(d->batch, d->seqlen, d->ngroups, d->d_state);
 }
 
-ssd_status ssd_prefill(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params, const void* x,
-                       const void* dt, const void* B, const void* C, const void* z, const float* init_state,
-                       const void* init_conv_state, void* y, float* final_state, void* conv_state,
-                       void* workspace, size_t workspace_bytes, void* stream) {
+// ssd_prefill with optional input row strides (nullptr: contiguous rows).
+static ssd_status prefill_impl(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params,
+                               const ssd_row_strides* rs, const void* x, const void* dt, const void* B,
+                               const void* C, const void* z, const float* init_state, const void* init_conv_state,
+                               void* y, float* final_state, void* conv_state, void* workspace,
+                               size_t workspace_bytes, void* stream) {
     ssd_status st = check_dims(d, dtype, true);
     if (st != SSD_OK) return st;
     if ((st = check_params(params)) != SSD_OK) return st;
@@ -84,12 +97,17 @@ ssd_status ssd_prefill(const ssd_dims* d, ssd_dtype dtype, const ssd_params* par
         if (!aligned16(p)) return SSD_ERR_ALIGN;
     if ((tokens && (y == x || y == z)) || (init_conv_state && init_conv_state == conv_state))
         return SSD_ERR_UNSUPPORTED;
+    const ssd::Shape s = ssd::make_shape(*d);
+    ssd_row_strides r{s.HP, s.HP, s.H, s.GN, s.GN};
+    if (rs) {
+        if ((st = check_strides(*rs, s, dtype)) != SSD_OK) return st;
+        r = *rs;
+    }
     const int path = ssd_prefill_path(d, dtype);
     const size_t need = path == 1 ? ssd::prefill_tc_workspace_bytes(d->batch, d->seqlen, d->ngroups, d->d_state) : 0;
     if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
     if (d->batch == 0) return SSD_OK;
 
-    const ssd::Shape s = ssd::make_shape(*d);
     ssd::PrefillArgs a;
     a.batch = s.batch;
     a.L = s.seqlen;
@@ -102,12 +120,30 @@ ssd_status ssd_prefill(const ssd_dims* d, ssd_dtype dtype, const ssd_params* par
     a.init_state = init_state; a.init_conv_state = init_conv_state;
     a.y = y; a.final_state = final_state; a.conv_state = conv_state;
     a.workspace = workspace;
+    a.rs_x = r.x; a.rs_z = r.z; a.rs_dt = r.dt; a.rs_B = r.B; a.rs_C = r.C;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
                                                                                         : ssd::ActKind::BF16_YF32);
     cudaError_t e = path == 1 ? ssd::launch_prefill_tc(a, kind, cs, g_hook)
                               : ssd::launch_prefill_simt(a, kind, cs, g_hook);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_prefill(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params, const void* x,
+                       const void* dt, const void* B, const void* C, const void* z, const float* init_state,
+                       const void* init_conv_state, void* y, float* final_state, void* conv_state,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    return prefill_impl(d, dtype, params, nullptr, x, dt, B, C, z, init_state, init_conv_state, y, final_state,
+                        conv_state, workspace, workspace_bytes, stream);
+}
+
+ssd_status ssd_prefill_strided(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params,
+                               const ssd_row_strides* row_strides, const void* x, const void* dt, const void* B,
+                               const void* C, const void* z, const float* init_state, const void* init_conv_state,
+                               void* y, float* final_state, void* conv_state, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    return prefill_impl(d, dtype, params, row_strides, x, dt, B, C, z, init_state, init_conv_state, y,
+                        final_state, conv_state, workspace, workspace_bytes, stream);
 }
 
 size_t ssd_prefill_varlen_workspace_bytes(const ssd_dims* d, ssd_dtype dtype) {
@@ -156,6 +192,7 @@ ssd_status ssd_prefill_varlen(const ssd_dims* d, ssd_dtype dtype, const ssd_para
     a.workspace = workspace;
     a.cu = cu_seqlens;
     a.err = err;
+    a.rs_x = s.HP; a.rs_z = s.HP; a.rs_dt = s.H; a.rs_B = s.GN; a.rs_C = s.GN;
     const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
                                                                                         : ssd::ActKind::BF16_YF32);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);

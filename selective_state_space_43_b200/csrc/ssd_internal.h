@@ -45,6 +45,9 @@ struct PrefillArgs {
     // sequence b is rows cu[b] .. cu[b+1]-1 of [L][...] activations.  nullptr: batch x L layout.
     const int64_t* cu = nullptr;
     int* err = nullptr;  // device error word (bit 1: a sequence's offsets were invalid)
+    // Elements between consecutive rows (tokens) of each input; a batch is L rows.  The contiguous
+    // widths HP, HP, H, GN, GN unless the inputs are views into a wider array (e.g. the in_proj output).
+    int64_t rs_x = 0, rs_z = 0, rs_dt = 0, rs_B = 0, rs_C = 0;
 };
 
 // Device error word bits, read back by ssd_device_status.

@@ -45,9 +45,9 @@ __device__ __forceinline__ float raw_at(const PrefillArgs& a, int64_t b, int64_t
         return to_f32(static_cast<const T*>(a.init_conv_state)[((size_t)b * a.conv_dim + c) * 3 + (s + 3)]);
     }
     const size_t row = (size_t)(row0 + s);
-    if (c < a.HP) return to_f32(static_cast<const T*>(a.x)[row * a.HP + c]);
-    if (c < a.HP + a.GN) return to_f32(static_cast<const T*>(a.B)[row * a.GN + (c - a.HP)]);
-    return to_f32(static_cast<const T*>(a.C)[row * a.GN + (c - a.HP - a.GN)]);
+    if (c < a.HP) return to_f32(static_cast<const T*>(a.x)[row * a.rs_x + c]);
+    if (c < a.HP + a.GN) return to_f32(static_cast<const T*>(a.B)[row * a.rs_B + (c - a.HP)]);
+    return to_f32(static_cast<const T*>(a.C)[row * a.rs_C + (c - a.HP - a.GN)]);
 }
 
 template <typename T, typename TY, int N, int Q>
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
                 const int t = lane * PER + k;
                 float dA = 0.f;
                 if (t < Qc) {
-                    const float dtv = softplus_f(to_f32(static_cast<const T*>(a.dt)[((size_t)span.row0 + t0 + t) * a.H + h]) + dtb);
+                    const float dtv = softplus_f(to_f32(static_cast<const T*>(a.dt)[((size_t)span.row0 + t0 + t) * a.rs_dt + h]) + dtb);
                     sDt[t] = dtv;
                     dA = dtv * A;
                 } else {
@@ -152,8 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
 #pragma unroll 8
                 for (int n = 0; n < N; ++n) off += sC[t * N + n] * sS[p * NB + n];
                 const float yv = acc + dec * off + Dh * sX[t * kP + p];
-                const size_t o = ((size_t)span.row0 + t0 + t) * a.HP + cx + p;
-                const float zv = to_f32(static_cast<const T*>(a.z)[o]);
+                const size_t row = (size_t)span.row0 + t0 + t;
+                const size_t o = row * a.HP + cx + p;
+                const float zv = to_f32(static_cast<const T*>(a.z)[row * a.rs_z + cx + p]);
                 static_cast<TY*>(a.y)[o] = from_f32<TY>(yv * silu_f(zv));
             }
             __syncwarp();

@@ -713,9 +713,9 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
         __nv_bfloat16 v;
         if (t >= 0) {
             const size_t row = (size_t)(sp.row0 + t);
-            if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[row * a.HP + c];
-            else if (c < a.HP + a.GN) v = static_cast<const __nv_bfloat16*>(a.B)[row * a.GN + (c - a.HP)];
-            else v = static_cast<const __nv_bfloat16*>(a.C)[row * a.GN + (c - a.HP - a.GN)];
+            if (c < a.HP) v = static_cast<const __nv_bfloat16*>(a.x)[row * a.rs_x + c];
+            else if (c < a.HP + a.GN) v = static_cast<const __nv_bfloat16*>(a.B)[row * a.rs_B + (c - a.HP)];
+            else v = static_cast<const __nv_bfloat16*>(a.C)[row * a.rs_C + (c - a.HP - a.GN)];
         } else {
             v = conv_history(a, b, c, t);
         }
@@ -730,7 +730,8 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
     const int sel = pair >= half_gn;                // 0 = B, 1 = C
     const int cp = pair - sel * half_gn;            // pair index within the array
     const int cglob = a.HP + sel * a.GN + 2 * cp;   // conv channel of the pair's first element
-    const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B) + (size_t)b * a.L * half_gn + cp;
+    const int64_t rs = (sel ? a.rs_C : a.rs_B) / 2;  // row stride in channel pairs
+    const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B) + (size_t)b * a.L * rs + cp;
     uint32_t* dst = static_cast<uint32_t*>(a.workspace) + ((size_t)b * a.L * 2 + sel) * half_gn + cp;
     const float4 w0 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cglob * 4);
     const float4 w1 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(cglob + 1) * 4);
@@ -740,7 +741,7 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
 #pragma unroll
     for (int k = 0; k < kProTok + 3; ++k) {
         const int64_t t = t0 - 3 + k;
-        raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * half_gn] : 0u;
+        raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * rs] : 0u;
     }
 #pragma unroll
     for (int k = 0; k < kProTok + 3; ++k) {
@@ -814,12 +815,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D bf16 map over [batch][L][width] with a [1][128][64] box and 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int64_t width, int64_t L, int64_t batch) {
+// 3-D bf16 map over [batch][L][width] (rows row_stride elements apart) with a [1][128][64] box and
+// 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t width, int64_t row_stride, int64_t L, int64_t batch) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)L, (cuuint64_t)batch};
-    const cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)(width * L * 2)};
+    const cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)(row_stride * L * 2)};
     const cuuint32_t box[3] = {64, 128, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -828,11 +830,11 @@ bool make_map(CUtensorMap* m, const void* base, int64_t width, int64_t L, int64_
 }
 
 // 3-D bf16 map over dt [batch][L][H] with a [1][128][8] box (8 heads x 128 tokens, no swizzle); needs H % 8 == 0.
-bool make_dt_map(CUtensorMap* m, const void* base, int64_t H, int64_t L, int64_t batch) {
+bool make_dt_map(CUtensorMap* m, const void* base, int64_t H, int64_t row_stride, int64_t L, int64_t batch) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || H % 8 != 0) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)batch};
-    const cuuint64_t strides[2] = {(cuuint64_t)H * 2, (cuuint64_t)(H * L * 2)};
+    const cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)(row_stride * L * 2)};
     const cuuint32_t box[3] = {8, 128, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -855,10 +857,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     TcParams prm;
     prm.a = a;
     const int64_t mbatch = a.cu ? 1 : a.batch;  // a packed batch is one [L] row of the maps
-    if (!make_map(&prm.tm_x, a.x, a.HP, a.L, mbatch) || !make_map(&prm.tm_z, a.z, a.HP, a.L, mbatch) ||
-        (kind == ActKind::BF16 && !make_map(&prm.tm_y, a.y, a.HP, a.L, mbatch)) ||
-        !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, a.L, mbatch) ||
-        !make_dt_map(&prm.tm_dt, a.dt, a.H, a.L, mbatch))
+    if (!make_map(&prm.tm_x, a.x, a.HP, a.rs_x, a.L, mbatch) || !make_map(&prm.tm_z, a.z, a.HP, a.rs_z, a.L, mbatch) ||
+        (kind == ActKind::BF16 && !make_map(&prm.tm_y, a.y, a.HP, a.HP, a.L, mbatch)) ||
+        !make_map(&prm.tm_bc, a.workspace, 2 * a.GN, 2 * a.GN, a.L, mbatch) ||
+        !make_dt_map(&prm.tm_dt, a.dt, a.H, a.rs_dt, a.L, mbatch))
         return cudaErrorInvalidValue;
     const int ntok = (int)((a.L + kProTok - 1) / kProTok);
     const int64_t tail = a.batch * (int64_t)a.conv_dim * 3;

@@ -32,6 +32,11 @@ class SsdParams(ctypes.Structure):
                 ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p)]
 
 
+class SsdRowStrides(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_int64), ("z", ctypes.c_int64), ("dt", ctypes.c_int64), ("B", ctypes.c_int64),
+                ("C", ctypes.c_int64)]
+
+
 class SsdError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {STATUS.get(status, status)} ({lib().ssd_status_string(status).decode()})")
@@ -67,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_varlen_workspace_bytes.argtypes = [dimp, ctypes.c_int]
         L.ssd_prefill_varlen.restype = ctypes.c_int
         L.ssd_prefill_varlen.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 12 + [sz, vp]
+        L.ssd_prefill_strided.restype = ctypes.c_int
+        L.ssd_prefill_strided.argtypes = [dimp, ctypes.c_int, parp, ctypes.POINTER(SsdRowStrides)] + [vp] * 11 + [sz, vp]
         L.ssd_prefill_noalloc.restype = ctypes.c_int
         L.ssd_prefill_noalloc.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 10 + [vp]
         L.ssd_device_status.restype = ctypes.c_int
@@ -105,6 +112,35 @@ def _check(t, name, shape, dtype, device):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _row_stride(t, name, shape, dtype, device) -> int:
+    """Elements between consecutive tokens of a [Bt, L, ...] input.  Contiguous tensors, and views
+    whose per-token part is contiguous with batches L rows apart (e.g. slices of a block's in_proj
+    output), are accepted; the library reads the views in place."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    width = 1
+    for n in shape[2:]:
+        width *= n
+    if t.is_contiguous():
+        return width
+    expect = 1
+    for dim in range(t.dim() - 1, 1, -1):
+        if t.shape[dim] > 1 and t.stride(dim) != expect:
+            raise ValueError(f"{name}: the elements of one token must be contiguous")
+        expect *= t.shape[dim]
+    Bt, L = shape[0], shape[1]
+    rs = t.stride(1) if L > 1 else (t.stride(0) if Bt > 1 else width)
+    if Bt > 1 and L > 1 and t.stride(0) != L * rs:
+        raise ValueError(f"{name}: consecutive sequences must be seqlen rows apart")
+    return rs
+
+
 def _stream_ptr(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
@@ -134,7 +170,8 @@ def prefill(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=None, init
             workspace=None, y=None, final_state=None, conv_state=None, y_dtype=None):
     """Chunked SSD prefill on the GPU.
 
-    x, z [Bt, L, H*P]; dt [Bt, L, H]; B, C [Bt, L, G, N] (bf16 or fp32, one dtype);
+    x, z [Bt, L, H*P]; dt [Bt, L, H]; B, C [Bt, L, G, N] (bf16 or fp32, one dtype), contiguous or
+    views with strided rows (e.g. slices of the in_proj output [Bt, L, z | x | B | C | dt]);
     A, D, dt_bias [H], conv_w [conv_dim, 4], conv_b [conv_dim] fp32;
     init_state [Bt, H, P, N] fp32 or None; init_conv_state [Bt, conv_dim, 3] or None.
     y_dtype: the dtype of y (default: the activation dtype; float32 with bf16
@@ -148,9 +185,10 @@ def prefill(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=None, init
     G, N = B.shape[2], B.shape[3]
     act = x.dtype
     conv_dim = HP + 2 * G * N
-    for name, t, shp in (("x", x, (Bt, L, HP)), ("z", z, (Bt, L, HP)), ("dt", dt, (Bt, L, H)),
-                         ("B", B, (Bt, L, G, N)), ("C", C, (Bt, L, G, N))):
-        _check(t, name, shp, act, dev)
+    rs = SsdRowStrides(*[_row_stride(t, name, shp, act, dev) for name, t, shp in (
+        ("x", x, (Bt, L, HP)), ("z", z, (Bt, L, HP)), ("dt", dt, (Bt, L, H)), ("B", B, (Bt, L, G, N)),
+        ("C", C, (Bt, L, G, N)))])
+    strided = (rs.x, rs.z, rs.dt, rs.B, rs.C) != (HP, HP, H, G * N, G * N)
     if init_state is not None:
         _check(init_state, "init_state", (Bt, H, P, N), torch.float32, dev)
     if init_conv_state is not None:
@@ -172,11 +210,14 @@ def prefill(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=None, init
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().ssd_prefill(ctypes.byref(dims), code, ctypes.byref(params), _ptr(x), _ptr(dt), _ptr(B),
-                           _ptr(C), _ptr(z), _ptr(init_state), _ptr(init_conv_state), _ptr(y), _ptr(final_state),
-                           _ptr(conv_state), _ptr(workspace), ws_bytes, _stream_ptr(dev))
+    args = (_ptr(x), _ptr(dt), _ptr(B), _ptr(C), _ptr(z), _ptr(init_state), _ptr(init_conv_state), _ptr(y),
+            _ptr(final_state), _ptr(conv_state), _ptr(workspace), ws_bytes, _stream_ptr(dev))
+    if strided:
+        st = lib().ssd_prefill_strided(ctypes.byref(dims), code, ctypes.byref(params), ctypes.byref(rs), *args)
+    else:
+        st = lib().ssd_prefill(ctypes.byref(dims), code, ctypes.byref(params), *args)
     if st != 0:
-        raise SsdError(st, "ssd_prefill")
+        raise SsdError(st, "ssd_prefill_strided" if strided else "ssd_prefill")
     return y, final_state, conv_state
 
 

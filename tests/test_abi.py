@@ -161,3 +161,19 @@ def test_varlen_rejects_bad_arguments_before_launch(L):
         assert _call_varlen(L, d, ws=0x90000, ws_bytes=need - 16) == 7
     # fp32 activations take the CUDA-core path, which needs no workspace
     assert ops.prefill_varlen_workspace_bytes(dims(d_state=32, chunk=64, nheads=4, ngroups=1), torch.float32) == 0
+
+
+def test_strided_prefill_checks_the_row_strides(L):
+    d = dims(batch=2, seqlen=300, nheads=16, ngroups=2)
+    base = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, None, 0x60000, 0x70000, 0x80000]
+
+    def call(rs):
+        return L.ssd_prefill_strided(ctypes.byref(d), 1, ctypes.byref(_fake_params()),
+                                     None if rs is None else ctypes.byref(ops.SsdRowStrides(*rs)), *base, None, 0,
+                                     None)
+    wide = 2 * 1024 + 2 * 256 + 16                      # z | x | B | C | dt per token
+    assert call((wide, wide, wide, wide, wide)) == 7    # valid strides: fails only for want of a workspace
+    assert call((1000, wide, wide, wide, wide)) == 2    # x rows narrower than H*P
+    assert call((wide, wide, 8, wide, wide)) == 2       # dt rows narrower than H
+    assert call((wide + 4, wide, wide, wide, wide)) == 4  # not a multiple of 16 bytes
+    assert call(None) == 7                              # NULL: contiguous rows, as ssd_prefill

@@ -170,3 +170,25 @@ def test_layer_shapes_take_the_tensor_core_path():
         d = WORKLOADS[name]["dims"]
         dims = ops.make_dims(d.batch, d.seqlen, d.nheads, d.headdim, d.d_state, d.ngroups, d.chunk)
         assert ops.prefill_path(dims, torch.bfloat16) == 1, name
+
+
+@pytest.mark.parametrize("d,dt", [(Dims(2, 300, 16, 64, 128, 2, 128), torch.bfloat16),
+                                  (Dims(2, 140, 4, 64, 32, 1, 64), torch.float32)])
+def test_prefill_reads_views_of_the_in_proj_output(d, dt):
+    # x, z, dt, B, C as slices of one [Bt, L, z | x | B | C | dt] array (a Mamba-2 block's in_proj
+    # output): the strided call must give exactly the contiguous call's results
+    inp = make_prefill_inputs(d, dtype=dt, seed=111, init_state=True, init_conv_state=True)
+    dev = dev_inputs(inp)
+    HP, GN, H = d.nheads * d.headdim, d.ngroups * d.d_state, d.nheads
+    zxbcdt = torch.empty((d.batch, d.seqlen, 2 * HP + 2 * GN + H), dtype=dt, device="cuda")
+    views = {"z": zxbcdt[..., :HP], "x": zxbcdt[..., HP:2 * HP],
+             "B": zxbcdt[..., 2 * HP:2 * HP + GN].unflatten(-1, (d.ngroups, d.d_state)),
+             "C": zxbcdt[..., 2 * HP + GN:2 * HP + 2 * GN].unflatten(-1, (d.ngroups, d.d_state)),
+             "dt": zxbcdt[..., 2 * HP + 2 * GN:]}
+    for k, v in views.items():
+        v.copy_(dev[k])
+        assert not v.is_contiguous()
+    ys, fss, css = gpu_prefill({**dev, **views}, d.chunk)
+    yc, fsc, csc = gpu_prefill(dev, d.chunk)
+    ops.device_status()
+    assert torch.equal(ys, yc) and torch.equal(fss, fsc) and torch.equal(css, csc)
