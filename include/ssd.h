@@ -230,6 +230,36 @@ SSD_API ssd_status ssd_prefill_varlen(const ssd_dims* dims, ssd_dtype dtype, con
                                       void* conv_state, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Context parallelism: one sequence split into W consecutive segments, one per
+ * rank.  The state after a segment is affine in the state before it,
+ * S_out = exp(A * sum_t dt_t) * S_in + S_loc, with S_loc the state the segment
+ * reaches from zero, so one exchange suffices: each rank scans its segment
+ * from zero (ssd_prefill, final_state = S_loc) with the 3 pre-conv tokens
+ * before the segment as its init_conv_state (ssd_conv_window of the previous
+ * rank's segment), sums its dt (ssd_dt_sum), all ranks gather (S_loc, sums),
+ * each folds the segments before its own into its initial state
+ * (ssd_cp_combine) and scans its segment again from that state.  Segments
+ * must be at least 3 tokens long.  The library provides the three steps; the
+ * gather is the caller's (see selective_state_space_43_b200/cp.py).
+ *
+ * ssd_conv_window: conv_state [batch][conv_dim][3] (out) = pre-conv x|B|C of
+ *   tokens seqlen-3 .. seqlen-1 (from init_conv_state, or zero, before token 0);
+ *   the conv_state output of ssd_prefill, without the scan.
+ * ssd_dt_sum: dt_sum [batch][H] fp32 (out) = sum over the seqlen tokens of
+ *   softplus(dt_raw + dt_bias[h]); deterministic.
+ * ssd_cp_combine: state_in [batch][H][P][N] fp32 (out) = init_state (or zero)
+ *   folded with segments 0 .. upto-1: S <- exp(A_h dt_sums[q]) S + seg_states[q],
+ *   with dt_sums [nseg][batch][H] and seg_states [nseg][batch][H][P][N].
+ *   dims supplies batch, nheads, headdim and d_state; seqlen is ignored.
+ */
+SSD_API ssd_status ssd_conv_window(const ssd_dims* dims, ssd_dtype dtype, const void* x, const void* B,
+                                   const void* C, const void* init_conv_state, void* conv_state, void* stream);
+SSD_API ssd_status ssd_dt_sum(const ssd_dims* dims, ssd_dtype dtype, const float* dt_bias, const void* dt,
+                              float* dt_sum, void* stream);
+SSD_API ssd_status ssd_cp_combine(const ssd_dims* dims, int nseg, int upto, const float* A, const float* dt_sums,
+                                  const float* seg_states, const float* init_state, float* state_in, void* stream);
+
+/*
  * Synchronises `stream` and reports whether a kernel launched by this library
  * gave up on a bounded device-side wait since the last call (SSD_ERR_TIMEOUT;
  * its outputs are then incomplete), or whether the stream holds a CUDA error

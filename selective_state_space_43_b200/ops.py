@@ -74,6 +74,12 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_varlen.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 12 + [sz, vp]
         L.ssd_prefill_strided.restype = ctypes.c_int
         L.ssd_prefill_strided.argtypes = [dimp, ctypes.c_int, parp, ctypes.POINTER(SsdRowStrides)] + [vp] * 11 + [sz, vp]
+        L.ssd_conv_window.restype = ctypes.c_int
+        L.ssd_conv_window.argtypes = [dimp, ctypes.c_int] + [vp] * 5 + [vp]
+        L.ssd_dt_sum.restype = ctypes.c_int
+        L.ssd_dt_sum.argtypes = [dimp, ctypes.c_int, vp, vp, vp, vp]
+        L.ssd_cp_combine.restype = ctypes.c_int
+        L.ssd_cp_combine.argtypes = [dimp, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, vp]
         L.ssd_prefill_noalloc.restype = ctypes.c_int
         L.ssd_prefill_noalloc.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 10 + [vp]
         L.ssd_device_status.restype = ctypes.c_int
@@ -281,6 +287,61 @@ def prefill_varlen(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, cu_seqlens, in
     if st != 0:
         raise SsdError(st, "ssd_prefill_varlen")
     return y, final_state, conv_state
+
+
+def conv_window(x, B, C, init_conv_state=None, out=None):
+    """Pre-conv x|B|C of the last 3 tokens of each sequence, [Bt, conv_dim, 3] (history before token 0):
+    the conv_state that ssd_prefill would return, without the scan."""
+    dev = x.device
+    Bt, L, HP = x.shape
+    G, N = B.shape[2], B.shape[3]
+    conv_dim = HP + 2 * G * N
+    for name, t, shp in (("x", x, (Bt, L, HP)), ("B", B, (Bt, L, G, N)), ("C", C, (Bt, L, G, N))):
+        _check(t, name, shp, x.dtype, dev)
+    if init_conv_state is not None:
+        _check(init_conv_state, "init_conv_state", (Bt, conv_dim, 3), x.dtype, dev)
+    if out is None:
+        out = torch.empty((Bt, conv_dim, 3), dtype=x.dtype, device=dev)
+    dims = make_dims(Bt, L, HP // 64, 64, N, G)
+    st = lib().ssd_conv_window(ctypes.byref(dims), SSD_F32 if x.dtype == torch.float32 else SSD_BF16, _ptr(x),
+                               _ptr(B), _ptr(C), _ptr(init_conv_state), _ptr(out), _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_conv_window")
+    return out
+
+
+def dt_sum(dt, dt_bias, ngroups=1, d_state=128):
+    """sum_t softplus(dt_raw + dt_bias[h]) per sequence and head, [Bt, H] fp32."""
+    dev = dt.device
+    Bt, L, H = dt.shape
+    _check(dt, "dt", (Bt, L, H), dt.dtype, dev)
+    _check(dt_bias, "dt_bias", (H,), torch.float32, dev)
+    out = torch.empty((Bt, H), dtype=torch.float32, device=dev)
+    dims = make_dims(Bt, L, H, 64, d_state, ngroups)
+    st = lib().ssd_dt_sum(ctypes.byref(dims), SSD_F32 if dt.dtype == torch.float32 else SSD_BF16, _ptr(dt_bias),
+                          _ptr(dt), _ptr(out), _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_dt_sum")
+    return out
+
+
+def cp_combine(seg_states, dt_sums, A, upto, init_state=None):
+    """Initial state of segment ``upto``: init_state (or zero) folded with segments 0 .. upto-1,
+    S <- exp(A_h dt_sums[q]) S + seg_states[q].  seg_states [W, Bt, H, P, N], dt_sums [W, Bt, H]."""
+    dev = seg_states.device
+    W, Bt, H, P, N = seg_states.shape
+    _check(seg_states, "seg_states", (W, Bt, H, P, N), torch.float32, dev)
+    _check(dt_sums, "dt_sums", (W, Bt, H), torch.float32, dev)
+    _check(A, "A", (H,), torch.float32, dev)
+    if init_state is not None:
+        _check(init_state, "init_state", (Bt, H, P, N), torch.float32, dev)
+    out = torch.empty((Bt, H, P, N), dtype=torch.float32, device=dev)
+    dims = make_dims(Bt, 0, H, P, N, 1)
+    st = lib().ssd_cp_combine(ctypes.byref(dims), W, int(upto), _ptr(A), _ptr(dt_sums), _ptr(seg_states),
+                              _ptr(init_state), _ptr(out), _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_cp_combine")
+    return out
 
 
 def decode_step(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, conv_state, ssm_state, y=None, y_dtype=None):

@@ -177,3 +177,17 @@ def test_strided_prefill_checks_the_row_strides(L):
     assert call((wide, wide, 8, wide, wide)) == 2       # dt rows narrower than H
     assert call((wide + 4, wide, wide, wide, wide)) == 4  # not a multiple of 16 bytes
     assert call(None) == 7                              # NULL: contiguous rows, as ssd_prefill
+
+
+def test_context_parallel_helpers_check_arguments(L):
+    d = dims(batch=2, seqlen=300, nheads=16, ngroups=2)
+    assert L.ssd_conv_window(None, 1, 0x10000, 0x30000, 0x40000, None, 0x80000, None) == 1
+    assert L.ssd_conv_window(ctypes.byref(d), 1, None, 0x30000, 0x40000, None, 0x80000, None) == 1
+    assert L.ssd_conv_window(ctypes.byref(d), 1, 0x10000, 0x30008, 0x40000, None, 0x80000, None) == 4
+    assert L.ssd_conv_window(ctypes.byref(d), 1, 0x10000, 0x30000, 0x40000, 0x80000, 0x80000, None) == 5
+    assert L.ssd_dt_sum(ctypes.byref(d), 1, None, 0x20000, 0x90000, None) == 1
+    assert L.ssd_dt_sum(ctypes.byref(dims(headdim=32)), 1, 0x1000, 0x20000, 0x90000, None) == 2
+    assert L.ssd_cp_combine(ctypes.byref(d), 4, 5, 0x1000, 0x2000, 0x3000, None, 0x4000, None) == 2  # upto > nseg
+    assert L.ssd_cp_combine(ctypes.byref(d), 0, 0, 0x1000, 0x2000, 0x3000, None, 0x4000, None) == 2
+    assert L.ssd_cp_combine(ctypes.byref(d), 4, 2, 0x1000, None, 0x3000, None, 0x4000, None) == 1
+    assert L.ssd_cp_combine(ctypes.byref(d), 4, 2, 0x1000, 0x2000, 0x3000, 0x4000, 0x4000, None) == 5
