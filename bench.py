@@ -292,6 +292,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a CUDA graph replay")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed variable-length prefill line")
+    ap.add_argument("--no-norm", action="store_true", help="skip the gated RMSNorm line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -395,6 +396,40 @@ def main():
     tc = {"algorithmic_tflops": tflops, "frac_bf16_peak": tflops / peaks["bf16_tflops"],
           "frac_bf16_sustained": tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
           "algorithmic_flops_per_step": pflops, "peak_source": peak_src}
+
+    # ---- gated RMSNorm of the prefill output (grouped, ngroups groups), HBM-bound ---------------------------
+    norm = None
+    if not args.no_norm and path == 1:
+        wn = torch.rand(d.d_inner, generator=torch.Generator().manual_seed(11)).add_(0.5).to(dev)
+        yn = torch.empty_like(y)
+
+        def norm_once():
+            ops.gated_rmsnorm(y, wn, d.ngroups, out=yn)
+        for _ in range(args.warmup):
+            norm_once()
+        torch.cuda.synchronize(dev)
+        nstep = norm_once
+        if launch != "eager":
+            ngraph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ngraph):
+                norm_once()
+            nstep = ngraph.replay
+        ns = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ne = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for k in range(K):
+            flush.zero_()
+            ns[k].record()
+            nstep()
+            ne[k].record()
+        torch.cuda.synchronize(dev)
+        nms = sum(a.elapsed_time(b) for a, b in zip(ns, ne)) / K
+        nbytes = 2 * y.numel() * y.element_size() + d.d_inner * 4
+        ngbs = nbytes / (nms * 1e-3) / 1e9
+        norm = {"kernel": "group_rmsnorm_kernel", "us_per_call": nms * 1e3, "groups": d.ngroups,
+                "algorithmic_bytes": nbytes,
+                "roofline": {"bound": "hbm", "achieved": ngbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": ngbs / peaks["hbm_gbs"], "traffic": kernel_traffic("group_rmsnorm_kernel")}}
+        del yn
 
     # ---- e2e through the public API from pinned host memory ------------------------------------------------
     e2e = None
@@ -548,7 +583,7 @@ def main():
                        "l2": "flushed between timed steps (256 MB write outside the step events)",
                        "kernel_path": "tcgen05 tensor-core" if path == 1 else "CUDA-core", "launch": launch},
             "tensor": tc, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
-            "varlen": varlen,
+            "varlen": varlen, "gated_rmsnorm": norm,
             "gpu_launches": K * (2 if path == 1 else 1), "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -260,6 +260,19 @@ SSD_API ssd_status ssd_cp_combine(const ssd_dims* dims, int nseg, int upto, cons
                                   const float* seg_states, const float* init_state, float* state_in, void* stream);
 
 /*
+ * RMSNorm of the gated output before a block's output projection (the
+ * "Mamba-3" page, 정규화 section: Mamba-2's norm, kept in hybrids).  Applied
+ * after the gate, over norm_groups contiguous channel groups of each row
+ * (norm_groups = ngroups for Mamba-2's grouped norm, 1 for one norm over all
+ * channels):  out[r][c] = y[r][c] * rsqrt(mean over c's group of y^2 + eps) * weight[c].
+ *   y, out      [rows][channels] in dtype (SSD_BF16 or SSD_F32); out may equal y
+ *   weight      [channels] fp32
+ * channels / norm_groups must be a multiple of 8; pointers 16-byte aligned.
+ */
+SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t norm_groups, float eps,
+                                     ssd_dtype dtype, const void* y, const float* weight, void* out, void* stream);
+
+/*
  * Synchronises `stream` and reports whether a kernel launched by this library
  * gave up on a bounded device-side wait since the last call (SSD_ERR_TIMEOUT;
  * its outputs are then incomplete), or whether the stream holds a CUDA error

@@ -179,3 +179,18 @@ def decode_step(step: dict, params: dict, conv_state, ssm_state, unit_mask=None)
     _load().oracle_decode_step(ctypes.byref(d), *[_ptr(a) for a in arrs],
                                None if mask is None else mask.ctypes.data_as(ctypes.c_void_p), _ptr(y))
     return y
+
+
+def gated_rmsnorm(y, weight, ngroups: int, eps: float = 1e-5):
+    """RMSNorm of the gated output, as the norm that Mamba-2 blocks apply before their output
+    projection (the "Mamba-3: 추론을 우선한 상태 공간 모델" page, 정규화 section, keeps it for hybrid
+    models and names its variants: before or after the gate, grouped or over all channels).  Reading
+    taken: after the SiLU(z) gate, over ``ngroups`` contiguous channel groups (1 = all channels):
+    out = v / sqrt(mean over the group of v^2 + eps) * weight, v = the gated y of ``prefill``.
+    y [..., H*P], weight [H*P].  Plain fp64 definition."""
+    v = _f64(y)
+    w = _f64(weight)
+    shp = v.shape
+    g = v.reshape(shp[:-1] + (ngroups, shp[-1] // ngroups))
+    ms = np.mean(g * g, axis=-1, keepdims=True)
+    return (g / np.sqrt(ms + eps)).reshape(shp) * w

@@ -743,16 +743,8 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
         const int64_t t = t0 - 3 + k;
         raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * rs] : 0u;
     }
-#pragma unroll
-    for (int k = 0; k < kProTok + 3; ++k) {
-        const int64_t t = t0 - 3 + k;
-        if (!kVarlen && t < 0)
-            v[k] = make_float2(__bfloat162float(conv_history(a, b, cglob, t)),
-                               __bfloat162float(conv_history(a, b, cglob + 1, t)));
-        else
-            v[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
-    }
-    // packed batch: the sequence of row t0 and where the next one starts
+    // packed batch: the sequence of row t0 and where the next one starts (searched while the loads above
+    // are in flight)
     int64_t seq = 0, start = 0, next = a.L;
     if constexpr (kVarlen) {
         int64_t lo = 0, hi = a.batch;  // largest seq with cu[seq] <= t0 (empty sequences skipped)
@@ -764,6 +756,15 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
         seq = lo;
         start = a.cu[seq];
         next = a.cu[seq + 1];
+    }
+#pragma unroll
+    for (int k = 0; k < kProTok + 3; ++k) {
+        const int64_t t = t0 - 3 + k;
+        if (!kVarlen && t < 0)
+            v[k] = make_float2(__bfloat162float(conv_history(a, b, cglob, t)),
+                               __bfloat162float(conv_history(a, b, cglob + 1, t)));
+        else
+            v[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
     }
 #pragma unroll
     for (int k = 0; k < kProTok; ++k) {

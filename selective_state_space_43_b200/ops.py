@@ -80,6 +80,9 @@ def lib() -> ctypes.CDLL:
         L.ssd_dt_sum.argtypes = [dimp, ctypes.c_int, vp, vp, vp, vp]
         L.ssd_cp_combine.restype = ctypes.c_int
         L.ssd_cp_combine.argtypes = [dimp, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, vp]
+        L.ssd_gated_rmsnorm.restype = ctypes.c_int
+        L.ssd_gated_rmsnorm.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_float, ctypes.c_int,
+                                        vp, vp, vp, vp]
         L.ssd_prefill_noalloc.restype = ctypes.c_int
         L.ssd_prefill_noalloc.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 10 + [vp]
         L.ssd_device_status.restype = ctypes.c_int
@@ -341,6 +344,25 @@ def cp_combine(seg_states, dt_sums, A, upto, init_state=None):
                               _ptr(init_state), _ptr(out), _stream_ptr(dev))
     if st != 0:
         raise SsdError(st, "ssd_cp_combine")
+    return out
+
+
+def gated_rmsnorm(y, weight, norm_groups, eps=1e-5, out=None):
+    """RMSNorm over ``norm_groups`` contiguous channel groups of the gated output y [..., channels]
+    (bf16 or fp32), times the per-channel fp32 ``weight``; ``out`` may be ``y`` (in place)."""
+    dev = y.device
+    channels = y.shape[-1]
+    if not y.is_contiguous():
+        raise ValueError("y must be contiguous")
+    _check(weight, "weight", (channels,), torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(y)
+    _check(out, "out", tuple(y.shape), y.dtype, dev)
+    code = SSD_F32 if y.dtype == torch.float32 else SSD_BF16
+    st = lib().ssd_gated_rmsnorm(y.numel() // channels, channels, int(norm_groups), float(eps), code, _ptr(y),
+                                 _ptr(weight), _ptr(out), _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_gated_rmsnorm")
     return out
 
 

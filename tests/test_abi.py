@@ -191,3 +191,14 @@ def test_context_parallel_helpers_check_arguments(L):
     assert L.ssd_cp_combine(ctypes.byref(d), 0, 0, 0x1000, 0x2000, 0x3000, None, 0x4000, None) == 2
     assert L.ssd_cp_combine(ctypes.byref(d), 4, 2, 0x1000, None, 0x3000, None, 0x4000, None) == 1
     assert L.ssd_cp_combine(ctypes.byref(d), 4, 2, 0x1000, 0x2000, 0x3000, 0x4000, 0x4000, None) == 5
+
+
+def test_gated_rmsnorm_checks_arguments(L):
+    f = L.ssd_gated_rmsnorm
+    assert f(4, 1024, 3, 1e-5, 1, 0x10000, 0x20000, 0x30000, None) == 2    # groups must divide the channels
+    assert f(4, 1020, 2, 1e-5, 1, 0x10000, 0x20000, 0x30000, None) == 2    # group of 510: not a multiple of 8
+    assert f(4, 1024, 8, -1.0, 1, 0x10000, 0x20000, 0x30000, None) == 2    # eps < 0
+    assert f(4, 1024, 8, 1e-5, 7, 0x10000, 0x20000, 0x30000, None) == 3
+    assert f(4, 1024, 8, 1e-5, 1, None, 0x20000, 0x30000, None) == 1
+    assert f(4, 1024, 8, 1e-5, 1, 0x10008, 0x20000, 0x30000, None) == 4
+    assert f(0, 1024, 8, 1e-5, 1, None, None, None, None) == 0             # no rows: nothing to do

@@ -192,3 +192,36 @@ def test_prefill_reads_views_of_the_in_proj_output(d, dt):
     yc, fsc, csc = gpu_prefill(dev, d.chunk)
     ops.device_status()
     assert torch.equal(ys, yc) and torch.equal(fss, fsc) and torch.equal(css, csc)
+
+
+@pytest.mark.parametrize("norm_groups", [2, 1])
+def test_gated_rmsnorm_after_prefill_matches_oracle(norm_groups):
+    d = Dims(2, 300, 16, 64, 128, 2, 128)
+    host = make_prefill_inputs(d, dtype=torch.bfloat16, seed=121, init_state=True)
+    dev = dev_inputs(host)
+    y32, y, _, _ = run_both(dev, d.chunk)
+    w = torch.rand(d.nheads * d.headdim, generator=torch.Generator().manual_seed(7)) + 0.5
+    wd = w.cuda()
+    n32 = ops.gated_rmsnorm(y32, wd, norm_groups)
+    ops.device_status()
+    yo, _, _ = oracle.prefill(host)
+    assert_close(np64(n32), oracle.gated_rmsnorm(yo, w.numpy(), norm_groups), "gated rmsnorm")
+    # bf16 in and out: the same fp32 arithmetic on the bf16 values, rounded once at the end
+    n16 = ops.gated_rmsnorm(y, wd, norm_groups)
+    assert_bf16_is_rounded(n16, ops.gated_rmsnorm(y.float(), wd, norm_groups), "gated rmsnorm bf16")
+    # in place
+    y_copy = y.clone()
+    ops.gated_rmsnorm(y_copy, wd, norm_groups, out=y_copy)
+    assert torch.equal(y_copy, n16)
+
+
+@pytest.mark.parametrize("groups", [1, 2, 4, 8])
+def test_gated_rmsnorm_group_sizes(groups):
+    # 4096 channels: groups of 4096 and 2048 take the two-read path, 1024 and 512 the register-held one
+    g = torch.Generator().manual_seed(groups)
+    y = torch.randn((37, 4096), generator=g) * 2.0
+    w = torch.rand(4096, generator=g) + 0.5
+    out = ops.gated_rmsnorm(y.cuda(), w.cuda(), groups)
+    ops.device_status()
+    assert_close(np64(out), oracle.gated_rmsnorm(y.double().numpy(), w.double().numpy(), groups),
+                 f"rmsnorm, {groups} groups", rel_tol=1e-5, abs_tol=1e-4)

@@ -245,3 +245,38 @@ def test_decode_inputs_deterministic():
     b = make_decode_inputs(d, steps=2, seed=9)
     assert torch.equal(a["ssm_state"], b["ssm_state"])
     assert torch.equal(a["steps"][1]["x"], b["steps"][1]["x"])
+
+
+# --- gated RMSNorm: closed forms and invariants -------------------------------------------------
+
+def test_rmsnorm_hand_example():
+    # one group [3, 4]: mean square 12.5, so out = [3, 4] / sqrt(12.5 + eps) * w
+    y = np.array([[3.0, 4.0]])
+    w = np.array([2.0, 0.5])
+    out = oracle.gated_rmsnorm(y, w, 1, eps=0.5)
+    np.testing.assert_allclose(out, [[3.0 * 2.0 / math.sqrt(13.0), 4.0 * 0.5 / math.sqrt(13.0)]], rtol=1e-15)
+
+
+def test_rmsnorm_constant_group_and_group_independence():
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((3, 7, 64))
+    y[:, :, 16:32] = -2.5                          # group 1 of 4 is constant: out = -2.5/sqrt(6.25 + eps) * w
+    w = rng.uniform(0.5, 1.5, 64)
+    out = oracle.gated_rmsnorm(y, w, 4, eps=1e-5)
+    want = np.broadcast_to(-2.5 / math.sqrt(6.25 + 1e-5) * w[16:32], out[:, :, 16:32].shape)
+    np.testing.assert_allclose(out[:, :, 16:32], want, rtol=1e-13)
+    y2 = y.copy()
+    y2[:, :, 48:] *= 10.0                          # another group changes: group 0 does not
+    np.testing.assert_array_equal(oracle.gated_rmsnorm(y2, w, 4)[:, :, :16], out[:, :, :16])
+
+
+def test_rmsnorm_output_has_unit_rms_and_is_scale_free():
+    rng = np.random.default_rng(6)
+    y = rng.standard_normal((5, 256)) * 3.0
+    w = np.ones(256)
+    out = oracle.gated_rmsnorm(y, w, 8, eps=0.0)
+    ms = (out.reshape(5, 8, 32) ** 2).mean(axis=-1)
+    np.testing.assert_allclose(ms, 1.0, rtol=1e-13)
+    np.testing.assert_allclose(oracle.gated_rmsnorm(7.0 * y, w, 8, eps=0.0), out, rtol=1e-13)
+    # one group over all channels is not the mean of the per-group norms
+    assert not np.allclose(oracle.gated_rmsnorm(y, w, 1, eps=0.0), out)
