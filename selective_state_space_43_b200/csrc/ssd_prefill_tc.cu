@@ -27,9 +27,10 @@
 //                           ring), z of the current chunk (one buffer, which
 //                           the epilogue overwrites with y for the TMA store)
 //                  warp 1  TMEM allocator + single-thread tcgen05.mma issuer
-//                  warp 2  each chunk's dt, cumsum of dt*A and mask factors,
-//                           one chunk ahead (double-buffered), from a raw dt
-//                           tile that warp 0 loads with the chunk's raw x
+//                  warp 2  each chunk's dt and cumsum of dt*A one chunk ahead
+//                           (double-buffered), from a raw dt tile that warp 0
+//                           loads with the chunk's raw x; then the chunk's
+//                           decay tables, once the previous chunk's mask is done
 //                  warp 3  TMA producer: post-conv B and C tiles
 //                  warps 4-19 512 compute threads, four per token row i (= TMEM
 //                           lane i), each owning 16 channels / state / output
@@ -38,12 +39,14 @@
 //                           in TMEM for the D skip), decay mask, state pass,
 //                           epilogue (D skip, z gate, y store).  Elementwise
 //                           math uses the packed fp32x2 FMA / MUL of sm_100.
-// The decay mask exp(cs_i - cs_j) is formed per 8-column group: exactly (one
-// exp per element) for the rows inside the group, and as the product of a row
-// factor exp(cs_i - cs_r) and a column factor exp(cs_r - cs_j) dt_j, with r the
-// group's last column, for the rows below it.  Both factors are <= 1, so
-// neither overflows, and either underflows only where the true product is
-// below ~1e-38.
+// The decay exp(cs_i - cs_j) dt_j of M is assembled from tables that the
+// cumsum warp writes for each chunk, so the mask itself needs no MUFU work.
+// With g(i) the 8-row group of i and cs_end(g) the cumsum at the group's last
+// row: inside a group an exact table exp(cs_i - cs_j) dt_j; below it the
+// product exp(cs_i - cs_end(g(i)-1)) exp(cs_end(g(i)-1) - cs_end(g(j)))
+// exp(cs_end(g(j)) - cs_j) dt_j.  With A < 0 the cumsum does not increase, so
+// every factor is <= 1: none overflows, and one underflows only where the true
+// product is below ~1e-38.
 // Every mbarrier wait is bounded; a wait that gives up raises a device error
 // flag (read back by ssd_device_status) and the CTA drains and exits.
 #include <cuda.h>
@@ -81,11 +84,15 @@ constexpr uint32_t OFF_WT = OFF_DTRAW + 2 * 2048;      // conv taps of the head'
 constexpr uint32_t OFF_CB = OFF_WT + 4 * 64 * 4;       // conv bias [64] float
 constexpr uint32_t OFF_HALO = OFF_CB + 64 * 4;         // [2][3][64] bf16 raw x history
 constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;  // cs [2][128] float (double-buffered by chunk parity)
-constexpr uint32_t OFF_DT = OFF_CS + 2 * 128 * 4;      // dt [2][128]
-constexpr uint32_t OFF_COLF = OFF_DT + 2 * 128 * 4;    // column factors of the decay mask [2][128] (8-col groups)
+constexpr uint32_t OFF_COLF = OFF_CS + 2 * 128 * 4;    // exp(cs_end(g(j)) - cs_j) dt_j [2][128]
 constexpr uint32_t OFF_WX = OFF_COLF + 2 * 128 * 4;    // weight of x_j in the chunk state [2][128]
-constexpr uint32_t OFF_BAR = OFF_WX + 2 * 128 * 4;     // mbarriers (8 B each)
-constexpr int NBAR = 17;
+// decay tables of one chunk (single buffer: rewritten once every thread's mask of the previous chunk is done);
+// g = 8-row group, cs_end(g) = cs at the group's last row
+constexpr uint32_t OFF_RFAC = OFF_WX + 2 * 128 * 4;    // exp(cs_i - cs_end(g(i)-1)) [128]
+constexpr uint32_t OFF_PG = OFF_RFAC + 128 * 4;        // exp(cs_end(gi-1) - cs_end(g)), g < gi: [16 gi][4 q][4 kb]
+constexpr uint32_t OFF_DG = OFF_PG + 256 * 4;          // exp(cs_i - cs_j) dt_j inside a group, j <= i: [16][8][8]
+constexpr uint32_t OFF_BAR = OFF_DG + 1024 * 4;        // mbarriers (8 B each)
+constexpr int NBAR = 18;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;  // TMEM base address
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
@@ -95,7 +102,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // FULL_RAW / XREADY / CS_* come in pairs by chunk parity; EPI_DONE = a chunk's epilogue is complete
 // (its Y / Y2 / z read, its y written); EMPTY_BC = the chunk's last B / C reader (Y2) is complete.
 enum Bar { FULL_RAW0 = 0, FULL_RAW1, XREADY0, XREADY1, FULL_Z, EPI_DONE, FULL_BC, EMPTY_BC, MREADY, G_FULL, SC_FULL,
-           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1 };
+           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, TAB_READY };
 
 // TMEM columns (fp32, 128 lanes): G = C B^T, Y = M X, Y2 = C S^T, S_c, the running state, and the
 // post-conv x of two chunks (for the D skip)
@@ -253,7 +260,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
     float* s_cs = reinterpret_cast<float*>(sm + OFF_CS);      // [2][128] per chunk parity
-    float* s_dt = reinterpret_cast<float*>(sm + OFF_DT);
     float* s_colf = reinterpret_cast<float*>(sm + OFF_COLF);
     float* s_wx = reinterpret_cast<float*>(sm + OFF_WX);
     constexpr bool kTmaStoreY = sizeof(TY) == 2;  // bf16 y goes out through TMA from the stage it was written in
@@ -276,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             uint32_t cnt = 1;
             if (k == XREADY0 || k == XREADY1 || k == EPI_DONE || k == MREADY || k == CS_FREE0 || k == CS_FREE1)
                 cnt = kComputeThreads;
-            if (k == CS_READY0 || k == CS_READY1) cnt = 32;
+            if (k == CS_READY0 || k == CS_READY1 || k == TAB_READY) cnt = 32;
             mbar_init(&bars[k], cnt);
         }
         *abort_flag = 0;
@@ -409,21 +415,96 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 if (lane >= o) incl += up;
             }
             const float excl = incl - run;
-            const float cs_last = __shfl_sync(0xffffffffu, incl, 31);
-            // cs at the last row of the 8-row group (rows 8m .. 8m+7 live on lanes 2m, 2m+1)
-            const float cs_g8 = __shfl_sync(0xffffffffu, incl, lane | 1);
+            // The decay factors of the chunk are products of the per-row decays a_r = exp(dt_r A):
+            // exp(cs_i - cs_j) = a_{j+1} ... a_i.  Lane l holds rows 4l .. 4l+3 of the 8-row group gi = l/2;
+            // the pair (2gi, 2gi+1) shares the group's 8 decays, and T_g = a_{8g} ... a_{8g+7}.
+            const int gi = lane >> 1;
+            float ga[8], gdt[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float ak = __expf(dtv[k] * A);
+                const float oak = __shfl_xor_sync(0xffffffffu, ak, 1), odt = __shfl_xor_sync(0xffffffffu, dtv[k], 1);
+                ga[k] = (lane & 1) ? oak : ak;
+                ga[4 + k] = (lane & 1) ? ak : oak;
+                gdt[k] = (lane & 1) ? odt : dtv[k];
+                gdt[4 + k] = (lane & 1) ? dtv[k] : odt;
+            }
+            float pre[8], suf[8];  // a_{8gi} .. a_m  and  a_{m+1} .. a_{8gi+7}
+            {
+                float p = 1.f, q = 1.f;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    p *= ga[m];
+                    pre[m] = p;
+                    suf[7 - m] = q;
+                    q *= ga[7 - m];
+                }
+            }
+            const float tg = pre[7];
+            float tall[16];  // T_g of every group of the chunk
+#pragma unroll
+            for (int g = 0; g < 16; ++g) tall[g] = __shfl_sync(0xffffffffu, tg, 2 * g);
+            float later = 1.f;  // T_{gi+1} ... T_15
+#pragma unroll
+            for (int g = 15; g > 0; --g)
+                if (g > gi) later *= tall[g];
+            const bool odd = lane & 1;  // this lane holds rows 4..7 of its group (else 0..3)
             float csr[4], cf[4], wx[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
+                const float sm_k = odd ? suf[4 + k] : suf[k];  // (register selects, no indexed local array)
                 csr[k] = cs[k] + excl;
-                cf[k] = __expf(cs_g8 - csr[k]) * dtv[k];
-                wx[k] = __expf(cs_last - csr[k]) * dtv[k];
+                cf[k] = sm_k * dtv[k];             // exp(cs_end(gi) - cs_j) dt_j
+                wx[k] = sm_k * later * dtv[k];     // exp(cs_last - cs_j) dt_j
             }
             reinterpret_cast<float4*>(s_cs + buf * 128)[lane] = make_float4(csr[0], csr[1], csr[2], csr[3]);
-            reinterpret_cast<float4*>(s_dt + buf * 128)[lane] = make_float4(dtv[0], dtv[1], dtv[2], dtv[3]);
             reinterpret_cast<float4*>(s_colf + buf * 128)[lane] = make_float4(cf[0], cf[1], cf[2], cf[3]);
             reinterpret_cast<float4*>(s_wx + buf * 128)[lane] = make_float4(wx[0], wx[1], wx[2], wx[3]);
             mbar_arrive(&bars[CS_READY0 + buf]);
+
+            // decay tables of this chunk, once every thread's mask of the previous chunk has read them
+            if (c >= 1 && !warp_wait(&bars[MREADY], (c - 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            float rfac[4];  // exp(cs_i - cs_end(gi-1)) = a_{8gi} ... a_i
+#pragma unroll
+            for (int k = 0; k < 4; ++k) rfac[k] = gi > 0 ? (odd ? pre[4 + k] : pre[k]) : 0.f;
+            reinterpret_cast<float4*>(sm + OFF_RFAC)[lane] = make_float4(rfac[0], rfac[1], rfac[2], rfac[3]);
+            // group-to-group factors of row group gi, exp(cs_end(gi-1) - cs_end(g)) = T_{g+1} ... T_{gi-1}
+            // for g < gi: entries e = 8 (l&1) .. +7 of [4 q][4 kb], g = 4 kb + q
+            float between[16];
+            {
+                float p = 1.f;
+#pragma unroll
+                for (int g = 15; g >= 0; --g) {
+                    between[g] = g < gi ? p : 0.f;
+                    if (g < gi) p *= tall[g];
+                }
+            }
+            float pg[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {  // e = 8 (l&1) + k: g = 4 (k & 3) + (k >> 2) + 2 (l&1)
+                const int g0 = 4 * (k & 3) + (k >> 2);
+                pg[k] = odd ? between[g0 + 2] : between[g0];
+            }
+            float4* pg4 = reinterpret_cast<float4*>(sm + OFF_PG) + gi * 4 + (lane & 1) * 2;
+            pg4[0] = make_float4(pg[0], pg[1], pg[2], pg[3]);
+            pg4[1] = make_float4(pg[4], pg[5], pg[6], pg[7]);
+            // in-group decay of this lane's rows r = 4 (l&1) + k against the group's 8 columns:
+            // exp(cs_r - cs_j) dt_j = a_{j+1} ... a_r dt_j for j <= r, zero above
+            float4* dg4 = reinterpret_cast<float4*>(sm + OFF_DG) + (gi * 8 + 4 * (lane & 1)) * 2;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = 4 * (lane & 1) + k;
+                float dv[8];
+                float prod = 1.f;  // a_{j+1} ... a_r, built from j = r downwards
+#pragma unroll
+                for (int cix = 7; cix >= 0; --cix) {
+                    dv[cix] = cix <= r ? prod * gdt[cix] : 0.f;
+                    if (cix <= r) prod *= ga[cix];
+                }
+                dg4[2 * k] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+                dg4[2 * k + 1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
+            }
+            mbar_arrive(&bars[TAB_READY]);
         }
     } else if (warp == kWarpMma) {
         // ---------------- tcgen05.mma issuer ----------------
@@ -513,14 +594,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             const int Qc = (int)(Ls - t0 < kQ ? Ls - t0 : kQ);
             const bool tma_y = kTmaStoreY && tma_y_chunk<kVarlen>(Ls, c);  // else y is stored from registers
             const float* cs_b = s_cs + buf * 128;
-            const float cs_i = cs_b[i];
             const float cs_last = cs_b[kQ - 1];
 
             // (e) decay mask of row i, columns 8*quarter .. +7 of each 32-column block
             if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
+            // the decay tables of this chunk
+            if (!warp_wait(&bars[TAB_READY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             {
-                const float* dt_b = s_dt + buf * 128;
+                // decay of row i (group gi) against column group g = 4 kb + quarter (columns 8g .. 8g+7):
+                //   g < gi: exp(cs_i - cs_end(gi-1)) exp(cs_end(gi-1) - cs_end(g)) exp(cs_end(g) - cs_j) dt_j
+                //   g = gi: the in-group table;  g > gi: zero
+                const int gi = i >> 3;
+                const float rfac = reinterpret_cast<const float*>(sm + OFF_RFAC)[i];
+                const float4 p4 = reinterpret_cast<const float4*>(sm + OFF_PG)[gi * 4 + quarter];
+                const float pk[4] = {p4.x, p4.y, p4.z, p4.w};
+                const float4* drow = reinterpret_cast<const float4*>(sm + OFF_DG) + (gi * 8 + (i & 7)) * 2;
                 float gv[4][8];
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb)  // warp-uniform: groups right of the diagonal block are zero
@@ -528,40 +617,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 tmem_wait_ld();
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb) {
-                    const int j0 = kb * 32 + quarter * 8;  // first column of this 8-column group
+                    const int g = 4 * kb + quarter;
                     uint4 packed = make_uint4(0u, 0u, 0u, 0u);
-                    if (kb <= q && i >= j0) {
-                        float m[8];
-                        if (i > j0 + 7) {
-                            // below the group: exp(cs_i - cs_j) = exp(cs_i - cs_r) exp(cs_r - cs_j), r = j0 + 7
-                            const float rowf = __expf(cs_i - cs_b[j0 + 7]);
-                            const float2 rf = make_float2(rowf, rowf);
-                            const float4* colf = reinterpret_cast<const float4*>(s_colf + buf * 128 + j0);
-#pragma unroll
-                            for (int e = 0; e < 8; e += 4) {
-                                const float4 cf = colf[e >> 2];
-                                const float2 v0 = __fmul2_rn(__fmul2_rn(make_float2(gv[kb][e], gv[kb][e + 1]),
-                                                                        make_float2(cf.x, cf.y)), rf);
-                                const float2 v1 = __fmul2_rn(__fmul2_rn(make_float2(gv[kb][e + 2], gv[kb][e + 3]),
-                                                                        make_float2(cf.z, cf.w)), rf);
-                                m[e] = v0.x;
-                                m[e + 1] = v0.y;
-                                m[e + 2] = v1.x;
-                                m[e + 3] = v1.y;
-                            }
+                    if (kb <= q && g <= gi) {
+                        float4 fa, fb;
+                        if (g < gi) {
+                            const float4* colf = reinterpret_cast<const float4*>(s_colf + buf * 128 + 8 * g);
+                            const float rf = rfac * pk[kb];
+                            fa = colf[0];
+                            fb = colf[1];
+                            fa = make_float4(fa.x * rf, fa.y * rf, fa.z * rf, fa.w * rf);
+                            fb = make_float4(fb.x * rf, fb.y * rf, fb.z * rf, fb.w * rf);
                         } else {
-                            // the row lies inside the group: exact decay for j <= i
-                            const float4* c4 = reinterpret_cast<const float4*>(cs_b + j0);
-                            const float4* d4 = reinterpret_cast<const float4*>(dt_b + j0);
-                            const float4 ca = c4[0], cb = c4[1], da = d4[0], db = d4[1];
-                            const float cj[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-                            const float dj[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                m[e] = j0 + e <= i ? gv[kb][e] * __expf(cs_i - cj[e]) * dj[e] : 0.f;
+                            fa = drow[0];
+                            fb = drow[1];
                         }
-                        packed = make_uint4(pack_bf2(m[0], m[1]), pack_bf2(m[2], m[3]), pack_bf2(m[4], m[5]),
-                                            pack_bf2(m[6], m[7]));
+                        const float2 m0 = __fmul2_rn(make_float2(gv[kb][0], gv[kb][1]), make_float2(fa.x, fa.y));
+                        const float2 m1 = __fmul2_rn(make_float2(gv[kb][2], gv[kb][3]), make_float2(fa.z, fa.w));
+                        const float2 m2 = __fmul2_rn(make_float2(gv[kb][4], gv[kb][5]), make_float2(fb.x, fb.y));
+                        const float2 m3 = __fmul2_rn(make_float2(gv[kb][6], gv[kb][7]), make_float2(fb.z, fb.w));
+                        packed = make_uint4(pack_bf2(m0.x, m0.y), pack_bf2(m1.x, m1.y), pack_bf2(m2.x, m2.y),
+                                            pack_bf2(m3.x, m3.y));
                     }
                     *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 + sw128_off(i, (kb & 1) * 4 + quarter)) = packed;
                 }
