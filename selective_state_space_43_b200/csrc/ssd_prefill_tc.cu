@@ -774,7 +774,7 @@ __device__ __forceinline__ __nv_bfloat16 conv_history(const PrefillArgs& a, int6
 }
 
 template <bool kVarlen>
-__global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int ntok) {
+__global__ void __launch_bounds__(256, kVarlen ? 3 : 5) bc_prologue_kernel(PrefillArgs a, int ntok) {
     // the chunk scan may start its launch now; it waits for this grid before reading the workspace
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if ((int)blockIdx.x >= ntok) {
@@ -800,6 +800,21 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
     }
     const int64_t b = blockIdx.y;  // 0 for a packed batch
     const int64_t t0 = (int64_t)blockIdx.x * kProTok;  // first row of the window within [0, L)
+    // packed batch: the sequence of row t0 (the largest s with cu[s] <= t0; empty sequences are skipped),
+    // searched once per block
+    __shared__ int64_t s_seq;
+    if constexpr (kVarlen) {
+        if (threadIdx.x == 0) {
+            int64_t lo = 0, hi = a.batch;
+            while (hi - lo > 1) {
+                const int64_t mid = (lo + hi) >> 1;
+                if (a.cu[mid] <= t0) lo = mid;
+                else hi = mid;
+            }
+            s_seq = lo;
+        }
+        __syncthreads();
+    }
     const int half_gn = a.GN / 2;                    // channel pairs per array
     const int pair = blockIdx.z * 256 + threadIdx.x;  // 0 .. GN-1 over both arrays
     if (pair >= a.GN) return;
@@ -819,17 +834,10 @@ __global__ void __launch_bounds__(256) bc_prologue_kernel(PrefillArgs a, int nto
         const int64_t t = t0 - 3 + k;
         raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * rs] : 0u;
     }
-    // packed batch: the sequence of row t0 and where the next one starts (searched while the loads above
-    // are in flight)
+    // packed batch: the sequence of row t0 and where the next one starts
     int64_t seq = 0, start = 0, next = a.L;
     if constexpr (kVarlen) {
-        int64_t lo = 0, hi = a.batch;  // largest seq with cu[seq] <= t0 (empty sequences skipped)
-        while (hi - lo > 1) {
-            const int64_t mid = (lo + hi) >> 1;
-            if (a.cu[mid] <= t0) lo = mid;
-            else hi = mid;
-        }
-        seq = lo;
+        seq = s_seq;
         start = a.cu[seq];
         next = a.cu[seq + 1];
     }
