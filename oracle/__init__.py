@@ -43,6 +43,8 @@ def _bind(lib):
     lib.oracle_prefill.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 12 + [ctypes.c_void_p] + [dp] * 3 + [
         ctypes.c_int]
     lib.oracle_decode_step.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 12 + [ctypes.c_void_p, dp]
+    if hasattr(lib, "oracle_prefill_backward"):
+        lib.oracle_prefill_backward.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 26 + [ctypes.c_int]
     return lib
 
 
@@ -179,6 +181,37 @@ def decode_step(step: dict, params: dict, conv_state, ssm_state, unit_mask=None)
     _load().oracle_decode_step(ctypes.byref(d), *[_ptr(a) for a in arrs],
                                None if mask is None else mask.ctypes.data_as(ctypes.c_void_p), _ptr(y))
     return y
+
+
+def prefill_backward(inp: dict, dy, d_final=None, nthreads: int | None = None):
+    """Gradients of the fp64 prefill (the adjoint of the token-by-token recurrence, for training:
+    "Nemotron-H 스타일 Hybrid Mamba-Transformer 3B 모델 구현 타당성 분석" §3.1/§3.2 checks the new
+    Mamba-2 layer's forward and backward).  The loss whose gradients are returned is
+    sum(dy * y) + sum(d_final * final_state), y and final_state from ``prefill(inp)``; the conv_state
+    output carries none.  ``inp`` as for ``prefill``; dy [Bt, L, H*P]; d_final [Bt, H, P, N] or None.
+    Returns a dict of float64 arrays shaped like the inputs they belong to: x, z, dt, B, C (B/C as
+    [Bt, L, G, N]), A, D, dt_bias, conv_w, conv_b, init_state, init_conv_state (the last two are the
+    gradients for the given initial states, or for zero ones when they are None).
+    """
+    x = _f64(inp["x"])
+    Bt, L, HP = x.shape
+    Bm = _f64(inp["B"])
+    G, N = Bm.shape[2], Bm.shape[3]
+    H = inp["A"].shape[0]
+    P = HP // H
+    conv_dim = HP + 2 * G * N
+    d = _dims(Bt, L, H, P, N, G)
+    arrs = [x, _f64(inp["dt"]), Bm, _f64(inp["C"]), _f64(inp["z"]), _f64(inp["A"]), _f64(inp["D"]),
+            _f64(inp["dt_bias"]), _f64(inp["conv_w"]), _f64(inp["conv_b"]), _f64(inp.get("init_state")),
+            _f64(inp.get("init_conv_state")), _f64(dy), _f64(d_final)]
+    out = {"x": np.empty((Bt, L, HP)), "dt": np.empty((Bt, L, H)), "B": np.empty((Bt, L, G, N)),
+           "C": np.empty((Bt, L, G, N)), "z": np.empty((Bt, L, HP)), "A": np.empty(H), "D": np.empty(H),
+           "dt_bias": np.empty(H), "conv_w": np.empty((conv_dim, 4)), "conv_b": np.empty(conv_dim),
+           "init_state": np.empty((Bt, H, P, N)), "init_conv_state": np.empty((Bt, conv_dim, 3))}
+    order = ("x", "dt", "B", "C", "z", "A", "D", "dt_bias", "conv_w", "conv_b", "init_state", "init_conv_state")
+    _load().oracle_prefill_backward(ctypes.byref(d), *[_ptr(a) for a in arrs], *[_ptr(out[k]) for k in order],
+                                    int(nthreads or default_threads()))
+    return out
 
 
 def gated_rmsnorm(y, weight, ngroups: int, eps: float = 1e-5):

@@ -110,6 +110,17 @@ def make_prefill_inputs(dims: Dims, dtype=torch.bfloat16, seed: int = 43, init_s
     return out
 
 
+def make_backward_grads(dims: Dims, dtype=torch.bfloat16, seed: int = 53, d_final: bool = True) -> dict:
+    """Incoming gradients of one prefill backward call, on the CPU: dy [B, L, H*P] ~ N(0, 1) rounded to
+    ``dtype`` (the gradient of a loss with respect to y) and d_final [B, H, P, N] ~ N(0, 0.1^2) fp32 (the
+    gradient with respect to final_state, present when the next segment's loss depends on it)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    Bt, L, H, P, N = dims.batch, dims.seqlen, dims.nheads, dims.headdim, dims.d_state
+    dy = torch.randn((Bt, L, H * P), generator=g).to(dtype)
+    df = torch.randn((Bt, H, P, N), generator=g) * 0.1
+    return dict(dy=dy, d_final=df if d_final else None)
+
+
 def varlen_lengths(nseq: int, lo: int, hi: int, seed: int) -> list:
     """``nseq`` sequence lengths drawn log-uniformly from [lo, hi] (a continuous-batching mix)."""
     g = torch.Generator(device="cpu").manual_seed(seed)

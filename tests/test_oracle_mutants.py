@@ -10,6 +10,7 @@ import tempfile
 import pytest
 
 import oracle
+import test_oracle_backward_pins as bpins
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssd_oracle.c")
@@ -34,6 +35,29 @@ MUTANTS = {
     "decode missing D": ("const double yv = acc + D[h] * xt[p];", "const double yv = acc;"),
     "decode wrong B group": ("const double* Bt = u + HP + (size_t)g * N;", "const double* Bt = u + HP;"),
     "softplus branch wrong": ("if (v > 30.0) return v + log1p(exp(-v));", "if (v > 0.0) return v;"),
+}
+
+# mistakes in the backward (the adjoint recurrence and the conv backward)
+BACKWARD_MUTANTS = {
+    "adjoint not decayed": ("for (int i2 = 0; i2 < P * N; i2++) lam[i2] *= av[t];",
+                            "for (int i2 = 0; i2 < P * N; i2++) lam[i2] *= 1.0;"),
+    "read-out adjoint after the decay": ("lam[p * N + n] += g_[p] * Ct[n];", "lam[p * N + n] += 0.0 * Ct[n];"),
+    "dC from the previous state": ("duC[t * N + n] += g_[p] * St[p * N + n];",
+                                   "duC[t * N + n] += g_[p] * Sprev[p * N + n];"),
+    "dB without dt": ("duB[t * N + n] += dtv[t] * xt[p] * lam[p * N + n];",
+                      "duB[t * N + n] += xt[p] * lam[p * N + n];"),
+    "decay term of ddt dropped": ("ddt[t] += dxB + lamS * av[t] * j->A[h];", "ddt[t] += dxB;"),
+    "dA without dt": ("dA_h += lamS * av[t] * dtv[t];", "dA_h += lamS * av[t];"),
+    "softplus derivative missing": ("const double v = ddt[t] * o_sigmoid(j->dt_raw[i] + j->dt_bias[h]);",
+                                    "const double v = ddt[t];"),
+    "silu derivative wrong": ("return s * (1.0 + v * (1.0 - s));", "return s;"),
+    "gate gradient ungated": ("g_[p] = j->dy[yi] * o_silu(zv);", "g_[p] = j->dy[yi];"),
+    "D skip gradient dropped": ("dux[t * P + p] += j->D[h] * g_[p];", "dux[t * P + p] += 0.0 * g_[p];"),
+    "conv taps not flipped": ("long t = s + 3 - k;\n            if (t >= 0 && t < L) acc += w[k] * dv[t];",
+                              "long t = s + k;\n            if (t >= 0 && t < L) acc += w[k] * dv[t];"),
+    "conv bias gradient dropped": ("*db += dv[t];", "*db += 0.0;"),
+    "history gradient misplaced": ("else if (d_hist) d_hist[s + 3] = acc;", "else if (d_hist) d_hist[-s - 1] = acc;"),
+    "checkpoint off by one": ("if (t % RECOMP_SEG == 0) memcpy(", "if (t % RECOMP_SEG == 1) memcpy("),
 }
 
 PINS = [
@@ -81,7 +105,34 @@ def test_unmutated_copy_passes_every_pin():
         so = _compile(open(SRC).read(), tmp, "clean")
         oracle.use_library(so)
         try:
-            for pin in PINS:
+            for pin in PINS + BACKWARD_PINS:
                 pin()
+        finally:
+            oracle.use_library(None)
+
+
+BACKWARD_PINS = [
+    lambda: bpins.test_directional_finite_differences(True, True),
+    lambda: bpins.test_elementwise_finite_differences_of_parameters(),
+    lambda: bpins.test_segment_recomputation_boundary(),
+]
+
+
+@pytest.mark.parametrize("name", sorted(BACKWARD_MUTANTS))
+def test_planted_backward_mistake_is_caught(name):
+    src = open(SRC).read()
+    old, new = BACKWARD_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for '{name}' not unique"
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _compile(src.replace(old, new), tmp, "mutant")
+        oracle.use_library(so)
+        try:
+            failed = 0
+            for pin in BACKWARD_PINS:
+                try:
+                    pin()
+                except AssertionError:
+                    failed += 1
+            assert failed > 0, f"no pin caught the planted mistake '{name}'"
         finally:
             oracle.use_library(None)
