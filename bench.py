@@ -38,9 +38,9 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from selective_state_space_43_b200.synth import (Dims, WORKLOADS, make_decode_inputs,  # noqa: E402
-                                                 make_prefill_inputs, make_varlen_inputs, seed_of,
-                                                 varlen_lengths)
+from selective_state_space_43_b200.synth import (Dims, WORKLOADS, make_backward_grads,  # noqa: E402
+                                                 make_decode_inputs, make_prefill_inputs, make_varlen_inputs,
+                                                 seed_of, varlen_lengths)
 
 METRIC = "SSD prefill tokens/s per layer (% bf16 TC peak); decode GB/s (% of HBM peak)"
 PREFILL_WORKLOAD = "nemotron_h_8b"
@@ -49,6 +49,10 @@ L2_FLUSH_BYTES = 256 << 20
 # continuous-batching mix for the packed variable-length prefill: this many sequences of the prefill
 # workload's layer, lengths log-uniform in [VARLEN_MIN, VARLEN_MAX], each with its own initial state
 VARLEN_NSEQ, VARLEN_MIN, VARLEN_MAX = 32, 64, 4096
+# fp32 FMA peak of the CUDA cores, for the backward's SIMT chunk kernel: 148 SMs x 128 fp32 lanes x 2 flops
+# per FMA x the 1965 MHz maximum SM clock
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+BWD_Q = 64  # the backward's chunk length
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -78,6 +82,81 @@ def prefill_flops(d: Dims) -> int:
     # Q x Q times X (2QP), the chunk state B^T X (2NP) and C times the state (2NP)
     per_tok = 2 * d.chunk * d.d_state * d.ngroups + d.nheads * (2 * d.chunk * d.headdim + 4 * d.d_state * d.headdim)
     return d.batch * d.seqlen * per_tok
+
+
+def backward_bytes(d: Dims, act_bytes: int) -> int:
+    """Bytes the backward must move: the forward inputs and dy read (activation dtype), d_final read,
+    the fp32 gradients of the activations and of the initial state written."""
+    rows = d.batch * d.seqlen
+    act_in = rows * (2 * d.d_inner + d.nheads + 2 * d.ngroups * d.d_state) * act_bytes
+    dy = rows * d.d_inner * act_bytes
+    grads = rows * (2 * d.d_inner + d.nheads + 2 * d.ngroups * d.d_state) * 4
+    states = 2 * d.batch * d.nheads * d.headdim * d.d_state * 4
+    return act_in + dy + grads + states
+
+
+def backward_chunk_flops(d: Dims) -> int:
+    """Algorithmic flops of the per-chunk backward (chunk_bwd_kernel) for Q = 64 chunks: per (chunk, head)
+    the four Q x P x N contractions (Sp C, g Sp, Lm B, x Lm), the full Q x Q x P product g.x and the two
+    causal-triangle Q x Q x P (y, dx) and Q x Q x N (dB, dC) sums; per (chunk, group) C.B."""
+    Q, P, N = BWD_Q, d.headdim, d.d_state
+    nc = -(-d.seqlen // Q)
+    per_head = 8 * Q * P * N + 2 * Q * Q * P + 2 * Q * Q * P + 2 * Q * Q * N
+    per_group = 2 * Q * Q * N
+    return d.batch * nc * (d.nheads * per_head + d.ngroups * per_group)
+
+
+def bench_backward(ops, d: Dims, act, dev, flush, K: int, warmup: int, world: int, sampler):
+    """Times ssd_prefill_backward on the prefill workload (bf16 activations and dy, d_final given)."""
+    inp = make_prefill_inputs(d, dtype=act, seed=seed_of(PREFILL_WORKLOAD) + 7)
+    gr = make_backward_grads(d, dtype=act, seed=seed_of(PREFILL_WORKLOAD) + 8)
+    g = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    dy, dfin = gr["dy"].to(dev), gr["d_final"].to(dev)
+    dims = ops.make_dims(d.batch, d.seqlen, d.nheads, d.headdim, d.d_state, d.ngroups, d.chunk)
+    ws = torch.empty(max(ops.prefill_backward_workspace_bytes(dims), 16), dtype=torch.uint8, device=dev)
+
+    def once():
+        return ops.prefill_backward(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"],
+                                    g["conv_w"], g["conv_b"], dy, None, None, dfin, workspace=ws)
+    for _ in range(warmup):
+        flush.zero_()
+        once()
+    torch.cuda.synchronize(dev)
+    KB = max(3, min(K, 10))
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(KB)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(KB)]
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(KB)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(KB)]
+    barrier(world)
+    sampler.load(True)
+    for k in range(KB):
+        flush.zero_()
+        ops.set_timing_events(ks[k], ke[k])
+        st[k].record()
+        once()
+        en[k].record()
+    torch.cuda.synchronize(dev)
+    ops.set_timing_events(None, None)
+    sampler.load(False)
+    barrier(world)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(st, en)) / KB, world, dev)
+    kms = sum(a.elapsed_time(b) for a, b in zip(ks, ke)) / KB
+    tokens = d.batch * d.seqlen
+    flops = backward_chunk_flops(d)
+    tf = flops / (kms * 1e-3) / 1e12
+    nbytes = backward_bytes(d, 2 if act == torch.bfloat16 else 4)
+    return {"value": tokens * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": KB,
+            "workload": f"gradients of the {PREFILL_WORKLOAD} layer prefill (bf16 inputs and dy, fp32 d_final; "
+                        "every input, parameter and initial-state gradient, fp32)",
+            "launch": "eager (7 kernels: post-conv, dt, chunk states, state scans, chunk backward, "
+                      "conv backward, reductions)",
+            "algorithmic_bytes_per_step": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "dominant_kernel": {"kernel": "chunk_bwd_kernel", "ms": kms, "share": kms / ms,
+                                "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_ALU_TFLOPS,
+                                             "unit": "TFLOP/s", "frac": tf / FP32_ALU_TFLOPS, "traffic": None,
+                                             "algorithmic_flops_per_launch": flops,
+                                             "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1965 MHz"}},
+            "l2": "flushed between timed steps (256 MB write outside the step events)"}
 
 
 def decode_bytes(d: Dims, act_bytes: int) -> tuple[int, int]:
@@ -293,6 +372,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a CUDA graph replay")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed variable-length prefill line")
     ap.add_argument("--no-norm", action="store_true", help="skip the gated RMSNorm line")
+    ap.add_argument("--no-backward", action="store_true", help="skip the training-backward line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -564,6 +644,14 @@ def main():
                   "l2": "flushed between timed steps (256 MB write outside the step events)"}
         del gv, vy, vws
 
+    # ---- training backward of the same layer -------------------------------------------------------------
+    backward = None
+    if not args.no_backward:
+        try:
+            backward = bench_backward(ops, d, act, dev, flush, K, args.warmup, world, sampler)
+        except (RuntimeError, ValueError) as exc:  # report it and keep the forward numbers
+            backward = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     clocks = sampler.stop()
 
     # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------------------------------------
@@ -583,7 +671,7 @@ def main():
                        "l2": "flushed between timed steps (256 MB write outside the step events)",
                        "kernel_path": "tcgen05 tensor-core" if path == 1 else "CUDA-core", "launch": launch},
             "tensor": tc, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
-            "varlen": varlen, "gated_rmsnorm": norm,
+            "varlen": varlen, "gated_rmsnorm": norm, "backward": backward,
             "gpu_launches": K * (2 if path == 1 else 1), "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

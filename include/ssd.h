@@ -273,6 +273,48 @@ SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t nor
                                      ssd_dtype dtype, const void* y, const float* weight, void* out, void* stream);
 
 /*
+ * Gradients of ssd_prefill, for training ("Nemotron-H 스타일 Hybrid Mamba-Transformer
+ * 3B 모델 구현 타당성 분석" §3.1/§3.2: the hybrid is trained from scratch and the
+ * new Mamba-2 layer's forward and backward are checked).  The gradients are
+ * those of the loss  sum(dy * y) + sum(d_final_state * final_state)  with y and
+ * final_state the outputs of ssd_prefill on the same inputs; the conv_state
+ * output carries none.  Every gradient is fp32 and is written, never added to.
+ *
+ *   inputs        exactly as for ssd_prefill (contiguous rows; dims->chunk is
+ *                 validated but the backward uses its own 64-token chunks)
+ *   dy            [batch][seqlen][H*P]: bf16 for SSD_BF16, fp32 for SSD_F32 and
+ *                 SSD_BF16_YF32 (the dtype of the forward's y)
+ *   d_final_state [batch][H][P][N] fp32, or NULL for zero
+ *   grads         dx, dz [batch][seqlen][H*P]; ddt [batch][seqlen][H] (of dt_raw);
+ *                 dB, dC [batch][seqlen][G][N] (pre-conv inputs);
+ *                 dA, dD, ddt_bias [H]; dconv_w [conv_dim][4]; dconv_b [conv_dim]
+ *                 (summed over the batch); d_init_state [batch][H][P][N] and
+ *                 d_init_conv_state [batch][conv_dim][3], each NULL when not
+ *                 wanted (they are the gradients for the given initial states,
+ *                 or for zero ones when those are NULL)
+ *   workspace     device scratch of ssd_prefill_backward_workspace_bytes()
+ *                 (the post-conv channels and their gradients, fp32, plus two
+ *                 fp32 [batch][ceil(seqlen/64)][H][P][N] state arrays)
+ * All pointers device memory, 16-byte aligned; gradients must not overlap the
+ * inputs or one another.  The result is deterministic (every sum is taken in a
+ * fixed order).  seqlen == 0 is valid: d_init_state = d_final_state (or zero),
+ * the parameter gradients and d_init_conv_state are zero.  Errors as for
+ * ssd_prefill; SSD_ERR_SHAPE also when ceil(seqlen/64) or batch exceeds 65535.
+ */
+typedef struct {
+    float *dx, *ddt, *dB, *dC, *dz;
+    float *dA, *dD, *ddt_bias, *dconv_w, *dconv_b;
+    float *d_init_state, *d_init_conv_state;
+} ssd_grads;
+
+SSD_API size_t ssd_prefill_backward_workspace_bytes(const ssd_dims* dims);
+SSD_API ssd_status ssd_prefill_backward(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
+                                        const void* x, const void* dt, const void* B, const void* C, const void* z,
+                                        const float* init_state, const void* init_conv_state, const void* dy,
+                                        const float* d_final_state, const ssd_grads* grads, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream` and reports whether a kernel launched by this library
  * gave up on a bounded device-side wait since the last call (SSD_ERR_TIMEOUT;
  * its outputs are then incomplete), or whether the stream holds a CUDA error

@@ -3,6 +3,7 @@
 #include <stdint.h>
 
 #include "ssd.h"
+#include "ssd_backward.h"
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
 
@@ -224,6 +225,55 @@ ssd_status ssd_decode_step(const ssd_dims* d, ssd_dtype dtype, const ssd_params*
     const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
                                                                                         : ssd::ActKind::BF16_YF32);
     cudaError_t e = ssd::launch_decode(a, s.batch, kind, static_cast<cudaStream_t>(stream), g_hook);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+size_t ssd_prefill_backward_workspace_bytes(const ssd_dims* d) {
+    if (!d || check_dims(d, SSD_F32, true) != SSD_OK) return 0;
+    return ssd::bwd::workspace_bytes(d->batch, d->seqlen, d->nheads, d->headdim, d->d_state, d->ngroups);
+}
+
+ssd_status ssd_prefill_backward(const ssd_dims* d, ssd_dtype dtype, const ssd_params* params, const void* x,
+                                const void* dt, const void* B, const void* C, const void* z,
+                                const float* init_state, const void* init_conv_state, const void* dy,
+                                const float* d_final_state, const ssd_grads* g, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    ssd_status st = check_dims(d, dtype, true);
+    if (st != SSD_OK) return st;
+    if ((st = check_params(params)) != SSD_OK) return st;
+    if (!g) return SSD_ERR_NULL;
+    // grid limits of the backward's launches: 64-token chunks and the batch on the y / z grid axes
+    if ((d->seqlen + 63) / 64 > 65535 || d->batch > 65535) return SSD_ERR_SHAPE;
+    const bool tokens = d->batch > 0 && d->seqlen > 0;
+    if (tokens && (!x || !dt || !B || !C || !z || !dy || !g->dx || !g->ddt || !g->dB || !g->dC || !g->dz))
+        return SSD_ERR_NULL;
+    if (!g->dA || !g->dD || !g->ddt_bias || !g->dconv_w || !g->dconv_b) return SSD_ERR_NULL;
+    const void* ptrs[] = {x, dt, B, C, z, init_state, init_conv_state, dy, d_final_state, g->dx, g->ddt, g->dB,
+                          g->dC, g->dz, g->dA, g->dD, g->ddt_bias, g->dconv_w, g->dconv_b, g->d_init_state,
+                          g->d_init_conv_state, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return SSD_ERR_ALIGN;
+    const size_t need = ssd::bwd::workspace_bytes(d->batch, d->seqlen, d->nheads, d->headdim, d->d_state,
+                                                  d->ngroups);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
+
+    ssd::bwd::BwdArgs a{};
+    a.batch = d->batch;
+    a.L = d->seqlen;
+    a.H = d->nheads; a.P = d->headdim; a.N = d->d_state; a.G = d->ngroups;
+    a.act_bf16 = dtype != SSD_F32;
+    a.dy_bf16 = dtype == SSD_BF16;
+    a.A = params->A; a.D = params->D; a.dt_bias = params->dt_bias;
+    a.conv_w = params->conv_w; a.conv_b = params->conv_b;
+    a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z; a.dy = dy;
+    a.init_state = init_state; a.init_conv_state = init_conv_state; a.d_final = d_final_state;
+    a.dx = g->dx; a.ddt = g->ddt; a.dB = g->dB; a.dC = g->dC; a.dz = g->dz;
+    a.dA = g->dA; a.dD = g->dD; a.ddt_bias = g->ddt_bias; a.dconv_w = g->dconv_w; a.dconv_b = g->dconv_b;
+    a.d_init_state = g->d_init_state; a.d_init_conv_state = g->d_init_conv_state;
+    a.workspace = workspace;
+    a.ev_before = g_hook.ev_before;
+    a.ev_after = g_hook.ev_after;
+    cudaError_t e = ssd::bwd::launch_prefill_backward(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

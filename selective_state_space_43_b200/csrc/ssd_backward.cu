@@ -1,0 +1,698 @@
+// ssd_backward.cu -- gradients of the chunked SSD prefill (the training backward).
+//
+// The layer is trained from scratch in "Nemotron-H 스타일 Hybrid Mamba-Transformer
+// 3B 모델 구현 타당성 분석" (§3.1: the new Mamba-2 layer needs its forward and
+// backward checked; §3.2 phase 2).  The backward differentiates the loss
+//   sum dy . y + sum d_final . final_state
+// through the whole layer core: conv1d (k=4) + SiLU on [x | B | C], dt =
+// softplus(dt_raw + dt_bias), the scalar-decay state recurrence, the D skip
+// and the SiLU(z) gate.
+//
+// It works on its own 64-token chunks (the chunk length is an implementation
+// choice; the gradients do not depend on it beyond rounding).  With, inside a
+// chunk, cs_i the inclusive cumulative sum of dt*A, L_ij = exp(cs_i - cs_j)
+// (i >= j), g_i = dy_i * silu(z_i), Sp the state entering the chunk and Lm the
+// adjoint of the state leaving it:
+//
+//   y_i   = sum_{j<=i} (C_i.B_j) L_ij dt_j x_j + exp(cs_i) Sp C_i + D x_i
+//   dx_j  = dt_j [sum_{i>=j} (C_i.B_j) L_ij g_i + exp(cs_last - cs_j) Lm B_j] + D g_j
+//   dB_j  = dt_j [sum_{i>=j} (g_i.x_j) L_ij C_i + exp(cs_last - cs_j) x_j Lm]     (summed over the group's heads)
+//   dC_i  = sum_{j<=i} (g_i.x_j) L_ij dt_j B_j + exp(cs_i) g_i Sp                  (summed over the group's heads)
+//   d(dA_k) = sum_{i>=k} sum_{j<k} M_ij + sum_{i>=k} E_i + F + sum_{j<k} W_j,
+//     M_ij = (g_i.x_j)(C_i.B_j) L_ij dt_j,  E_i = exp(cs_i) g_i.(Sp C_i),
+//     F = exp(cs_last) <Lm, Sp>,  W_j = exp(cs_last - cs_j) dt_j x_j.(Lm B_j)
+//   ddt_j = sum_i M_ij / dt_j + W_j / dt_j + A d(dA_j)   (the first two formed without dividing)
+//   Lm of chunk c-1 = exp(cs_last,c) Lm_c + sum_{i in c} exp(cs_i) g_i (outer) C_i
+//
+// Kernels, in launch order (all fp32 arithmetic):
+//   post_conv_kernel    u = silu(conv(xBC)) of every channel and token           -> U
+//   dt_kernel           dt and the in-chunk cumsum of dt*A                       -> DT, CS
+//   chunk_state_kernel  per (chunk, head): sum exp(cs_last-cs_j) dt_j x_j B_j^T and
+//                       sum exp(cs_i) g_i C_i^T                                   -> SP, LM
+//   state_pass_kernel   per head: forward scan of SP into the entering states,
+//                       reverse scan of LM into the leaving adjoints, F per chunk,
+//                       d_init_state
+//   chunk_bwd_kernel    per (chunk, group), heads in turn: dz, ddt, the post-conv
+//                       gradients of x (per head) and of B, C (summed over the group)
+//   conv_bwd_kernel     per (channel, 64-token tile): through SiLU' and the taps to
+//                       the pre-conv gradients, per-tile conv_w/conv_b partial sums,
+//                       d_init_conv_state
+//   reduce_kernel       sums of the per-tile / per-chunk partials in a fixed order
+//                       -> dconv_w, dconv_b, dA, dD, ddt_bias (deterministic)
+//
+// SSD_EMU: compiled as plain C++ by the tests' host emulation (one thread per
+// CUDA thread, a real barrier for __syncthreads), which runs this same source
+// on the CPU under AddressSanitizer; the library is always built with nvcc.
+#ifdef SSD_EMU
+#include "emu_cuda.h"
+#define SSD_LAUNCH(kern, grid, block, smem, st, ...) \
+    ((void)(st), ::emu::launch((grid), (block), (smem), [&]() { kern(__VA_ARGS__); }))
+#define SSD_SET_SMEM(kern, bytes) cudaSuccess
+#define SSD_DYN_SMEM() (::emu::smem())
+#else
+#include <cuda_runtime.h>
+#define SSD_LAUNCH(kern, grid, block, smem, st, ...) kern<<<(grid), (block), (smem), (st)>>>(__VA_ARGS__)
+#define SSD_SET_SMEM(kern, bytes) \
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes))
+extern __shared__ __align__(16) unsigned char ssd_bwd_smem[];
+#define SSD_DYN_SMEM() (ssd_bwd_smem)
+#endif
+
+#include "ssd_backward.h"
+
+namespace ssd {
+namespace bwd {
+
+constexpr int kQ = 64;    // backward chunk (tokens); also the conv backward's tile
+constexpr int kT = 256;   // threads per block
+constexpr int kP = 64;    // head dimension
+constexpr int kS = kQ + 1;  // padded row stride of the 64-wide shared tiles
+
+struct Ws {
+    float* U;   // [batch][L][conv_dim]  post-conv, post-SiLU channels
+    float* DU;  // [batch][L][conv_dim]  their gradients
+    float* DT;  // [batch][H][L]         dt
+    float* CS;  // [batch][H][L]         in-chunk inclusive cumsum of dt*A
+    float* SP;  // [batch][nc][H][P][N]  chunk-local states, then the states entering each chunk
+    float* LM;  // [batch][nc][H][P][N]  chunk-local adjoints, then the adjoints leaving each chunk
+    float* PF;  // [batch][nc][H]        F = exp(cs_last) <Lm, Sp>
+    float* PH;  // [batch][nc][H][3]     per-chunk partial dA, dD, ddt_bias
+    float* PW;  // [batch][ntile][conv_dim][5]  per-tile partial dconv_w (4), dconv_b
+};
+
+namespace {
+
+__host__ __device__ inline int64_t nchunks(int64_t L) { return (L + kQ - 1) / kQ; }
+__host__ __device__ inline int64_t ntiles(int64_t L) { return L > 0 ? nchunks(L) : 1; }
+inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Carves the workspace; returns the bytes used (base may be null to only count).
+size_t carve(int64_t batch, int64_t L, int H, int P, int N, int G, char* base, Ws* ws) {
+    const int64_t conv_dim = (int64_t)H * P + 2LL * G * N, nc = nchunks(L), nt = ntiles(L);
+    const size_t sizes[9] = {
+        (size_t)(batch * L * conv_dim), (size_t)(batch * L * conv_dim), (size_t)(batch * H * L),
+        (size_t)(batch * H * L),        (size_t)(batch * nc * H * P * N), (size_t)(batch * nc * H * P * N),
+        (size_t)(batch * nc * H),       (size_t)(batch * nc * H * 3),     (size_t)(batch * nt * conv_dim * 5)};
+    float** slots[9] = {&ws->U, &ws->DU, &ws->DT, &ws->CS, &ws->SP, &ws->LM, &ws->PF, &ws->PH, &ws->PW};
+    size_t off = 0;
+    for (int k = 0; k < 9; ++k) {
+        if (base) *slots[k] = reinterpret_cast<float*>(base + off);
+        off += round256(sizes[k] * sizeof(float));
+    }
+    return off;
+}
+
+__device__ __forceinline__ float ld_act(const void* p, int64_t i, bool bf16) {
+    if (bf16) return __uint_as_float(static_cast<unsigned>(static_cast<const unsigned short*>(p)[i]) << 16);
+    return static_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ float sigmoid_f(float v) { return 1.f / (1.f + expf(-v)); }
+__device__ __forceinline__ float silu_f(float v) { return v * sigmoid_f(v); }
+__device__ __forceinline__ float dsilu_f(float v) {
+    const float s = sigmoid_f(v);
+    return s * (1.f + v * (1.f - s));
+}
+__device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(expf(v)); }
+
+// Pre-conv value of channel c at token s of sequence b (s in [-3, L)); history or zero before 0.
+__device__ __forceinline__ float raw_at(const BwdArgs& a, int64_t b, int64_t s, int64_t c) {
+    const int64_t HP = (int64_t)a.H * a.P, GN = (int64_t)a.G * a.N, conv_dim = HP + 2 * GN;
+    if (s < 0)
+        return a.init_conv_state ? ld_act(a.init_conv_state, (b * conv_dim + c) * 3 + (s + 3), a.act_bf16) : 0.f;
+    const int64_t row = b * a.L + s;
+    if (c < HP) return ld_act(a.x, row * HP + c, a.act_bf16);
+    if (c < HP + GN) return ld_act(a.B, row * GN + (c - HP), a.act_bf16);
+    return ld_act(a.C, row * GN + (c - HP - GN), a.act_bf16);
+}
+
+// grid (ceil(conv_dim / kT), nchunks, batch): one thread per (channel, 64-token tile).
+__global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
+    const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N;
+    const int64_t c = (int64_t)blockIdx.x * kT + threadIdx.x;
+    if (c >= conv_dim) return;
+    const int64_t b = blockIdx.z, t0 = (int64_t)blockIdx.y * kQ;
+    const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
+    const float w0 = a.conv_w[c * 4 + 0], w1 = a.conv_w[c * 4 + 1], w2 = a.conv_w[c * 4 + 2],
+                w3 = a.conv_w[c * 4 + 3], bias = a.conv_b[c];
+    float r0 = raw_at(a, b, t0 - 3, c), r1 = raw_at(a, b, t0 - 2, c), r2 = raw_at(a, b, t0 - 1, c);
+    for (int64_t t = t0; t < t1; ++t) {
+        const float r3 = raw_at(a, b, t, c);
+        ws.U[(b * a.L + t) * conv_dim + c] = silu_f(bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * r3);
+        r0 = r1;
+        r1 = r2;
+        r2 = r3;
+    }
+}
+
+// grid (ceil(H * nchunks / kT), batch): one thread per (head, chunk).
+__global__ void __launch_bounds__(kT) dt_kernel(BwdArgs a, Ws ws) {
+    const int64_t nc = nchunks(a.L);
+    const int64_t idx = (int64_t)blockIdx.x * kT + threadIdx.x;
+    if (idx >= nc * a.H) return;
+    const int h = static_cast<int>(idx % a.H);
+    const int64_t c = idx / a.H, b = blockIdx.y, t0 = c * kQ;
+    const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
+    const float Ah = a.A[h], bias = a.dt_bias[h];
+    float cs = 0.f;
+    for (int64_t t = t0; t < t1; ++t) {
+        const float dt = softplus_f(ld_act(a.dt, (b * a.L + t) * a.H + h, a.act_bf16) + bias);
+        cs += dt * Ah;
+        ws.DT[(b * a.H + h) * a.L + t] = dt;
+        ws.CS[(b * a.H + h) * a.L + t] = cs;
+    }
+}
+
+// grid (nchunks, H, batch), kT threads.  Chunk-local state and adjoint sums of one head:
+//   SP[p][n] = sum_j exp(cs_last - cs_j) dt_j x_j[p] B_j[n],  LM[p][n] = sum_i exp(cs_i) g_i[p] C_i[n].
+template <int N>
+__global__ void __launch_bounds__(kT) chunk_state_kernel(BwdArgs a, Ws ws) {
+    constexpr int M = kP * N / kT;  // outputs per thread
+    const int64_t nc = nchunks(a.L), HP = (int64_t)a.H * kP, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
+    const int64_t c = blockIdx.x, b = blockIdx.z;
+    const int h = blockIdx.y, g = h / (a.H / a.G), tid = threadIdx.x;
+    const int64_t t0 = c * kQ;
+    const int Qv = static_cast<int>(a.L - t0 < kQ ? a.L - t0 : kQ);
+
+    float* sm = reinterpret_cast<float*>(SSD_DYN_SMEM());
+    float* wx = sm;               // [kQ][kP]
+    float* wg = wx + kQ * kP;     // [kQ][kP]
+    float* Bs = wg + kQ * kP;     // [kQ][N]
+    float* Cs = Bs + kQ * N;      // [kQ][N]
+    float* fx = Cs + kQ * N;      // [kQ]
+    float* fg = fx + kQ;          // [kQ]
+
+    const float* dtp = ws.DT + (b * a.H + h) * a.L + t0;
+    const float* csp = ws.CS + (b * a.H + h) * a.L + t0;
+    if (tid < kQ) {
+        if (tid < Qv) {
+            fx[tid] = dtp[tid] * expf(csp[Qv - 1] - csp[tid]);
+            fg[tid] = expf(csp[tid]);
+        } else {
+            fx[tid] = 0.f;
+            fg[tid] = 0.f;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < kQ * kP; e += kT) {
+        const int j = e / kP, p = e % kP;
+        if (j < Qv) {
+            const int64_t row = b * a.L + t0 + j;
+            wx[e] = ws.U[row * conv_dim + (int64_t)h * kP + p] * fx[j];
+            const int64_t yi = row * HP + (int64_t)h * kP + p;
+            wg[e] = ld_act(a.dy, yi, a.dy_bf16) * silu_f(ld_act(a.z, yi, a.act_bf16)) * fg[j];
+        } else {
+            wx[e] = 0.f;
+            wg[e] = 0.f;
+        }
+    }
+    for (int e = tid; e < kQ * N; e += kT) {
+        const int j = e / N, n = e % N;
+        if (j < Qv) {
+            const int64_t row = (b * a.L + t0 + j) * conv_dim;
+            Bs[e] = ws.U[row + HP + (int64_t)g * N + n];
+            Cs[e] = ws.U[row + HP + GN + (int64_t)g * N + n];
+        } else {
+            Bs[e] = 0.f;
+            Cs[e] = 0.f;
+        }
+    }
+    __syncthreads();
+    const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const int e = tid + kT * m, p = e / N, n = e % N;
+        float s = 0.f, l = 0.f;
+        for (int j = 0; j < Qv; ++j) {
+            s += wx[j * kP + p] * Bs[j * N + n];
+            l += wg[j * kP + p] * Cs[j * N + n];
+        }
+        ws.SP[base + e] = s;
+        ws.LM[base + e] = l;
+    }
+}
+
+// Sum of v over the block (kT threads); every thread gets the total.  red: kT floats.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+    const int tid = threadIdx.x;
+    red[tid] = v;
+    __syncthreads();
+    for (int s = kT / 2; s > 0; s >>= 1) {
+        if (tid < s) red[tid] += red[tid + s];
+        __syncthreads();
+    }
+    const float total = red[0];
+    __syncthreads();
+    return total;
+}
+
+// grid (H, batch), kT threads; each thread owns P*N/kT state elements of one head.
+template <int N>
+__global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
+    constexpr int M = kP * N / kT;
+    const int64_t nc = nchunks(a.L), b = blockIdx.y;
+    const int h = blockIdx.x, tid = threadIdx.x;
+    float* red = reinterpret_cast<float*>(SSD_DYN_SMEM());
+    const int64_t head = (b * a.H + h) * (int64_t)kP * N;
+
+    float s[M], l[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) s[m] = a.init_state ? a.init_state[head + tid + kT * m] : 0.f;
+    for (int64_t c = 0; c < nc; ++c) {
+        const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
+        const float decay = expf(ws.CS[(b * a.H + h) * a.L + last]);
+        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const int64_t i = base + tid + kT * m;
+            const float loc = ws.SP[i];
+            ws.SP[i] = s[m];
+            s[m] = decay * s[m] + loc;
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) l[m] = a.d_final ? a.d_final[head + tid + kT * m] : 0.f;
+    for (int64_t c = nc - 1; c >= 0; --c) {
+        const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
+        const float decay = expf(ws.CS[(b * a.H + h) * a.L + last]);
+        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
+        float f = 0.f;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const int64_t i = base + tid + kT * m;
+            const float loc = ws.LM[i];
+            ws.LM[i] = l[m];
+            f += l[m] * ws.SP[i];
+            l[m] = decay * l[m] + loc;
+        }
+        f = block_sum(f, red);
+        if (tid == 0) ws.PF[(b * nc + c) * a.H + h] = decay * f;
+    }
+    if (a.d_init_state) {
+#pragma unroll
+        for (int m = 0; m < M; ++m) a.d_init_state[head + tid + kT * m] = l[m];
+    }
+}
+
+template <int N>
+constexpr size_t chunk_bwd_floats() {
+    // Bs, Cs [kQ][N+1]; CB, LCB, LGX, T, xs, gs [kQ][kS]; X [kP][N+1]; 7 vectors of kQ; 3 x kT reduction
+    return 2 * (size_t)kQ * (N + 1) + 6 * (size_t)kQ * kS + (size_t)kP * (N + 1) + 7 * (size_t)kQ + 3 * (size_t)kT;
+}
+
+// grid (nchunks, G, batch), kT threads.  One chunk of one group; the group's heads in turn.
+template <int N>
+__global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
+    constexpr int NS = N + 1;         // padded row stride of the N-wide tiles
+    constexpr int M = kQ * N / kT;    // dB / dC entries per thread
+    const int64_t nc = nchunks(a.L), HP = (int64_t)a.H * kP, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
+    const int64_t c = blockIdx.x, b = blockIdx.z, t0 = c * kQ;
+    const int g = blockIdx.y, hpg = a.H / a.G, tid = threadIdx.x;
+    const int Qv = static_cast<int>(a.L - t0 < kQ ? a.L - t0 : kQ);
+
+    float* sm = reinterpret_cast<float*>(SSD_DYN_SMEM());
+    float* Bs = sm;                  // [kQ][NS]  post-conv B of the group
+    float* Cs = Bs + kQ * NS;        // [kQ][NS]
+    float* CB = Cs + kQ * NS;        // [kQ][kS]  C_i . B_j
+    float* LCB = CB + kQ * kS;       // [kQ][kS]  L_ij C_i . B_j   (i >= j, else 0)
+    float* LGX = LCB + kQ * kS;      // [kQ][kS]  L_ij g_i . x_j   (i >= j, else 0)
+    float* T = LGX + kQ * kS;        // [kQ][kS]  Sp C_i, then Lm B_j, then row prefix sums of M
+    float* xs = T + kQ * kS;         // [kQ][kS]  post-conv x of the head
+    float* gs = xs + kQ * kS;        // [kQ][kS]  g = dy * silu(z)
+    float* X = gs + kQ * kS;         // [kP][NS]  Sp, then Lm
+    float* dts = X + kP * NS;        // [kQ]
+    float* css = dts + kQ;
+    float* ex = css + kQ;            // exp(cs_i)
+    float* el = ex + kQ;             // exp(cs_last - cs_j)
+    float* Ev = el + kQ;
+    float* Wv = Ev + kQ;             // exp(cs_last - cs_j) x_j . (Lm B_j)
+    float* Dr = Wv + kQ;             // ddt without the decay term
+    float* red = Dr + kQ;            // [3][kT]
+
+    // the group's post-conv B and C, and C_i . B_j
+    for (int e = tid; e < kQ * N; e += kT) {
+        const int j = e / N, n = e % N;
+        float bv = 0.f, cv = 0.f;
+        if (j < Qv) {
+            const int64_t row = (b * a.L + t0 + j) * conv_dim;
+            bv = ws.U[row + HP + (int64_t)g * N + n];
+            cv = ws.U[row + HP + GN + (int64_t)g * N + n];
+        }
+        Bs[j * NS + n] = bv;
+        Cs[j * NS + n] = cv;
+    }
+    __syncthreads();
+    for (int e = tid; e < kQ * kQ; e += kT) {
+        const int i = e / kQ, j = e % kQ;
+        float acc = 0.f;
+        for (int n = 0; n < N; ++n) acc += Cs[i * NS + n] * Bs[j * NS + n];
+        CB[i * kS + j] = acc;
+    }
+
+    float dBa[M], dCa[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        dBa[m] = 0.f;
+        dCa[m] = 0.f;
+    }
+
+    for (int hl = 0; hl < hpg; ++hl) {
+        const int h = g * hpg + hl;
+        const float Dh = a.D[h], Ah = a.A[h], bias = a.dt_bias[h];
+        const int64_t hrow = (b * a.H + h) * a.L + t0;
+        const int64_t sbase = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
+
+        // 1: dt, cs, x and g of the head
+        if (tid < kQ) {
+            dts[tid] = tid < Qv ? ws.DT[hrow + tid] : 0.f;
+            css[tid] = tid < Qv ? ws.CS[hrow + tid] : 0.f;
+        }
+        for (int e = tid; e < kQ * kP; e += kT) {
+            const int j = e / kP, p = e % kP;
+            float xv = 0.f, gv = 0.f;
+            if (j < Qv) {
+                const int64_t row = b * a.L + t0 + j;
+                xv = ws.U[row * conv_dim + (int64_t)h * kP + p];
+                const int64_t yi = row * HP + (int64_t)h * kP + p;
+                gv = ld_act(a.dy, yi, a.dy_bf16) * silu_f(ld_act(a.z, yi, a.act_bf16));
+            }
+            xs[j * kS + p] = xv;
+            gs[j * kS + p] = gv;
+        }
+        __syncthreads();
+
+        // 2: decay factors, L-weighted C.B and g.x, the entering state
+        const float cl = css[Qv - 1];
+        if (tid < kQ) {
+            ex[tid] = tid < Qv ? expf(css[tid]) : 0.f;
+            el[tid] = tid < Qv ? expf(cl - css[tid]) : 0.f;
+        }
+        for (int e = tid; e < kQ * kQ; e += kT) {
+            const int i = e / kQ, j = e % kQ;
+            float lcb = 0.f, lgx = 0.f;
+            if (j <= i && i < Qv) {
+                const float Lij = expf(css[i] - css[j]);
+                float gx = 0.f;
+                for (int p = 0; p < kP; ++p) gx += gs[i * kS + p] * xs[j * kS + p];
+                lcb = CB[i * kS + j] * Lij;
+                lgx = gx * Lij;
+            }
+            LCB[i * kS + j] = lcb;
+            LGX[i * kS + j] = lgx;
+        }
+        for (int e = tid; e < kP * N; e += kT) X[(e / N) * NS + e % N] = ws.SP[sbase + e];
+        __syncthreads();
+
+        // 3: T = Sp C_i;  dC_i += exp(cs_i) g_i Sp
+        for (int e = tid; e < kQ * kP; e += kT) {
+            const int i = e / kP, p = e % kP;
+            float acc = 0.f;
+            for (int n = 0; n < N; ++n) acc += X[p * NS + n] * Cs[i * NS + n];
+            T[i * kS + p] = acc;
+        }
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const int e = tid + kT * m, i = e / N, n = e % N;
+            float acc = 0.f;
+            for (int p = 0; p < kP; ++p) acc += gs[i * kS + p] * X[p * NS + n];
+            dCa[m] += ex[i] * acc;
+        }
+        __syncthreads();
+
+        // 4: y recomputed for dz;  E_i
+        for (int e = tid; e < kQ * kP; e += kT) {
+            const int i = e / kP, p = e % kP;
+            if (i < Qv) {
+                float acc = 0.f;
+                for (int j = 0; j <= i; ++j) acc += LCB[i * kS + j] * dts[j] * xs[j * kS + p];
+                const float yv = acc + ex[i] * T[i * kS + p] + Dh * xs[i * kS + p];
+                const int64_t yi = (b * a.L + t0 + i) * HP + (int64_t)h * kP + p;
+                a.dz[yi] = ld_act(a.dy, yi, a.dy_bf16) * yv * dsilu_f(ld_act(a.z, yi, a.act_bf16));
+            }
+        }
+        if (tid < kQ) {
+            float acc = 0.f;
+            for (int p = 0; p < kP; ++p) acc += gs[tid * kS + p] * T[tid * kS + p];
+            Ev[tid] = ex[tid] * acc;
+        }
+        __syncthreads();
+
+        // 5: the leaving adjoint; T = Lm B_j;  dB_j += dt_j exp(cs_last - cs_j) x_j Lm
+        for (int e = tid; e < kP * N; e += kT) X[(e / N) * NS + e % N] = ws.LM[sbase + e];
+        __syncthreads();
+        for (int e = tid; e < kQ * kP; e += kT) {
+            const int j = e / kP, p = e % kP;
+            float acc = 0.f;
+            for (int n = 0; n < N; ++n) acc += X[p * NS + n] * Bs[j * NS + n];
+            T[j * kS + p] = acc;
+        }
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const int e = tid + kT * m, j = e / N, n = e % N;
+            float acc = 0.f;
+            for (int p = 0; p < kP; ++p) acc += xs[j * kS + p] * X[p * NS + n];
+            dBa[m] += dts[j] * el[j] * acc;
+        }
+        __syncthreads();
+
+        // 6: dx (post-conv, this head's channels);  W_j and the direct part of ddt
+        for (int e = tid; e < kQ * kP; e += kT) {
+            const int j = e / kP, p = e % kP;
+            if (j < Qv) {
+                float acc = 0.f;
+                for (int i = j; i < Qv; ++i) acc += LCB[i * kS + j] * gs[i * kS + p];
+                const float d = dts[j] * (acc + el[j] * T[j * kS + p]) + Dh * gs[j * kS + p];
+                ws.DU[(b * a.L + t0 + j) * conv_dim + (int64_t)h * kP + p] = d;
+            }
+        }
+        if (tid < kQ) {
+            float w = 0.f;
+            for (int p = 0; p < kP; ++p) w += xs[tid * kS + p] * T[tid * kS + p];
+            w *= el[tid];
+            float dr = w;
+            for (int i = tid; i < Qv; ++i) dr += LGX[i * kS + tid] * CB[i * kS + tid];
+            Wv[tid] = w;
+            Dr[tid] = dr;
+        }
+        // 7: the intra-chunk parts of dB and dC
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const int e = tid + kT * m, r = e / N, n = e % N;
+            float accb = 0.f, accc = 0.f;
+            for (int i = r; i < Qv; ++i) accb += LGX[i * kS + r] * Cs[i * NS + n];
+            for (int j = 0; j <= r && j < Qv; ++j) accc += LGX[r * kS + j] * dts[j] * Bs[j * NS + n];
+            dBa[m] += dts[r] * accb;
+            dCa[m] += accc;
+        }
+        __syncthreads();
+
+        // 8: d(dA): T[i][k] = sum_{j<k} M_ij, then column sums over i >= k
+        if (tid < kQ) {
+            float run = 0.f;
+            for (int k = 0; k <= tid; ++k) {
+                T[tid * kS + k] = run;
+                run += LGX[tid * kS + k] * CB[tid * kS + k] * dts[k];
+            }
+        }
+        __syncthreads();
+        const float F = ws.PF[(b * nc + c) * a.H + h];
+        float pdA = 0.f, pbias = 0.f, pD = 0.f;
+        if (tid < Qv) {
+            const int k = tid;
+            float R = 0.f, Es = 0.f, Wsum = 0.f;
+            for (int i = k; i < Qv; ++i) {
+                R += T[i * kS + k];
+                Es += Ev[i];
+            }
+            for (int j = 0; j < k; ++j) Wsum += dts[j] * Wv[j];
+            const float dda = R + Es + F + Wsum;
+            const float ddt = Dr[k] + Ah * dda;
+            const int64_t di = (b * a.L + t0 + k) * a.H + h;
+            const float dr = ddt * sigmoid_f(ld_act(a.dt, di, a.act_bf16) + bias);
+            a.ddt[di] = dr;
+            pdA = dts[k] * dda;
+            pbias = dr;
+        }
+        for (int e = tid; e < kQ * kP; e += kT) pD += gs[(e / kP) * kS + e % kP] * xs[(e / kP) * kS + e % kP];
+        const float sA = block_sum(pdA, red), sD = block_sum(pD, red + kT), sB = block_sum(pbias, red + 2 * kT);
+        if (tid == 0) {
+            float* ph = ws.PH + ((b * nc + c) * a.H + h) * 3;
+            ph[0] = sA;
+            ph[1] = sD;
+            ph[2] = sB;
+        }
+        __syncthreads();
+    }
+
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const int e = tid + kT * m, j = e / N, n = e % N;
+        if (j < Qv) {
+            const int64_t row = (b * a.L + t0 + j) * conv_dim;
+            ws.DU[row + HP + (int64_t)g * N + n] = dBa[m];
+            ws.DU[row + HP + GN + (int64_t)g * N + n] = dCa[m];
+        }
+    }
+}
+
+// grid (ceil(conv_dim / kT), ntiles, batch): one thread per (channel, 64-token tile).
+// Streams t over the tile and the 3 tokens after it: dv_t = du_t silu'(v_t), and the pre-conv
+// gradient of token s = t - 3 is w0 dv_t + w1 dv_{t-1} + w2 dv_{t-2} + w3 dv_{t-3}.
+__global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
+    const int64_t HP = (int64_t)a.H * a.P, GN = (int64_t)a.G * a.N, conv_dim = HP + 2 * GN;
+    const int64_t c = (int64_t)blockIdx.x * kT + threadIdx.x;
+    if (c >= conv_dim) return;
+    const int64_t b = blockIdx.z, tile = blockIdx.y, nt = ntiles(a.L), t0 = tile * kQ;
+    const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
+    const float w0 = a.conv_w[c * 4 + 0], w1 = a.conv_w[c * 4 + 1], w2 = a.conv_w[c * 4 + 2],
+                w3 = a.conv_w[c * 4 + 3], bias = a.conv_b[c];
+    float* out;
+    int64_t ostride, ocol;
+    if (c < HP) {
+        out = a.dx, ostride = HP, ocol = c;
+    } else if (c < HP + GN) {
+        out = a.dB, ostride = GN, ocol = c - HP;
+    } else {
+        out = a.dC, ostride = GN, ocol = c - HP - GN;
+    }
+    float r0 = raw_at(a, b, t0 - 3, c), r1 = raw_at(a, b, t0 - 2, c), r2 = raw_at(a, b, t0 - 1, c);
+    float d1 = 0.f, d2 = 0.f, d3 = 0.f;  // dv at t-1, t-2, t-3 (zero before token 0)
+    float gw0 = 0.f, gw1 = 0.f, gw2 = 0.f, gw3 = 0.f, gb = 0.f;
+    for (int64_t t = t0; t < t1 + 3; ++t) {
+        float dv = 0.f;
+        if (t < a.L) {
+            const float r3 = raw_at(a, b, t, c);
+            const float v = bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * r3;
+            dv = ws.DU[(b * a.L + t) * conv_dim + c] * dsilu_f(v);
+            if (t < t1) {
+                gw0 += dv * r0;
+                gw1 += dv * r1;
+                gw2 += dv * r2;
+                gw3 += dv * r3;
+                gb += dv;
+            }
+            r0 = r1;
+            r1 = r2;
+            r2 = r3;
+        }
+        const int64_t s = t - 3;
+        const float gs = w0 * dv + w1 * d1 + w2 * d2 + w3 * d3;
+        if (s >= t0 && s < t1) {
+            out[(b * a.L + s) * ostride + ocol] = gs;
+        } else if (s < 0 && a.d_init_conv_state) {
+            a.d_init_conv_state[(b * conv_dim + c) * 3 + (s + 3)] = gs;
+        }
+        d3 = d2;
+        d2 = d1;
+        d1 = dv;
+    }
+    float* pw = ws.PW + ((b * nt + tile) * conv_dim + c) * 5;
+    pw[0] = gw0;
+    pw[1] = gw1;
+    pw[2] = gw2;
+    pw[3] = gw3;
+    pw[4] = gb;
+}
+
+// grid ceil((conv_dim + H) / kT): per channel the conv parameter gradients, per head dA, dD, ddt_bias;
+// partials summed in (batch, tile) order.
+__global__ void __launch_bounds__(kT) reduce_kernel(BwdArgs a, Ws ws) {
+    const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N, nc = nchunks(a.L), nt = ntiles(a.L);
+    const int64_t idx = (int64_t)blockIdx.x * kT + threadIdx.x;
+    if (idx < conv_dim) {
+        float s[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int64_t b = 0; b < a.batch; ++b)
+            for (int64_t t = 0; t < nt; ++t) {
+                const float* pw = ws.PW + ((b * nt + t) * conv_dim + idx) * 5;
+                for (int k = 0; k < 5; ++k) s[k] += pw[k];
+            }
+        for (int k = 0; k < 4; ++k) a.dconv_w[idx * 4 + k] = s[k];
+        a.dconv_b[idx] = s[4];
+    } else if (idx < conv_dim + a.H) {
+        const int64_t h = idx - conv_dim;
+        float s[3] = {0.f, 0.f, 0.f};
+        for (int64_t b = 0; b < a.batch; ++b)
+            for (int64_t c = 0; c < nc; ++c) {
+                const float* ph = ws.PH + ((b * nc + c) * a.H + h) * 3;
+                for (int k = 0; k < 3; ++k) s[k] += ph[k];
+            }
+        a.dA[h] = s[0];
+        a.dD[h] = s[1];
+        a.ddt_bias[h] = s[2];
+    }
+}
+
+// grid ceil(batch * H * P * N / kT): d_init_state = d_final when there are no tokens.
+__global__ void __launch_bounds__(kT) copy_adjoint_kernel(BwdArgs a) {
+    const int64_t n = a.batch * a.H * (int64_t)a.P * a.N;
+    const int64_t i = (int64_t)blockIdx.x * kT + threadIdx.x;
+    if (i < n) a.d_init_state[i] = a.d_final ? a.d_final[i] : 0.f;
+}
+
+template <int N>
+cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
+    const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N, nc = nchunks(a.L), nt = ntiles(a.L);
+    const unsigned cgrid = static_cast<unsigned>((conv_dim + kT - 1) / kT);
+    cudaError_t err;
+    if (a.batch > 0 && nc > 0) {
+        const size_t state_smem = (2 * (size_t)kQ * kP + 2 * (size_t)kQ * N + 2 * kQ) * sizeof(float);
+        const size_t chunk_smem = chunk_bwd_floats<N>() * sizeof(float);
+        if ((err = SSD_SET_SMEM(chunk_state_kernel<N>, state_smem)) != cudaSuccess) return err;
+        if ((err = SSD_SET_SMEM(chunk_bwd_kernel<N>, chunk_smem)) != cudaSuccess) return err;
+        const dim3 tiles(cgrid, static_cast<unsigned>(nc), static_cast<unsigned>(a.batch));
+        SSD_LAUNCH(post_conv_kernel, tiles, dim3(kT), 0, st, a, ws);
+        SSD_LAUNCH(dt_kernel, dim3(static_cast<unsigned>((nc * a.H + kT - 1) / kT), static_cast<unsigned>(a.batch)),
+                   dim3(kT), 0, st, a, ws);
+        const dim3 chunk_heads(static_cast<unsigned>(nc), static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+        SSD_LAUNCH(chunk_state_kernel<N>, chunk_heads, dim3(kT), state_smem, st, a, ws);
+        SSD_LAUNCH(state_pass_kernel<N>, dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch)), dim3(kT),
+                   kT * sizeof(float), st, a, ws);
+        const dim3 chunk_groups(static_cast<unsigned>(nc), static_cast<unsigned>(a.G), static_cast<unsigned>(a.batch));
+#ifndef SSD_EMU
+        if (a.ev_before) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_before), st);
+#endif
+        SSD_LAUNCH(chunk_bwd_kernel<N>, chunk_groups, dim3(kT), chunk_smem, st, a, ws);
+#ifndef SSD_EMU
+        if (a.ev_after) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_after), st);
+#endif
+    } else if (a.batch > 0 && a.d_init_state) {
+        const int64_t n = a.batch * a.H * (int64_t)a.P * a.N;
+        SSD_LAUNCH(copy_adjoint_kernel, dim3(static_cast<unsigned>((n + kT - 1) / kT)), dim3(kT), 0, st, a);
+    }
+    if (a.batch > 0)
+        SSD_LAUNCH(conv_bwd_kernel, dim3(cgrid, static_cast<unsigned>(nt), static_cast<unsigned>(a.batch)), dim3(kT),
+                   0, st, a, ws);
+    SSD_LAUNCH(reduce_kernel, dim3(static_cast<unsigned>((conv_dim + a.H + kT - 1) / kT)), dim3(kT), 0, st, a, ws);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t workspace_bytes(int64_t batch, int64_t L, int H, int P, int N, int G) {
+    Ws ws;
+    return carve(batch, L, H, P, N, G, nullptr, &ws);
+}
+
+size_t chunk_bwd_smem_bytes(int N) {
+    switch (N) {
+        case 16: return chunk_bwd_floats<16>() * sizeof(float);
+        case 32: return chunk_bwd_floats<32>() * sizeof(float);
+        case 64: return chunk_bwd_floats<64>() * sizeof(float);
+        default: return chunk_bwd_floats<128>() * sizeof(float);
+    }
+}
+
+// Runs the backward on `st`.  Sizes, pointers and the workspace are validated by the caller
+// (P = 64, N in {16, 32, 64, 128}, H % G == 0, workspace >= workspace_bytes()).
+cudaError_t launch_prefill_backward(const BwdArgs& a, cudaStream_t st) {
+    Ws ws;
+    carve(a.batch, a.L, a.H, a.P, a.N, a.G, static_cast<char*>(a.workspace), &ws);
+    switch (a.N) {
+        case 16: return launch_n<16>(a, ws, st);
+        case 32: return launch_n<32>(a, ws, st);
+        case 64: return launch_n<64>(a, ws, st);
+        default: return launch_n<128>(a, ws, st);
+    }
+}
+
+}  // namespace bwd
+}  // namespace ssd

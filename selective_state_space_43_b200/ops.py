@@ -37,6 +37,11 @@ class SsdRowStrides(ctypes.Structure):
                 ("C", ctypes.c_int64)]
 
 
+class SsdGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dx", "ddt", "dB", "dC", "dz", "dA", "dD", "ddt_bias", "dconv_w",
+                                               "dconv_b", "d_init_state", "d_init_conv_state")]
+
+
 class SsdError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {STATUS.get(status, status)} ({lib().ssd_status_string(status).decode()})")
@@ -85,6 +90,11 @@ def lib() -> ctypes.CDLL:
                                         vp, vp, vp, vp]
         L.ssd_prefill_noalloc.restype = ctypes.c_int
         L.ssd_prefill_noalloc.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 10 + [vp]
+        L.ssd_prefill_backward_workspace_bytes.restype = sz
+        L.ssd_prefill_backward_workspace_bytes.argtypes = [dimp]
+        L.ssd_prefill_backward.restype = ctypes.c_int
+        L.ssd_prefill_backward.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 9 + [ctypes.POINTER(SsdGrads)] + [
+            vp, sz, vp]
         L.ssd_device_status.restype = ctypes.c_int
         L.ssd_device_status.argtypes = [vp]
         L.ssd_set_timing_events.restype = ctypes.c_int
@@ -228,6 +238,64 @@ def prefill(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=None, init
     if st != 0:
         raise SsdError(st, "ssd_prefill_strided" if strided else "ssd_prefill")
     return y, final_state, conv_state
+
+
+def prefill_backward_workspace_bytes(dims: SsdDims) -> int:
+    return int(lib().ssd_prefill_backward_workspace_bytes(ctypes.byref(dims)))
+
+
+def prefill_backward(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, dy, init_state=None, init_conv_state=None,
+                     d_final_state=None, want_init_grads=True, workspace=None, chunk=128):
+    """Gradients of ``prefill`` on the GPU (the training backward).
+
+    Inputs as for ``prefill`` (contiguous); dy [Bt, L, H*P] is the gradient of y (the activation dtype,
+    or fp32 with bf16 activations when y was fp32); d_final_state [Bt, H, P, N] fp32 or None.
+    Returns a dict of fp32 tensors keyed by the input they belong to: x, dt, B, C, z, A, D, dt_bias,
+    conv_w, conv_b, and (with ``want_init_grads``) init_state, init_conv_state -- the gradients of
+    sum(dy * y) + sum(d_final_state * final_state).
+    """
+    dev = x.device
+    Bt, L, HP = x.shape
+    H = A.shape[0]
+    P = HP // H
+    G, N = B.shape[2], B.shape[3]
+    act = x.dtype
+    conv_dim = HP + 2 * G * N
+    for name, t, shp in (("x", x, (Bt, L, HP)), ("z", z, (Bt, L, HP)), ("dt", dt, (Bt, L, H)),
+                         ("B", B, (Bt, L, G, N)), ("C", C, (Bt, L, G, N))):
+        _check(t, name, shp, act, dev)
+    _check(dy, "dy", (Bt, L, HP), dy.dtype, dev)
+    code = _dtype_code(x, dy.dtype)
+    if init_state is not None:
+        _check(init_state, "init_state", (Bt, H, P, N), torch.float32, dev)
+    if init_conv_state is not None:
+        _check(init_conv_state, "init_conv_state", (Bt, conv_dim, 3), act, dev)
+    if d_final_state is not None:
+        _check(d_final_state, "d_final_state", (Bt, H, P, N), torch.float32, dev)
+    params = _params(A, D, dt_bias, conv_w, conv_b, H, conv_dim, dev)
+    dims = make_dims(Bt, L, H, P, N, G, chunk)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"x": torch.empty((Bt, L, HP), **f32), "dt": torch.empty((Bt, L, H), **f32),
+           "B": torch.empty((Bt, L, G, N), **f32), "C": torch.empty((Bt, L, G, N), **f32),
+           "z": torch.empty((Bt, L, HP), **f32), "A": torch.empty(H, **f32), "D": torch.empty(H, **f32),
+           "dt_bias": torch.empty(H, **f32), "conv_w": torch.empty((conv_dim, 4), **f32),
+           "conv_b": torch.empty(conv_dim, **f32)}
+    if want_init_grads:
+        out["init_state"] = torch.empty((Bt, H, P, N), **f32)
+        out["init_conv_state"] = torch.empty((Bt, conv_dim, 3), **f32)
+    grads = SsdGrads(*[None if out.get(k) is None else out[k].data_ptr() for k in (
+        "x", "dt", "B", "C", "z", "A", "D", "dt_bias", "conv_w", "conv_b", "init_state", "init_conv_state")])
+    need = prefill_backward_workspace_bytes(dims)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().ssd_prefill_backward(ctypes.byref(dims), code, ctypes.byref(params), _ptr(x), _ptr(dt), _ptr(B),
+                                    _ptr(C), _ptr(z), _ptr(init_state), _ptr(init_conv_state), _ptr(dy),
+                                    _ptr(d_final_state), ctypes.byref(grads), _ptr(workspace), ws_bytes,
+                                    _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_prefill_backward")
+    return out
 
 
 def prefill_varlen_workspace_bytes(dims: SsdDims, dtype: torch.dtype) -> int:

@@ -202,3 +202,44 @@ def test_gated_rmsnorm_checks_arguments(L):
     assert f(4, 1024, 8, 1e-5, 1, None, 0x20000, 0x30000, None) == 1
     assert f(4, 1024, 8, 1e-5, 1, 0x10008, 0x20000, 0x30000, None) == 4
     assert f(0, 1024, 8, 1e-5, 1, None, None, None, None) == 0             # no rows: nothing to do
+
+
+def _call_backward(L, d, dtype=1, params=True, ptrs=None, grads=None, ws=None, ws_bytes=0):
+    p = ops.SsdParams(0x1000, 0x2000, 0x3000, 0x4000, 0x5000) if params is True else (params or None)
+    ptrs = ptrs or dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, init=None, init_conv=None,
+                        dy=0x60000, dfin=None)
+    g = ops.SsdGrads(*([0x100000 * (k + 1) for k in range(10)] + [None, None])) if grads is None else grads
+    return L.ssd_prefill_backward(ctypes.byref(d), dtype, ctypes.byref(p) if p else None, ptrs["x"], ptrs["dt"],
+                                  ptrs["B"], ptrs["C"], ptrs["z"], ptrs["init"], ptrs["init_conv"], ptrs["dy"],
+                                  ptrs["dfin"], ctypes.byref(g) if g is not False else None, ws, ws_bytes, None)
+
+
+def test_backward_rejects_bad_arguments_before_launch(L):
+    small = dims(seqlen=16, nheads=4, d_state=32, ngroups=1)
+    # post-conv channels and their gradients, dt and its cumsum, two chunk-state arrays and the partials
+    conv_dim = 4 * 64 + 2 * 32
+    assert L.ssd_prefill_backward_workspace_bytes(ctypes.byref(small)) >= 4 * (
+        2 * 16 * conv_dim + 2 * 4 * 16 + 2 * 1 * 4 * 64 * 32)
+    d = dims()
+    need = L.ssd_prefill_backward_workspace_bytes(ctypes.byref(d))
+    assert L.ssd_prefill_backward_workspace_bytes(ctypes.byref(dims(headdim=32))) == 0
+    assert L.ssd_prefill_backward(None, 1, None, *([None] * 9), None, None, 0, None) == 1
+    assert _call_backward(L, dims(headdim=32)) == 2
+    assert _call_backward(L, d, dtype=7) == 3
+    assert _call_backward(L, d, params=False) == 1
+    assert _call_backward(L, d, grads=False) == 1
+    base = dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, init=None, init_conv=None, dy=0x60000,
+                dfin=None)
+    assert _call_backward(L, d, ptrs={**base, "dy": None}) == 1
+    assert _call_backward(L, d, ptrs={**base, "z": 0x50004}) == 4
+    missing = ops.SsdGrads(*([0x100000 * (k + 1) for k in range(4)] + [None] + [0x600000] * 5 + [None, None]))
+    assert _call_backward(L, d, grads=missing) == 1                      # dz is required
+    odd = ops.SsdGrads(*([0x100000 * (k + 1) for k in range(10)] + [0x100008, None]))
+    assert _call_backward(L, d, grads=odd) == 4                          # d_init_state misaligned
+    assert _call_backward(L, d) == 7                                     # no workspace
+    assert _call_backward(L, d, ws=0x900000, ws_bytes=need - 1) == 7
+    assert _call_backward(L, dims(seqlen=64 * 65536)) == 2               # beyond the chunk grid
+    # zero tokens: the activations and per-token gradients may be NULL, the parameter gradients may not
+    none_act = {**base, "x": None, "dt": None, "B": None, "C": None, "z": None, "dy": None}
+    no_param = ops.SsdGrads(*([None] * 5 + [0x100000] * 4 + [None] + [None, None]))
+    assert _call_backward(L, dims(seqlen=0), ptrs=none_act, grads=no_param) == 1

@@ -61,3 +61,15 @@ def test_algorithmic_byte_and_flop_counts_match_the_survey_figures():
     dd = WORKLOADS["decode_nemotron_h_8b"]["dims"]
     total, _ = bench.decode_bytes(dd, 2)
     assert abs(total / 1e6 - 2192.6) < 0.1
+
+
+def test_backward_work_counts():
+    from selective_state_space_43_b200.synth import WORKLOADS
+    d = WORKLOADS["nemotron_h_8b"]["dims"]
+    # per token: x, z, dt, B, C and dy read as bf16, their fp32 gradients written; two fp32 states
+    per_token = (2 * 8192 + 128 + 2 * 1024) * 2 + 8192 * 2 + (2 * 8192 + 128 + 2 * 1024) * 4
+    assert bench.backward_bytes(d, 2) == 4096 * per_token + 2 * 128 * 64 * 128 * 4
+    # 64 chunks of 64 tokens; per head 8QPN + 4Q^2P + 2Q^2N, per group 2Q^2N
+    per_head = 8 * 64 * 64 * 128 + 4 * 64 * 64 * 64 + 2 * 64 * 64 * 128
+    assert bench.backward_chunk_flops(d) == 64 * (128 * per_head + 8 * 2 * 64 * 64 * 128)
+    assert abs(bench.FP32_ALU_TFLOPS - 74.45) < 0.01

@@ -1,0 +1,115 @@
+"""GPU parity of ssd_prefill_backward (the training backward) against the fp64 oracle's backward
+(needs a B200).  Every gradient the library returns is compared element by element.
+
+Tolerance, per gradient tensor: relative L2 error <= 5e-3 (the layer's parity bound) and max-abs
+error <= 2e-2 * max(1, max |reference|).  The max-abs bound is relative to the tensor's scale
+because the parameter gradients (dA, dD, ddt_bias, dconv_w, dconv_b) are sums over every token of
+the batch, with magnitudes up to 1e3 at the full workload; the backward accumulates in fp32 over
+64-token chunks and the chunk-to-chunk scans, so its error grows like fp32 rounding of those sums
+(about 1e-6 relative at the test sizes, measured on the same source through the host emulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import dev_inputs, np64
+from selective_state_space_43_b200 import ops
+from selective_state_space_43_b200.synth import WORKLOADS, Dims, make_backward_grads, make_prefill_inputs, seed_of
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 5e-3
+MAX_ABS_SCALED = 2e-2
+
+
+def gpu_backward(dev, dy, d_final, want_init=True):
+    return ops.prefill_backward(dev["x"], dev["dt"], dev["B"], dev["C"], dev["z"], dev["A"], dev["D"],
+                                dev["dt_bias"], dev["conv_w"], dev["conv_b"], dy, dev.get("init_state"),
+                                dev.get("init_conv_state"), d_final, want_init_grads=want_init)
+
+
+def compare(got, want, tag):
+    for k, ref in want.items():
+        if k not in got:
+            continue
+        g = np64(got[k])
+        assert g.shape == ref.shape, (tag, k)
+        if ref.size == 0:
+            continue
+        assert np.isfinite(g).all(), f"{tag} d{k}: non-finite values"
+        rel = float(np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30))
+        mx = float(np.max(np.abs(g - ref)))
+        bound = MAX_ABS_SCALED * max(1.0, float(np.max(np.abs(ref))))
+        assert rel <= REL_L2 and mx <= bound, f"{tag} d{k}: rel-L2 {rel:.3e}, max-abs {mx:.3e} (<= {bound:.3e})"
+
+
+def run_case(d, dtype, init, dfin, seed, dy_dtype=None):
+    inp = make_prefill_inputs(d, dtype=dtype, seed=seed, init_state=init, init_conv_state=init, random_D=True)
+    gr = make_backward_grads(d, dtype=dy_dtype or dtype, seed=seed + 1, d_final=dfin)
+    dev = dev_inputs(inp)
+    dy = gr["dy"].cuda()
+    df = None if gr["d_final"] is None else gr["d_final"].cuda()
+    got = gpu_backward(dev, dy, df)
+    torch.cuda.synchronize()
+    want = oracle.prefill_backward(inp, gr["dy"], gr["d_final"])
+    return got, want
+
+
+CASES = [
+    # batch, L, H, G, N, dtype, init states, d_final
+    (2, 300, 8, 2, 64, torch.bfloat16, True, True),     # ragged last chunk, 4 heads per group
+    (1, 129, 4, 4, 32, torch.float32, False, False),    # 1-token last chunk, zero states
+    (1, 512, 16, 2, 128, torch.bfloat16, True, True),   # the production d_state, 8 chunks
+    (3, 64, 2, 1, 16, torch.float32, True, True),       # exactly one chunk per sequence
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}L{c[1]}H{c[2]}G{c[3]}N{c[4]}")
+def test_backward_matches_oracle(case):
+    Bt, L, H, G, N, dtype, init, dfin = case
+    got, want = run_case(Dims(Bt, L, H, 64, N, G, 128), dtype, init, dfin, seed=7 * L + N)
+    compare(got, want, f"B{Bt} L{L} H{H} G{G} N{N}")
+
+
+def test_backward_fp32_dy_with_bf16_activations():
+    got, want = run_case(Dims(1, 200, 4, 64, 64, 2, 128), torch.bfloat16, True, True, seed=21,
+                         dy_dtype=torch.float32)
+    compare(got, want, "bf16 activations, fp32 dy")
+
+
+def test_backward_full_nemotron_h_8b_layer():
+    # the benchmark workload: B1 L4096 H128 P64 N128 G8, bf16, every gradient element compared
+    w = WORKLOADS["nemotron_h_8b"]
+    got, want = run_case(w["dims"], torch.bfloat16, False, True, seed=seed_of("nemotron_h_8b"))
+    compare(got, want, "nemotron_h_8b")
+
+
+def test_backward_is_deterministic():
+    d = Dims(2, 200, 8, 64, 128, 2, 128)
+    inp = make_prefill_inputs(d, dtype=torch.bfloat16, seed=3, init_state=True, init_conv_state=True)
+    gr = make_backward_grads(d, seed=4)
+    dev = dev_inputs(inp)
+    a = gpu_backward(dev, gr["dy"].cuda(), gr["d_final"].cuda())
+    b = gpu_backward(dev, gr["dy"].cuda(), gr["d_final"].cuda())
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("L", [0, 2])
+def test_backward_short_and_empty_sequences(L):
+    d = Dims(2, L, 4, 64, 32, 2, 128)
+    got, want = run_case(d, torch.float32, True, True, seed=30 + L)
+    compare(got, want, f"L{L}")
+    if L == 0:
+        assert torch.equal(got["init_state"].cpu(), make_backward_grads(d, dtype=torch.float32, seed=31)["d_final"])
+        assert not got["conv_w"].any() and not got["init_conv_state"].any()
+
+
+def test_backward_without_initial_state_gradients():
+    d = Dims(1, 100, 4, 64, 32, 1, 128)
+    inp = make_prefill_inputs(d, dtype=torch.bfloat16, seed=5)
+    gr = make_backward_grads(d, seed=6, d_final=False)
+    got = gpu_backward(dev_inputs(inp), gr["dy"].cuda(), None, want_init=False)
+    assert "init_state" not in got and "init_conv_state" not in got
+    compare(got, oracle.prefill_backward(inp, gr["dy"], None), "no initial-state gradients")
