@@ -43,6 +43,8 @@ def _bind(lib):
     lib.oracle_prefill.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 12 + [ctypes.c_void_p] + [dp] * 3 + [
         ctypes.c_int]
     lib.oracle_decode_step.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 12 + [ctypes.c_void_p, dp]
+    if hasattr(lib, "oracle_mimo_decode_step"):
+        lib.oracle_mimo_decode_step.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int] + [dp] * 10
     if hasattr(lib, "oracle_prefill_backward"):
         lib.oracle_prefill_backward.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 26 + [ctypes.c_int]
     return lib
@@ -212,6 +214,24 @@ def prefill_backward(inp: dict, dy, d_final=None, nthreads: int | None = None):
     _load().oracle_prefill_backward(ctypes.byref(d), *[_ptr(a) for a in arrs], *[_ptr(out[k]) for k in order],
                                     int(nthreads or default_threads()))
     return out
+
+
+def mimo_decode_step(step: dict, params: dict, ssm_state):
+    """One fp64 MIMO decode step (Mamba-3's multi-input multi-output SSM on the Mamba-2 scalar decay, no
+    short conv; "Mamba-3: 추론을 우선한 상태 공간 모델", opening section and 아키텍처).  step holds x, z
+    [Bt, H, R, P], dt [Bt, H], B, C [Bt, G, R, N]; params A, D, dt_bias [H].  ``ssm_state`` (float64
+    [Bt, H, P, N], C-contiguous) is updated in place.  Returns y [Bt, H, R, P]."""
+    assert ssm_state.dtype == np.float64 and ssm_state.flags.c_contiguous
+    x = _f64(step["x"])
+    Bt, H, R, P = x.shape
+    Bm = _f64(step["B"])
+    G, N = Bm.shape[1], Bm.shape[3]
+    d = _dims(Bt, 1, H, P, N, G)
+    y = np.empty((Bt, H, R, P))
+    arrs = [x, _f64(step["dt"]), Bm, _f64(step["C"]), _f64(step["z"]), _f64(params["A"]), _f64(params["D"]),
+            _f64(params["dt_bias"]), ssm_state, y]
+    _load().oracle_mimo_decode_step(ctypes.byref(d), int(R), *[_ptr(a) for a in arrs])
+    return y
 
 
 def gated_rmsnorm(y, weight, ngroups: int, eps: float = 1e-5):

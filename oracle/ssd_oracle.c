@@ -610,3 +610,55 @@ void oracle_prefill_backward(const oracle_dims* d, const double* x, const double
     }
     free(jobs); free(th); free(pdA); free(pdD); free(pddt_bias); free(pdconv_w); free(pdconv_b);
 }
+
+/* ===========================================================================
+ * MIMO decode step (Mamba-3's multi-input multi-output SSM).
+ *
+ * "Mamba-3: 추론을 우선한 상태 공간 모델" (opening section, third change; 아키텍처:
+ * the MIMO projection widens B and C) replaces the single-input single-output
+ * SSM by several SSMs modelled in parallel, at almost no cost to decode
+ * latency.  The page gives no equations; the plainest reading, kept on the
+ * Mamba-2 scalar decay (the new discretisation and complex states are other
+ * changes), is a rank-R input and R read-outs per head:
+ *
+ *   dt = softplus(dt_raw + dt_bias[h]),  a = exp(dt A[h])
+ *   S[h] <- a S[h] + dt sum_{k<R} x_k[h] (outer) B_k[g]
+ *   y_k[h] = (S[h] C_k[g] + D[h] x_k[h]) silu(z_k[h])        k = 0..R-1
+ *
+ * with no short conv (the same page: Mamba-3 drops it).  R = 1 is the Mamba-2
+ * decode step without its conv.
+ * Layouts: x, z, y [Bt][H][R][P]; dt_raw [Bt][H]; Bm, Cm [Bt][G][R][N];
+ * state [Bt][H][P][N] (in/out).
+ * ------------------------------------------------------------------------- */
+void oracle_mimo_decode_step(const oracle_dims* d, int R, const double* x, const double* dt_raw,
+                             const double* Bm, const double* Cm, const double* z, const double* A,
+                             const double* D, const double* dt_bias, double* state, double* y) {
+    const int H = d->nheads, P = d->headdim, N = d->d_state, G = d->ngroups;
+    for (long b = 0; b < d->batch; b++) {
+        for (int h = 0; h < H; h++) {
+            const int g = h / (H / G);
+            const double dt = o_softplus(dt_raw[(size_t)b * H + h] + dt_bias[h]);
+            const double a = exp(dt * A[h]);
+            double* S = state + ((size_t)b * H + h) * P * N;
+            const double* xh = x + ((size_t)b * H + h) * R * P;
+            const double* zh = z + ((size_t)b * H + h) * R * P;
+            const double* Bg = Bm + ((size_t)b * G + g) * R * N;
+            const double* Cg = Cm + ((size_t)b * G + g) * R * N;
+            for (int p = 0; p < P; p++) {
+                for (int n = 0; n < N; n++) {
+                    double in = 0.0;
+                    for (int k = 0; k < R; k++) in += xh[k * P + p] * Bg[k * N + n];
+                    S[(size_t)p * N + n] = a * S[(size_t)p * N + n] + dt * in;
+                }
+            }
+            for (int k = 0; k < R; k++) {
+                for (int p = 0; p < P; p++) {
+                    double acc = 0.0;
+                    for (int n = 0; n < N; n++) acc += S[(size_t)p * N + n] * Cg[k * N + n];
+                    const double yv = acc + D[h] * xh[k * P + p];
+                    y[(((size_t)b * H + h) * R + k) * P + p] = yv * o_silu(zh[k * P + p]);
+                }
+            }
+        }
+    }
+}

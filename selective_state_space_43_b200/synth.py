@@ -168,6 +168,27 @@ def make_decode_inputs(dims: Dims, steps: int, dtype=torch.bfloat16, seed: int =
     return dict(params=params, ssm_state=ssm_state, conv_state=conv_state, steps=per_step)
 
 
+def make_mimo_decode_inputs(dims: Dims, rank: int, steps: int, dtype=torch.bfloat16, seed: int = 59,
+                            random_D: bool = False) -> dict:
+    """Initial state and ``steps`` rounds of one-token inputs for the rank-``rank`` MIMO decode: x, z
+    [B, H, R, P] ~ N(0, 1), dt [B, H] ~ N(0, 1), B, C [B, G, R, N] ~ N(0, 1)/sqrt(N), rounded to ``dtype``;
+    fp32 state ~ N(0, 0.1^2); A, D, dt_bias as for the other workloads (the conv parameters are drawn too,
+    so the draw order matches, but the MIMO step has no conv)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    Bt, H, P, N, G = dims.batch, dims.nheads, dims.headdim, dims.d_state, dims.ngroups
+    params = make_params(dims, g, random_D=random_D)
+    ssm_state = torch.randn((Bt, H, P, N), generator=g) * 0.1
+    per_step = []
+    for _ in range(steps):
+        x = torch.randn((Bt, H, rank, P), generator=g)
+        z = torch.randn((Bt, H, rank, P), generator=g)
+        dt = torch.randn((Bt, H), generator=g)
+        Bm = torch.randn((Bt, G, rank, N), generator=g) / math.sqrt(N)
+        Cm = torch.randn((Bt, G, rank, N), generator=g) / math.sqrt(N)
+        per_step.append(dict(x=x.to(dtype), z=z.to(dtype), dt=dt.to(dtype), B=Bm.to(dtype), C=Cm.to(dtype)))
+    return dict(params=params, ssm_state=ssm_state, steps=per_step)
+
+
 def workload(name: str, **overrides):
     """(dims, dtype, inputs) for one of the named workloads."""
     w = WORKLOADS[name]

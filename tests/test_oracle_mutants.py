@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 import test_oracle_backward_pins as bpins
+import test_oracle_mimo_pins as mpins
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssd_oracle.c")
@@ -60,6 +61,19 @@ BACKWARD_MUTANTS = {
     "checkpoint off by one": ("if (t % RECOMP_SEG == 0) memcpy(", "if (t % RECOMP_SEG == 1) memcpy("),
 }
 
+# mistakes in the MIMO decode step
+MIMO_MUTANTS = {
+    "MIMO input from slot 0's B": ("in += xh[k * P + p] * Bg[k * N + n];", "in += xh[k * P + p] * Bg[n];"),
+    "MIMO read-out from slot 0's C": ("acc += S[(size_t)p * N + n] * Cg[k * N + n];",
+                                      "acc += S[(size_t)p * N + n] * Cg[n];"),
+    "MIMO D skip from slot 0": ("const double yv = acc + D[h] * xh[k * P + p];", "const double yv = acc + D[h] * xh[p];"),
+    "MIMO gate from slot 0": ("yv * o_silu(zh[k * P + p]);", "yv * o_silu(zh[p]);"),
+    "MIMO input not scaled by dt": ("S[(size_t)p * N + n] = a * S[(size_t)p * N + n] + dt * in;",
+                                    "S[(size_t)p * N + n] = a * S[(size_t)p * N + n] + in;"),
+    "MIMO decay squared": ("S[(size_t)p * N + n] = a * S[(size_t)p * N + n] + dt * in;",
+                           "S[(size_t)p * N + n] = a * a * S[(size_t)p * N + n] + dt * in;"),
+}
+
 PINS = [
     lambda: pins.test_conv_silu_matches_library_fir(True),
     lambda: pins.test_prefill_matches_quadratic_form(1, True),
@@ -105,7 +119,7 @@ def test_unmutated_copy_passes_every_pin():
         so = _compile(open(SRC).read(), tmp, "clean")
         oracle.use_library(so)
         try:
-            for pin in PINS + BACKWARD_PINS:
+            for pin in PINS + BACKWARD_PINS + MIMO_PINS:
                 pin()
         finally:
             oracle.use_library(None)
@@ -129,6 +143,33 @@ def test_planted_backward_mistake_is_caught(name):
         try:
             failed = 0
             for pin in BACKWARD_PINS:
+                try:
+                    pin()
+                except AssertionError:
+                    failed += 1
+            assert failed > 0, f"no pin caught the planted mistake '{name}'"
+        finally:
+            oracle.use_library(None)
+
+
+MIMO_PINS = [
+    lambda: mpins.test_closed_form_over_steps(2),
+    lambda: mpins.test_rank_one_is_the_mamba2_decode_without_conv(),
+    lambda: mpins.test_slot_permutation(),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MIMO_MUTANTS))
+def test_planted_mimo_mistake_is_caught(name):
+    src = open(SRC).read()
+    old, new = MIMO_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for '{name}' not unique"
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _compile(src.replace(old, new), tmp, "mutant")
+        oracle.use_library(so)
+        try:
+            failed = 0
+            for pin in MIMO_PINS:
                 try:
                     pin()
                 except AssertionError:
