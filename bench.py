@@ -39,8 +39,8 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from selective_state_space_43_b200.synth import (Dims, WORKLOADS, make_backward_grads,  # noqa: E402
-                                                 make_decode_inputs, make_prefill_inputs, make_varlen_inputs,
-                                                 seed_of, varlen_lengths)
+                                                 make_decode_inputs, make_mimo_decode_inputs, make_prefill_inputs,
+                                                 make_varlen_inputs, seed_of, varlen_lengths)
 
 METRIC = "SSD prefill tokens/s per layer (% bf16 TC peak); decode GB/s (% of HBM peak)"
 PREFILL_WORKLOAD = "nemotron_h_8b"
@@ -53,6 +53,8 @@ VARLEN_NSEQ, VARLEN_MIN, VARLEN_MAX = 32, 64, 4096
 # per FMA x the 1965 MHz maximum SM clock
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 BWD_Q = 64  # the backward's chunk length
+MIMO_RANK = 4     # rank of the MIMO decode line (the pages give no rank; 4 = a few SSMs per head)
+MIMO_INPUTS = 4   # distinct step inputs the MIMO decode line cycles through
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -169,6 +171,56 @@ def decode_bytes(d: Dims, act_bytes: int) -> tuple[int, int]:
     roll = B * 2 * d.ngroups * d.d_state * (3 + 3) * act_bytes     # B/C conv window rewritten by the roll kernel
     total = state + conv + inputs + y
     return total, total - roll
+
+
+def mimo_decode_bytes(d: Dims, rank: int, act_bytes: int) -> int:
+    """Bytes of one MIMO decode step: the fp32 state read and written, x, z, B, C, dt read, y written."""
+    B = d.batch
+    state = 2 * B * d.nheads * d.headdim * d.d_state * 4
+    xzy = 3 * B * d.nheads * rank * d.headdim * act_bytes
+    bc = 2 * B * d.ngroups * rank * d.d_state * act_bytes
+    return state + xzy + bc + B * d.nheads * act_bytes
+
+
+def bench_mimo(ops, d: Dims, act, dev, world: int, sampler, peaks, nsteps: int):
+    """Times ssd_mimo_decode_step (rank MIMO_RANK) on the decode workload's layer and batch."""
+    data = make_mimo_decode_inputs(d, MIMO_RANK, MIMO_INPUTS, dtype=act, seed=seed_of(DECODE_WORKLOAD) + 5)
+    p = {k: v.to(dev) for k, v in data["params"].items()}
+    ssm = data["ssm_state"].to(dev)
+    steps = [{k: v.to(dev) for k, v in s.items()} for s in data["steps"]]
+    ys = [torch.empty_like(s["x"]) for s in steps]
+    del data
+
+    def mstep(i):
+        s = steps[i % len(steps)]
+        ops.mimo_decode_step(s["x"], s["dt"], s["B"], s["C"], s["z"], p["A"], p["D"], p["dt_bias"], ssm,
+                             y=ys[i % len(steps)])
+    for i in range(3):
+        mstep(i)
+    torch.cuda.synchronize(dev)
+    ms_ = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+    me = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+    barrier(world)
+    sampler.load(True)
+    for k in range(nsteps):
+        ms_[k].record()
+        mstep(k)
+        me[k].record()
+    torch.cuda.synchronize(dev)
+    sampler.load(False)
+    barrier(world)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(ms_, me)) / nsteps, world, dev)
+    nbytes = mimo_decode_bytes(d, MIMO_RANK, 2 if act == torch.bfloat16 else 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    flops = 4 * MIMO_RANK * d.batch * d.nheads * d.headdim * d.d_state
+    return {"value": gbs * world, "unit": "GB/s", "ms_per_step": ms, "steps": nsteps, "rank": MIMO_RANK,
+            "workload": f"MIMO decode step, rank {MIMO_RANK}, on the {DECODE_WORKLOAD} layer and batch "
+                        f"({d.batch} sequences, H{d.nheads} P{d.headdim} N{d.d_state} G{d.ngroups}), bf16 "
+                        "activations, fp32 state, no conv",
+            "algorithmic_bytes_per_step": nbytes, "algorithmic_flops_per_step": flops,
+            "roofline": {"bound": "hbm", "kernel": "mimo_decode_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None},
+            "l2": "state (1.07 GB) larger than L2; no flush"}
 
 
 # ---------------------------------------------------------------------------------------------------------
@@ -373,6 +425,7 @@ def main():
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed variable-length prefill line")
     ap.add_argument("--no-norm", action="store_true", help="skip the gated RMSNorm line")
     ap.add_argument("--no-backward", action="store_true", help="skip the training-backward line")
+    ap.add_argument("--no-mimo", action="store_true", help="skip the MIMO decode line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -652,6 +705,15 @@ def main():
         except (RuntimeError, ValueError) as exc:  # report it and keep the forward numbers
             backward = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
+    # ---- MIMO decode step on the decode workload ------------------------------------------------------------
+    mimo = None
+    if not args.no_mimo:
+        try:
+            wd = WORKLOADS[DECODE_WORKLOAD]
+            mimo = bench_mimo(ops, wd["dims"], wd["dtype"], dev, world, sampler, peaks, max(3, min(K, 16)))
+        except (RuntimeError, ValueError) as exc:  # report it and keep the other numbers
+            mimo = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     clocks = sampler.stop()
 
     # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------------------------------------
@@ -672,6 +734,7 @@ def main():
                        "kernel_path": "tcgen05 tensor-core" if path == 1 else "CUDA-core", "launch": launch},
             "tensor": tc, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
             "varlen": varlen, "gated_rmsnorm": norm, "backward": backward,
+            "mimo_decode": mimo,
             "gpu_launches": K * (2 if path == 1 else 1), "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -6,6 +6,7 @@
 #include "ssd_backward.h"
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_mimo.h"
 
 namespace {
 
@@ -274,6 +275,35 @@ ssd_status ssd_prefill_backward(const ssd_dims* d, ssd_dtype dtype, const ssd_pa
     a.ev_before = g_hook.ev_before;
     a.ev_after = g_hook.ev_after;
     cudaError_t e = ssd::bwd::launch_prefill_backward(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_mimo_decode_step(const ssd_dims* d, int32_t rank, ssd_dtype dtype, const ssd_params* params,
+                                const void* x, const void* dt, const void* B, const void* C, const void* z,
+                                float* ssm_state, void* y, void* stream) {
+    ssd_status st = check_dims(d, dtype, false);
+    if (st != SSD_OK) return st;
+    if (!(rank == 1 || rank == 2 || rank == 4 || rank == 8)) return SSD_ERR_SHAPE;
+    if (!params || !params->A || !params->D || !params->dt_bias) return SSD_ERR_NULL;
+    if (!aligned16(params->A) || !aligned16(params->D) || !aligned16(params->dt_bias)) return SSD_ERR_ALIGN;
+    if (!x || !dt || !B || !C || !z || !ssm_state || !y) return SSD_ERR_NULL;
+    const void* ptrs[] = {x, dt, B, C, z, ssm_state, y};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return SSD_ERR_ALIGN;
+    if (y == x || y == z) return SSD_ERR_UNSUPPORTED;
+    if (d->batch == 0) return SSD_OK;
+    ssd::mimo::MimoArgs a{};
+    a.batch = d->batch;
+    a.H = d->nheads; a.P = d->headdim; a.N = d->d_state; a.G = d->ngroups; a.R = rank;
+    a.act_bf16 = dtype != SSD_F32;
+    a.y_bf16 = dtype == SSD_BF16;
+    a.A = params->A; a.D = params->D; a.dt_bias = params->dt_bias;
+    a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z;
+    a.ssm_state = ssm_state;
+    a.y = y;
+    a.ev_before = g_hook.ev_before;
+    a.ev_after = g_hook.ev_after;
+    cudaError_t e = ssd::mimo::launch_mimo_decode(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

@@ -81,6 +81,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
 // Synchronises `st`, then reads and clears the tensor-core kernel's timeout flag.
 cudaError_t read_and_clear_tc_error(int* flag, cudaStream_t st);
 
+namespace mimo {
+struct MimoArgs;
+// The MIMO decode step (ssd_mimo.cu); sizes and pointers validated by the caller.
+cudaError_t launch_mimo_decode(const MimoArgs& a, cudaStream_t st);
+}  // namespace mimo
+
 namespace bwd {
 struct BwdArgs;
 // The prefill backward (ssd_backward.cu); sizes and pointers validated by the caller.

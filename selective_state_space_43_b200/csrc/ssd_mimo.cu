@@ -1,0 +1,173 @@
+// ssd_mimo.cu -- one decode token of the multi-input multi-output (MIMO) SSM for a batch.
+//
+// "Mamba-3: 추론을 우선한 상태 공간 모델" (opening section, third change; 아키텍처: the MIMO
+// projection widens B and C) models several SSMs in parallel per head instead of one, at almost
+// no cost to decode latency.  Read here on the Mamba-2 scalar decay, with no short conv (the
+// same page drops it):
+//   dt = softplus(dt_raw + dt_bias[h]),  a = exp(dt A[h])
+//   S  <- a S + dt sum_{k<R} x_k (outer) B_k           (a rank-R update of the P x N state)
+//   y_k = (S C_k + D x_k) silu(z_k),   k < R
+// The state is still read once and written once, now with 2R FMAs per element instead of 2, so
+// the step stays bound by HBM bandwidth for R <= 8 (at most 4 flops per state byte against a
+// B200 fp32/HBM ridge of about 11): this is why MIMO leaves decode latency nearly unchanged.
+//
+// Design (as the Mamba-2 decode kernel): one 256-thread CTA per (sequence, head); the P x N fp32
+// state streamed with 16-byte vectors, every load of the CTA issued before the first FMA; a row
+// of N floats covered by N/4 lanes; the R read-outs are segmented warp reductions over those
+// lanes; x, B, C and y of the head staged in shared memory.
+//
+// SSD_EMU: compiled as plain C++ by the tests' host emulation (one thread per CUDA thread, real
+// barriers for __syncthreads and the warp shuffles) under AddressSanitizer; the library is
+// always built with nvcc.
+#ifdef SSD_EMU
+#include "emu_cuda.h"
+#define SSD_LAUNCH(kern, grid, block, smem, st, ...) \
+    ((void)(st), ::emu::launch((grid), (block), (smem), [&]() { kern(__VA_ARGS__); }))
+#define SSD_DYN_SMEM() (::emu::smem())
+#else
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#define SSD_LAUNCH(kern, grid, block, smem, st, ...) kern<<<(grid), (block), (smem), (st)>>>(__VA_ARGS__)
+extern __shared__ __align__(16) unsigned char ssd_mimo_smem[];
+#define SSD_DYN_SMEM() (ssd_mimo_smem)
+#endif
+
+#include "ssd_mimo.h"
+
+namespace ssd {
+namespace mimo {
+namespace {
+
+constexpr int kT = 256;
+constexpr int kP = 64;
+#define COMMA ,
+
+__device__ __forceinline__ float ld_act(const void* p, int64_t i, bool bf16) {
+    if (bf16) return __uint_as_float(static_cast<unsigned>(static_cast<const unsigned short*>(p)[i]) << 16);
+    return static_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ void st_out(void* p, int64_t i, float v, bool bf16) {
+    if (bf16)
+        static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+    else
+        static_cast<float*>(p)[i] = v;
+}
+__device__ __forceinline__ float silu_f(float v) { return v / (1.f + __expf(-v)); }
+__device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(__expf(v)); }
+
+// grid batch * H, kT threads.
+template <int R, int N>
+__global__ void __launch_bounds__(kT) mimo_decode_kernel(MimoArgs a) {
+    constexpr int LPR = N / 4;            // lanes per state row (a float4 each)
+    constexpr int RPW = 32 / LPR;         // rows per warp per pass
+    constexpr int ITER = kP / (8 * RPW);  // passes over the P rows with 8 warps
+    float* s_x = reinterpret_cast<float*>(SSD_DYN_SMEM());  // [R][P]
+    float* s_B = s_x + R * kP;                               // [R][N]
+    float* s_C = s_B + R * N;                                // [R][N]
+    float* s_y = s_C + R * N;                                // [R][P]
+
+    const int64_t bh = blockIdx.x;
+    const int64_t b = bh / a.H;
+    const int h = static_cast<int>(bh - b * a.H);
+    const int g = h / (a.H / a.G);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rsub = lane / LPR, n0 = (lane % LPR) * 4;
+
+    // the state loads first: they are the step's traffic
+    float4* S = reinterpret_cast<float4*>(a.ssm_state + bh * kP * N);
+    float4 v[ITER];
+#pragma unroll
+    for (int it = 0; it < ITER; ++it) {
+        const int p = (it * 8 + warp) * RPW + rsub;
+        v[it] = __ldcs(S + ((p * N + n0) >> 2));
+    }
+    const int64_t xo = bh * R * kP, bo = (b * a.G + g) * R * N;
+    for (int i = tid; i < R * kP; i += kT) s_x[i] = ld_act(a.x, xo + i, a.act_bf16);
+    for (int i = tid; i < R * N; i += kT) {
+        s_B[i] = ld_act(a.B, bo + i, a.act_bf16);
+        s_C[i] = ld_act(a.C, bo + i, a.act_bf16);
+    }
+    const float dtv = softplus_f(ld_act(a.dt, bh, a.act_bf16) + a.dt_bias[h]);
+    const float decay = __expf(dtv * a.A[h]);
+    __syncthreads();
+
+    float4 bq[R], cq[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+        bq[k] = make_float4(s_B[k * N + n0], s_B[k * N + n0 + 1], s_B[k * N + n0 + 2], s_B[k * N + n0 + 3]);
+        cq[k] = make_float4(s_C[k * N + n0], s_C[k * N + n0 + 1], s_C[k * N + n0 + 2], s_C[k * N + n0 + 3]);
+    }
+#pragma unroll
+    for (int it = 0; it < ITER; ++it) {
+        const int p = (it * 8 + warp) * RPW + rsub;
+        float ix = 0.f, iy = 0.f, iz = 0.f, iw = 0.f;
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const float xk = s_x[k * kP + p];
+            ix += xk * bq[k].x;
+            iy += xk * bq[k].y;
+            iz += xk * bq[k].z;
+            iw += xk * bq[k].w;
+        }
+        float4 s = v[it];
+        s.x = fmaf(decay, s.x, dtv * ix);
+        s.y = fmaf(decay, s.y, dtv * iy);
+        s.z = fmaf(decay, s.z, dtv * iz);
+        s.w = fmaf(decay, s.w, dtv * iw);
+        __stcs(S + ((p * N + n0) >> 2), s);
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            float part = s.x * cq[k].x + s.y * cq[k].y + s.z * cq[k].z + s.w * cq[k].w;
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if ((lane % LPR) == 0) s_y[k * kP + p] = part;
+        }
+    }
+    __syncthreads();
+    const float Dh = a.D[h];
+    for (int i = tid; i < R * kP; i += kT) {
+        const float yv = s_y[i] + Dh * s_x[i];
+        st_out(a.y, xo + i, yv * silu_f(ld_act(a.z, xo + i, a.act_bf16)), a.y_bf16);
+    }
+}
+
+template <int R, int N>
+void launch_rn(const MimoArgs& a, cudaStream_t st) {
+    const dim3 grid(static_cast<unsigned>(a.batch * a.H));
+    SSD_LAUNCH(mimo_decode_kernel<R COMMA N>, grid, dim3(kT), smem_bytes(R, kP, N), st, a);
+}
+
+template <int R>
+cudaError_t launch_r(const MimoArgs& a, cudaStream_t st) {
+    switch (a.N) {
+        case 16: launch_rn<R, 16>(a, st); break;
+        case 32: launch_rn<R, 32>(a, st); break;
+        case 64: launch_rn<R, 64>(a, st); break;
+        default: launch_rn<R, 128>(a, st); break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Runs the step on `st`.  Validated by the caller: P = 64, N in {16, 32, 64, 128}, R in {1, 2, 4, 8},
+// H % G == 0, batch * H >= 1 and below 2^31.
+cudaError_t launch_mimo_decode(const MimoArgs& a, cudaStream_t st) {
+#ifndef SSD_EMU
+    if (a.ev_before) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_before), st);
+#endif
+    cudaError_t e;
+    switch (a.R) {
+        case 1: e = launch_r<1>(a, st); break;
+        case 2: e = launch_r<2>(a, st); break;
+        case 4: e = launch_r<4>(a, st); break;
+        default: e = launch_r<8>(a, st); break;
+    }
+#ifndef SSD_EMU
+    if (a.ev_after) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_after), st);
+#endif
+    return e;
+}
+
+}  // namespace mimo
+}  // namespace ssd

@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_backward.restype = ctypes.c_int
         L.ssd_prefill_backward.argtypes = [dimp, ctypes.c_int, parp] + [vp] * 9 + [ctypes.POINTER(SsdGrads)] + [
             vp, sz, vp]
+        L.ssd_mimo_decode_step.restype = ctypes.c_int
+        L.ssd_mimo_decode_step.argtypes = [dimp, ctypes.c_int32, ctypes.c_int, parp] + [vp] * 7 + [vp]
         L.ssd_device_status.restype = ctypes.c_int
         L.ssd_device_status.argtypes = [vp]
         L.ssd_set_timing_events.restype = ctypes.c_int
@@ -507,6 +509,34 @@ def prefill_noalloc(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, init_state=No
     if st != 0:
         raise SsdError(st, "ssd_prefill_noalloc")
     return y, final_state, conv_state
+
+
+def mimo_decode_step(x, dt, B, C, z, A, D, dt_bias, ssm_state, y=None, y_dtype=None):
+    """One MIMO decode step on the GPU (rank R = x.shape[2]; see include/ssd.h).  x, z [Bt, H, R, P];
+    dt [Bt, H]; B, C [Bt, G, R, N] (bf16 or fp32, one dtype); A, D, dt_bias [H] fp32; ssm_state
+    [Bt, H, P, N] fp32, updated in place.  Returns y [Bt, H, R, P] (the activation dtype, or y_dtype)."""
+    dev = x.device
+    Bt, H, R, P = x.shape
+    G, N = B.shape[1], B.shape[3]
+    act = x.dtype
+    for name, t, shp in (("x", x, (Bt, H, R, P)), ("z", z, (Bt, H, R, P)), ("dt", dt, (Bt, H)),
+                         ("B", B, (Bt, G, R, N)), ("C", C, (Bt, G, R, N))):
+        _check(t, name, shp, act, dev)
+    for name, t in (("A", A), ("D", D), ("dt_bias", dt_bias)):
+        _check(t, name, (H,), torch.float32, dev)
+    _check(ssm_state, "ssm_state", (Bt, H, P, N), torch.float32, dev)
+    ydt = y_dtype or (y.dtype if y is not None else act)
+    code = _dtype_code(x, ydt)
+    if y is None:
+        y = torch.empty((Bt, H, R, P), dtype=ydt, device=dev)
+    _check(y, "y", (Bt, H, R, P), ydt, dev)
+    params = SsdParams(A.data_ptr(), D.data_ptr(), dt_bias.data_ptr(), None, None)
+    dims = make_dims(Bt, 1, H, P, N, G)
+    st = lib().ssd_mimo_decode_step(ctypes.byref(dims), int(R), code, ctypes.byref(params), _ptr(x), _ptr(dt),
+                                    _ptr(B), _ptr(C), _ptr(z), _ptr(ssm_state), _ptr(y), _stream_ptr(dev))
+    if st != 0:
+        raise SsdError(st, "ssd_mimo_decode_step")
+    return y
 
 
 def device_status(device="cuda"):

@@ -40,6 +40,9 @@ struct Ctx {
     dim3 tid, bid;
     std::barrier<>* bar = nullptr;
     unsigned char* smem = nullptr;
+    std::barrier<>* warp_bar = nullptr;  // the 32 threads of this thread's warp
+    float* warp_buf = nullptr;           // 32 exchange slots of this warp
+    unsigned lane = 0;
 };
 inline thread_local Ctx ctx;
 inline dim3 g_grid, g_block;
@@ -57,6 +60,11 @@ void launch(dim3 grid, dim3 block, size_t smem_bytes, F&& body) {
                 std::unique_ptr<unsigned char[]> sm(new unsigned char[smem_bytes ? smem_bytes : 1]);
                 memset(sm.get(), 0xFF, smem_bytes ? smem_bytes : 1);
                 std::barrier<> bar(nt);
+                const unsigned nw = (nt + 31) / 32;
+                std::vector<std::unique_ptr<std::barrier<>>> wbar;
+                for (unsigned w = 0; w < nw; ++w)
+                    wbar.emplace_back(new std::barrier<>(static_cast<ptrdiff_t>(w + 1 < nw ? 32 : nt - 32 * w)));
+                std::unique_ptr<float[]> wbuf(new float[32 * nw]);
                 std::vector<std::thread> th;
                 th.reserve(nt);
                 for (unsigned t = 0; t < nt; ++t)
@@ -65,9 +73,13 @@ void launch(dim3 grid, dim3 block, size_t smem_bytes, F&& body) {
                         ctx.bid = dim3(bx, by, bz);
                         ctx.bar = &bar;
                         ctx.smem = sm.get();
+                        ctx.warp_bar = wbar[t / 32].get();
+                        ctx.warp_buf = wbuf.get() + 32 * (t / 32);
+                        ctx.lane = t % 32;
                         body();
-                        // a thread that returns early leaves the barrier's later phases to the others
+                        // a thread that returns early leaves the barriers' later phases to the others
                         bar.arrive_and_drop();
+                        ctx.warp_bar->arrive_and_drop();
                     });
                 for (auto& x : th) x.join();
             }
@@ -85,4 +97,36 @@ inline float __uint_as_float(unsigned u) {
     float f;
     memcpy(&f, &u, 4);
     return f;
+}
+
+// 16-byte vector, streaming loads and stores (plain accesses here)
+struct float4 {
+    float x, y, z, w;
+};
+inline float4 make_float4(float a, float b, float c, float d) { return float4{a, b, c, d}; }
+inline float4 __ldcs(const float4* p) { return *p; }
+inline void __stcs(float4* p, float4 v) { *p = v; }
+inline float __expf(float v) { return expf(v); }
+
+// bf16 storage: round to nearest, ties to even, on the 16 dropped bits (NaN kept quiet)
+struct __nv_bfloat16 {
+    unsigned short bits;
+};
+inline __nv_bfloat16 __float2bfloat16_rn(float f) {
+    unsigned u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) return __nv_bfloat16{(unsigned short)((u >> 16) | 0x40u)};
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return __nv_bfloat16{(unsigned short)(u >> 16)};
+}
+
+// Warp shuffle: every lane of the warp posts its value, waits for the others, reads its partner's.
+// All 32 lanes must call it (the kernels only shuffle in warp-uniform code).
+inline float __shfl_xor_sync(unsigned, float v, int lanemask) {
+    ::emu::Ctx& c = ::emu::ctx;
+    c.warp_buf[c.lane] = v;
+    c.warp_bar->arrive_and_wait();
+    const float r = c.warp_buf[c.lane ^ static_cast<unsigned>(lanemask)];
+    c.warp_bar->arrive_and_wait();
+    return r;
 }

@@ -243,3 +243,27 @@ def test_backward_rejects_bad_arguments_before_launch(L):
     none_act = {**base, "x": None, "dt": None, "B": None, "C": None, "z": None, "dy": None}
     no_param = ops.SsdGrads(*([None] * 5 + [0x100000] * 4 + [None] + [None, None]))
     assert _call_backward(L, dims(seqlen=0), ptrs=none_act, grads=no_param) == 1
+
+
+def _call_mimo(L, d, rank=4, dtype=1, params=True, ptrs=None):
+    p = ops.SsdParams(0x1000, 0x2000, 0x3000, None, None) if params is True else params
+    q = ptrs or dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, S=0x60000, y=0x70000)
+    return L.ssd_mimo_decode_step(ctypes.byref(d), rank, dtype, ctypes.byref(p) if p else None, q["x"], q["dt"],
+                                  q["B"], q["C"], q["z"], q["S"], q["y"], None)
+
+
+def test_mimo_decode_rejects_bad_arguments_before_launch(L):
+    d = dims(batch=256, seqlen=1)
+    assert _call_mimo(L, d, rank=3) == 2
+    assert _call_mimo(L, d, rank=16) == 2
+    assert _call_mimo(L, dims(headdim=32), rank=4) == 2
+    assert _call_mimo(L, d, dtype=9) == 3
+    assert _call_mimo(L, d, params=None) == 1
+    assert _call_mimo(L, d, params=ops.SsdParams(0x1000, None, 0x3000, None, None)) == 1
+    assert _call_mimo(L, d, params=ops.SsdParams(0x1008, 0x2000, 0x3000, None, None)) == 4
+    base = dict(x=0x10000, dt=0x20000, B=0x30000, C=0x40000, z=0x50000, S=0x60000, y=0x70000)
+    assert _call_mimo(L, d, ptrs={**base, "S": None}) == 1
+    assert _call_mimo(L, d, ptrs={**base, "C": 0x40004}) == 4
+    assert _call_mimo(L, d, ptrs={**base, "y": base["z"]}) == 5
+    # no sequences: nothing to do, valid
+    assert _call_mimo(L, dims(batch=0, seqlen=1)) == 0

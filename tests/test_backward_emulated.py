@@ -13,14 +13,14 @@ import numpy as np
 import pytest
 import torch
 
-import emu_backward
+import emu_harness
 import oracle
 from selective_state_space_43_b200.synth import Dims, make_backward_grads, make_prefill_inputs
 
 
 @pytest.fixture(scope="module")
 def exe(tmp_path_factory):
-    return emu_backward.build(str(tmp_path_factory.mktemp("emu")))
+    return emu_harness.build(str(tmp_path_factory.mktemp("emu")))
 
 
 def rel_l2(a, b):
@@ -53,7 +53,7 @@ def test_emulated_backward_matches_oracle(exe, case):
     d = Dims(Bt, L, H, 64, N, G, 64)
     inp = make_prefill_inputs(d, dtype=dtype, seed=L + N, init_state=init, init_conv_state=init, random_D=True)
     gr = make_backward_grads(d, dtype=torch.float32 if dy32 else dtype, seed=L + N + 1, d_final=dfin)
-    got = emu_backward.run(exe, inp, gr["dy"], gr["d_final"], dy_bf16=(dtype == torch.bfloat16 and not dy32))
+    got = emu_harness.run_backward(exe, inp, gr["dy"], gr["d_final"], dy_bf16=(dtype == torch.bfloat16 and not dy32))
     want = oracle.prefill_backward(inp, gr["dy"], gr["d_final"])
     check(got, want)
 
@@ -63,7 +63,7 @@ def test_emulated_backward_short_sequences(exe, L):
     d = Dims(2, L, 2, 64, 16, 1, 64)
     inp = make_prefill_inputs(d, dtype=torch.float32, seed=9, init_state=True, init_conv_state=True)
     gr = make_backward_grads(d, dtype=torch.float32, seed=10, d_final=True)
-    got = emu_backward.run(exe, inp, gr["dy"], gr["d_final"], dy_bf16=False)
+    got = emu_harness.run_backward(exe, inp, gr["dy"], gr["d_final"], dy_bf16=False)
     want = oracle.prefill_backward(inp, gr["dy"], gr["d_final"])
     check(got, want)
     if L == 0:

@@ -73,3 +73,13 @@ def test_backward_work_counts():
     per_head = 8 * 64 * 64 * 128 + 4 * 64 * 64 * 64 + 2 * 64 * 64 * 128
     assert bench.backward_chunk_flops(d) == 64 * (128 * per_head + 8 * 2 * 64 * 64 * 128)
     assert abs(bench.FP32_ALU_TFLOPS - 74.45) < 0.01
+
+
+def test_mimo_decode_byte_count():
+    from selective_state_space_43_b200.synth import WORKLOADS
+    d = WORKLOADS["decode_nemotron_h_8b"]["dims"]
+    # the fp32 state read and written dominates: 2 x 1.07 GB, plus x, z, y (rank 4) and B, C (rank 4)
+    state = 2 * 256 * 128 * 64 * 128 * 4
+    assert bench.mimo_decode_bytes(d, 4, 2) == state + 3 * 256 * 128 * 4 * 64 * 2 + 2 * 256 * 8 * 4 * 128 * 2 + \
+        256 * 128 * 2
+    assert bench.mimo_decode_bytes(d, 1, 2) < bench.mimo_decode_bytes(d, 4, 2) < 1.03 * state
