@@ -162,14 +162,46 @@ __global__ void __launch_bounds__(kT) dt_kernel(BwdArgs a, Ws ws) {
     }
 }
 
+// Register-tiled product of two shared-memory operands, the building block of the chunk kernels:
+//   acc[r][c] += sum_{k < K} A(ty + 16 r, k) * B(tx + 16 c, k),
+//   A(m, k) = A[m * sam + k * sak],  B(n, k) = B[n * sbn + k * sbk],
+// with the kT threads as a 16 x 16 grid (ty = tid / 16, tx = tid % 16).  Each k costs TM + TN
+// shared loads for TM * TN FMAs.  Rows and columns are interleaved by 16, so a warp (two ty, all 16
+// tx) reads two A addresses and 16 B addresses per k: bank-conflict free when sam is not a multiple
+// of 32 and sbn is odd.
+template <int TM, int TN>
+__device__ __forceinline__ void tile_mma(float (&acc)[TM][TN], const float* A, int sam, int sak, const float* B,
+                                         int sbn, int sbk, int K, int ty, int tx) {
+    for (int k = 0; k < K; ++k) {
+        float av[TM], bv[TN];
+#pragma unroll
+        for (int r = 0; r < TM; ++r) av[r] = A[(ty + 16 * r) * sam + k * sak];
+#pragma unroll
+        for (int c = 0; c < TN; ++c) bv[c] = B[(tx + 16 * c) * sbn + k * sbk];
+#pragma unroll
+        for (int r = 0; r < TM; ++r)
+#pragma unroll
+            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+}
+
+template <int TM, int TN>
+__device__ __forceinline__ void tile_zero(float (&acc)[TM][TN]) {
+#pragma unroll
+    for (int r = 0; r < TM; ++r)
+#pragma unroll
+        for (int c = 0; c < TN; ++c) acc[r][c] = 0.f;
+}
+
 // grid (nchunks, H, batch), kT threads.  Chunk-local state and adjoint sums of one head:
 //   SP[p][n] = sum_j exp(cs_last - cs_j) dt_j x_j[p] B_j[n],  LM[p][n] = sum_i exp(cs_i) g_i[p] C_i[n].
+// Each thread owns rows p = ty + 16 r (r < 4) and columns n = tx + 16 c (c < N/16) of both.
 template <int N>
 __global__ void __launch_bounds__(kT) chunk_state_kernel(BwdArgs a, Ws ws) {
-    constexpr int M = kP * N / kT;  // outputs per thread
+    constexpr int TN = N / 16;
     const int64_t nc = nchunks(a.L), HP = (int64_t)a.H * kP, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
     const int64_t c = blockIdx.x, b = blockIdx.z;
-    const int h = blockIdx.y, g = h / (a.H / a.G), tid = threadIdx.x;
+    const int h = blockIdx.y, g = h / (a.H / a.G), tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     const int64_t t0 = c * kQ;
     const int Qv = static_cast<int>(a.L - t0 < kQ ? a.L - t0 : kQ);
 
@@ -218,17 +250,19 @@ __global__ void __launch_bounds__(kT) chunk_state_kernel(BwdArgs a, Ws ws) {
     }
     __syncthreads();
     const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
+    float acc[4][TN];
+    tile_zero(acc);
+    tile_mma(acc, wx, 1, kP, Bs, 1, N, Qv, ty, tx);
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        const int e = tid + kT * m, p = e / N, n = e % N;
-        float s = 0.f, l = 0.f;
-        for (int j = 0; j < Qv; ++j) {
-            s += wx[j * kP + p] * Bs[j * N + n];
-            l += wg[j * kP + p] * Cs[j * N + n];
-        }
-        ws.SP[base + e] = s;
-        ws.LM[base + e] = l;
-    }
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int q = 0; q < TN; ++q) ws.SP[base + (int64_t)(ty + 16 * r) * N + tx + 16 * q] = acc[r][q];
+    tile_zero(acc);
+    tile_mma(acc, wg, 1, kP, Cs, 1, N, Qv, ty, tx);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int q = 0; q < TN; ++q) ws.LM[base + (int64_t)(ty + 16 * r) * N + tx + 16 * q] = acc[r][q];
 }
 
 // Sum of v over the block (kT threads); every thread gets the total.  red: kT floats.
@@ -295,38 +329,46 @@ __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
 
 template <int N>
 constexpr size_t chunk_bwd_floats() {
-    // Bs, Cs [kQ][N+1]; CB, LCB, LGX, T, xs, gs [kQ][kS]; X [kP][N+1]; 7 vectors of kQ; 3 x kT reduction
-    return 2 * (size_t)kQ * (N + 1) + 6 * (size_t)kQ * kS + (size_t)kP * (N + 1) + 7 * (size_t)kQ + 3 * (size_t)kT;
+    // Bs, Cs [kQ][N+1]; CB, LCB, LGX, Tm, xs, gs [kQ][kS]; X [kP][N+1]; red [kQ][17]; 7 vectors of kQ;
+    // 3 x kT block sums
+    return 2 * (size_t)kQ * (N + 1) + 6 * (size_t)kQ * kS + (size_t)kP * (N + 1) + (size_t)kQ * 17 +
+           7 * (size_t)kQ + 3 * (size_t)kT;
 }
 
-// grid (nchunks, G, batch), kT threads.  One chunk of one group; the group's heads in turn.
+// grid (nchunks, G, batch), kT threads.  One chunk of one group; the group's heads in turn.  The
+// contractions are register-tiled shared-memory products (tile_mma): a thread owns rows ty + 16 r and
+// columns tx + 16 c of every 64-row result, and of the group's dB / dC, which stay in registers across
+// the heads.  The causal (triangular) sums run over the whole chunk: the operands are zero above the
+// diagonal.
 template <int N>
 __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
-    constexpr int NS = N + 1;         // padded row stride of the N-wide tiles
-    constexpr int M = kQ * N / kT;    // dB / dC entries per thread
+    constexpr int NS = N + 1;      // padded row stride of the N-wide tiles
+    constexpr int TN = N / 16;     // columns per thread of the N-wide results
+    constexpr int RS = 17;         // row stride of the per-row partial sums
     const int64_t nc = nchunks(a.L), HP = (int64_t)a.H * kP, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
     const int64_t c = blockIdx.x, b = blockIdx.z, t0 = c * kQ;
-    const int g = blockIdx.y, hpg = a.H / a.G, tid = threadIdx.x;
+    const int g = blockIdx.y, hpg = a.H / a.G, tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     const int Qv = static_cast<int>(a.L - t0 < kQ ? a.L - t0 : kQ);
 
     float* sm = reinterpret_cast<float*>(SSD_DYN_SMEM());
     float* Bs = sm;                  // [kQ][NS]  post-conv B of the group
     float* Cs = Bs + kQ * NS;        // [kQ][NS]
     float* CB = Cs + kQ * NS;        // [kQ][kS]  C_i . B_j
-    float* LCB = CB + kQ * kS;       // [kQ][kS]  L_ij C_i . B_j   (i >= j, else 0)
-    float* LGX = LCB + kQ * kS;      // [kQ][kS]  L_ij g_i . x_j   (i >= j, else 0)
-    float* T = LGX + kQ * kS;        // [kQ][kS]  Sp C_i, then Lm B_j, then row prefix sums of M
-    float* xs = T + kQ * kS;         // [kQ][kS]  post-conv x of the head
+    float* LCB = CB + kQ * kS;       // [kQ][kS]  L_ij dt_j C_i . B_j         (i >= j, else 0)
+    float* LGX = LCB + kQ * kS;      // [kQ][kS]  L_ij g_i . x_j, then times dt_j (i >= j, else 0)
+    float* Tm = LGX + kQ * kS;       // [kQ][kS]  row prefix sums of M
+    float* xs = Tm + kQ * kS;        // [kQ][kS]  post-conv x of the head
     float* gs = xs + kQ * kS;        // [kQ][kS]  g = dy * silu(z)
     float* X = gs + kQ * kS;         // [kP][NS]  Sp, then Lm
-    float* dts = X + kP * NS;        // [kQ]
+    float* red = X + kP * NS;        // [kQ][RS]  per-row partial sums over the 16 column threads
+    float* dts = red + kQ * RS;      // [kQ]
     float* css = dts + kQ;
     float* ex = css + kQ;            // exp(cs_i)
     float* el = ex + kQ;             // exp(cs_last - cs_j)
-    float* Ev = el + kQ;
+    float* Ev = el + kQ;             // exp(cs_i) g_i . (Sp C_i)
     float* Wv = Ev + kQ;             // exp(cs_last - cs_j) x_j . (Lm B_j)
     float* Dr = Wv + kQ;             // ddt without the decay term
-    float* red = Dr + kQ;            // [3][kT]
+    float* bsum = Dr + kQ;           // [3][kT]
 
     // the group's post-conv B and C, and C_i . B_j
     for (int e = tid; e < kQ * N; e += kT) {
@@ -341,19 +383,19 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         Cs[j * NS + n] = cv;
     }
     __syncthreads();
-    for (int e = tid; e < kQ * kQ; e += kT) {
-        const int i = e / kQ, j = e % kQ;
-        float acc = 0.f;
-        for (int n = 0; n < N; ++n) acc += Cs[i * NS + n] * Bs[j * NS + n];
-        CB[i * kS + j] = acc;
+    {
+        float acc[4][4];
+        tile_zero(acc);
+        tile_mma(acc, Cs, NS, 1, Bs, NS, 1, N, ty, tx);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) CB[(ty + 16 * r) * kS + tx + 16 * q] = acc[r][q];
     }
 
-    float dBa[M], dCa[M];
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-        dBa[m] = 0.f;
-        dCa[m] = 0.f;
-    }
+    float dBa[4][TN], dCa[4][TN];  // rows j (or i) = ty + 16 r, columns n = tx + 16 c
+    tile_zero(dBa);
+    tile_zero(dCa);
 
     for (int hl = 0; hl < hpg; ++hl) {
         const int h = g * hpg + hl;
@@ -380,127 +422,160 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         }
         __syncthreads();
 
-        // 2: decay factors, L-weighted C.B and g.x, the entering state
+        // 2: decay factors; L-weighted g.x (LGX, without dt for now) and dt-weighted C.B (LCB); Sp
         const float cl = css[Qv - 1];
         if (tid < kQ) {
             ex[tid] = tid < Qv ? expf(css[tid]) : 0.f;
             el[tid] = tid < Qv ? expf(cl - css[tid]) : 0.f;
         }
-        for (int e = tid; e < kQ * kQ; e += kT) {
-            const int i = e / kQ, j = e % kQ;
-            float lcb = 0.f, lgx = 0.f;
-            if (j <= i && i < Qv) {
-                const float Lij = expf(css[i] - css[j]);
-                float gx = 0.f;
-                for (int p = 0; p < kP; ++p) gx += gs[i * kS + p] * xs[j * kS + p];
-                lcb = CB[i * kS + j] * Lij;
-                lgx = gx * Lij;
-            }
-            LCB[i * kS + j] = lcb;
-            LGX[i * kS + j] = lgx;
+        {
+            float acc[4][4];
+            tile_zero(acc);
+            tile_mma(acc, gs, kS, 1, xs, kS, 1, kP, ty, tx);
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = ty + 16 * r, j = tx + 16 * q;
+                    float lgx = 0.f, lcb = 0.f;
+                    if (j <= i && i < Qv) {
+                        const float Lij = expf(css[i] - css[j]);
+                        lgx = acc[r][q] * Lij;
+                        lcb = CB[i * kS + j] * Lij * dts[j];
+                    }
+                    LGX[i * kS + j] = lgx;
+                    LCB[i * kS + j] = lcb;
+                }
         }
         for (int e = tid; e < kP * N; e += kT) X[(e / N) * NS + e % N] = ws.SP[sbase + e];
         __syncthreads();
 
-        // 3: T = Sp C_i;  dC_i += exp(cs_i) g_i Sp
-        for (int e = tid; e < kQ * kP; e += kT) {
-            const int i = e / kP, p = e % kP;
-            float acc = 0.f;
-            for (int n = 0; n < N; ++n) acc += X[p * NS + n] * Cs[i * NS + n];
-            T[i * kS + p] = acc;
-        }
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const int e = tid + kT * m, i = e / N, n = e % N;
-            float acc = 0.f;
-            for (int p = 0; p < kP; ++p) acc += gs[i * kS + p] * X[p * NS + n];
-            dCa[m] += ex[i] * acc;
-        }
-        __syncthreads();
-
-        // 4: y recomputed for dz;  E_i
-        for (int e = tid; e < kQ * kP; e += kT) {
-            const int i = e / kP, p = e % kP;
-            if (i < Qv) {
-                float acc = 0.f;
-                for (int j = 0; j <= i; ++j) acc += LCB[i * kS + j] * dts[j] * xs[j * kS + p];
-                const float yv = acc + ex[i] * T[i * kS + p] + Dh * xs[i * kS + p];
-                const int64_t yi = (b * a.L + t0 + i) * HP + (int64_t)h * kP + p;
-                a.dz[yi] = ld_act(a.dy, yi, a.dy_bf16) * yv * dsilu_f(ld_act(a.z, yi, a.act_bf16));
-            }
-        }
+        // 3: y recomputed for dz (Sp C_i and the intra-chunk sum), E_i, dC_i += exp(cs_i) g_i Sp;
+        //    the direct part of ddt from the pairs (before LGX takes dt)
         if (tid < kQ) {
-            float acc = 0.f;
-            for (int p = 0; p < kP; ++p) acc += gs[tid * kS + p] * T[tid * kS + p];
-            Ev[tid] = ex[tid] * acc;
-        }
-        __syncthreads();
-
-        // 5: the leaving adjoint; T = Lm B_j;  dB_j += dt_j exp(cs_last - cs_j) x_j Lm
-        for (int e = tid; e < kP * N; e += kT) X[(e / N) * NS + e % N] = ws.LM[sbase + e];
-        __syncthreads();
-        for (int e = tid; e < kQ * kP; e += kT) {
-            const int j = e / kP, p = e % kP;
-            float acc = 0.f;
-            for (int n = 0; n < N; ++n) acc += X[p * NS + n] * Bs[j * NS + n];
-            T[j * kS + p] = acc;
-        }
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const int e = tid + kT * m, j = e / N, n = e % N;
-            float acc = 0.f;
-            for (int p = 0; p < kP; ++p) acc += xs[j * kS + p] * X[p * NS + n];
-            dBa[m] += dts[j] * el[j] * acc;
-        }
-        __syncthreads();
-
-        // 6: dx (post-conv, this head's channels);  W_j and the direct part of ddt
-        for (int e = tid; e < kQ * kP; e += kT) {
-            const int j = e / kP, p = e % kP;
-            if (j < Qv) {
-                float acc = 0.f;
-                for (int i = j; i < Qv; ++i) acc += LCB[i * kS + j] * gs[i * kS + p];
-                const float d = dts[j] * (acc + el[j] * T[j * kS + p]) + Dh * gs[j * kS + p];
-                ws.DU[(b * a.L + t0 + j) * conv_dim + (int64_t)h * kP + p] = d;
-            }
-        }
-        if (tid < kQ) {
-            float w = 0.f;
-            for (int p = 0; p < kP; ++p) w += xs[tid * kS + p] * T[tid * kS + p];
-            w *= el[tid];
-            float dr = w;
+            float dr = 0.f;
             for (int i = tid; i < Qv; ++i) dr += LGX[i * kS + tid] * CB[i * kS + tid];
-            Wv[tid] = w;
             Dr[tid] = dr;
         }
-        // 7: the intra-chunk parts of dB and dC
+        float pD = 0.f;
+        {
+            float spc[4][4], yin[4][4];
+            tile_zero(spc);
+            tile_zero(yin);
+            tile_mma(spc, Cs, NS, 1, X, NS, 1, N, ty, tx);       // [i][p] = sum_n C_i[n] Sp[p][n]
+            tile_mma(yin, LCB, kS, 1, xs, 1, kS, Qv, ty, tx);    // [i][p] = sum_j LCB[i][j] x_j[p]
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const int e = tid + kT * m, r = e / N, n = e % N;
-            float accb = 0.f, accc = 0.f;
-            for (int i = r; i < Qv; ++i) accb += LGX[i * kS + r] * Cs[i * NS + n];
-            for (int j = 0; j <= r && j < Qv; ++j) accc += LGX[r * kS + j] * dts[j] * Bs[j * NS + n];
-            dBa[m] += dts[r] * accb;
-            dCa[m] += accc;
+            for (int r = 0; r < 4; ++r) {
+                const int i = ty + 16 * r;
+                float epart = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int p = tx + 16 * q;
+                    const float gv = gs[i * kS + p], xv = xs[i * kS + p];
+                    epart += gv * spc[r][q];
+                    pD += gv * xv;
+                    if (i < Qv) {
+                        const float yv = yin[r][q] + ex[i] * spc[r][q] + Dh * xv;
+                        const int64_t yi = (b * a.L + t0 + i) * HP + (int64_t)h * kP + p;
+                        a.dz[yi] = ld_act(a.dy, yi, a.dy_bf16) * yv * dsilu_f(ld_act(a.z, yi, a.act_bf16));
+                    }
+                }
+                red[i * RS + tx] = epart;
+            }
+        }
+        {
+            float acc[4][TN];
+            tile_zero(acc);
+            tile_mma(acc, gs, kS, 1, X, 1, NS, kP, ty, tx);      // [i][n] = sum_p g_i[p] Sp[p][n]
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int q = 0; q < TN; ++q) dCa[r][q] += ex[ty + 16 * r] * acc[r][q];
         }
         __syncthreads();
 
-        // 8: d(dA): T[i][k] = sum_{j<k} M_ij, then column sums over i >= k
+        // 4: E_i; LGX takes dt_j; the leaving adjoint Lm
         if (tid < kQ) {
+            float e = 0.f;
+            for (int k = 0; k < 16; ++k) e += red[tid * RS + k];
+            Ev[tid] = ex[tid] * e;
+        }
+        for (int e = tid; e < kQ * kQ; e += kT) LGX[(e / kQ) * kS + e % kQ] *= dts[e % kQ];
+        for (int e = tid; e < kP * N; e += kT) X[(e / N) * NS + e % N] = ws.LM[sbase + e];
+        __syncthreads();
+
+        // 5: dx (Lm B_j and the intra-chunk sum), W_j; dB_j += dt_j exp(cs_last - cs_j) x_j Lm and the
+        //    intra-chunk parts of dB and dC
+        {
+            float lmb[4][4], dxi[4][4];
+            tile_zero(lmb);
+            tile_zero(dxi);
+            tile_mma(lmb, Bs, NS, 1, X, NS, 1, N, ty, tx);       // [j][p] = sum_n B_j[n] Lm[p][n]
+            tile_mma(dxi, LCB, 1, kS, gs, 1, kS, Qv, ty, tx);    // [j][p] = sum_i LCB[i][j] g_i[p]
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = ty + 16 * r;
+                float wpart = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int p = tx + 16 * q;
+                    wpart += xs[j * kS + p] * lmb[r][q];
+                    if (j < Qv) {
+                        const float d = dxi[r][q] + dts[j] * el[j] * lmb[r][q] + Dh * gs[j * kS + p];
+                        ws.DU[(b * a.L + t0 + j) * conv_dim + (int64_t)h * kP + p] = d;
+                    }
+                }
+                red[j * RS + tx] = wpart;
+            }
+        }
+        {
+            float acc[4][TN];
+            tile_zero(acc);
+            tile_mma(acc, xs, kS, 1, X, 1, NS, kP, ty, tx);      // [j][n] = sum_p x_j[p] Lm[p][n]
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = ty + 16 * r;
+#pragma unroll
+                for (int q = 0; q < TN; ++q) dBa[r][q] += dts[j] * el[j] * acc[r][q];
+            }
+            tile_zero(acc);
+            tile_mma(acc, LGX, 1, kS, Cs, 1, NS, Qv, ty, tx);    // [j][n] = sum_i LGX[i][j] dt_j C_i[n]
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int q = 0; q < TN; ++q) dBa[r][q] += acc[r][q];
+            tile_zero(acc);
+            tile_mma(acc, LGX, kS, 1, Bs, 1, NS, Qv, ty, tx);    // [i][n] = sum_j LGX[i][j] dt_j B_j[n]
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int q = 0; q < TN; ++q) dCa[r][q] += acc[r][q];
+        }
+        __syncthreads();
+
+        // 6: W_j and the rest of the direct part of ddt; row prefix sums of M_ij = LGX[i][j] C_i . B_j
+        if (tid < kQ) {
+            float w = 0.f;
+            for (int k = 0; k < 16; ++k) w += red[tid * RS + k];
+            w *= el[tid];
+            Wv[tid] = w;
+            Dr[tid] += w;
             float run = 0.f;
             for (int k = 0; k <= tid; ++k) {
-                T[tid * kS + k] = run;
-                run += LGX[tid * kS + k] * CB[tid * kS + k] * dts[k];
+                Tm[tid * kS + k] = run;
+                run += LGX[tid * kS + k] * CB[tid * kS + k];
             }
         }
         __syncthreads();
+
+        // 7: d(dA_k) = sum_{i>=k} sum_{j<k} M_ij + sum_{i>=k} E_i + F + sum_{j<k} dt_j W_j; ddt; partials
         const float F = ws.PF[(b * nc + c) * a.H + h];
-        float pdA = 0.f, pbias = 0.f, pD = 0.f;
+        float pdA = 0.f, pbias = 0.f;
         if (tid < Qv) {
             const int k = tid;
             float R = 0.f, Es = 0.f, Wsum = 0.f;
             for (int i = k; i < Qv; ++i) {
-                R += T[i * kS + k];
+                R += Tm[i * kS + k];
                 Es += Ev[i];
             }
             for (int j = 0; j < k; ++j) Wsum += dts[j] * Wv[j];
@@ -512,8 +587,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             pdA = dts[k] * dda;
             pbias = dr;
         }
-        for (int e = tid; e < kQ * kP; e += kT) pD += gs[(e / kP) * kS + e % kP] * xs[(e / kP) * kS + e % kP];
-        const float sA = block_sum(pdA, red), sD = block_sum(pD, red + kT), sB = block_sum(pbias, red + 2 * kT);
+        const float sA = block_sum(pdA, bsum), sD = block_sum(pD, bsum + kT), sB = block_sum(pbias, bsum + 2 * kT);
         if (tid == 0) {
             float* ph = ws.PH + ((b * nc + c) * a.H + h) * 3;
             ph[0] = sA;
@@ -524,12 +598,15 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     }
 
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        const int e = tid + kT * m, j = e / N, n = e % N;
+    for (int r = 0; r < 4; ++r) {
+        const int j = ty + 16 * r;
         if (j < Qv) {
             const int64_t row = (b * a.L + t0 + j) * conv_dim;
-            ws.DU[row + HP + (int64_t)g * N + n] = dBa[m];
-            ws.DU[row + HP + GN + (int64_t)g * N + n] = dCa[m];
+#pragma unroll
+            for (int q = 0; q < TN; ++q) {
+                ws.DU[row + HP + (int64_t)g * N + tx + 16 * q] = dBa[r][q];
+                ws.DU[row + HP + GN + (int64_t)g * N + tx + 16 * q] = dCa[r][q];
+            }
         }
     }
 }
