@@ -55,9 +55,42 @@ __device__ __forceinline__ void st_out(void* p, int64_t i, float v, bool bf16) {
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + __expf(-v)); }
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(__expf(v)); }
 
+// Segmented reduce-scatter of CNT partial sums over the lanes of a state row (offsets O, O/2, .., 1
+// inside segments of 2*O lanes).  While more than one sum is left, each level swaps half of them with
+// the partner lane (lane ^ o): the lane keeps the upper half if its bit o is set, else the lower half,
+// and adds what it receives; then the remaining single sum is reduced plainly.  Costs CNT/2 + CNT/4 +
+// .. shuffles for the scatter levels instead of CNT per level.  On return vals[0 .. left) hold the
+// full sums of outputs first .. first+left-1 (first built from the lane's scatter bits), the same in
+// every lane that shares those bits.
+template <int CNT, int O>
+struct RowReduce {
+    static __device__ __forceinline__ void run(float* vals, int lane, int& first, int& left) {
+        if constexpr (O == 0) {
+            left = CNT;
+        } else if constexpr (CNT > 1) {
+            constexpr int HALF = CNT / 2;
+            const bool upper = (lane & O) != 0;
+            float keep[HALF];
+#pragma unroll
+            for (int i = 0; i < HALF; ++i) {
+                const float send = upper ? vals[i] : vals[HALF + i];
+                const float mine = upper ? vals[HALF + i] : vals[i];
+                keep[i] = mine + __shfl_xor_sync(0xffffffffu, send, O);
+            }
+#pragma unroll
+            for (int i = 0; i < HALF; ++i) vals[i] = keep[i];
+            if (upper) first += HALF;
+            RowReduce<HALF, O / 2>::run(vals, lane, first, left);
+        } else {
+            vals[0] += __shfl_xor_sync(0xffffffffu, vals[0], O);
+            RowReduce<1, O / 2>::run(vals, lane, first, left);
+        }
+    }
+};
+
 // grid batch * H, kT threads.
 template <int R, int N>
-__global__ void __launch_bounds__(kT) mimo_decode_kernel(MimoArgs a) {
+__global__ void __launch_bounds__(kT, (R <= 4 ? 3 : 2)) mimo_decode_kernel(MimoArgs a) {
     constexpr int LPR = N / 4;            // lanes per state row (a float4 each)
     constexpr int RPW = 32 / LPR;         // rows per warp per pass
     constexpr int ITER = kP / (8 * RPW);  // passes over the P rows with 8 warps
@@ -91,12 +124,10 @@ __global__ void __launch_bounds__(kT) mimo_decode_kernel(MimoArgs a) {
     const float decay = __expf(dtv * a.A[h]);
     __syncthreads();
 
-    float4 bq[R], cq[R];
-#pragma unroll
-    for (int k = 0; k < R; ++k) {
-        bq[k] = make_float4(s_B[k * N + n0], s_B[k * N + n0 + 1], s_B[k * N + n0 + 2], s_B[k * N + n0 + 3]);
-        cq[k] = make_float4(s_C[k * N + n0], s_C[k * N + n0 + 1], s_C[k * N + n0 + 2], s_C[k * N + n0 + 3]);
-    }
+    // the lane's 4 columns of B_k and C_k are re-read from shared memory (16-byte loads) where they are
+    // used, rather than held in 8R registers, to keep 3 CTAs per SM at R = 4
+    const float4* sB4 = reinterpret_cast<const float4*>(s_B + n0);
+    const float4* sC4 = reinterpret_cast<const float4*>(s_C + n0);
 #pragma unroll
     for (int it = 0; it < ITER; ++it) {
         const int p = (it * 8 + warp) * RPW + rsub;
@@ -104,10 +135,11 @@ __global__ void __launch_bounds__(kT) mimo_decode_kernel(MimoArgs a) {
 #pragma unroll
         for (int k = 0; k < R; ++k) {
             const float xk = s_x[k * kP + p];
-            ix += xk * bq[k].x;
-            iy += xk * bq[k].y;
-            iz += xk * bq[k].z;
-            iw += xk * bq[k].w;
+            const float4 bq = sB4[k * (N / 4)];
+            ix += xk * bq.x;
+            iy += xk * bq.y;
+            iz += xk * bq.z;
+            iw += xk * bq.w;
         }
         float4 s = v[it];
         s.x = fmaf(decay, s.x, dtv * ix);
@@ -115,12 +147,21 @@ __global__ void __launch_bounds__(kT) mimo_decode_kernel(MimoArgs a) {
         s.z = fmaf(decay, s.z, dtv * iz);
         s.w = fmaf(decay, s.w, dtv * iw);
         __stcs(S + ((p * N + n0) >> 2), s);
+        float part[R];
 #pragma unroll
         for (int k = 0; k < R; ++k) {
-            float part = s.x * cq[k].x + s.y * cq[k].y + s.z * cq[k].z + s.w * cq[k].w;
+            const float4 cq = sC4[k * (N / 4)];
+            part[k] = s.x * cq.x + s.y * cq.y + s.z * cq.z + s.w * cq.w;
+        }
+        int first = 0, left = R;
+        RowReduce<R, LPR / 2>::run(part, lane, first, left);
+        // the scatter levels used the lane's highest segment bits; the lanes whose remaining bits are
+        // zero write the sums they hold
+        constexpr int SCAT = (R < LPR ? R : LPR);  // lanes that end up with distinct sums
+        if ((lane % (LPR / SCAT)) == 0) {
 #pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if ((lane % LPR) == 0) s_y[k * kP + p] = part;
+            for (int k = 0; k < R; ++k)
+                if (k < left) s_y[(first + k) * kP + p] = part[k];
         }
     }
     __syncthreads();
