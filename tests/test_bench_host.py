@@ -83,3 +83,65 @@ def test_mimo_decode_byte_count():
     assert bench.mimo_decode_bytes(d, 4, 2) == state + 3 * 256 * 128 * 4 * 64 * 2 + 2 * 256 * 8 * 4 * 128 * 2 + \
         256 * 128 * 2
     assert bench.mimo_decode_bytes(d, 1, 2) < bench.mimo_decode_bytes(d, 4, 2) < 1.03 * state
+
+
+class _FakeEvent:
+    def __init__(self, enable_timing=False):
+        pass
+
+    def record(self, *a):
+        pass
+
+    def elapsed_time(self, other):
+        return 2.0  # ms
+
+
+class _FakeSampler:
+    def load(self, on):
+        pass
+
+
+class _FakeOps:
+    """Stands in for the binding: checks the call shapes the bench legs make, computes nothing."""
+
+    def __init__(self):
+        from selective_state_space_43_b200 import ops
+        self.make_dims = ops.make_dims
+        self.calls = {"backward": 0, "mimo": 0, "events": []}
+
+    def prefill_backward_workspace_bytes(self, dims):
+        return 1024
+
+    def prefill_backward(self, x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, dy, init_state, init_conv_state,
+                         d_final_state, workspace=None):
+        assert dy.shape == x.shape and d_final_state.shape[0] == x.shape[0] and workspace.numel() >= 1024
+        self.calls["backward"] += 1
+        return {}
+
+    def mimo_decode_step(self, x, dt, B, C, z, A, D, dt_bias, ssm_state, y=None):
+        assert x.shape[2] == bench.MIMO_RANK and y.shape == x.shape and ssm_state.dtype == torch.float32
+        self.calls["mimo"] += 1
+        return y
+
+    def set_timing_events(self, before, after):
+        self.calls["events"].append(before is None)
+
+
+def test_backward_and_mimo_bench_legs_on_a_fake_device(monkeypatch):
+    from selective_state_space_43_b200.synth import Dims
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    fake = _FakeOps()
+    d = Dims(1, 256, 4, 64, 32, 2, 128)
+    flush = torch.empty(16)
+    peaks = {"hbm_gbs": 6554.6}
+    b = bench.bench_backward(fake, d, torch.bfloat16, torch.device("cpu"), flush, 5, 3, 1, _FakeSampler())
+    assert fake.calls["backward"] == 3 + 5 and fake.calls["events"][-1] is True   # hook cleared afterwards
+    assert b["ms_per_step"] == 2.0 and b["value"] == 256 / 2e-3
+    rf = b["dominant_kernel"]["roofline"]
+    assert rf["bound"] == "alu" and rf["unit"] == "TFLOP/s"
+    assert abs(rf["achieved"] - bench.backward_chunk_flops(d) / 2e-3 / 1e12) < 1e-9
+    m = bench.bench_mimo(fake, d, torch.bfloat16, torch.device("cpu"), 1, _FakeSampler(), peaks, 4)
+    assert fake.calls["mimo"] == 3 + 4
+    assert abs(m["value"] - bench.mimo_decode_bytes(d, bench.MIMO_RANK, 2) / 2e-3 / 1e9) < 1e-6
+    assert m["roofline"]["frac"] == m["roofline"]["achieved"] / 6554.6
