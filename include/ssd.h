@@ -296,7 +296,7 @@ SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t nor
  *                 (the post-conv channels and their gradients, fp32, plus two
  *                 fp32 [batch][ceil(seqlen/64)][H][P][N] state arrays)
  * All pointers device memory, 16-byte aligned; gradients must not overlap the
- * inputs or one another.  The result is deterministic (every sum is taken in a
+ * inputs, the workspace or one another (SSD_ERR_UNSUPPORTED otherwise).  The result is deterministic (every sum is taken in a
  * fixed order).  seqlen == 0 is valid: d_init_state = d_final_state (or zero),
  * the parameter gradients and d_init_conv_state are zero.  Errors as for
  * ssd_prefill; SSD_ERR_SHAPE also when ceil(seqlen/64) or batch exceeds 65535.
@@ -317,6 +317,7 @@ SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t nor
  *   ssm_state   [batch][H][P][N] fp32, updated in place
  *   y           [batch][H][R][P]     dtype, fp32 for SSD_BF16_YF32 (out)
  * params: A, D, dt_bias are used; conv_w and conv_b are ignored (may be NULL).
+ * y must not overlap any input or the state (SSD_ERR_UNSUPPORTED).
  * dims->seqlen and dims->chunk are ignored.  Same size limits as the decode
  * step; SSD_ERR_SHAPE for any other rank.
  */

@@ -49,6 +49,29 @@ ssd_status check_params(const ssd_params* p) {
     return SSD_OK;
 }
 
+// A byte range [p, p + n) of a caller's buffer (p may be null: no buffer).
+struct Span {
+    const void* p;
+    uint64_t n;
+};
+
+bool overlap(const Span& a, const Span& b) {
+    if (!a.p || !b.p || a.n == 0 || b.n == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    return a0 < b0 + b.n && b0 < a0 + a.n;
+}
+
+// Whether any output range overlaps another output or any input range.
+bool outputs_alias(const Span* outs, int nout, const Span* ins, int nin) {
+    for (int i = 0; i < nout; ++i) {
+        for (int j = i + 1; j < nout; ++j)
+            if (overlap(outs[i], outs[j])) return true;
+        for (int j = 0; j < nin; ++j)
+            if (overlap(outs[i], ins[j])) return true;
+    }
+    return false;
+}
+
 }  // namespace
 
 extern "C" {
@@ -257,6 +280,24 @@ ssd_status ssd_prefill_backward(const ssd_dims* d, ssd_dtype dtype, const ssd_pa
     const size_t need = ssd::bwd::workspace_bytes(d->batch, d->seqlen, d->nheads, d->headdim, d->d_state,
                                                   d->ngroups);
     if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
+    {
+        const uint64_t rows = (uint64_t)d->batch * (uint64_t)d->seqlen, H = d->nheads;
+        const uint64_t HP = H * d->headdim, GN = (uint64_t)d->ngroups * d->d_state, cd = HP + 2 * GN;
+        const uint64_t st = (uint64_t)d->batch * HP * d->d_state, ae = dtype == SSD_F32 ? 4 : 2;
+        const uint64_t de = dtype == SSD_BF16 ? 2 : 4;
+        const Span ins[] = {{x, rows * HP * ae},         {dt, rows * H * ae},          {B, rows * GN * ae},
+                            {C, rows * GN * ae},         {z, rows * HP * ae},          {dy, rows * HP * de},
+                            {init_state, st * 4},        {init_conv_state, (uint64_t)d->batch * cd * 3 * ae},
+                            {d_final_state, st * 4},     {params->A, H * 4},           {params->D, H * 4},
+                            {params->dt_bias, H * 4},    {params->conv_w, cd * 16},    {params->conv_b, cd * 4},
+                            {workspace, need}};
+        const Span outs[] = {{g->dx, rows * HP * 4},     {g->ddt, rows * H * 4},       {g->dB, rows * GN * 4},
+                             {g->dC, rows * GN * 4},     {g->dz, rows * HP * 4},       {g->dA, H * 4},
+                             {g->dD, H * 4},             {g->ddt_bias, H * 4},         {g->dconv_w, cd * 16},
+                             {g->dconv_b, cd * 4},       {g->d_init_state, st * 4},
+                             {g->d_init_conv_state, (uint64_t)d->batch * cd * 3 * 4}};
+        if (outputs_alias(outs, 12, ins, 15)) return SSD_ERR_UNSUPPORTED;
+    }
 
     ssd::bwd::BwdArgs a{};
     a.batch = d->batch;
@@ -290,7 +331,15 @@ ssd_status ssd_mimo_decode_step(const ssd_dims* d, int32_t rank, ssd_dtype dtype
     const void* ptrs[] = {x, dt, B, C, z, ssm_state, y};
     for (const void* p : ptrs)
         if (!aligned16(p)) return SSD_ERR_ALIGN;
-    if (y == x || y == z) return SSD_ERR_UNSUPPORTED;
+    {
+        const uint64_t bh = (uint64_t)d->batch * d->nheads, ae = dtype == SSD_F32 ? 4 : 2;
+        const uint64_t ye = dtype == SSD_BF16 ? 2 : 4, R = (uint64_t)rank;
+        const uint64_t bc = (uint64_t)d->batch * d->ngroups * R * d->d_state * ae;
+        const Span ins[] = {{x, bh * R * d->headdim * ae}, {dt, bh * ae}, {B, bc}, {C, bc},
+                            {z, bh * R * d->headdim * ae}, {ssm_state, bh * d->headdim * d->d_state * 4}};
+        const Span outs[] = {{y, bh * R * d->headdim * ye}};
+        if (outputs_alias(outs, 1, ins, 6)) return SSD_ERR_UNSUPPORTED;
+    }
     if (d->batch == 0) return SSD_OK;
     ssd::mimo::MimoArgs a{};
     a.batch = d->batch;

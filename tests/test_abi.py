@@ -267,3 +267,33 @@ def test_mimo_decode_rejects_bad_arguments_before_launch(L):
     assert _call_mimo(L, d, ptrs={**base, "y": base["z"]}) == 5
     # no sequences: nothing to do, valid
     assert _call_mimo(L, dims(batch=0, seqlen=1)) == 0
+
+
+def test_backward_rejects_overlapping_gradients(L):
+    d = dims(seqlen=64, nheads=4, d_state=32, ngroups=1)
+    need = L.ssd_prefill_backward_workspace_bytes(ctypes.byref(d))
+    rows, HP = 64, 256
+    base = dict(x=0x1000000, dt=0x2000000, B=0x3000000, C=0x4000000, z=0x5000000, init=None, init_conv=None,
+                dy=0x6000000, dfin=None)
+    ws = 0x40000000
+    ok = [0x10000000 + 0x1000000 * k for k in range(10)] + [None, None]
+    # every call below overlaps two ranges, so it fails validation before any launch
+    g = list(ok)
+    g[0] = base["x"] + 64                                   # dx inside x
+    assert _call_backward(L, d, ptrs=base, grads=ops.SsdGrads(*g), ws=ws, ws_bytes=need) == 5
+    g = list(ok)
+    g[6] = g[5]                                             # dD == dA
+    assert _call_backward(L, d, ptrs=base, grads=ops.SsdGrads(*g), ws=ws, ws_bytes=need) == 5
+    g = list(ok)
+    g[10] = ws + 256                                        # d_init_state inside the workspace
+    assert _call_backward(L, d, ptrs=base, grads=ops.SsdGrads(*g), ws=ws, ws_bytes=need) == 5
+    g = list(ok)
+    g[4] = ok[0] + rows * HP * 4 - 16                       # dz starts 16 bytes before the end of dx
+    assert _call_backward(L, d, ptrs=base, grads=ops.SsdGrads(*g), ws=ws, ws_bytes=need) == 5
+
+
+def test_mimo_rejects_an_overlapping_output(L):
+    d = dims(batch=2, seqlen=1, nheads=4, d_state=32, ngroups=1)
+    base = dict(x=0x1000000, dt=0x2000000, B=0x3000000, C=0x4000000, z=0x5000000, S=0x6000000, y=0x7000000)
+    assert _call_mimo(L, d, ptrs={**base, "y": base["S"] + 1024}) == 5
+    assert _call_mimo(L, d, ptrs={**base, "y": base["B"]}) == 5
