@@ -1,0 +1,84 @@
+"""The host emulation of the kernels is a strong enough check: faults planted in temporary copies of
+the backward kernels' source (an access outside a buffer, a read of shared memory that was never
+written, a dropped term) each make the emulated run fail, through AddressSanitizer, through the
+NaN-filled outputs and shared memory, or through the comparison with the oracle.  CPU only; the
+faults are planted in copies, never in the library's source."""
+import concurrent.futures as cf
+import os
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import emu_harness
+import oracle
+from selective_state_space_43_b200.synth import Dims, make_backward_grads, make_prefill_inputs
+
+SRC = os.path.join(emu_harness.CSRC, "ssd_backward.cu")
+
+MUTANTS = {
+    # reads x one token past the tile: beyond the array for the last tile of the last sequence
+    "post-conv reads past its tile": ("        const float r3 = raw_at(a, b, t, c);\n"
+                                      "        ws.U[(b * a.L + t) * conv_dim + c]",
+                                      "        const float r3 = raw_at(a, b, t + 1, c);\n"
+                                      "        ws.U[(b * a.L + t) * conv_dim + c]"),
+    # writes each pre-conv gradient one token late: beyond dx / dB / dC for the last token
+    "conv backward writes one row late": ("out[(b * a.L + s) * ostride + ocol] = gs;",
+                                          "out[(b * a.L + s + 1) * ostride + ocol] = gs;"),
+    # leaves the rows of a ragged chunk past its end as they were (NaN bytes for the first head)
+    "ragged rows not cleared": ("            xs[j * kS + p] = xv;", "            if (j < Qv) xs[j * kS + p] = xv;"),
+    # drops the D skip term of dx
+    "dx without the D skip": ("dts[j] * el[j] * lmb[r][q] + Dh * gs[j * kS + p];", "dts[j] * el[j] * lmb[r][q];"),
+}
+
+
+def _build(name, old, new, tmp):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for '{name}' not unique"
+    d = os.path.join(tmp, name.replace(" ", "_"))
+    os.makedirs(d)
+    with open(os.path.join(d, "ssd_backward.cu"), "w") as f:
+        f.write(src.replace(old, new))
+    exe = os.path.join(d, "run_backward")
+    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
+           "-fno-omit-frame-pointer", "-w", "-I", d, "-I", emu_harness.EMU, "-I", emu_harness.CSRC, "-o", exe,
+           os.path.join(emu_harness.EMU, "run_backward.cpp"), "-pthread"]
+    subprocess.check_call(cmd)
+    return exe
+
+
+@pytest.fixture(scope="module")
+def mutant_exes(tmp_path_factory):
+    tmp = str(tmp_path_factory.mktemp("emu_mutants"))
+    with cf.ThreadPoolExecutor(max_workers=len(MUTANTS)) as ex:
+        futs = {name: ex.submit(_build, name, old, new, tmp) for name, (old, new) in MUTANTS.items()}
+        return {name: f.result() for name, f in futs.items()}
+
+
+def _case():
+    d = Dims(2, 150, 4, 64, 32, 2, 64)
+    inp = make_prefill_inputs(d, dtype=torch.float32, seed=8, init_state=True, init_conv_state=True, random_D=True)
+    gr = make_backward_grads(d, dtype=torch.float32, seed=9)
+    return inp, gr
+
+
+def _caught(exe, inp, gr, want):
+    try:
+        got = emu_harness.run_backward(exe, inp, gr["dy"], gr["d_final"], dy_bf16=False)
+    except RuntimeError:
+        return True                                   # sanitizer report or a failed run
+    for k, ref in want.items():
+        g = got[k].astype(np.float64)
+        if np.isnan(g).any():
+            return True
+        if np.linalg.norm(g - ref) > 2e-5 * max(np.linalg.norm(ref), 1e-30):
+            return True
+    return False
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_kernel_fault_is_caught(mutant_exes, name):
+    inp, gr = _case()
+    want = oracle.prefill_backward(inp, gr["dy"], gr["d_final"])
+    assert _caught(mutant_exes[name], inp, gr, want), f"the emulation missed the planted fault '{name}'"
