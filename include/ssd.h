@@ -293,8 +293,9 @@ SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t nor
  *                 wanted (they are the gradients for the given initial states,
  *                 or for zero ones when those are NULL)
  *   workspace     device scratch of ssd_prefill_backward_workspace_bytes()
- *                 (the post-conv channels and their gradients, fp32, plus two
- *                 fp32 [batch][ceil(seqlen/64)][H][P][N] state arrays)
+ *                 (the post-conv channels and their gradients, fp32, a second
+ *                 copy of the B/C gradients, and two fp32
+ *                 [batch][ceil(seqlen/64)][H][P][N] state arrays)
  * All pointers device memory, 16-byte aligned; gradients must not overlap the
  * inputs, the workspace or one another (SSD_ERR_UNSUPPORTED otherwise).  The result is deterministic (every sum is taken in a
  * fixed order).  seqlen == 0 is valid: d_init_state = d_final_state (or zero),

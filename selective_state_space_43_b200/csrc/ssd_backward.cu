@@ -29,11 +29,12 @@
 //   dt_kernel           dt and the in-chunk cumsum of dt*A                       -> DT, CS
 //   chunk_state_kernel  per (chunk, head): sum exp(cs_last-cs_j) dt_j x_j B_j^T and
 //                       sum exp(cs_i) g_i C_i^T                                   -> SP, LM
-//   state_pass_kernel   per head: forward scan of SP into the entering states,
-//                       reverse scan of LM into the leaving adjoints, F per chunk,
-//                       d_init_state
-//   chunk_bwd_kernel    per (chunk, group), heads in turn: dz, ddt, the post-conv
-//                       gradients of x (per head) and of B, C (summed over the group)
+//   state_pass_kernel   per head (4 CTAs, one slice of the state each): forward scan of
+//                       SP into the entering states, reverse scan of LM into the leaving
+//                       adjoints, F per chunk (4 partial sums), d_init_state
+//   chunk_bwd_kernel    per (chunk, group, half of the group's heads), heads in turn: dz,
+//                       ddt, the post-conv gradients of x (per head) and of B, C (summed
+//                       over the half; the conv backward adds the two halves)
 //   conv_bwd_kernel     per (channel, 64-token tile): through SiLU' and the taps to
 //                       the pre-conv gradients, per-tile conv_w/conv_b partial sums,
 //                       d_init_conv_state
@@ -67,6 +68,7 @@ constexpr int kQ = 64;    // backward chunk (tokens); also the conv backward's t
 constexpr int kT = 256;   // threads per block
 constexpr int kP = 64;    // head dimension
 constexpr int kS = kQ + 1;  // padded row stride of the 64-wide shared tiles
+constexpr int kSplit = 4;   // CTAs per head in the chunk-to-chunk state scans
 
 struct Ws {
     float* U;   // [batch][L][conv_dim]  post-conv, post-SiLU channels
@@ -75,27 +77,32 @@ struct Ws {
     float* CS;  // [batch][H][L]         in-chunk inclusive cumsum of dt*A
     float* SP;  // [batch][nc][H][P][N]  chunk-local states, then the states entering each chunk
     float* LM;  // [batch][nc][H][P][N]  chunk-local adjoints, then the adjoints leaving each chunk
-    float* PF;  // [batch][nc][H]        F = exp(cs_last) <Lm, Sp>
+    float* PF;  // [batch][nc][H][kSplit]  F = exp(cs_last) <Lm, Sp>, in kSplit partial sums
     float* PH;  // [batch][nc][H][3]     per-chunk partial dA, dD, ddt_bias
     float* PW;  // [batch][ntile][conv_dim][5]  per-tile partial dconv_w (4), dconv_b
+    float* DU2; // [batch][L][2 G N]     dB | dC of the second half of each group's heads (when split)
 };
 
 namespace {
 
 __host__ __device__ inline int64_t nchunks(int64_t L) { return (L + kQ - 1) / kQ; }
 __host__ __device__ inline int64_t ntiles(int64_t L) { return L > 0 ? nchunks(L) : 1; }
+// CTAs per (chunk, group) in the chunk backward: the group's heads in two halves when there are two or more
+__host__ __device__ inline int head_split(int H, int G) { return H / G >= 2 ? 2 : 1; }
 inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Carves the workspace; returns the bytes used (base may be null to only count).
 size_t carve(int64_t batch, int64_t L, int H, int P, int N, int G, char* base, Ws* ws) {
     const int64_t conv_dim = (int64_t)H * P + 2LL * G * N, nc = nchunks(L), nt = ntiles(L);
-    const size_t sizes[9] = {
+    const size_t sizes[10] = {
         (size_t)(batch * L * conv_dim), (size_t)(batch * L * conv_dim), (size_t)(batch * H * L),
         (size_t)(batch * H * L),        (size_t)(batch * nc * H * P * N), (size_t)(batch * nc * H * P * N),
-        (size_t)(batch * nc * H),       (size_t)(batch * nc * H * 3),     (size_t)(batch * nt * conv_dim * 5)};
-    float** slots[9] = {&ws->U, &ws->DU, &ws->DT, &ws->CS, &ws->SP, &ws->LM, &ws->PF, &ws->PH, &ws->PW};
+        (size_t)(batch * nc * H * kSplit), (size_t)(batch * nc * H * 3),  (size_t)(batch * nt * conv_dim * 5),
+        (size_t)(batch * L * 2 * G * N)};
+    float** slots[10] = {&ws->U,  &ws->DU, &ws->DT, &ws->CS, &ws->SP,
+                         &ws->LM, &ws->PF, &ws->PH, &ws->PW, &ws->DU2};
     size_t off = 0;
-    for (int k = 0; k < 9; ++k) {
+    for (int k = 0; k < 10; ++k) {
         if (base) *slots[k] = reinterpret_cast<float*>(base + off);
         off += round256(sizes[k] * sizeof(float));
     }
@@ -279,47 +286,87 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return total;
 }
 
-// grid (H, batch), kT threads; each thread owns P*N/kT state elements of one head.
+// grid (H * kSplit, batch), kT threads: the P*N state elements of a head in kSplit contiguous slices,
+// P*N / (kSplit * kT) per thread.  The forward scan turns SP into the states entering each chunk, the
+// reverse scan turns LM into the adjoints leaving each chunk and leaves each slice's part of F; the next
+// chunk's values are loaded before the current chunk's are stored, so the loads of consecutive chunks
+// overlap.
 template <int N>
 __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
-    constexpr int M = kP * N / kT;
+    constexpr int M = kP * N / (kSplit * kT);
+    constexpr int SLICE = kP * N / kSplit;
     const int64_t nc = nchunks(a.L), b = blockIdx.y;
-    const int h = blockIdx.x, tid = threadIdx.x;
+    const int h = blockIdx.x / kSplit, sp = blockIdx.x % kSplit, tid = threadIdx.x;
     float* red = reinterpret_cast<float*>(SSD_DYN_SMEM());
-    const int64_t head = (b * a.H + h) * (int64_t)kP * N;
+    const int64_t head = (b * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
+    const float* csh = ws.CS + (b * a.H + h) * a.L;
 
-    float s[M], l[M];
+    float s[M], cur[M], nxt[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) s[m] = a.init_state ? a.init_state[head + tid + kT * m] : 0.f;
+    for (int m = 0; m < M; ++m) {
+        s[m] = a.init_state ? a.init_state[head + tid + kT * m] : 0.f;
+        cur[m] = 0.f;
+        nxt[m] = 0.f;
+    }
+    if (nc > 0) {
+        const int64_t base = ((b * nc) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
+#pragma unroll
+        for (int m = 0; m < M; ++m) cur[m] = ws.SP[base + tid + kT * m];
+    }
     for (int64_t c = 0; c < nc; ++c) {
         const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
-        const float decay = expf(ws.CS[(b * a.H + h) * a.L + last]);
-        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
+        const float decay = expf(csh[last]);
+        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
+        if (c + 1 < nc) {
+            const int64_t nb = base + (int64_t)a.H * kP * N;
+#pragma unroll
+            for (int m = 0; m < M; ++m) nxt[m] = ws.SP[nb + tid + kT * m];
+        }
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            const int64_t i = base + tid + kT * m;
-            const float loc = ws.SP[i];
-            ws.SP[i] = s[m];
-            s[m] = decay * s[m] + loc;
+            ws.SP[base + tid + kT * m] = s[m];
+            s[m] = decay * s[m] + cur[m];
+            cur[m] = nxt[m];
         }
     }
+
+    float l[M], sp_cur[M], sp_nxt[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) l[m] = a.d_final ? a.d_final[head + tid + kT * m] : 0.f;
+    for (int m = 0; m < M; ++m) {
+        l[m] = a.d_final ? a.d_final[head + tid + kT * m] : 0.f;
+        cur[m] = nxt[m] = sp_cur[m] = sp_nxt[m] = 0.f;
+    }
+    if (nc > 0) {
+        const int64_t base = ((b * nc + nc - 1) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            cur[m] = ws.LM[base + tid + kT * m];
+            sp_cur[m] = ws.SP[base + tid + kT * m];
+        }
+    }
     for (int64_t c = nc - 1; c >= 0; --c) {
         const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
-        const float decay = expf(ws.CS[(b * a.H + h) * a.L + last]);
-        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
+        const float decay = expf(csh[last]);
+        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
+        if (c > 0) {
+            const int64_t pb = base - (int64_t)a.H * kP * N;
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                nxt[m] = ws.LM[pb + tid + kT * m];
+                sp_nxt[m] = ws.SP[pb + tid + kT * m];
+            }
+        }
         float f = 0.f;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            const int64_t i = base + tid + kT * m;
-            const float loc = ws.LM[i];
-            ws.LM[i] = l[m];
-            f += l[m] * ws.SP[i];
-            l[m] = decay * l[m] + loc;
+            ws.LM[base + tid + kT * m] = l[m];
+            f += l[m] * sp_cur[m];
+            l[m] = decay * l[m] + cur[m];
+            cur[m] = nxt[m];
+            sp_cur[m] = sp_nxt[m];
         }
         f = block_sum(f, red);
-        if (tid == 0) ws.PF[(b * nc + c) * a.H + h] = decay * f;
+        if (tid == 0) ws.PF[((b * nc + c) * a.H + h) * kSplit + sp] = decay * f;
     }
     if (a.d_init_state) {
 #pragma unroll
@@ -347,7 +394,9 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     constexpr int RS = 17;         // row stride of the per-row partial sums
     const int64_t nc = nchunks(a.L), HP = (int64_t)a.H * kP, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
     const int64_t c = blockIdx.x, b = blockIdx.z, t0 = c * kQ;
-    const int g = blockIdx.y, hpg = a.H / a.G, tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    const int hpg = a.H / a.G, split = head_split(a.H, a.G), tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    const int g = blockIdx.y / split, half = blockIdx.y % split;
+    const int hl0 = half * hpg / split, hl1 = (half + 1) * hpg / split;  // this CTA's heads of the group
     const int Qv = static_cast<int>(a.L - t0 < kQ ? a.L - t0 : kQ);
 
     float* sm = reinterpret_cast<float*>(SSD_DYN_SMEM());
@@ -397,7 +446,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     tile_zero(dBa);
     tile_zero(dCa);
 
-    for (int hl = 0; hl < hpg; ++hl) {
+    for (int hl = hl0; hl < hl1; ++hl) {
         const int h = g * hpg + hl;
         const float Dh = a.D[h], Ah = a.A[h], bias = a.dt_bias[h];
         const int64_t hrow = (b * a.H + h) * a.L + t0;
@@ -569,7 +618,9 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         __syncthreads();
 
         // 7: d(dA_k) = sum_{i>=k} sum_{j<k} M_ij + sum_{i>=k} E_i + F + sum_{j<k} dt_j W_j; ddt; partials
-        const float F = ws.PF[(b * nc + c) * a.H + h];
+        float F = 0.f;
+#pragma unroll
+        for (int k = 0; k < kSplit; ++k) F += ws.PF[((b * nc + c) * a.H + h) * kSplit + k];
         float pdA = 0.f, pbias = 0.f;
         if (tid < Qv) {
             const int k = tid;
@@ -597,15 +648,18 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         __syncthreads();
     }
 
+    // this half's dB | dC: the first half into the B/C part of DU, the second into DU2; the conv
+    // backward adds the two in that order
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int j = ty + 16 * r;
         if (j < Qv) {
-            const int64_t row = (b * a.L + t0 + j) * conv_dim;
+            float* dst = half == 0 ? ws.DU + (b * a.L + t0 + j) * conv_dim + HP
+                                   : ws.DU2 + (b * a.L + t0 + j) * 2 * GN;
 #pragma unroll
             for (int q = 0; q < TN; ++q) {
-                ws.DU[row + HP + (int64_t)g * N + tx + 16 * q] = dBa[r][q];
-                ws.DU[row + HP + GN + (int64_t)g * N + tx + 16 * q] = dCa[r][q];
+                dst[(int64_t)g * N + tx + 16 * q] = dBa[r][q];
+                dst[GN + (int64_t)g * N + tx + 16 * q] = dCa[r][q];
             }
         }
     }
@@ -631,6 +685,7 @@ __global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
     } else {
         out = a.dC, ostride = GN, ocol = c - HP - GN;
     }
+    const bool two_halves = head_split(a.H, a.G) == 2;
     float r0 = raw_at(a, b, t0 - 3, c), r1 = raw_at(a, b, t0 - 2, c), r2 = raw_at(a, b, t0 - 1, c);
     float d1 = 0.f, d2 = 0.f, d3 = 0.f;  // dv at t-1, t-2, t-3 (zero before token 0)
     float gw0 = 0.f, gw1 = 0.f, gw2 = 0.f, gw3 = 0.f, gb = 0.f;
@@ -639,7 +694,9 @@ __global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
         if (t < a.L) {
             const float r3 = raw_at(a, b, t, c);
             const float v = bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * r3;
-            dv = ws.DU[(b * a.L + t) * conv_dim + c] * dsilu_f(v);
+            float du = ws.DU[(b * a.L + t) * conv_dim + c];
+            if (c >= HP && two_halves) du += ws.DU2[(b * a.L + t) * 2 * GN + (c - HP)];
+            dv = du * dsilu_f(v);
             if (t < t1) {
                 gw0 += dv * r0;
                 gw1 += dv * r1;
@@ -721,9 +778,10 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
                    dim3(kT), 0, st, a, ws);
         const dim3 chunk_heads(static_cast<unsigned>(nc), static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
         SSD_LAUNCH(chunk_state_kernel<N>, chunk_heads, dim3(kT), state_smem, st, a, ws);
-        SSD_LAUNCH(state_pass_kernel<N>, dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch)), dim3(kT),
-                   kT * sizeof(float), st, a, ws);
-        const dim3 chunk_groups(static_cast<unsigned>(nc), static_cast<unsigned>(a.G), static_cast<unsigned>(a.batch));
+        SSD_LAUNCH(state_pass_kernel<N>, dim3(static_cast<unsigned>(a.H * kSplit), static_cast<unsigned>(a.batch)),
+                   dim3(kT), kT * sizeof(float), st, a, ws);
+        const dim3 chunk_groups(static_cast<unsigned>(nc), static_cast<unsigned>(a.G * head_split(a.H, a.G)),
+                                static_cast<unsigned>(a.batch));
 #ifndef SSD_EMU
         if (a.ev_before) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_before), st);
 #endif
