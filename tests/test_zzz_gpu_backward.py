@@ -62,6 +62,7 @@ CASES = [
     (1, 129, 4, 4, 32, torch.float32, False, False),    # 1-token last chunk, zero states
     (1, 512, 16, 2, 128, torch.bfloat16, True, True),   # the production d_state, 8 chunks
     (3, 64, 2, 1, 16, torch.float32, True, True),       # exactly one chunk per sequence
+    (1, 100, 6, 2, 32, torch.bfloat16, True, True),     # three heads per group: uneven halves
 ]
 
 
