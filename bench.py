@@ -380,6 +380,37 @@ def cpu_baseline(inp, d: Dims, budget_s: float):
                       f"tokens/s = pairs x L / H / seconds"}
 
 
+def cpu_backward_baseline(d: Dims, act):
+    """The oracle's backward timed on one group of the prefill workload's layer (H/G heads, all L tokens,
+    the same per-head shapes), reported as tokens/s of the whole layer: one group is 1/G of the work."""
+    import oracle
+    sub = Dims(d.batch, d.seqlen, d.nheads // d.ngroups, d.headdim, d.d_state, 1, d.chunk)
+    inp = make_prefill_inputs(sub, dtype=act, seed=seed_of(PREFILL_WORKLOAD) + 7)
+    gr = make_backward_grads(sub, dtype=act, seed=seed_of(PREFILL_WORKLOAD) + 8)
+    t0 = time.perf_counter()
+    oracle.prefill_backward(inp, gr["dy"], gr["d_final"])
+    el = time.perf_counter() - t0
+    tokens = d.batch * d.seqlen / d.ngroups
+    return {"value": tokens / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"one group ({sub.nheads} of {d.nheads} heads, {d.seqlen} tokens) of the {PREFILL_WORKLOAD} "
+                      f"layer, fp64 adjoint of the token recurrence, {el:.1f} s; tokens/s = L / G / seconds"}
+
+
+def cpu_mimo_baseline(d: Dims, act, nseq: int = 16):
+    """The oracle's MIMO step timed on ``nseq`` of the decode workload's sequences, as GB/s of the
+    step's algorithmic bytes for those sequences."""
+    import oracle
+    sub = Dims(nseq, 1, d.nheads, d.headdim, d.d_state, d.ngroups, d.chunk)
+    data = make_mimo_decode_inputs(sub, MIMO_RANK, 1, dtype=act, seed=seed_of(DECODE_WORKLOAD) + 5)
+    state = data["ssm_state"].double().numpy().copy()
+    t0 = time.perf_counter()
+    oracle.mimo_decode_step(data["steps"][0], data["params"], state)
+    el = time.perf_counter() - t0
+    nbytes = mimo_decode_bytes(sub, MIMO_RANK, 2 if act == torch.bfloat16 else 4)
+    return {"value": nbytes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{nseq} of the {d.batch} sequences of one step, rank {MIMO_RANK}, fp64, {el:.2f} s"}
+
+
 # ---------------------------------------------------------------------------------------------------------
 
 def run_reference(args):
@@ -720,6 +751,11 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(inp, d, args.cpu_seconds)
+        if backward is not None and "error" not in backward:
+            backward["cpu_baseline"] = cpu_backward_baseline(d, act)
+        if mimo is not None and "error" not in mimo:
+            wd = WORKLOADS[DECODE_WORKLOAD]
+            mimo["cpu_baseline"] = cpu_mimo_baseline(wd["dims"], wd["dtype"])
 
     if rank == 0:
         line = {

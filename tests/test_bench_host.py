@@ -145,3 +145,12 @@ def test_backward_and_mimo_bench_legs_on_a_fake_device(monkeypatch):
     assert fake.calls["mimo"] == 3 + 4
     assert abs(m["value"] - bench.mimo_decode_bytes(d, bench.MIMO_RANK, 2) / 2e-3 / 1e9) < 1e-6
     assert m["roofline"]["frac"] == m["roofline"]["achieved"] / 6554.6
+
+
+def test_oracle_baselines_of_the_backward_and_mimo_lines():
+    from selective_state_space_43_b200.synth import Dims
+    d = Dims(1, 96, 4, 64, 16, 2, 64)
+    b = bench.cpu_backward_baseline(d, torch.bfloat16)
+    assert b["kind"] == "oracle" and b["unit"] == "tokens/s" and b["value"] > 0 and "2 of 4 heads" in b["sample"]
+    m = bench.cpu_mimo_baseline(Dims(4, 1, 4, 64, 16, 2, 64), torch.bfloat16, nseq=2)
+    assert m["kind"] == "oracle" and m["unit"] == "GB/s" and m["value"] > 0
