@@ -560,12 +560,100 @@ def set_timing_events(before, after):
         raise SsdError(st, "ssd_set_timing_events")
 
 
-def prefill_host(inputs: dict, chunk=128, device="cuda", stream=None):
-    """End-to-end prefill from HOST tensors: copies the inputs to the device
-    (pinned memory -> HBM, asynchronous), runs ssd_prefill and copies y,
-    final_state and conv_state back into pinned host tensors.  Returns the
-    host outputs and the number of bytes moved each way."""
+_side_streams = {}
+
+
+def _host_streams(dev):
+    """Two side streams per device (host->device copies, device->host copies), created once."""
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _side_streams:
+        _side_streams[key] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    return _side_streams[key]
+
+
+def host_pieces(L: int, chunk: int, segments=None) -> list:
+    """Row ranges [r0, r1) of the pieces prefill_host cuts a sequence of L tokens into: ``segments`` pieces
+    (default: as many as fit at two chunks each, at most 8) of equal length rounded up to whole chunks,
+    the last one shorter; one piece when L fits in one."""
+    if segments is None:
+        segments = max(1, min(8, L // (2 * chunk)))
+    seg = -(-L // max(1, int(segments)))
+    seg = max(chunk, -(-seg // chunk) * chunk)
+    return [(r0, min(L, r0 + seg)) for r0 in range(0, L, seg)] if L > 0 else [(0, 0)]
+
+
+def prefill_host(inputs: dict, chunk=128, device="cuda", stream=None, segments=None):
+    """End-to-end prefill from HOST tensors (pinned for asynchronous copies): the inputs go to the device,
+    ssd_prefill runs, and y, final_state and conv_state come back into pinned host tensors.
+
+    The sequence is cut into ``segments`` pieces on chunk boundaries (default: up to 8 pieces of at least
+    two chunks).  Piece k is copied in on one side stream while piece k-1 is scanned on the current stream
+    and piece k-2's y is copied out on another, so the two copy directions and the scan overlap.  Each piece
+    starts from the states the previous one left (final_state and conv_state as init_state and
+    init_conv_state), which on chunk boundaries gives the same values as one call over the whole sequence.
+    The current stream waits for every copy before the call returns, so events recorded on it around the
+    call time the whole transfer.  Returns ([y, final_state, conv_state] on the host, bytes in, bytes out).
+    """
     dev = torch.device(device)
+    x = inputs["x"]
+    Bt, L = x.shape[0], x.shape[1]
+    h2d = sum(t.numel() * t.element_size() for t in inputs.values() if t is not None)
+    pieces = host_pieces(L, chunk, segments)
+    if len(pieces) <= 1:
+        return _prefill_host_whole(inputs, chunk, dev, h2d)
+
+    cur = torch.cuda.current_stream(dev)
+    s_in, s_out = _host_streams(dev)
+    s_in.wait_stream(cur)
+    s_out.wait_stream(cur)
+    names = ("A", "D", "dt_bias", "conv_w", "conv_b", "init_state", "init_conv_state")
+    with torch.cuda.stream(s_in):
+        p = {k: (None if inputs.get(k) is None else inputs[k].to(dev, non_blocking=True)) for k in names}
+    for t in p.values():
+        if t is not None:
+            t.record_stream(cur)
+    y_host = torch.empty(tuple(x.shape), dtype=x.dtype, pin_memory=True)
+    fs_prev, cs_prev = p["init_state"], p["init_conv_state"]
+    for r0, r1 in pieces:
+        with torch.cuda.stream(s_in):
+            d = {}
+            for k in ("x", "dt", "B", "C", "z"):
+                h = inputs[k]
+                t = torch.empty((Bt, r1 - r0) + tuple(h.shape[2:]), dtype=h.dtype, device=dev)
+                for b in range(Bt):
+                    t[b].copy_(h[b, r0:r1], non_blocking=True)
+                d[k] = t
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+        cur.wait_event(ready)
+        for t in d.values():
+            t.record_stream(cur)
+        y, fs, cs = prefill(d["x"], d["dt"], d["B"], d["C"], d["z"], p["A"], p["D"], p["dt_bias"], p["conv_w"],
+                            p["conv_b"], fs_prev, cs_prev, chunk=chunk)
+        done = torch.cuda.Event()
+        done.record(cur)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            for b in range(Bt):
+                y_host[b, r0:r1].copy_(y[b], non_blocking=True)
+        y.record_stream(s_out)
+        fs_prev, cs_prev = fs, cs
+    fs_host = torch.empty(tuple(fs_prev.shape), dtype=fs_prev.dtype, pin_memory=True)
+    cs_host = torch.empty(tuple(cs_prev.shape), dtype=cs_prev.dtype, pin_memory=True)
+    with torch.cuda.stream(s_out):
+        fs_host.copy_(fs_prev, non_blocking=True)
+        cs_host.copy_(cs_prev, non_blocking=True)
+    fs_prev.record_stream(s_out)
+    cs_prev.record_stream(s_out)
+    out_done = torch.cuda.Event()
+    out_done.record(s_out)
+    cur.wait_event(out_done)
+    outs = [y_host, fs_host, cs_host]
+    return outs, h2d, sum(t.numel() * t.element_size() for t in outs)
+
+
+def _prefill_host_whole(inputs: dict, chunk, dev, h2d):
+    """prefill_host in one piece on the current stream: copy in, scan, copy out."""
     names = ("x", "dt", "B", "C", "z", "A", "D", "dt_bias", "conv_w", "conv_b", "init_state", "init_conv_state")
     d = {k: (None if inputs.get(k) is None else inputs[k].to(dev, non_blocking=True)) for k in names}
     y, fs, cs = prefill(d["x"], d["dt"], d["B"], d["C"], d["z"], d["A"], d["D"], d["dt_bias"], d["conv_w"],
@@ -573,6 +661,4 @@ def prefill_host(inputs: dict, chunk=128, device="cuda", stream=None):
     outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (y, fs, cs)]
     for o, t in zip(outs, (y, fs, cs)):
         o.copy_(t, non_blocking=True)
-    h2d = sum(t.numel() * t.element_size() for t in inputs.values() if t is not None)
-    d2h = sum(t.numel() * t.element_size() for t in outs)
-    return outs, h2d, d2h
+    return outs, h2d, sum(t.numel() * t.element_size() for t in outs)

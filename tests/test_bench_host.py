@@ -154,3 +154,18 @@ def test_oracle_baselines_of_the_backward_and_mimo_lines():
     assert b["kind"] == "oracle" and b["unit"] == "tokens/s" and b["value"] > 0 and "2 of 4 heads" in b["sample"]
     m = bench.cpu_mimo_baseline(Dims(4, 1, 4, 64, 16, 2, 64), torch.bfloat16, nseq=2)
     assert m["kind"] == "oracle" and m["unit"] == "GB/s" and m["value"] > 0
+
+
+def test_host_prefill_pieces():
+    from selective_state_space_43_b200.ops import host_pieces
+    assert host_pieces(4096, 128) == [(r, r + 512) for r in range(0, 4096, 512)]   # 8 pieces of 4 chunks
+    assert host_pieces(1000, 128, 3) == [(0, 384), (384, 768), (768, 1000)]       # rounded up to chunks
+    assert host_pieces(300, 128) == [(0, 300)]                                       # one piece
+    assert host_pieces(300, 128, 8) == [(0, 128), (128, 256), (256, 300)]
+    assert host_pieces(0, 128) == [(0, 0)]
+    for L in (1, 127, 129, 777, 5000):
+        for segs in (None, 1, 2, 5, 9):
+            p = host_pieces(L, 64, segs)
+            assert p[0][0] == 0 and p[-1][1] == L
+            assert all(a[1] == b[0] for a, b in zip(p, p[1:]))
+            assert all(r0 % 64 == 0 for r0, _ in p)                                 # chunk-aligned starts
