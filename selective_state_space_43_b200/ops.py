@@ -582,7 +582,7 @@ def host_pieces(L: int, chunk: int, segments=None) -> list:
     return [(r0, min(L, r0 + seg)) for r0 in range(0, L, seg)] if L > 0 else [(0, 0)]
 
 
-def prefill_host(inputs: dict, chunk=128, device="cuda", stream=None, segments=None):
+def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None):
     """End-to-end prefill from HOST tensors (pinned for asynchronous copies): the inputs go to the device,
     ssd_prefill runs, and y, final_state and conv_state come back into pinned host tensors.
 
