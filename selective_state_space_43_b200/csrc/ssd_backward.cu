@@ -67,7 +67,8 @@ namespace bwd {
 constexpr int kQ = 64;    // backward chunk (tokens); also the conv backward's tile
 constexpr int kT = 256;   // threads per block
 constexpr int kP = 64;    // head dimension
-constexpr int kS = kQ + 1;  // padded row stride of the 64-wide shared tiles
+constexpr int kS = kQ + 4;  // row stride of the 64-wide shared tiles: a multiple of 4 floats (16-byte rows)
+constexpr int kTS = kQ + 1; // row stride of the prefix-sum tile (written row by row, one row per thread)
 constexpr int kSplit = 4;   // CTAs per head in the chunk-to-chunk state scans
 
 struct Ws {
@@ -189,6 +190,58 @@ __device__ __forceinline__ void tile_mma(float (&acc)[TM][TN], const float* A, i
         for (int r = 0; r < TM; ++r)
 #pragma unroll
             for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+}
+
+// 16-byte shared load (the address must be 16-byte aligned; the host emulation checks it).
+__device__ __forceinline__ float4 lds4(const float* p) {
+#ifdef SSD_EMU
+    emu_check_aligned(p, 16);
+#endif
+    return *reinterpret_cast<const float4*>(p);
+}
+
+__device__ __forceinline__ float f4c(const float4& v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+// tile_mma for A and B both contiguous along k (sak = sbk = 1), four k per 16-byte load of each:
+// per four k, TM + TN loads (a warp's A loads: two rows, one wavefront; its B loads: 16 rows, two
+// wavefronts) for 4 TM TN FMAs.  K a multiple of 4; rows and the bases 16-byte aligned.
+template <int TM, int TN>
+__device__ __forceinline__ void tile_mma_kk(float (&acc)[TM][TN], const float* A, int sam, const float* B, int sbn,
+                                            int K, int ty, int tx) {
+    for (int k = 0; k < K; k += 4) {
+        float4 av[TM], bv[TN];
+#pragma unroll
+        for (int r = 0; r < TM; ++r) av[r] = lds4(A + (ty + 16 * r) * sam + k);
+#pragma unroll
+        for (int c = 0; c < TN; ++c) bv[c] = lds4(B + (tx + 16 * c) * sbn + k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int r = 0; r < TM; ++r)
+#pragma unroll
+                for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(f4c(av[r], i), f4c(bv[c], i), acc[r][c]);
+    }
+}
+
+// tile_mma for A contiguous along k (sak = 1), B any: A four k per 16-byte load, B scalar.
+template <int TM, int TN>
+__device__ __forceinline__ void tile_mma_ak(float (&acc)[TM][TN], const float* A, int sam, const float* B, int sbn,
+                                            int sbk, int K, int ty, int tx) {
+    for (int k = 0; k < K; k += 4) {
+        float4 av[TM];
+#pragma unroll
+        for (int r = 0; r < TM; ++r) av[r] = lds4(A + (ty + 16 * r) * sam + k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float bv[TN];
+#pragma unroll
+            for (int c = 0; c < TN; ++c) bv[c] = B[(tx + 16 * c) * sbn + (k + i) * sbk];
+#pragma unroll
+            for (int r = 0; r < TM; ++r)
+#pragma unroll
+                for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(f4c(av[r], i), bv[c], acc[r][c]);
+        }
     }
 }
 
@@ -376,10 +429,10 @@ __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
 
 template <int N>
 constexpr size_t chunk_bwd_floats() {
-    // Bs, Cs [kQ][N+1]; CB, LCB, LGX, Tm, xs, gs [kQ][kS]; X [kP][N+1]; red [kQ][17]; 7 vectors of kQ;
-    // 3 x kT block sums
-    return 2 * (size_t)kQ * (N + 1) + 6 * (size_t)kQ * kS + (size_t)kP * (N + 1) + (size_t)kQ * 17 +
-           7 * (size_t)kQ + 3 * (size_t)kT;
+    // Bs, Cs [kQ][N+4]; CB, LCB, LGX, xs, gs [kQ][kS]; Tm [kQ][kTS] (+3 to keep 16-byte alignment);
+    // X [kP][N+4]; red [kQ][17] (+4); 7 vectors of kQ; 3 x kT block sums
+    return 2 * (size_t)kQ * (N + 4) + 5 * (size_t)kQ * kS + ((size_t)kQ * kTS + 3) / 4 * 4 + (size_t)kP * (N + 4) +
+           ((size_t)kQ * 17 + 3) / 4 * 4 + 7 * (size_t)kQ + 3 * (size_t)kT;
 }
 
 // grid (nchunks, G, batch), kT threads.  One chunk of one group; the group's heads in turn.  The
@@ -389,7 +442,7 @@ constexpr size_t chunk_bwd_floats() {
 // diagonal.
 template <int N>
 __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
-    constexpr int NS = N + 1;      // padded row stride of the N-wide tiles
+    constexpr int NS = N + 4;      // row stride of the N-wide tiles (16-byte rows)
     constexpr int TN = N / 16;     // columns per thread of the N-wide results
     constexpr int RS = 17;         // row stride of the per-row partial sums
     const int64_t nc = nchunks(a.L), HP = (int64_t)a.H * kP, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
@@ -398,6 +451,8 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     const int g = blockIdx.y / split, half = blockIdx.y % split;
     const int hl0 = half * hpg / split, hl1 = (half + 1) * hpg / split;  // this CTA's heads of the group
     const int Qv = static_cast<int>(a.L - t0 < kQ ? a.L - t0 : kQ);
+    // causal sums over the chunk's rows, rounded up to whole 16-byte loads: the operands are zero past Qv
+    const int Q4 = (Qv + 3) & ~3;
 
     float* sm = reinterpret_cast<float*>(SSD_DYN_SMEM());
     float* Bs = sm;                  // [kQ][NS]  post-conv B of the group
@@ -405,12 +460,12 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     float* CB = Cs + kQ * NS;        // [kQ][kS]  C_i . B_j
     float* LCB = CB + kQ * kS;       // [kQ][kS]  L_ij dt_j C_i . B_j         (i >= j, else 0)
     float* LGX = LCB + kQ * kS;      // [kQ][kS]  L_ij g_i . x_j, then times dt_j (i >= j, else 0)
-    float* Tm = LGX + kQ * kS;       // [kQ][kS]  row prefix sums of M
-    float* xs = Tm + kQ * kS;        // [kQ][kS]  post-conv x of the head
+    float* xs = LGX + kQ * kS;       // [kQ][kS]  post-conv x of the head
     float* gs = xs + kQ * kS;        // [kQ][kS]  g = dy * silu(z)
     float* X = gs + kQ * kS;         // [kP][NS]  Sp, then Lm
-    float* red = X + kP * NS;        // [kQ][RS]  per-row partial sums over the 16 column threads
-    float* dts = red + kQ * RS;      // [kQ]
+    float* Tm = X + kP * NS;         // [kQ][kTS] row prefix sums of M
+    float* red = Tm + (kQ * kTS + 3) / 4 * 4;    // [kQ][RS]  per-row partial sums over the 16 column threads
+    float* dts = red + (kQ * RS + 3) / 4 * 4;    // [kQ]
     float* css = dts + kQ;
     float* ex = css + kQ;            // exp(cs_i)
     float* el = ex + kQ;             // exp(cs_last - cs_j)
@@ -435,7 +490,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     {
         float acc[4][4];
         tile_zero(acc);
-        tile_mma(acc, Cs, NS, 1, Bs, NS, 1, N, ty, tx);
+        tile_mma_kk(acc, Cs, NS, Bs, NS, N, ty, tx);
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -480,7 +535,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         {
             float acc[4][4];
             tile_zero(acc);
-            tile_mma(acc, gs, kS, 1, xs, kS, 1, kP, ty, tx);
+            tile_mma_kk(acc, gs, kS, xs, kS, kP, ty, tx);
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -511,8 +566,8 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             float spc[4][4], yin[4][4];
             tile_zero(spc);
             tile_zero(yin);
-            tile_mma(spc, Cs, NS, 1, X, NS, 1, N, ty, tx);       // [i][p] = sum_n C_i[n] Sp[p][n]
-            tile_mma(yin, LCB, kS, 1, xs, 1, kS, Qv, ty, tx);    // [i][p] = sum_j LCB[i][j] x_j[p]
+            tile_mma_kk(spc, Cs, NS, X, NS, N, ty, tx);            // [i][p] = sum_n C_i[n] Sp[p][n]
+            tile_mma_ak(yin, LCB, kS, xs, 1, kS, Q4, ty, tx);      // [i][p] = sum_j LCB[i][j] x_j[p]
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 const int i = ty + 16 * r;
@@ -535,7 +590,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         {
             float acc[4][TN];
             tile_zero(acc);
-            tile_mma(acc, gs, kS, 1, X, 1, NS, kP, ty, tx);      // [i][n] = sum_p g_i[p] Sp[p][n]
+            tile_mma_ak(acc, gs, kS, X, 1, NS, kP, ty, tx);        // [i][n] = sum_p g_i[p] Sp[p][n]
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -559,7 +614,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             float lmb[4][4], dxi[4][4];
             tile_zero(lmb);
             tile_zero(dxi);
-            tile_mma(lmb, Bs, NS, 1, X, NS, 1, N, ty, tx);       // [j][p] = sum_n B_j[n] Lm[p][n]
+            tile_mma_kk(lmb, Bs, NS, X, NS, N, ty, tx);            // [j][p] = sum_n B_j[n] Lm[p][n]
             tile_mma(dxi, LCB, 1, kS, gs, 1, kS, Qv, ty, tx);    // [j][p] = sum_i LCB[i][j] g_i[p]
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -580,7 +635,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         {
             float acc[4][TN];
             tile_zero(acc);
-            tile_mma(acc, xs, kS, 1, X, 1, NS, kP, ty, tx);      // [j][n] = sum_p x_j[p] Lm[p][n]
+            tile_mma_ak(acc, xs, kS, X, 1, NS, kP, ty, tx);        // [j][n] = sum_p x_j[p] Lm[p][n]
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 const int j = ty + 16 * r;
@@ -594,7 +649,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
 #pragma unroll
                 for (int q = 0; q < TN; ++q) dBa[r][q] += acc[r][q];
             tile_zero(acc);
-            tile_mma(acc, LGX, kS, 1, Bs, 1, NS, Qv, ty, tx);    // [i][n] = sum_j LGX[i][j] dt_j B_j[n]
+            tile_mma_ak(acc, LGX, kS, Bs, 1, NS, Q4, ty, tx);      // [i][n] = sum_j LGX[i][j] dt_j B_j[n]
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -611,7 +666,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             Dr[tid] += w;
             float run = 0.f;
             for (int k = 0; k <= tid; ++k) {
-                Tm[tid * kS + k] = run;
+                Tm[tid * kTS + k] = run;
                 run += LGX[tid * kS + k] * CB[tid * kS + k];
             }
         }
@@ -626,7 +681,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             const int k = tid;
             float R = 0.f, Es = 0.f, Wsum = 0.f;
             for (int i = k; i < Qv; ++i) {
-                R += Tm[i * kS + k];
+                R += Tm[i * kTS + k];
                 Es += Ev[i];
             }
             for (int j = 0; j < k; ++j) Wsum += dts[j] * Wv[j];

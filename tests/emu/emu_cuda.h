@@ -11,6 +11,8 @@
 
 #include <math.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <barrier>
@@ -93,6 +95,14 @@ void launch(dim3 grid, dim3 block, size_t smem_bytes, F&& body) {
 #define gridDim (::emu::g_grid)
 
 inline void __syncthreads() { ::emu::ctx.bar->arrive_and_wait(); }
+
+// Vector accesses must be aligned to their size on the GPU; the host would not fault, so check here.
+inline void emu_check_aligned(const void* p, unsigned bytes) {
+    if (reinterpret_cast<uintptr_t>(p) % bytes) {
+        fprintf(stderr, "emu: misaligned %u-byte access at %p\n", bytes, p);
+        abort();
+    }
+}
 inline float __uint_as_float(unsigned u) {
     float f;
     memcpy(&f, &u, 4);

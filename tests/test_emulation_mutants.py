@@ -1,7 +1,8 @@
 """The host emulation of the kernels is a strong enough check: faults planted in temporary copies of
-the backward kernels' source (an access outside a buffer, a read of shared memory that was never
-written, a dropped term) each make the emulated run fail, through AddressSanitizer, through the
-NaN-filled outputs and shared memory, or through the comparison with the oracle.  CPU only; the
+the backward kernels' source (an access outside a buffer, a misaligned 16-byte shared load, a read of
+shared memory that was never written, a dropped term) each make the emulated run fail, through
+AddressSanitizer, the emulator's alignment check, the NaN-filled outputs and shared memory, or the
+comparison with the oracle.  CPU only; the
 faults are planted in copies, never in the library's source."""
 import concurrent.futures as cf
 import os
@@ -28,6 +29,8 @@ MUTANTS = {
                                           "out[(b * a.L + s + 1) * ostride + ocol] = gs;"),
     # leaves the rows of a ragged chunk past its end as they were (NaN bytes for the first head)
     "ragged rows not cleared": ("            xs[j * kS + p] = xv;", "            if (j < Qv) xs[j * kS + p] = xv;"),
+    # shared rows no longer 16-byte aligned: the emulation's alignment check must stop the vector loads
+    "unaligned shared rows": ("constexpr int kS = kQ + 4;", "constexpr int kS = kQ + 1;"),
     # drops the D skip term of dx
     "dx without the D skip": ("dts[j] * el[j] * lmb[r][q] + Dh * gs[j * kS + p];", "dts[j] * el[j] * lmb[r][q];"),
 }
