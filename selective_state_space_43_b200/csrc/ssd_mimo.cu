@@ -52,6 +52,13 @@ __device__ __forceinline__ void st_out(void* p, int64_t i, float v, bool bf16) {
     else
         static_cast<float*>(p)[i] = v;
 }
+// 16-byte shared load (the address must be 16-byte aligned; the host emulation checks it).
+__device__ __forceinline__ float4 lds4(const float* p) {
+#ifdef SSD_EMU
+    emu_check_aligned(p, 16);
+#endif
+    return *reinterpret_cast<const float4*>(p);
+}
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + __expf(-v)); }
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(__expf(v)); }
 
@@ -126,8 +133,8 @@ __global__ void __launch_bounds__(kT, (R <= 4 ? 3 : 2)) mimo_decode_kernel(MimoA
 
     // the lane's 4 columns of B_k and C_k are re-read from shared memory (16-byte loads) where they are
     // used, rather than held in 8R registers, to keep 3 CTAs per SM at R = 4
-    const float4* sB4 = reinterpret_cast<const float4*>(s_B + n0);
-    const float4* sC4 = reinterpret_cast<const float4*>(s_C + n0);
+    const float* sB4 = s_B + n0;
+    const float* sC4 = s_C + n0;
 #pragma unroll
     for (int it = 0; it < ITER; ++it) {
         const int p = (it * 8 + warp) * RPW + rsub;
@@ -135,7 +142,7 @@ __global__ void __launch_bounds__(kT, (R <= 4 ? 3 : 2)) mimo_decode_kernel(MimoA
 #pragma unroll
         for (int k = 0; k < R; ++k) {
             const float xk = s_x[k * kP + p];
-            const float4 bq = sB4[k * (N / 4)];
+            const float4 bq = lds4(sB4 + k * N);
             ix += xk * bq.x;
             iy += xk * bq.y;
             iz += xk * bq.z;
@@ -150,7 +157,7 @@ __global__ void __launch_bounds__(kT, (R <= 4 ? 3 : 2)) mimo_decode_kernel(MimoA
         float part[R];
 #pragma unroll
         for (int k = 0; k < R; ++k) {
-            const float4 cq = sC4[k * (N / 4)];
+            const float4 cq = lds4(sC4 + k * N);
             part[k] = s.x * cq.x + s.y * cq.y + s.z * cq.z + s.w * cq.w;
         }
         int first = 0, left = R;
