@@ -245,6 +245,79 @@ __device__ __forceinline__ void tile_mma_ak(float (&acc)[TM][TN], const float* A
     }
 }
 
+// Column n of a thread's c-th output column in the products whose B runs along n (N-wide results, TN =
+// N/16 columns per thread): contiguous groups of four, 4 tx .. 4 tx + 3 within each 64-column block, so
+// that the 16 column threads of a warp read 256 contiguous bytes per load (two wavefronts).  TN = 2:
+// pairs 2 tx, 2 tx + 1; TN = 1: column tx.
+template <int TN>
+__device__ __forceinline__ int ncol(int tx, int c) {
+    if constexpr (TN >= 4) return 64 * (c / 4) + 4 * tx + (c % 4);
+    else if constexpr (TN == 2) return 2 * tx + c;
+    else return tx;
+}
+
+// The TN values of row k of B (B(n, k) = B[n + k * sbk], n = ncol(tx, c)) in as few loads as the
+// layout allows: 16-byte loads for TN >= 4, 8-byte for TN = 2 (sbk a multiple of 4, base 16-byte aligned).
+template <int TN>
+__device__ __forceinline__ void load_ncols(float (&bv)[TN], const float* Bk, int tx) {
+    if constexpr (TN >= 4) {
+#pragma unroll
+        for (int h = 0; h < TN / 4; ++h) {
+            const float4 v = lds4(Bk + 64 * h + 4 * tx);
+            bv[4 * h] = v.x;
+            bv[4 * h + 1] = v.y;
+            bv[4 * h + 2] = v.z;
+            bv[4 * h + 3] = v.w;
+        }
+    } else if constexpr (TN == 2) {
+        const float* p = Bk + 2 * tx;
+#ifdef SSD_EMU
+        emu_check_aligned(p, 8);
+#endif
+        const float2 v = *reinterpret_cast<const float2*>(p);
+        bv[0] = v.x;
+        bv[1] = v.y;
+    } else {
+        bv[0] = Bk[tx];
+    }
+}
+
+// tile_mma with B running along n (columns ncol(tx, c)): A(m, k) = A[m * sam + k * sak], scalar loads.
+template <int TM, int TN>
+__device__ __forceinline__ void tile_mma_nc(float (&acc)[TM][TN], const float* A, int sam, int sak, const float* B,
+                                            int sbk, int K, int ty, int tx) {
+    for (int k = 0; k < K; ++k) {
+        float av[TM], bv[TN];
+#pragma unroll
+        for (int r = 0; r < TM; ++r) av[r] = A[(ty + 16 * r) * sam + k * sak];
+        load_ncols(bv, B + k * sbk, tx);
+#pragma unroll
+        for (int r = 0; r < TM; ++r)
+#pragma unroll
+            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+}
+
+// tile_mma with A contiguous along k (four k per 16-byte load) and B running along n (ncol columns).
+template <int TM, int TN>
+__device__ __forceinline__ void tile_mma_ak_nc(float (&acc)[TM][TN], const float* A, int sam, const float* B,
+                                               int sbk, int K, int ty, int tx) {
+    for (int k = 0; k < K; k += 4) {
+        float4 av[TM];
+#pragma unroll
+        for (int r = 0; r < TM; ++r) av[r] = lds4(A + (ty + 16 * r) * sam + k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float bv[TN];
+            load_ncols(bv, B + (k + i) * sbk, tx);
+#pragma unroll
+            for (int r = 0; r < TM; ++r)
+#pragma unroll
+                for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(f4c(av[r], i), bv[c], acc[r][c]);
+        }
+    }
+}
+
 template <int TM, int TN>
 __device__ __forceinline__ void tile_zero(float (&acc)[TM][TN]) {
 #pragma unroll
@@ -255,7 +328,7 @@ __device__ __forceinline__ void tile_zero(float (&acc)[TM][TN]) {
 
 // grid (nchunks, H, batch), kT threads.  Chunk-local state and adjoint sums of one head:
 //   SP[p][n] = sum_j exp(cs_last - cs_j) dt_j x_j[p] B_j[n],  LM[p][n] = sum_i exp(cs_i) g_i[p] C_i[n].
-// Each thread owns rows p = ty + 16 r (r < 4) and columns n = tx + 16 c (c < N/16) of both.
+// Each thread owns rows p = ty + 16 r (r < 4) and columns n = ncol(tx, c) (c < N/16) of both.
 template <int N>
 __global__ void __launch_bounds__(kT) chunk_state_kernel(BwdArgs a, Ws ws) {
     constexpr int TN = N / 16;
@@ -312,17 +385,17 @@ __global__ void __launch_bounds__(kT) chunk_state_kernel(BwdArgs a, Ws ws) {
     const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
     float acc[4][TN];
     tile_zero(acc);
-    tile_mma(acc, wx, 1, kP, Bs, 1, N, Qv, ty, tx);
+    tile_mma_nc(acc, wx, 1, kP, Bs, N, Qv, ty, tx);
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int q = 0; q < TN; ++q) ws.SP[base + (int64_t)(ty + 16 * r) * N + tx + 16 * q] = acc[r][q];
+        for (int q = 0; q < TN; ++q) ws.SP[base + (int64_t)(ty + 16 * r) * N + ncol<TN>(tx, q)] = acc[r][q];
     tile_zero(acc);
-    tile_mma(acc, wg, 1, kP, Cs, 1, N, Qv, ty, tx);
+    tile_mma_nc(acc, wg, 1, kP, Cs, N, Qv, ty, tx);
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int q = 0; q < TN; ++q) ws.LM[base + (int64_t)(ty + 16 * r) * N + tx + 16 * q] = acc[r][q];
+        for (int q = 0; q < TN; ++q) ws.LM[base + (int64_t)(ty + 16 * r) * N + ncol<TN>(tx, q)] = acc[r][q];
 }
 
 // Sum of v over the block (kT threads); every thread gets the total.  red: kT floats.
@@ -497,7 +570,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             for (int q = 0; q < 4; ++q) CB[(ty + 16 * r) * kS + tx + 16 * q] = acc[r][q];
     }
 
-    float dBa[4][TN], dCa[4][TN];  // rows j (or i) = ty + 16 r, columns n = tx + 16 c
+    float dBa[4][TN], dCa[4][TN];  // rows j (or i) = ty + 16 r, columns n = ncol(tx, c)
     tile_zero(dBa);
     tile_zero(dCa);
 
@@ -590,7 +663,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         {
             float acc[4][TN];
             tile_zero(acc);
-            tile_mma_ak(acc, gs, kS, X, 1, NS, kP, ty, tx);        // [i][n] = sum_p g_i[p] Sp[p][n]
+            tile_mma_ak_nc(acc, gs, kS, X, NS, kP, ty, tx);        // [i][n] = sum_p g_i[p] Sp[p][n]
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -635,7 +708,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
         {
             float acc[4][TN];
             tile_zero(acc);
-            tile_mma_ak(acc, xs, kS, X, 1, NS, kP, ty, tx);        // [j][n] = sum_p x_j[p] Lm[p][n]
+            tile_mma_ak_nc(acc, xs, kS, X, NS, kP, ty, tx);        // [j][n] = sum_p x_j[p] Lm[p][n]
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 const int j = ty + 16 * r;
@@ -643,13 +716,13 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
                 for (int q = 0; q < TN; ++q) dBa[r][q] += dts[j] * el[j] * acc[r][q];
             }
             tile_zero(acc);
-            tile_mma(acc, LGX, 1, kS, Cs, 1, NS, Qv, ty, tx);    // [j][n] = sum_i LGX[i][j] dt_j C_i[n]
+            tile_mma_nc(acc, LGX, 1, kS, Cs, NS, Qv, ty, tx);      // [j][n] = sum_i LGX[i][j] dt_j C_i[n]
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
                 for (int q = 0; q < TN; ++q) dBa[r][q] += acc[r][q];
             tile_zero(acc);
-            tile_mma_ak(acc, LGX, kS, Bs, 1, NS, Q4, ty, tx);      // [i][n] = sum_j LGX[i][j] dt_j B_j[n]
+            tile_mma_ak_nc(acc, LGX, kS, Bs, NS, Q4, ty, tx);      // [i][n] = sum_j LGX[i][j] dt_j B_j[n]
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -713,8 +786,8 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
                                    : ws.DU2 + (b * a.L + t0 + j) * 2 * GN;
 #pragma unroll
             for (int q = 0; q < TN; ++q) {
-                dst[(int64_t)g * N + tx + 16 * q] = dBa[r][q];
-                dst[GN + (int64_t)g * N + tx + 16 * q] = dCa[r][q];
+                dst[(int64_t)g * N + ncol<TN>(tx, q)] = dBa[r][q];
+                dst[GN + (int64_t)g * N + ncol<TN>(tx, q)] = dCa[r][q];
             }
         }
     }

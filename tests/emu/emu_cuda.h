@@ -113,6 +113,9 @@ inline float __uint_as_float(unsigned u) {
 struct float4 {
     float x, y, z, w;
 };
+struct float2 {
+    float x, y;
+};
 inline float4 make_float4(float a, float b, float c, float d) { return float4{a, b, c, d}; }
 inline float4 __ldcs(const float4* p) { return *p; }
 inline void __stcs(float4* p, float4 v) { *p = v; }
