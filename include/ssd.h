@@ -273,6 +273,30 @@ SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t nor
                                      ssd_dtype dtype, const void* y, const float* weight, void* out, void* stream);
 
 /*
+ * One decode token of the multi-input multi-output (MIMO) SSM for a batch of
+ * sequences ("Mamba-3: 추론을 우선한 상태 공간 모델", opening section: several SSMs
+ * modelled in parallel per head at almost no cost to decode latency; 아키텍처:
+ * the MIMO projection widens B and C).  Rank R = `rank` (1, 2, 4 or 8), on the
+ * Mamba-2 scalar decay and without the short conv (the page drops it):
+ *   dt = softplus(dt_raw + dt_bias[h]),  a = exp(dt * A[h])
+ *   S[h] <- a * S[h] + dt * sum_{k<R} x_k[h] (outer) B_k[g]
+ *   y_k[h] = (S[h] . C_k[g] + D[h] * x_k[h]) * silu(z_k[h])
+ * R = 1 is the Mamba-2 decode step without its conv.
+ *   x, z        [batch][H][R][P]     dtype (post-projection, no conv)
+ *   dt          [batch][H]           dtype (dt_raw)
+ *   B, C        [batch][G][R][N]     dtype
+ *   ssm_state   [batch][H][P][N] fp32, updated in place
+ *   y           [batch][H][R][P]     dtype, fp32 for SSD_BF16_YF32 (out)
+ * params: A, D, dt_bias are used; conv_w and conv_b are ignored (may be NULL).
+ * y must not overlap any input or the state (SSD_ERR_UNSUPPORTED).
+ * dims->seqlen and dims->chunk are ignored.  Same size limits as the decode
+ * step; SSD_ERR_SHAPE for any other rank.
+ */
+SSD_API ssd_status ssd_mimo_decode_step(const ssd_dims* dims, int32_t rank, ssd_dtype dtype,
+                                        const ssd_params* params, const void* x, const void* dt, const void* B,
+                                        const void* C, const void* z, float* ssm_state, void* y, void* stream);
+
+/*
  * Gradients of ssd_prefill, for training ("Nemotron-H 스타일 Hybrid Mamba-Transformer
  * 3B 모델 구현 타당성 분석" §3.1/§3.2: the hybrid is trained from scratch and the
  * new Mamba-2 layer's forward and backward are checked).  The gradients are
@@ -302,30 +326,6 @@ SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t nor
  * the parameter gradients and d_init_conv_state are zero.  Errors as for
  * ssd_prefill; SSD_ERR_SHAPE also when ceil(seqlen/64) or batch exceeds 65535.
  */
-/*
- * One decode token of the multi-input multi-output (MIMO) SSM for a batch of
- * sequences ("Mamba-3: 추론을 우선한 상태 공간 모델", opening section: several SSMs
- * modelled in parallel per head at almost no cost to decode latency; 아키텍처:
- * the MIMO projection widens B and C).  Rank R = `rank` (1, 2, 4 or 8), on the
- * Mamba-2 scalar decay and without the short conv (the page drops it):
- *   dt = softplus(dt_raw + dt_bias[h]),  a = exp(dt * A[h])
- *   S[h] <- a * S[h] + dt * sum_{k<R} x_k[h] (outer) B_k[g]
- *   y_k[h] = (S[h] . C_k[g] + D[h] * x_k[h]) * silu(z_k[h])
- * R = 1 is the Mamba-2 decode step without its conv.
- *   x, z        [batch][H][R][P]     dtype (post-projection, no conv)
- *   dt          [batch][H]           dtype (dt_raw)
- *   B, C        [batch][G][R][N]     dtype
- *   ssm_state   [batch][H][P][N] fp32, updated in place
- *   y           [batch][H][R][P]     dtype, fp32 for SSD_BF16_YF32 (out)
- * params: A, D, dt_bias are used; conv_w and conv_b are ignored (may be NULL).
- * y must not overlap any input or the state (SSD_ERR_UNSUPPORTED).
- * dims->seqlen and dims->chunk are ignored.  Same size limits as the decode
- * step; SSD_ERR_SHAPE for any other rank.
- */
-SSD_API ssd_status ssd_mimo_decode_step(const ssd_dims* dims, int32_t rank, ssd_dtype dtype,
-                                        const ssd_params* params, const void* x, const void* dt, const void* B,
-                                        const void* C, const void* z, float* ssm_state, void* y, void* stream);
-
 typedef struct {
     float *dx, *ddt, *dB, *dC, *dz;
     float *dA, *dD, *ddt_bias, *dconv_w, *dconv_b;
