@@ -45,6 +45,7 @@ CASES = [
     (1, 70, 2, 1, 128, torch.bfloat16, True, True, True),    # d_state 128 (largest shared tile)
     (1, 129, 3, 3, 64, torch.float32, True, False, False),   # one head per group, 1-token last chunk
     (1, 100, 6, 2, 32, torch.bfloat16, True, True, False),   # three heads per group: halves of 1 and 2 heads
+    (1, 200, 8, 2, 128, torch.bfloat16, True, True, False),  # d_state 128, 4 heads per group, 4 chunks (8-token tail)
 ]
 
 
