@@ -143,12 +143,23 @@ __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
     const float w0 = a.conv_w[c * 4 + 0], w1 = a.conv_w[c * 4 + 1], w2 = a.conv_w[c * 4 + 2],
                 w3 = a.conv_w[c * 4 + 3], bias = a.conv_b[c];
     float r0 = raw_at(a, b, t0 - 3, c), r1 = raw_at(a, b, t0 - 2, c), r2 = raw_at(a, b, t0 - 1, c);
-    for (int64_t t = t0; t < t1; ++t) {
-        const float r3 = raw_at(a, b, t, c);
-        ws.U[(b * a.L + t) * conv_dim + c] = silu_f(bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * r3);
-        r0 = r1;
-        r1 = r2;
-        r2 = r3;
+    // kBatch tokens' inputs are loaded before any of their outputs is stored (the stores could alias
+    // the inputs as far as the compiler knows, so it would not move later loads above them)
+    constexpr int kBatch = 8;
+#pragma unroll 1
+    for (int64_t tb = t0; tb < t1; tb += kBatch) {
+        float rin[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) rin[i] = tb + i < t1 ? raw_at(a, b, tb + i, c) : 0.f;
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            if (tb + i < t1) {
+                ws.U[(b * a.L + tb + i) * conv_dim + c] = silu_f(bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * rin[i]);
+                r0 = r1;
+                r1 = r2;
+                r2 = rin[i];
+            }
+        }
     }
 }
 
@@ -318,6 +329,23 @@ __device__ __forceinline__ void tile_mma_ak_nc(float (&acc)[TM][TN], const float
     }
 }
 
+// tile_mma for the chunk-state sums: rows m = 4 ty + r (four contiguous rows per thread, A(m, k) =
+// A[m + k * sak], one 16-byte load per k; a warp's two ty read 32 contiguous bytes) and B along n
+// (ncol columns).  sak a multiple of 4, A 16-byte aligned.
+template <int TN>
+__device__ __forceinline__ void tile_mma_mc_nc(float (&acc)[4][TN], const float* A, int sak, const float* B,
+                                               int sbk, int K, int ty, int tx) {
+    for (int k = 0; k < K; ++k) {
+        const float4 a4 = lds4(A + 4 * ty + k * sak);
+        float bv[TN];
+        load_ncols(bv, B + k * sbk, tx);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(f4c(a4, r), bv[c], acc[r][c]);
+    }
+}
+
 template <int TM, int TN>
 __device__ __forceinline__ void tile_zero(float (&acc)[TM][TN]) {
 #pragma unroll
@@ -328,7 +356,7 @@ __device__ __forceinline__ void tile_zero(float (&acc)[TM][TN]) {
 
 // grid (nchunks, H, batch), kT threads.  Chunk-local state and adjoint sums of one head:
 //   SP[p][n] = sum_j exp(cs_last - cs_j) dt_j x_j[p] B_j[n],  LM[p][n] = sum_i exp(cs_i) g_i[p] C_i[n].
-// Each thread owns rows p = ty + 16 r (r < 4) and columns n = ncol(tx, c) (c < N/16) of both.
+// Each thread owns rows p = 4 ty + r (r < 4) and columns n = ncol(tx, c) (c < N/16) of both.
 template <int N>
 __global__ void __launch_bounds__(kT) chunk_state_kernel(BwdArgs a, Ws ws) {
     constexpr int TN = N / 16;
@@ -385,17 +413,17 @@ __global__ void __launch_bounds__(kT) chunk_state_kernel(BwdArgs a, Ws ws) {
     const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N;
     float acc[4][TN];
     tile_zero(acc);
-    tile_mma_nc(acc, wx, 1, kP, Bs, N, Qv, ty, tx);
+    tile_mma_mc_nc(acc, wx, kP, Bs, N, Qv, ty, tx);
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int q = 0; q < TN; ++q) ws.SP[base + (int64_t)(ty + 16 * r) * N + ncol<TN>(tx, q)] = acc[r][q];
+        for (int q = 0; q < TN; ++q) ws.SP[base + (int64_t)(4 * ty + r) * N + ncol<TN>(tx, q)] = acc[r][q];
     tile_zero(acc);
-    tile_mma_nc(acc, wg, 1, kP, Cs, N, Qv, ty, tx);
+    tile_mma_mc_nc(acc, wg, kP, Cs, N, Qv, ty, tx);
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int q = 0; q < TN; ++q) ws.LM[base + (int64_t)(ty + 16 * r) * N + ncol<TN>(tx, q)] = acc[r][q];
+        for (int q = 0; q < TN; ++q) ws.LM[base + (int64_t)(4 * ty + r) * N + ncol<TN>(tx, q)] = acc[r][q];
 }
 
 // Sum of v over the block (kT threads); every thread gets the total.  red: kT floats.
@@ -804,48 +832,72 @@ __global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
     const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
     const float w0 = a.conv_w[c * 4 + 0], w1 = a.conv_w[c * 4 + 1], w2 = a.conv_w[c * 4 + 2],
                 w3 = a.conv_w[c * 4 + 3], bias = a.conv_b[c];
+    // this channel's input array and gradient array (x / B / C and dx / dB / dC), row stride, column
+    const void* src;
     float* out;
     int64_t ostride, ocol;
     if (c < HP) {
-        out = a.dx, ostride = HP, ocol = c;
+        src = a.x, out = a.dx, ostride = HP, ocol = c;
     } else if (c < HP + GN) {
-        out = a.dB, ostride = GN, ocol = c - HP;
+        src = a.B, out = a.dB, ostride = GN, ocol = c - HP;
     } else {
-        out = a.dC, ostride = GN, ocol = c - HP - GN;
+        src = a.C, out = a.dC, ostride = GN, ocol = c - HP - GN;
     }
+    const int64_t row0 = b * a.L;
     const bool two_halves = head_split(a.H, a.G) == 2;
     float r0 = raw_at(a, b, t0 - 3, c), r1 = raw_at(a, b, t0 - 2, c), r2 = raw_at(a, b, t0 - 1, c);
     float d1 = 0.f, d2 = 0.f, d3 = 0.f;  // dv at t-1, t-2, t-3 (zero before token 0)
     float gw0 = 0.f, gw1 = 0.f, gw2 = 0.f, gw3 = 0.f, gb = 0.f;
-    for (int64_t t = t0; t < t1 + 3; ++t) {
-        float dv = 0.f;
-        if (t < a.L) {
-            const float r3 = raw_at(a, b, t, c);
-            const float v = bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * r3;
-            float du = ws.DU[(b * a.L + t) * conv_dim + c];
-            if (c >= HP && two_halves) du += ws.DU2[(b * a.L + t) * 2 * GN + (c - HP)];
-            dv = du * dsilu_f(v);
-            if (t < t1) {
-                gw0 += dv * r0;
-                gw1 += dv * r1;
-                gw2 += dv * r2;
-                gw3 += dv * r3;
-                gb += dv;
+    // the loads of kBatch tokens are issued before their gradients are stored (see post_conv_kernel);
+    // 2 keeps the thread at 64 registers (4 CTAs per SM): the same loads in flight per SM as larger
+    // batches with fewer resident CTAs
+    constexpr int kBatch = 2;
+#pragma unroll 1
+    for (int64_t tb = t0; tb < t1 + 3; tb += kBatch) {
+        float rin[kBatch], din[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const int64_t tt = tb + i;
+            rin[i] = 0.f;
+            din[i] = 0.f;
+            if (tt < a.L && tt < t1 + 3) {
+                rin[i] = ld_act(src, (row0 + tt) * ostride + ocol, a.act_bf16);
+                din[i] = ws.DU[(row0 + tt) * conv_dim + c];
+                if (c >= HP && two_halves) din[i] += ws.DU2[(row0 + tt) * 2 * GN + (c - HP)];
             }
-            r0 = r1;
-            r1 = r2;
-            r2 = r3;
         }
-        const int64_t s = t - 3;
-        const float gs = w0 * dv + w1 * d1 + w2 * d2 + w3 * d3;
-        if (s >= t0 && s < t1) {
-            out[(b * a.L + s) * ostride + ocol] = gs;
-        } else if (s < 0 && a.d_init_conv_state) {
-            a.d_init_conv_state[(b * conv_dim + c) * 3 + (s + 3)] = gs;
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const int64_t t = tb + i;
+            if (t < t1 + 3) {
+                float dv = 0.f;
+                if (t < a.L) {
+                    const float r3 = rin[i];
+                    const float v = bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * r3;
+                    dv = din[i] * dsilu_f(v);
+                    if (t < t1) {
+                        gw0 += dv * r0;
+                        gw1 += dv * r1;
+                        gw2 += dv * r2;
+                        gw3 += dv * r3;
+                        gb += dv;
+                    }
+                    r0 = r1;
+                    r1 = r2;
+                    r2 = r3;
+                }
+                const int64_t s = t - 3;
+                const float gs = w0 * dv + w1 * d1 + w2 * d2 + w3 * d3;
+                if (s >= t0 && s < t1) {
+                    out[(row0 + s) * ostride + ocol] = gs;
+                } else if (s < 0 && a.d_init_conv_state) {
+                    a.d_init_conv_state[(b * conv_dim + c) * 3 + (s + 3)] = gs;
+                }
+                d3 = d2;
+                d2 = d1;
+                d1 = dv;
+            }
         }
-        d3 = d2;
-        d2 = d1;
-        d1 = dv;
     }
     float* pw = ws.PW + ((b * nt + tile) * conv_dim + c) * 5;
     pw[0] = gw0;

@@ -20,13 +20,11 @@ SRC = os.path.join(emu_harness.CSRC, "ssd_backward.cu")
 
 MUTANTS = {
     # reads x one token past the tile: beyond the array for the last tile of the last sequence
-    "post-conv reads past its tile": ("        const float r3 = raw_at(a, b, t, c);\n"
-                                      "        ws.U[(b * a.L + t) * conv_dim + c]",
-                                      "        const float r3 = raw_at(a, b, t + 1, c);\n"
-                                      "        ws.U[(b * a.L + t) * conv_dim + c]"),
+    "post-conv reads past its tile": ("rin[i] = tb + i < t1 ? raw_at(a, b, tb + i, c) : 0.f;",
+                                      "rin[i] = tb + i < t1 ? raw_at(a, b, tb + i + 1, c) : 0.f;"),
     # writes each pre-conv gradient one token late: beyond dx / dB / dC for the last token
-    "conv backward writes one row late": ("out[(b * a.L + s) * ostride + ocol] = gs;",
-                                          "out[(b * a.L + s + 1) * ostride + ocol] = gs;"),
+    "conv backward writes one row late": ("out[(row0 + s) * ostride + ocol] = gs;",
+                                          "out[(row0 + s + 1) * ostride + ocol] = gs;"),
     # leaves the rows of a ragged chunk past its end as they were (NaN bytes for the first head)
     "ragged rows not cleared": ("            xs[j * kS + p] = xv;", "            if (j < Qv) xs[j * kS + p] = xv;"),
     # shared rows no longer 16-byte aligned: the emulation's alignment check must stop the vector loads
