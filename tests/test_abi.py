@@ -297,3 +297,23 @@ def test_mimo_rejects_an_overlapping_output(L):
     base = dict(x=0x1000000, dt=0x2000000, B=0x3000000, C=0x4000000, z=0x5000000, S=0x6000000, y=0x7000000)
     assert _call_mimo(L, d, ptrs={**base, "y": base["S"] + 1024}) == 5
     assert _call_mimo(L, d, ptrs={**base, "y": base["B"]}) == 5
+
+
+def test_binding_checks_tensors_before_calling_the_library(L):
+    import torch
+    from selective_state_space_43_b200.synth import Dims, make_backward_grads, make_mimo_decode_inputs, \
+        make_prefill_inputs
+    d = Dims(1, 32, 4, 64, 16, 2, 64)
+    inp = make_prefill_inputs(d, dtype=torch.bfloat16, seed=1)
+    gr = make_backward_grads(d, seed=2)
+    args = [inp[k] for k in ("x", "dt", "B", "C", "z", "A", "D", "dt_bias", "conv_w", "conv_b")]
+    # host tensors are refused: there is no CPU path
+    with pytest.raises(ValueError, match="must be on"):
+        ops.prefill_backward(*args, gr["dy"])
+    data = make_mimo_decode_inputs(d, 2, 1, dtype=torch.bfloat16, seed=3)
+    s = data["steps"][0]
+    with pytest.raises(ValueError, match="must be on"):
+        ops.mimo_decode_step(s["x"], s["dt"], s["B"], s["C"], s["z"], data["params"]["A"], data["params"]["D"],
+                             data["params"]["dt_bias"], data["ssm_state"])
+    with pytest.raises(ValueError, match="must be on"):
+        ops.prefill(*args)
