@@ -289,8 +289,9 @@ SSD_API ssd_status ssd_gated_rmsnorm(int64_t rows, int32_t channels, int32_t nor
  *   y           [batch][H][R][P]     dtype, fp32 for SSD_BF16_YF32 (out)
  * params: A, D, dt_bias are used; conv_w and conv_b are ignored (may be NULL).
  * y must not overlap any input or the state (SSD_ERR_UNSUPPORTED).
- * dims->seqlen and dims->chunk are ignored.  Same size limits as the decode
- * step; SSD_ERR_SHAPE for any other rank.
+ * dims->seqlen and dims->chunk are ignored; the other fields are validated as
+ * for the decode step (d_conv included, although the MIMO step has no conv).
+ * SSD_ERR_SHAPE for any other rank.
  */
 SSD_API ssd_status ssd_mimo_decode_step(const ssd_dims* dims, int32_t rank, ssd_dtype dtype,
                                         const ssd_params* params, const void* x, const void* dt, const void* B,
