@@ -293,30 +293,16 @@ __device__ __forceinline__ void load_ncols(float (&bv)[TN], const float* Bk, int
     }
 }
 
-// tile_mma with B running along n (columns ncol(tx, c)): A(m, k) = A[m * sam + k * sak], scalar loads.
-template <int TM, int TN>
-__device__ __forceinline__ void tile_mma_nc(float (&acc)[TM][TN], const float* A, int sam, int sak, const float* B,
-                                            int sbk, int K, int ty, int tx) {
-    for (int k = 0; k < K; ++k) {
-        float av[TM], bv[TN];
-#pragma unroll
-        for (int r = 0; r < TM; ++r) av[r] = A[(ty + 16 * r) * sam + k * sak];
-        load_ncols(bv, B + k * sbk, tx);
-#pragma unroll
-        for (int r = 0; r < TM; ++r)
-#pragma unroll
-            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-}
-
-// tile_mma with A contiguous along k (four k per 16-byte load) and B running along n (ncol columns).
+// tile_mma with A contiguous along k (four k per 16-byte load) and B running along n (ncol columns);
+// rows 4 ty + r (four contiguous rows per thread: with sam = 68 a warp's two ty read rows 4 apart, 16
+// banks apart, one wavefront).
 template <int TM, int TN>
 __device__ __forceinline__ void tile_mma_ak_nc(float (&acc)[TM][TN], const float* A, int sam, const float* B,
                                                int sbk, int K, int ty, int tx) {
     for (int k = 0; k < K; k += 4) {
         float4 av[TM];
 #pragma unroll
-        for (int r = 0; r < TM; ++r) av[r] = lds4(A + (ty + 16 * r) * sam + k);
+        for (int r = 0; r < TM; ++r) av[r] = lds4(A + (TM * ty + r) * sam + k);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float bv[TN];
@@ -598,7 +584,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             for (int q = 0; q < 4; ++q) CB[(ty + 16 * r) * kS + tx + 16 * q] = acc[r][q];
     }
 
-    float dBa[4][TN], dCa[4][TN];  // rows j (or i) = ty + 16 r, columns n = ncol(tx, c)
+    float dBa[4][TN], dCa[4][TN];  // rows j (or i) = 4 ty + r, columns n = ncol(tx, c)
     tile_zero(dBa);
     tile_zero(dCa);
 
@@ -695,7 +681,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int q = 0; q < TN; ++q) dCa[r][q] += ex[ty + 16 * r] * acc[r][q];
+                for (int q = 0; q < TN; ++q) dCa[r][q] += ex[4 * ty + r] * acc[r][q];
         }
         __syncthreads();
 
@@ -739,12 +725,12 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
             tile_mma_ak_nc(acc, xs, kS, X, NS, kP, ty, tx);        // [j][n] = sum_p x_j[p] Lm[p][n]
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const int j = ty + 16 * r;
+                const int j = 4 * ty + r;
 #pragma unroll
                 for (int q = 0; q < TN; ++q) dBa[r][q] += dts[j] * el[j] * acc[r][q];
             }
             tile_zero(acc);
-            tile_mma_nc(acc, LGX, 1, kS, Cs, NS, Qv, ty, tx);      // [j][n] = sum_i LGX[i][j] dt_j C_i[n]
+            tile_mma_mc_nc(acc, LGX, kS, Cs, NS, Qv, ty, tx);      // [j][n] = sum_i LGX[i][j] dt_j C_i[n]
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -808,7 +794,7 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     // backward adds the two in that order
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const int j = ty + 16 * r;
+        const int j = 4 * ty + r;
         if (j < Qv) {
             float* dst = half == 0 ? ws.DU + (b * a.L + t0 + j) * conv_dim + HP
                                    : ws.DU2 + (b * a.L + t0 + j) * 2 * GN;
