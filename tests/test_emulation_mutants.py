@@ -1,5 +1,5 @@
 """The host emulation of the kernels is a strong enough check: faults planted in temporary copies of
-the backward kernels' source (an access outside a buffer, a misaligned 16-byte shared load, a read of
+the backward and MIMO kernels' source (an access outside a buffer, a misaligned 16-byte shared load, a read of
 shared memory that was never written, a dropped term) each make the emulated run fail, through
 AddressSanitizer, the emulator's alignment check, the NaN-filled outputs and shared memory, or the
 comparison with the oracle.  CPU only; the
@@ -83,3 +83,57 @@ def test_planted_kernel_fault_is_caught(mutant_exes, name):
     inp, gr = _case()
     want = oracle.prefill_backward(inp, gr["dy"], gr["d_final"])
     assert _caught(mutant_exes[name], inp, gr, want), f"the emulation missed the planted fault '{name}'"
+
+
+MIMO_SRC = os.path.join(emu_harness.CSRC, "ssd_mimo.cu")
+
+MIMO_MUTANTS = {
+    # the reduce-scatter keeps the other half: each lane writes another output's sum
+    "read-out keeps the wrong half": ("if (upper) first += HALF;", "if (!upper) first += HALF;"),
+    # only the first lane of each row writes: the other outputs stay unwritten (NaN)
+    "read-outs written by too few lanes": ("if ((lane % (LPR / SCAT)) == 0) {", "if ((lane % LPR) == 0) {"),
+    # each state vector read one vector late: past the state array for the last head
+    "state read one vector late": ("v[it] = __ldcs(S + ((p * N + n0) >> 2));",
+                                   "v[it] = __ldcs(S + ((p * N + n0) >> 2) + 1);"),
+}
+
+
+def _build_mimo(name, old, new, tmp):
+    src = open(MIMO_SRC).read()
+    assert src.count(old) == 1, f"mutation site for '{name}' not unique"
+    d = os.path.join(tmp, name.replace(" ", "_"))
+    os.makedirs(d)
+    with open(os.path.join(d, "ssd_mimo.cu"), "w") as f:
+        f.write(src.replace(old, new))
+    exe = os.path.join(d, "run_mimo")
+    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
+           "-fno-omit-frame-pointer", "-w", "-I", d, "-I", emu_harness.EMU, "-I", emu_harness.CSRC, "-o", exe,
+           os.path.join(emu_harness.EMU, "run_mimo.cpp"), "-pthread"]
+    subprocess.check_call(cmd)
+    return exe
+
+
+@pytest.fixture(scope="module")
+def mimo_mutant_exes(tmp_path_factory):
+    tmp = str(tmp_path_factory.mktemp("emu_mimo_mutants"))
+    with cf.ThreadPoolExecutor(max_workers=len(MIMO_MUTANTS)) as ex:
+        futs = {name: ex.submit(_build_mimo, name, old, new, tmp) for name, (old, new) in MIMO_MUTANTS.items()}
+        return {name: f.result() for name, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MIMO_MUTANTS))
+def test_planted_mimo_kernel_fault_is_caught(mimo_mutant_exes, name):
+    from pins import f64
+    from selective_state_space_43_b200.synth import make_mimo_decode_inputs
+    d = Dims(2, 1, 4, 64, 64, 2, 64)
+    data = make_mimo_decode_inputs(d, 4, 2, dtype=torch.float32, seed=3, random_D=True)
+    prm = {k: f64(v) for k, v in data["params"].items()}
+    S = f64(data["ssm_state"]).copy()
+    want = [oracle.mimo_decode_step(s, prm, S) for s in data["steps"]]
+    try:
+        ys, _ = emu_harness.run_mimo(mimo_mutant_exes[name], data, 4, y_bf16=False)
+    except RuntimeError:
+        return                                         # sanitizer report or a failed run
+    caught = any(np.isnan(y).any() or np.max(np.abs(y - w)) > 2e-5 * max(1.0, np.max(np.abs(w)))
+                 for y, w in zip(ys, want))
+    assert caught, f"the emulation missed the planted fault '{name}'"
