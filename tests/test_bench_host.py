@@ -169,3 +169,29 @@ def test_host_prefill_pieces():
             assert p[0][0] == 0 and p[-1][1] == L
             assert all(a[1] == b[0] for a, b in zip(p, p[1:]))
             assert all(r0 % 64 == 0 for r0, _ in p)                                 # chunk-aligned starts
+
+
+def test_oracle_baselines_of_the_prefill_and_decode_lines():
+    from selective_state_space_43_b200.synth import Dims, make_decode_inputs, make_prefill_inputs
+    d = Dims(2, 96, 4, 64, 16, 2, 64)
+    inp = make_prefill_inputs(d, dtype=torch.bfloat16, seed=5, init_state=True)
+    p = bench.cpu_baseline(inp, d, 0.0, "tiny")
+    assert p["kind"] == "oracle" and p["unit"] == "tokens/s" and p["value"] > 0 and "of the tiny workload" in p["sample"]
+    dd = Dims(4, 1, 4, 64, 16, 2, 64)
+    data = make_decode_inputs(dd, steps=3, seed=6)
+    sample = {"params": data["params"], "ssm_state": data["ssm_state"][:2].clone(),
+              "conv_state": data["conv_state"][:2].clone(),
+              "steps": [{k: v[:2].clone() for k, v in s.items()} for s in data["steps"]]}
+    r = bench.cpu_decode_baseline(sample, dd, 3, 2)
+    assert r["kind"] == "oracle" and r["unit"] == "GB/s" and r["value"] > 0 and "2 of the 4 sequences" in r["sample"]
+    # the baseline leaves the sample's states untouched (it steps copies)
+    assert torch.equal(sample["ssm_state"], data["ssm_state"][:2])
+
+
+def test_headline_is_the_largest_single_gpu_prefill_workload():
+    from selective_state_space_43_b200.synth import WORKLOADS
+    prefill = [n for n in WORKLOADS if not n.startswith("decode")]
+    tokens = {n: WORKLOADS[n]["dims"].batch * WORKLOADS[n]["dims"].seqlen for n in prefill}
+    nbytes = {n: bench.prefill_bytes(WORKLOADS[n]["dims"], 2, WORKLOADS[n]["init_state"]) for n in prefill}
+    assert bench.HEADLINE_WORKLOAD == max(prefill, key=lambda n: (nbytes[n], tokens[n]))
+    assert set(bench.OTHER_PREFILL_WORKLOADS) == set(prefill) - {bench.HEADLINE_WORKLOAD}
