@@ -192,7 +192,9 @@ SSD_API ssd_status ssd_decode_step(const ssd_dims* dims, ssd_dtype dtype, const 
  *    scratch than that (ssd_prefill_workspace_bytes() > SSD_NOALLOC_SCRATCH_BYTES).
  *  - Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
  *  - The first call on a device (with that device current) looks up the
- *    array's address there; make it before any stream capture.
+ *    array's address there; make it before any stream capture.  The address
+ *    stays cached for the process: do not use this entry point across a
+ *    cudaDeviceReset (the cached address would be stale).
  *  - All calls share the array: calls whose kernels overlap on the GPU race.
  *    Each call rewrites every scratch element it reads, so no clearing is
  *    needed between calls.
@@ -348,6 +350,20 @@ SSD_API ssd_status ssd_prefill_backward(const ssd_dims* dims, ssd_dtype dtype, c
  * (about 2 s), so a kernel can never hang the device.
  */
 SSD_API ssd_status ssd_device_status(void* stream);
+
+/*
+ * Testing aid for the timeout path (no counterpart in the pages; off unless
+ * a test calls it).  While wait_ns is nonzero, every tensor-core prefill
+ * (ssd_prefill, ssd_prefill_strided, ssd_prefill_varlen, ssd_prefill_noalloc)
+ * launched from this host thread makes each CTA wait wait_ns nanoseconds on a
+ * barrier that nothing arrives on before its first tensor-core step; the wait
+ * gives up, the CTA lets its copies in flight land, frees its tensor memory
+ * and exits, and ssd_device_status() then reports SSD_ERR_TIMEOUT (the
+ * outputs of that call are incomplete).  Pass 0 to switch it off.  Nothing
+ * faults or hangs: it exercises the same bounded-wait exit a real stall would
+ * take.  Thread-local; always returns SSD_OK.
+ */
+SSD_API ssd_status ssd_test_stall_prefill(uint64_t wait_ns);
 
 /*
  * Optional timing hook for benchmarks.  When both are non-NULL, the next

@@ -11,6 +11,7 @@
 namespace {
 
 thread_local ssd::TimingHook g_hook;
+thread_local uint64_t g_test_stall_ns = 0;  // ssd_test_stall_prefill
 
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -146,6 +147,7 @@ static ssd_status prefill_impl(const ssd_dims* d, ssd_dtype dtype, const ssd_par
     a.y = y; a.final_state = final_state; a.conv_state = conv_state;
     a.workspace = workspace;
     a.rs_x = r.x; a.rs_z = r.z; a.rs_dt = r.dt; a.rs_B = r.B; a.rs_C = r.C;
+    a.stall_ns = g_test_stall_ns;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
                                                                                         : ssd::ActKind::BF16_YF32);
@@ -218,6 +220,7 @@ ssd_status ssd_prefill_varlen(const ssd_dims* d, ssd_dtype dtype, const ssd_para
     a.cu = cu_seqlens;
     a.err = err;
     a.rs_x = s.HP; a.rs_z = s.HP; a.rs_dt = s.H; a.rs_B = s.GN; a.rs_C = s.GN;
+    a.stall_ns = g_test_stall_ns;
     const ssd::ActKind kind = dtype == SSD_F32 ? ssd::ActKind::F32 : (dtype == SSD_BF16 ? ssd::ActKind::BF16
                                                                                         : ssd::ActKind::BF16_YF32);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -359,8 +362,15 @@ ssd_status ssd_mimo_decode_step(const ssd_dims* d, int32_t rank, ssd_dtype dtype
 ssd_status ssd_device_status(void* stream) {
     int flag = 0;
     if (ssd::read_and_clear_tc_error(&flag, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSD_ERR_CUDA;
-    if (flag & ssd::kErrTimeout) return SSD_ERR_TIMEOUT;
+    int mimo_flag = 0;
+    if (ssd::mimo::read_and_clear_mimo_error(&mimo_flag) != cudaSuccess) return SSD_ERR_CUDA;
+    if ((flag & ssd::kErrTimeout) || mimo_flag) return SSD_ERR_TIMEOUT;
     return flag & ssd::kErrBadSeqlens ? SSD_ERR_SHAPE : SSD_OK;
+}
+
+ssd_status ssd_test_stall_prefill(uint64_t wait_ns) {
+    g_test_stall_ns = wait_ns;
+    return SSD_OK;
 }
 
 ssd_status ssd_set_timing_events(void* before_main, void* after_main) {

@@ -48,6 +48,9 @@ struct PrefillArgs {
     // Elements between consecutive rows (tokens) of each input; a batch is L rows.  The contiguous
     // widths HP, HP, H, GN, GN unless the inputs are views into a wider array (e.g. the in_proj output).
     int64_t rs_x = 0, rs_z = 0, rs_dt = 0, rs_B = 0, rs_C = 0;
+    // Tests of the timeout path only (0 otherwise): the tensor-core scan's MMA warp first waits this
+    // many ns on a barrier that nothing arrives on, then gives up and aborts its CTA.
+    uint64_t stall_ns = 0;
 };
 
 // Device error word bits, read back by ssd_device_status.
@@ -85,6 +88,9 @@ namespace mimo {
 struct MimoArgs;
 // The MIMO decode step (ssd_mimo.cu); sizes and pointers validated by the caller.
 cudaError_t launch_mimo_decode(const MimoArgs& a, cudaStream_t st);
+// Reads and clears the MIMO kernel's error word (nonzero: a state load never landed).  Does not
+// synchronise: call after the stream is idle.
+cudaError_t read_and_clear_mimo_error(int* flag);
 }  // namespace mimo
 
 namespace bwd {

@@ -51,6 +51,8 @@
 // flag (read back by ssd_device_status) and the CTA drains and exits.
 #include <cuda.h>
 
+#include <mutex>
+
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
 #include "ssd_sm100.cuh"
@@ -92,7 +94,7 @@ constexpr uint32_t OFF_RFAC = OFF_WX + 2 * 128 * 4;    // exp(cs_i - cs_end(g(i)
 constexpr uint32_t OFF_PG = OFF_RFAC + 128 * 4;        // exp(cs_end(gi-1) - cs_end(g)), g < gi: [16 gi][4 q][4 kb]
 constexpr uint32_t OFF_DG = OFF_PG + 256 * 4;          // exp(cs_i - cs_j) dt_j inside a group, j <= i: [16][8][8]
 constexpr uint32_t OFF_BAR = OFF_DG + 1024 * 4;        // mbarriers (8 B each)
-constexpr int NBAR = 18;
+constexpr int NBAR = 19;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;  // TMEM base address
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
@@ -102,7 +104,8 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // FULL_RAW / XREADY / CS_* come in pairs by chunk parity; EPI_DONE = a chunk's epilogue is complete
 // (its Y / Y2 / z read, its y written); EMPTY_BC = the chunk's last B / C reader (Y2) is complete.
 enum Bar { FULL_RAW0 = 0, FULL_RAW1, XREADY0, XREADY1, FULL_Z, EPI_DONE, FULL_BC, EMPTY_BC, MREADY, G_FULL, SC_FULL,
-           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, TAB_READY };
+           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, TAB_READY,
+           NEVER };  // NEVER: nothing arrives on it (the test stall of the timeout path waits on it)
 
 // TMEM columns (fp32, 128 lanes): G = C B^T, Y = M X, Y2 = C S^T, S_c, the running state, and the
 // post-conv x of two chunks (for the D skip)
@@ -358,11 +361,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 if (c + 1 < nc) load_z(c + 1);
             }
             if constexpr (kTmaStoreY) bulk_wait_all();
-            if (*abort_flag) {  // let copies still in flight land before the CTA exits
-                if (issued_x0 >= 0) mbar_wait(&bars[FULL_RAW0], (issued_x0 >> 1) & 1, nullptr, 100000000ull);
-                if (issued_x1 >= 0) mbar_wait(&bars[FULL_RAW1], (issued_x1 >> 1) & 1, nullptr, 100000000ull);
-                if (issued_z >= 0) mbar_wait(&bars[FULL_Z], issued_z & 1, nullptr, 100000000ull);
-            }
+            // Every load this thread issued lands before the CTA exits.  Normally each was consumed
+            // already and the waits return at once; after an abort (which another warp may raise after
+            // this loop has ended) a load can still be in flight.
+            if (issued_x0 >= 0) mbar_wait(&bars[FULL_RAW0], (issued_x0 >> 1) & 1, nullptr, 100000000ull);
+            if (issued_x1 >= 0) mbar_wait(&bars[FULL_RAW1], (issued_x1 >> 1) & 1, nullptr, 100000000ull);
+            if (issued_z >= 0) mbar_wait(&bars[FULL_Z], issued_z & 1, nullptr, 100000000ull);
         }
     } else if (warp == kWarpBc) {
         // ---------------- post-conv B / C producer ----------------
@@ -382,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, tok0 + c * kQ, mb);
                 last = c;
             }
-            if (*abort_flag && last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
+            // the last B / C load lands before the CTA exits (at once unless a consumer aborted)
+            if (last >= 0) mbar_wait(&bars[FULL_BC], last & 1, nullptr, 100000000ull);
         }
     } else if (warp == kWarpCs) {
         // ---------------- chunk dt / cumsum (whole warp; lane l owns rows 4l .. 4l+3) ----------------
@@ -522,6 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             const uint64_t dM = sw128_desc(smem_u32(sm + OFF_M), 16, 1024);
             const uint64_t dS = sw128_desc(smem_u32(sm + OFF_S), 16384, 1024);
             const uint64_t dX0 = sw128_desc(smem_u32(sm + OFF_X), 16384, 1024);
+            // test stall of the timeout path: a wait on a barrier nothing arrives on, bounded by
+            // a.stall_ns, gives up and aborts the CTA before its first MMA (off unless a test sets it)
+            if (a.stall_ns && !mbar_wait(&bars[NEVER], 0, abort_flag, a.stall_ns)) raise_abort(abort_flag);
             for (int c = 0; c < nc; ++c) {
                 const uint64_t dX = dX0 + (uint64_t)((c & 1) * (16384 >> 4));
                 if (!mbar_wait(&bars[FULL_BC], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
@@ -979,10 +987,14 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     return cudaGetLastError();
 }
 
+// The flag's address is looked up once per device and cached for the process (like every device
+// symbol here, it does not survive a cudaDeviceReset).
 int* device_error_flag() {
     static int* ptrs[64] = {};
+    static std::mutex lock;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> guard(lock);
     if (!ptrs[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_tc_error) != cudaSuccess) return nullptr;

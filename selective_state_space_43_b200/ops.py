@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_mimo_decode_step.argtypes = [dimp, ctypes.c_int32, ctypes.c_int, parp] + [vp] * 7 + [vp]
         L.ssd_device_status.restype = ctypes.c_int
         L.ssd_device_status.argtypes = [vp]
+        L.ssd_test_stall_prefill.restype = ctypes.c_int
+        L.ssd_test_stall_prefill.argtypes = [ctypes.c_uint64]
         L.ssd_set_timing_events.restype = ctypes.c_int
         L.ssd_set_timing_events.argtypes = [vp, vp]
         _lib = L
