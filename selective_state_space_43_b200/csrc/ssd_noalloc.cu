@@ -11,7 +11,10 @@
 // The array is SSD_NOALLOC_SCRATCH_BYTES (16 MiB) and every GPU that loads
 // the library holds it until the process exits.  Its device address is looked
 // up once per device, on the first call made with that device current; make
-// that first call before any stream capture.  All calls share the one array:
+// that first call before any stream capture.  The address is cached by device
+// index for the life of the process: a cudaDeviceReset (or any other teardown
+// of the device's primary context) between calls leaves it stale, so this
+// entry point must not be used across a device reset in one process.  All calls share the one array:
 // calls whose kernels overlap on the GPU (e.g. on two streams) race on it.
 // Nothing in it has to start at zero: the B/C prologue writes every element
 // that the chunk scan then reads, so leftovers from the previous call are

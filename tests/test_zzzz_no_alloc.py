@@ -1,18 +1,20 @@
 """ssd_prefill_noalloc: the prefill entry point for callers that cannot
 allocate device memory (no allocator they may use, or an allocation would
 break their memory plan), which keeps its scratch in a fixed array inside the
-library.  Its results must match ssd_prefill's on two calls in a row (the
-second call finds the first call's leftovers in the shared array).
+library.  The same kernels run on the same inputs as ssd_prefill, so its
+results must equal ssd_prefill's bit for bit, on two calls in a row (the second
+call finds the first call's leftovers in the shared array), and after a longer
+call has filled more of the array than a shorter one with a ragged last chunk
+rewrites (the shorter call must read none of the longer call's rows).
 
 Collected last on purpose (file name), so that a run stopping at the first
 failure has already run every other test."""
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
-from gpu_util import assert_close, dev_inputs, np64
+from gpu_util import dev_inputs
 from selective_state_space_43_b200 import ops
 from selective_state_space_43_b200.synth import Dims, make_prefill_inputs
 
@@ -26,21 +28,39 @@ def _run(fn, d, seed, y_dtype):
               y_dtype=y_dtype)
 
 
+def _scratch_bytes(d):
+    dims = ops.make_dims(d.batch, d.seqlen, d.nheads, d.headdim, d.d_state, d.ngroups, d.chunk)
+    return ops.prefill_workspace_bytes(dims, torch.bfloat16)
+
+
+def _assert_equal(got, want, what):
+    torch.cuda.synchronize()
+    ops.device_status()
+    for name, g, w in zip(("y", "final_state", "conv_state"), got, want):
+        assert torch.equal(g, w), f"{what}: {name} differs from ssd_prefill's"
+
+
 @pytest.mark.parametrize("y_dtype", [torch.float32, torch.bfloat16])
 def test_noalloc_matches_prefill_on_two_calls_in_a_row(y_dtype):
-    # Nemotron-H 8B layer shape (16 heads per group), 2 x 1000 tokens with a
-    # ragged last chunk: 8 MB of scratch, inside the 16 MiB built-in array
+    # Nemotron-H 8B layer shape (16 heads per group), 2 x 1000 tokens with a ragged last chunk:
+    # 2 * 1000 * 2 * 2 * 128 * 2 bytes of post-conv B/C scratch, inside the 16 MiB built-in array
     d = Dims(2, 1000, 32, 64, 128, 2, 128)
-    dims = ops.make_dims(d.batch, d.seqlen, d.nheads, d.headdim, d.d_state, d.ngroups, d.chunk)
-    assert 0 < ops.prefill_workspace_bytes(dims, torch.bfloat16) <= ops.NOALLOC_SCRATCH_BYTES
+    assert _scratch_bytes(d) == 2 * 1000 * 2 * 2 * 128 * 2 <= ops.NOALLOC_SCRATCH_BYTES
     for seed in (201, 202):
         want = _run(ops.prefill, d, seed, y_dtype)
         got = _run(ops.prefill_noalloc, d, seed, y_dtype)
-        torch.cuda.synchronize()
-        ops.device_status()
-        assert_close(np64(got[0]), np64(want[0]), f"noalloc y (seed {seed})")
-        assert_close(np64(got[1]), np64(want[1]), f"noalloc final_state (seed {seed})")
-        assert np.array_equal(np64(got[2]), np64(want[2]))
+        _assert_equal(got, want, f"seed {seed}")
+
+
+def test_noalloc_shorter_call_after_a_longer_one():
+    # a call over 2 x 2000 tokens fills 4 MB of the array; the next call (2 x 1000 tokens, last chunk
+    # of 104 rows) reuses its first 2 MB, and must match ssd_prefill with a fresh workspace
+    long_d, short_d = Dims(2, 2000, 32, 64, 128, 2, 128), Dims(2, 1000, 32, 64, 128, 2, 128)
+    assert _scratch_bytes(short_d) < _scratch_bytes(long_d) <= ops.NOALLOC_SCRATCH_BYTES
+    _run(ops.prefill_noalloc, long_d, 211, torch.bfloat16)
+    want = _run(ops.prefill, short_d, 212, torch.bfloat16)
+    got = _run(ops.prefill_noalloc, short_d, 212, torch.bfloat16)
+    _assert_equal(got, want, "after a longer call")
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
