@@ -24,8 +24,11 @@ struct MimoArgs {
     void* ev_after = nullptr;
 };
 
-// Dynamic shared memory of the step kernel: x, B, C and y of one (sequence, head).
-inline size_t smem_bytes(int R, int P, int N) { return (size_t)(2 * R * P + 2 * R * N) * sizeof(float); }
+// Dynamic shared memory of the step kernel: the head's P x N fp32 state, x, B, C and y of one
+// (sequence, head), and the state load's mbarrier.
+inline size_t smem_bytes(int R, int P, int N) {
+    return (size_t)(P * N + 2 * R * P + 2 * R * N) * sizeof(float) + 16;
+}
 
 }  // namespace mimo
 }  // namespace ssd

@@ -15,6 +15,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <barrier>
 #include <memory>
 #include <thread>
@@ -41,6 +42,7 @@ namespace emu {
 struct Ctx {
     dim3 tid, bid;
     std::barrier<>* bar = nullptr;
+    std::atomic<int>* or_flag = nullptr;  // __syncthreads_or's slot of this block
     unsigned char* smem = nullptr;
     std::barrier<>* warp_bar = nullptr;  // the 32 threads of this thread's warp
     float* warp_buf = nullptr;           // 32 exchange slots of this warp
@@ -48,6 +50,7 @@ struct Ctx {
 };
 inline thread_local Ctx ctx;
 inline dim3 g_grid, g_block;
+inline int g_error = 0;  // a kernel's device error word (set by an emulated bounded wait that gave up)
 
 inline unsigned char* smem() { return ctx.smem; }
 
@@ -62,6 +65,7 @@ void launch(dim3 grid, dim3 block, size_t smem_bytes, F&& body) {
                 std::unique_ptr<unsigned char[]> sm(new unsigned char[smem_bytes ? smem_bytes : 1]);
                 memset(sm.get(), 0xFF, smem_bytes ? smem_bytes : 1);
                 std::barrier<> bar(nt);
+                std::atomic<int> or_flag(0);
                 const unsigned nw = (nt + 31) / 32;
                 std::vector<std::unique_ptr<std::barrier<>>> wbar;
                 for (unsigned w = 0; w < nw; ++w)
@@ -74,6 +78,7 @@ void launch(dim3 grid, dim3 block, size_t smem_bytes, F&& body) {
                         ctx.tid = dim3(t % block.x, (t / block.x) % block.y, t / (block.x * block.y));
                         ctx.bid = dim3(bx, by, bz);
                         ctx.bar = &bar;
+                        ctx.or_flag = &or_flag;
                         ctx.smem = sm.get();
                         ctx.warp_bar = wbar[t / 32].get();
                         ctx.warp_buf = wbuf.get() + 32 * (t / 32);
@@ -95,6 +100,30 @@ void launch(dim3 grid, dim3 block, size_t smem_bytes, F&& body) {
 #define gridDim (::emu::g_grid)
 
 inline void __syncthreads() { ::emu::ctx.bar->arrive_and_wait(); }
+// Block-wide OR of v: every thread of the block calls it (three barrier phases, so the slot can be
+// reset before any thread can reach the next call).
+inline int __syncthreads_or(int v) {
+    ::emu::Ctx& c = ::emu::ctx;
+    c.bar->arrive_and_wait();
+    if (v) c.or_flag->store(1);
+    c.bar->arrive_and_wait();
+    const int r = c.or_flag->load();
+    c.bar->arrive_and_wait();
+    if (c.tid.x == 0 && c.tid.y == 0 && c.tid.z == 0) c.or_flag->store(0);
+    return r;
+}
+
+// mbarriers and untiled bulk copies: a bulk copy is a plain copy made when it is issued, so every
+// wait on its barrier succeeds at once (the copies' bounds are still checked by AddressSanitizer).
+inline void mbar_init(uint64_t*, unsigned) {}
+inline void fence_mbar_init() {}
+inline void mbar_arrive_expect_tx(uint64_t*, unsigned) {}
+inline bool mbar_wait(uint64_t*, unsigned, volatile int*, uint64_t = 0) { return true; }
+inline void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t*) { memcpy(dst, src, bytes); }
+inline void bulk_store(void* dst, const void* src, unsigned bytes) { memcpy(dst, src, bytes); }
+inline void bulk_commit() {}
+inline void bulk_wait_read_all() {}
+inline void fence_async_smem() {}
 
 // Vector accesses must be aligned to their size on the GPU; the host would not fault, so check here.
 inline void emu_check_aligned(const void* p, unsigned bytes) {

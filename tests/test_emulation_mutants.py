@@ -92,9 +92,13 @@ MIMO_MUTANTS = {
     "read-out keeps the wrong half": ("if (upper) first += HALF;", "if (!upper) first += HALF;"),
     # only the first lane of each row writes: the other outputs stay unwritten (NaN)
     "read-outs written by too few lanes": ("if ((lane % (LPR / SCAT)) == 0) {", "if ((lane % LPR) == 0) {"),
-    # each state vector read one vector late: past the state array for the last head
-    "state read one vector late": ("v[it] = __ldcs(S + ((p * N + n0) >> 2));",
-                                   "v[it] = __ldcs(S + ((p * N + n0) >> 2) + 1);"),
+    # the head's state loaded one vector late: past the state array for the last head
+    "state read one vector late": ("bulk_load(s_st, gstate, kStateBytes, bar);",
+                                   "bulk_load(s_st, gstate + 4, kStateBytes, bar);"),
+    # each lane updates the next lane's columns: the last lane of a row reads and writes past the row
+    "state columns one vector late": ("float* srow = s_st + p * N + n0;", "float* srow = s_st + p * N + n0 + 4;"),
+    # the updated state is never written back
+    "state store dropped": ("bulk_store(gstate, s_st, kStateBytes);", "(void)gstate;"),
 }
 
 
