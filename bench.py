@@ -168,7 +168,8 @@ def bench_backward(ops, d: Dims, act, dev, flush, K: int, warmup: int, world: in
             "algorithmic_bytes_per_step": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
             "dominant_kernel": {"kernel": "chunk_bwd_kernel", "ms": kms, "share": kms / ms,
                                 "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_ALU_TFLOPS,
-                                             "unit": "TFLOP/s", "frac": tf / FP32_ALU_TFLOPS, "traffic": None,
+                                             "unit": "TFLOP/s", "frac": tf / FP32_ALU_TFLOPS,
+                                             "traffic": kernel_traffic("chunk_bwd_kernel"),
                                              "algorithmic_flops_per_launch": flops,
                                              "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1965 MHz"}},
             "l2": "flushed between timed steps (256 MB write outside the step events)"}
@@ -232,7 +233,7 @@ def bench_mimo(ops, d: Dims, act, dev, world: int, sampler, peaks, nsteps: int):
                         "activations, fp32 state, no conv",
             "algorithmic_bytes_per_step": nbytes, "algorithmic_flops_per_step": flops,
             "roofline": {"bound": "hbm", "kernel": "mimo_decode_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None},
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": kernel_traffic("mimo_decode_kernel")},
             "l2": "state (1.07 GB) larger than L2; no flush"}
 
 
