@@ -104,8 +104,11 @@ SSD_API size_t ssd_prefill_workspace_bytes(const ssd_dims* dims, ssd_dtype dtype
 
 /*
  * Which kernel path ssd_prefill takes for these sizes:
- *   1 = tcgen05 tensor-core chunk scan (bf16 activations, P=64, Q=128, N=128,
- *       nheads a multiple of 8);
+ *   1 = tcgen05 tensor-core chunk scan (bf16 activations, P=64, N in {64, 128},
+ *       Q in {64, 128}, nheads a multiple of 8).  It always works in chunks of
+ *       128 tokens (Q = 64 gives the same result up to rounding: the chunk
+ *       length is a tiling choice), and runs N = 64 in the N = 128 tiles with
+ *       the upper 64 state channels zero;
  *   2 = CUDA-core chunk scan (every other supported shape, and fp32);
  *  <0 = -(ssd_status) for invalid sizes.
  */

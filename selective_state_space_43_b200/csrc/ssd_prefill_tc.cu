@@ -32,13 +32,19 @@
 //                           loads with the chunk's raw x; then the chunk's
 //                           decay tables, once the previous chunk's mask is done
 //                  warp 3  TMA producer: post-conv B and C tiles
-//                  warps 4-19 512 compute threads, four per token row i (= TMEM
-//                           lane i), each owning 16 channels / state / output
-//                           columns and one 8-column group of each of the 4
-//                           decay-mask column blocks: x conv (fp32 output kept
-//                           in TMEM for the D skip), decay mask, state pass,
-//                           epilogue (D skip, z gate, y store).  Elementwise
-//                           math uses the packed fp32x2 FMA / MUL of sm_100.
+//                  warps 4-11  group A, two threads per token row i (= TMEM
+//                           lane i), each owning two 8-column groups of each of
+//                           the 4 decay-mask column blocks and 32 output
+//                           columns: the decay mask of chunk c, then its
+//                           epilogue (D skip, z gate, y store)
+//                  warps 12-19 group B, two threads per row: the x conv of
+//                           chunk c+1 (32 channels each; fp32 output kept in
+//                           TMEM for the D skip), then the state pass of chunk
+//                           c+1 (32 state columns of row n = i)
+//                The two groups run a chunk apart, so the mask / epilogue of one
+//                chunk overlaps the conv / state pass of the next instead of all
+//                16 warps walking the four phases in lock step.  Elementwise
+//                math uses the packed fp32x2 FMA / MUL of sm_100.
 // The decay exp(cs_i - cs_j) dt_j of M is assembled from tables that the
 // cumsum warp writes for each chunk, so the mask itself needs no MUFU work.
 // With g(i) the 8-row group of i and cs_end(g) the cumsum at the group's last
@@ -68,7 +74,11 @@ using namespace sm100;
 constexpr int kQ = 128, kP = 64, kN = 128;
 constexpr int kThreads = 640;
 constexpr int kWarpRaw = 0, kWarpMma = 1, kWarpCs = 2, kWarpBc = 3, kFirstCompute = 4;
-constexpr int kComputeThreads = 512;  // 16 warps: four per TMEM lane quadrant
+// The 16 compute warps form two groups of 8 (two warps per TMEM lane quadrant in each), specialised by
+// phase so that the phases of neighbouring chunks overlap: group A (warps 4-11) builds each chunk's decay
+// mask and runs its epilogue, group B (warps 12-19) runs the x conv and the state pass.
+constexpr int kFirstGroupB = 12;
+constexpr int kGroupThreads = 256;
 
 // shared memory map (bytes from a 1024-byte aligned base)
 constexpr uint32_t OFF_C = 0;          // u_C tile: two boxes [128 tok][64 n] bf16, 128B swizzle
@@ -94,17 +104,19 @@ constexpr uint32_t OFF_RFAC = OFF_WX + 2 * 128 * 4;    // exp(cs_i - cs_end(g(i)
 constexpr uint32_t OFF_PG = OFF_RFAC + 128 * 4;        // exp(cs_end(gi-1) - cs_end(g)), g < gi: [16 gi][4 q][4 kb]
 constexpr uint32_t OFF_DG = OFF_PG + 256 * 4;          // exp(cs_i - cs_j) dt_j inside a group, j <= i: [16][8][8]
 constexpr uint32_t OFF_BAR = OFF_DG + 1024 * 4;        // mbarriers (8 B each)
-constexpr int NBAR = 19;
+constexpr int NBAR = 21;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;  // TMEM base address
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// FULL_RAW / XREADY / CS_* come in pairs by chunk parity; EPI_DONE = a chunk's epilogue is complete
-// (its Y / Y2 / z read, its y written); EMPTY_BC = the chunk's last B / C reader (Y2) is complete.
-enum Bar { FULL_RAW0 = 0, FULL_RAW1, XREADY0, XREADY1, FULL_Z, EPI_DONE, FULL_BC, EMPTY_BC, MREADY, G_FULL, SC_FULL,
-           Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, TAB_READY,
+// FULL_RAW / XREADY / EPI_DONE / CS_* come in pairs by chunk parity (a waiter of one group may be a whole
+// chunk behind the other group, and a barrier must never run two phases past a waiter); EPI_DONE = a
+// chunk's epilogue is complete (its Y / Y2 / z / conv output read, its y written); EMPTY_BC = the chunk's
+// last B / C reader (Y2) is complete; SREADY = the state entering the next chunk is in shared memory.
+enum Bar { FULL_RAW0 = 0, FULL_RAW1, XREADY0, XREADY1, FULL_Z, EPI_DONE0, EPI_DONE1, FULL_BC, EMPTY_BC, MREADY,
+           G_FULL, SC_FULL, Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, TAB_READY, SREADY,
            NEVER };  // NEVER: nothing arrives on it (the test stall of the timeout path waits on it)
 
 // TMEM columns (fp32, 128 lanes): G = C B^T, Y = M X, Y2 = C S^T, S_c, the running state, and the
@@ -175,17 +187,19 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
     atomicOr(&g_tc_error, kErrTimeout);
 }
 
-// Row-major x conv of chunk cc for the calling thread: token row i, channels 16*quarter .. +15.
-// Writes X and X' (bf16, smem operands) and the fp32 conv output into TMEM (for the D skip), and the
-// raw history of the next chunk.  Returns false if a wait gave up.
+// Row-major x conv of chunk cc for the calling thread of group B: token row i, channels 32*half .. +31
+// (two 16-channel quarters).  Writes X and X' (bf16, smem operands) and the fp32 conv output into TMEM
+// (for the D skip), and the raw history of the next chunk.  Returns false if a wait gave up.
 __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, uint64_t* bars, volatile int* abort_flag,
                                            uint32_t tmem, uint32_t lane_base, int cc, int nc, int64_t Ls, int i,
-                                           int quarter) {
+                                           int half) {
     const int buf = cc & 1;
     if (!warp_wait(&bars[CS_READY0 + buf], (cc >> 1) & 1, abort_flag)) return false;
     if (!warp_wait(&bars[FULL_RAW0 + buf], (cc >> 1) & 1, abort_flag)) return false;
     // the raw history rows were written by other threads in the previous chunk's conv
     if (cc >= 1 && !warp_wait(&bars[XREADY0 + ((cc - 1) & 1)], ((cc - 1) >> 1) & 1, abort_flag)) return false;
+    // the X tile and the conv output of this parity were last read by chunk cc-2's Y MMA and epilogue
+    if (cc >= 2 && !warp_wait(&bars[EPI_DONE0 + buf], ((cc - 2) >> 1) & 1, abort_flag)) return false;
     const int64_t t0 = (int64_t)cc * kQ;
     const int Qc = (int)(Ls - t0 < kQ ? Ls - t0 : kQ);
     const bool valid = i < Qc;
@@ -193,58 +207,64 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
     const uint4* halo_in = reinterpret_cast<const uint4*>(sm + OFF_HALO + (cc & 1) * 384);
     const float4* wt = reinterpret_cast<const float4*>(sm + OFF_WT);   // [tap][64 channels]
     const float4* cb = reinterpret_cast<const float4*>(sm + OFF_CB);
-    float2 acc[8];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const float4 bv = cb[quarter * 4 + m];
-        acc[2 * m] = make_float2(bv.x, bv.y);
-        acc[2 * m + 1] = make_float2(bv.z, bv.w);
-    }
-#pragma unroll
-    for (int tap = 0; tap < 4; ++tap) {
-        const int r = i - 3 + tap;
-        uint4 w[2];
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-            w[k] = r >= 0 ? *reinterpret_cast<const uint4*>(rx + sw128_off(r, quarter * 2 + k))
-                          : halo_in[(r + 3) * 8 + quarter * 2 + k];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float4 tv = wt[tap * 16 + quarter * 4 + m];
-            const uint32_t lo = (m & 1) ? w[m >> 1].z : w[m >> 1].x;
-            const uint32_t hi = (m & 1) ? w[m >> 1].w : w[m >> 1].y;
-            acc[2 * m] = __ffma2_rn(make_float2(tv.x, tv.y), make_float2(bf_lo(lo), bf_hi(lo)), acc[2 * m]);
-            acc[2 * m + 1] = __ffma2_rn(make_float2(tv.z, tv.w), make_float2(bf_lo(hi), bf_hi(hi)), acc[2 * m + 1]);
-        }
-    }
     const float wxr = s_wx_at(sm, buf, i);
-    float u[16];
-    uint32_t xo[8], xpo[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float2 uv = valid ? silu2(acc[k]) : make_float2(0.f, 0.f);
-        u[2 * k] = uv.x;
-        u[2 * k + 1] = uv.y;
-        xo[k] = pack_bf2(uv.x, uv.y);
-        const float2 up = __fmul2_rn(uv, make_float2(wxr, wxr));
-        xpo[k] = pack_bf2(up.x, up.y);
-    }
-    tmem_st16(tmem + lane_base + COL_U + buf * 64 + quarter * 16, u);
     uint8_t* sX = sm + OFF_X + buf * 16384;
     uint8_t* sXp = sm + OFF_XP;
+#pragma unroll 1
+    for (int sub = 0; sub < 2; ++sub) {
+        const int quarter = 2 * half + sub;
+        float2 acc[8];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        *reinterpret_cast<uint4*>(sX + sw128_off(i, quarter * 2 + k)) =
-            make_uint4(xo[4 * k], xo[4 * k + 1], xo[4 * k + 2], xo[4 * k + 3]);
-        *reinterpret_cast<uint4*>(sXp + sw128_off(i, quarter * 2 + k)) =
-            make_uint4(xpo[4 * k], xpo[4 * k + 1], xpo[4 * k + 2], xpo[4 * k + 3]);
-    }
-    if (i >= kQ - 3 && cc + 1 < nc) {  // raw history (rows 125..127) of the next chunk
-        uint4* halo_out = reinterpret_cast<uint4*>(sm + OFF_HALO + ((cc + 1) & 1) * 384);
+        for (int m = 0; m < 4; ++m) {
+            const float4 bv = cb[quarter * 4 + m];
+            acc[2 * m] = make_float2(bv.x, bv.y);
+            acc[2 * m + 1] = make_float2(bv.z, bv.w);
+        }
 #pragma unroll
-        for (int k = 0; k < 2; ++k)
-            halo_out[(i - (kQ - 3)) * 8 + quarter * 2 + k] = *reinterpret_cast<const uint4*>(rx + sw128_off(i, quarter * 2 + k));
+        for (int tap = 0; tap < 4; ++tap) {
+            const int r = i - 3 + tap;
+            uint4 w[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                w[k] = r >= 0 ? *reinterpret_cast<const uint4*>(rx + sw128_off(r, quarter * 2 + k))
+                              : halo_in[(r + 3) * 8 + quarter * 2 + k];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 tv = wt[tap * 16 + quarter * 4 + m];
+                const uint32_t lo = (m & 1) ? w[m >> 1].z : w[m >> 1].x;
+                const uint32_t hi = (m & 1) ? w[m >> 1].w : w[m >> 1].y;
+                acc[2 * m] = __ffma2_rn(make_float2(tv.x, tv.y), make_float2(bf_lo(lo), bf_hi(lo)), acc[2 * m]);
+                acc[2 * m + 1] = __ffma2_rn(make_float2(tv.z, tv.w), make_float2(bf_lo(hi), bf_hi(hi)), acc[2 * m + 1]);
+            }
+        }
+        float u[16];
+        uint32_t xo[8], xpo[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float2 uv = valid ? silu2(acc[k]) : make_float2(0.f, 0.f);
+            u[2 * k] = uv.x;
+            u[2 * k + 1] = uv.y;
+            xo[k] = pack_bf2(uv.x, uv.y);
+            const float2 up = __fmul2_rn(uv, make_float2(wxr, wxr));
+            xpo[k] = pack_bf2(up.x, up.y);
+        }
+        tmem_st16(tmem + lane_base + COL_U + buf * 64 + quarter * 16, u);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            *reinterpret_cast<uint4*>(sX + sw128_off(i, quarter * 2 + k)) =
+                make_uint4(xo[4 * k], xo[4 * k + 1], xo[4 * k + 2], xo[4 * k + 3]);
+            *reinterpret_cast<uint4*>(sXp + sw128_off(i, quarter * 2 + k)) =
+                make_uint4(xpo[4 * k], xpo[4 * k + 1], xpo[4 * k + 2], xpo[4 * k + 3]);
+        }
+        if (i >= kQ - 3 && cc + 1 < nc) {  // raw history (rows 125..127) of the next chunk
+            uint4* halo_out = reinterpret_cast<uint4*>(sm + OFF_HALO + ((cc + 1) & 1) * 384);
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                halo_out[(i - (kQ - 3)) * 8 + quarter * 2 + k] =
+                    *reinterpret_cast<const uint4*>(rx + sw128_off(i, quarter * 2 + k));
+        }
     }
+    tmem_wait_st();  // the conv output is read by a group-A thread, the running state again by this one
     fence_async_smem();
     tc_fence_before();
     mbar_arrive(&bars[XREADY0 + buf]);
@@ -283,8 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int k = 0; k < NBAR; ++k) {
             uint32_t cnt = 1;
-            if (k == XREADY0 || k == XREADY1 || k == EPI_DONE || k == MREADY || k == CS_FREE0 || k == CS_FREE1)
-                cnt = kComputeThreads;
+            if (k == XREADY0 || k == XREADY1 || k == SREADY) cnt = kGroupThreads;       // group B
+            if (k == EPI_DONE0 || k == EPI_DONE1 || k == MREADY) cnt = kGroupThreads;   // group A
+            if (k == CS_FREE0 || k == CS_FREE1) cnt = 2 * kGroupThreads;               // both
             if (k == CS_READY0 || k == CS_READY1 || k == TAB_READY) cnt = 32;
             mbar_init(&bars[k], cnt);
         }
@@ -297,6 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     }
     if (warp >= kFirstCompute) {
         const int i = threadIdx.x - kFirstCompute * 32;
+        if (a.N < kN) {  // d_state 64: the upper 64 channels of the B / C tiles are zero for the whole launch
+            for (int e = i; e < 16384 / 16; e += 2 * kGroupThreads) {
+                reinterpret_cast<uint4*>(sm + OFF_C + 16384)[e] = make_uint4(0u, 0u, 0u, 0u);
+                reinterpret_cast<uint4*>(sm + OFF_B + 16384)[e] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_async_smem();
+        }
         if (i < kP) {
             const int ch = h * kP + i;
             // conv taps [tap][channel], bias, and the history of token 0 (initial conv state or zeros)
@@ -352,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                     load_x(c + 2);
                 }
                 // y(c) out of the z buffer once chunk c's epilogue is complete, then z(c+1) in
-                if (!mbar_wait(&bars[EPI_DONE], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
+                if (!mbar_wait(&bars[EPI_DONE0 + (c & 1)], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 if (kTmaStoreY && tma_y_chunk<kVarlen>(Ls, c)) {
                     tma_store_3d(&prm.tm_y, sm + OFF_Z, h * kP, tok0 + c * kQ, mb);
                     bulk_commit();
@@ -378,12 +406,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             for (int c = 0; c < nc; ++c) {
                 // B / C of chunk c, once chunk c-1's last reader of the tiles (Y2) is complete
                 if (c >= 1 && !mbar_wait(&bars[EMPTY_BC], (c - 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
-                mbar_arrive_expect_tx(&bars[FULL_BC], 4 * 16384);
-                const int xc = a.GN + g * kN, xb = g * kN;
+                // one 64-wide box per 64 state channels; with N = 64 the upper boxes stay zero
+                mbar_arrive_expect_tx(&bars[FULL_BC], (a.N == kN ? 4 : 2) * 16384);
+                const int xc = a.GN + g * a.N, xb = g * a.N;
                 tma_load_3d(sm + OFF_C, &prm.tm_bc, &bars[FULL_BC], xc, tok0 + c * kQ, mb);
-                tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, tok0 + c * kQ, mb);
                 tma_load_3d(sm + OFF_B, &prm.tm_bc, &bars[FULL_BC], xb, tok0 + c * kQ, mb);
-                tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, tok0 + c * kQ, mb);
+                if (a.N == kN) {
+                    tma_load_3d(sm + OFF_C + 16384, &prm.tm_bc, &bars[FULL_BC], xc + 64, tok0 + c * kQ, mb);
+                    tma_load_3d(sm + OFF_B + 16384, &prm.tm_bc, &bars[FULL_BC], xb + 64, tok0 + c * kQ, mb);
+                }
                 last = c;
             }
             // the last B / C load lands before the CTA exits (at once unless a consumer aborted)
@@ -542,8 +573,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 tc_fence_after();
                 mma_k128<true, true>(tmem + COL_SC, dBt, dXp, ID_SC);
                 mma_commit(&bars[SC_FULL]);
-                // Y2 = C S_prev^T, once the previous chunk's epilogue has read the previous Y2
-                if (c >= 1 && !mbar_wait(&bars[EPI_DONE], (c - 1) & 1, abort_flag)) {
+                // Y2 = C S_prev^T, once the previous chunk's epilogue has read the previous Y2 and the state
+                // pass has written S_prev
+                if (c >= 1 && (!mbar_wait(&bars[EPI_DONE0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag) ||
+                               !mbar_wait(&bars[SREADY], (c - 1) & 1, abort_flag))) {
                     raise_abort(abort_flag);
                     break;
                 }
@@ -560,54 +593,26 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             mma_commit(&bars[MMA_DONE]);
             mbar_wait(&bars[MMA_DONE], 0, nullptr, 100000000ull);
         }
-    } else {
-        // ---------------- compute warps ----------------
-        // Per chunk c: decay mask (c), state pass (c), x conv (c+1), epilogue (c), so that the next
-        // chunk's conv and its S_c / Y2 tensor-core work overlap this chunk's Y = M X and epilogue.
-        const int wc = warp - kFirstCompute;               // 0..15
+    } else if (warp < kFirstGroupB) {
+        // ---------------- group A: decay mask and epilogue of each chunk ----------------
+        // Thread (quadrant q, half) owns token row i = TMEM lane i, the 8-column groups 2*half and 2*half+1
+        // of each 32-column mask block, and output columns 32*half .. +31.
         const int q = warp & 3;                            // TMEM lane quadrant of this warp
-        const int quarter = wc >> 2;                       // columns 16*quarter .. +15 (mask: 8-column groups)
-        const int i = q * 32 + lane;                       // token row / TMEM lane / state row n
+        const int half = (warp - kFirstCompute) >> 2;      // 0 or 1
+        const int i = q * 32 + lane;                       // token row / TMEM lane
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float Dh = a.D[h];
-        uint8_t* sXp = sm + OFF_XP;
         uint8_t* sMm = sm + OFF_M;
-        uint8_t* sS = sm + OFF_S;
-        (void)sXp;
-
-        // initial state (this thread's 16 columns): S_run in TMEM, bf16 copy in smem
-        {
-            const float* init = a.init_state ? a.init_state + ((size_t)b * a.H + h) * kP * kN : nullptr;
-            float v[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = init ? init[(size_t)(quarter * 16 + k) * kN + i] : 0.f;
-            tmem_st16(tmem + lane_base + COL_SRUN + quarter * 16, v);
-#pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-                uint4 w;
-                w.x = pack_bf2(v[k2 * 8 + 0], v[k2 * 8 + 1]);
-                w.y = pack_bf2(v[k2 * 8 + 2], v[k2 * 8 + 3]);
-                w.z = pack_bf2(v[k2 * 8 + 4], v[k2 * 8 + 5]);
-                w.w = pack_bf2(v[k2 * 8 + 6], v[k2 * 8 + 7]);
-                *reinterpret_cast<uint4*>(sS + sw128_off(i, quarter * 2 + k2)) = w;
-            }
-            tmem_wait_st();
-        }
-
-        bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, Ls, i, quarter);
-        if (!ok) raise_abort(abort_flag);
-        for (int c = 0; c < nc && ok; ++c) {
+        for (int c = 0; c < nc; ++c) {
             const int buf = c & 1;
             const int64_t t0 = (int64_t)c * kQ;
             const int Qc = (int)(Ls - t0 < kQ ? Ls - t0 : kQ);
             const bool tma_y = kTmaStoreY && tma_y_chunk<kVarlen>(Ls, c);  // else y is stored from registers
-            const float* cs_b = s_cs + buf * 128;
-            const float cs_last = cs_b[kQ - 1];
 
-            // (e) decay mask of row i, columns 8*quarter .. +7 of each 32-column block
+            // (e) decay mask of row i
             if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
-            // the decay tables of this chunk
+            // the decay tables of this chunk (written after its cumsum, so the cumsum buffer is ready too)
             if (!warp_wait(&bars[TAB_READY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             {
                 // decay of row i (group gi) against column group g = 4 kb + quarter (columns 8g .. 8g+7):
@@ -615,147 +620,218 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 //   g = gi: the in-group table;  g > gi: zero
                 const int gi = i >> 3;
                 const float rfac = reinterpret_cast<const float*>(sm + OFF_RFAC)[i];
-                const float4 p4 = reinterpret_cast<const float4*>(sm + OFF_PG)[gi * 4 + quarter];
-                const float pk[4] = {p4.x, p4.y, p4.z, p4.w};
+                const float4 p4a = reinterpret_cast<const float4*>(sm + OFF_PG)[gi * 4 + 2 * half];
+                const float4 p4b = reinterpret_cast<const float4*>(sm + OFF_PG)[gi * 4 + 2 * half + 1];
+                const float pk[2][4] = {{p4a.x, p4a.y, p4a.z, p4a.w}, {p4b.x, p4b.y, p4b.z, p4b.w}};
                 const float4* drow = reinterpret_cast<const float4*>(sm + OFF_DG) + (gi * 8 + (i & 7)) * 2;
-                float gv[4][8];
-#pragma unroll
-                for (int kb = 0; kb < 4; ++kb)  // warp-uniform: groups right of the diagonal block are zero
-                    if (kb <= q) tmem_ld8(tmem + lane_base + COL_G + kb * 32 + quarter * 8, gv[kb]);
-                tmem_wait_ld();
+                const float* colf_b = s_colf + buf * 128;
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb) {
-                    const int g = 4 * kb + quarter;
-                    uint4 packed = make_uint4(0u, 0u, 0u, 0u);
-                    if (kb <= q && g <= gi) {
-                        float4 fa, fb;
-                        if (g < gi) {
-                            const float4* colf = reinterpret_cast<const float4*>(s_colf + buf * 128 + 8 * g);
-                            const float rf = rfac * pk[kb];
-                            fa = colf[0];
-                            fb = colf[1];
-                            fa = make_float4(fa.x * rf, fa.y * rf, fa.z * rf, fa.w * rf);
-                            fb = make_float4(fb.x * rf, fb.y * rf, fb.z * rf, fb.w * rf);
-                        } else {
-                            fa = drow[0];
-                            fb = drow[1];
-                        }
-                        const float2 m0 = __fmul2_rn(make_float2(gv[kb][0], gv[kb][1]), make_float2(fa.x, fa.y));
-                        const float2 m1 = __fmul2_rn(make_float2(gv[kb][2], gv[kb][3]), make_float2(fa.z, fa.w));
-                        const float2 m2 = __fmul2_rn(make_float2(gv[kb][4], gv[kb][5]), make_float2(fb.x, fb.y));
-                        const float2 m3 = __fmul2_rn(make_float2(gv[kb][6], gv[kb][7]), make_float2(fb.z, fb.w));
-                        packed = make_uint4(pack_bf2(m0.x, m0.y), pack_bf2(m1.x, m1.y), pack_bf2(m2.x, m2.y),
-                                            pack_bf2(m3.x, m3.y));
+                    float gv[16];
+                    if (kb <= q) {  // warp-uniform: blocks right of the diagonal block are zero
+                        tmem_ld16(tmem + lane_base + COL_G + kb * 32 + half * 16, gv);
+                        tmem_wait_ld();
                     }
-                    *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 + sw128_off(i, (kb & 1) * 4 + quarter)) = packed;
+#pragma unroll
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int quarter = 2 * half + sub;
+                        const int g = 4 * kb + quarter;
+                        uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+                        if (kb <= q && g <= gi) {
+                            float4 fa, fb;
+                            if (g < gi) {
+                                const float4* colf = reinterpret_cast<const float4*>(colf_b + 8 * g);
+                                const float rf = rfac * pk[sub][kb];
+                                fa = colf[0];
+                                fb = colf[1];
+                                fa = make_float4(fa.x * rf, fa.y * rf, fa.z * rf, fa.w * rf);
+                                fb = make_float4(fb.x * rf, fb.y * rf, fb.z * rf, fb.w * rf);
+                            } else {
+                                fa = drow[0];
+                                fb = drow[1];
+                            }
+                            const float* gg = gv + 8 * sub;
+                            const float2 m0 = __fmul2_rn(make_float2(gg[0], gg[1]), make_float2(fa.x, fa.y));
+                            const float2 m1 = __fmul2_rn(make_float2(gg[2], gg[3]), make_float2(fa.z, fa.w));
+                            const float2 m2 = __fmul2_rn(make_float2(gg[4], gg[5]), make_float2(fb.x, fb.y));
+                            const float2 m3 = __fmul2_rn(make_float2(gg[6], gg[7]), make_float2(fb.z, fb.w));
+                            packed = make_uint4(pack_bf2(m0.x, m0.y), pack_bf2(m1.x, m1.y), pack_bf2(m2.x, m2.y),
+                                                pack_bf2(m3.x, m3.y));
+                        }
+                        *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 + sw128_off(i, (kb & 1) * 4 + quarter)) =
+                            packed;
+                    }
                 }
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[MREADY]);
 
-            // (f) state passing: S_run <- exp(cs_last) S_run + S_c  (lane i = state row n; 16 columns p)
-            if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
-            tc_fence_after();
-            {
-                const float dl = __expf(cs_last);
-                const float2 dl2 = make_float2(dl, dl);
-                float sc[16], sr[16];
-                tmem_ld16(tmem + lane_base + COL_SC + quarter * 16, sc);
-                tmem_ld16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 16; k += 2) {
-                    const float2 v = __ffma2_rn(dl2, make_float2(sr[k], sr[k + 1]), make_float2(sc[k], sc[k + 1]));
-                    sr[k] = v.x;
-                    sr[k + 1] = v.y;
-                }
-                tmem_st16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
-                // S_prev is overwritten once Y2 = C S_prev^T of this chunk has read it
-                if (!warp_wait(&bars[EMPTY_BC], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
-#pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                    uint4 w;
-                    w.x = pack_bf2(sr[k2 * 8 + 0], sr[k2 * 8 + 1]);
-                    w.y = pack_bf2(sr[k2 * 8 + 2], sr[k2 * 8 + 3]);
-                    w.z = pack_bf2(sr[k2 * 8 + 4], sr[k2 * 8 + 5]);
-                    w.w = pack_bf2(sr[k2 * 8 + 6], sr[k2 * 8 + 7]);
-                    // the state entering chunk c+1
-                    *reinterpret_cast<uint4*>(sS + sw128_off(i, quarter * 2 + k2)) = w;
-                }
-            }
-
-            // (c) the next chunk's x conv (its S_c then overlaps this chunk's Y = M X and epilogue)
-            if (c + 1 < nc && !conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, c + 1, nc, Ls, i, quarter)) {
-                raise_abort(abort_flag);
-                break;
-            }
-
-            // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 16*quarter .. +15
+            // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 32*half .. +31
             if (!warp_wait(&bars[FULL_Z], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            // the conv output of this chunk (written by group B; complete before the Y MMA was issued, waited
+            // on here as well so that the TMEM stores are ordered before this group's loads directly)
+            if (!warp_wait(&bars[XREADY0 + buf], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
             tc_fence_after();
-            tmem_wait_st();  // this thread's TMEM stores (the conv output read below, the running state) are done
             {
                 uint8_t* rz = sm + OFF_Z;  // z in, y out (same positions, this thread's only)
-                const float ecs = __expf(cs_b[i]);  // decay of S_prev up to row i
+                const float ecs = __expf(s_cs[buf * 128 + i]);  // decay of S_prev up to row i
                 const float2 e2 = make_float2(ecs, ecs), d2 = make_float2(Dh, Dh);
-                // the gate SiLU(z) of this thread's 16 columns
-                float2 gz[8];
+#pragma unroll 1
+                for (int sub = 0; sub < 2; ++sub) {
+                    const int quarter = 2 * half + sub;
+                    // the gate SiLU(z) of these 16 columns
+                    float2 gz[8];
 #pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                    const uint4 zw = *reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2 + k2));
-                    const uint32_t zr[4] = {zw.x, zw.y, zw.z, zw.w};
+                    for (int k2 = 0; k2 < 2; ++k2) {
+                        const uint4 zw = *reinterpret_cast<const uint4*>(rz + sw128_off(i, quarter * 2 + k2));
+                        const uint32_t zr[4] = {zw.x, zw.y, zw.z, zw.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) gz[k2 * 4 + e] = silu2(make_float2(bf_lo(zr[e]), bf_hi(zr[e])));
-                }
-#pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {  // 8 columns per TMEM round trip
-                    float y1[8], y2[8], uu[8];
-                    tmem_ld8(tmem + lane_base + COL_Y + quarter * 16 + k2 * 8, y1);
-                    tmem_ld8(tmem + lane_base + COL_Y2 + quarter * 16 + k2 * 8, y2);
-                    tmem_ld8(tmem + lane_base + COL_U + buf * 64 + quarter * 16 + k2 * 8, uu);
-                    tmem_wait_ld();
-                    float o[8];
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        float2 yv = __ffma2_rn(e2, make_float2(y2[e], y2[e + 1]), make_float2(y1[e], y1[e + 1]));
-                        yv = __ffma2_rn(d2, make_float2(uu[e], uu[e + 1]), yv);
-                        const float2 ov = __fmul2_rn(yv, gz[k2 * 4 + (e >> 1)]);
-                        o[e] = ov.x;
-                        o[e + 1] = ov.y;
+                        for (int e = 0; e < 4; ++e) gz[k2 * 4 + e] = silu2(make_float2(bf_lo(zr[e]), bf_hi(zr[e])));
                     }
-                    if (tma_y) {
-                        *reinterpret_cast<uint4*>(rz + sw128_off(i, quarter * 2 + k2)) =
-                            make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]),
-                                       pack_bf2(o[6], o[7]));
-                    } else if (i < Qc) {
-                        TY* yrow = static_cast<TY*>(a.y) + ((size_t)span.row0 + t0 + i) * a.HP + (size_t)h * kP + quarter * 16;
-                        if constexpr (sizeof(TY) == 2) {
-                            *reinterpret_cast<uint4*>(yrow + k2 * 8) =
+#pragma unroll
+                    for (int k2 = 0; k2 < 2; ++k2) {  // 8 columns per TMEM round trip
+                        float y1[8], y2[8], uu[8];
+                        tmem_ld8(tmem + lane_base + COL_Y + quarter * 16 + k2 * 8, y1);
+                        tmem_ld8(tmem + lane_base + COL_Y2 + quarter * 16 + k2 * 8, y2);
+                        tmem_ld8(tmem + lane_base + COL_U + buf * 64 + quarter * 16 + k2 * 8, uu);
+                        tmem_wait_ld();
+                        float o[8];
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            float2 yv = __ffma2_rn(e2, make_float2(y2[e], y2[e + 1]), make_float2(y1[e], y1[e + 1]));
+                            yv = __ffma2_rn(d2, make_float2(uu[e], uu[e + 1]), yv);
+                            const float2 ov = __fmul2_rn(yv, gz[k2 * 4 + (e >> 1)]);
+                            o[e] = ov.x;
+                            o[e + 1] = ov.y;
+                        }
+                        if (tma_y) {
+                            *reinterpret_cast<uint4*>(rz + sw128_off(i, quarter * 2 + k2)) =
                                 make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]),
                                            pack_bf2(o[6], o[7]));
-                        } else {
-                            float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
-                            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-                            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+                        } else if (i < Qc) {
+                            TY* yrow = static_cast<TY*>(a.y) + ((size_t)span.row0 + t0 + i) * a.HP + (size_t)h * kP +
+                                       quarter * 16;
+                            if constexpr (sizeof(TY) == 2) {
+                                *reinterpret_cast<uint4*>(yrow + k2 * 8) =
+                                    make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]),
+                                               pack_bf2(o[6], o[7]));
+                            } else {
+                                float4* dst = reinterpret_cast<float4*>(yrow + k2 * 8);
+                                dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                                dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+                            }
                         }
                     }
                 }
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars[EPI_DONE]);
-            mbar_arrive(&bars[CS_FREE0 + buf]);  // this chunk's dt / cumsum buffer is no longer read
+            mbar_arrive(&bars[EPI_DONE0 + buf]);
+            mbar_arrive(&bars[CS_FREE0 + buf]);  // group A's reads of this chunk's cumsum buffer are done
         }
-        // final state: the running state after the last chunk (this thread's 16 columns p of row n = i)
-        if (!*abort_flag) {  // (an empty sequence passes its initial state through)
-            float sr[16];
-            tmem_ld16(tmem + lane_base + COL_SRUN + quarter * 16, sr);
-            tmem_wait_ld();
-            float* fs = a.final_state + ((size_t)b * a.H + h) * kP * kN;
+    } else {
+        // ---------------- group B: x conv and state pass ----------------
+        // Thread (quadrant q, half) owns token row i = TMEM lane i of the conv (channels 32*half .. +31) and
+        // state row n = i of the state pass (columns p = 32*half .. +31).
+        const int q = warp & 3;
+        const int half = (warp - kFirstGroupB) >> 2;
+        const int i = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        uint8_t* sS = sm + OFF_S;
+
+        // initial state (this thread's 32 columns): S_run in TMEM, bf16 copy in smem
+        {
+            // state row n = i exists for i < N; with N = 64 the rows 64..127 stay zero throughout
+            const float* init = a.init_state && i < a.N ? a.init_state + ((size_t)b * a.H + h) * kP * a.N : nullptr;
+#pragma unroll 1
+            for (int sub = 0; sub < 2; ++sub) {
+                const int col = 32 * half + 16 * sub;
+                float v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) fs[(size_t)(quarter * 16 + k) * kN + i] = sr[k];
+                for (int k = 0; k < 16; ++k) v[k] = init ? init[(size_t)(col + k) * a.N + i] : 0.f;
+                tmem_st16(tmem + lane_base + COL_SRUN + col, v);
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    uint4 w;
+                    w.x = pack_bf2(v[k2 * 8 + 0], v[k2 * 8 + 1]);
+                    w.y = pack_bf2(v[k2 * 8 + 2], v[k2 * 8 + 3]);
+                    w.z = pack_bf2(v[k2 * 8 + 4], v[k2 * 8 + 5]);
+                    w.w = pack_bf2(v[k2 * 8 + 6], v[k2 * 8 + 7]);
+                    *reinterpret_cast<uint4*>(sS + sw128_off(i, col / 8 + k2)) = w;
+                }
+            }
+            tmem_wait_st();
+        }
+
+        bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, Ls, i, half);
+        if (!ok) raise_abort(abort_flag);
+        for (int c = 0; c < nc && ok; ++c) {
+            const int buf = c & 1;
+            const float cs_last = s_cs[buf * 128 + kQ - 1];
+
+            // (f) state passing: S_run <- exp(cs_last) S_run + S_c  (lane i = state row n; 32 columns p)
+            if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            tc_fence_after();
+            {
+                const float dl = __expf(cs_last);
+                const float2 dl2 = make_float2(dl, dl);
+#pragma unroll 1
+                for (int sub = 0; sub < 2; ++sub) {
+                    const int col = 32 * half + 16 * sub;
+                    float sc[16], sr[16];
+                    tmem_ld16(tmem + lane_base + COL_SC + col, sc);
+                    tmem_ld16(tmem + lane_base + COL_SRUN + col, sr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 16; k += 2) {
+                        const float2 v = __ffma2_rn(dl2, make_float2(sr[k], sr[k + 1]), make_float2(sc[k], sc[k + 1]));
+                        sr[k] = v.x;
+                        sr[k + 1] = v.y;
+                    }
+                    tmem_st16(tmem + lane_base + COL_SRUN + col, sr);
+                    // S_prev is overwritten once Y2 = C S_prev^T of this chunk has read it
+                    if (sub == 0 && !warp_wait(&bars[EMPTY_BC], c & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int k2 = 0; k2 < 2; ++k2) {
+                        uint4 w;
+                        w.x = pack_bf2(sr[k2 * 8 + 0], sr[k2 * 8 + 1]);
+                        w.y = pack_bf2(sr[k2 * 8 + 2], sr[k2 * 8 + 3]);
+                        w.z = pack_bf2(sr[k2 * 8 + 4], sr[k2 * 8 + 5]);
+                        w.w = pack_bf2(sr[k2 * 8 + 6], sr[k2 * 8 + 7]);
+                        // the state entering chunk c+1
+                        *reinterpret_cast<uint4*>(sS + sw128_off(i, col / 8 + k2)) = w;
+                    }
+                }
+            }
+            if (!ok) { raise_abort(abort_flag); break; }
+            fence_async_smem();
+            mbar_arrive(&bars[SREADY]);          // S_prev(c+1) is in smem for Y2 of chunk c+1
+            mbar_arrive(&bars[CS_FREE0 + buf]);  // group B's reads of this chunk's cumsum buffer are done
+
+            // (c) the next chunk's x conv (its S_c then overlaps this chunk's Y = M X and epilogue)
+            if (c + 1 < nc && !conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, c + 1, nc, Ls, i, half)) {
+                raise_abort(abort_flag);
+                break;
+            }
+        }
+        // final state: the running state after the last chunk (this thread's 32 columns p of row n = i)
+        if (!*abort_flag && i < a.N) {  // (an empty sequence passes its initial state through)
+            tmem_wait_st();
+            float* fs = a.final_state + ((size_t)b * a.H + h) * kP * a.N;
+#pragma unroll 1
+            for (int sub = 0; sub < 2; ++sub) {
+                const int col = 32 * half + 16 * sub;
+                float sr[16];
+                tmem_ld16(tmem + lane_base + COL_SRUN + col, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 16; ++k) fs[(size_t)(col + k) * a.N + i] = sr[k];
+            }
         }
     }
 
@@ -937,8 +1013,11 @@ bool make_dt_map(CUtensorMap* m, const void* base, int64_t H, int64_t row_stride
 
 }  // namespace
 
+// d_state 64 runs the d_state 128 tiles with the upper 64 channels zero; a requested chunk of 64 runs in
+// chunks of 128 (the chunk length is a tiling choice: the results agree up to rounding).  The dt tiles are
+// loaded 8 heads wide, and dt rows must be a multiple of 16 bytes for the tensor map.
 bool prefill_tc_supported(int P, int N, int Q, int H, bool bf16) {
-    return bf16 && P == kP && N == kN && Q == kQ && H % 8 == 0;  // dt tiles are loaded 8 heads wide
+    return bf16 && P == kP && (N == kN || N == 64) && (Q == kQ || Q == 64) && H % 8 == 0;
 }
 
 size_t prefill_tc_workspace_bytes(int64_t batch, int64_t L, int G, int N) {

@@ -67,6 +67,14 @@ def test_path_and_workspace_queries(L):
     assert ops.prefill_path(dims(d_state=48), torch.bfloat16) == -2
     # fp32 activations and small shapes always take the CUDA-core path
     assert ops.prefill_path(dims(d_state=32, chunk=64, nheads=4, ngroups=1), torch.float32) == 2
+    # bf16 with P = 64, d_state 64 or 128, chunk 64 or 128 and nheads a multiple of 8: tensor cores
+    for N in (64, 128):
+        for Q in (64, 128):
+            assert ops.prefill_path(dims(d_state=N, chunk=Q), torch.bfloat16) == 1, (N, Q)
+            assert ops.prefill_path(dims(d_state=N, chunk=Q), torch.float32) == 2
+    assert ops.prefill_path(dims(d_state=32), torch.bfloat16) == 2
+    assert ops.prefill_path(dims(d_state=16), torch.bfloat16) == 2
+    assert ops.prefill_path(dims(nheads=12, ngroups=4), torch.bfloat16) == 2
     assert ops.prefill_workspace_bytes(dims(headdim=32), torch.bfloat16) == 0
 
 

@@ -45,6 +45,7 @@ SMALL = {
     "n16_per_head_groups": (Dims(1, 200, 4, 64, 16, 4, 128), torch.bfloat16, False),
     "n32_fp32_q128": (Dims(2, 140, 6, 64, 32, 3, 128), torch.float32, True),
     "n64_bf16": (Dims(1, 390, 8, 64, 64, 1, 128), torch.bfloat16, False),
+    "n32_bf16_cuda_core": (Dims(1, 200, 8, 64, 32, 2, 128), torch.bfloat16, True),
 }
 
 
@@ -92,13 +93,18 @@ def test_final_state_may_overwrite_init_state():
 
 
 def test_prefill_chunk_size_independence():
-    # Q is a tiling parameter of the method: Q = 64 and Q = 128 agree within rounding
+    # Q is a tiling parameter of the method: Q = 64 and Q = 128 agree within rounding.  The tensor-core
+    # path works in 128-token chunks whatever Q is asked for (so its Q = 64 call is bit-equal to its
+    # Q = 128 call); the CUDA-core path, fed the same values in fp32, scans in 64-token chunks.
     d = Dims(1, 700, 8, 64, 128, 2, 128)
     inp = dev_inputs(make_prefill_inputs(d, dtype=torch.bfloat16, seed=6, init_state=True))
     y1, f1, _ = gpu_prefill(inp, 128, y_dtype=torch.float32)
     y2, f2, _ = gpu_prefill(inp, 64, y_dtype=torch.float32)
-    assert_close(np64(y2), np64(y1), "y Q64 vs Q128", rel_tol=5e-3, abs_tol=2e-2)
-    assert_close(np64(f2), np64(f1), "final_state Q64 vs Q128", rel_tol=5e-3, abs_tol=2e-2)
+    assert torch.equal(y1, y2) and torch.equal(f1, f2)
+    inp32 = {k: (v.float() if v is not None and v.dtype == torch.bfloat16 else v) for k, v in inp.items()}
+    y3, f3, _ = gpu_prefill(inp32, 64)
+    assert_close(np64(y3), np64(y1), "y Q64 (CUDA cores) vs Q128 (tensor cores)", rel_tol=5e-3, abs_tol=2e-2)
+    assert_close(np64(f3), np64(f1), "final_state Q64 vs Q128", rel_tol=5e-3, abs_tol=2e-2)
 
 
 def test_prefill_split_sequence_continuation():
@@ -162,6 +168,16 @@ def test_prefill_full_size_sampled(name):
         assert_close(yg[b, :, h * P:(h + 1) * P], yo[b, :, h * P:(h + 1) * P], f"{name} y (b={b}, h={h})")
         assert_close(fg[b, h], fo[b, h], f"{name} final_state (b={b}, h={h})")
     assert np.array_equal(np64(cs), co)
+
+
+def test_tensor_core_path_covers_d_state_64_and_chunk_64():
+    # the 64-state and 64-token-chunk layers run on the tensor cores (chunks of 128 internally, the upper
+    # 64 state channels zero for d_state 64); results agree with the oracle as for the other shapes
+    for N, Q in ((64, 128), (64, 64), (128, 64)):
+        assert ops.prefill_path(ops.make_dims(2, 300, 16, 64, N, 2, Q), torch.bfloat16) == 1, (N, Q)
+    d = Dims(2, 300, 16, 64, 128, 2, 64)
+    inp = make_prefill_inputs(d, dtype=torch.bfloat16, seed=103, init_state=True, init_conv_state=True)
+    _check_full(inp, d.chunk, "n128_q64")
 
 
 def test_layer_shapes_take_the_tensor_core_path():

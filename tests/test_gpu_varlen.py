@@ -52,9 +52,15 @@ def test_varlen_tensor_core_path_matches_oracle(init):
     check_varlen(d, torch.bfloat16, EDGE, init, seed=301, tag=f"varlen tc init={init}")
 
 
+def test_varlen_tensor_core_path_d_state_64():
+    d = Dims(1, 1, 8, 64, 64, 2, 64)
+    assert ops.prefill_path(ops.make_dims(len(EDGE), sum(EDGE), 8, 64, 64, 2, 64), torch.bfloat16) == 1
+    check_varlen(d, torch.bfloat16, EDGE, True, seed=306, tag="varlen tc n64")
+
+
 @pytest.mark.parametrize("name,d,dtype", [
     ("fp32_q64", Dims(1, 1, 4, 64, 32, 1, 64), torch.float32),
-    ("bf16_n64", Dims(1, 1, 8, 64, 64, 2, 128), torch.bfloat16),
+    ("bf16_n32", Dims(1, 1, 8, 64, 32, 2, 128), torch.bfloat16),
 ])
 def test_varlen_cuda_core_path_matches_oracle(name, d, dtype):
     assert ops.prefill_path(ops.make_dims(len(EDGE), sum(EDGE), d.nheads, 64, d.d_state, d.ngroups, d.chunk),
