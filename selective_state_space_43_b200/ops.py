@@ -584,9 +584,29 @@ def host_pieces(L: int, chunk: int, segments=None) -> list:
     return [(r0, min(L, r0 + seg)) for r0 in range(0, L, seg)] if L > 0 else [(0, 0)]
 
 
-def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None):
+def _host_outputs(inputs: dict, out):
+    """The pinned host tensors prefill_host writes y, final_state and conv_state into: the caller's ``out``
+    (checked) or new ones."""
+    x = inputs["x"]
+    Bt, L, HP = x.shape
+    H = inputs["A"].shape[0]
+    G, N = inputs["B"].shape[2], inputs["B"].shape[3]
+    shapes = ((Bt, L, HP), (Bt, H, HP // H, N), (Bt, HP + 2 * G * N, 3))
+    dtypes = (x.dtype, torch.float32, x.dtype)
+    if out is None:
+        return [torch.empty(sh, dtype=dt, pin_memory=True) for sh, dt in zip(shapes, dtypes)]
+    out = list(out)
+    for name, t, sh, dt in zip(("y", "final_state", "conv_state"), out, shapes, dtypes):
+        if t.is_cuda or tuple(t.shape) != sh or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"out {name} must be a contiguous host tensor {sh} of {dt}")
+    return out
+
+
+def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None, out=None):
     """End-to-end prefill from HOST tensors (pinned for asynchronous copies): the inputs go to the device,
-    ssd_prefill runs, and y, final_state and conv_state come back into pinned host tensors.
+    ssd_prefill runs, and y, final_state and conv_state come back into pinned host tensors -- the caller's
+    ``out`` = (y, final_state, conv_state) when given (reused across calls, no host allocation), else new
+    ones (a pinned allocation of y's size per call).
 
     The sequence is cut into ``segments`` pieces on chunk boundaries (default: up to 8 pieces of at least
     two chunks).  Piece k is copied in on one side stream while piece k-1 is scanned on the current stream
@@ -601,8 +621,9 @@ def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None):
     Bt, L = x.shape[0], x.shape[1]
     h2d = sum(t.numel() * t.element_size() for t in inputs.values() if t is not None)
     pieces = host_pieces(L, chunk, segments)
+    y_host, fs_host, cs_host = _host_outputs(inputs, out)
     if len(pieces) <= 1:
-        return _prefill_host_whole(inputs, chunk, dev, h2d)
+        return _prefill_host_whole(inputs, chunk, dev, h2d, (y_host, fs_host, cs_host))
 
     cur = torch.cuda.current_stream(dev)
     s_in, s_out = _host_streams(dev)
@@ -614,7 +635,6 @@ def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None):
     for t in p.values():
         if t is not None:
             t.record_stream(cur)
-    y_host = torch.empty(tuple(x.shape), dtype=x.dtype, pin_memory=True)
     fs_prev, cs_prev = p["init_state"], p["init_conv_state"]
     for r0, r1 in pieces:
         with torch.cuda.stream(s_in):
@@ -640,8 +660,6 @@ def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None):
                 y_host[b, r0:r1].copy_(y[b], non_blocking=True)
         y.record_stream(s_out)
         fs_prev, cs_prev = fs, cs
-    fs_host = torch.empty(tuple(fs_prev.shape), dtype=fs_prev.dtype, pin_memory=True)
-    cs_host = torch.empty(tuple(cs_prev.shape), dtype=cs_prev.dtype, pin_memory=True)
     with torch.cuda.stream(s_out):
         fs_host.copy_(fs_prev, non_blocking=True)
         cs_host.copy_(cs_prev, non_blocking=True)
@@ -654,13 +672,13 @@ def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None):
     return outs, h2d, sum(t.numel() * t.element_size() for t in outs)
 
 
-def _prefill_host_whole(inputs: dict, chunk, dev, h2d):
+def _prefill_host_whole(inputs: dict, chunk, dev, h2d, outs):
     """prefill_host in one piece on the current stream: copy in, scan, copy out."""
     names = ("x", "dt", "B", "C", "z", "A", "D", "dt_bias", "conv_w", "conv_b", "init_state", "init_conv_state")
     d = {k: (None if inputs.get(k) is None else inputs[k].to(dev, non_blocking=True)) for k in names}
     y, fs, cs = prefill(d["x"], d["dt"], d["B"], d["C"], d["z"], d["A"], d["D"], d["dt_bias"], d["conv_w"],
                         d["conv_b"], d["init_state"], d["init_conv_state"], chunk=chunk)
-    outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (y, fs, cs)]
+    outs = list(outs)
     for o, t in zip(outs, (y, fs, cs)):
         o.copy_(t, non_blocking=True)
     return outs, h2d, sum(t.numel() * t.element_size() for t in outs)

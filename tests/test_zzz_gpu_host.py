@@ -56,3 +56,22 @@ def test_repeated_calls_reuse_memory_safely():
         y, fs, _ = gpu_prefill(dev_inputs(i), d.chunk)
         torch.cuda.synchronize()
         assert torch.equal(o[0], y.cpu()) and torch.equal(o[1], fs.cpu())
+
+
+@pytest.mark.parametrize("segments", [1, 4])
+def test_host_prefill_into_callers_pinned_outputs(segments):
+    # the caller's pinned output buffers are written in place and returned, on both the one-piece and the
+    # pipelined path; reusing them on the next call gives that call's results
+    d = Dims(2, 700, 16, 64, 128, 2, 128)
+    first = make_prefill_inputs(d, dtype=torch.bfloat16, seed=31, init_state=True, init_conv_state=True)
+    second = make_prefill_inputs(d, dtype=torch.bfloat16, seed=32, init_state=True, init_conv_state=True)
+    want = [ops.prefill_host(pinned(i), chunk=d.chunk, segments=segments)[0] for i in (first, second)]
+    torch.cuda.synchronize()
+    out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in want[0]]
+    for inp, w in zip((first, second), want):
+        got, _, _ = ops.prefill_host(pinned(inp), chunk=d.chunk, segments=segments, out=out)
+        torch.cuda.synchronize()
+        assert all(g is o for g, o in zip(got, out))
+        assert all(torch.equal(g, x) for g, x in zip(got, w))
+    with pytest.raises(ValueError):
+        ops.prefill_host(pinned(first), chunk=d.chunk, out=[out[0], out[1], out[1]])
