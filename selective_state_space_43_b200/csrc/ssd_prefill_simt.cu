@@ -83,20 +83,35 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
         const int Qc = (int)(Ls - t0 < Q ? Ls - t0 : Q);
         __syncthreads();  // previous chunk fully consumed
 
-        // 1. conv + SiLU of the head's channels, dt and the in-chunk cumsum.
+        // 1. conv + SiLU of the head's channels, dt and the in-chunk cumsum.  Channel-major: a thread slides
+        //    a 4-tap window down its channel's rows, the loads of kRowBlk rows issued before their FMAs
+        //    (neighbouring threads read neighbouring channels of a row).
         constexpr int CH = kP + 2 * N;
-        for (int i = tid; i < Q * CH; i += kThreads) {
-            const int t = i / CH, j = i % CH;
-            if (t >= Qc) continue;
+        constexpr int kRowBlk = 8;
+        for (int j = tid; j < CH; j += kThreads) {
             const int ch = j < kP ? cx + j : (j < kP + N ? cb + (j - kP) : cc + (j - kP - N));
-            const float* w = a.conv_w + (size_t)ch * 4;
-            float acc = a.conv_b[ch];
+            const float4 w = *reinterpret_cast<const float4*>(a.conv_w + (size_t)ch * 4);
+            const float bias = a.conv_b[ch];
+            float h0 = raw_at<T>(a, b, span.row0, t0 - 3, ch), h1 = raw_at<T>(a, b, span.row0, t0 - 2, ch),
+                  h2 = raw_at<T>(a, b, span.row0, t0 - 1, ch);
+            for (int tb = 0; tb < Qc; tb += kRowBlk) {
+                float r[kRowBlk];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc += w[k] * raw_at<T>(a, b, span.row0, t0 + t - 3 + k, ch);
-            const float u = silu_f(acc);
-            if (j < kP) sX[t * kP + j] = u;
-            else if (j < kP + N) sB[t * NB + (j - kP)] = u;
-            else sC[t * N + (j - kP - N)] = u;
+                for (int k = 0; k < kRowBlk; ++k) r[k] = tb + k < Qc ? raw_at<T>(a, b, span.row0, t0 + tb + k, ch) : 0.f;
+#pragma unroll
+                for (int k = 0; k < kRowBlk; ++k) {
+                    const int t = tb + k;
+                    const float u = silu_f(bias + w.x * h0 + w.y * h1 + w.z * h2 + w.w * r[k]);
+                    h0 = h1;
+                    h1 = h2;
+                    h2 = r[k];
+                    if (t < Qc) {
+                        if (j < kP) sX[t * kP + j] = u;
+                        else if (j < kP + N) sB[t * NB + (j - kP)] = u;
+                        else sC[t * N + (j - kP - N)] = u;
+                    }
+                }
+            }
         }
         if (warp == 0) {
             constexpr int PER = Q / 32;
@@ -130,27 +145,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
         const float cs_last = sCs[Qc - 1];
         for (int s = tid; s < Q; s += kThreads) sE[s] = s < Qc ? __expf(cs_last - sCs[s]) * sDt[s] : 0.f;
 
-        // 2. outputs, one row t per warp at a time (state S is the previous chunk's)
+        // 2. outputs, one row t per warp at a time (state S is the previous chunk's); the dot products run
+        //    four independent partial sums so that their shared-memory loads overlap
         float* wrow = sW + warp * Q;
         for (int t = warp; t < Qc; t += kWarps) {
             const float cst = sCs[t];
             for (int s = lane; s < Q; s += 32) {
                 float gsum = 0.f;
                 if (s <= t) {
-#pragma unroll 8
-                    for (int n = 0; n < N; ++n) gsum += sC[t * N + n] * sB[s * NB + n];
-                    gsum *= __expf(cst - sCs[s]) * sDt[s];
+                    float g4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                    for (int n = 0; n < N; n += 4) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) g4[e] += sC[t * N + n + e] * sB[s * NB + n + e];
+                    }
+                    gsum = ((g4[0] + g4[1]) + (g4[2] + g4[3])) * (__expf(cst - sCs[s]) * sDt[s]);
                 }
                 wrow[s] = gsum;
             }
             __syncwarp();
             const float dec = __expf(cst);
             for (int p = lane; p < kP; p += 32) {
-                float acc = 0.f;
-                for (int s = 0; s <= t; ++s) acc += wrow[s] * sX[s * kP + p];
-                float off = 0.f;
-#pragma unroll 8
-                for (int n = 0; n < N; ++n) off += sC[t * N + n] * sS[p * NB + n];
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                int s = 0;
+                for (; s + 3 <= t; s += 4) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) a4[e] += wrow[s + e] * sX[(s + e) * kP + p];
+                }
+                for (; s <= t; ++s) a4[0] += wrow[s] * sX[s * kP + p];
+                const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+                float o4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int n = 0; n < N; n += 4) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o4[e] += sC[t * N + n + e] * sS[p * NB + n + e];
+                }
+                const float off = (o4[0] + o4[1]) + (o4[2] + o4[3]);
                 const float yv = acc + dec * off + Dh * sX[t * kP + p];
                 const size_t row = (size_t)span.row0 + t0 + t;
                 const size_t o = row * a.HP + cx + p;
@@ -165,9 +195,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
         const float dl = __expf(cs_last);
         for (int i = tid; i < kP * N; i += kThreads) {
             const int p = i / N, n = i % N;
-            float acc = 0.f;
-            for (int s = 0; s < Qc; ++s) acc += sE[s] * sX[s * kP + p] * sB[s * NB + n];
-            sS[p * NB + n] = dl * sS[p * NB + n] + acc;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            int s = 0;
+            for (; s + 4 <= Qc; s += 4) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) a4[e] += sE[s + e] * sX[(s + e) * kP + p] * sB[(s + e) * NB + n];
+            }
+            for (; s < Qc; ++s) a4[0] += sE[s] * sX[s * kP + p] * sB[s * NB + n];
+            sS[p * NB + n] = dl * sS[p * NB + n] + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
         }
     }
     __syncthreads();
