@@ -140,6 +140,20 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
+// Two (three) phases at once: the try_waits are issued back to back, so when the phases have completed
+// (the usual case in the pipeline's steady state) their latencies overlap; otherwise one by one.
+__device__ __forceinline__ bool warp_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1,
+                                           volatile int* abort_flag) {
+    const bool r0 = mbar_try_wait(b0, p0), r1 = mbar_try_wait(b1, p1);
+    if (__all_sync(0xffffffffu, r0 & r1)) return true;
+    return warp_wait(b0, p0, abort_flag) && warp_wait(b1, p1, abort_flag);
+}
+__device__ __forceinline__ bool warp_wait3(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
+                                           uint32_t p2, volatile int* abort_flag) {
+    const bool r0 = mbar_try_wait(b0, p0), r1 = mbar_try_wait(b1, p1), r2 = mbar_try_wait(b2, p2);
+    if (__all_sync(0xffffffffu, r0 & r1 & r2)) return true;
+    return warp_wait(b0, p0, abort_flag) && warp_wait(b1, p1, abort_flag) && warp_wait(b2, p2, abort_flag);
+}
 
 // SiLU(v) = v sigmoid(v) with sigmoid(v) = (1 + tanh(v/2)) / 2: one MUFU
 // operation (the hardware tanh approximation, relative error ~2^-11) instead
@@ -194,12 +208,18 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
                                            uint32_t tmem, uint32_t lane_base, int cc, int nc, int64_t Ls, int i,
                                            int half) {
     const int buf = cc & 1;
-    if (!warp_wait(&bars[CS_READY0 + buf], (cc >> 1) & 1, abort_flag)) return false;
-    if (!warp_wait(&bars[FULL_RAW0 + buf], (cc >> 1) & 1, abort_flag)) return false;
-    // the raw history rows were written by other threads in the previous chunk's conv
-    if (cc >= 1 && !warp_wait(&bars[XREADY0 + ((cc - 1) & 1)], ((cc - 1) >> 1) & 1, abort_flag)) return false;
-    // the X tile and the conv output of this parity were last read by chunk cc-2's Y MMA and epilogue
-    if (cc >= 2 && !warp_wait(&bars[EPI_DONE0 + buf], ((cc - 2) >> 1) & 1, abort_flag)) return false;
+    // this chunk's cumsum (its raw x tile arrived before it) and raw x
+    if (!warp_wait2(&bars[CS_READY0 + buf], (cc >> 1) & 1, &bars[FULL_RAW0 + buf], (cc >> 1) & 1, abort_flag))
+        return false;
+    // the raw history rows were written by other threads in the previous chunk's conv; the X tile and the
+    // conv output of this parity were last read by chunk cc-2's Y MMA and epilogue
+    if (cc >= 2) {
+        if (!warp_wait2(&bars[XREADY0 + ((cc - 1) & 1)], ((cc - 1) >> 1) & 1, &bars[EPI_DONE0 + buf],
+                        ((cc - 2) >> 1) & 1, abort_flag))
+            return false;
+    } else if (cc == 1 && !warp_wait(&bars[XREADY0], 0, abort_flag)) {
+        return false;
+    }
     const int64_t t0 = (int64_t)cc * kQ;
     const int Qc = (int)(Ls - t0 < kQ ? Ls - t0 : kQ);
     const bool valid = i < Qc;
@@ -249,6 +269,8 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
             xpo[k] = pack_bf2(up.x, up.y);
         }
         tmem_st16(tmem + lane_base + COL_U + buf * 64 + quarter * 16, u);
+        // X' is single-buffered: the previous chunk's S_c must have read it
+        if (sub == 0 && cc >= 1 && !warp_wait(&bars[SC_FULL], (cc - 1) & 1, abort_flag)) return false;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
             *reinterpret_cast<uint4*>(sX + sw128_off(i, quarter * 2 + k)) =
@@ -269,6 +291,87 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
     tc_fence_before();
     mbar_arrive(&bars[XREADY0 + buf]);
     return true;
+}
+
+// The running state is split between the two compute groups by columns: the thread (quadrant q, half) of
+// group A owns state columns 32*half .. +15 of row n = i (= TMEM lane i), the matching thread of group B
+// columns 32*half + 16 .. +31.  Each writes its part of the bf16 copy that is the Y2 operand and arrives on
+// SREADY (256 + 256 arrivals per phase; phase 0 = the initial state, phase c+1 = the state entering chunk c+1).
+
+// Initial state (or zeros) of the calling thread's 16 columns col .. col+15: S_run in TMEM, bf16 in smem.
+__device__ __forceinline__ void state_init(const PrefillArgs& a, uint8_t* sm, uint64_t* bars, uint32_t tmem,
+                                           uint32_t lane_base, int b, int h, int i, int col) {
+    // state row n = i exists for i < N; with N = 64 the rows 64..127 stay zero throughout
+    const float* init = a.init_state && i < a.N ? a.init_state + ((size_t)b * a.H + h) * kP * a.N : nullptr;
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = init ? init[(size_t)(col + k) * a.N + i] : 0.f;
+    tmem_st16(tmem + lane_base + COL_SRUN + col, v);
+    uint8_t* sS = sm + OFF_S;
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2) {
+        uint4 w;
+        w.x = pack_bf2(v[k2 * 8 + 0], v[k2 * 8 + 1]);
+        w.y = pack_bf2(v[k2 * 8 + 2], v[k2 * 8 + 3]);
+        w.z = pack_bf2(v[k2 * 8 + 4], v[k2 * 8 + 5]);
+        w.w = pack_bf2(v[k2 * 8 + 6], v[k2 * 8 + 7]);
+        *reinterpret_cast<uint4*>(sS + sw128_off(i, col / 8 + k2)) = w;
+    }
+    tmem_wait_st();
+    fence_async_smem();
+    mbar_arrive(&bars[SREADY]);
+}
+
+// State pass of chunk c for the calling thread's 16 columns: S_run <- exp(cs_last) S_run + S_c (TMEM), then,
+// once Y2 and S_c of chunk c are complete, the bf16 state entering chunk c+1 into smem.  Returns false if a
+// wait gave up.
+__device__ __forceinline__ bool state_half(uint8_t* sm, uint64_t* bars, volatile int* abort_flag, uint32_t tmem,
+                                           uint32_t lane_base, int c, float cs_last, int i, int col) {
+    if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) return false;
+    tc_fence_after();
+    const float dl = __expf(cs_last);
+    const float2 dl2 = make_float2(dl, dl);
+    float sc[16], sr[16];
+    tmem_ld16(tmem + lane_base + COL_SC + col, sc);
+    tmem_ld16(tmem + lane_base + COL_SRUN + col, sr);
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 16; k += 2) {
+        const float2 v = __ffma2_rn(dl2, make_float2(sr[k], sr[k + 1]), make_float2(sc[k], sc[k + 1]));
+        sr[k] = v.x;
+        sr[k + 1] = v.y;
+    }
+    tmem_st16(tmem + lane_base + COL_SRUN + col, sr);
+    // S_prev is overwritten once Y2 = C S_prev^T of this chunk has read it
+    if (!warp_wait(&bars[EMPTY_BC], c & 1, abort_flag)) return false;
+    uint8_t* sS = sm + OFF_S;
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2) {
+        uint4 w;
+        w.x = pack_bf2(sr[k2 * 8 + 0], sr[k2 * 8 + 1]);
+        w.y = pack_bf2(sr[k2 * 8 + 2], sr[k2 * 8 + 3]);
+        w.z = pack_bf2(sr[k2 * 8 + 4], sr[k2 * 8 + 5]);
+        w.w = pack_bf2(sr[k2 * 8 + 6], sr[k2 * 8 + 7]);
+        *reinterpret_cast<uint4*>(sS + sw128_off(i, col / 8 + k2)) = w;  // the state entering chunk c+1
+    }
+    tmem_wait_st();
+    tc_fence_before();  // this chunk's S_c reads are done before the next S_c MMA may overwrite it
+    fence_async_smem();
+    mbar_arrive(&bars[SREADY]);
+    return true;
+}
+
+// Final state of the calling thread's 16 columns (rows n < N).
+__device__ __forceinline__ void state_final(const PrefillArgs& a, uint32_t tmem, uint32_t lane_base, int b, int h,
+                                            int i, int col) {
+    if (i >= a.N) return;
+    tmem_wait_st();
+    float sr[16];
+    tmem_ld16(tmem + lane_base + COL_SRUN + col, sr);
+    tmem_wait_ld();
+    float* fs = a.final_state + ((size_t)b * a.H + h) * kP * a.N;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) fs[(size_t)(col + k) * a.N + i] = sr[k];
 }
 
 // kVarlen: a packed variable-length batch (a.cu set); the batch x L layout otherwise.
@@ -303,9 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int k = 0; k < NBAR; ++k) {
             uint32_t cnt = 1;
-            if (k == XREADY0 || k == XREADY1 || k == SREADY) cnt = kGroupThreads;       // group B
+            if (k == XREADY0 || k == XREADY1) cnt = kGroupThreads;                      // group B
             if (k == EPI_DONE0 || k == EPI_DONE1 || k == MREADY) cnt = kGroupThreads;   // group A
-            if (k == CS_FREE0 || k == CS_FREE1) cnt = 2 * kGroupThreads;               // both
+            if (k == CS_FREE0 || k == CS_FREE1 || k == SREADY) cnt = 2 * kGroupThreads; // both
             if (k == CS_READY0 || k == CS_READY1 || k == TAB_READY) cnt = 32;
             mbar_init(&bars[k], cnt);
         }
@@ -568,21 +671,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 tc_fence_after();
                 mma_k128<false, false>(tmem + COL_G, dC, dB, ID_G);
                 mma_commit(&bars[G_FULL]);
-                // chunk state S_c = B^T X'  (needs this chunk's conv)
-                if (!mbar_wait(&bars[XREADY0 + (c & 1)], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
-                tc_fence_after();
-                mma_k128<true, true>(tmem + COL_SC, dBt, dXp, ID_SC);
-                mma_commit(&bars[SC_FULL]);
-                // Y2 = C S_prev^T, once the previous chunk's epilogue has read the previous Y2 and the state
-                // pass has written S_prev
-                if (c >= 1 && (!mbar_wait(&bars[EPI_DONE0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag) ||
-                               !mbar_wait(&bars[SREADY], (c - 1) & 1, abort_flag))) {
+                // Y2 = C S_prev^T, once the state passes of the previous chunk (or the initial state, phase 0)
+                // have written S_prev and the previous chunk's epilogue has read the previous Y2
+                if (!mbar_wait(&bars[SREADY], c & 1, abort_flag) ||
+                    (c >= 1 && !mbar_wait(&bars[EPI_DONE0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag))) {
                     raise_abort(abort_flag);
                     break;
                 }
                 tc_fence_after();
                 mma_k128<false, true>(tmem + COL_Y2, dC, dS, ID_Y2);
-                mma_commit(&bars[EMPTY_BC]);  // B / C tiles and S_prev free
+                // chunk state S_c = B^T X' (needs this chunk's conv; the S_c columns are free since both state
+                // passes of the previous chunk, in the SREADY phase waited above, have read them)
+                if (!mbar_wait(&bars[XREADY0 + (c & 1)], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+                tc_fence_after();
+                mma_k128<true, true>(tmem + COL_SC, dBt, dXp, ID_SC);
+                mma_commit(&bars[SC_FULL]);
+                mma_commit(&bars[EMPTY_BC]);  // B / C tiles and S_prev free (Y2 and S_c complete)
                 // Y = M X, once every row's decay mask is written
                 if (!mbar_wait(&bars[MREADY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
                 tc_fence_after();
@@ -594,26 +698,29 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             mbar_wait(&bars[MMA_DONE], 0, nullptr, 100000000ull);
         }
     } else if (warp < kFirstGroupB) {
-        // ---------------- group A: decay mask and epilogue of each chunk ----------------
+        // ---------------- group A: decay mask, half of the state pass, epilogue ----------------
         // Thread (quadrant q, half) owns token row i = TMEM lane i, the 8-column groups 2*half and 2*half+1
-        // of each 32-column mask block, and output columns 32*half .. +31.
+        // of each 32-column mask block, state columns 32*half .. +15 and output columns 32*half .. +31.
         const int q = warp & 3;                            // TMEM lane quadrant of this warp
         const int half = (warp - kFirstCompute) >> 2;      // 0 or 1
         const int i = q * 32 + lane;                       // token row / TMEM lane
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float Dh = a.D[h];
         uint8_t* sMm = sm + OFF_M;
+        state_init(a, sm, bars, tmem, lane_base, b, h, i, 32 * half);
         for (int c = 0; c < nc; ++c) {
             const int buf = c & 1;
             const int64_t t0 = (int64_t)c * kQ;
             const int Qc = (int)(Ls - t0 < kQ ? Ls - t0 : kQ);
             const bool tma_y = kTmaStoreY && tma_y_chunk<kVarlen>(Ls, c);  // else y is stored from registers
 
-            // (e) decay mask of row i
-            if (!warp_wait(&bars[G_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            // (e) decay mask of row i, once G and this chunk's decay tables (written after its cumsum, so the
+            // cumsum buffer is ready too) are
+            if (!warp_wait2(&bars[G_FULL], c & 1, &bars[TAB_READY], c & 1, abort_flag)) {
+                raise_abort(abort_flag);
+                break;
+            }
             tc_fence_after();
-            // the decay tables of this chunk (written after its cumsum, so the cumsum buffer is ready too)
-            if (!warp_wait(&bars[TAB_READY], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
             {
                 // decay of row i (group gi) against column group g = 4 kb + quarter (columns 8g .. 8g+7):
                 //   g < gi: exp(cs_i - cs_end(gi-1)) exp(cs_end(gi-1) - cs_end(g)) exp(cs_end(g) - cs_j) dt_j
@@ -626,40 +733,44 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 const float4* drow = reinterpret_cast<const float4*>(sm + OFF_DG) + (gi * 8 + (i & 7)) * 2;
                 const float* colf_b = s_colf + buf * 128;
 #pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    float gv[16];
-                    if (kb <= q) {  // warp-uniform: blocks right of the diagonal block are zero
-                        tmem_ld16(tmem + lane_base + COL_G + kb * 32 + half * 16, gv);
-                        tmem_wait_ld();
-                    }
+                for (int kb2 = 0; kb2 < 4; kb2 += 2) {
+                    float gv[2][16];  // two 32-column blocks per TMEM round trip (warp-uniform: blocks right of
+                                      // the diagonal block are zero and not loaded)
+                    if (kb2 <= q) tmem_ld16(tmem + lane_base + COL_G + kb2 * 32 + half * 16, gv[0]);
+                    if (kb2 + 1 <= q) tmem_ld16(tmem + lane_base + COL_G + (kb2 + 1) * 32 + half * 16, gv[1]);
+                    if (kb2 <= q) tmem_wait_ld();
 #pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
-                        const int quarter = 2 * half + sub;
-                        const int g = 4 * kb + quarter;
-                        uint4 packed = make_uint4(0u, 0u, 0u, 0u);
-                        if (kb <= q && g <= gi) {
-                            float4 fa, fb;
-                            if (g < gi) {
-                                const float4* colf = reinterpret_cast<const float4*>(colf_b + 8 * g);
-                                const float rf = rfac * pk[sub][kb];
-                                fa = colf[0];
-                                fb = colf[1];
-                                fa = make_float4(fa.x * rf, fa.y * rf, fa.z * rf, fa.w * rf);
-                                fb = make_float4(fb.x * rf, fb.y * rf, fb.z * rf, fb.w * rf);
-                            } else {
-                                fa = drow[0];
-                                fb = drow[1];
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const int kb = kb2 + kk;
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub) {
+                            const int quarter = 2 * half + sub;
+                            const int g = 4 * kb + quarter;
+                            uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+                            if (kb <= q && g <= gi) {
+                                float4 fa, fb;
+                                if (g < gi) {
+                                    const float4* colf = reinterpret_cast<const float4*>(colf_b + 8 * g);
+                                    const float rf = rfac * pk[sub][kb];
+                                    fa = colf[0];
+                                    fb = colf[1];
+                                    fa = make_float4(fa.x * rf, fa.y * rf, fa.z * rf, fa.w * rf);
+                                    fb = make_float4(fb.x * rf, fb.y * rf, fb.z * rf, fb.w * rf);
+                                } else {
+                                    fa = drow[0];
+                                    fb = drow[1];
+                                }
+                                const float* gg = gv[kk] + 8 * sub;
+                                const float2 m0 = __fmul2_rn(make_float2(gg[0], gg[1]), make_float2(fa.x, fa.y));
+                                const float2 m1 = __fmul2_rn(make_float2(gg[2], gg[3]), make_float2(fa.z, fa.w));
+                                const float2 m2 = __fmul2_rn(make_float2(gg[4], gg[5]), make_float2(fb.x, fb.y));
+                                const float2 m3 = __fmul2_rn(make_float2(gg[6], gg[7]), make_float2(fb.z, fb.w));
+                                packed = make_uint4(pack_bf2(m0.x, m0.y), pack_bf2(m1.x, m1.y), pack_bf2(m2.x, m2.y),
+                                                    pack_bf2(m3.x, m3.y));
                             }
-                            const float* gg = gv + 8 * sub;
-                            const float2 m0 = __fmul2_rn(make_float2(gg[0], gg[1]), make_float2(fa.x, fa.y));
-                            const float2 m1 = __fmul2_rn(make_float2(gg[2], gg[3]), make_float2(fa.z, fa.w));
-                            const float2 m2 = __fmul2_rn(make_float2(gg[4], gg[5]), make_float2(fb.x, fb.y));
-                            const float2 m3 = __fmul2_rn(make_float2(gg[6], gg[7]), make_float2(fb.z, fb.w));
-                            packed = make_uint4(pack_bf2(m0.x, m0.y), pack_bf2(m1.x, m1.y), pack_bf2(m2.x, m2.y),
-                                                pack_bf2(m3.x, m3.y));
+                            *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 +
+                                                      sw128_off(i, (kb & 1) * 4 + quarter)) = packed;
                         }
-                        *reinterpret_cast<uint4*>(sMm + (kb >> 1) * 16384 + sw128_off(i, (kb & 1) * 4 + quarter)) =
-                            packed;
                     }
                 }
             }
@@ -667,12 +778,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             tc_fence_before();
             mbar_arrive(&bars[MREADY]);
 
-            // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 32*half .. +31
-            if (!warp_wait(&bars[FULL_Z], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
-            if (!warp_wait(&bars[Y_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
-            // the conv output of this chunk (written by group B; complete before the Y MMA was issued, waited
-            // on here as well so that the TMEM stores are ordered before this group's loads directly)
-            if (!warp_wait(&bars[XREADY0 + buf], (c >> 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
+            // (f) this thread's half of the state pass of chunk c
+            if (!state_half(sm, bars, abort_flag, tmem, lane_base, c, s_cs[buf * 128 + kQ - 1], i, 32 * half)) {
+                raise_abort(abort_flag);
+                break;
+            }
+
+            // (g) epilogue: y = (Y + exp(cs_i) Y2 + D x) SiLU(z), columns 32*half .. +31, once z, Y (Y2 before
+            // it) and this chunk's conv output (written by group B; complete before the Y MMA was issued,
+            // waited on here as well so that its TMEM stores are ordered before these loads directly) are in
+            if (!warp_wait3(&bars[FULL_Z], c & 1, &bars[Y_FULL], c & 1, &bars[XREADY0 + buf], (c >> 1) & 1,
+                            abort_flag)) {
+                raise_abort(abort_flag);
+                break;
+            }
             tc_fence_after();
             {
                 uint8_t* rz = sm + OFF_Z;  // z in, y out (same positions, this thread's only)
@@ -681,7 +800,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
 #pragma unroll 1
                 for (int sub = 0; sub < 2; ++sub) {
                     const int quarter = 2 * half + sub;
-                    // the gate SiLU(z) of these 16 columns
+                    float y1[16], y2[16], uu[16];
+                    tmem_ld16(tmem + lane_base + COL_Y + quarter * 16, y1);
+                    tmem_ld16(tmem + lane_base + COL_Y2 + quarter * 16, y2);
+                    tmem_ld16(tmem + lane_base + COL_U + buf * 64 + quarter * 16, uu);
+                    // the gate SiLU(z) of these 16 columns while the TMEM loads are in flight
                     float2 gz[8];
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
@@ -690,18 +813,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
 #pragma unroll
                         for (int e = 0; e < 4; ++e) gz[k2 * 4 + e] = silu2(make_float2(bf_lo(zr[e]), bf_hi(zr[e])));
                     }
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int k2 = 0; k2 < 2; ++k2) {  // 8 columns per TMEM round trip
-                        float y1[8], y2[8], uu[8];
-                        tmem_ld8(tmem + lane_base + COL_Y + quarter * 16 + k2 * 8, y1);
-                        tmem_ld8(tmem + lane_base + COL_Y2 + quarter * 16 + k2 * 8, y2);
-                        tmem_ld8(tmem + lane_base + COL_U + buf * 64 + quarter * 16 + k2 * 8, uu);
-                        tmem_wait_ld();
+                    for (int k2 = 0; k2 < 2; ++k2) {
                         float o[8];
 #pragma unroll
                         for (int e = 0; e < 8; e += 2) {
-                            float2 yv = __ffma2_rn(e2, make_float2(y2[e], y2[e + 1]), make_float2(y1[e], y1[e + 1]));
-                            yv = __ffma2_rn(d2, make_float2(uu[e], uu[e + 1]), yv);
+                            const int f = k2 * 8 + e;
+                            float2 yv = __ffma2_rn(e2, make_float2(y2[f], y2[f + 1]), make_float2(y1[f], y1[f + 1]));
+                            yv = __ffma2_rn(d2, make_float2(uu[f], uu[f + 1]), yv);
                             const float2 ov = __fmul2_rn(yv, gz[k2 * 4 + (e >> 1)]);
                             o[e] = ov.x;
                             o[e + 1] = ov.y;
@@ -731,108 +851,34 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             mbar_arrive(&bars[EPI_DONE0 + buf]);
             mbar_arrive(&bars[CS_FREE0 + buf]);  // group A's reads of this chunk's cumsum buffer are done
         }
+        // final state of this thread's columns (an empty sequence passes its initial state through)
+        if (!*abort_flag) state_final(a, tmem, lane_base, b, h, i, 32 * half);
     } else {
-        // ---------------- group B: x conv and state pass ----------------
+        // ---------------- group B: x conv (one chunk ahead), the other half of the state pass ----------------
         // Thread (quadrant q, half) owns token row i = TMEM lane i of the conv (channels 32*half .. +31) and
-        // state row n = i of the state pass (columns p = 32*half .. +31).
+        // state columns 32*half + 16 .. +31 of row n = i.
         const int q = warp & 3;
         const int half = (warp - kFirstGroupB) >> 2;
         const int i = q * 32 + lane;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        uint8_t* sS = sm + OFF_S;
-
-        // initial state (this thread's 32 columns): S_run in TMEM, bf16 copy in smem
-        {
-            // state row n = i exists for i < N; with N = 64 the rows 64..127 stay zero throughout
-            const float* init = a.init_state && i < a.N ? a.init_state + ((size_t)b * a.H + h) * kP * a.N : nullptr;
-#pragma unroll 1
-            for (int sub = 0; sub < 2; ++sub) {
-                const int col = 32 * half + 16 * sub;
-                float v[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) v[k] = init ? init[(size_t)(col + k) * a.N + i] : 0.f;
-                tmem_st16(tmem + lane_base + COL_SRUN + col, v);
-#pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                    uint4 w;
-                    w.x = pack_bf2(v[k2 * 8 + 0], v[k2 * 8 + 1]);
-                    w.y = pack_bf2(v[k2 * 8 + 2], v[k2 * 8 + 3]);
-                    w.z = pack_bf2(v[k2 * 8 + 4], v[k2 * 8 + 5]);
-                    w.w = pack_bf2(v[k2 * 8 + 6], v[k2 * 8 + 7]);
-                    *reinterpret_cast<uint4*>(sS + sw128_off(i, col / 8 + k2)) = w;
-                }
-            }
-            tmem_wait_st();
-        }
-
+        state_init(a, sm, bars, tmem, lane_base, b, h, i, 32 * half + 16);
         bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, Ls, i, half);
         if (!ok) raise_abort(abort_flag);
         for (int c = 0; c < nc && ok; ++c) {
             const int buf = c & 1;
-            const float cs_last = s_cs[buf * 128 + kQ - 1];
-
-            // (f) state passing: S_run <- exp(cs_last) S_run + S_c  (lane i = state row n; 32 columns p)
-            if (!warp_wait(&bars[SC_FULL], c & 1, abort_flag)) { raise_abort(abort_flag); break; }
-            tc_fence_after();
-            {
-                const float dl = __expf(cs_last);
-                const float2 dl2 = make_float2(dl, dl);
-#pragma unroll 1
-                for (int sub = 0; sub < 2; ++sub) {
-                    const int col = 32 * half + 16 * sub;
-                    float sc[16], sr[16];
-                    tmem_ld16(tmem + lane_base + COL_SC + col, sc);
-                    tmem_ld16(tmem + lane_base + COL_SRUN + col, sr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 16; k += 2) {
-                        const float2 v = __ffma2_rn(dl2, make_float2(sr[k], sr[k + 1]), make_float2(sc[k], sc[k + 1]));
-                        sr[k] = v.x;
-                        sr[k + 1] = v.y;
-                    }
-                    tmem_st16(tmem + lane_base + COL_SRUN + col, sr);
-                    // S_prev is overwritten once Y2 = C S_prev^T of this chunk has read it
-                    if (sub == 0 && !warp_wait(&bars[EMPTY_BC], c & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int k2 = 0; k2 < 2; ++k2) {
-                        uint4 w;
-                        w.x = pack_bf2(sr[k2 * 8 + 0], sr[k2 * 8 + 1]);
-                        w.y = pack_bf2(sr[k2 * 8 + 2], sr[k2 * 8 + 3]);
-                        w.z = pack_bf2(sr[k2 * 8 + 4], sr[k2 * 8 + 5]);
-                        w.w = pack_bf2(sr[k2 * 8 + 6], sr[k2 * 8 + 7]);
-                        // the state entering chunk c+1
-                        *reinterpret_cast<uint4*>(sS + sw128_off(i, col / 8 + k2)) = w;
-                    }
-                }
-            }
-            if (!ok) { raise_abort(abort_flag); break; }
-            fence_async_smem();
-            mbar_arrive(&bars[SREADY]);          // S_prev(c+1) is in smem for Y2 of chunk c+1
-            mbar_arrive(&bars[CS_FREE0 + buf]);  // group B's reads of this chunk's cumsum buffer are done
-
-            // (c) the next chunk's x conv (its S_c then overlaps this chunk's Y = M X and epilogue)
+            // (c) the next chunk's x conv first: this chunk's S_c (needed below) completes meanwhile
             if (c + 1 < nc && !conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, c + 1, nc, Ls, i, half)) {
                 raise_abort(abort_flag);
                 break;
             }
-        }
-        // final state: the running state after the last chunk (this thread's 32 columns p of row n = i)
-        if (!*abort_flag && i < a.N) {  // (an empty sequence passes its initial state through)
-            tmem_wait_st();
-            float* fs = a.final_state + ((size_t)b * a.H + h) * kP * a.N;
-#pragma unroll 1
-            for (int sub = 0; sub < 2; ++sub) {
-                const int col = 32 * half + 16 * sub;
-                float sr[16];
-                tmem_ld16(tmem + lane_base + COL_SRUN + col, sr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 16; ++k) fs[(size_t)(col + k) * a.N + i] = sr[k];
+            // (f) this thread's half of the state pass of chunk c
+            if (!state_half(sm, bars, abort_flag, tmem, lane_base, c, s_cs[buf * 128 + kQ - 1], i, 32 * half + 16)) {
+                raise_abort(abort_flag);
+                break;
             }
+            mbar_arrive(&bars[CS_FREE0 + buf]);  // group B's reads of this chunk's cumsum buffer are done
         }
+        if (!*abort_flag) state_final(a, tmem, lane_base, b, h, i, 32 * half + 16);
     }
 
     __syncthreads();

@@ -52,10 +52,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // try_wait (whose own short, system-chosen suspension returns as soon as the
 // phase completes) rather than a long suspend hint, which was seen to wake the
 // thread up to ~1000 cycles late.
+// A phase that has already completed returns at once, before the abort flag is read (one try_wait on the
+// fast path); once the flag is set, a wait that has to wait gives up within 64 polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns = 2000000000ull) {
-    if (abort && *abort) return false;
     if (mbar_try_wait(bar, parity)) return true;
+    if (abort && *abort) return false;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
