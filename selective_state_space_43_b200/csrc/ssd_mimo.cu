@@ -129,7 +129,7 @@ using sm100::mbar_wait;
 
 // grid batch * H, kT threads, smem_bytes(R, P, N) of dynamic shared memory.
 template <int R, int N>
-__global__ void __launch_bounds__(kT, (R <= 4 ? 4 : 3)) mimo_decode_kernel(MimoArgs a) {
+__global__ void __launch_bounds__(kT, (R <= 4 ? 5 : 3)) mimo_decode_kernel(MimoArgs a) {
     constexpr int LPR = N / 4;            // lanes per state row (a float4 each)
     constexpr int RPW = 32 / LPR;         // rows per warp per pass
     constexpr int ITER = kP / (8 * RPW);  // passes over the P rows with 8 warps
