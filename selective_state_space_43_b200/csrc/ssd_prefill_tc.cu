@@ -957,7 +957,8 @@ __global__ void __launch_bounds__(256, kVarlen ? 3 : 5) bc_prologue_kernel(Prefi
     const float4 w0 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cglob * 4);
     const float4 w1 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(cglob + 1) * 4);
     const float2 bias = make_float2(a.conv_b[cglob], a.conv_b[cglob + 1]);
-    uint32_t raw[kProTok + 3];  // rows t0-3 .. t0+kProTok-1, channels (2cp, 2cp+1)
+    float2 v[kProTok + 3];  // rows t0-3 .. t0+kProTok-1, channels (2cp, 2cp+1)
+    uint32_t raw[kProTok + 3];
 #pragma unroll
     for (int k = 0; k < kProTok + 3; ++k) {
         const int64_t t = t0 - 3 + k;
@@ -970,21 +971,20 @@ __global__ void __launch_bounds__(256, kVarlen ? 3 : 5) bc_prologue_kernel(Prefi
         start = a.cu[seq];
         next = a.cu[seq + 1];
     }
-    // row t0-3+k of the window as fp32 (history before token 0 of an unpacked batch)
-    auto row_val = [&](int k) -> float2 {
+#pragma unroll
+    for (int k = 0; k < kProTok + 3; ++k) {
         const int64_t t = t0 - 3 + k;
         if (!kVarlen && t < 0)
-            return make_float2(__bfloat162float(conv_history(a, b, cglob, t)),
+            v[k] = make_float2(__bfloat162float(conv_history(a, b, cglob, t)),
                                __bfloat162float(conv_history(a, b, cglob + 1, t)));
-        return make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
-    };
-    float2 win0 = row_val(0), win1 = row_val(1), win2 = row_val(2);  // the three rows before the current one
+        else
+            v[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
+    }
 #pragma unroll
     for (int k = 0; k < kProTok; ++k) {
         const int64_t t = t0 + k;
-        const float2 win3 = row_val(k + 3);
         if (t < a.L) {
-            float2 x4[4] = {win0, win1, win2, win3};
+            float2 x4[4] = {v[k], v[k + 1], v[k + 2], v[k + 3]};
             if constexpr (kVarlen) {
                 while (t >= next && seq + 1 < a.batch) {  // row t opens a later sequence
                     ++seq;
@@ -1009,9 +1009,6 @@ __global__ void __launch_bounds__(256, kVarlen ? 3 : 5) bc_prologue_kernel(Prefi
             const float2 u = silu2(p);
             dst[(size_t)t * 2 * half_gn] = pack_bf2(u.x, u.y);
         }
-        win0 = win1;
-        win1 = win2;
-        win2 = win3;
     }
 }
 
