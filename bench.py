@@ -163,8 +163,8 @@ def bench_backward(ops, d: Dims, act, dev, flush, K: int, warmup: int, world: in
     return {"value": tokens * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": KB,
             "workload": f"gradients of the {BACKWARD_WORKLOAD} layer prefill (bf16 inputs and dy, fp32 d_final; "
                         "every input, parameter and initial-state gradient, fp32)",
-            "launch": "eager (7 kernels: post-conv, dt, chunk states, state scans, chunk backward, "
-                      "conv backward, reductions)",
+            "launch": "eager (7 kernels: post-conv, dt, chunk states (tcgen05 for bf16, d_state 64/128), state "
+                      "scans, chunk backward, conv backward, reductions)",
             "algorithmic_bytes_per_step": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
             "dominant_kernel": {"kernel": "chunk_bwd_kernel", "ms": kms, "share": kms / ms,
                                 "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_ALU_TFLOPS,

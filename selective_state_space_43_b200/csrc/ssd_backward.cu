@@ -64,6 +64,13 @@ extern __shared__ __align__(16) unsigned char ssd_bwd_smem[];
 namespace ssd {
 namespace bwd {
 
+#ifndef SSD_EMU
+// The tensor-core per-chunk state sums (ssd_backward_tc.cu), used in place of chunk_state_kernel for bf16
+// activations with P = 64 and N in {64, 128}.
+bool chunk_state_tc_supported(int P, int N, bool act_bf16);
+cudaError_t launch_chunk_state_tc(const ChunkStateTcArgs& a, int64_t nchunks, cudaStream_t st);
+#endif
+
 constexpr int kQ = 64;    // backward chunk (tokens); also the conv backward's tile
 constexpr int kT = 256;   // threads per block
 constexpr int kP = 64;    // head dimension
@@ -943,7 +950,17 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         SSD_LAUNCH(dt_kernel, dim3(static_cast<unsigned>((nc * a.H + kT - 1) / kT), static_cast<unsigned>(a.batch)),
                    dim3(kT), 0, st, a, ws);
         const dim3 chunk_heads(static_cast<unsigned>(nc), static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+#ifndef SSD_EMU
+        if (chunk_state_tc_supported(a.P, N, a.act_bf16)) {
+            ChunkStateTcArgs t{a.batch, a.L, a.H, a.G, N, a.act_bf16, a.dy_bf16, ws.U, ws.DT, ws.CS, a.dy, a.z,
+                               ws.SP, ws.LM};
+            if ((err = launch_chunk_state_tc(t, nc, st)) != cudaSuccess) return err;
+        } else {
+            SSD_LAUNCH(chunk_state_kernel<N>, chunk_heads, dim3(kT), state_smem, st, a, ws);
+        }
+#else
         SSD_LAUNCH(chunk_state_kernel<N>, chunk_heads, dim3(kT), state_smem, st, a, ws);
+#endif
         SSD_LAUNCH(state_pass_kernel<N>, dim3(static_cast<unsigned>(a.H * kSplit), static_cast<unsigned>(a.batch)),
                    dim3(kT), kT * sizeof(float), st, a, ws);
         const dim3 chunk_groups(static_cast<unsigned>(nc), static_cast<unsigned>(a.G * head_split(a.H, a.G)),

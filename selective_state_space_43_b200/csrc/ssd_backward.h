@@ -32,6 +32,18 @@ struct BwdArgs {
     void* ev_after = nullptr;
 };
 
+// Inputs and outputs of the tensor-core version of the per-chunk state sums (ssd_backward_tc.cu): the
+// workspace's post-conv channels U [batch][L][conv_dim], dt and in-chunk cumsum DT, CS [batch][H][L], and
+// the chunk-local sums SP, LM [batch][nchunks][H][P][N] it writes.
+struct ChunkStateTcArgs {
+    int64_t batch, L;
+    int H, G, N;
+    bool act_bf16, dy_bf16;
+    const float *U, *DT, *CS;
+    const void *dy, *z;
+    float *SP, *LM;
+};
+
 // Bytes of workspace launch_prefill_backward needs (every region 256-byte aligned).
 size_t workspace_bytes(int64_t batch, int64_t L, int H, int P, int N, int G);
 

@@ -1,0 +1,194 @@
+// ssd_backward_tc.cu -- the per-chunk state sums of the prefill backward on the sm_100a tensor cores.
+//
+// For every 64-token chunk c and head h the backward needs two P x N sums over the chunk's tokens j
+// ("Nemotron-H 스타일 Hybrid Mamba-Transformer 3B 모델 구현 타당성 분석" §3.1/§3.2 train the layer, so its
+// backward is needed; the sums are the chunked form of the adjoint recurrence, as in ssd_backward.cu):
+//   SP_c = sum_j exp(cs_last - cs_j) dt_j x_j (outer) B_j      (the state a chunk adds, from zero)
+//   LM_c = sum_i exp(cs_i) g_i (outer) C_i,  g = dy * silu(z)   (the adjoint a chunk adds)
+// with x, B, C the post-conv channels.  Both are dense contractions over the chunk (K = 64 tokens), so
+// they run as tcgen05 MMAs, transposed so that the 128 state rows n are the MMA's M:
+//   SP_c^T = B^T X',  X'_j = exp(cs_last - cs_j) dt_j x_j        [N x P], K = the chunk's tokens
+//   LM_c^T = C^T G'', G''_i = exp(cs_i) g_i
+// (the same operand shapes as the forward's chunk-state MMA: A = B^T read MN-major from a [token][n]
+// tile, B = X' MN-major from a [token][p] tile; bf16 operands, fp32 accumulators in TMEM).  One
+// 128-thread CTA per (chunk, head, sequence): the threads convert their slices of the fp32 post-conv
+// channels, dy and z into the bf16 tiles (128-byte swizzle), one thread issues the two MMAs, and each
+// thread reads its TMEM lane n (state row n) back and writes SP[p][n] / LM[p][n] for p = 0..63.  For
+// d_state 64 the upper 64 rows of the B / C tiles are zero.  The wait for the MMAs is bounded; a wait that
+// gives up sets this file's error word (reported by ssd_device_status) and writes nothing.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ssd_backward.h"
+#include "ssd_sm100.cuh"
+
+namespace ssd {
+namespace bwd {
+
+__device__ int g_bwd_tc_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kQc = 64;       // the backward's chunk (tokens) = the MMAs' K
+constexpr int kPc = 64;       // head dimension
+constexpr int kNc = 128;      // state rows in the tiles (d_state 64 uses the first 64)
+constexpr int kThreadsC = 128;
+
+// shared memory (bytes from a 1024-byte aligned base); every tile is [64 tokens][64 columns] bf16 with
+// 128-byte rows and the 128-byte swizzle, 8 KB
+constexpr uint32_t OFF_BT = 0;        // B: two tiles, n 0..63 and 64..127
+constexpr uint32_t OFF_CT = 16384;    // C: two tiles
+constexpr uint32_t OFF_XW = 32768;    // X' [j][p]
+constexpr uint32_t OFF_GW = 40960;    // G'' [i][p]
+constexpr uint32_t OFF_BAR = 49152;   // mbarrier
+constexpr uint32_t OFF_TMH = OFF_BAR + 8;
+constexpr uint32_t SMEM_C = OFF_TMH + 8 + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS_C = 128;            // SP^T in columns 0..63, LM^T in 64..127
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float act_at(const void* p, int64_t i, bool bf16) {
+    if (bf16) return __uint_as_float(static_cast<uint32_t>(static_cast<const unsigned short*>(p)[i]) << 16);
+    return static_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ float silu_c(float v) { return v / (1.f + expf(-v)); }
+
+// grid (nchunks, H, batch), kThreadsC threads, SMEM_C bytes of dynamic shared memory
+__global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkStateTcArgs a) {
+    extern __shared__ uint8_t smem_c[];
+    uint8_t* sm = smem_c + ((1024u - (smem_u32(smem_c) & 1023u)) & 1023u);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint32_t* tm_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMH);
+    const int64_t c = blockIdx.x, b = blockIdx.z;
+    const int h = blockIdx.y, g = h / (a.H / a.G);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t t0 = c * kQc, nc = (a.L + kQc - 1) / kQc;
+    const int Qv = static_cast<int>(a.L - t0 < kQc ? a.L - t0 : kQc);
+    const int64_t HP = (int64_t)a.H * kPc, GN = (int64_t)a.G * a.N, conv_dim = HP + 2 * GN;
+
+    if (warp == 0) {
+        tmem_alloc(tm_holder, TMEM_COLS_C);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+
+    // B and C of the chunk (rows j >= Qv and channels n >= N zero): 64 rows x 16 chunks of 8 channels each
+    for (int e = tid; e < kQc * (kNc / 8); e += kThreadsC) {
+        const int r = e >> 4, k8 = e & 15, n0 = 8 * k8;
+        uint4 pb = make_uint4(0u, 0u, 0u, 0u), pc = pb;
+        if (r < Qv && n0 < a.N) {
+            const float* row = a.U + (b * a.L + t0 + r) * conv_dim + HP + (int64_t)g * a.N + n0;
+            const float4 b0 = *reinterpret_cast<const float4*>(row), b1 = *reinterpret_cast<const float4*>(row + 4);
+            const float4 c0 = *reinterpret_cast<const float4*>(row + GN);
+            const float4 c1 = *reinterpret_cast<const float4*>(row + GN + 4);
+            pb = make_uint4(pack_bf2(b0.x, b0.y), pack_bf2(b0.z, b0.w), pack_bf2(b1.x, b1.y), pack_bf2(b1.z, b1.w));
+            pc = make_uint4(pack_bf2(c0.x, c0.y), pack_bf2(c0.z, c0.w), pack_bf2(c1.x, c1.y), pack_bf2(c1.z, c1.w));
+        }
+        const uint32_t off = (uint32_t)(k8 >> 3) * 8192u + sw128_off(r, k8 & 7);
+        *reinterpret_cast<uint4*>(sm + OFF_BT + off) = pb;
+        *reinterpret_cast<uint4*>(sm + OFF_CT + off) = pc;
+    }
+    // X' and G'' (64 rows x 8 chunks of 8 head channels)
+    const float* dtp = a.DT + (b * a.H + h) * a.L + t0;
+    const float* csp = a.CS + (b * a.H + h) * a.L + t0;
+    const float cs_last = csp[Qv - 1];
+    for (int e = tid; e < kQc * (kPc / 8); e += kThreadsC) {
+        const int r = e >> 3, k8 = e & 7, p0 = 8 * k8;
+        uint4 px = make_uint4(0u, 0u, 0u, 0u), pg = px;
+        if (r < Qv) {
+            const float fx = dtp[r] * expf(cs_last - csp[r]), fg = expf(csp[r]);
+            const int64_t row = b * a.L + t0 + r;
+            const float* xr = a.U + row * conv_dim + (int64_t)h * kPc + p0;
+            const float4 x0 = *reinterpret_cast<const float4*>(xr), x1 = *reinterpret_cast<const float4*>(xr + 4);
+            px = make_uint4(pack_bf2(x0.x * fx, x0.y * fx), pack_bf2(x0.z * fx, x0.w * fx),
+                            pack_bf2(x1.x * fx, x1.y * fx), pack_bf2(x1.z * fx, x1.w * fx));
+            const int64_t yi = row * HP + (int64_t)h * kPc + p0;
+            float gv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) gv[k] = act_at(a.dy, yi + k, a.dy_bf16) * silu_c(act_at(a.z, yi + k, a.act_bf16)) * fg;
+            pg = make_uint4(pack_bf2(gv[0], gv[1]), pack_bf2(gv[2], gv[3]), pack_bf2(gv[4], gv[5]), pack_bf2(gv[6], gv[7]));
+        }
+        *reinterpret_cast<uint4*>(sm + OFF_XW + sw128_off(r, k8)) = px;
+        *reinterpret_cast<uint4*>(sm + OFF_GW + sw128_off(r, k8)) = pg;
+    }
+    fence_async_smem();  // the tiles are read by the tensor cores (async proxy)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tm_holder;
+
+    if (tid == 0) {
+        constexpr uint32_t ID = idesc_bf16_f32(128, 64, true, true);  // A MN-major (B^T / C^T), B MN-major (X' / G'')
+        const uint64_t dB = sw128_desc(smem_u32(sm + OFF_BT), 8192, 1024);
+        const uint64_t dC = sw128_desc(smem_u32(sm + OFF_CT), 8192, 1024);
+        const uint64_t dX = sw128_desc(smem_u32(sm + OFF_XW), 8192, 1024);
+        const uint64_t dG = sw128_desc(smem_u32(sm + OFF_GW), 8192, 1024);
+        // K = 64 tokens in four steps of 16 rows; an MN-major operand advances 16 rows x 128 bytes per step
+#pragma unroll
+        for (uint32_t kk = 0; kk < 4; ++kk) mma_bf16(tmem, dB + kk * (2048 >> 4), dX + kk * (2048 >> 4), ID, kk > 0);
+#pragma unroll
+        for (uint32_t kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + 64, dC + kk * (2048 >> 4), dG + kk * (2048 >> 4), ID, kk > 0);
+        mma_commit(bar);
+    }
+    const bool done = __all_sync(0xffffffffu, mbar_wait(bar, 0, nullptr));
+    tc_fence_after();
+    const int n = warp * 32 + lane;  // this thread's TMEM lane = state row n
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    if (done) {
+        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kPc * a.N;
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+            float* out = which ? a.LM : a.SP;
+#pragma unroll 1
+            for (int p0 = 0; p0 < kPc; p0 += 16) {
+                float v[16];
+                tmem_ld16(tmem + lane_base + which * 64 + p0, v);
+                tmem_wait_ld();
+                if (n < a.N) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) out[base + (int64_t)(p0 + k) * a.N + n] = v[k];
+                }
+            }
+        }
+    } else if (tid == 0) {
+        atomicOr(&g_bwd_tc_error, 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS_C);
+    }
+}
+
+}  // namespace
+
+bool chunk_state_tc_supported(int P, int N, bool act_bf16) { return act_bf16 && P == kPc && (N == 64 || N == kNc); }
+
+cudaError_t launch_chunk_state_tc(const ChunkStateTcArgs& a, int64_t nchunks, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_C);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>(nchunks), static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+    chunk_state_tc_kernel<<<grid, kThreadsC, SMEM_C, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_bwd_tc_error(int* flag) {
+    cudaError_t e = cudaMemcpyFromSymbol(flag, g_bwd_tc_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_bwd_tc_error, &zero, sizeof(int));
+}
+
+}  // namespace bwd
+}  // namespace ssd

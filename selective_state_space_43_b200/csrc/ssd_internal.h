@@ -97,6 +97,9 @@ namespace bwd {
 struct BwdArgs;
 // The prefill backward (ssd_backward.cu); sizes and pointers validated by the caller.
 cudaError_t launch_prefill_backward(const BwdArgs& a, cudaStream_t st);
+// Reads and clears the error word of the backward's tensor-core kernel (ssd_backward_tc.cu; nonzero: a
+// bounded wait gave up).  Does not synchronise: call after the stream is idle.
+cudaError_t read_and_clear_bwd_tc_error(int* flag);
 }  // namespace bwd
 
 }  // namespace ssd
