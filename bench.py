@@ -121,7 +121,23 @@ def backward_chunk_flops(d: Dims) -> int:
     return d.batch * nc * (d.nheads * per_head + d.ngroups * per_group)
 
 
-def bench_backward(ops, d: Dims, act, dev, flush, K: int, warmup: int, world: int, sampler):
+def backward_chunk_bytes(d: Dims, act_bytes: int) -> int:
+    """Algorithmic bytes of one launch of the tensor-core per-chunk backward (chunk_bwd_tc_kernel), Q = 64:
+    reads the fp32 post-conv x, B, C, dt and in-chunk cumsum (workspace), dy and z and the raw dt (activation
+    dtype), the entering states and leaving adjoints (fp32 [nc][H][P][N] each) and the per-chunk F partials;
+    writes dz, the post-conv gradients of x (fp32), of B and C (fp32, one copy per half of each group's heads),
+    ddt and the per-chunk partials.  Each byte counted once."""
+    Q, P, N = BWD_Q, d.headdim, d.d_state
+    rows, nc = d.batch * d.seqlen, d.batch * -(-d.seqlen // Q)
+    HP, GN = d.nheads * P, d.ngroups * N
+    halves = 2 if d.nheads // d.ngroups >= 2 else 1
+    reads = rows * (HP + 2 * GN) * 4 + rows * 2 * d.nheads * 4 + rows * (2 * HP + d.nheads) * act_bytes + \
+        2 * nc * d.nheads * P * N * 4 + nc * d.nheads * 4 * 4
+    writes = rows * 2 * HP * 4 + halves * rows * 2 * GN * 4 + rows * d.nheads * 4 + nc * d.nheads * 3 * 4
+    return reads + writes
+
+
+def bench_backward(ops, d: Dims, act, dev, flush, K: int, warmup: int, world: int, sampler, peaks):
     """Times ssd_prefill_backward on the prefill workload (bf16 activations and dy, d_final given)."""
     inp = make_prefill_inputs(d, dtype=act, seed=seed_of(BACKWARD_WORKLOAD) + 7)
     gr = make_backward_grads(d, dtype=act, seed=seed_of(BACKWARD_WORKLOAD) + 8)
@@ -157,21 +173,22 @@ def bench_backward(ops, d: Dims, act, dev, flush, K: int, warmup: int, world: in
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(st, en)) / KB, world, dev)
     kms = sum(a.elapsed_time(b) for a, b in zip(ks, ke)) / KB
     tokens = d.batch * d.seqlen
-    flops = backward_chunk_flops(d)
-    tf = flops / (kms * 1e-3) / 1e12
-    nbytes = backward_bytes(d, 2 if act == torch.bfloat16 else 4)
+    abytes = 2 if act == torch.bfloat16 else 4
+    nbytes = backward_bytes(d, abytes)
+    kbytes = backward_chunk_bytes(d, abytes)
+    kgbs = kbytes / (kms * 1e-3) / 1e9
     return {"value": tokens * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": KB,
             "workload": f"gradients of the {BACKWARD_WORKLOAD} layer prefill (bf16 inputs and dy, fp32 d_final; "
                         "every input, parameter and initial-state gradient, fp32)",
-            "launch": "eager (7 kernels: post-conv, dt, chunk states (tcgen05 for bf16, d_state 64/128), state "
-                      "scans, chunk backward, conv backward, reductions)",
+            "launch": "eager (7 kernels: post-conv, dt, chunk states (tcgen05), state scans, chunk backward "
+                      "(tcgen05), conv backward, reductions; the tcgen05 kernels for bf16, d_state 64/128)",
             "algorithmic_bytes_per_step": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
-            "dominant_kernel": {"kernel": "chunk_bwd_kernel", "ms": kms, "share": kms / ms,
-                                "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_ALU_TFLOPS,
-                                             "unit": "TFLOP/s", "frac": tf / FP32_ALU_TFLOPS,
-                                             "traffic": kernel_traffic("chunk_bwd_kernel"),
-                                             "algorithmic_flops_per_launch": flops,
-                                             "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1965 MHz"}},
+            "dominant_kernel": {"kernel": "chunk_bwd_tc_kernel", "ms": kms, "share": kms / ms,
+                                "algorithmic_flops_per_launch": backward_chunk_flops(d),
+                                "roofline": {"bound": "hbm", "achieved": kgbs, "peak": peaks["hbm_gbs"],
+                                             "unit": "GB/s", "frac": kgbs / peaks["hbm_gbs"],
+                                             "traffic": kernel_traffic(f"chunk_bwd_tc_kernel@{BACKWARD_WORKLOAD}"),
+                                             "algorithmic_bytes_per_launch": kbytes}},
             "l2": "flushed between timed steps (256 MB write outside the step events)"}
 
 
@@ -886,7 +903,7 @@ def main():
     if not args.no_backward:
         try:
             wb = WORKLOADS[BACKWARD_WORKLOAD]
-            backward = bench_backward(ops, wb["dims"], wb["dtype"], dev, flush, K, args.warmup, world, sampler)
+            backward = bench_backward(ops, wb["dims"], wb["dtype"], dev, flush, K, args.warmup, world, sampler, peaks)
         except (RuntimeError, ValueError) as exc:  # report it and keep the forward numbers
             backward = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         torch.cuda.empty_cache()

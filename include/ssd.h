@@ -60,7 +60,8 @@ typedef enum {
     SSD_ERR_UNSUPPORTED = 5, /* valid but not implemented (e.g. aliasing outputs)      */
     SSD_ERR_CUDA = 6,        /* a CUDA runtime call failed (launch or query)            */
     SSD_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than ssd_prefill_workspace_bytes */
-    SSD_ERR_TIMEOUT = 8      /* a bounded device-side wait gave up                      */
+    SSD_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up                      */
+    SSD_ERR_RANGE = 9        /* a backward operand beyond the tensor-core path's fp16 range */
 } ssd_status;
 
 /* Activation dtype.  SSD_BF16_YF32 reads bf16 activations (and keeps the conv
@@ -348,8 +349,10 @@ SSD_API ssd_status ssd_prefill_backward(const ssd_dims* dims, ssd_dtype dtype, c
 /*
  * Synchronises `stream` and reports whether a kernel launched by this library
  * gave up on a bounded device-side wait since the last call (SSD_ERR_TIMEOUT;
- * its outputs are then incomplete), or whether the stream holds a CUDA error
- * (SSD_ERR_CUDA).  Clears the flag.  Every wait inside the kernels is bounded
+ * its outputs are then incomplete), whether a tensor-core backward kernel met
+ * an operand that fp16 cannot hold even after its power-of-two state scaling
+ * (SSD_ERR_RANGE; |value| >= 65504, the gradients of that call are invalid),
+ * or whether the stream holds a CUDA error (SSD_ERR_CUDA).  Clears the flags.  Every wait inside the kernels is bounded
  * (about 2 s), so a kernel can never hang the device.
  */
 SSD_API ssd_status ssd_device_status(void* stream);

@@ -69,6 +69,10 @@ namespace bwd {
 // activations with P = 64 and N in {64, 128}.
 bool chunk_state_tc_supported(int P, int N, bool act_bf16);
 cudaError_t launch_chunk_state_tc(const ChunkStateTcArgs& a, int64_t nchunks, cudaStream_t st);
+// The tensor-core per-chunk backward (ssd_chunk_bwd_tc.cu), used in place of chunk_bwd_kernel under the
+// same conditions (and 16-byte aligned dy, z, dz).
+bool chunk_bwd_tc_supported(int P, int N, bool act_bf16, const void* dy, const void* z, const void* dz);
+cudaError_t launch_chunk_bwd_tc(const ChunkBwdTcArgs& a, int64_t nchunks, cudaStream_t st);
 #endif
 
 constexpr int kQ = 64;    // backward chunk (tokens); also the conv backward's tile
@@ -968,7 +972,18 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
 #ifndef SSD_EMU
         if (a.ev_before) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_before), st);
 #endif
+#ifndef SSD_EMU
+        if (chunk_bwd_tc_supported(a.P, N, a.act_bf16, a.dy, a.z, a.dz)) {
+            ChunkBwdTcArgs t{a.batch, a.L,  a.H,   a.G,  N,     head_split(a.H, a.G), kSplit, a.act_bf16, a.dy_bf16,
+                             a.A,     a.D,  a.dt_bias, a.dt, a.z, a.dy,  ws.U,  ws.DT, ws.CS, ws.SP, ws.LM, ws.PF,
+                             a.dz,    a.ddt, ws.DU, ws.DU2, ws.PH};
+            if ((err = launch_chunk_bwd_tc(t, nc, st)) != cudaSuccess) return err;
+        } else {
+            SSD_LAUNCH(chunk_bwd_kernel<N>, chunk_groups, dim3(kT), chunk_smem, st, a, ws);
+        }
+#else
         SSD_LAUNCH(chunk_bwd_kernel<N>, chunk_groups, dim3(kT), chunk_smem, st, a, ws);
+#endif
 #ifndef SSD_EMU
         if (a.ev_after) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_after), st);
 #endif

@@ -44,6 +44,19 @@ struct ChunkStateTcArgs {
     float *SP, *LM;
 };
 
+// Inputs and outputs of the tensor-core per-chunk backward (ssd_backward_tc.cu), which writes exactly what
+// the CUDA-core chunk kernel writes: dz, ddt, the post-conv gradients of x (DU) and of B, C (DU for the
+// first half of each group's heads, DU2 for the second), and the per-chunk partials PH.
+struct ChunkBwdTcArgs {
+    int64_t batch, L;
+    int H, G, N, split, nsplit_pf;  // heads-per-group halves (1 or 2); partial sums per chunk in PF
+    bool act_bf16, dy_bf16;
+    const float *A, *D, *dt_bias;
+    const void *dt, *z, *dy;
+    const float *U, *DT, *CS, *SP, *LM, *PF;
+    float *dz, *ddt, *DU, *DU2, *PH;
+};
+
 // Bytes of workspace launch_prefill_backward needs (every region 256-byte aligned).
 size_t workspace_bytes(int64_t batch, int64_t L, int H, int P, int N, int G);
 

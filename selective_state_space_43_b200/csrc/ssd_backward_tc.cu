@@ -10,14 +10,18 @@
 //   SP_c^T = B^T X',  X'_j = exp(cs_last - cs_j) dt_j x_j        [N x P], K = the chunk's tokens
 //   LM_c^T = C^T G'', G''_i = exp(cs_i) g_i
 // (the same operand shapes as the forward's chunk-state MMA: A = B^T read MN-major from a [token][n]
-// tile, B = X' MN-major from a [token][p] tile; bf16 operands, fp32 accumulators in TMEM).  One
+// tile, B = X' MN-major from a [token][p] tile; fp16 operands, whose 11-bit significand keeps the
+// gradients that flow through these sums (the initial-state gradient, dA, ddt_bias) well inside the
+// layer's tolerance where bf16's 8 bits do not; fp32 accumulators in TMEM).  The operands are activations
+// (post-conv B, C, x and g scaled by decays <= 1 and dt): a magnitude fp16 cannot hold (>= 65504) sets
+// bit 1 of the error word, which ssd_device_status reports as SSD_ERR_RANGE.  One
 // 128-thread CTA per (chunk, head, sequence): the threads convert their slices of the fp32 post-conv
-// channels, dy and z into the bf16 tiles (128-byte swizzle), one thread issues the two MMAs, and each
+// channels, dy and z into the fp16 tiles (128-byte swizzle), one thread issues the two MMAs, and each
 // thread reads its TMEM lane n (state row n) back and writes SP[p][n] / LM[p][n] for p = 0..63.  For
 // d_state 64 the upper 64 rows of the B / C tiles are zero.  The wait for the MMAs is bounded; a wait that
 // gives up sets this file's error word (reported by ssd_device_status) and writes nothing.
 #include <cuda.h>
-#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "ssd_backward.h"
@@ -37,7 +41,7 @@ constexpr int kPc = 64;       // head dimension
 constexpr int kNc = 128;      // state rows in the tiles (d_state 64 uses the first 64)
 constexpr int kThreadsC = 128;
 
-// shared memory (bytes from a 1024-byte aligned base); every tile is [64 tokens][64 columns] bf16 with
+// shared memory (bytes from a 1024-byte aligned base); every tile is [64 tokens][64 columns] fp16 with
 // 128-byte rows and the 128-byte swizzle, 8 KB
 constexpr uint32_t OFF_BT = 0;        // B: two tiles, n 0..63 and 64..127
 constexpr uint32_t OFF_CT = 16384;    // C: two tiles
@@ -48,8 +52,9 @@ constexpr uint32_t OFF_TMH = OFF_BAR + 8;
 constexpr uint32_t SMEM_C = OFF_TMH + 8 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS_C = 128;            // SP^T in columns 0..63, LM^T in 64..127
 
-__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi, float& range) {
+    range = fmaxf(range, fmaxf(fabsf(lo), fabsf(hi)));
+    __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 __device__ __forceinline__ float act_at(const void* p, int64_t i, bool bf16) {
@@ -80,6 +85,7 @@ __global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkSt
         fence_mbar_init();
     }
 
+    float range = 0.f;  // largest magnitude this thread writes to an fp16 tile
     // B and C of the chunk (rows j >= Qv and channels n >= N zero): 64 rows x 16 chunks of 8 channels each
     for (int e = tid; e < kQc * (kNc / 8); e += kThreadsC) {
         const int r = e >> 4, k8 = e & 15, n0 = 8 * k8;
@@ -89,8 +95,10 @@ __global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkSt
             const float4 b0 = *reinterpret_cast<const float4*>(row), b1 = *reinterpret_cast<const float4*>(row + 4);
             const float4 c0 = *reinterpret_cast<const float4*>(row + GN);
             const float4 c1 = *reinterpret_cast<const float4*>(row + GN + 4);
-            pb = make_uint4(pack_bf2(b0.x, b0.y), pack_bf2(b0.z, b0.w), pack_bf2(b1.x, b1.y), pack_bf2(b1.z, b1.w));
-            pc = make_uint4(pack_bf2(c0.x, c0.y), pack_bf2(c0.z, c0.w), pack_bf2(c1.x, c1.y), pack_bf2(c1.z, c1.w));
+            pb = make_uint4(pack_h2(b0.x, b0.y, range), pack_h2(b0.z, b0.w, range), pack_h2(b1.x, b1.y, range),
+                            pack_h2(b1.z, b1.w, range));
+            pc = make_uint4(pack_h2(c0.x, c0.y, range), pack_h2(c0.z, c0.w, range), pack_h2(c1.x, c1.y, range),
+                            pack_h2(c1.z, c1.w, range));
         }
         const uint32_t off = (uint32_t)(k8 >> 3) * 8192u + sw128_off(r, k8 & 7);
         *reinterpret_cast<uint4*>(sm + OFF_BT + off) = pb;
@@ -108,17 +116,19 @@ __global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkSt
             const int64_t row = b * a.L + t0 + r;
             const float* xr = a.U + row * conv_dim + (int64_t)h * kPc + p0;
             const float4 x0 = *reinterpret_cast<const float4*>(xr), x1 = *reinterpret_cast<const float4*>(xr + 4);
-            px = make_uint4(pack_bf2(x0.x * fx, x0.y * fx), pack_bf2(x0.z * fx, x0.w * fx),
-                            pack_bf2(x1.x * fx, x1.y * fx), pack_bf2(x1.z * fx, x1.w * fx));
+            px = make_uint4(pack_h2(x0.x * fx, x0.y * fx, range), pack_h2(x0.z * fx, x0.w * fx, range),
+                            pack_h2(x1.x * fx, x1.y * fx, range), pack_h2(x1.z * fx, x1.w * fx, range));
             const int64_t yi = row * HP + (int64_t)h * kPc + p0;
             float gv[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) gv[k] = act_at(a.dy, yi + k, a.dy_bf16) * silu_c(act_at(a.z, yi + k, a.act_bf16)) * fg;
-            pg = make_uint4(pack_bf2(gv[0], gv[1]), pack_bf2(gv[2], gv[3]), pack_bf2(gv[4], gv[5]), pack_bf2(gv[6], gv[7]));
+            pg = make_uint4(pack_h2(gv[0], gv[1], range), pack_h2(gv[2], gv[3], range), pack_h2(gv[4], gv[5], range),
+                            pack_h2(gv[6], gv[7], range));
         }
         *reinterpret_cast<uint4*>(sm + OFF_XW + sw128_off(r, k8)) = px;
         *reinterpret_cast<uint4*>(sm + OFF_GW + sw128_off(r, k8)) = pg;
     }
+    if (!(range < 65504.f)) atomicOr(&g_bwd_tc_error, 2);
     fence_async_smem();  // the tiles are read by the tensor cores (async proxy)
     tc_fence_before();
     __syncthreads();
@@ -126,7 +136,8 @@ __global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkSt
     const uint32_t tmem = *tm_holder;
 
     if (tid == 0) {
-        constexpr uint32_t ID = idesc_bf16_f32(128, 64, true, true);  // A MN-major (B^T / C^T), B MN-major (X' / G'')
+        // fp16 A and B (format 0), fp32 D; A MN-major (B^T / C^T), B MN-major (X' / G'')
+        constexpr uint32_t ID = (1u << 4) | (1u << 15) | (1u << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
         const uint64_t dB = sw128_desc(smem_u32(sm + OFF_BT), 8192, 1024);
         const uint64_t dC = sw128_desc(smem_u32(sm + OFF_CT), 8192, 1024);
         const uint64_t dX = sw128_desc(smem_u32(sm + OFF_XW), 8192, 1024);
@@ -160,7 +171,7 @@ __global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkSt
             }
         }
     } else if (tid == 0) {
-        atomicOr(&g_bwd_tc_error, 1);
+        atomicOr(&g_bwd_tc_error, 1);  // bit 0: the wait gave up
     }
     tc_fence_before();
     __syncthreads();

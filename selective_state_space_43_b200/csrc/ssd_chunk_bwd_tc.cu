@@ -1,0 +1,719 @@
+// ssd_chunk_bwd_tc.cu -- the per-chunk backward of the prefill on the sm_100a tensor cores.
+//
+// The layer is trained ("Nemotron-H 스타일 Hybrid Mamba-Transformer 3B 모델 구현 타당성 분석" §3.1/§3.2), so the
+// SSD prefill needs its backward.  Inside one 64-token chunk, with cs the in-chunk cumulative sum of dt*A,
+// L_ij = exp(cs_i - cs_j) (i >= j), g = dy * silu(z), Sp the state entering the chunk and Lm the adjoint
+// of the state leaving it, every gradient of the chunk is built from ten dense products over the chunk
+// (K = 64 tokens or 64 head channels) or over the state (K = N):
+//   CB  = C B^T                  GX  = g x^T                 (token x token)
+//   SPC = C Sp^T   LMB = B Lm^T  YIN = LCB x   DXI = LCB^T g  (token x head channel)
+//   dB^T += Lm^T X'^T + C^T LGX'   dC^T += Sp^T G''^T + B^T LGX'^T   (state x token, summed over heads)
+// with LCB_ij = CB_ij L_ij dt_j and LGX'_ij = GX_ij L_ij dt_j (zero above the diagonal), X'_j =
+// exp(cs_last - cs_j) dt_j x_j and G''_i = exp(cs_i) g_i.  From them, elementwise:
+//   y_i  = YIN_i + exp(cs_i) SPC_i + D x_i,  dz_i = dy_i silu'(z_i) y_i
+//   dx_j = DXI_j + dt_j exp(cs_last - cs_j) LMB_j + D g_j
+//   E_i  = exp(cs_i) g_i . SPC_i,  W_j = exp(cs_last - cs_j) x_j . LMB_j
+//   M_ij = LGX'_ij CB_ij,  Dr_j = sum_i GX_ij L_ij CB_ij (the column sums of M / dt_j)
+//   d(dA_k) = R_k + sum_{i>=k} E_i + F + sum_{j<k} dt_j W_j,
+//     R_k = sum_{i>=k} sum_{j<k} M_ij = sum_{m<k} (colsum_m(M) - rowsum_m(M))  (M is lower triangular)
+//   ddt_k = Dr_k + W_k + A d(dA_k), then through softplus
+// (the same quantities, in the same fp32 epilogue arithmetic, as the CUDA-core chunk kernel of
+// ssd_backward.cu; there R comes from explicit prefix sums of M).
+//
+// One CTA per (chunk, group, half of the group's heads), heads in turn; 256 threads in two roles:
+//   row warps 0, 1, 4, 5  (TMEM lanes 0..63 = the chunk's tokens; warps 0/4 tokens 0..31, 1/5 tokens
+//                         32..63; warps 0, 1 columns 0..31, warps 4, 5 columns 32..63): the elementwise
+//                         work above, the LCB / LGX' tiles, dz, dx and the per-head scalars; lane 0 of
+//                         warp 0 also allocates TMEM (the whole warp) and issues the MMAs, at the points
+//                         where warp 0 waits for their operands anyway;
+//   loader warps 2, 3, 6, 7: the head's operand tiles (x, X', g, G'', Sp, Lm) as bf16 in 128-byte-swizzled
+//                         shared memory, two heads deep.
+// Every MMA is M = 128, N = 64 with bf16 operands and fp32 accumulators in TMEM (512 columns: CB, GX,
+// SPC, LMB, YIN, DXI, dB^T, dC^T).  The token-major products use only rows 0..63 of their 128-row
+// result: the A tile's rows 64..127 are whatever follows it in shared memory (always in bounds), and the
+// result lanes 64..127 are never read.  dB^T and dC^T have the state index n as M (rows past N unused).
+// All waits are bounded mbarrier waits that also watch a shared abort word; a wait that gives up sets
+// this file's error word (reported by ssd_device_status), and the CTA leaves without
+// writing its dB / dC.  No atomics: every sum runs in a fixed order (deterministic).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "ssd_backward.h"
+#include "ssd_sm100.cuh"
+
+namespace ssd {
+namespace bwd {
+
+__device__ int g_chunk_bwd_tc_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kQb = 64;   // chunk (tokens)
+constexpr int kPb = 64;   // head dimension
+constexpr int kThreadsB = 256;
+
+// shared memory (bytes from a 1024-byte aligned base).  A "box" is [64 rows][64 bf16] with 128-byte rows
+// and the 128-byte swizzle (8 KB); an N-wide tile is one box per 64 state columns.
+constexpr uint32_t OFF_TC = 0;          // C [i][n], two boxes
+constexpr uint32_t OFF_TB = 16384;      // B [j][n], two boxes
+constexpr uint32_t OFF_LCB = 32768;     // LCB [i][j]
+constexpr uint32_t OFF_LGX = 40960;     // LGX' [i][j]
+constexpr uint32_t OFF_BUF = 49152;     // two per-head buffers of BUF_BYTES:
+constexpr uint32_t B_SP = 0;            //   Sp [p][n], two boxes
+constexpr uint32_t B_LM = 16384;        //   Lm [p][n], two boxes
+constexpr uint32_t B_X = 32768;         //   x [j][p]
+constexpr uint32_t B_XP = 40960;        //   X' [j][p]
+constexpr uint32_t B_G = 49152;         //   g [i][p]
+constexpr uint32_t B_GP = 57344;        //   G'' [i][p]
+constexpr uint32_t BUF_BYTES = 65536;
+constexpr uint32_t OFF_VEC = OFF_BUF + 2 * BUF_BYTES;  // fp32 vectors:
+constexpr uint32_t V_DT = 0;            //   dt [2 buffers][64]
+constexpr uint32_t V_CS = 512;          //   cs [2][64]
+constexpr uint32_t V_COL = 1024;        //   column sums of GX L CB [2 head parities][2 token halves][64]
+constexpr uint32_t V_ROWM = 2048;       //   row sums of M [2][2 column halves][64]
+constexpr uint32_t V_E = 3072;          //   g_i . SPC_i partials [2][2][64]
+constexpr uint32_t V_W = 4096;          //   W_j partials [2][2][64]
+constexpr uint32_t V_PD = 5120;         //   sum g . x per row warp [2][4]
+constexpr uint32_t V_MAX = 5152;        //   largest |Sp|, |Lm| per loader warp [2 head parities][4][2]
+constexpr uint32_t V_SC = 5216;         //   the Sp, Lm scales of each buffer [2][2]
+constexpr uint32_t VEC_BYTES = 5248;
+constexpr uint32_t OFF_BAR = OFF_VEC + VEC_BYTES;
+enum : int { TILE_FULL0, TILE_FULL1, TILE_FREE0, TILE_FREE1, B1_DONE, LT_FULL, B2_DONE, ACC_FREE, WSYNC, FINAL,
+             LMAX, NBAR };
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // abort word, TMEM base
+constexpr uint32_t SMEM_B = OFF_MISC + 16 + 1024;  // + alignment slack
+
+// TMEM columns (lane = token or state row)
+constexpr uint32_t COL_CB = 0, COL_GX = 64, COL_SPC = 128, COL_LMB = 192, COL_YIN = 256, COL_DXI = 320,
+                   COL_DB = 384, COL_DC = 448, TMEM_COLS_B = 512;
+
+// The MMA operands are fp16 (11-bit significand): bf16's 8 bits lose too much in the sums behind ddt.
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+// Instruction descriptor for kind::f16 with fp16 A/B (format 0) and an fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float sigm(float v) { return 1.f / (1.f + expf(-v)); }
+
+// Eight consecutive activations from element i (a multiple of 8) of a bf16 or fp32 array (16-byte aligned).
+__device__ __forceinline__ void load8(const void* p, int64_t i, bool bf16, float (&v)[8]) {
+    if (bf16) {
+        const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(p) + i);
+        v[0] = bf_lo(w.x), v[1] = bf_hi(w.x), v[2] = bf_lo(w.y), v[3] = bf_hi(w.y);
+        v[4] = bf_lo(w.z), v[5] = bf_hi(w.z), v[6] = bf_lo(w.w), v[7] = bf_hi(w.w);
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+        const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i + 4);
+        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+    }
+}
+// Eight values times s as fp16; `range` keeps the largest magnitude packed (>= 65504 does not fit).
+__device__ __forceinline__ uint4 pack8(const float (&v)[8], float s, float& range) {
+    float w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        w[q] = v[q] * s;
+        range = fmaxf(range, fabsf(w[q]));
+    }
+    return make_uint4(pack_h2(w[0], w[1]), pack_h2(w[2], w[3]), pack_h2(w[4], w[5]), pack_h2(w[6], w[7]));
+}
+// The power of two s <= 1 that brings a tile whose largest magnitude is m below 2^14 (1 when it already is).
+__device__ __forceinline__ float state_scale(float m) {
+    if (m < 16384.f) return 1.f;
+    const int e = min(((__float_as_int(m) >> 23) & 0xff) - 127, 128);  // m in [2^e, 2^(e+1))
+    return __int_as_float((127 + 13 - e) << 23);                        // m * s in [2^13, 2^14)
+}
+
+// D (+)= A B over K = 16 * steps; a K-major operand steps 32 bytes inside a box and 8 KB from box to box,
+// an MN-major one 16 rows (2 KB) per step.  The first step overwrites D unless acc.
+__device__ __forceinline__ void mma_steps(uint32_t d, uint64_t a0, bool a_mn, uint64_t b0, bool b_mn, uint32_t idesc,
+                                          int steps, bool acc) {
+    for (int kk = 0; kk < steps; ++kk) {
+        const uint32_t kmaj = ((uint32_t)(kk >> 2) * 8192u + (uint32_t)(kk & 3) * 32u) >> 4;
+        const uint32_t mnmaj = ((uint32_t)kk * 2048u) >> 4;
+        mma_bf16(d, a0 + (a_mn ? mnmaj : kmaj), b0 + (b_mn ? mnmaj : kmaj), idesc, (acc || kk > 0) ? 1u : 0u);
+    }
+}
+
+constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, false, false);
+constexpr uint32_t ID_KM = idesc_f16_f32(128, 64, false, true);
+constexpr uint32_t ID_MK = idesc_f16_f32(128, 64, true, false);
+constexpr uint32_t ID_MM = idesc_f16_f32(128, 64, true, true);
+__device__ __forceinline__ uint64_t kdesc(const uint8_t* p) { return sw128_desc(smem_u32(p), 16, 1024); }
+__device__ __forceinline__ uint64_t mdesc(const uint8_t* p) { return sw128_desc(smem_u32(p), 8192, 1024); }
+
+// The first MMAs of head k (operands: the head's buffer and C, B): GX, SPC, LMB and the Sp / Lm parts of
+// dB^T, dC^T (which the first head starts).
+__device__ __forceinline__ void issue_batch1(const uint8_t* sm, uint32_t tmem, int k, int nbox, uint64_t* done) {
+    const uint8_t* bo = sm + OFF_BUF + (k & 1) * BUF_BYTES;
+    mma_steps(tmem + COL_GX, kdesc(bo + B_G), false, kdesc(bo + B_X), false, ID_KK, 4, false);
+    mma_steps(tmem + COL_SPC, kdesc(sm + OFF_TC), false, kdesc(bo + B_SP), false, ID_KK, 4 * nbox, false);
+    mma_steps(tmem + COL_LMB, kdesc(sm + OFF_TB), false, kdesc(bo + B_LM), false, ID_KK, 4 * nbox, false);
+    mma_steps(tmem + COL_DB, mdesc(bo + B_LM), true, kdesc(bo + B_XP), false, ID_MK, 4, k > 0);
+    mma_steps(tmem + COL_DC, mdesc(bo + B_SP), true, kdesc(bo + B_GP), false, ID_MK, 4, k > 0);
+    mma_commit(done);
+}
+// The MMAs that need the row warps' LCB / LGX' tiles: YIN, DXI and the intra-chunk parts of dB^T, dC^T.
+__device__ __forceinline__ void issue_batch2(const uint8_t* sm, uint32_t tmem, int k, uint64_t* done,
+                                             uint64_t* free_buf) {
+    const uint8_t* bo = sm + OFF_BUF + (k & 1) * BUF_BYTES;
+    mma_steps(tmem + COL_YIN, kdesc(sm + OFF_LCB), false, mdesc(bo + B_X), true, ID_KM, 4, false);
+    mma_steps(tmem + COL_DXI, mdesc(sm + OFF_LCB), true, mdesc(bo + B_G), true, ID_MM, 4, false);
+    mma_steps(tmem + COL_DB, mdesc(sm + OFF_TC), true, mdesc(sm + OFF_LGX), true, ID_MM, 4, true);
+    mma_steps(tmem + COL_DC, mdesc(sm + OFF_TB), true, kdesc(sm + OFF_LGX), false, ID_MK, 4, true);
+    mma_commit(done);
+    mma_commit(free_buf);
+}
+
+// A warp-uniform bounded wait: true when the phase of `parity` completed for every lane.
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+__device__ __forceinline__ void give_up(volatile int* abort) {
+    *abort = 1;
+    atomicOr(&g_chunk_bwd_tc_error, 1);
+}
+
+// Sum over the warp's 32 lanes of each of v[0..31]: lane l ends with the sum of v[l] (butterfly; at each
+// step a lane keeps the half of its values whose index bit matches its lane bit and adds the partner's).
+__device__ __forceinline__ float column_sums(float (&v)[32], int lane) {
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const bool up = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+            const float send = up ? v[i] : v[i + s];
+            const float keep = up ? v[i + s] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+        }
+    }
+    return v[0];
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+    return v;
+}
+
+// grid (nchunks, G * split, batch), kThreadsB threads, SMEM_B bytes of dynamic shared memory
+__global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkBwdTcArgs a) {
+    extern __shared__ uint8_t smem_b[];
+    uint8_t* sm = smem_b + ((1024u - (smem_u32(smem_b) & 1023u)) & 1023u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_MISC);
+    uint32_t* tm_holder = reinterpret_cast<uint32_t*>(sm + OFF_MISC + 8);
+    float* vec = reinterpret_cast<float*>(sm + OFF_VEC);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t c = blockIdx.x, b = blockIdx.z, t0 = c * kQb, nc = (a.L + kQb - 1) / kQb;
+    const int hpg = a.H / a.G, g = blockIdx.y / a.split, half = blockIdx.y % a.split;
+    const int hl0 = half * hpg / a.split, nh = (half + 1) * hpg / a.split - hl0;
+    const int Qv = static_cast<int>(a.L - t0 < kQb ? a.L - t0 : kQb);
+    const int N = a.N, nbox = N / 64;
+    const int64_t HP = (int64_t)a.H * kPb, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
+    const int64_t row0 = b * a.L + t0;  // first token row of the chunk
+
+    if (warp == 0) {
+        tmem_alloc(tm_holder, TMEM_COLS_B);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        *abort = 0;
+        mbar_init(&bars[TILE_FULL0], 128);
+        mbar_init(&bars[TILE_FULL1], 128);
+        mbar_init(&bars[TILE_FREE0], 129);  // the MMAs' commit + the 128 row threads
+        mbar_init(&bars[TILE_FREE1], 129);
+        mbar_init(&bars[B1_DONE], 1);
+        mbar_init(&bars[LT_FULL], 128);
+        mbar_init(&bars[B2_DONE], 1);
+        mbar_init(&bars[ACC_FREE], 128);
+        mbar_init(&bars[WSYNC], 128);
+        mbar_init(&bars[FINAL], 1);
+        mbar_init(&bars[LMAX], 128);
+        fence_mbar_init();
+    }
+    // the group's post-conv B and C (rows past Qv zero): 64 rows x N/8 chunks of 8 channels
+    for (int e = tid; e < kQb * (N / 8); e += kThreadsB) {
+        const int r = e / (N / 8), k8 = e % (N / 8);
+        uint4 pb = make_uint4(0u, 0u, 0u, 0u), pc = pb;
+        if (r < Qv) {
+            const float* src = a.U + (row0 + r) * conv_dim + HP + (int64_t)g * N + 8 * k8;
+            float v[8], range = 0.f;
+            load8(src, 0, false, v);
+            pb = pack8(v, 1.f, range);
+            load8(src + GN, 0, false, v);
+            pc = pack8(v, 1.f, range);
+            if (!(range < 65504.f)) atomicOr(&g_chunk_bwd_tc_error, 2);
+        }
+        const uint32_t off = (uint32_t)(k8 >> 3) * 8192u + sw128_off(r, k8 & 7);
+        *reinterpret_cast<uint4*>(sm + OFF_TB + off) = pb;
+        *reinterpret_cast<uint4*>(sm + OFF_TC + off) = pc;
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tm_holder;
+
+    if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
+        // ---------------- loaders ----------------
+        const int lt = ((warp & 3) - 2 + 2 * (warp >> 2)) * 32 + lane;  // 0..127
+        for (int k = 0; k < nh; ++k) {
+            const int buf = k & 1;
+            if (k >= 2 && !wait_all(&bars[TILE_FREE0 + buf], ((k >> 1) - 1) & 1, abort)) {
+                give_up(abort);
+                break;
+            }
+            uint8_t* bo = sm + OFF_BUF + buf * BUF_BYTES;
+            const int h = g * hpg + hl0 + k;
+            const int64_t hrow = (b * a.H + h) * a.L + t0;
+            // Sp and Lm: 64 rows p x N/8 chunks; every value in registers first (8 chunks of each per thread
+            // for N = 128, 4 for N = 64)
+            const int64_t sbase = ((b * nc + c) * a.H + h) * (int64_t)kPb * N;
+            const int per = kPb * (N / 8) / 128;
+            float4 v[2][16];
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const float* src = (which ? a.LM : a.SP) + sbase;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    if (m < per) {
+                        const int e = lt + 128 * m;
+                        const float* sp = src + (int64_t)(e / (N / 8)) * N + 8 * (e % (N / 8));
+                        v[which][2 * m] = *reinterpret_cast<const float4*>(sp);
+                        v[which][2 * m + 1] = *reinterpret_cast<const float4*>(sp + 4);
+                    }
+                }
+            }
+            // their largest magnitudes over the loader warps -> the power-of-two scales (<= 1) that keep the
+            // fp16 tiles below 2^14; the partners of the accumulating products (X' of Lm, G'' of Sp) take the
+            // inverse, the row warps unscale SPC and LMB
+            float mx[2] = {0.f, 0.f};
+#pragma unroll
+            for (int which = 0; which < 2; ++which)
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    if (m < 2 * per)
+                        mx[which] = fmaxf(mx[which], fmaxf(fmaxf(fabsf(v[which][m].x), fabsf(v[which][m].y)),
+                                                           fmaxf(fabsf(v[which][m].z), fabsf(v[which][m].w))));
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+                mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
+            }
+            float* slots = vec + (V_MAX >> 2) + (k & 1) * 8;
+            if (lane == 0) {
+                slots[2 * (lt >> 5)] = mx[0];
+                slots[2 * (lt >> 5) + 1] = mx[1];
+            }
+            mbar_arrive(&bars[LMAX]);
+            if (!wait_all(&bars[LMAX], k & 1, abort)) {
+                give_up(abort);
+                break;
+            }
+            float sc[2];
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const float m = fmaxf(fmaxf(slots[which], slots[2 + which]), fmaxf(slots[4 + which], slots[6 + which]));
+                sc[which] = state_scale(m);
+            }
+            float range = 0.f;  // largest magnitude written to an fp16 tile
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                uint8_t* dst = bo + (which ? B_LM : B_SP);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    if (m < per) {
+                        const int e = lt + 128 * m, p = e / (N / 8), k8 = e % (N / 8);
+                        const float4 x0 = v[which][2 * m], x1 = v[which][2 * m + 1];
+                        const float f[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                        *reinterpret_cast<uint4*>(dst + (k8 >> 3) * 8192 + sw128_off(p, k8 & 7)) =
+                            pack8(f, sc[which], range);
+                    }
+                }
+            }
+            // x, X', g, G'': 64 rows x 8 chunks of 8 channels, four chunks per thread (rows lt / 8 + 16 m),
+            // all loads first
+            const float cs_last = a.CS[hrow + Qv - 1];
+            const int k8 = lt & 7;
+            float xv[4][8], gv[4][8], zv[4][8], dtr[4], csr[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int r = (lt >> 3) + 16 * m;
+                if (r < Qv) {
+                    dtr[m] = a.DT[hrow + r];
+                    csr[m] = a.CS[hrow + r];
+                    load8(a.U, (row0 + r) * conv_dim + (int64_t)h * kPb + 8 * k8, false, xv[m]);
+                    const int64_t yi = (row0 + r) * HP + (int64_t)h * kPb + 8 * k8;
+                    load8(a.dy, yi, a.dy_bf16, gv[m]);
+                    load8(a.z, yi, a.act_bf16, zv[m]);
+                } else {
+                    dtr[m] = csr[m] = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) xv[m][q] = gv[m][q] = zv[m][q] = 0.f;
+                }
+            }
+            const float inv_sp = 1.f / sc[0], inv_lm = 1.f / sc[1];  // exact: powers of two
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int r = (lt >> 3) + 16 * m;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) gv[m][q] = gv[m][q] * zv[m][q] * sigm(zv[m][q]);
+                const bool on = r < Qv;
+                const uint32_t off = sw128_off(r, k8);
+                *reinterpret_cast<uint4*>(bo + B_X + off) = pack8(xv[m], 1.f, range);
+                *reinterpret_cast<uint4*>(bo + B_XP + off) =
+                    pack8(xv[m], on ? dtr[m] * expf(cs_last - csr[m]) * inv_lm : 0.f, range);
+                *reinterpret_cast<uint4*>(bo + B_G + off) = pack8(gv[m], 1.f, range);
+                *reinterpret_cast<uint4*>(bo + B_GP + off) = pack8(gv[m], on ? expf(csr[m]) * inv_sp : 0.f, range);
+                if (k8 == 0) {
+                    vec[(V_DT >> 2) + buf * 64 + r] = dtr[m];
+                    vec[(V_CS >> 2) + buf * 64 + r] = csr[m];
+                }
+            }
+            if (lt == 0) {
+                vec[(V_SC >> 2) + buf * 2] = sc[0];
+                vec[(V_SC >> 2) + buf * 2 + 1] = sc[1];
+            }
+            if (!(range < 65504.f)) atomicOr(&g_chunk_bwd_tc_error, 2);
+            fence_async_smem();
+            mbar_arrive(&bars[TILE_FULL0 + buf]);
+        }
+    } else {
+        // ---------------- row warps 0, 1, 4, 5 ----------------
+        const int rq = warp & 3;           // token half: rows 32 rq .. 32 rq + 31
+        const int ch = warp >> 2;          // column half: 32 ch .. 32 ch + 31
+        const int r = 32 * rq + lane, c0 = 32 * ch;
+        const int wi = rq + 2 * ch;        // 0..3
+        const uint32_t lb = (uint32_t)(32 * rq) << 16;
+        bool ok = true;
+        if (warp == 0) {
+            if (lane == 0) mma_steps(tmem + COL_CB, kdesc(sm + OFF_TC), false, kdesc(sm + OFF_TB), false, ID_KK, 4 * nbox,
+                                     false);
+            ok = wait_all(&bars[TILE_FULL0], 0, abort);
+            if (ok) {
+                tc_fence_after();
+                if (lane == 0) issue_batch1(sm, tmem, 0, nbox, &bars[B1_DONE]);
+                __syncwarp();
+            }
+        }
+        for (int k = 0; k < nh && ok; ++k) {
+            const int buf = k & 1, par = k & 1;
+            const int h = g * hpg + hl0 + k;
+            const float Dh = a.D[h];
+            // this row's fp32 x, g and dy silu'(z) over the thread's 32 columns (zero past Qv)
+            float xr[32], gr[32], dyds[32];
+            {
+                const int64_t xi = (row0 + r) * conv_dim + (int64_t)h * kPb + c0;
+                const int64_t yi = (row0 + r) * HP + (int64_t)h * kPb + c0;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float xv[8], dy[8], zv[8];
+                    if (r < Qv) {
+                        load8(a.U, xi + 8 * q8, false, xv);
+                        load8(a.dy, yi + 8 * q8, a.dy_bf16, dy);
+                        load8(a.z, yi + 8 * q8, a.act_bf16, zv);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) xv[q] = dy[q] = zv[q] = 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float s = sigm(zv[q]);
+                        xr[8 * q8 + q] = xv[q];
+                        gr[8 * q8 + q] = dy[q] * zv[q] * s;
+                        dyds[8 * q8 + q] = dy[q] * s * (1.f + zv[q] * (1.f - s));
+                    }
+                }
+            }
+            // the loader's dt / cs of this head (TILE_FULL), then the first MMAs (B1_DONE)
+            if (!wait_all(&bars[TILE_FULL0 + buf], (k >> 1) & 1, abort) || !wait_all(&bars[B1_DONE], par, abort)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float* dts = vec + (V_DT >> 2) + buf * 64;
+            const float* css = vec + (V_CS >> 2) + buf * 64;
+            const float cs_r = css[r], dt_r = dts[r], cs_last = css[Qv - 1];
+            // the loader's scales of Sp and Lm: SPC and LMB come out of TMEM multiplied by them
+            const float usp = 1.f / vec[(V_SC >> 2) + buf * 2], ulm = 1.f / vec[(V_SC >> 2) + buf * 2 + 1];
+            // phase B: LCB and LGX' rows, the row sums of M and the column sums of GX L CB
+            float rowm = 0.f, range = 0.f;
+            {
+                float gx[32], cb[32];
+                tmem_ld32(tmem + lb + COL_GX + c0, gx);
+                tmem_ld32(tmem + lb + COL_CB + c0, cb);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t plcb[4], plgx[4];
+#pragma unroll
+                    for (int w2 = 0; w2 < 4; ++w2) {
+                        float lc[2], lg[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int q = 8 * q8 + 2 * w2 + u, j = c0 + q;
+                            const bool on = j <= r && r < Qv;
+                            const float L = on ? expf(cs_r - css[j]) : 0.f;
+                            const float lgx = gx[q] * L, dtj = dts[j];
+                            lc[u] = cb[q] * L * dtj;
+                            lg[u] = lgx * dtj;
+                            rowm += lg[u] * cb[q];
+                            gx[q] = lgx * cb[q];  // becomes this row's share of column j's sum
+                        }
+                        plcb[w2] = pack_h2(lc[0], lc[1]);
+                        plgx[w2] = pack_h2(lg[0], lg[1]);
+                        range = fmaxf(range, fmaxf(fmaxf(fabsf(lc[0]), fabsf(lc[1])), fmaxf(fabsf(lg[0]), fabsf(lg[1]))));
+                    }
+                    const uint32_t off = sw128_off(r, 4 * ch + q8);
+                    *reinterpret_cast<uint4*>(sm + OFF_LCB + off) = make_uint4(plcb[0], plcb[1], plcb[2], plcb[3]);
+                    *reinterpret_cast<uint4*>(sm + OFF_LGX + off) = make_uint4(plgx[0], plgx[1], plgx[2], plgx[3]);
+                }
+                fence_async_smem();
+                mbar_arrive(&bars[LT_FULL]);
+                if (!(range < 65504.f)) atomicOr(&g_chunk_bwd_tc_error, 2);
+                const float col = column_sums(gx, lane);
+                vec[(V_COL >> 2) + (par * 2 + rq) * 64 + c0 + lane] = col;
+            }
+            vec[(V_ROWM >> 2) + (par * 2 + ch) * 64 + r] = rowm;
+            float pd = 0.f;
+            {
+                float spc[32];
+                tmem_ld32(tmem + lb + COL_SPC + c0, spc);
+                tmem_wait_ld();
+                float e = 0.f;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    e += gr[q] * spc[q];
+                    pd += gr[q] * xr[q];
+                }
+                vec[(V_E >> 2) + (par * 2 + ch) * 64 + r] = e * usp;
+            }
+            if (warp == 0) {
+                if (!wait_all(&bars[LT_FULL], par, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) issue_batch2(sm, tmem, k, &bars[B2_DONE], &bars[TILE_FREE0 + buf]);
+                __syncwarp();
+            }
+            if (!wait_all(&bars[B2_DONE], par, abort)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // phase C: dz from the recomputed y; dx; W
+            const float ex_r = r < Qv ? expf(cs_r) : 0.f, el_r = r < Qv ? expf(cs_last - cs_r) : 0.f;
+            const float exu = ex_r * usp;
+            {
+                float yin[32], spc[32];
+                tmem_ld32(tmem + lb + COL_YIN + c0, yin);
+                tmem_ld32(tmem + lb + COL_SPC + c0, spc);
+                tmem_wait_ld();
+                if (r < Qv) {
+                    float* dz = a.dz + (row0 + r) * HP + (int64_t)h * kPb + c0;
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4) {
+                        float4 o;
+                        o.x = dyds[q] * (yin[q] + exu * spc[q] + Dh * xr[q]);
+                        o.y = dyds[q + 1] * (yin[q + 1] + exu * spc[q + 1] + Dh * xr[q + 1]);
+                        o.z = dyds[q + 2] * (yin[q + 2] + exu * spc[q + 2] + Dh * xr[q + 2]);
+                        o.w = dyds[q + 3] * (yin[q + 3] + exu * spc[q + 3] + Dh * xr[q + 3]);
+                        *reinterpret_cast<float4*>(dz + q) = o;
+                    }
+                }
+            }
+            float wpart = 0.f;
+            {
+                float lmb[32], dxi[32];
+                tmem_ld32(tmem + lb + COL_LMB + c0, lmb);
+                tmem_ld32(tmem + lb + COL_DXI + c0, dxi);
+                tmem_wait_ld();
+                const float f = dt_r * el_r * ulm;
+                float* du = a.DU + (row0 + r) * conv_dim + (int64_t)h * kPb + c0;
+#pragma unroll
+                for (int q = 0; q < 32; q += 4) {
+                    float4 o;
+                    o.x = dxi[q] + f * lmb[q] + Dh * gr[q];
+                    o.y = dxi[q + 1] + f * lmb[q + 1] + Dh * gr[q + 1];
+                    o.z = dxi[q + 2] + f * lmb[q + 2] + Dh * gr[q + 2];
+                    o.w = dxi[q + 3] + f * lmb[q + 3] + Dh * gr[q + 3];
+                    if (r < Qv) *reinterpret_cast<float4*>(du + q) = o;
+                    wpart += xr[q] * lmb[q] + xr[q + 1] * lmb[q + 1] + xr[q + 2] * lmb[q + 2] + xr[q + 3] * lmb[q + 3];
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[ACC_FREE]);
+            if (warp == 0 && k + 1 < nh) {
+                if (!wait_all(&bars[ACC_FREE], par, abort) ||
+                    !wait_all(&bars[TILE_FULL0 + (buf ^ 1)], ((k + 1) >> 1) & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) issue_batch1(sm, tmem, k + 1, nbox, &bars[B1_DONE]);
+                __syncwarp();
+            }
+            vec[(V_W >> 2) + (par * 2 + ch) * 64 + r] = el_r * ulm * wpart;
+            pd = warp_sum(pd);
+            if (lane == 0) vec[(V_PD >> 2) + par * 4 + wi] = pd;
+            mbar_arrive(&bars[WSYNC]);
+            if (warp == 0) {
+                // the head's per-token scalars: tokens lane and lane + 32
+                if (!wait_all(&bars[WSYNC], par, abort)) {
+                    ok = false;
+                    break;
+                }
+                const float* col = vec + (V_COL >> 2) + par * 128;
+                const float* rwm = vec + (V_ROWM >> 2) + par * 128;
+                const float* ev = vec + (V_E >> 2) + par * 128;
+                const float* wv = vec + (V_W >> 2) + par * 128;
+                const float Ah = a.A[h], bias = a.dt_bias[h];
+                float dr0[2], dtk[2], d[2], e[2], w[2], dw[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int kk = lane + 32 * u;
+                    dr0[u] = col[kk] + col[64 + kk];
+                    dtk[u] = dts[kk];
+                    d[u] = dtk[u] * dr0[u] - (rwm[kk] + rwm[64 + kk]);
+                    e[u] = (kk < Qv ? expf(css[kk]) : 0.f) * (ev[kk] + ev[64 + kk]);
+                    w[u] = wv[kk] + wv[64 + kk];
+                    dw[u] = dtk[u] * w[u];
+                }
+                // exclusive prefix sums of d and dt W, inclusive suffix sums of E, over the 64 tokens
+                auto scan_excl = [&](const float (&v)[2], float (&out)[2]) {
+                    float s0 = v[0];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float t = __shfl_up_sync(0xffffffffu, s0, o);
+                        if (lane >= o) s0 += t;
+                    }
+                    const float tot0 = __shfl_sync(0xffffffffu, s0, 31);
+                    float s1 = v[1];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float t = __shfl_up_sync(0xffffffffu, s1, o);
+                        if (lane >= o) s1 += t;
+                    }
+                    out[0] = s0 - v[0];
+                    out[1] = tot0 + s1 - v[1];
+                };
+                float R[2], Wp[2], Es[2];
+                scan_excl(d, R);
+                scan_excl(dw, Wp);
+                {
+                    float ex_[2];
+                    scan_excl(e, ex_);
+                    const float etot = __shfl_sync(0xffffffffu, ex_[1] + e[1], 31);
+                    Es[0] = etot - ex_[0];
+                    Es[1] = etot - ex_[1];
+                }
+                float F = 0.f;
+                for (int s = 0; s < a.nsplit_pf; ++s) F += a.PF[((b * nc + c) * a.H + h) * a.nsplit_pf + s];
+                float pdA = 0.f, pbias = 0.f;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int kk = lane + 32 * u;
+                    if (kk < Qv) {
+                        const float dda = R[u] + Es[u] + F + Wp[u];
+                        const float ddt = dr0[u] + w[u] + Ah * dda;
+                        const int64_t di = (row0 + kk) * a.H + h;
+                        const float raw = a.act_bf16 ? bf_lo(static_cast<const unsigned short*>(a.dt)[di])
+                                                     : static_cast<const float*>(a.dt)[di];
+                        const float dr = ddt * sigm(raw + bias);
+                        a.ddt[di] = dr;
+                        pdA += dtk[u] * dda;
+                        pbias += dr;
+                    }
+                }
+                pdA = warp_sum(pdA);
+                pbias = warp_sum(pbias);
+                if (lane == 0) {
+                    const float* pdw = vec + (V_PD >> 2) + par * 4;
+                    float* ph = a.PH + ((b * nc + c) * a.H + h) * 3;
+                    ph[0] = pdA;
+                    ph[1] = (pdw[0] + pdw[1]) + (pdw[2] + pdw[3]);
+                    ph[2] = pbias;
+                }
+                __syncwarp();
+            }
+            mbar_arrive(&bars[TILE_FREE0 + buf]);
+        }
+        if (!ok) give_up(abort);
+        if (warp == 0) {
+            if (lane == 0) mma_commit(&bars[FINAL]);  // every MMA issued so far
+            __syncwarp();
+        }
+    }
+
+    // every role is done issuing; dB^T and dC^T are final once the last MMAs complete
+    const bool done = __all_sync(0xffffffffu, mbar_wait(&bars[FINAL], 0, nullptr));
+    tc_fence_after();
+    __syncthreads();
+    if (done && *abort == 0) {
+        const int n = 32 * (warp & 3) + lane, j0 = 32 * (warp >> 2);
+        const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
+        float db[32], dc[32];
+        tmem_ld32(tmem + lb + COL_DB + j0, db);
+        tmem_ld32(tmem + lb + COL_DC + j0, dc);
+        tmem_wait_ld();
+        if (n < N) {
+            for (int q = 0; q < 32; ++q) {
+                const int j = j0 + q;
+                if (j < Qv) {
+                    float* dst = half == 0 ? a.DU + (row0 + j) * conv_dim + HP : a.DU2 + (row0 + j) * 2 * GN;
+                    dst[(int64_t)g * N + n] = db[q];
+                    dst[GN + (int64_t)g * N + n] = dc[q];
+                }
+            }
+        }
+    } else if (tid == 0 && !done) {
+        atomicOr(&g_chunk_bwd_tc_error, 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS_B);
+    }
+}
+
+}  // namespace
+
+bool chunk_bwd_tc_supported(int P, int N, bool act_bf16, const void* dy, const void* z, const void* dz) {
+    const uintptr_t bits = reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(z) |
+                           reinterpret_cast<uintptr_t>(dz);
+    return act_bf16 && P == kPb && (N == 64 || N == 128) && (bits & 15u) == 0;
+}
+
+cudaError_t read_and_clear_chunk_bwd_tc_error(int* flag) {
+    cudaError_t e = cudaMemcpyFromSymbol(flag, g_chunk_bwd_tc_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_chunk_bwd_tc_error, &zero, sizeof(int));
+}
+
+cudaError_t launch_chunk_bwd_tc(const ChunkBwdTcArgs& a, int64_t nchunks, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_B);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>(nchunks), static_cast<unsigned>(a.G * a.split),
+                    static_cast<unsigned>(a.batch));
+    chunk_bwd_tc_kernel<<<grid, kThreadsB, SMEM_B, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace bwd
+}  // namespace ssd

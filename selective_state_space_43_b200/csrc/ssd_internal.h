@@ -100,6 +100,8 @@ cudaError_t launch_prefill_backward(const BwdArgs& a, cudaStream_t st);
 // Reads and clears the error word of the backward's tensor-core kernel (ssd_backward_tc.cu; nonzero: a
 // bounded wait gave up).  Does not synchronise: call after the stream is idle.
 cudaError_t read_and_clear_bwd_tc_error(int* flag);
+// The same for the tensor-core per-chunk backward (ssd_chunk_bwd_tc.cu).
+cudaError_t read_and_clear_chunk_bwd_tc_error(int* flag);
 }  // namespace bwd
 
 }  // namespace ssd

@@ -123,7 +123,8 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 }
 
 // ---- MMA (single thread issues) ----------------------------------------------------------------------------
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
+// D[tmem] (+)= A[smem] * B[smem]^T, 16-bit inputs (kind::f16: the instruction descriptor says bf16 or fp16,
+// the same for A and B), fp32 accumulate.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          uint32_t accumulate) {
     asm volatile(

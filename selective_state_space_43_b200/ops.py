@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libssd_b200.so")
 
 SSD_F32, SSD_BF16, SSD_BF16_YF32 = 0, 1, 2
 STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE", 4: "SSD_ERR_ALIGN",
-          5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_WORKSPACE", 8: "SSD_ERR_TIMEOUT"}
+          5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA", 7: "SSD_ERR_WORKSPACE", 8: "SSD_ERR_TIMEOUT",
+          9: "SSD_ERR_RANGE"}
 
 
 class SsdDims(ctypes.Structure):
@@ -543,7 +544,8 @@ def mimo_decode_step(x, dt, B, C, z, A, D, dt_bias, ssm_state, y=None, y_dtype=N
 
 def device_status(device="cuda"):
     """Synchronise the current stream; raise if a kernel gave up on a bounded device-side wait
-    (SSD_ERR_TIMEOUT) or met invalid packed-sequence offsets (SSD_ERR_SHAPE)."""
+    (SSD_ERR_TIMEOUT), met invalid packed-sequence offsets (SSD_ERR_SHAPE) or, in the tensor-core backward,
+    an operand beyond fp16 range (SSD_ERR_RANGE)."""
     st = lib().ssd_device_status(_stream_ptr(torch.device(device)))
     if st != 0:
         raise SsdError(st, "ssd_device_status")

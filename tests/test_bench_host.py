@@ -73,6 +73,12 @@ def test_backward_work_counts():
     per_head = 8 * 64 * 64 * 128 + 4 * 64 * 64 * 64 + 2 * 64 * 64 * 128
     assert bench.backward_chunk_flops(d) == 64 * (128 * per_head + 8 * 2 * 64 * 64 * 128)
     assert abs(bench.FP32_ALU_TFLOPS - 74.45) < 0.01
+    # the tensor-core chunk backward: fp32 post-conv x|B|C, dt, cs; bf16 dy, z, dt; fp32 states and adjoints;
+    # dz, dx, two halves of dB|dC, ddt written (fp32), and the small per-chunk partials
+    reads = 4096 * (8192 + 2048) * 4 + 4096 * 2 * 128 * 4 + 4096 * (2 * 8192 + 128) * 2 + \
+        2 * 64 * 128 * 64 * 128 * 4 + 64 * 128 * 16
+    writes = 4096 * 2 * 8192 * 4 + 2 * 4096 * 2048 * 4 + 4096 * 128 * 4 + 64 * 128 * 12
+    assert bench.backward_chunk_bytes(d, 2) == reads + writes
 
 
 def test_mimo_decode_byte_count():
@@ -135,12 +141,12 @@ def test_backward_and_mimo_bench_legs_on_a_fake_device(monkeypatch):
     d = Dims(1, 256, 4, 64, 32, 2, 128)
     flush = torch.empty(16)
     peaks = {"hbm_gbs": 6554.6}
-    b = bench.bench_backward(fake, d, torch.bfloat16, torch.device("cpu"), flush, 5, 3, 1, _FakeSampler())
+    b = bench.bench_backward(fake, d, torch.bfloat16, torch.device("cpu"), flush, 5, 3, 1, _FakeSampler(), peaks)
     assert fake.calls["backward"] == 3 + 5 and fake.calls["events"][-1] is True   # hook cleared afterwards
     assert b["ms_per_step"] == 2.0 and b["value"] == 256 / 2e-3
     rf = b["dominant_kernel"]["roofline"]
-    assert rf["bound"] == "alu" and rf["unit"] == "TFLOP/s"
-    assert abs(rf["achieved"] - bench.backward_chunk_flops(d) / 2e-3 / 1e12) < 1e-9
+    assert rf["bound"] == "hbm" and rf["unit"] == "GB/s" and rf["peak"] == 6554.6
+    assert abs(rf["achieved"] - bench.backward_chunk_bytes(d, 2) / 2e-3 / 1e9) < 1e-6
     m = bench.bench_mimo(fake, d, torch.bfloat16, torch.device("cpu"), 1, _FakeSampler(), peaks, 4)
     assert fake.calls["mimo"] == 3 + 4
     assert abs(m["value"] - bench.mimo_decode_bytes(d, bench.MIMO_RANK, 2) / 2e-3 / 1e9) < 1e-6
