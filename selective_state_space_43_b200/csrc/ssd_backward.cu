@@ -51,6 +51,7 @@
 #define SSD_SET_SMEM(kern, bytes) cudaSuccess
 #define SSD_DYN_SMEM() (::emu::smem())
 #else
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #define SSD_LAUNCH(kern, grid, block, smem, st, ...) kern<<<(grid), (block), (smem), (st)>>>(__VA_ARGS__)
 #define SSD_SET_SMEM(kern, bytes) \
@@ -93,6 +94,14 @@ struct Ws {
     float* PH;  // [batch][nc][H][3]     per-chunk partial dA, dD, ddt_bias
     float* PW;  // [batch][ntile][conv_dim][5]  per-tile partial dconv_w (4), dconv_b
     float* DU2; // [batch][L][2 G N]     dB | dC of the second half of each group's heads (when split)
+    // for the tensor-core chunk backward (else unused): the entering states and leaving adjoints as fp16
+    // tiles, [batch][nc][H][N/64 boxes][64 rows p][64 n] with 128-byte rows and the 128-byte swizzle (the
+    // shared-memory image its MMAs read), each row p scaled by a power of two s_p <= 1 that keeps it below
+    // 2^14, and the inverses 1/s_p [batch][nc][H][64]
+    float* SPH;
+    float* LMH;
+    float* SPS;
+    float* LMS;
 };
 
 namespace {
@@ -106,15 +115,16 @@ inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 // Carves the workspace; returns the bytes used (base may be null to only count).
 size_t carve(int64_t batch, int64_t L, int H, int P, int N, int G, char* base, Ws* ws) {
     const int64_t conv_dim = (int64_t)H * P + 2LL * G * N, nc = nchunks(L), nt = ntiles(L);
-    const size_t sizes[10] = {
+    const size_t sizes[14] = {
         (size_t)(batch * L * conv_dim), (size_t)(batch * L * conv_dim), (size_t)(batch * H * L),
         (size_t)(batch * H * L),        (size_t)(batch * nc * H * P * N), (size_t)(batch * nc * H * P * N),
         (size_t)(batch * nc * H * kSplit), (size_t)(batch * nc * H * 3),  (size_t)(batch * nt * conv_dim * 5),
-        (size_t)(batch * L * 2 * G * N)};
-    float** slots[10] = {&ws->U,  &ws->DU, &ws->DT, &ws->CS, &ws->SP,
-                         &ws->LM, &ws->PF, &ws->PH, &ws->PW, &ws->DU2};
+        (size_t)(batch * L * 2 * G * N), (size_t)(batch * nc * H * P * N / 2), (size_t)(batch * nc * H * P * N / 2),
+        (size_t)(batch * nc * H * P),   (size_t)(batch * nc * H * P)};
+    float** slots[14] = {&ws->U,  &ws->DU, &ws->DT,  &ws->CS,  &ws->SP,  &ws->LM,  &ws->PF,
+                         &ws->PH, &ws->PW, &ws->DU2, &ws->SPH, &ws->LMH, &ws->SPS, &ws->LMS};
     size_t off = 0;
-    for (int k = 0; k < 10; ++k) {
+    for (int k = 0; k < 14; ++k) {
         if (base) *slots[k] = reinterpret_cast<float*>(base + off);
         off += round256(sizes[k] * sizeof(float));
     }
@@ -437,11 +447,68 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return total;
 }
 
-// grid (H * kSplit, batch), kT threads: the P*N state elements of a head in kSplit contiguous slices,
-// P*N / (kSplit * kT) per thread.  The forward scan turns SP into the states entering each chunk, the
-// reverse scan turns LM into the adjoints leaving each chunk and leaves each slice's part of F; the next
-// chunk's values are loaded before the current chunk's are stored, so the loads of consecutive chunks
-// overlap.
+// M consecutive floats (16-byte aligned when M is a multiple of 4).
+template <int M>
+__device__ __forceinline__ void ld_vec(const float* p, float (&v)[M]) {
+    if constexpr (M % 4 == 0) {
+#pragma unroll
+        for (int m = 0; m < M; m += 4) {
+            const float4 t = *reinterpret_cast<const float4*>(p + m);
+            v[m] = t.x, v[m + 1] = t.y, v[m + 2] = t.z, v[m + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < M; ++m) v[m] = p[m];
+    }
+}
+template <int M>
+__device__ __forceinline__ void st_vec(float* p, const float (&v)[M]) {
+    if constexpr (M % 4 == 0) {
+#pragma unroll
+        for (int m = 0; m < M; m += 4) *reinterpret_cast<float4*>(p + m) = make_float4(v[m], v[m + 1], v[m + 2], v[m + 3]);
+    } else {
+#pragma unroll
+        for (int m = 0; m < M; ++m) p[m] = v[m];
+    }
+}
+
+#ifndef SSD_EMU
+// Writes this thread's M (8 or 4) consecutive elements n0.. of state row p as fp16 into the swizzled tile of one
+// (chunk, head) (see Ws::SPH), scaled by the row's power of two s_p <= 1 (the 16 lanes that hold row p agree on
+// it), and 1/s_p into the row's scale slot.
+template <int M>
+__device__ __forceinline__ void store_half_row(const float (&v)[M], int p, int n0, char* tile, float* inv_scale) {
+    float mx = 0.f;
+#pragma unroll
+    for (int m = 0; m < M; ++m) mx = fmaxf(mx, fabsf(v[m]));
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sc = 1.f;
+    if (!(mx < 16384.f)) {
+        const int e = min(((__float_as_int(mx) >> 23) & 0xff) - 127, 128);  // mx in [2^e, 2^(e+1))
+        sc = __int_as_float((127 + 13 - e) << 23);                           // mx * sc in [2^13, 2^14)
+    }
+    uint32_t w[M / 2];
+#pragma unroll
+    for (int m = 0; m < M; m += 2) {
+        __half2 hv = __floats2half2_rn(v[m] * sc, v[m + 1] * sc);
+        w[m / 2] = *reinterpret_cast<uint32_t*>(&hv);
+    }
+    const int k8 = n0 >> 3;
+    char* dst = tile + (k8 >> 3) * 8192 + p * 128 + (((k8 & 7) ^ (p & 7)) << 4) + ((n0 & 7) ? 8 : 0);
+    if constexpr (M == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    else *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    if ((threadIdx.x & 15) == 0) inv_scale[p] = 1.f / sc;
+}
+#endif
+
+// grid (H * kSplit, batch), kT threads: the P*N state elements of a head in kSplit slices of P / kSplit whole
+// rows p; a thread holds M = P*N / (kSplit * kT) consecutive elements of one row (16 threads per row).  The
+// forward scan turns SP into the states entering each chunk, the reverse scan turns LM into the adjoints
+// leaving each chunk and leaves each slice's part of F; the next chunk's values are loaded before the
+// current chunk's are stored, so the loads of consecutive chunks overlap.  For the tensor-core chunk
+// backward (ws.SPH set) the entering states are also written as scaled fp16 tiles, and the leaving adjoints
+// only as such tiles (the fp32 ones have no other reader).
 template <int N>
 __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
     constexpr int M = kP * N / (kSplit * kT);
@@ -449,33 +516,32 @@ __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
     const int64_t nc = nchunks(a.L), b = blockIdx.y;
     const int h = blockIdx.x / kSplit, sp = blockIdx.x % kSplit, tid = threadIdx.x;
     float* red = reinterpret_cast<float*>(SSD_DYN_SMEM());
-    const int64_t head = (b * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
+    const int64_t off = (int64_t)sp * SLICE + (int64_t)tid * M;  // this thread's first element in a P x N block
+    const int64_t head = (b * a.H + h) * (int64_t)kP * N + off;
+    const int prow = static_cast<int>(off / N), n0 = static_cast<int>(off % N);
     const float* csh = ws.CS + (b * a.H + h) * a.L;
+    const bool half_tiles = ws.SPH != nullptr;
+    auto blk = [&](int64_t c) { return ((b * nc + c) * a.H + h) * (int64_t)kP * N; };
 
     float s[M], cur[M], nxt[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        s[m] = a.init_state ? a.init_state[head + tid + kT * m] : 0.f;
-        cur[m] = 0.f;
-        nxt[m] = 0.f;
-    }
-    if (nc > 0) {
-        const int64_t base = ((b * nc) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
-#pragma unroll
-        for (int m = 0; m < M; ++m) cur[m] = ws.SP[base + tid + kT * m];
-    }
+    for (int m = 0; m < M; ++m) s[m] = cur[m] = nxt[m] = 0.f;
+    if (a.init_state) ld_vec<M>(a.init_state + head, s);
+    if (nc > 0) ld_vec<M>(ws.SP + blk(0) + off, cur);
     for (int64_t c = 0; c < nc; ++c) {
         const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
         const float decay = expf(csh[last]);
-        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
-        if (c + 1 < nc) {
-            const int64_t nb = base + (int64_t)a.H * kP * N;
-#pragma unroll
-            for (int m = 0; m < M; ++m) nxt[m] = ws.SP[nb + tid + kT * m];
+        if (c + 1 < nc) ld_vec<M>(ws.SP + blk(c + 1) + off, nxt);
+        st_vec<M>(ws.SP + blk(c) + off, s);
+#ifndef SSD_EMU
+        if constexpr (M == 4 || M == 8) {
+            if (half_tiles)
+                store_half_row<M>(s, prow, n0, reinterpret_cast<char*>(ws.SPH) + blk(c) * 2,
+                                  ws.SPS + ((b * nc + c) * a.H + h) * kP);
         }
+#endif
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            ws.SP[base + tid + kT * m] = s[m];
             s[m] = decay * s[m] + cur[m];
             cur[m] = nxt[m];
         }
@@ -483,34 +549,35 @@ __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
 
     float l[M], sp_cur[M], sp_nxt[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        l[m] = a.d_final ? a.d_final[head + tid + kT * m] : 0.f;
-        cur[m] = nxt[m] = sp_cur[m] = sp_nxt[m] = 0.f;
-    }
+    for (int m = 0; m < M; ++m) l[m] = cur[m] = nxt[m] = sp_cur[m] = sp_nxt[m] = 0.f;
+    if (a.d_final) ld_vec<M>(a.d_final + head, l);
     if (nc > 0) {
-        const int64_t base = ((b * nc + nc - 1) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            cur[m] = ws.LM[base + tid + kT * m];
-            sp_cur[m] = ws.SP[base + tid + kT * m];
-        }
+        ld_vec<M>(ws.LM + blk(nc - 1) + off, cur);
+        ld_vec<M>(ws.SP + blk(nc - 1) + off, sp_cur);
     }
     for (int64_t c = nc - 1; c >= 0; --c) {
         const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
         const float decay = expf(csh[last]);
-        const int64_t base = ((b * nc + c) * a.H + h) * (int64_t)kP * N + (int64_t)sp * SLICE;
         if (c > 0) {
-            const int64_t pb = base - (int64_t)a.H * kP * N;
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                nxt[m] = ws.LM[pb + tid + kT * m];
-                sp_nxt[m] = ws.SP[pb + tid + kT * m];
-            }
+            ld_vec<M>(ws.LM + blk(c - 1) + off, nxt);
+            ld_vec<M>(ws.SP + blk(c - 1) + off, sp_nxt);
         }
+#ifndef SSD_EMU
+        if constexpr (M == 4 || M == 8) {
+            if (half_tiles)
+                store_half_row<M>(l, prow, n0, reinterpret_cast<char*>(ws.LMH) + blk(c) * 2,
+                                  ws.LMS + ((b * nc + c) * a.H + h) * kP);
+            else
+                st_vec<M>(ws.LM + blk(c) + off, l);
+        } else {
+            st_vec<M>(ws.LM + blk(c) + off, l);
+        }
+#else
+        st_vec<M>(ws.LM + blk(c) + off, l);
+#endif
         float f = 0.f;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            ws.LM[base + tid + kT * m] = l[m];
             f += l[m] * sp_cur[m];
             l[m] = decay * l[m] + cur[m];
             cur[m] = nxt[m];
@@ -519,10 +586,7 @@ __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
         f = block_sum(f, red);
         if (tid == 0) ws.PF[((b * nc + c) * a.H + h) * kSplit + sp] = decay * f;
     }
-    if (a.d_init_state) {
-#pragma unroll
-        for (int m = 0; m < M; ++m) a.d_init_state[head + tid + kT * m] = l[m];
-    }
+    if (a.d_init_state) st_vec<M>(a.d_init_state + head, l);
 }
 
 template <int N>
@@ -954,6 +1018,13 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         SSD_LAUNCH(dt_kernel, dim3(static_cast<unsigned>((nc * a.H + kT - 1) / kT), static_cast<unsigned>(a.batch)),
                    dim3(kT), 0, st, a, ws);
         const dim3 chunk_heads(static_cast<unsigned>(nc), static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+        Ws wsp = ws;  // the state pass writes the fp16 state tiles only for the tensor-core chunk backward
+#ifndef SSD_EMU
+        const bool tc_chunk = chunk_bwd_tc_supported(a.P, N, a.act_bf16, a.dy, a.z, a.dz);
+#else
+        const bool tc_chunk = false;
+#endif
+        if (!tc_chunk) wsp.SPH = wsp.LMH = wsp.SPS = wsp.LMS = nullptr;
 #ifndef SSD_EMU
         if (chunk_state_tc_supported(a.P, N, a.act_bf16)) {
             ChunkStateTcArgs t{a.batch, a.L, a.H, a.G, N, a.act_bf16, a.dy_bf16, ws.U, ws.DT, ws.CS, a.dy, a.z,
@@ -966,17 +1037,17 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         SSD_LAUNCH(chunk_state_kernel<N>, chunk_heads, dim3(kT), state_smem, st, a, ws);
 #endif
         SSD_LAUNCH(state_pass_kernel<N>, dim3(static_cast<unsigned>(a.H * kSplit), static_cast<unsigned>(a.batch)),
-                   dim3(kT), kT * sizeof(float), st, a, ws);
+                   dim3(kT), kT * sizeof(float), st, a, wsp);
         const dim3 chunk_groups(static_cast<unsigned>(nc), static_cast<unsigned>(a.G * head_split(a.H, a.G)),
                                 static_cast<unsigned>(a.batch));
 #ifndef SSD_EMU
         if (a.ev_before) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_before), st);
 #endif
 #ifndef SSD_EMU
-        if (chunk_bwd_tc_supported(a.P, N, a.act_bf16, a.dy, a.z, a.dz)) {
-            ChunkBwdTcArgs t{a.batch, a.L,  a.H,   a.G,  N,     head_split(a.H, a.G), kSplit, a.act_bf16, a.dy_bf16,
-                             a.A,     a.D,  a.dt_bias, a.dt, a.z, a.dy,  ws.U,  ws.DT, ws.CS, ws.SP, ws.LM, ws.PF,
-                             a.dz,    a.ddt, ws.DU, ws.DU2, ws.PH};
+        if (tc_chunk) {
+            ChunkBwdTcArgs t{a.batch,  a.L,   a.H,    a.G,    N,      head_split(a.H, a.G), kSplit, a.act_bf16,
+                             a.dy_bf16, a.A,  a.D,    a.dt_bias, a.dt, a.z, a.dy, ws.U, ws.DT, ws.CS, ws.SPH, ws.LMH,
+                             ws.SPS,   ws.LMS, ws.PF, a.dz,   a.ddt,  ws.DU,  ws.DU2, ws.PH};
             if ((err = launch_chunk_bwd_tc(t, nc, st)) != cudaSuccess) return err;
         } else {
             SSD_LAUNCH(chunk_bwd_kernel<N>, chunk_groups, dim3(kT), chunk_smem, st, a, ws);

@@ -47,13 +47,18 @@ struct ChunkStateTcArgs {
 // Inputs and outputs of the tensor-core per-chunk backward (ssd_backward_tc.cu), which writes exactly what
 // the CUDA-core chunk kernel writes: dz, ddt, the post-conv gradients of x (DU) and of B, C (DU for the
 // first half of each group's heads, DU2 for the second), and the per-chunk partials PH.
+// The entering states and leaving adjoints come as the state pass's fp16 tiles SPH, LMH
+// [batch][nchunks][H][N/64][64][64] (128-byte swizzled rows, row p scaled by s_p) with the inverse row
+// scales SPS, LMS [batch][nchunks][H][64].
 struct ChunkBwdTcArgs {
     int64_t batch, L;
     int H, G, N, split, nsplit_pf;  // heads-per-group halves (1 or 2); partial sums per chunk in PF
     bool act_bf16, dy_bf16;
     const float *A, *D, *dt_bias;
     const void *dt, *z, *dy;
-    const float *U, *DT, *CS, *SP, *LM, *PF;
+    const float *U, *DT, *CS;
+    const void *SPH, *LMH;
+    const float *SPS, *LMS, *PF;
     float *dz, *ddt, *DU, *DU2, *PH;
 };
 

@@ -78,12 +78,11 @@ constexpr uint32_t V_ROWM = 2048;       //   row sums of M [2][2 column halves][
 constexpr uint32_t V_E = 3072;          //   g_i . SPC_i partials [2][2][64]
 constexpr uint32_t V_W = 4096;          //   W_j partials [2][2][64]
 constexpr uint32_t V_PD = 5120;         //   sum g . x per row warp [2][4]
-constexpr uint32_t V_MAX = 5152;        //   largest |Sp|, |Lm| per loader warp [2 head parities][4][2]
-constexpr uint32_t V_SC = 5216;         //   the Sp, Lm scales of each buffer [2][2]
-constexpr uint32_t VEC_BYTES = 5248;
+constexpr uint32_t V_ISC = 5248;        //   inverse row scales of each buffer's Sp, Lm tiles [2][2][64]
+constexpr uint32_t VEC_BYTES = 6272;
 constexpr uint32_t OFF_BAR = OFF_VEC + VEC_BYTES;
 enum : int { TILE_FULL0, TILE_FULL1, TILE_FREE0, TILE_FREE1, B1_DONE, LT_FULL, B2_DONE, ACC_FREE, WSYNC, FINAL,
-             LMAX, NBAR };
+             SPLM_FULL0, SPLM_FULL1, NBAR };
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // abort word, TMEM base
 constexpr uint32_t SMEM_B = OFF_MISC + 16 + 1024;  // + alignment slack
 
@@ -127,11 +126,12 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8], float s, float& rang
     }
     return make_uint4(pack_h2(w[0], w[1]), pack_h2(w[2], w[3]), pack_h2(w[4], w[5]), pack_h2(w[6], w[7]));
 }
-// The power of two s <= 1 that brings a tile whose largest magnitude is m below 2^14 (1 when it already is).
-__device__ __forceinline__ float state_scale(float m) {
-    if (m < 16384.f) return 1.f;
-    const int e = min(((__float_as_int(m) >> 23) & 0xff) - 127, 128);  // m in [2^e, 2^(e+1))
-    return __int_as_float((127 + 13 - e) << 23);                        // m * s in [2^13, 2^14)
+// Eight values v[q] f[q] s as fp16 (the per-column inverse state scales f), tracking `range` likewise.
+__device__ __forceinline__ uint4 pack8s(const float (&v)[8], const float (&f)[8], float s, float& range) {
+    float w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) w[q] = v[q] * f[q];
+    return pack8(w, s, range);
 }
 
 // D (+)= A B over K = 16 * steps; a K-major operand steps 32 bytes inside a box and 8 KB from box to box,
@@ -240,7 +240,8 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
         mbar_init(&bars[ACC_FREE], 128);
         mbar_init(&bars[WSYNC], 128);
         mbar_init(&bars[FINAL], 1);
-        mbar_init(&bars[LMAX], 128);
+        mbar_init(&bars[SPLM_FULL0], 1);  // the bulk copies' transaction bytes
+        mbar_init(&bars[SPLM_FULL1], 1);
         fence_mbar_init();
     }
     // the group's post-conv B and C (rows past Qv zero): 64 rows x N/8 chunks of 8 channels
@@ -278,70 +279,18 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             uint8_t* bo = sm + OFF_BUF + buf * BUF_BYTES;
             const int h = g * hpg + hl0 + k;
             const int64_t hrow = (b * a.H + h) * a.L + t0;
-            // Sp and Lm: 64 rows p x N/8 chunks; every value in registers first (8 chunks of each per thread
-            // for N = 128, 4 for N = 64)
-            const int64_t sbase = ((b * nc + c) * a.H + h) * (int64_t)kPb * N;
-            const int per = kPb * (N / 8) / 128;
-            float4 v[2][16];
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const float* src = (which ? a.LM : a.SP) + sbase;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    if (m < per) {
-                        const int e = lt + 128 * m;
-                        const float* sp = src + (int64_t)(e / (N / 8)) * N + 8 * (e % (N / 8));
-                        v[which][2 * m] = *reinterpret_cast<const float4*>(sp);
-                        v[which][2 * m + 1] = *reinterpret_cast<const float4*>(sp + 4);
-                    }
-                }
-            }
-            // their largest magnitudes over the loader warps -> the power-of-two scales (<= 1) that keep the
-            // fp16 tiles below 2^14; the partners of the accumulating products (X' of Lm, G'' of Sp) take the
-            // inverse, the row warps unscale SPC and LMB
-            float mx[2] = {0.f, 0.f};
-#pragma unroll
-            for (int which = 0; which < 2; ++which)
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    if (m < 2 * per)
-                        mx[which] = fmaxf(mx[which], fmaxf(fmaxf(fabsf(v[which][m].x), fabsf(v[which][m].y)),
-                                                           fmaxf(fabsf(v[which][m].z), fabsf(v[which][m].w))));
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
-                mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
-            }
-            float* slots = vec + (V_MAX >> 2) + (k & 1) * 8;
-            if (lane == 0) {
-                slots[2 * (lt >> 5)] = mx[0];
-                slots[2 * (lt >> 5) + 1] = mx[1];
-            }
-            mbar_arrive(&bars[LMAX]);
-            if (!wait_all(&bars[LMAX], k & 1, abort)) {
-                give_up(abort);
-                break;
-            }
-            float sc[2];
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const float m = fmaxf(fmaxf(slots[which], slots[2 + which]), fmaxf(slots[4 + which], slots[6 + which]));
-                sc[which] = state_scale(m);
-            }
-            float range = 0.f;  // largest magnitude written to an fp16 tile
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                uint8_t* dst = bo + (which ? B_LM : B_SP);
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    if (m < per) {
-                        const int e = lt + 128 * m, p = e / (N / 8), k8 = e % (N / 8);
-                        const float4 x0 = v[which][2 * m], x1 = v[which][2 * m + 1];
-                        const float f[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                        *reinterpret_cast<uint4*>(dst + (k8 >> 3) * 8192 + sw128_off(p, k8 & 7)) =
-                            pack8(f, sc[which], range);
-                    }
-                }
+            // Sp and Lm: the state pass's fp16 tiles (each row p scaled by s_p) and their inverse row scales,
+            // four bulk copies onto this buffer's barrier
+            const int64_t ti = (b * nc + c) * a.H + h;
+            const uint32_t tile_bytes = 8192u * (uint32_t)nbox;
+            float* isc = vec + (V_ISC >> 2) + buf * 128;  // 1/s_p of Sp [64], then of Lm [64]
+            if (lt == 0) {
+                uint64_t* bar = &bars[SPLM_FULL0 + buf];
+                mbar_arrive_expect_tx(bar, 2 * tile_bytes + 2 * 256);
+                bulk_load(bo + B_SP, static_cast<const char*>(a.SPH) + ti * tile_bytes, tile_bytes, bar);
+                bulk_load(bo + B_LM, static_cast<const char*>(a.LMH) + ti * tile_bytes, tile_bytes, bar);
+                bulk_load(isc, a.SPS + ti * 64, 256, bar);
+                bulk_load(isc + 64, a.LMS + ti * 64, 256, bar);
             }
             // x, X', g, G'': 64 rows x 8 chunks of 8 channels, four chunks per thread (rows lt / 8 + 16 m),
             // all loads first
@@ -364,7 +313,18 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                     for (int q = 0; q < 8; ++q) xv[m][q] = gv[m][q] = zv[m][q] = 0.f;
                 }
             }
-            const float inv_sp = 1.f / sc[0], inv_lm = 1.f / sc[1];  // exact: powers of two
+            float range = 0.f;  // largest magnitude written to an fp16 tile
+            if (!wait_all(&bars[SPLM_FULL0 + buf], (k >> 1) & 1, abort)) {
+                give_up(abort);
+                break;
+            }
+            // X' takes Lm's inverse row scales and G'' Sp's (column p of X', G'' meets row p of Lm, Sp)
+            float il[8], is[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                is[q] = isc[8 * k8 + q];
+                il[q] = isc[64 + 8 * k8 + q];
+            }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int r = (lt >> 3) + 16 * m;
@@ -374,17 +334,13 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 const uint32_t off = sw128_off(r, k8);
                 *reinterpret_cast<uint4*>(bo + B_X + off) = pack8(xv[m], 1.f, range);
                 *reinterpret_cast<uint4*>(bo + B_XP + off) =
-                    pack8(xv[m], on ? dtr[m] * expf(cs_last - csr[m]) * inv_lm : 0.f, range);
+                    pack8s(xv[m], il, on ? dtr[m] * expf(cs_last - csr[m]) : 0.f, range);
                 *reinterpret_cast<uint4*>(bo + B_G + off) = pack8(gv[m], 1.f, range);
-                *reinterpret_cast<uint4*>(bo + B_GP + off) = pack8(gv[m], on ? expf(csr[m]) * inv_sp : 0.f, range);
+                *reinterpret_cast<uint4*>(bo + B_GP + off) = pack8s(gv[m], is, on ? expf(csr[m]) : 0.f, range);
                 if (k8 == 0) {
                     vec[(V_DT >> 2) + buf * 64 + r] = dtr[m];
                     vec[(V_CS >> 2) + buf * 64 + r] = csr[m];
                 }
-            }
-            if (lt == 0) {
-                vec[(V_SC >> 2) + buf * 2] = sc[0];
-                vec[(V_SC >> 2) + buf * 2 + 1] = sc[1];
             }
             if (!(range < 65504.f)) atomicOr(&g_chunk_bwd_tc_error, 2);
             fence_async_smem();
@@ -401,7 +357,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
         if (warp == 0) {
             if (lane == 0) mma_steps(tmem + COL_CB, kdesc(sm + OFF_TC), false, kdesc(sm + OFF_TB), false, ID_KK, 4 * nbox,
                                      false);
-            ok = wait_all(&bars[TILE_FULL0], 0, abort);
+            ok = wait_all(&bars[TILE_FULL0], 0, abort) && wait_all(&bars[SPLM_FULL0], 0, abort);
             if (ok) {
                 tc_fence_after();
                 if (lane == 0) issue_batch1(sm, tmem, 0, nbox, &bars[B1_DONE]);
@@ -447,7 +403,9 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             const float* css = vec + (V_CS >> 2) + buf * 64;
             const float cs_r = css[r], dt_r = dts[r], cs_last = css[Qv - 1];
             // the loader's scales of Sp and Lm: SPC and LMB come out of TMEM multiplied by them
-            const float usp = 1.f / vec[(V_SC >> 2) + buf * 2], ulm = 1.f / vec[(V_SC >> 2) + buf * 2 + 1];
+            // the inverse row scales of this head's Sp, Lm tiles: SPC and LMB column p come out of TMEM times s_p
+            const float* isp = vec + (V_ISC >> 2) + buf * 128 + c0;
+            const float* ilm = isp + 64;
             // phase B: LCB and LGX' rows, the row sums of M and the column sums of GX L CB
             float rowm = 0.f, range = 0.f;
             {
@@ -495,10 +453,10 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 float e = 0.f;
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    e += gr[q] * spc[q];
+                    e += gr[q] * spc[q] * isp[q];
                     pd += gr[q] * xr[q];
                 }
-                vec[(V_E >> 2) + (par * 2 + ch) * 64 + r] = e * usp;
+                vec[(V_E >> 2) + (par * 2 + ch) * 64 + r] = e;
             }
             if (warp == 0) {
                 if (!wait_all(&bars[LT_FULL], par, abort)) {
@@ -516,21 +474,22 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             tc_fence_after();
             // phase C: dz from the recomputed y; dx; W
             const float ex_r = r < Qv ? expf(cs_r) : 0.f, el_r = r < Qv ? expf(cs_last - cs_r) : 0.f;
-            const float exu = ex_r * usp;
             {
                 float yin[32], spc[32];
                 tmem_ld32(tmem + lb + COL_YIN + c0, yin);
                 tmem_ld32(tmem + lb + COL_SPC + c0, spc);
                 tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) spc[q] *= ex_r * isp[q];
                 if (r < Qv) {
                     float* dz = a.dz + (row0 + r) * HP + (int64_t)h * kPb + c0;
 #pragma unroll
                     for (int q = 0; q < 32; q += 4) {
                         float4 o;
-                        o.x = dyds[q] * (yin[q] + exu * spc[q] + Dh * xr[q]);
-                        o.y = dyds[q + 1] * (yin[q + 1] + exu * spc[q + 1] + Dh * xr[q + 1]);
-                        o.z = dyds[q + 2] * (yin[q + 2] + exu * spc[q + 2] + Dh * xr[q + 2]);
-                        o.w = dyds[q + 3] * (yin[q + 3] + exu * spc[q + 3] + Dh * xr[q + 3]);
+                        o.x = dyds[q] * (yin[q] + spc[q] + Dh * xr[q]);
+                        o.y = dyds[q + 1] * (yin[q + 1] + spc[q + 1] + Dh * xr[q + 1]);
+                        o.z = dyds[q + 2] * (yin[q + 2] + spc[q + 2] + Dh * xr[q + 2]);
+                        o.w = dyds[q + 3] * (yin[q + 3] + spc[q + 3] + Dh * xr[q + 3]);
                         *reinterpret_cast<float4*>(dz + q) = o;
                     }
                 }
@@ -541,7 +500,9 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 tmem_ld32(tmem + lb + COL_LMB + c0, lmb);
                 tmem_ld32(tmem + lb + COL_DXI + c0, dxi);
                 tmem_wait_ld();
-                const float f = dt_r * el_r * ulm;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) lmb[q] *= ilm[q];
+                const float f = dt_r * el_r;
                 float* du = a.DU + (row0 + r) * conv_dim + (int64_t)h * kPb + c0;
 #pragma unroll
                 for (int q = 0; q < 32; q += 4) {
@@ -558,7 +519,8 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             mbar_arrive(&bars[ACC_FREE]);
             if (warp == 0 && k + 1 < nh) {
                 if (!wait_all(&bars[ACC_FREE], par, abort) ||
-                    !wait_all(&bars[TILE_FULL0 + (buf ^ 1)], ((k + 1) >> 1) & 1, abort)) {
+                    !wait_all(&bars[TILE_FULL0 + (buf ^ 1)], ((k + 1) >> 1) & 1, abort) ||
+                    !wait_all(&bars[SPLM_FULL0 + (buf ^ 1)], ((k + 1) >> 1) & 1, abort)) {
                     ok = false;
                     break;
                 }
@@ -566,7 +528,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 if (lane == 0) issue_batch1(sm, tmem, k + 1, nbox, &bars[B1_DONE]);
                 __syncwarp();
             }
-            vec[(V_W >> 2) + (par * 2 + ch) * 64 + r] = el_r * ulm * wpart;
+            vec[(V_W >> 2) + (par * 2 + ch) * 64 + r] = el_r * wpart;
             pd = warp_sum(pd);
             if (lane == 0) vec[(V_PD >> 2) + par * 4 + wi] = pd;
             mbar_arrive(&bars[WSYNC]);
