@@ -20,23 +20,29 @@
 // (the same quantities, in the same fp32 epilogue arithmetic, as the CUDA-core chunk kernel of
 // ssd_backward.cu; there R comes from explicit prefix sums of M).
 //
-// One CTA per (chunk, group, half of the group's heads), heads in turn; 256 threads in two roles:
+// Operands are fp16 (11-bit significand; bf16's 8 bits lose too much in the sums behind ddt).  The
+// entering states and leaving adjoints arrive as the state pass's fp16 tiles, row p scaled by a power of
+// two s_p <= 1 that keeps it below 2^14; SPC and LMB column p are multiplied back by 1/s_p, and the
+// partners of the head-summed products (X', G'') take 1/s_p on their column p.  Any other value fp16
+// cannot hold (>= 65504) sets bit 1 of this file's error word (SSD_ERR_RANGE).  The elementwise terms
+// read x, g and dy silu'(z) back from the same fp16 tiles the MMAs use.
+//
+// One CTA per (chunk, group, half of the group's heads), heads in turn; 288 threads in three roles:
 //   row warps 0, 1, 4, 5  (TMEM lanes 0..63 = the chunk's tokens; warps 0/4 tokens 0..31, 1/5 tokens
 //                         32..63; warps 0, 1 columns 0..31, warps 4, 5 columns 32..63): the elementwise
-//                         work above, the LCB / LGX' tiles, dz, dx and the per-head scalars; lane 0 of
-//                         warp 0 also allocates TMEM (the whole warp) and issues the MMAs, at the points
-//                         where warp 0 waits for their operands anyway;
-//   loader warps 2, 3, 6, 7: the head's operand tiles (x, X', g, G'', Sp, Lm) as bf16 in 128-byte-swizzled
-//                         shared memory, two heads deep.
-// Every MMA is M = 128, N = 64 with bf16 operands and fp32 accumulators in TMEM (512 columns: CB, GX,
-// SPC, LMB, YIN, DXI, dB^T, dC^T).  The token-major products use only rows 0..63 of their 128-row
-// result: the A tile's rows 64..127 are whatever follows it in shared memory (always in bounds), and the
-// result lanes 64..127 are never read.  dB^T and dC^T have the state index n as M (rows past N unused).
+//                         work above, the LCB / LGX' tiles, dz, dx; warp 0 also the per-head scalars
+//                         (ddt and the partial sums);
+//   loader warps 2, 3, 6, 7: the head's tiles, two heads deep: Sp and Lm by bulk copy, x, X', g, G'' and
+//                         dy silu'(z) converted from global memory;
+//   warp 8              : TMEM allocation and, on one thread, the MMAs.
+// Every MMA is M = 128, N = 64 with fp32 accumulators in TMEM (512 columns: CB, GX, SPC, LMB, YIN, DXI,
+// dB^T, dC^T).  The token-major products use only rows 0..63 of their 128-row result: the A tile's rows
+// 64..127 are whatever follows it in shared memory (always in bounds), and the result lanes 64..127 are
+// never read.  dB^T and dC^T have the state index n as M (rows past N unused).
 // All waits are bounded mbarrier waits that also watch a shared abort word; a wait that gives up sets
-// this file's error word (reported by ssd_device_status), and the CTA leaves without
-// writing its dB / dC.  No atomics: every sum runs in a fixed order (deterministic).
+// bit 0 of the error word (SSD_ERR_TIMEOUT from ssd_device_status), and the CTA leaves without writing
+// its dB / dC.  No atomics on results: every sum runs in a fixed order (deterministic).
 #include <cuda.h>
-#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -54,22 +60,23 @@ using namespace sm100;
 
 constexpr int kQb = 64;   // chunk (tokens)
 constexpr int kPb = 64;   // head dimension
-constexpr int kThreadsB = 256;
+constexpr int kThreadsB = 288;
 
-// shared memory (bytes from a 1024-byte aligned base).  A "box" is [64 rows][64 bf16] with 128-byte rows
+// shared memory (bytes from a 1024-byte aligned base).  A "box" is [64 rows][64 fp16] with 128-byte rows
 // and the 128-byte swizzle (8 KB); an N-wide tile is one box per 64 state columns.
 constexpr uint32_t OFF_TC = 0;          // C [i][n], two boxes
 constexpr uint32_t OFF_TB = 16384;      // B [j][n], two boxes
 constexpr uint32_t OFF_LCB = 32768;     // LCB [i][j]
 constexpr uint32_t OFF_LGX = 40960;     // LGX' [i][j]
 constexpr uint32_t OFF_BUF = 49152;     // two per-head buffers of BUF_BYTES:
-constexpr uint32_t B_SP = 0;            //   Sp [p][n], two boxes
-constexpr uint32_t B_LM = 16384;        //   Lm [p][n], two boxes
+constexpr uint32_t B_SP = 0;            //   s Sp [p][n], two boxes
+constexpr uint32_t B_LM = 16384;        //   s Lm [p][n], two boxes
 constexpr uint32_t B_X = 32768;         //   x [j][p]
 constexpr uint32_t B_XP = 40960;        //   X' [j][p]
 constexpr uint32_t B_G = 49152;         //   g [i][p]
 constexpr uint32_t B_GP = 57344;        //   G'' [i][p]
-constexpr uint32_t BUF_BYTES = 65536;
+constexpr uint32_t B_DS = 65536;        //   dy silu'(z) [i][p]
+constexpr uint32_t BUF_BYTES = 73728;
 constexpr uint32_t OFF_VEC = OFF_BUF + 2 * BUF_BYTES;  // fp32 vectors:
 constexpr uint32_t V_DT = 0;            //   dt [2 buffers][64]
 constexpr uint32_t V_CS = 512;          //   cs [2][64]
@@ -81,8 +88,8 @@ constexpr uint32_t V_PD = 5120;         //   sum g . x per row warp [2][4]
 constexpr uint32_t V_ISC = 5248;        //   inverse row scales of each buffer's Sp, Lm tiles [2][2][64]
 constexpr uint32_t VEC_BYTES = 6272;
 constexpr uint32_t OFF_BAR = OFF_VEC + VEC_BYTES;
-enum : int { TILE_FULL0, TILE_FULL1, TILE_FREE0, TILE_FREE1, B1_DONE, LT_FULL, B2_DONE, ACC_FREE, WSYNC, FINAL,
-             SPLM_FULL0, SPLM_FULL1, NBAR };
+enum : int { TILE_FULL0, TILE_FULL1, TILE_FREE0, TILE_FREE1, SPLM_FULL0, SPLM_FULL1, GX_DONE, B1_DONE, LT_FULL,
+             B2_DONE, ACC_FREE, WSYNC, FINAL, NBAR };
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // abort word, TMEM base
 constexpr uint32_t SMEM_B = OFF_MISC + 16 + 1024;  // + alignment slack
 
@@ -90,7 +97,6 @@ constexpr uint32_t SMEM_B = OFF_MISC + 16 + 1024;  // + alignment slack
 constexpr uint32_t COL_CB = 0, COL_GX = 64, COL_SPC = 128, COL_LMB = 192, COL_YIN = 256, COL_DXI = 320,
                    COL_DB = 384, COL_DC = 448, TMEM_COLS_B = 512;
 
-// The MMA operands are fp16 (11-bit significand): bf16's 8 bits lose too much in the sums behind ddt.
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -126,12 +132,24 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8], float s, float& rang
     }
     return make_uint4(pack_h2(w[0], w[1]), pack_h2(w[2], w[3]), pack_h2(w[4], w[5]), pack_h2(w[6], w[7]));
 }
-// Eight values v[q] f[q] s as fp16 (the per-column inverse state scales f), tracking `range` likewise.
-__device__ __forceinline__ uint4 pack8s(const float (&v)[8], const float (&f)[8], float s, float& range) {
+// Eight values v[q] f[q] s as fp16 (f: the per-column inverse state scales, in shared memory), tracking
+// `range` likewise.
+__device__ __forceinline__ uint4 pack8s(const float (&v)[8], const float* f, float s, float& range) {
     float w[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) w[q] = v[q] * f[q];
     return pack8(w, s, range);
+}
+// The eight fp16 values of 16-byte chunk `chunk` of row r of a swizzled tile, as fp32.
+__device__ __forceinline__ void unpack8(const uint8_t* tile, int r, int chunk, float (&v)[8]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + sw128_off(r, chunk));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
 }
 
 // D (+)= A B over K = 16 * steps; a K-major operand steps 32 bytes inside a box and 8 KB from box to box,
@@ -152,26 +170,29 @@ constexpr uint32_t ID_MM = idesc_f16_f32(128, 64, true, true);
 __device__ __forceinline__ uint64_t kdesc(const uint8_t* p) { return sw128_desc(smem_u32(p), 16, 1024); }
 __device__ __forceinline__ uint64_t mdesc(const uint8_t* p) { return sw128_desc(smem_u32(p), 8192, 1024); }
 
-// The first MMAs of head k (operands: the head's buffer and C, B): GX, SPC, LMB and the Sp / Lm parts of
-// dB^T, dC^T (which the first head starts).
-__device__ __forceinline__ void issue_batch1(const uint8_t* sm, uint32_t tmem, int k, int nbox, uint64_t* done) {
+// The first MMAs of head k (operands: the head's buffer and C, B): GX first (the row warps start on it), then
+// SPC, LMB and the Sp / Lm parts of dB^T, dC^T (which the first head starts).
+__device__ __forceinline__ void issue_batch1(const uint8_t* sm, uint32_t tmem, int k, int nbox, uint64_t* gx_done,
+                                             uint64_t* done) {
     const uint8_t* bo = sm + OFF_BUF + (k & 1) * BUF_BYTES;
     mma_steps(tmem + COL_GX, kdesc(bo + B_G), false, kdesc(bo + B_X), false, ID_KK, 4, false);
+    mma_commit(gx_done);
     mma_steps(tmem + COL_SPC, kdesc(sm + OFF_TC), false, kdesc(bo + B_SP), false, ID_KK, 4 * nbox, false);
     mma_steps(tmem + COL_LMB, kdesc(sm + OFF_TB), false, kdesc(bo + B_LM), false, ID_KK, 4 * nbox, false);
     mma_steps(tmem + COL_DB, mdesc(bo + B_LM), true, kdesc(bo + B_XP), false, ID_MK, 4, k > 0);
     mma_steps(tmem + COL_DC, mdesc(bo + B_SP), true, kdesc(bo + B_GP), false, ID_MK, 4, k > 0);
     mma_commit(done);
 }
-// The MMAs that need the row warps' LCB / LGX' tiles: YIN, DXI and the intra-chunk parts of dB^T, dC^T.
+// The MMAs that need the row warps' LCB / LGX' tiles: YIN, DXI (then `done`), and the intra-chunk parts of
+// dB^T, dC^T (then `free_buf`: the head's buffer and the LCB / LGX' tiles are free).
 __device__ __forceinline__ void issue_batch2(const uint8_t* sm, uint32_t tmem, int k, uint64_t* done,
                                              uint64_t* free_buf) {
     const uint8_t* bo = sm + OFF_BUF + (k & 1) * BUF_BYTES;
     mma_steps(tmem + COL_YIN, kdesc(sm + OFF_LCB), false, mdesc(bo + B_X), true, ID_KM, 4, false);
     mma_steps(tmem + COL_DXI, mdesc(sm + OFF_LCB), true, mdesc(bo + B_G), true, ID_MM, 4, false);
+    mma_commit(done);
     mma_steps(tmem + COL_DB, mdesc(sm + OFF_TC), true, mdesc(sm + OFF_LGX), true, ID_MM, 4, true);
     mma_steps(tmem + COL_DC, mdesc(sm + OFF_TB), true, kdesc(sm + OFF_LGX), false, ID_MK, 4, true);
-    mma_commit(done);
     mma_commit(free_buf);
 }
 
@@ -206,6 +227,22 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Exclusive prefix sums over the 64 tokens held two per lane (token lane and lane + 32).
+__device__ __forceinline__ void scan_excl(const float (&v)[2], float (&out)[2], int lane) {
+    float s0 = v[0], s1 = v[1];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float t0 = __shfl_up_sync(0xffffffffu, s0, o), t1 = __shfl_up_sync(0xffffffffu, s1, o);
+        if (lane >= o) {
+            s0 += t0;
+            s1 += t1;
+        }
+    }
+    const float tot0 = __shfl_sync(0xffffffffu, s0, 31);
+    out[0] = s0 - v[0];
+    out[1] = tot0 + s1 - v[1];
+}
+
 // grid (nchunks, G * split, batch), kThreadsB threads, SMEM_B bytes of dynamic shared memory
 __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkBwdTcArgs a) {
     extern __shared__ uint8_t smem_b[];
@@ -224,7 +261,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
     const int64_t HP = (int64_t)a.H * kPb, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
     const int64_t row0 = b * a.L + t0;  // first token row of the chunk
 
-    if (warp == 0) {
+    if (warp == 8) {
         tmem_alloc(tm_holder, TMEM_COLS_B);
         tmem_relinquish();
     }
@@ -234,14 +271,15 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
         mbar_init(&bars[TILE_FULL1], 128);
         mbar_init(&bars[TILE_FREE0], 129);  // the MMAs' commit + the 128 row threads
         mbar_init(&bars[TILE_FREE1], 129);
+        mbar_init(&bars[SPLM_FULL0], 1);    // the bulk copies' transaction bytes
+        mbar_init(&bars[SPLM_FULL1], 1);
+        mbar_init(&bars[GX_DONE], 1);
         mbar_init(&bars[B1_DONE], 1);
         mbar_init(&bars[LT_FULL], 128);
         mbar_init(&bars[B2_DONE], 1);
         mbar_init(&bars[ACC_FREE], 128);
         mbar_init(&bars[WSYNC], 128);
         mbar_init(&bars[FINAL], 1);
-        mbar_init(&bars[SPLM_FULL0], 1);  // the bulk copies' transaction bytes
-        mbar_init(&bars[SPLM_FULL1], 1);
         fence_mbar_init();
     }
     // the group's post-conv B and C (rows past Qv zero): 64 rows x N/8 chunks of 8 channels
@@ -267,9 +305,32 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
     tc_fence_after();
     const uint32_t tmem = *tm_holder;
 
-    if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
+    if (warp == 8) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            mma_steps(tmem + COL_CB, kdesc(sm + OFF_TC), false, kdesc(sm + OFF_TB), false, ID_KK, 4 * nbox, false);
+            bool ok = true;
+            for (int k = 0; k < nh && ok; ++k) {
+                const int buf = k & 1;
+                ok = mbar_wait(&bars[TILE_FULL0 + buf], (k >> 1) & 1, abort) &&
+                     mbar_wait(&bars[SPLM_FULL0 + buf], (k >> 1) & 1, abort) &&
+                     (k == 0 || mbar_wait(&bars[ACC_FREE], (k - 1) & 1, abort));
+                if (!ok) break;
+                tc_fence_after();
+                issue_batch1(sm, tmem, k, nbox, &bars[GX_DONE], &bars[B1_DONE]);
+                ok = mbar_wait(&bars[LT_FULL], k & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                issue_batch2(sm, tmem, k, &bars[B2_DONE], &bars[TILE_FREE0 + buf]);
+            }
+            if (!ok) give_up(abort);
+            mma_commit(&bars[FINAL]);  // every MMA issued so far
+        }
+        __syncwarp();
+    } else if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
         // ---------------- loaders ----------------
         const int lt = ((warp & 3) - 2 + 2 * (warp >> 2)) * 32 + lane;  // 0..127
+        const int k8 = lt & 7;  // this thread's 16-byte chunk (8 head channels) of rows lt / 8 + 16 m
         for (int k = 0; k < nh; ++k) {
             const int buf = k & 1;
             if (k >= 2 && !wait_all(&bars[TILE_FREE0 + buf], ((k >> 1) - 1) & 1, abort)) {
@@ -279,8 +340,8 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             uint8_t* bo = sm + OFF_BUF + buf * BUF_BYTES;
             const int h = g * hpg + hl0 + k;
             const int64_t hrow = (b * a.H + h) * a.L + t0;
-            // Sp and Lm: the state pass's fp16 tiles (each row p scaled by s_p) and their inverse row scales,
-            // four bulk copies onto this buffer's barrier
+            // Sp and Lm: the state pass's fp16 tiles and their inverse row scales, four bulk copies onto this
+            // buffer's barrier
             const int64_t ti = (b * nc + c) * a.H + h;
             const uint32_t tile_bytes = 8192u * (uint32_t)nbox;
             float* isc = vec + (V_ISC >> 2) + buf * 128;  // 1/s_p of Sp [64], then of Lm [64]
@@ -292,10 +353,8 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 bulk_load(isc, a.SPS + ti * 64, 256, bar);
                 bulk_load(isc + 64, a.LMS + ti * 64, 256, bar);
             }
-            // x, X', g, G'': 64 rows x 8 chunks of 8 channels, four chunks per thread (rows lt / 8 + 16 m),
-            // all loads first
+            // x, X', g, G'', dy silu'(z): 64 rows x 8 chunks of 8 channels, four chunks per thread, all loads first
             const float cs_last = a.CS[hrow + Qv - 1];
-            const int k8 = lt & 7;
             float xv[4][8], gv[4][8], zv[4][8], dtr[4], csr[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -319,24 +378,26 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 break;
             }
             // X' takes Lm's inverse row scales and G'' Sp's (column p of X', G'' meets row p of Lm, Sp)
-            float il[8], is[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                is[q] = isc[8 * k8 + q];
-                il[q] = isc[64 + 8 * k8 + q];
-            }
+            const float* is = isc + 8 * k8;
+            const float* il = isc + 64 + 8 * k8;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int r = (lt >> 3) + 16 * m;
+                float ds[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) gv[m][q] = gv[m][q] * zv[m][q] * sigm(zv[m][q]);
+                for (int q = 0; q < 8; ++q) {
+                    const float zq = zv[m][q], s = __fdividef(1.f, 1.f + __expf(-zq)), dy = gv[m][q];
+                    gv[m][q] = dy * zq * s;                       // g = dy silu(z)
+                    ds[q] = dy * s * (1.f + zq * (1.f - s));      // dy silu'(z)
+                }
                 const bool on = r < Qv;
                 const uint32_t off = sw128_off(r, k8);
                 *reinterpret_cast<uint4*>(bo + B_X + off) = pack8(xv[m], 1.f, range);
                 *reinterpret_cast<uint4*>(bo + B_XP + off) =
-                    pack8s(xv[m], il, on ? dtr[m] * expf(cs_last - csr[m]) : 0.f, range);
+                    pack8s(xv[m], il, on ? dtr[m] * __expf(cs_last - csr[m]) : 0.f, range);
                 *reinterpret_cast<uint4*>(bo + B_G + off) = pack8(gv[m], 1.f, range);
-                *reinterpret_cast<uint4*>(bo + B_GP + off) = pack8s(gv[m], is, on ? expf(csr[m]) : 0.f, range);
+                *reinterpret_cast<uint4*>(bo + B_GP + off) = pack8s(gv[m], is, on ? __expf(csr[m]) : 0.f, range);
+                *reinterpret_cast<uint4*>(bo + B_DS + off) = pack8(ds, 1.f, range);
                 if (k8 == 0) {
                     vec[(V_DT >> 2) + buf * 64 + r] = dtr[m];
                     vec[(V_CS >> 2) + buf * 64 + r] = csr[m];
@@ -354,55 +415,37 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
         const int wi = rq + 2 * ch;        // 0..3
         const uint32_t lb = (uint32_t)(32 * rq) << 16;
         bool ok = true;
-        if (warp == 0) {
-            if (lane == 0) mma_steps(tmem + COL_CB, kdesc(sm + OFF_TC), false, kdesc(sm + OFF_TB), false, ID_KK, 4 * nbox,
-                                     false);
-            ok = wait_all(&bars[TILE_FULL0], 0, abort) && wait_all(&bars[SPLM_FULL0], 0, abort);
-            if (ok) {
-                tc_fence_after();
-                if (lane == 0) issue_batch1(sm, tmem, 0, nbox, &bars[B1_DONE]);
-                __syncwarp();
-            }
-        }
         for (int k = 0; k < nh && ok; ++k) {
             const int buf = k & 1, par = k & 1;
             const int h = g * hpg + hl0 + k;
             const float Dh = a.D[h];
-            // this row's fp32 x, g and dy silu'(z) over the thread's 32 columns (zero past Qv)
-            float xr[32], gr[32], dyds[32];
-            {
-                const int64_t xi = (row0 + r) * conv_dim + (int64_t)h * kPb + c0;
-                const int64_t yi = (row0 + r) * HP + (int64_t)h * kPb + c0;
+            // warp 0's per-head scalars from global memory, ahead of the waits: F, the raw dt of its two
+            // tokens, A, dt_bias
+            float F = 0.f, raw[2] = {0.f, 0.f}, Ah = 0.f, bias = 0.f;
+            if (warp == 0) {
+                for (int s = 0; s < a.nsplit_pf; ++s) F += a.PF[((b * nc + c) * a.H + h) * a.nsplit_pf + s];
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float xv[8], dy[8], zv[8];
-                    if (r < Qv) {
-                        load8(a.U, xi + 8 * q8, false, xv);
-                        load8(a.dy, yi + 8 * q8, a.dy_bf16, dy);
-                        load8(a.z, yi + 8 * q8, a.act_bf16, zv);
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) xv[q] = dy[q] = zv[q] = 0.f;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float s = sigm(zv[q]);
-                        xr[8 * q8 + q] = xv[q];
-                        gr[8 * q8 + q] = dy[q] * zv[q] * s;
-                        dyds[8 * q8 + q] = dy[q] * s * (1.f + zv[q] * (1.f - s));
+                for (int u = 0; u < 2; ++u) {
+                    const int kk = lane + 32 * u;
+                    if (kk < Qv) {
+                        const int64_t di = (row0 + kk) * a.H + h;
+                        raw[u] = a.act_bf16 ? bf_lo(static_cast<const unsigned short*>(a.dt)[di])
+                                            : static_cast<const float*>(a.dt)[di];
                     }
                 }
+                Ah = a.A[h];
+                bias = a.dt_bias[h];
             }
-            // the loader's dt / cs of this head (TILE_FULL), then the first MMAs (B1_DONE)
-            if (!wait_all(&bars[TILE_FULL0 + buf], (k >> 1) & 1, abort) || !wait_all(&bars[B1_DONE], par, abort)) {
+            // the head's tiles (TILE_FULL), then GX (GX_DONE)
+            if (!wait_all(&bars[TILE_FULL0 + buf], (k >> 1) & 1, abort) || !wait_all(&bars[GX_DONE], par, abort)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            const uint8_t* bo = sm + OFF_BUF + buf * BUF_BYTES;
             const float* dts = vec + (V_DT >> 2) + buf * 64;
             const float* css = vec + (V_CS >> 2) + buf * 64;
             const float cs_r = css[r], dt_r = dts[r], cs_last = css[Qv - 1];
-            // the loader's scales of Sp and Lm: SPC and LMB come out of TMEM multiplied by them
             // the inverse row scales of this head's Sp, Lm tiles: SPC and LMB column p come out of TMEM times s_p
             const float* isp = vec + (V_ISC >> 2) + buf * 128 + c0;
             const float* ilm = isp + 64;
@@ -423,7 +466,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                         for (int u = 0; u < 2; ++u) {
                             const int q = 8 * q8 + 2 * w2 + u, j = c0 + q;
                             const bool on = j <= r && r < Qv;
-                            const float L = on ? expf(cs_r - css[j]) : 0.f;
+                            const float L = on ? __expf(cs_r - css[j]) : 0.f;
                             const float lgx = gx[q] * L, dtj = dts[j];
                             lc[u] = cb[q] * L * dtj;
                             lg[u] = lgx * dtj;
@@ -445,6 +488,12 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 vec[(V_COL >> 2) + (par * 2 + rq) * 64 + c0 + lane] = col;
             }
             vec[(V_ROWM >> 2) + (par * 2 + ch) * 64 + r] = rowm;
+            // E partial (g . SPC) and sum g . x over this thread's columns, once SPC is there (B1_DONE)
+            if (!wait_all(&bars[B1_DONE], par, abort)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
             float pd = 0.f;
             {
                 float spc[32];
@@ -452,20 +501,17 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 tmem_wait_ld();
                 float e = 0.f;
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    e += gr[q] * spc[q] * isp[q];
-                    pd += gr[q] * xr[q];
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float gq[8], xq[8];
+                    unpack8(bo + B_G, r, 4 * ch + q8, gq);
+                    unpack8(bo + B_X, r, 4 * ch + q8, xq);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        e += gq[q] * spc[8 * q8 + q] * isp[8 * q8 + q];
+                        pd += gq[q] * xq[q];
+                    }
                 }
                 vec[(V_E >> 2) + (par * 2 + ch) * 64 + r] = e;
-            }
-            if (warp == 0) {
-                if (!wait_all(&bars[LT_FULL], par, abort)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) issue_batch2(sm, tmem, k, &bars[B2_DONE], &bars[TILE_FREE0 + buf]);
-                __syncwarp();
             }
             if (!wait_all(&bars[B2_DONE], par, abort)) {
                 ok = false;
@@ -479,18 +525,20 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 tmem_ld32(tmem + lb + COL_YIN + c0, yin);
                 tmem_ld32(tmem + lb + COL_SPC + c0, spc);
                 tmem_wait_ld();
+                float* dz = a.dz + (row0 + r) * HP + (int64_t)h * kPb + c0;
 #pragma unroll
-                for (int q = 0; q < 32; ++q) spc[q] *= ex_r * isp[q];
-                if (r < Qv) {
-                    float* dz = a.dz + (row0 + r) * HP + (int64_t)h * kPb + c0;
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float xq[8], dq[8], o[8];
+                    unpack8(bo + B_X, r, 4 * ch + q8, xq);
+                    unpack8(bo + B_DS, r, 4 * ch + q8, dq);
 #pragma unroll
-                    for (int q = 0; q < 32; q += 4) {
-                        float4 o;
-                        o.x = dyds[q] * (yin[q] + spc[q] + Dh * xr[q]);
-                        o.y = dyds[q + 1] * (yin[q + 1] + spc[q + 1] + Dh * xr[q + 1]);
-                        o.z = dyds[q + 2] * (yin[q + 2] + spc[q + 2] + Dh * xr[q + 2]);
-                        o.w = dyds[q + 3] * (yin[q + 3] + spc[q + 3] + Dh * xr[q + 3]);
-                        *reinterpret_cast<float4*>(dz + q) = o;
+                    for (int q = 0; q < 8; ++q) {
+                        const int qq = 8 * q8 + q;
+                        o[q] = dq[q] * (yin[qq] + ex_r * isp[qq] * spc[qq] + Dh * xq[q]);
+                    }
+                    if (r < Qv) {
+                        *reinterpret_cast<float4*>(dz + 8 * q8) = make_float4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<float4*>(dz + 8 * q8 + 4) = make_float4(o[4], o[5], o[6], o[7]);
                     }
                 }
             }
@@ -500,33 +548,27 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 tmem_ld32(tmem + lb + COL_LMB + c0, lmb);
                 tmem_ld32(tmem + lb + COL_DXI + c0, dxi);
                 tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) lmb[q] *= ilm[q];
+                tc_fence_before();
+                mbar_arrive(&bars[ACC_FREE]);  // the head's last TMEM read: the next head's MMAs may start
                 const float f = dt_r * el_r;
                 float* du = a.DU + (row0 + r) * conv_dim + (int64_t)h * kPb + c0;
 #pragma unroll
-                for (int q = 0; q < 32; q += 4) {
-                    float4 o;
-                    o.x = dxi[q] + f * lmb[q] + Dh * gr[q];
-                    o.y = dxi[q + 1] + f * lmb[q + 1] + Dh * gr[q + 1];
-                    o.z = dxi[q + 2] + f * lmb[q + 2] + Dh * gr[q + 2];
-                    o.w = dxi[q + 3] + f * lmb[q + 3] + Dh * gr[q + 3];
-                    if (r < Qv) *reinterpret_cast<float4*>(du + q) = o;
-                    wpart += xr[q] * lmb[q] + xr[q + 1] * lmb[q + 1] + xr[q + 2] * lmb[q + 2] + xr[q + 3] * lmb[q + 3];
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float xq[8], gq[8], o[8];
+                    unpack8(bo + B_X, r, 4 * ch + q8, xq);
+                    unpack8(bo + B_G, r, 4 * ch + q8, gq);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int qq = 8 * q8 + q;
+                        const float lm = lmb[qq] * ilm[qq];
+                        o[q] = dxi[qq] + f * lm + Dh * gq[q];
+                        wpart += xq[q] * lm;
+                    }
+                    if (r < Qv) {
+                        *reinterpret_cast<float4*>(du + 8 * q8) = make_float4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<float4*>(du + 8 * q8 + 4) = make_float4(o[4], o[5], o[6], o[7]);
+                    }
                 }
-            }
-            tc_fence_before();
-            mbar_arrive(&bars[ACC_FREE]);
-            if (warp == 0 && k + 1 < nh) {
-                if (!wait_all(&bars[ACC_FREE], par, abort) ||
-                    !wait_all(&bars[TILE_FULL0 + (buf ^ 1)], ((k + 1) >> 1) & 1, abort) ||
-                    !wait_all(&bars[SPLM_FULL0 + (buf ^ 1)], ((k + 1) >> 1) & 1, abort)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) issue_batch1(sm, tmem, k + 1, nbox, &bars[B1_DONE]);
-                __syncwarp();
             }
             vec[(V_W >> 2) + (par * 2 + ch) * 64 + r] = el_r * wpart;
             pd = warp_sum(pd);
@@ -542,7 +584,6 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 const float* rwm = vec + (V_ROWM >> 2) + par * 128;
                 const float* ev = vec + (V_E >> 2) + par * 128;
                 const float* wv = vec + (V_W >> 2) + par * 128;
-                const float Ah = a.A[h], bias = a.dt_bias[h];
                 float dr0[2], dtk[2], d[2], e[2], w[2], dw[2];
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
@@ -555,35 +596,13 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                     dw[u] = dtk[u] * w[u];
                 }
                 // exclusive prefix sums of d and dt W, inclusive suffix sums of E, over the 64 tokens
-                auto scan_excl = [&](const float (&v)[2], float (&out)[2]) {
-                    float s0 = v[0];
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float t = __shfl_up_sync(0xffffffffu, s0, o);
-                        if (lane >= o) s0 += t;
-                    }
-                    const float tot0 = __shfl_sync(0xffffffffu, s0, 31);
-                    float s1 = v[1];
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float t = __shfl_up_sync(0xffffffffu, s1, o);
-                        if (lane >= o) s1 += t;
-                    }
-                    out[0] = s0 - v[0];
-                    out[1] = tot0 + s1 - v[1];
-                };
-                float R[2], Wp[2], Es[2];
-                scan_excl(d, R);
-                scan_excl(dw, Wp);
-                {
-                    float ex_[2];
-                    scan_excl(e, ex_);
-                    const float etot = __shfl_sync(0xffffffffu, ex_[1] + e[1], 31);
-                    Es[0] = etot - ex_[0];
-                    Es[1] = etot - ex_[1];
-                }
-                float F = 0.f;
-                for (int s = 0; s < a.nsplit_pf; ++s) F += a.PF[((b * nc + c) * a.H + h) * a.nsplit_pf + s];
+                float R[2], Wp[2], Ex[2], Es[2];
+                scan_excl(d, R, lane);
+                scan_excl(dw, Wp, lane);
+                scan_excl(e, Ex, lane);
+                const float etot = __shfl_sync(0xffffffffu, Ex[1] + e[1], 31);
+                Es[0] = etot - Ex[0];
+                Es[1] = etot - Ex[1];
                 float pdA = 0.f, pbias = 0.f;
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
@@ -591,11 +610,8 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                     if (kk < Qv) {
                         const float dda = R[u] + Es[u] + F + Wp[u];
                         const float ddt = dr0[u] + w[u] + Ah * dda;
-                        const int64_t di = (row0 + kk) * a.H + h;
-                        const float raw = a.act_bf16 ? bf_lo(static_cast<const unsigned short*>(a.dt)[di])
-                                                     : static_cast<const float*>(a.dt)[di];
-                        const float dr = ddt * sigm(raw + bias);
-                        a.ddt[di] = dr;
+                        const float dr = ddt * sigm(raw[u] + bias);
+                        a.ddt[(row0 + kk) * a.H + h] = dr;
                         pdA += dtk[u] * dda;
                         pbias += dr;
                     }
@@ -614,17 +630,13 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             mbar_arrive(&bars[TILE_FREE0 + buf]);
         }
         if (!ok) give_up(abort);
-        if (warp == 0) {
-            if (lane == 0) mma_commit(&bars[FINAL]);  // every MMA issued so far
-            __syncwarp();
-        }
     }
 
     // every role is done issuing; dB^T and dC^T are final once the last MMAs complete
     const bool done = __all_sync(0xffffffffu, mbar_wait(&bars[FINAL], 0, nullptr));
     tc_fence_after();
     __syncthreads();
-    if (done && *abort == 0) {
+    if (warp < 8 && done && *abort == 0) {
         const int n = 32 * (warp & 3) + lane, j0 = 32 * (warp >> 2);
         const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
         float db[32], dc[32];
@@ -646,7 +658,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS_B);
     }
