@@ -27,14 +27,15 @@
 // cannot hold (>= 65504) sets bit 1 of this file's error word (SSD_ERR_RANGE).  The elementwise terms
 // read x, g and dy silu'(z) back from the same fp16 tiles the MMAs use.
 //
-// One CTA per (chunk, group, half of the group's heads), heads in turn; 288 threads in three roles:
+// One CTA per (chunk, group, half of the group's heads), heads in turn; 384 threads in four roles:
 //   row warps 0, 1, 4, 5  (TMEM lanes 0..63 = the chunk's tokens; warps 0/4 tokens 0..31, 1/5 tokens
 //                         32..63; warps 0, 1 columns 0..31, warps 4, 5 columns 32..63): the elementwise
-//                         work above, the LCB / LGX' tiles, dz, dx; warp 0 also the per-head scalars
-//                         (ddt and the partial sums);
-//   loader warps 2, 3, 6, 7: the head's tiles, two heads deep: Sp and Lm by bulk copy, x, X', g, G'' and
-//                         dy silu'(z) converted from global memory;
-//   warp 8              : TMEM allocation and, on one thread, the MMAs.
+//                         work above, the LCB / LGX' tiles, dz, dx and per-row partial sums;
+//   loader warps 2, 3, 6, 7, 10, 11: the head's tiles, two heads deep: Sp and Lm by bulk copy, x, X', g, G''
+//                         and dy silu'(z) converted from global memory;
+//   warp 8              : TMEM allocation and, on one thread, the MMAs;
+//   warp 9              : each head's per-token scalars from the partial sums (the prefix / suffix sums
+//                         behind d(dA), ddt) and the per-chunk partials of dA, dD, ddt_bias.
 // Every MMA is M = 128, N = 64 with fp32 accumulators in TMEM (512 columns: CB, GX, SPC, LMB, YIN, DXI,
 // dB^T, dC^T).  The token-major products use only rows 0..63 of their 128-row result: the A tile's rows
 // 64..127 are whatever follows it in shared memory (always in bounds), and the result lanes 64..127 are
@@ -60,7 +61,9 @@ using namespace sm100;
 
 constexpr int kQb = 64;   // chunk (tokens)
 constexpr int kPb = 64;   // head dimension
-constexpr int kThreadsB = 288;
+constexpr int kThreadsB = 384;
+constexpr int kLoaders = 192;  // loader threads (warps 2, 3, 6, 7, 10, 11)
+constexpr int kSplitPf = 4;    // partial sums of F per (chunk, head) from the state pass
 
 // shared memory (bytes from a 1024-byte aligned base).  A "box" is [64 rows][64 fp16] with 128-byte rows
 // and the 128-byte swizzle (8 KB); an N-wide tile is one box per 64 state columns.
@@ -89,7 +92,7 @@ constexpr uint32_t V_ISC = 5248;        //   inverse row scales of each buffer's
 constexpr uint32_t VEC_BYTES = 6272;
 constexpr uint32_t OFF_BAR = OFF_VEC + VEC_BYTES;
 enum : int { TILE_FULL0, TILE_FULL1, TILE_FREE0, TILE_FREE1, SPLM_FULL0, SPLM_FULL1, GX_DONE, B1_DONE, LT_FULL,
-             B2_DONE, ACC_FREE, WSYNC, FINAL, NBAR };
+             B2_DONE, ACC_FREE, WSYNC, SCALAR_FREE, FINAL, NBAR };
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // abort word, TMEM base
 constexpr uint32_t SMEM_B = OFF_MISC + 16 + 1024;  // + alignment slack
 
@@ -267,10 +270,10 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
     }
     if (tid == 0) {
         *abort = 0;
-        mbar_init(&bars[TILE_FULL0], 128);
-        mbar_init(&bars[TILE_FULL1], 128);
-        mbar_init(&bars[TILE_FREE0], 129);  // the MMAs' commit + the 128 row threads
-        mbar_init(&bars[TILE_FREE1], 129);
+        mbar_init(&bars[TILE_FULL0], kLoaders);
+        mbar_init(&bars[TILE_FULL1], kLoaders);
+        mbar_init(&bars[TILE_FREE0], 1 + 128 + 32);  // the MMAs' commit, the row threads, the scalar warp
+        mbar_init(&bars[TILE_FREE1], 1 + 128 + 32);
         mbar_init(&bars[SPLM_FULL0], 1);    // the bulk copies' transaction bytes
         mbar_init(&bars[SPLM_FULL1], 1);
         mbar_init(&bars[GX_DONE], 1);
@@ -279,6 +282,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
         mbar_init(&bars[B2_DONE], 1);
         mbar_init(&bars[ACC_FREE], 128);
         mbar_init(&bars[WSYNC], 128);
+        mbar_init(&bars[SCALAR_FREE], 32);
         mbar_init(&bars[FINAL], 1);
         fence_mbar_init();
     }
@@ -327,10 +331,94 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             mma_commit(&bars[FINAL]);  // every MMA issued so far
         }
         __syncwarp();
-    } else if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
-        // ---------------- loaders ----------------
-        const int lt = ((warp & 3) - 2 + 2 * (warp >> 2)) * 32 + lane;  // 0..127
-        const int k8 = lt & 7;  // this thread's 16-byte chunk (8 head channels) of rows lt / 8 + 16 m
+    } else if (warp == 9) {
+        // ---------------- scalar warp: each head's ddt and per-chunk partial sums (tokens lane, lane + 32) -------
+        bool ok = true;
+        for (int k = 0; k < nh && ok; ++k) {
+            const int buf = k & 1, par = k & 1;
+            const int h = g * hpg + hl0 + k;
+            // the global inputs first: F, the raw dt of the two tokens, A, dt_bias
+            const float* pf = a.PF + ((b * nc + c) * a.H + h) * kSplitPf;
+            const float F = (pf[0] + pf[1]) + (pf[2] + pf[3]);
+            float raw[2] = {0.f, 0.f};
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int kk = lane + 32 * u;
+                if (kk < Qv) raw[u] = bf_lo(static_cast<const unsigned short*>(a.dt)[(row0 + kk) * a.H + h]);
+            }
+            const float Ah = a.A[h], bias = a.dt_bias[h];
+            // dt and exp(cs) of the two tokens from the head's buffer (TILE_FULL), then the row warps' sums (WSYNC)
+            if (!wait_all(&bars[TILE_FULL0 + buf], (k >> 1) & 1, abort)) {
+                ok = false;
+                break;
+            }
+            const float* dts = vec + (V_DT >> 2) + buf * 64;
+            const float* css = vec + (V_CS >> 2) + buf * 64;
+            float dtk[2], exk[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int kk = lane + 32 * u;
+                dtk[u] = dts[kk];
+                exk[u] = kk < Qv ? expf(css[kk]) : 0.f;
+            }
+            if (!wait_all(&bars[WSYNC], par, abort)) {
+                ok = false;
+                break;
+            }
+            const float* col = vec + (V_COL >> 2) + par * 128;
+            const float* rwm = vec + (V_ROWM >> 2) + par * 128;
+            const float* ev = vec + (V_E >> 2) + par * 128;
+            const float* wv = vec + (V_W >> 2) + par * 128;
+            const float* pdw = vec + (V_PD >> 2) + par * 4;
+            float dr0[2], d[2], e[2], w[2], dw[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int kk = lane + 32 * u;
+                dr0[u] = col[kk] + col[64 + kk];
+                d[u] = dtk[u] * dr0[u] - (rwm[kk] + rwm[64 + kk]);
+                e[u] = exk[u] * (ev[kk] + ev[64 + kk]);
+                w[u] = wv[kk] + wv[64 + kk];
+                dw[u] = dtk[u] * w[u];
+            }
+            const float pD = (pdw[0] + pdw[1]) + (pdw[2] + pdw[3]);
+            __syncwarp();
+            mbar_arrive(&bars[SCALAR_FREE]);  // the partial sums are read: the row warps may write the next ones
+            // exclusive prefix sums of d and dt W, inclusive suffix sums of E, over the 64 tokens
+            float R[2], Wp[2], Ex[2], Es[2];
+            scan_excl(d, R, lane);
+            scan_excl(dw, Wp, lane);
+            scan_excl(e, Ex, lane);
+            const float etot = __shfl_sync(0xffffffffu, Ex[1] + e[1], 31);
+            Es[0] = etot - Ex[0];
+            Es[1] = etot - Ex[1];
+            float pdA = 0.f, pbias = 0.f;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int kk = lane + 32 * u;
+                if (kk < Qv) {
+                    const float dda = R[u] + Es[u] + F + Wp[u];
+                    const float ddt = dr0[u] + w[u] + Ah * dda;
+                    const float dr = ddt * sigm(raw[u] + bias);
+                    a.ddt[(row0 + kk) * a.H + h] = dr;
+                    pdA += dtk[u] * dda;
+                    pbias += dr;
+                }
+            }
+            pdA = warp_sum(pdA);
+            pbias = warp_sum(pbias);
+            if (lane == 0) {
+                float* ph = a.PH + ((b * nc + c) * a.H + h) * 3;
+                ph[0] = pdA;
+                ph[1] = pD;
+                ph[2] = pbias;
+            }
+            mbar_arrive(&bars[TILE_FREE0 + buf]);
+        }
+        if (!ok) give_up(abort);
+    } else if ((warp & 3) >= 2) {
+        // ---------------- loaders: warps 2, 3, 6, 7, 10, 11 ----------------
+        const int lt = ((warp >> 2) * 2 + (warp & 3) - 2) * 32 + lane;  // 0..kLoaders-1
+        const int k8 = lt & 7;  // this thread's 16-byte chunk (8 head channels) of rows lt / 8 + 24 m
         for (int k = 0; k < nh; ++k) {
             const int buf = k & 1;
             if (k >= 2 && !wait_all(&bars[TILE_FREE0 + buf], ((k >> 1) - 1) & 1, abort)) {
@@ -353,12 +441,13 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 bulk_load(isc, a.SPS + ti * 64, 256, bar);
                 bulk_load(isc + 64, a.LMS + ti * 64, 256, bar);
             }
-            // x, X', g, G'', dy silu'(z): 64 rows x 8 chunks of 8 channels, four chunks per thread, all loads first
+            // x, X', g, G'', dy silu'(z): 64 rows x 8 chunks of 8 channels, up to three chunks per thread (rows
+            // lt / 8 + 24 m below 64), all loads first
             const float cs_last = a.CS[hrow + Qv - 1];
-            float xv[4][8], gv[4][8], zv[4][8], dtr[4], csr[4];
+            float xv[3][8], gv[3][8], zv[3][8], dtr[3], csr[3];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int r = (lt >> 3) + 16 * m;
+            for (int m = 0; m < 3; ++m) {
+                const int r = (lt >> 3) + 24 * m;
                 if (r < Qv) {
                     dtr[m] = a.DT[hrow + r];
                     csr[m] = a.CS[hrow + r];
@@ -381,8 +470,9 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             const float* is = isc + 8 * k8;
             const float* il = isc + 64 + 8 * k8;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int r = (lt >> 3) + 16 * m;
+            for (int m = 0; m < 3; ++m) {
+                const int r = (lt >> 3) + 24 * m;
+                if (r >= kQb) break;
                 float ds[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -419,23 +509,6 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             const int buf = k & 1, par = k & 1;
             const int h = g * hpg + hl0 + k;
             const float Dh = a.D[h];
-            // warp 0's per-head scalars from global memory, ahead of the waits: F, the raw dt of its two
-            // tokens, A, dt_bias
-            float F = 0.f, raw[2] = {0.f, 0.f}, Ah = 0.f, bias = 0.f;
-            if (warp == 0) {
-                for (int s = 0; s < a.nsplit_pf; ++s) F += a.PF[((b * nc + c) * a.H + h) * a.nsplit_pf + s];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int kk = lane + 32 * u;
-                    if (kk < Qv) {
-                        const int64_t di = (row0 + kk) * a.H + h;
-                        raw[u] = a.act_bf16 ? bf_lo(static_cast<const unsigned short*>(a.dt)[di])
-                                            : static_cast<const float*>(a.dt)[di];
-                    }
-                }
-                Ah = a.A[h];
-                bias = a.dt_bias[h];
-            }
             // the head's tiles (TILE_FULL), then GX (GX_DONE)
             if (!wait_all(&bars[TILE_FULL0 + buf], (k >> 1) & 1, abort) || !wait_all(&bars[GX_DONE], par, abort)) {
                 ok = false;
@@ -484,6 +557,11 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 fence_async_smem();
                 mbar_arrive(&bars[LT_FULL]);
                 if (!(range < 65504.f)) atomicOr(&g_chunk_bwd_tc_error, 2);
+                // the scalar warp is done with the previous head's partial sums before these are written
+                if (k > 0 && !wait_all(&bars[SCALAR_FREE], (k - 1) & 1, abort)) {
+                    ok = false;
+                    break;
+                }
                 const float col = column_sums(gx, lane);
                 vec[(V_COL >> 2) + (par * 2 + rq) * 64 + c0 + lane] = col;
             }
@@ -574,59 +652,6 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             pd = warp_sum(pd);
             if (lane == 0) vec[(V_PD >> 2) + par * 4 + wi] = pd;
             mbar_arrive(&bars[WSYNC]);
-            if (warp == 0) {
-                // the head's per-token scalars: tokens lane and lane + 32
-                if (!wait_all(&bars[WSYNC], par, abort)) {
-                    ok = false;
-                    break;
-                }
-                const float* col = vec + (V_COL >> 2) + par * 128;
-                const float* rwm = vec + (V_ROWM >> 2) + par * 128;
-                const float* ev = vec + (V_E >> 2) + par * 128;
-                const float* wv = vec + (V_W >> 2) + par * 128;
-                float dr0[2], dtk[2], d[2], e[2], w[2], dw[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int kk = lane + 32 * u;
-                    dr0[u] = col[kk] + col[64 + kk];
-                    dtk[u] = dts[kk];
-                    d[u] = dtk[u] * dr0[u] - (rwm[kk] + rwm[64 + kk]);
-                    e[u] = (kk < Qv ? expf(css[kk]) : 0.f) * (ev[kk] + ev[64 + kk]);
-                    w[u] = wv[kk] + wv[64 + kk];
-                    dw[u] = dtk[u] * w[u];
-                }
-                // exclusive prefix sums of d and dt W, inclusive suffix sums of E, over the 64 tokens
-                float R[2], Wp[2], Ex[2], Es[2];
-                scan_excl(d, R, lane);
-                scan_excl(dw, Wp, lane);
-                scan_excl(e, Ex, lane);
-                const float etot = __shfl_sync(0xffffffffu, Ex[1] + e[1], 31);
-                Es[0] = etot - Ex[0];
-                Es[1] = etot - Ex[1];
-                float pdA = 0.f, pbias = 0.f;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int kk = lane + 32 * u;
-                    if (kk < Qv) {
-                        const float dda = R[u] + Es[u] + F + Wp[u];
-                        const float ddt = dr0[u] + w[u] + Ah * dda;
-                        const float dr = ddt * sigm(raw[u] + bias);
-                        a.ddt[(row0 + kk) * a.H + h] = dr;
-                        pdA += dtk[u] * dda;
-                        pbias += dr;
-                    }
-                }
-                pdA = warp_sum(pdA);
-                pbias = warp_sum(pbias);
-                if (lane == 0) {
-                    const float* pdw = vec + (V_PD >> 2) + par * 4;
-                    float* ph = a.PH + ((b * nc + c) * a.H + h) * 3;
-                    ph[0] = pdA;
-                    ph[1] = (pdw[0] + pdw[1]) + (pdw[2] + pdw[3]);
-                    ph[2] = pbias;
-                }
-                __syncwarp();
-            }
             mbar_arrive(&bars[TILE_FREE0 + buf]);
         }
         if (!ok) give_up(abort);
@@ -680,6 +705,7 @@ cudaError_t read_and_clear_chunk_bwd_tc_error(int* flag) {
 }
 
 cudaError_t launch_chunk_bwd_tc(const ChunkBwdTcArgs& a, int64_t nchunks, cudaStream_t st) {
+    if (a.nsplit_pf != kSplitPf || !a.act_bf16) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_B);
     if (e != cudaSuccess) return e;
