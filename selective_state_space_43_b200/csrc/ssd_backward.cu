@@ -154,28 +154,61 @@ __device__ __forceinline__ float raw_at(const BwdArgs& a, int64_t b, int64_t s, 
     return ld_act(a.C, row * GN + (c - HP - GN), a.act_bf16);
 }
 
-// grid (ceil(conv_dim / kT), nchunks, batch): one thread per (channel, 64-token tile).
+constexpr int kCPT = 2;  // channels per thread of the conv kernels (conv_dim is even, and so is every array's width)
+
+// The pre-conv array (x, B or C) of an even channel c and of c + 1, its row stride and column.
+struct ChanPair {
+    const void* src;
+    int64_t stride, col;
+};
+__device__ __forceinline__ ChanPair chan_pair(const BwdArgs& a, int64_t c) {
+    const int64_t HP = (int64_t)a.H * a.P, GN = (int64_t)a.G * a.N;
+    if (c < HP) return {a.x, HP, c};
+    if (c < HP + GN) return {a.B, GN, c - HP};
+    return {a.C, GN, c - HP - GN};
+}
+// Channels c, c + 1 at token s: the inputs for s >= 0, the conv history (or zero) before.
+__device__ __forceinline__ float2 raw_pair(const BwdArgs& a, const ChanPair& q, int64_t b, int64_t s, int64_t c) {
+    if (s < 0) return make_float2(raw_at(a, b, s, c), raw_at(a, b, s, c + 1));
+    const int64_t i = (b * a.L + s) * q.stride + q.col;
+    if (a.act_bf16) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(static_cast<const unsigned short*>(q.src) + i);
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    return *reinterpret_cast<const float2*>(static_cast<const float*>(q.src) + i);
+}
+
+// grid (ceil(conv_dim / (kT * kCPT)), nchunks, batch): one thread per (pair of channels, 64-token tile), streaming
+// the tile with kBatch tokens' inputs loaded before their outputs are stored (the stores could alias the
+// inputs as far as the compiler knows, so it would not move later loads above them).
 __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
     const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N;
-    const int64_t c = (int64_t)blockIdx.x * kT + threadIdx.x;
+    const int64_t c = ((int64_t)blockIdx.x * kT + threadIdx.x) * kCPT;
     if (c >= conv_dim) return;
     const int64_t b = blockIdx.z, t0 = (int64_t)blockIdx.y * kQ;
     const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
-    const float w0 = a.conv_w[c * 4 + 0], w1 = a.conv_w[c * 4 + 1], w2 = a.conv_w[c * 4 + 2],
-                w3 = a.conv_w[c * 4 + 3], bias = a.conv_b[c];
-    float r0 = raw_at(a, b, t0 - 3, c), r1 = raw_at(a, b, t0 - 2, c), r2 = raw_at(a, b, t0 - 1, c);
-    // kBatch tokens' inputs are loaded before any of their outputs is stored (the stores could alias
-    // the inputs as far as the compiler knows, so it would not move later loads above them)
+    float w[2][4], bias[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float4 wv = *reinterpret_cast<const float4*>(a.conv_w + (c + k) * 4);
+        w[k][0] = wv.x, w[k][1] = wv.y, w[k][2] = wv.z, w[k][3] = wv.w;
+        bias[k] = a.conv_b[c + k];
+    }
+    const ChanPair q = chan_pair(a, c);
+    float2 r0 = raw_pair(a, q, b, t0 - 3, c), r1 = raw_pair(a, q, b, t0 - 2, c), r2 = raw_pair(a, q, b, t0 - 1, c);
     constexpr int kBatch = 8;
 #pragma unroll 1
     for (int64_t tb = t0; tb < t1; tb += kBatch) {
-        float rin[kBatch];
+        float2 rin[kBatch];
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) rin[i] = tb + i < t1 ? raw_at(a, b, tb + i, c) : 0.f;
+        for (int i = 0; i < kBatch; ++i) rin[i] = tb + i < t1 ? raw_pair(a, q, b, tb + i, c) : make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < kBatch; ++i) {
             if (tb + i < t1) {
-                ws.U[(b * a.L + tb + i) * conv_dim + c] = silu_f(bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * rin[i]);
+                float2 u;
+                u.x = silu_f(bias[0] + w[0][0] * r0.x + w[0][1] * r1.x + w[0][2] * r2.x + w[0][3] * rin[i].x);
+                u.y = silu_f(bias[1] + w[1][0] * r0.y + w[1][1] * r1.y + w[1][2] * r2.y + w[1][3] * rin[i].y);
+                *reinterpret_cast<float2*>(ws.U + (b * a.L + tb + i) * conv_dim + c) = u;
                 r0 = r1;
                 r1 = r2;
                 r2 = rin[i];
@@ -184,21 +217,39 @@ __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
     }
 }
 
-// grid (ceil(H * nchunks / kT), batch): one thread per (head, chunk).
+// grid (nchunks, ceil(H / (kT / 32)), batch), kT threads: one warp per (chunk, head), lane l holding tokens
+// t0 + l and t0 + l + 32: dt = softplus(dt_raw + dt_bias) and the in-chunk inclusive cumulative sum of dt * A
+// (a warp scan), stored with consecutive lanes on consecutive tokens.
 __global__ void __launch_bounds__(kT) dt_kernel(BwdArgs a, Ws ws) {
-    const int64_t nc = nchunks(a.L);
-    const int64_t idx = (int64_t)blockIdx.x * kT + threadIdx.x;
-    if (idx >= nc * a.H) return;
-    const int h = static_cast<int>(idx % a.H);
-    const int64_t c = idx / a.H, b = blockIdx.y, t0 = c * kQ;
+    const int lane = threadIdx.x & 31;
+    const int64_t h = (int64_t)blockIdx.y * (kT / 32) + (threadIdx.x >> 5);
+    if (h >= a.H) return;
+    const int64_t b = blockIdx.z, t0 = (int64_t)blockIdx.x * kQ;
     const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
     const float Ah = a.A[h], bias = a.dt_bias[h];
-    float cs = 0.f;
-    for (int64_t t = t0; t < t1; ++t) {
-        const float dt = softplus_f(ld_act(a.dt, (b * a.L + t) * a.H + h, a.act_bf16) + bias);
-        cs += dt * Ah;
-        ws.DT[(b * a.H + h) * a.L + t] = dt;
-        ws.CS[(b * a.H + h) * a.L + t] = cs;
+    float dt[2], v[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int64_t t = t0 + lane + 32 * u;
+        dt[u] = t < t1 ? softplus_f(ld_act(a.dt, (b * a.L + t) * a.H + h, a.act_bf16) + bias) : 0.f;
+        v[u] = dt[u] * Ah;
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float p0 = __shfl_up_sync(0xffffffffu, v[0], o), p1 = __shfl_up_sync(0xffffffffu, v[1], o);
+        if (lane >= o) {
+            v[0] += p0;
+            v[1] += p1;
+        }
+    }
+    v[1] += __shfl_sync(0xffffffffu, v[0], 31);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int64_t t = t0 + lane + 32 * u;
+        if (t < t1) {
+            ws.DT[(b * a.H + h) * a.L + t] = dt[u];
+            ws.CS[(b * a.H + h) * a.L + t] = v[u];
+        }
     }
 }
 
@@ -502,37 +553,91 @@ __device__ __forceinline__ void store_half_row(const float (&v)[M], int p, int n
 }
 #endif
 
+#ifndef SSD_EMU
+// The M (8 or 4) elements n0.. of row p of one (chunk, head) fp16 tile (see Ws::SPH), unscaled.
+template <int M>
+__device__ __forceinline__ void load_half_row(const char* tile, const float* inv_scale, int p, int n0, float (&v)[M]) {
+    const int k8 = n0 >> 3;
+    const char* src = tile + (k8 >> 3) * 8192 + p * 128 + (((k8 & 7) ^ (p & 7)) << 4) + ((n0 & 7) ? 8 : 0);
+    uint32_t w[M / 2];
+    if constexpr (M == 8) {
+        const uint4 q = *reinterpret_cast<const uint4*>(src);
+        w[0] = q.x, w[1] = q.y, w[2] = q.z, w[3] = q.w;
+    } else {
+        const uint2 q = *reinterpret_cast<const uint2*>(src);
+        w[0] = q.x, w[1] = q.y;
+    }
+    const float is = inv_scale[p];
+#pragma unroll
+    for (int m = 0; m < M; m += 2) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[m / 2]));
+        v[m] = f.x * is;
+        v[m + 1] = f.y * is;
+    }
+}
+#endif
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+constexpr int kWin = 32;  // chunks per window of the state pass (one decay per lane, one F flush)
+
+// Shared memory of the state pass: the per-warp partial F sums of a window, by window parity.
+constexpr size_t state_pass_smem() { return 2 * (size_t)kWin * (kT / 32) * sizeof(float); }
+
 // grid (H * kSplit, batch), kT threads: the P*N state elements of a head in kSplit slices of P / kSplit whole
 // rows p; a thread holds M = P*N / (kSplit * kT) consecutive elements of one row (16 threads per row).  The
 // forward scan turns SP into the states entering each chunk, the reverse scan turns LM into the adjoints
-// leaving each chunk and leaves each slice's part of F; the next chunk's values are loaded before the
-// current chunk's are stored, so the loads of consecutive chunks overlap.  For the tensor-core chunk
-// backward (ws.SPH set) the entering states are also written as scaled fp16 tiles, and the leaving adjoints
-// only as such tiles (the fp32 ones have no other reader).
+// leaving each chunk and leaves each slice's part of F.  The next chunk's values are loaded before the
+// current chunk's are stored, so the loads of consecutive chunks overlap; the chunks' decays are loaded 32 at
+// a time (one per lane) and F is reduced per warp, with one block barrier per 32 chunks.  For the
+// tensor-core chunk backward (ws.SPH set) the entering states are written only as scaled fp16 tiles, the
+// reverse scan takes them from there for F, and the leaving adjoints are written only as such tiles (the fp32
+// arrays have no other reader).
 template <int N>
 __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
     constexpr int M = kP * N / (kSplit * kT);
     constexpr int SLICE = kP * N / kSplit;
+    constexpr int NW = kT / 32;
     const int64_t nc = nchunks(a.L), b = blockIdx.y;
     const int h = blockIdx.x / kSplit, sp = blockIdx.x % kSplit, tid = threadIdx.x;
-    float* red = reinterpret_cast<float*>(SSD_DYN_SMEM());
+    const int lane = tid & 31, wid = tid >> 5;
+    float* fw = reinterpret_cast<float*>(SSD_DYN_SMEM());  // [2][kWin][NW]
     const int64_t off = (int64_t)sp * SLICE + (int64_t)tid * M;  // this thread's first element in a P x N block
     const int64_t head = (b * a.H + h) * (int64_t)kP * N + off;
     const int prow = static_cast<int>(off / N), n0 = static_cast<int>(off % N);
     const float* csh = ws.CS + (b * a.H + h) * a.L;
-    const bool half_tiles = ws.SPH != nullptr;
+#ifndef SSD_EMU
+    const bool half_tiles = (M == 4 || M == 8) && ws.SPH != nullptr;
+#else
+    const bool half_tiles = false;
+#endif
     auto blk = [&](int64_t c) { return ((b * nc + c) * a.H + h) * (int64_t)kP * N; };
+    // exp(cs at the last token) of chunk w * kWin + lane, for the window w
+    auto window_decays = [&](int64_t w) {
+        const int64_t c = w * kWin + lane;
+        float d = 0.f;
+        if (c < nc) {
+            const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
+            d = expf(csh[last]);
+        }
+        return d;
+    };
 
     float s[M], cur[M], nxt[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) s[m] = cur[m] = nxt[m] = 0.f;
     if (a.init_state) ld_vec<M>(a.init_state + head, s);
     if (nc > 0) ld_vec<M>(ws.SP + blk(0) + off, cur);
+    float dwin = 0.f;
     for (int64_t c = 0; c < nc; ++c) {
-        const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
-        const float decay = expf(csh[last]);
+        if ((c % kWin) == 0) dwin = window_decays(c / kWin);
+        const float decay = __shfl_sync(0xffffffffu, dwin, static_cast<int>(c % kWin));
         if (c + 1 < nc) ld_vec<M>(ws.SP + blk(c + 1) + off, nxt);
-        st_vec<M>(ws.SP + blk(c) + off, s);
+        if (!half_tiles) st_vec<M>(ws.SP + blk(c) + off, s);
 #ifndef SSD_EMU
         if constexpr (M == 4 || M == 8) {
             if (half_tiles)
@@ -547,20 +652,36 @@ __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
         }
     }
 
-    float l[M], sp_cur[M], sp_nxt[M];
+    // reverse: the adjoints leaving each chunk, and F = decay <Lm, Sp> per chunk (this slice's part)
+    float l[M], lcur[M], lnxt[M], scur[M], snxt[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) l[m] = cur[m] = nxt[m] = sp_cur[m] = sp_nxt[m] = 0.f;
+    for (int m = 0; m < M; ++m) l[m] = lcur[m] = lnxt[m] = scur[m] = snxt[m] = 0.f;
     if (a.d_final) ld_vec<M>(a.d_final + head, l);
+    // the state entering chunk c: the fp32 array, or the fp16 tile and its row scale
+    auto load_sp = [&](int64_t c, float (&v)[M]) {
+#ifndef SSD_EMU
+        if constexpr (M == 4 || M == 8) {
+            if (half_tiles) {
+                load_half_row<M>(reinterpret_cast<const char*>(ws.SPH) + blk(c) * 2,
+                                 ws.SPS + ((b * nc + c) * a.H + h) * kP, prow, n0, v);
+                return;
+            }
+        }
+#endif
+        ld_vec<M>(ws.SP + blk(c) + off, v);
+    };
     if (nc > 0) {
-        ld_vec<M>(ws.LM + blk(nc - 1) + off, cur);
-        ld_vec<M>(ws.SP + blk(nc - 1) + off, sp_cur);
+        ld_vec<M>(ws.LM + blk(nc - 1) + off, lcur);
+        load_sp(nc - 1, scur);
     }
     for (int64_t c = nc - 1; c >= 0; --c) {
-        const int64_t last = (c * kQ + kQ - 1 < a.L ? c * kQ + kQ - 1 : a.L - 1);
-        const float decay = expf(csh[last]);
+        const int64_t w = c / kWin;
+        const int ci = static_cast<int>(c % kWin);
+        if (c == nc - 1 || ci == kWin - 1) dwin = window_decays(w);
+        const float decay = __shfl_sync(0xffffffffu, dwin, ci);
         if (c > 0) {
-            ld_vec<M>(ws.LM + blk(c - 1) + off, nxt);
-            ld_vec<M>(ws.SP + blk(c - 1) + off, sp_nxt);
+            ld_vec<M>(ws.LM + blk(c - 1) + off, lnxt);
+            load_sp(c - 1, snxt);
         }
 #ifndef SSD_EMU
         if constexpr (M == 4 || M == 8) {
@@ -578,13 +699,24 @@ __global__ void __launch_bounds__(kT) state_pass_kernel(BwdArgs a, Ws ws) {
         float f = 0.f;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            f += l[m] * sp_cur[m];
-            l[m] = decay * l[m] + cur[m];
-            cur[m] = nxt[m];
-            sp_cur[m] = sp_nxt[m];
+            f += l[m] * scur[m];
+            l[m] = decay * l[m] + lcur[m];
+            lcur[m] = lnxt[m];
+            scur[m] = snxt[m];
         }
-        f = block_sum(f, red);
-        if (tid == 0) ws.PF[((b * nc + c) * a.H + h) * kSplit + sp] = decay * f;
+        f = warp_sum_f(f);
+        if (lane == 0) fw[((w & 1) * kWin + ci) * NW + wid] = f;
+        if (ci == 0) {
+            // the window is done: its chunks' F, the warps' sums in a fixed order, times the chunk's decay
+            // (lane t of every warp holds chunk w * kWin + t's)
+            __syncthreads();
+            if (tid < kWin && w * kWin + tid < nc) {
+                float t = 0.f;
+#pragma unroll
+                for (int q = 0; q < NW; ++q) t += fw[((w & 1) * kWin + tid) * NW + q];
+                ws.PF[((b * nc + w * kWin + tid) * a.H + h) * kSplit + sp] = dwin * t;
+            }
+        }
     }
     if (a.d_init_state) st_vec<M>(a.d_init_state + head, l);
 }
@@ -1006,7 +1138,7 @@ __global__ void __launch_bounds__(kT) copy_adjoint_kernel(BwdArgs a) {
 template <int N>
 cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
     const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N, nc = nchunks(a.L), nt = ntiles(a.L);
-    const unsigned cgrid = static_cast<unsigned>((conv_dim + kT - 1) / kT);
+    const unsigned cgrid = static_cast<unsigned>((conv_dim + kT * kCPT - 1) / (kT * kCPT));  // post-conv channel pairs
     cudaError_t err;
     if (a.batch > 0 && nc > 0) {
         const size_t state_smem = (2 * (size_t)kQ * kP + 2 * (size_t)kQ * N + 2 * kQ) * sizeof(float);
@@ -1015,7 +1147,9 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         if ((err = SSD_SET_SMEM(chunk_bwd_kernel<N>, chunk_smem)) != cudaSuccess) return err;
         const dim3 tiles(cgrid, static_cast<unsigned>(nc), static_cast<unsigned>(a.batch));
         SSD_LAUNCH(post_conv_kernel, tiles, dim3(kT), 0, st, a, ws);
-        SSD_LAUNCH(dt_kernel, dim3(static_cast<unsigned>((nc * a.H + kT - 1) / kT), static_cast<unsigned>(a.batch)),
+        SSD_LAUNCH(dt_kernel,
+                   dim3(static_cast<unsigned>(nc), static_cast<unsigned>((a.H + kT / 32 - 1) / (kT / 32)),
+                        static_cast<unsigned>(a.batch)),
                    dim3(kT), 0, st, a, ws);
         const dim3 chunk_heads(static_cast<unsigned>(nc), static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
         Ws wsp = ws;  // the state pass writes the fp16 state tiles only for the tensor-core chunk backward
@@ -1037,7 +1171,7 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         SSD_LAUNCH(chunk_state_kernel<N>, chunk_heads, dim3(kT), state_smem, st, a, ws);
 #endif
         SSD_LAUNCH(state_pass_kernel<N>, dim3(static_cast<unsigned>(a.H * kSplit), static_cast<unsigned>(a.batch)),
-                   dim3(kT), kT * sizeof(float), st, a, wsp);
+                   dim3(kT), state_pass_smem(), st, a, wsp);
         const dim3 chunk_groups(static_cast<unsigned>(nc), static_cast<unsigned>(a.G * head_split(a.H, a.G)),
                                 static_cast<unsigned>(a.batch));
 #ifndef SSD_EMU
@@ -1063,8 +1197,10 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         SSD_LAUNCH(copy_adjoint_kernel, dim3(static_cast<unsigned>((n + kT - 1) / kT)), dim3(kT), 0, st, a);
     }
     if (a.batch > 0)
-        SSD_LAUNCH(conv_bwd_kernel, dim3(cgrid, static_cast<unsigned>(nt), static_cast<unsigned>(a.batch)), dim3(kT),
-                   0, st, a, ws);
+        SSD_LAUNCH(conv_bwd_kernel,
+                   dim3(static_cast<unsigned>((conv_dim + kT - 1) / kT), static_cast<unsigned>(nt),
+                        static_cast<unsigned>(a.batch)),
+                   dim3(kT), 0, st, a, ws);
     SSD_LAUNCH(reduce_kernel, dim3(static_cast<unsigned>((conv_dim + a.H + kT - 1) / kT)), dim3(kT), 0, st, a, ws);
     return cudaGetLastError();
 }

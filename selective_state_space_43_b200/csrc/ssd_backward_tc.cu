@@ -57,11 +57,13 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi, float& range) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ float act_at(const void* p, int64_t i, bool bf16) {
-    if (bf16) return __uint_as_float(static_cast<uint32_t>(static_cast<const unsigned short*>(p)[i]) << 16);
-    return static_cast<const float*>(p)[i];
+// Eight values (two float4) times s as fp16, tracking `range`.
+__device__ __forceinline__ uint4 pack8f(float4 a, float4 b, float s, float& range) {
+    return make_uint4(pack_h2(a.x * s, a.y * s, range), pack_h2(a.z * s, a.w * s, range), pack_h2(b.x * s, b.y * s, range),
+                      pack_h2(b.z * s, b.w * s, range));
 }
-__device__ __forceinline__ float silu_c(float v) { return v / (1.f + expf(-v)); }
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // grid (nchunks, H, batch), kThreadsC threads, SMEM_C bytes of dynamic shared memory
 __global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkStateTcArgs a) {
@@ -86,47 +88,81 @@ __global__ void __launch_bounds__(kThreadsC) chunk_state_tc_kernel(const ChunkSt
     }
 
     float range = 0.f;  // largest magnitude this thread writes to an fp16 tile
-    // B and C of the chunk (rows j >= Qv and channels n >= N zero): 64 rows x 16 chunks of 8 channels each
-    for (int e = tid; e < kQc * (kNc / 8); e += kThreadsC) {
-        const int r = e >> 4, k8 = e & 15, n0 = 8 * k8;
-        uint4 pb = make_uint4(0u, 0u, 0u, 0u), pc = pb;
-        if (r < Qv && n0 < a.N) {
-            const float* row = a.U + (b * a.L + t0 + r) * conv_dim + HP + (int64_t)g * a.N + n0;
-            const float4 b0 = *reinterpret_cast<const float4*>(row), b1 = *reinterpret_cast<const float4*>(row + 4);
-            const float4 c0 = *reinterpret_cast<const float4*>(row + GN);
-            const float4 c1 = *reinterpret_cast<const float4*>(row + GN + 4);
-            pb = make_uint4(pack_h2(b0.x, b0.y, range), pack_h2(b0.z, b0.w, range), pack_h2(b1.x, b1.y, range),
-                            pack_h2(b1.z, b1.w, range));
-            pc = make_uint4(pack_h2(c0.x, c0.y, range), pack_h2(c0.z, c0.w, range), pack_h2(c1.x, c1.y, range),
-                            pack_h2(c1.z, c1.w, range));
+    // B and C of the chunk (rows j >= Qv and channels n >= N zero): 64 rows x 16 chunks of 8 channels, eight
+    // per thread in two passes of four, each pass's loads issued before its stores (the stores could alias
+    // the loads as far as the compiler knows, so it would not move later loads above them)
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+        float4 v[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + kThreadsC * (4 * pass + i), r = e >> 4, n0 = 8 * (e & 15);
+            if (r < Qv && n0 < a.N) {
+                const float* row = a.U + (b * a.L + t0 + r) * conv_dim + HP + (int64_t)g * a.N + n0;
+                v[i][0] = *reinterpret_cast<const float4*>(row);
+                v[i][1] = *reinterpret_cast<const float4*>(row + 4);
+                v[i][2] = *reinterpret_cast<const float4*>(row + GN);
+                v[i][3] = *reinterpret_cast<const float4*>(row + GN + 4);
+            } else {
+                v[i][0] = v[i][1] = v[i][2] = v[i][3] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
-        const uint32_t off = (uint32_t)(k8 >> 3) * 8192u + sw128_off(r, k8 & 7);
-        *reinterpret_cast<uint4*>(sm + OFF_BT + off) = pb;
-        *reinterpret_cast<uint4*>(sm + OFF_CT + off) = pc;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + kThreadsC * (4 * pass + i), r = e >> 4, k8 = e & 15;
+            const uint32_t off = (uint32_t)(k8 >> 3) * 8192u + sw128_off(r, k8 & 7);
+            *reinterpret_cast<uint4*>(sm + OFF_BT + off) = pack8f(v[i][0], v[i][1], 1.f, range);
+            *reinterpret_cast<uint4*>(sm + OFF_CT + off) = pack8f(v[i][2], v[i][3], 1.f, range);
+        }
     }
-    // X' and G'' (64 rows x 8 chunks of 8 head channels)
+    // X' and G'' (64 rows x 8 chunks of 8 head channels; rows tid / 8 + 16 i), all loads first
     const float* dtp = a.DT + (b * a.H + h) * a.L + t0;
     const float* csp = a.CS + (b * a.H + h) * a.L + t0;
     const float cs_last = csp[Qv - 1];
-    for (int e = tid; e < kQc * (kPc / 8); e += kThreadsC) {
-        const int r = e >> 3, k8 = e & 7, p0 = 8 * k8;
-        uint4 px = make_uint4(0u, 0u, 0u, 0u), pg = px;
+    const int k8 = tid & 7, p0 = 8 * k8;
+    float4 xv[4][2], dyv[4][2];
+    uint4 zw[4];
+    float dtr[4], csr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = (tid >> 3) + 16 * i;
+        xv[i][0] = xv[i][1] = dyv[i][0] = dyv[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        zw[i] = make_uint4(0u, 0u, 0u, 0u);
+        dtr[i] = csr[i] = 0.f;
         if (r < Qv) {
-            const float fx = dtp[r] * expf(cs_last - csp[r]), fg = expf(csp[r]);
+            dtr[i] = dtp[r];
+            csr[i] = csp[r];
             const int64_t row = b * a.L + t0 + r;
             const float* xr = a.U + row * conv_dim + (int64_t)h * kPc + p0;
-            const float4 x0 = *reinterpret_cast<const float4*>(xr), x1 = *reinterpret_cast<const float4*>(xr + 4);
-            px = make_uint4(pack_h2(x0.x * fx, x0.y * fx, range), pack_h2(x0.z * fx, x0.w * fx, range),
-                            pack_h2(x1.x * fx, x1.y * fx, range), pack_h2(x1.z * fx, x1.w * fx, range));
+            xv[i][0] = *reinterpret_cast<const float4*>(xr);
+            xv[i][1] = *reinterpret_cast<const float4*>(xr + 4);
             const int64_t yi = row * HP + (int64_t)h * kPc + p0;
-            float gv[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) gv[k] = act_at(a.dy, yi + k, a.dy_bf16) * silu_c(act_at(a.z, yi + k, a.act_bf16)) * fg;
-            pg = make_uint4(pack_h2(gv[0], gv[1], range), pack_h2(gv[2], gv[3], range), pack_h2(gv[4], gv[5], range),
-                            pack_h2(gv[6], gv[7], range));
+            if (a.dy_bf16) {
+                const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(a.dy) + yi);
+                dyv[i][0] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+                dyv[i][1] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+            } else {
+                dyv[i][0] = *reinterpret_cast<const float4*>(static_cast<const float*>(a.dy) + yi);
+                dyv[i][1] = *reinterpret_cast<const float4*>(static_cast<const float*>(a.dy) + yi + 4);
+            }
+            zw[i] = *reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(a.z) + yi);
         }
-        *reinterpret_cast<uint4*>(sm + OFF_XW + sw128_off(r, k8)) = px;
-        *reinterpret_cast<uint4*>(sm + OFF_GW + sw128_off(r, k8)) = pg;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = (tid >> 3) + 16 * i;
+        const bool on = r < Qv;
+        const float fx = on ? dtr[i] * __expf(cs_last - csr[i]) : 0.f, fg = on ? __expf(csr[i]) : 0.f;
+        const float zf[8] = {bf_lo(zw[i].x), bf_hi(zw[i].x), bf_lo(zw[i].y), bf_hi(zw[i].y),
+                             bf_lo(zw[i].z), bf_hi(zw[i].z), bf_lo(zw[i].w), bf_hi(zw[i].w)};
+        const float dyf[8] = {dyv[i][0].x, dyv[i][0].y, dyv[i][0].z, dyv[i][0].w,
+                              dyv[i][1].x, dyv[i][1].y, dyv[i][1].z, dyv[i][1].w};
+        float4 g0, g1;
+        float* gp[8] = {&g0.x, &g0.y, &g0.z, &g0.w, &g1.x, &g1.y, &g1.z, &g1.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) *gp[q] = dyf[q] * zf[q] * __fdividef(1.f, 1.f + __expf(-zf[q]));
+        *reinterpret_cast<uint4*>(sm + OFF_XW + sw128_off(r, k8)) = pack8f(xv[i][0], xv[i][1], fx, range);
+        *reinterpret_cast<uint4*>(sm + OFF_GW + sw128_off(r, k8)) = pack8f(g0, g1, fg, range);
     }
     if (!(range < 65504.f)) atomicOr(&g_bwd_tc_error, 2);
     fence_async_smem();  // the tiles are read by the tensor cores (async proxy)

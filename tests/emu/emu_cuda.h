@@ -146,6 +146,8 @@ struct float2 {
     float x, y;
 };
 inline float4 make_float4(float a, float b, float c, float d) { return float4{a, b, c, d}; }
+inline float2 make_float2(float a, float b) { return float2{a, b}; }
+
 inline float4 __ldcs(const float4* p) { return *p; }
 inline void __stcs(float4* p, float4 v) { *p = v; }
 inline float __expf(float v) { return expf(v); }
@@ -160,6 +162,26 @@ inline __nv_bfloat16 __float2bfloat16_rn(float f) {
     if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) return __nv_bfloat16{(unsigned short)((u >> 16) | 0x40u)};
     u += 0x7fffu + ((u >> 16) & 1u);
     return __nv_bfloat16{(unsigned short)(u >> 16)};
+}
+
+// Warp broadcast: every lane of the warp posts its value and reads lane src's (all 32 lanes call it).
+inline float __shfl_sync(unsigned, float v, int src) {
+    ::emu::Ctx& c = ::emu::ctx;
+    c.warp_buf[c.lane] = v;
+    c.warp_bar->arrive_and_wait();
+    const float r = c.warp_buf[static_cast<unsigned>(src) & 31u];
+    c.warp_bar->arrive_and_wait();
+    return r;
+}
+
+// Warp shift: lane l reads lane l - delta's value (its own below delta); all 32 lanes call it.
+inline float __shfl_up_sync(unsigned, float v, int delta) {
+    ::emu::Ctx& c = ::emu::ctx;
+    c.warp_buf[c.lane] = v;
+    c.warp_bar->arrive_and_wait();
+    const float r = c.lane >= static_cast<unsigned>(delta) ? c.warp_buf[c.lane - delta] : v;
+    c.warp_bar->arrive_and_wait();
+    return r;
 }
 
 // Warp shuffle: every lane of the warp posts its value, waits for the others, reads its partner's.
