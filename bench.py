@@ -124,15 +124,15 @@ def backward_chunk_flops(d: Dims) -> int:
 def backward_chunk_bytes(d: Dims, act_bytes: int) -> int:
     """Algorithmic bytes of one launch of the tensor-core per-chunk backward (chunk_bwd_tc_kernel), Q = 64:
     reads the fp32 post-conv x, B, C, dt and in-chunk cumsum (workspace), dy and z and the raw dt (activation
-    dtype), the entering states and leaving adjoints (fp32 [nc][H][P][N] each) and the per-chunk F partials;
-    writes dz, the post-conv gradients of x (fp32), of B and C (fp32, one copy per half of each group's heads),
-    ddt and the per-chunk partials.  Each byte counted once."""
+    dtype), the entering states and leaving adjoints (the state pass's fp16 [nc][H][P][N] tiles, with an fp32
+    scale per row p) and the per-chunk F partials; writes dz, the post-conv gradients of x (fp32), of B and C
+    (fp32, one copy per half of each group's heads), ddt and the per-chunk partials.  Each byte counted once."""
     Q, P, N = BWD_Q, d.headdim, d.d_state
     rows, nc = d.batch * d.seqlen, d.batch * -(-d.seqlen // Q)
     HP, GN = d.nheads * P, d.ngroups * N
     halves = 2 if d.nheads // d.ngroups >= 2 else 1
     reads = rows * (HP + 2 * GN) * 4 + rows * 2 * d.nheads * 4 + rows * (2 * HP + d.nheads) * act_bytes + \
-        2 * nc * d.nheads * P * N * 4 + nc * d.nheads * 4 * 4
+        2 * nc * d.nheads * P * (N * 2 + 4) + nc * d.nheads * 4 * 4
     writes = rows * 2 * HP * 4 + halves * rows * 2 * GN * 4 + rows * d.nheads * 4 + nc * d.nheads * 3 * 4
     return reads + writes
 

@@ -88,6 +88,7 @@ const char* ssd_status_string(ssd_status s) {
         case SSD_ERR_CUDA: return "a CUDA runtime call failed";
         case SSD_ERR_WORKSPACE: return "workspace missing or too small";
         case SSD_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+        case SSD_ERR_RANGE: return "a backward operand beyond fp16 range (the gradients of that call are invalid)";
     }
     return "unknown status";
 }

@@ -40,8 +40,8 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings_and_version(L):
-    for code in range(0, 9):
-        assert L.ssd_status_string(code)
+    for code in range(0, 10):
+        assert L.ssd_status_string(code) and L.ssd_status_string(code) != b"unknown status"
     assert b"sm_100a" in L.ssd_version()
 
 

@@ -73,10 +73,10 @@ def test_backward_work_counts():
     per_head = 8 * 64 * 64 * 128 + 4 * 64 * 64 * 64 + 2 * 64 * 64 * 128
     assert bench.backward_chunk_flops(d) == 64 * (128 * per_head + 8 * 2 * 64 * 64 * 128)
     assert abs(bench.FP32_ALU_TFLOPS - 74.45) < 0.01
-    # the tensor-core chunk backward: fp32 post-conv x|B|C, dt, cs; bf16 dy, z, dt; fp32 states and adjoints;
-    # dz, dx, two halves of dB|dC, ddt written (fp32), and the small per-chunk partials
+    # the tensor-core chunk backward: fp32 post-conv x|B|C, dt, cs; bf16 dy, z, dt; fp16 states and adjoints
+    # with an fp32 scale per state row; dz, dx, two halves of dB|dC, ddt written (fp32), the per-chunk partials
     reads = 4096 * (8192 + 2048) * 4 + 4096 * 2 * 128 * 4 + 4096 * (2 * 8192 + 128) * 2 + \
-        2 * 64 * 128 * 64 * 128 * 4 + 64 * 128 * 16
+        2 * 64 * 128 * 64 * (128 * 2 + 4) + 64 * 128 * 16
     writes = 4096 * 2 * 8192 * 4 + 2 * 4096 * 2048 * 4 + 4096 * 128 * 4 + 64 * 128 * 12
     assert bench.backward_chunk_bytes(d, 2) == reads + writes
 

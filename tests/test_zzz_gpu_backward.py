@@ -114,3 +114,24 @@ def test_backward_without_initial_state_gradients():
     got = gpu_backward(dev_inputs(inp), gr["dy"].cuda(), None, want_init=False)
     assert "init_state" not in got and "init_conv_state" not in got
     compare(got, oracle.prefill_backward(inp, gr["dy"], None), "no initial-state gradients")
+
+
+def test_backward_reports_fp16_range():
+    # post-conv activations beyond fp16's range (bf16 holds them): the tensor-core kernels' fp16 operands
+    # cannot, and ssd_device_status says so (SSD_ERR_RANGE) instead of the call passing silently; the flag
+    # is cleared by the report
+    d = Dims(1, 128, 4, 64, 64, 2, 128)
+    inp = make_prefill_inputs(d, dtype=torch.bfloat16, seed=11)
+    inp["x"] = (inp["x"].float() * 1e7).to(torch.bfloat16)
+    gr = make_backward_grads(d, dtype=torch.bfloat16, seed=12)
+    dev = dev_inputs(inp)
+    ops.device_status()
+    gpu_backward(dev, gr["dy"].cuda(), gr["d_final"].cuda())
+    with pytest.raises(ops.SsdError) as err:
+        ops.device_status()
+    assert err.value.status == 9  # SSD_ERR_RANGE
+    ops.device_status()
+    # in-range inputs on the same path report nothing
+    inp2 = make_prefill_inputs(d, dtype=torch.bfloat16, seed=13)
+    gpu_backward(dev_inputs(inp2), gr["dy"].cuda(), gr["d_final"].cuda())
+    ops.device_status()
