@@ -605,10 +605,13 @@ def bench_prefill(run: PrefillRun, dev, flush, K: int, warmup: int, world: int, 
 
 
 def link_bandwidth(dev, nbytes: int = 256 << 20):
-    """One pinned host -> device and one device -> host copy of ``nbytes``, timed with CUDA events: the
-    link the end-to-end number is bound by."""
+    """Pinned host -> device and device -> host copies of ``nbytes``, timed with CUDA events: each direction
+    alone, then both at once on two streams (the PCIe link is full duplex, but each direction slows while
+    the other runs)."""
     h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    h2 = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
     dbuf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dbuf2 = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     out = {}
     for name, fn in (("h2d_gbs", lambda: dbuf.copy_(h, non_blocking=True)),
                      ("d2h_gbs", lambda: h.copy_(dbuf, non_blocking=True))):
@@ -621,7 +624,33 @@ def link_bandwidth(dev, nbytes: int = 256 << 20):
         e.record()
         torch.cuda.synchronize(dev)
         out[name] = 3 * nbytes / (s.elapsed_time(e) * 1e-3) / 1e9
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+    s = torch.cuda.Event(enable_timing=True)
+    e_in, e_out = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    s_in.wait_stream(cur)
+    s_out.wait_stream(cur)
+    with torch.cuda.stream(s_in):
+        dbuf.copy_(h, non_blocking=True)
+        e_in.record()
+    with torch.cuda.stream(s_out):
+        h2.copy_(dbuf2, non_blocking=True)
+        e_out.record()
+    torch.cuda.synchronize(dev)
+    # both streams run the whole time only until the first of them finishes: rate = bytes / own time
+    out["h2d_both_gbs"] = nbytes / (s.elapsed_time(e_in) * 1e-3) / 1e9
+    out["d2h_both_gbs"] = nbytes / (s.elapsed_time(e_out) * 1e-3) / 1e9
     return out
+
+
+def link_floor_bidir_ms(h2d: int, d2h: int, link: dict) -> float:
+    """The shortest time to move h2d bytes in and d2h bytes out over the link: both directions at once for as
+    long as both have bytes left, then the remainder alone (each direction's rates from link_bandwidth)."""
+    t_both = min(h2d / (link["h2d_both_gbs"] * 1e9), d2h / (link["d2h_both_gbs"] * 1e9))
+    rest_in = h2d - link["h2d_both_gbs"] * 1e9 * t_both
+    rest_out = d2h - link["d2h_both_gbs"] * 1e9 * t_both
+    return (t_both + rest_in / (link["h2d_gbs"] * 1e9) + rest_out / (link["d2h_gbs"] * 1e9)) * 1e3
 
 
 def bench_e2e(ops, run: PrefillRun, dev, K: int, world: int, sampler):
@@ -630,7 +659,7 @@ def bench_e2e(ops, run: PrefillRun, dev, K: int, world: int, sampler):
     host = {k: (None if v is None else v.pin_memory()) for k, v in run.inp.items()}
     # the outputs' pinned host buffers are allocated once and reused, as a serving loop would
     outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (run.y, run.fs, run.cs)]
-    segments = None   # the API's default: up to 8 pieces overlapped on three streams
+    segments = None   # the API's default: about 8 pieces overlapped on three streams
     try:
         for _ in range(3):
             ops.prefill_host(host, chunk=d.chunk, device=dev, segments=segments, out=outs)
@@ -659,11 +688,13 @@ def bench_e2e(ops, run: PrefillRun, dev, K: int, world: int, sampler):
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": KE, "workload": run.w["desc"],
             "link": link,
             "link_floor_ms": max(h2d / link["h2d_gbs"], d2h / link["d2h_gbs"]) / 1e6,
+            "link_floor_bidir_ms": link_floor_bidir_ms(h2d, d2h, link),
             "how": "ops.prefill_host: pinned host inputs -> device, ssd_prefill, outputs -> pinned host buffers "
                    "reused across steps; "
                    + ("one piece on one stream" if segments == 1 else
-                      "the sequence in up to 8 chunk-aligned pieces, copies in, scans and copies out "
-                      "overlapped on three streams, states chained piece to piece")
+                      "about 8 pieces of one sequence and a chunk-aligned token range (one contiguous copy per "
+                      "tensor), copies in, scans and copies out overlapped on three streams, states chained "
+                      "along each sequence")
                    + "; CUDA events on the calling stream around the whole call"}
 
 

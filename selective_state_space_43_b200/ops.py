@@ -610,21 +610,25 @@ def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None, out=None
     ``out`` = (y, final_state, conv_state) when given (reused across calls, no host allocation), else new
     ones (a pinned allocation of y's size per call).
 
-    The sequence is cut into ``segments`` pieces on chunk boundaries (default: up to 8 pieces of at least
-    two chunks).  Piece k is copied in on one side stream while piece k-1 is scanned on the current stream
-    and piece k-2's y is copied out on another, so the two copy directions and the scan overlap.  Each piece
-    starts from the states the previous one left (final_state and conv_state as init_state and
-    init_conv_state), which on chunk boundaries gives the same values as one call over the whole sequence.
-    The current stream waits for every copy before the call returns, so events recorded on it around the
-    call time the whole transfer.  Returns ([y, final_state, conv_state] on the host, bytes in, bytes out).
+    The work is cut into pieces of one sequence (batch row) and a chunk-aligned token range: ``segments``
+    ranges per sequence (default: about eight pieces in all, each at least two chunks long), so every
+    tensor of a piece is one contiguous host range and moves in one copy.  Piece k is copied in on one
+    side stream while piece k-1 is scanned on the current stream and piece k-2's y is copied out on
+    another, so the two copy directions and the scan overlap.  A piece starts from the states the previous
+    piece of its sequence left (final_state and conv_state as init_state and init_conv_state), which on
+    chunk boundaries gives the same values as one call over the whole sequence.  The current stream waits
+    for every copy before the call returns, so events recorded on it around the call time the whole
+    transfer.  Returns ([y, final_state, conv_state] on the host, bytes in, bytes out).
     """
     dev = torch.device(device)
     x = inputs["x"]
     Bt, L = x.shape[0], x.shape[1]
     h2d = sum(t.numel() * t.element_size() for t in inputs.values() if t is not None)
-    pieces = host_pieces(L, chunk, segments)
+    if segments is None:
+        segments = max(1, min(L // (2 * chunk), -(-8 // max(Bt, 1))))
+    ranges = host_pieces(L, chunk, segments)
     y_host, fs_host, cs_host = _host_outputs(inputs, out)
-    if len(pieces) <= 1:
+    if Bt * len(ranges) <= 1:
         return _prefill_host_whole(inputs, chunk, dev, h2d, (y_host, fs_host, cs_host))
 
     cur = torch.cuda.current_stream(dev)
@@ -637,36 +641,30 @@ def prefill_host(inputs: dict, chunk=128, device="cuda", segments=None, out=None
     for t in p.values():
         if t is not None:
             t.record_stream(cur)
-    fs_prev, cs_prev = p["init_state"], p["init_conv_state"]
-    for r0, r1 in pieces:
-        with torch.cuda.stream(s_in):
-            d = {}
-            for k in ("x", "dt", "B", "C", "z"):
-                h = inputs[k]
-                t = torch.empty((Bt, r1 - r0) + tuple(h.shape[2:]), dtype=h.dtype, device=dev)
-                for b in range(Bt):
-                    t[b].copy_(h[b, r0:r1], non_blocking=True)
-                d[k] = t
-            ready = torch.cuda.Event()
-            ready.record(s_in)
-        cur.wait_event(ready)
-        for t in d.values():
-            t.record_stream(cur)
-        y, fs, cs = prefill(d["x"], d["dt"], d["B"], d["C"], d["z"], p["A"], p["D"], p["dt_bias"], p["conv_w"],
-                            p["conv_b"], fs_prev, cs_prev, chunk=chunk)
-        done = torch.cuda.Event()
-        done.record(cur)
-        s_out.wait_event(done)
-        with torch.cuda.stream(s_out):
-            for b in range(Bt):
-                y_host[b, r0:r1].copy_(y[b], non_blocking=True)
-        y.record_stream(s_out)
-        fs_prev, cs_prev = fs, cs
-    with torch.cuda.stream(s_out):
-        fs_host.copy_(fs_prev, non_blocking=True)
-        cs_host.copy_(cs_prev, non_blocking=True)
-    fs_prev.record_stream(s_out)
-    cs_prev.record_stream(s_out)
+    for b in range(Bt):
+        fs_prev = None if p["init_state"] is None else p["init_state"][b:b + 1]
+        cs_prev = None if p["init_conv_state"] is None else p["init_conv_state"][b:b + 1]
+        for r0, r1 in ranges:
+            with torch.cuda.stream(s_in):
+                d = {k: inputs[k][b:b + 1, r0:r1].to(dev, non_blocking=True) for k in ("x", "dt", "B", "C", "z")}
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            cur.wait_event(ready)
+            for t in d.values():
+                t.record_stream(cur)
+            y, fs, cs = prefill(d["x"], d["dt"], d["B"], d["C"], d["z"], p["A"], p["D"], p["dt_bias"], p["conv_w"],
+                                p["conv_b"], fs_prev, cs_prev, chunk=chunk)
+            done = torch.cuda.Event()
+            done.record(cur)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                y_host[b, r0:r1].copy_(y[0], non_blocking=True)
+                if r1 == L:
+                    fs_host[b].copy_(fs[0], non_blocking=True)
+                    cs_host[b].copy_(cs[0], non_blocking=True)
+            for t in (y, fs, cs):
+                t.record_stream(s_out)
+            fs_prev, cs_prev = fs, cs
     out_done = torch.cuda.Event()
     out_done.record(s_out)
     cur.wait_event(out_done)

@@ -201,3 +201,13 @@ def test_headline_is_the_largest_single_gpu_prefill_workload():
     nbytes = {n: bench.prefill_bytes(WORKLOADS[n]["dims"], 2, WORKLOADS[n]["init_state"]) for n in prefill}
     assert bench.HEADLINE_WORKLOAD == max(prefill, key=lambda n: (nbytes[n], tokens[n]))
     assert set(bench.OTHER_PREFILL_WORKLOADS) == set(prefill) - {bench.HEADLINE_WORKLOAD}
+
+
+def test_bidirectional_link_floor():
+    # no slowdown when both directions run: the floor is the longer direction alone
+    same = {"h2d_gbs": 50.0, "d2h_gbs": 40.0, "h2d_both_gbs": 50.0, "d2h_both_gbs": 40.0}
+    assert abs(bench.link_floor_bidir_ms(500e6, 200e6, same) - 10.0) < 1e-9
+    # both directions at half rate while together: 100 MB out overlaps 4 ms of the way in
+    slow = {"h2d_gbs": 50.0, "d2h_gbs": 50.0, "h2d_both_gbs": 25.0, "d2h_both_gbs": 25.0}
+    # together 4 ms (100 MB in, 100 MB out), then 400 MB in alone at 50 GB/s = 8 ms
+    assert abs(bench.link_floor_bidir_ms(500e6, 100e6, slow) - 12.0) < 1e-9
