@@ -76,7 +76,7 @@ bool chunk_bwd_tc_supported(int P, int N, bool act_bf16, const void* dy, const v
 cudaError_t launch_chunk_bwd_tc(const ChunkBwdTcArgs& a, int64_t nchunks, cudaStream_t st);
 #endif
 
-constexpr int kQ = 64;    // backward chunk (tokens); also the conv backward's tile
+constexpr int kQ = 64;    // backward chunk (tokens)
 constexpr int kT = 256;   // threads per block
 constexpr int kP = 64;    // head dimension
 constexpr int kS = kQ + 4;  // row stride of the 64-wide shared tiles: a multiple of 4 floats (16-byte rows)
@@ -107,7 +107,8 @@ struct Ws {
 namespace {
 
 __host__ __device__ inline int64_t nchunks(int64_t L) { return (L + kQ - 1) / kQ; }
-__host__ __device__ inline int64_t ntiles(int64_t L) { return L > 0 ? nchunks(L) : 1; }
+constexpr int kCT = 32;   // tokens per tile of the two conv kernels (twice the threads of a 64-token tile)
+__host__ __device__ inline int64_t ntiles(int64_t L) { return L > 0 ? (L + kCT - 1) / kCT : 1; }
 // CTAs per (chunk, group) in the chunk backward: the group's heads in two halves when there are two or more
 __host__ __device__ inline int head_split(int H, int G) { return H / G >= 2 ? 2 : 1; }
 inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -178,15 +179,15 @@ __device__ __forceinline__ float2 raw_pair(const BwdArgs& a, const ChanPair& q, 
     return *reinterpret_cast<const float2*>(static_cast<const float*>(q.src) + i);
 }
 
-// grid (ceil(conv_dim / (kT * kCPT)), nchunks, batch): one thread per (pair of channels, 64-token tile), streaming
+// grid (ceil(conv_dim / (kT * kCPT)), ntiles, batch): one thread per (pair of channels, kCT-token tile), streaming
 // the tile with kBatch tokens' inputs loaded before their outputs are stored (the stores could alias the
 // inputs as far as the compiler knows, so it would not move later loads above them).
 __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
     const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N;
     const int64_t c = ((int64_t)blockIdx.x * kT + threadIdx.x) * kCPT;
     if (c >= conv_dim) return;
-    const int64_t b = blockIdx.z, t0 = (int64_t)blockIdx.y * kQ;
-    const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
+    const int64_t b = blockIdx.z, t0 = (int64_t)blockIdx.y * kCT;
+    const int64_t t1 = t0 + kCT < a.L ? t0 + kCT : a.L;
     float w[2][4], bias[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -1014,15 +1015,15 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     }
 }
 
-// grid (ceil(conv_dim / kT), ntiles, batch): one thread per (channel, 64-token tile).
+// grid (ceil(conv_dim / kT), ntiles, batch): one thread per (channel, kCT-token tile).
 // Streams t over the tile and the 3 tokens after it: dv_t = du_t silu'(v_t), and the pre-conv
 // gradient of token s = t - 3 is w0 dv_t + w1 dv_{t-1} + w2 dv_{t-2} + w3 dv_{t-3}.
 __global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
     const int64_t HP = (int64_t)a.H * a.P, GN = (int64_t)a.G * a.N, conv_dim = HP + 2 * GN;
     const int64_t c = (int64_t)blockIdx.x * kT + threadIdx.x;
     if (c >= conv_dim) return;
-    const int64_t b = blockIdx.z, tile = blockIdx.y, nt = ntiles(a.L), t0 = tile * kQ;
-    const int64_t t1 = t0 + kQ < a.L ? t0 + kQ : a.L;
+    const int64_t b = blockIdx.z, tile = blockIdx.y, nt = ntiles(a.L), t0 = tile * kCT;
+    const int64_t t1 = t0 + kCT < a.L ? t0 + kCT : a.L;
     const float w0 = a.conv_w[c * 4 + 0], w1 = a.conv_w[c * 4 + 1], w2 = a.conv_w[c * 4 + 2],
                 w3 = a.conv_w[c * 4 + 3], bias = a.conv_b[c];
     // this channel's input array and gradient array (x / B / C and dx / dB / dC), row stride, column
@@ -1100,31 +1101,51 @@ __global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
     pw[4] = gb;
 }
 
-// grid ceil((conv_dim + H) / kT): per channel the conv parameter gradients, per head dA, dD, ddt_bias;
-// partials summed in (batch, tile) order.
+// grid (ceil(conv_dim / 32) + ceil(H / 32)), kT threads: 32 channels (or heads) per CTA, each summed by
+// 8 threads over the tiles (chunks) t = j, j + 8, ... of every sequence, then the 8 partials in a fixed order
+// -> dconv_w, dconv_b per channel; dA, dD, ddt_bias per head (deterministic).
 __global__ void __launch_bounds__(kT) reduce_kernel(BwdArgs a, Ws ws) {
+    constexpr int NJ = kT / 32;
+    float(*part)[NJ][32] = reinterpret_cast<float(*)[NJ][32]>(SSD_DYN_SMEM());  // [5][NJ][32]
     const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N, nc = nchunks(a.L), nt = ntiles(a.L);
-    const int64_t idx = (int64_t)blockIdx.x * kT + threadIdx.x;
-    if (idx < conv_dim) {
-        float s[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int64_t b = 0; b < a.batch; ++b)
-            for (int64_t t = 0; t < nt; ++t) {
-                const float* pw = ws.PW + ((b * nt + t) * conv_dim + idx) * 5;
-                for (int k = 0; k < 5; ++k) s[k] += pw[k];
+    const int64_t cblocks = (conv_dim + 31) / 32;
+    const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;
+    const bool heads = blockIdx.x >= cblocks;
+    const int64_t idx = (heads ? blockIdx.x - cblocks : blockIdx.x) * 32 + lane;
+    const int K = heads ? 3 : 5;
+    const int64_t limit = heads ? a.H : conv_dim;
+    float s[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+    if (idx < limit) {
+        for (int64_t b = 0; b < a.batch; ++b) {
+            if (heads) {
+                for (int64_t c = j; c < nc; c += NJ) {
+                    const float* ph = ws.PH + ((b * nc + c) * a.H + idx) * 3;
+                    for (int k = 0; k < 3; ++k) s[k] += ph[k];
+                }
+            } else {
+                for (int64_t t = j; t < nt; t += NJ) {
+                    const float* pw = ws.PW + ((b * nt + t) * conv_dim + idx) * 5;
+                    for (int k = 0; k < 5; ++k) s[k] += pw[k];
+                }
             }
-        for (int k = 0; k < 4; ++k) a.dconv_w[idx * 4 + k] = s[k];
-        a.dconv_b[idx] = s[4];
-    } else if (idx < conv_dim + a.H) {
-        const int64_t h = idx - conv_dim;
-        float s[3] = {0.f, 0.f, 0.f};
-        for (int64_t b = 0; b < a.batch; ++b)
-            for (int64_t c = 0; c < nc; ++c) {
-                const float* ph = ws.PH + ((b * nc + c) * a.H + h) * 3;
-                for (int k = 0; k < 3; ++k) s[k] += ph[k];
-            }
-        a.dA[h] = s[0];
-        a.dD[h] = s[1];
-        a.ddt_bias[h] = s[2];
+        }
+    }
+    for (int k = 0; k < 5; ++k) part[k][j][lane] = s[k];
+    __syncthreads();
+    if (j == 0 && idx < limit) {
+        float t[5];
+        for (int k = 0; k < K; ++k) {
+            t[k] = 0.f;
+            for (int q = 0; q < NJ; ++q) t[k] += part[k][q][lane];
+        }
+        if (heads) {
+            a.dA[idx] = t[0];
+            a.dD[idx] = t[1];
+            a.ddt_bias[idx] = t[2];
+        } else {
+            for (int k = 0; k < 4; ++k) a.dconv_w[idx * 4 + k] = t[k];
+            a.dconv_b[idx] = t[4];
+        }
     }
 }
 
@@ -1145,7 +1166,7 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         const size_t chunk_smem = chunk_bwd_floats<N>() * sizeof(float);
         if ((err = SSD_SET_SMEM(chunk_state_kernel<N>, state_smem)) != cudaSuccess) return err;
         if ((err = SSD_SET_SMEM(chunk_bwd_kernel<N>, chunk_smem)) != cudaSuccess) return err;
-        const dim3 tiles(cgrid, static_cast<unsigned>(nc), static_cast<unsigned>(a.batch));
+        const dim3 tiles(cgrid, static_cast<unsigned>(ntiles(a.L)), static_cast<unsigned>(a.batch));
         SSD_LAUNCH(post_conv_kernel, tiles, dim3(kT), 0, st, a, ws);
         SSD_LAUNCH(dt_kernel,
                    dim3(static_cast<unsigned>(nc), static_cast<unsigned>((a.H + kT / 32 - 1) / (kT / 32)),
@@ -1201,7 +1222,8 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
                    dim3(static_cast<unsigned>((conv_dim + kT - 1) / kT), static_cast<unsigned>(nt),
                         static_cast<unsigned>(a.batch)),
                    dim3(kT), 0, st, a, ws);
-    SSD_LAUNCH(reduce_kernel, dim3(static_cast<unsigned>((conv_dim + a.H + kT - 1) / kT)), dim3(kT), 0, st, a, ws);
+    SSD_LAUNCH(reduce_kernel, dim3(static_cast<unsigned>((conv_dim + 31) / 32 + (a.H + 31) / 32)), dim3(kT),
+               5 * (size_t)kT * sizeof(float), st, a, ws);
     return cudaGetLastError();
 }
 
