@@ -20,8 +20,8 @@ SRC = os.path.join(emu_harness.CSRC, "ssd_backward.cu")
 
 MUTANTS = {
     # reads x one token past the tile: beyond the array for the last tile of the last sequence
-    "post-conv reads past its tile": ("rin[i] = tb + i < t1 ? raw_at(a, b, tb + i, c) : 0.f;",
-                                      "rin[i] = tb + i < t1 ? raw_at(a, b, tb + i + 1, c) : 0.f;"),
+    "post-conv reads past its tile": ("rin[i] = tb + i < t1 ? raw_pair(a, q, b, tb + i, c) : make_float2(0.f, 0.f);",
+                                      "rin[i] = tb + i < t1 ? raw_pair(a, q, b, tb + i + 1, c) : make_float2(0.f, 0.f);"),
     # writes each pre-conv gradient one token late: beyond dx / dB / dC for the last token
     "conv backward writes one row late": ("out[(row0 + s) * ostride + ocol] = gs;",
                                           "out[(row0 + s + 1) * ostride + ocol] = gs;"),
