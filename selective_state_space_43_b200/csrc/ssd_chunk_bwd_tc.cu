@@ -27,14 +27,15 @@
 // cannot hold (>= 65504) sets bit 1 of this file's error word (SSD_ERR_RANGE).  The elementwise terms
 // read x, g and dy silu'(z) back from the same fp16 tiles the MMAs use.
 //
-// One CTA per (chunk, group, half of the group's heads), heads in turn; 384 threads in four roles:
-//   row warps 0, 1, 4, 5  (TMEM lanes 0..63 = the chunk's tokens; warps 0/4 tokens 0..31, 1/5 tokens
-//                         32..63; warps 0, 1 columns 0..31, warps 4, 5 columns 32..63): the elementwise
-//                         work above, the LCB / LGX' tiles, dz, dx and per-row partial sums;
+// One CTA per (chunk, group, half of the group's heads), heads in turn; 512 threads in four roles:
+//   row warps 0, 1, 4, 5, 8, 9, 12, 13 (TMEM lanes 0..63 = the chunk's tokens; warp w takes tokens
+//                         32 (w & 3) .. +31 and columns 16 (w >> 2) .. +15): the elementwise work above,
+//                         the LCB / LGX' tiles, dz, dx and per-row partial sums (16 columns a thread keeps
+//                         each thread's dependent chains short; 16 warps cap registers at 128);
 //   loader warps 2, 3, 6, 7, 10, 11: the head's tiles, two heads deep: Sp and Lm by bulk copy, x, X', g, G''
 //                         and dy silu'(z) converted from global memory;
-//   warp 8              : TMEM allocation and, on one thread, the MMAs;
-//   warp 9              : each head's per-token scalars from the partial sums (the prefix / suffix sums
+//   warp 14             : TMEM allocation and, on one thread, the MMAs;
+//   warp 15             : each head's per-token scalars from the partial sums (the prefix / suffix sums
 //                         behind d(dA), ddt) and the per-chunk partials of dA, dD, ddt_bias.
 // Every MMA is M = 128, N = 64 with fp32 accumulators in TMEM (512 columns: CB, GX, SPC, LMB, YIN, DXI,
 // dB^T, dC^T).  The token-major products use only rows 0..63 of their 128-row result: the A tile's rows
@@ -61,7 +62,9 @@ using namespace sm100;
 
 constexpr int kQb = 64;   // chunk (tokens)
 constexpr int kPb = 64;   // head dimension
-constexpr int kThreadsB = 384;
+constexpr int kThreadsB = 512;
+constexpr int kRows = 256;     // row threads (warps 0, 1, 4, 5, 8, 9, 12, 13)
+constexpr int kWarpMma = 14, kWarpScalar = 15;
 constexpr int kLoaders = 192;  // loader threads (warps 2, 3, 6, 7, 10, 11)
 constexpr int kSplitPf = 4;    // partial sums of F per (chunk, head) from the state pass
 
@@ -84,12 +87,12 @@ constexpr uint32_t OFF_VEC = OFF_BUF + 2 * BUF_BYTES;  // fp32 vectors:
 constexpr uint32_t V_DT = 0;            //   dt [2 buffers][64]
 constexpr uint32_t V_CS = 512;          //   cs [2][64]
 constexpr uint32_t V_COL = 1024;        //   column sums of GX L CB [2 head parities][2 token halves][64]
-constexpr uint32_t V_ROWM = 2048;       //   row sums of M [2][2 column halves][64]
-constexpr uint32_t V_E = 3072;          //   g_i . SPC_i partials [2][2][64]
-constexpr uint32_t V_W = 4096;          //   W_j partials [2][2][64]
-constexpr uint32_t V_PD = 5120;         //   sum g . x per row warp [2][4]
-constexpr uint32_t V_ISC = 5248;        //   inverse row scales of each buffer's Sp, Lm tiles [2][2][64]
-constexpr uint32_t VEC_BYTES = 6272;
+constexpr uint32_t V_ROWM = 2048;       //   row sums of M [2][4 column quarters][64]
+constexpr uint32_t V_E = 4096;          //   g_i . SPC_i partials [2][4][64]
+constexpr uint32_t V_W = 6144;          //   W_j partials [2][4][64]
+constexpr uint32_t V_PD = 8192;         //   sum g . x per row warp [2][8]
+constexpr uint32_t V_ISC = 8256;        //   inverse row scales of each buffer's Sp, Lm tiles [2][2][64]
+constexpr uint32_t VEC_BYTES = 9280;
 constexpr uint32_t OFF_BAR = OFF_VEC + VEC_BYTES;
 enum : int { TILE_FULL0, TILE_FULL1, TILE_FREE0, TILE_FREE1, SPLM_FULL0, SPLM_FULL1, GX_DONE, B1_DONE, LT_FULL,
              B2_DONE, ACC_FREE, WSYNC, SCALAR_FREE, FINAL, NBAR };
@@ -208,11 +211,14 @@ __device__ __forceinline__ void give_up(volatile int* abort) {
     atomicOr(&g_chunk_bwd_tc_error, 1);
 }
 
-// Sum over the warp's 32 lanes of each of v[0..31]: lane l ends with the sum of v[l] (butterfly; at each
-// step a lane keeps the half of its values whose index bit matches its lane bit and adds the partner's).
-__device__ __forceinline__ float column_sums(float (&v)[32], int lane) {
+// Sum over the warp's 32 lanes of each of v[0..15]: lane l ends with the sum of v[l & 15] (both halves
+// of the warp add up, then a butterfly: at each step a lane keeps the half of its values whose index bit
+// matches its lane bit and adds the partner's).
+__device__ __forceinline__ float column_sums16(float (&v)[16], int lane) {
 #pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
+    for (int i = 0; i < 16; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 16);
+#pragma unroll
+    for (int s = 8; s >= 1; s >>= 1) {
         const bool up = (lane & s) != 0;
 #pragma unroll
         for (int i = 0; i < s; ++i) {
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
     const int64_t HP = (int64_t)a.H * kPb, GN = (int64_t)a.G * N, conv_dim = HP + 2 * GN;
     const int64_t row0 = b * a.L + t0;  // first token row of the chunk
 
-    if (warp == 8) {
+    if (warp == kWarpMma) {
         tmem_alloc(tm_holder, TMEM_COLS_B);
         tmem_relinquish();
     }
@@ -272,16 +278,16 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
         *abort = 0;
         mbar_init(&bars[TILE_FULL0], kLoaders);
         mbar_init(&bars[TILE_FULL1], kLoaders);
-        mbar_init(&bars[TILE_FREE0], 1 + 128 + 32);  // the MMAs' commit, the row threads, the scalar warp
-        mbar_init(&bars[TILE_FREE1], 1 + 128 + 32);
+        mbar_init(&bars[TILE_FREE0], 1 + kRows + 32);  // the MMAs' commit, the row threads, the scalar warp
+        mbar_init(&bars[TILE_FREE1], 1 + kRows + 32);
         mbar_init(&bars[SPLM_FULL0], 1);    // the bulk copies' transaction bytes
         mbar_init(&bars[SPLM_FULL1], 1);
         mbar_init(&bars[GX_DONE], 1);
         mbar_init(&bars[B1_DONE], 1);
-        mbar_init(&bars[LT_FULL], 128);
+        mbar_init(&bars[LT_FULL], kRows);
         mbar_init(&bars[B2_DONE], 1);
-        mbar_init(&bars[ACC_FREE], 128);
-        mbar_init(&bars[WSYNC], 128);
+        mbar_init(&bars[ACC_FREE], kRows);
+        mbar_init(&bars[WSYNC], kRows);
         mbar_init(&bars[SCALAR_FREE], 32);
         mbar_init(&bars[FINAL], 1);
         fence_mbar_init();
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
     tc_fence_after();
     const uint32_t tmem = *tm_holder;
 
-    if (warp == 8) {
+    if (warp == kWarpMma) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             mma_steps(tmem + COL_CB, kdesc(sm + OFF_TC), false, kdesc(sm + OFF_TB), false, ID_KK, 4 * nbox, false);
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             mma_commit(&bars[FINAL]);  // every MMA issued so far
         }
         __syncwarp();
-    } else if (warp == 9) {
+    } else if (warp == kWarpScalar) {
         // ---------------- scalar warp: each head's ddt and per-chunk partial sums (tokens lane, lane + 32) -------
         bool ok = true;
         for (int k = 0; k < nh && ok; ++k) {
@@ -366,21 +372,23 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                 break;
             }
             const float* col = vec + (V_COL >> 2) + par * 128;
-            const float* rwm = vec + (V_ROWM >> 2) + par * 128;
-            const float* ev = vec + (V_E >> 2) + par * 128;
-            const float* wv = vec + (V_W >> 2) + par * 128;
-            const float* pdw = vec + (V_PD >> 2) + par * 4;
+            const float* rwm = vec + (V_ROWM >> 2) + par * 256;
+            const float* ev = vec + (V_E >> 2) + par * 256;
+            const float* wv = vec + (V_W >> 2) + par * 256;
+            const float* pdw = vec + (V_PD >> 2) + par * 8;
+            // the four column quarters' partial sums of token kk, in a fixed order
+            auto q4 = [](const float* v, int kk) { return (v[kk] + v[64 + kk]) + (v[128 + kk] + v[192 + kk]); };
             float dr0[2], d[2], e[2], w[2], dw[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int kk = lane + 32 * u;
                 dr0[u] = col[kk] + col[64 + kk];
-                d[u] = dtk[u] * dr0[u] - (rwm[kk] + rwm[64 + kk]);
-                e[u] = exk[u] * (ev[kk] + ev[64 + kk]);
-                w[u] = wv[kk] + wv[64 + kk];
+                d[u] = dtk[u] * dr0[u] - q4(rwm, kk);
+                e[u] = exk[u] * q4(ev, kk);
+                w[u] = q4(wv, kk);
                 dw[u] = dtk[u] * w[u];
             }
-            const float pD = (pdw[0] + pdw[1]) + (pdw[2] + pdw[3]);
+            const float pD = ((pdw[0] + pdw[1]) + (pdw[2] + pdw[3])) + ((pdw[4] + pdw[5]) + (pdw[6] + pdw[7]));
             __syncwarp();
             mbar_arrive(&bars[SCALAR_FREE]);  // the partial sums are read: the row warps may write the next ones
             // exclusive prefix sums of d and dt W, inclusive suffix sums of E, over the 64 tokens
@@ -416,7 +424,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
         }
         if (!ok) give_up(abort);
     } else if ((warp & 3) >= 2) {
-        // ---------------- loaders: warps 2, 3, 6, 7, 10, 11 ----------------
+        // ---------------- loaders: warps 2, 3, 6, 7, 10, 11 (14 and 15 took the branches above) ----------------
         const int lt = ((warp >> 2) * 2 + (warp & 3) - 2) * 32 + lane;  // 0..kLoaders-1
         const int k8 = lt & 7;  // this thread's 16-byte chunk (8 head channels) of rows lt / 8 + 24 m
         for (int k = 0; k < nh; ++k) {
@@ -498,11 +506,11 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             mbar_arrive(&bars[TILE_FULL0 + buf]);
         }
     } else {
-        // ---------------- row warps 0, 1, 4, 5 ----------------
+        // ---------------- row warps 0, 1, 4, 5, 8, 9, 12, 13 ----------------
         const int rq = warp & 3;           // token half: rows 32 rq .. 32 rq + 31
-        const int ch = warp >> 2;          // column half: 32 ch .. 32 ch + 31
-        const int r = 32 * rq + lane, c0 = 32 * ch;
-        const int wi = rq + 2 * ch;        // 0..3
+        const int cq = warp >> 2;          // column quarter: 16 cq .. 16 cq + 15
+        const int r = 32 * rq + lane, c0 = 16 * cq;
+        const int wi = rq + 2 * cq;        // 0..7
         const uint32_t lb = (uint32_t)(32 * rq) << 16;
         bool ok = true;
         for (int k = 0; k < nh && ok; ++k) {
@@ -525,12 +533,12 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             // phase B: LCB and LGX' rows, the row sums of M and the column sums of GX L CB
             float rowm = 0.f, range = 0.f;
             {
-                float gx[32], cb[32];
-                tmem_ld32(tmem + lb + COL_GX + c0, gx);
-                tmem_ld32(tmem + lb + COL_CB + c0, cb);
+                float gx[16], cb[16];
+                tmem_ld16(tmem + lb + COL_GX + c0, gx);
+                tmem_ld16(tmem + lb + COL_CB + c0, cb);
                 tmem_wait_ld();
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
+                for (int q8 = 0; q8 < 2; ++q8) {
                     uint32_t plcb[4], plgx[4];
 #pragma unroll
                     for (int w2 = 0; w2 < 4; ++w2) {
@@ -550,7 +558,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                         plgx[w2] = pack_h2(lg[0], lg[1]);
                         range = fmaxf(range, fmaxf(fmaxf(fabsf(lc[0]), fabsf(lc[1])), fmaxf(fabsf(lg[0]), fabsf(lg[1]))));
                     }
-                    const uint32_t off = sw128_off(r, 4 * ch + q8);
+                    const uint32_t off = sw128_off(r, 2 * cq + q8);
                     *reinterpret_cast<uint4*>(sm + OFF_LCB + off) = make_uint4(plcb[0], plcb[1], plcb[2], plcb[3]);
                     *reinterpret_cast<uint4*>(sm + OFF_LGX + off) = make_uint4(plgx[0], plgx[1], plgx[2], plgx[3]);
                 }
@@ -562,10 +570,10 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                     ok = false;
                     break;
                 }
-                const float col = column_sums(gx, lane);
-                vec[(V_COL >> 2) + (par * 2 + rq) * 64 + c0 + lane] = col;
+                const float col = column_sums16(gx, lane);
+                if (lane < 16) vec[(V_COL >> 2) + (par * 2 + rq) * 64 + c0 + lane] = col;
             }
-            vec[(V_ROWM >> 2) + (par * 2 + ch) * 64 + r] = rowm;
+            vec[(V_ROWM >> 2) + (par * 4 + cq) * 64 + r] = rowm;
             // E partial (g . SPC) and sum g . x over this thread's columns, once SPC is there (B1_DONE)
             if (!wait_all(&bars[B1_DONE], par, abort)) {
                 ok = false;
@@ -574,22 +582,22 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             tc_fence_after();
             float pd = 0.f;
             {
-                float spc[32];
-                tmem_ld32(tmem + lb + COL_SPC + c0, spc);
+                float spc[16];
+                tmem_ld16(tmem + lb + COL_SPC + c0, spc);
                 tmem_wait_ld();
                 float e = 0.f;
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
+                for (int q8 = 0; q8 < 2; ++q8) {
                     float gq[8], xq[8];
-                    unpack8(bo + B_G, r, 4 * ch + q8, gq);
-                    unpack8(bo + B_X, r, 4 * ch + q8, xq);
+                    unpack8(bo + B_G, r, 2 * cq + q8, gq);
+                    unpack8(bo + B_X, r, 2 * cq + q8, xq);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         e += gq[q] * spc[8 * q8 + q] * isp[8 * q8 + q];
                         pd += gq[q] * xq[q];
                     }
                 }
-                vec[(V_E >> 2) + (par * 2 + ch) * 64 + r] = e;
+                vec[(V_E >> 2) + (par * 4 + cq) * 64 + r] = e;
             }
             if (!wait_all(&bars[B2_DONE], par, abort)) {
                 ok = false;
@@ -599,16 +607,16 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             // phase C: dz from the recomputed y; dx; W
             const float ex_r = r < Qv ? expf(cs_r) : 0.f, el_r = r < Qv ? expf(cs_last - cs_r) : 0.f;
             {
-                float yin[32], spc[32];
-                tmem_ld32(tmem + lb + COL_YIN + c0, yin);
-                tmem_ld32(tmem + lb + COL_SPC + c0, spc);
+                float yin[16], spc[16];
+                tmem_ld16(tmem + lb + COL_YIN + c0, yin);
+                tmem_ld16(tmem + lb + COL_SPC + c0, spc);
                 tmem_wait_ld();
                 float* dz = a.dz + (row0 + r) * HP + (int64_t)h * kPb + c0;
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
+                for (int q8 = 0; q8 < 2; ++q8) {
                     float xq[8], dq[8], o[8];
-                    unpack8(bo + B_X, r, 4 * ch + q8, xq);
-                    unpack8(bo + B_DS, r, 4 * ch + q8, dq);
+                    unpack8(bo + B_X, r, 2 * cq + q8, xq);
+                    unpack8(bo + B_DS, r, 2 * cq + q8, dq);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const int qq = 8 * q8 + q;
@@ -622,19 +630,19 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
             }
             float wpart = 0.f;
             {
-                float lmb[32], dxi[32];
-                tmem_ld32(tmem + lb + COL_LMB + c0, lmb);
-                tmem_ld32(tmem + lb + COL_DXI + c0, dxi);
+                float lmb[16], dxi[16];
+                tmem_ld16(tmem + lb + COL_LMB + c0, lmb);
+                tmem_ld16(tmem + lb + COL_DXI + c0, dxi);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&bars[ACC_FREE]);  // the head's last TMEM read: the next head's MMAs may start
                 const float f = dt_r * el_r;
                 float* du = a.DU + (row0 + r) * conv_dim + (int64_t)h * kPb + c0;
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
+                for (int q8 = 0; q8 < 2; ++q8) {
                     float xq[8], gq[8], o[8];
-                    unpack8(bo + B_X, r, 4 * ch + q8, xq);
-                    unpack8(bo + B_G, r, 4 * ch + q8, gq);
+                    unpack8(bo + B_X, r, 2 * cq + q8, xq);
+                    unpack8(bo + B_G, r, 2 * cq + q8, gq);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const int qq = 8 * q8 + q;
@@ -648,9 +656,9 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
                     }
                 }
             }
-            vec[(V_W >> 2) + (par * 2 + ch) * 64 + r] = el_r * wpart;
+            vec[(V_W >> 2) + (par * 4 + cq) * 64 + r] = el_r * wpart;
             pd = warp_sum(pd);
-            if (lane == 0) vec[(V_PD >> 2) + par * 4 + wi] = pd;
+            if (lane == 0) vec[(V_PD >> 2) + par * 8 + wi] = pd;
             mbar_arrive(&bars[WSYNC]);
             mbar_arrive(&bars[TILE_FREE0 + buf]);
         }
@@ -683,7 +691,7 @@ __global__ void __launch_bounds__(kThreadsB, 1) chunk_bwd_tc_kernel(const ChunkB
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS_B);
     }
