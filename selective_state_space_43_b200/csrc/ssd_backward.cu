@@ -35,7 +35,7 @@
 //   chunk_bwd_kernel    per (chunk, group, half of the group's heads), heads in turn: dz,
 //                       ddt, the post-conv gradients of x (per head) and of B, C (summed
 //                       over the half; the conv backward adds the two halves)
-//   conv_bwd_kernel     per (channel, 64-token tile): through SiLU' and the taps to
+//   conv_bwd_kernel     per (channel, 32-token tile): through SiLU' and the taps to
 //                       the pre-conv gradients, per-tile conv_w/conv_b partial sums,
 //                       d_init_conv_state
 //   reduce_kernel       sums of the per-tile / per-chunk partials in a fixed order
@@ -59,6 +59,8 @@
 extern __shared__ __align__(16) unsigned char ssd_bwd_smem[];
 #define SSD_DYN_SMEM() (ssd_bwd_smem)
 #endif
+
+#include <type_traits>
 
 #include "ssd_backward.h"
 
@@ -136,6 +138,8 @@ __device__ __forceinline__ float ld_act(const void* p, int64_t i, bool bf16) {
     if (bf16) return __uint_as_float(static_cast<unsigned>(static_cast<const unsigned short*>(p)[i]) << 16);
     return static_cast<const float*>(p)[i];
 }
+__device__ __forceinline__ float act_to_f(unsigned short v) { return __uint_as_float(static_cast<unsigned>(v) << 16); }
+__device__ __forceinline__ float act_to_f(float v) { return v; }
 __device__ __forceinline__ float sigmoid_f(float v) { return 1.f / (1.f + expf(-v)); }
 __device__ __forceinline__ float silu_f(float v) { return v * sigmoid_f(v); }
 __device__ __forceinline__ float dsilu_f(float v) {
@@ -143,6 +147,14 @@ __device__ __forceinline__ float dsilu_f(float v) {
     return s * (1.f + v * (1.f - s));
 }
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(expf(v)); }
+// The same with the fast exponential and division (a few ulp; 0 and 1 at the far ends): the two conv kernels
+// evaluate one per channel and token, and there the instruction count is what competes with HBM.
+__device__ __forceinline__ float sigmoid_fast(float v) { return __fdividef(1.f, 1.f + __expf(-v)); }
+__device__ __forceinline__ float silu_fast(float v) { return v * sigmoid_fast(v); }
+__device__ __forceinline__ float dsilu_fast(float v) {
+    const float s = sigmoid_fast(v);
+    return s * (1.f + v * (1.f - s));
+}
 
 // Pre-conv value of channel c at token s of sequence b (s in [-3, L)); history or zero before 0.
 __device__ __forceinline__ float raw_at(const BwdArgs& a, int64_t b, int64_t s, int64_t c) {
@@ -155,39 +167,35 @@ __device__ __forceinline__ float raw_at(const BwdArgs& a, int64_t b, int64_t s, 
     return ld_act(a.C, row * GN + (c - HP - GN), a.act_bf16);
 }
 
-constexpr int kCPT = 2;  // channels per thread of the conv kernels (conv_dim is even, and so is every array's width)
+// The two conv kernels spread a kCT-token tile over several threads per channel: each thread takes a short
+// window, loads all of it, then computes, so that many loads are in flight without long per-thread chains
+// (measured: both the 2-token streaming loop and one thread per whole tile leave HBM well under half busy).
+constexpr int kPC = 32;                // post_conv: channel pairs per CTA
+constexpr int kPST = kCT * kPC / kT;   // post_conv: tokens per thread (kT / kPC sub-tiles of the tile)
+constexpr int kCB = kT / 2;            // conv_bwd: channels per CTA
+constexpr int kBST = kCT / 2;          // conv_bwd: tokens per thread (two sub-tiles of the tile)
+static_assert(kPST * (kT / kPC) == kCT && kBST * 2 == kCT, "the sub-tiles cover the tile");
 
-// The pre-conv array (x, B or C) of an even channel c and of c + 1, its row stride and column.
-struct ChanPair {
-    const void* src;
-    int64_t stride, col;
-};
-__device__ __forceinline__ ChanPair chan_pair(const BwdArgs& a, int64_t c) {
-    const int64_t HP = (int64_t)a.H * a.P, GN = (int64_t)a.G * a.N;
-    if (c < HP) return {a.x, HP, c};
-    if (c < HP + GN) return {a.B, GN, c - HP};
-    return {a.C, GN, c - HP - GN};
+// Channels c, c + 1 of one token from its row: bf16 pairs as one 32-bit load, fp32 pairs as one 64-bit load.
+__device__ __forceinline__ float2 act_pair(const unsigned short* p) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
-// Channels c, c + 1 at token s: the inputs for s >= 0, the conv history (or zero) before.
-__device__ __forceinline__ float2 raw_pair(const BwdArgs& a, const ChanPair& q, int64_t b, int64_t s, int64_t c) {
-    if (s < 0) return make_float2(raw_at(a, b, s, c), raw_at(a, b, s, c + 1));
-    const int64_t i = (b * a.L + s) * q.stride + q.col;
-    if (a.act_bf16) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(static_cast<const unsigned short*>(q.src) + i);
-        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-    }
-    return *reinterpret_cast<const float2*>(static_cast<const float*>(q.src) + i);
-}
+__device__ __forceinline__ float2 act_pair(const float* p) { return *reinterpret_cast<const float2*>(p); }
 
-// grid (ceil(conv_dim / (kT * kCPT)), ntiles, batch): one thread per (pair of channels, kCT-token tile), streaming
-// the tile with kBatch tokens' inputs loaded before their outputs are stored (the stores could alias the
-// inputs as far as the compiler knows, so it would not move later loads above them).
+// grid (ceil(conv_dim / (2 kPC)), ntiles, batch), kT threads: thread (pair lc, sub-tile) takes channels
+// c, c + 1 and tokens t0 .. t0 + kPST - 1; it loads their pre-conv values and those of the 3 tokens before
+// (the conv history before token 0), then writes u = silu(conv) for its tokens.  Token indices are 32-bit
+// and every load is a 32-bit offset from one row pointer: the index arithmetic is most of the kernel's
+// instructions otherwise.  kBf16: the inputs are bf16 (a.act_bf16).
+template <bool kBf16>
 __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
-    const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N;
-    const int64_t c = ((int64_t)blockIdx.x * kT + threadIdx.x) * kCPT;
-    if (c >= conv_dim) return;
-    const int64_t b = blockIdx.z, t0 = (int64_t)blockIdx.y * kCT;
-    const int64_t t1 = t0 + kCT < a.L ? t0 + kCT : a.L;
+    using T = typename std::conditional<kBf16, unsigned short, float>::type;
+    const int HP = a.H * a.P, GN = a.G * a.N, conv_dim = HP + 2 * GN, L = static_cast<int>(a.L);
+    const int lc = threadIdx.x % kPC, sub = threadIdx.x / kPC;
+    const int c = (blockIdx.x * kPC + lc) * 2;
+    const int b = blockIdx.z, t0 = blockIdx.y * kCT + sub * kPST;
+    if (c >= conv_dim || t0 >= L) return;
     float w[2][4], bias[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -195,25 +203,36 @@ __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
         w[k][0] = wv.x, w[k][1] = wv.y, w[k][2] = wv.z, w[k][3] = wv.w;
         bias[k] = a.conv_b[c + k];
     }
-    const ChanPair q = chan_pair(a, c);
-    float2 r0 = raw_pair(a, q, b, t0 - 3, c), r1 = raw_pair(a, q, b, t0 - 2, c), r2 = raw_pair(a, q, b, t0 - 1, c);
-    constexpr int kBatch = 8;
-#pragma unroll 1
-    for (int64_t tb = t0; tb < t1; tb += kBatch) {
-        float2 rin[kBatch];
+    // the pre-conv array of channels c, c + 1 (x, B or C), its row stride, and the pointer at token t0
+    const T* src;
+    int rs;
+    if (c < HP) {
+        src = static_cast<const T*>(a.x) + c, rs = HP;
+    } else if (c < HP + GN) {
+        src = static_cast<const T*>(a.B) + (c - HP), rs = GN;
+    } else {
+        src = static_cast<const T*>(a.C) + (c - HP - GN), rs = GN;
+    }
+    src += ((int64_t)b * L + t0) * rs;
+    float2 r[kPST + 3];  // tokens t0 - 3 .. t0 + kPST - 1
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) rin[i] = tb + i < t1 ? raw_pair(a, q, b, tb + i, c) : make_float2(0.f, 0.f);
+    for (int i = 0; i < kPST + 3; ++i) {
+        const int s = t0 - 3 + i;
+        if (s >= L)
+            r[i] = make_float2(0.f, 0.f);
+        else if (i < 3 && s < 0)
+            r[i] = make_float2(raw_at(a, b, s, c), raw_at(a, b, s, c + 1));
+        else
+            r[i] = act_pair(src + (i - 3) * rs);
+    }
+    float* u = ws.U + ((int64_t)b * L + t0) * conv_dim + c;
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-            if (tb + i < t1) {
-                float2 u;
-                u.x = silu_f(bias[0] + w[0][0] * r0.x + w[0][1] * r1.x + w[0][2] * r2.x + w[0][3] * rin[i].x);
-                u.y = silu_f(bias[1] + w[1][0] * r0.y + w[1][1] * r1.y + w[1][2] * r2.y + w[1][3] * rin[i].y);
-                *reinterpret_cast<float2*>(ws.U + (b * a.L + tb + i) * conv_dim + c) = u;
-                r0 = r1;
-                r1 = r2;
-                r2 = rin[i];
-            }
+    for (int i = 0; i < kPST; ++i) {
+        if (t0 + i < L) {
+            float2 v;
+            v.x = silu_fast(bias[0] + w[0][0] * r[i].x + w[0][1] * r[i + 1].x + w[0][2] * r[i + 2].x + w[0][3] * r[i + 3].x);
+            v.y = silu_fast(bias[1] + w[1][0] * r[i].y + w[1][1] * r[i + 1].y + w[1][2] * r[i + 2].y + w[1][3] * r[i + 3].y);
+            *reinterpret_cast<float2*>(u + i * conv_dim) = v;
         }
     }
 }
@@ -1015,90 +1034,92 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     }
 }
 
-// grid (ceil(conv_dim / kT), ntiles, batch): one thread per (channel, kCT-token tile).
-// Streams t over the tile and the 3 tokens after it: dv_t = du_t silu'(v_t), and the pre-conv
-// gradient of token s = t - 3 is w0 dv_t + w1 dv_{t-1} + w2 dv_{t-2} + w3 dv_{t-3}.
-__global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
-    const int64_t HP = (int64_t)a.H * a.P, GN = (int64_t)a.G * a.N, conv_dim = HP + 2 * GN;
-    const int64_t c = (int64_t)blockIdx.x * kT + threadIdx.x;
-    if (c >= conv_dim) return;
-    const int64_t b = blockIdx.z, tile = blockIdx.y, nt = ntiles(a.L), t0 = tile * kCT;
-    const int64_t t1 = t0 + kCT < a.L ? t0 + kCT : a.L;
-    const float w0 = a.conv_w[c * 4 + 0], w1 = a.conv_w[c * 4 + 1], w2 = a.conv_w[c * 4 + 2],
-                w3 = a.conv_w[c * 4 + 3], bias = a.conv_b[c];
-    // this channel's input array and gradient array (x / B / C and dx / dB / dC), row stride, column
-    const void* src;
+// grid (ceil(conv_dim / kCB), ntiles, batch), kT threads, 2 * 5 * kCB floats of dynamic shared memory:
+// thread (channel lc, sub-tile) takes tokens t0 .. t0 + kBST - 1 of the tile.  With v_t the pre-SiLU conv
+// output, dv_t = du_t silu'(v_t), and the pre-conv gradient of token s is
+// w0 dv_{s+3} + w1 dv_{s+2} + w2 dv_{s+1} + w3 dv_s; so the thread loads the pre-conv values of tokens
+// t0 - 3 .. t0 + kBST + 2 and du of t0 .. t0 + kBST + 2 (the 3 tokens after its sub-tile reach back into it)
+// before any arithmetic.  The tile's conv_w / conv_b partials are its two sub-tiles' sums, in that order.
+// As in post_conv_kernel: 32-bit token indices and offsets from per-thread row pointers; kBf16 = a.act_bf16.
+template <bool kBf16>
+__global__ void __launch_bounds__(kT, 3) conv_bwd_kernel(BwdArgs a, Ws ws) {
+    using T = typename std::conditional<kBf16, unsigned short, float>::type;
+    float* part = reinterpret_cast<float*>(SSD_DYN_SMEM());  // [2 sub-tiles][5][kCB]
+    const int HP = a.H * a.P, GN = a.G * a.N, conv_dim = HP + 2 * GN, L = static_cast<int>(a.L);
+    const int lc = threadIdx.x % kCB, sub = threadIdx.x / kCB;
+    const int c = blockIdx.x * kCB + lc;
+    const bool live = c < conv_dim;  // threads past the last channel still meet the barrier
+    const int cc = live ? c : 0;
+    const int b = blockIdx.z, tile = blockIdx.y, t0 = tile * kCT + sub * kBST;
+    const float w0 = a.conv_w[cc * 4 + 0], w1 = a.conv_w[cc * 4 + 1], w2 = a.conv_w[cc * 4 + 2],
+                w3 = a.conv_w[cc * 4 + 3], bias = a.conv_b[cc];
+    // this channel's input array and gradient array (x / B / C and dx / dB / dC) and their row stride
+    const T* src;
     float* out;
-    int64_t ostride, ocol;
-    if (c < HP) {
-        src = a.x, out = a.dx, ostride = HP, ocol = c;
-    } else if (c < HP + GN) {
-        src = a.B, out = a.dB, ostride = GN, ocol = c - HP;
+    int rs;
+    if (cc < HP) {
+        src = static_cast<const T*>(a.x) + cc, out = a.dx + cc, rs = HP;
+    } else if (cc < HP + GN) {
+        src = static_cast<const T*>(a.B) + (cc - HP), out = a.dB + (cc - HP), rs = GN;
     } else {
-        src = a.C, out = a.dC, ostride = GN, ocol = c - HP - GN;
+        src = static_cast<const T*>(a.C) + (cc - HP - GN), out = a.dC + (cc - HP - GN), rs = GN;
     }
-    const int64_t row0 = b * a.L;
-    const bool two_halves = head_split(a.H, a.G) == 2;
-    float r0 = raw_at(a, b, t0 - 3, c), r1 = raw_at(a, b, t0 - 2, c), r2 = raw_at(a, b, t0 - 1, c);
-    float d1 = 0.f, d2 = 0.f, d3 = 0.f;  // dv at t-1, t-2, t-3 (zero before token 0)
+    const int64_t row = (int64_t)b * L + t0;  // this thread's first token, as a row of the [batch * L] arrays
+    src += row * rs;
+    out += row * rs;
+    const float* dp = ws.DU + row * conv_dim + cc;
+    // tokens of t0 .. t0 + kBST + 2 that exist (negative past the end: slot i reads token t0 - 3 + i only when
+    // i - 3 < n, so -3 turns every load of a thread past the last channel off)
+    const int n = live ? (L - t0 < kBST + 3 ? L - t0 : kBST + 3) : -3;
+    float r[kBST + 6], d[kBST + 3];  // r[i]: pre-conv value of token t0 - 3 + i; d[i]: du, then dv, of t0 + i
+#pragma unroll
+    for (int i = 0; i < kBST + 6; ++i) {
+        r[i] = 0.f;
+        if (i - 3 < n) r[i] = i >= 3 || t0 - 3 + i >= 0 ? act_to_f(src[(i - 3) * rs]) : raw_at(a, b, t0 - 3 + i, cc);
+    }
+#pragma unroll
+    for (int i = 0; i < kBST + 3; ++i) d[i] = i < n ? dp[i * conv_dim] : 0.f;
+    if (cc >= HP && head_split(a.H, a.G) == 2) {
+        const float* du2 = ws.DU2 + row * 2 * GN + (cc - HP);
+#pragma unroll
+        for (int i = 0; i < kBST + 3; ++i)
+            if (i < n) d[i] += du2[i * 2 * GN];
+    }
     float gw0 = 0.f, gw1 = 0.f, gw2 = 0.f, gw3 = 0.f, gb = 0.f;
-    // the loads of kBatch tokens are issued before their gradients are stored (see post_conv_kernel);
-    // 2 keeps the thread at 64 registers (4 CTAs per SM): the same loads in flight per SM as larger
-    // batches with fewer resident CTAs
-    constexpr int kBatch = 2;
-#pragma unroll 1
-    for (int64_t tb = t0; tb < t1 + 3; tb += kBatch) {
-        float rin[kBatch], din[kBatch];
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-            const int64_t tt = tb + i;
-            rin[i] = 0.f;
-            din[i] = 0.f;
-            if (tt < a.L && tt < t1 + 3) {
-                rin[i] = ld_act(src, (row0 + tt) * ostride + ocol, a.act_bf16);
-                din[i] = ws.DU[(row0 + tt) * conv_dim + c];
-                if (c >= HP && two_halves) din[i] += ws.DU2[(row0 + tt) * 2 * GN + (c - HP)];
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-            const int64_t t = tb + i;
-            if (t < t1 + 3) {
-                float dv = 0.f;
-                if (t < a.L) {
-                    const float r3 = rin[i];
-                    const float v = bias + w0 * r0 + w1 * r1 + w2 * r2 + w3 * r3;
-                    dv = din[i] * dsilu_f(v);
-                    if (t < t1) {
-                        gw0 += dv * r0;
-                        gw1 += dv * r1;
-                        gw2 += dv * r2;
-                        gw3 += dv * r3;
-                        gb += dv;
-                    }
-                    r0 = r1;
-                    r1 = r2;
-                    r2 = r3;
-                }
-                const int64_t s = t - 3;
-                const float gs = w0 * dv + w1 * d1 + w2 * d2 + w3 * d3;
-                if (s >= t0 && s < t1) {
-                    out[(row0 + s) * ostride + ocol] = gs;
-                } else if (s < 0 && a.d_init_conv_state) {
-                    a.d_init_conv_state[(b * conv_dim + c) * 3 + (s + 3)] = gs;
-                }
-                d3 = d2;
-                d2 = d1;
-                d1 = dv;
-            }
+    for (int i = 0; i < kBST + 3; ++i) {
+        const float v = bias + w0 * r[i] + w1 * r[i + 1] + w2 * r[i + 2] + w3 * r[i + 3];
+        d[i] = i < n ? d[i] * dsilu_fast(v) : 0.f;
+        if (i < kBST) {
+            gw0 += d[i] * r[i];
+            gw1 += d[i] * r[i + 1];
+            gw2 += d[i] * r[i + 2];
+            gw3 += d[i] * r[i + 3];
+            gb += d[i];
         }
     }
-    float* pw = ws.PW + ((b * nt + tile) * conv_dim + c) * 5;
-    pw[0] = gw0;
-    pw[1] = gw1;
-    pw[2] = gw2;
-    pw[3] = gw3;
-    pw[4] = gb;
+#pragma unroll
+    for (int j = 0; j < kBST; ++j)
+        if (j < n) out[j * rs] = w0 * d[j + 3] + w1 * d[j + 2] + w2 * d[j + 1] + w3 * d[j];
+    if (live && t0 == 0 && a.d_init_conv_state) {
+        // the history tokens s = -3, -2, -1 (dv is zero before token 0)
+        float* dh = a.d_init_conv_state + ((int64_t)b * conv_dim + cc) * 3;
+        dh[0] = w0 * d[0];
+        dh[1] = w0 * d[1] + w1 * d[0];
+        dh[2] = w0 * d[2] + w1 * d[1] + w2 * d[0];
+    }
+    float* mine = part + sub * 5 * kCB + lc;
+    mine[0] = gw0;
+    mine[kCB] = gw1;
+    mine[2 * kCB] = gw2;
+    mine[3 * kCB] = gw3;
+    mine[4 * kCB] = gb;
+    __syncthreads();
+    if (sub == 0 && live) {
+        float* pw = ws.PW + (((int64_t)b * ntiles(a.L) + tile) * conv_dim + c) * 5;
+#pragma unroll
+        for (int k = 0; k < 5; ++k) pw[k] = part[k * kCB + lc] + part[(5 + k) * kCB + lc];
+    }
 }
 
 // grid (ceil(conv_dim / 32) + ceil(H / 32)), kT threads: 32 channels (or heads) per CTA, each summed by
@@ -1159,7 +1180,7 @@ __global__ void __launch_bounds__(kT) copy_adjoint_kernel(BwdArgs a) {
 template <int N>
 cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
     const int64_t conv_dim = (int64_t)a.H * a.P + 2LL * a.G * a.N, nc = nchunks(a.L), nt = ntiles(a.L);
-    const unsigned cgrid = static_cast<unsigned>((conv_dim + kT * kCPT - 1) / (kT * kCPT));  // post-conv channel pairs
+    const unsigned cgrid = static_cast<unsigned>((conv_dim + 2 * kPC - 1) / (2 * kPC));  // post-conv channel pairs
     cudaError_t err;
     if (a.batch > 0 && nc > 0) {
         const size_t state_smem = (2 * (size_t)kQ * kP + 2 * (size_t)kQ * N + 2 * kQ) * sizeof(float);
@@ -1167,7 +1188,10 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         if ((err = SSD_SET_SMEM(chunk_state_kernel<N>, state_smem)) != cudaSuccess) return err;
         if ((err = SSD_SET_SMEM(chunk_bwd_kernel<N>, chunk_smem)) != cudaSuccess) return err;
         const dim3 tiles(cgrid, static_cast<unsigned>(ntiles(a.L)), static_cast<unsigned>(a.batch));
-        SSD_LAUNCH(post_conv_kernel, tiles, dim3(kT), 0, st, a, ws);
+        if (a.act_bf16)
+            SSD_LAUNCH(post_conv_kernel<true>, tiles, dim3(kT), 0, st, a, ws);
+        else
+            SSD_LAUNCH(post_conv_kernel<false>, tiles, dim3(kT), 0, st, a, ws);
         SSD_LAUNCH(dt_kernel,
                    dim3(static_cast<unsigned>(nc), static_cast<unsigned>((a.H + kT / 32 - 1) / (kT / 32)),
                         static_cast<unsigned>(a.batch)),
@@ -1217,11 +1241,15 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         const int64_t n = a.batch * a.H * (int64_t)a.P * a.N;
         SSD_LAUNCH(copy_adjoint_kernel, dim3(static_cast<unsigned>((n + kT - 1) / kT)), dim3(kT), 0, st, a);
     }
-    if (a.batch > 0)
-        SSD_LAUNCH(conv_bwd_kernel,
-                   dim3(static_cast<unsigned>((conv_dim + kT - 1) / kT), static_cast<unsigned>(nt),
-                        static_cast<unsigned>(a.batch)),
-                   dim3(kT), 0, st, a, ws);
+    if (a.batch > 0) {
+        const dim3 grid(static_cast<unsigned>((conv_dim + kCB - 1) / kCB), static_cast<unsigned>(nt),
+                        static_cast<unsigned>(a.batch));
+        const size_t smem = 2 * 5 * kCB * sizeof(float);
+        if (a.act_bf16)
+            SSD_LAUNCH(conv_bwd_kernel<true>, grid, dim3(kT), smem, st, a, ws);
+        else
+            SSD_LAUNCH(conv_bwd_kernel<false>, grid, dim3(kT), smem, st, a, ws);
+    }
     SSD_LAUNCH(reduce_kernel, dim3(static_cast<unsigned>((conv_dim + 31) / 32 + (a.H + 31) / 32)), dim3(kT),
                5 * (size_t)kT * sizeof(float), st, a, ws);
     return cudaGetLastError();

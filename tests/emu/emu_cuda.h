@@ -151,6 +151,7 @@ inline float2 make_float2(float a, float b) { return float2{a, b}; }
 inline float4 __ldcs(const float4* p) { return *p; }
 inline void __stcs(float4* p, float4 v) { *p = v; }
 inline float __expf(float v) { return expf(v); }
+inline float __fdividef(float a, float b) { return a / b; }
 
 // bf16 storage: round to nearest, ties to even, on the 16 dropped bits (NaN kept quiet)
 struct __nv_bfloat16 {

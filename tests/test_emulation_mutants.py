@@ -20,11 +20,9 @@ SRC = os.path.join(emu_harness.CSRC, "ssd_backward.cu")
 
 MUTANTS = {
     # reads x one token past the tile: beyond the array for the last tile of the last sequence
-    "post-conv reads past its tile": ("rin[i] = tb + i < t1 ? raw_pair(a, q, b, tb + i, c) : make_float2(0.f, 0.f);",
-                                      "rin[i] = tb + i < t1 ? raw_pair(a, q, b, tb + i + 1, c) : make_float2(0.f, 0.f);"),
+    "post-conv reads past its tile": ("r[i] = act_pair(src + (i - 3) * rs);", "r[i] = act_pair(src + (i - 2) * rs);"),
     # writes each pre-conv gradient one token late: beyond dx / dB / dC for the last token
-    "conv backward writes one row late": ("out[(row0 + s) * ostride + ocol] = gs;",
-                                          "out[(row0 + s + 1) * ostride + ocol] = gs;"),
+    "conv backward writes one row late": ("if (j < n) out[j * rs] =", "if (j < n) out[(j + 1) * rs] ="),
     # leaves the rows of a ragged chunk past its end as they were (NaN bytes for the first head)
     "ragged rows not cleared": ("            xs[j * kS + p] = xv;", "            if (j < Qv) xs[j * kS + p] = xv;"),
     # shared rows no longer 16-byte aligned: the emulation's alignment check must stop the vector loads
