@@ -140,6 +140,24 @@ __device__ __forceinline__ float ld_act(const void* p, int64_t i, bool bf16) {
 }
 __device__ __forceinline__ float act_to_f(unsigned short v) { return __uint_as_float(static_cast<unsigned>(v) << 16); }
 __device__ __forceinline__ float act_to_f(float v) { return v; }
+
+// A 16-byte global -> shared copy that takes no registers while in flight (cp.async, cached in L2 only); the
+// bytes past src_bytes (0 or 16) are zero-filled, and none is read when src_bytes is 0.
+#ifdef SSD_EMU
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+    memset(dst, 0, 16);
+    if (src_bytes) memcpy(dst, src, src_bytes);
+}
+__device__ __forceinline__ void cp_async_wait_all() {}
+#else
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sa), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+#endif
 __device__ __forceinline__ float sigmoid_f(float v) { return 1.f / (1.f + expf(-v)); }
 __device__ __forceinline__ float silu_f(float v) { return v * sigmoid_f(v); }
 __device__ __forceinline__ float dsilu_f(float v) {
@@ -172,9 +190,16 @@ __device__ __forceinline__ float raw_at(const BwdArgs& a, int64_t b, int64_t s, 
 // (measured: both the 2-token streaming loop and one thread per whole tile leave HBM well under half busy).
 constexpr int kPC = 32;                // post_conv: channel pairs per CTA
 constexpr int kPST = kCT * kPC / kT;   // post_conv: tokens per thread (kT / kPC sub-tiles of the tile)
-constexpr int kCB = kT / 2;            // conv_bwd: channels per CTA
-constexpr int kBST = kCT / 2;          // conv_bwd: tokens per thread (two sub-tiles of the tile)
-static_assert(kPST * (kT / kPC) == kCT && kBST * 2 == kCT, "the sub-tiles cover the tile");
+static_assert(kPST * (kT / kPC) == kCT, "the sub-tiles cover the tile");
+// conv_bwd stages its tile in shared memory instead: kCB channels x (kCT + 6) pre-conv rows and (kCT + 3) du
+// rows arrive by cp.async, so the loads in flight hold no registers; then kT / kCB sub-tiles of kBST tokens
+// per channel compute from shared memory.
+constexpr int kCB = 64;                      // channels per CTA
+constexpr int kBSUB = kT / kCB;              // sub-tiles per tile (4)
+constexpr int kBST = kCT / kBSUB;            // tokens per thread (8)
+constexpr int kRawRows = kCT + 6, kDuRows = kCT + 3;
+constexpr size_t kConvBwdSmem = (size_t)kRawRows * kCB * 4 + 2 * (size_t)kDuRows * kCB * 4 + (size_t)kBSUB * 5 * kCB * 4;
+static_assert(kBST * kBSUB == kCT && kCB % 8 == 0, "the sub-tiles cover the tile; whole 16-byte chunks per row");
 
 // Channels c, c + 1 of one token from its row: bf16 pairs as one 32-bit load, fp32 pairs as one 64-bit load.
 __device__ __forceinline__ float2 act_pair(const unsigned short* p) {
@@ -187,8 +212,9 @@ __device__ __forceinline__ float2 act_pair(const float* p) { return *reinterpret
 // c, c + 1 and tokens t0 .. t0 + kPST - 1; it loads their pre-conv values and those of the 3 tokens before
 // (the conv history before token 0), then writes u = silu(conv) for its tokens.  Token indices are 32-bit
 // and every load is a 32-bit offset from one row pointer: the index arithmetic is most of the kernel's
-// instructions otherwise.  kBf16: the inputs are bf16 (a.act_bf16).
-template <bool kBf16>
+// instructions otherwise.  kBf16: the inputs are bf16 (a.act_bf16); kHist: a conv history is given
+// (a.init_conv_state; without one the tokens before 0 are zero and take no registers).
+template <bool kBf16, bool kHist>
 __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
     using T = typename std::conditional<kBf16, unsigned short, float>::type;
     const int HP = a.H * a.P, GN = a.G * a.N, conv_dim = HP + 2 * GN, L = static_cast<int>(a.L);
@@ -218,7 +244,7 @@ __global__ void __launch_bounds__(kT) post_conv_kernel(BwdArgs a, Ws ws) {
 #pragma unroll
     for (int i = 0; i < kPST + 3; ++i) {
         const int s = t0 - 3 + i;
-        if (s >= L)
+        if (s >= L || (!kHist && i < 3 && s < 0))
             r[i] = make_float2(0.f, 0.f);
         else if (i < 3 && s < 0)
             r[i] = make_float2(raw_at(a, b, s, c), raw_at(a, b, s, c + 1));
@@ -1034,56 +1060,82 @@ __global__ void __launch_bounds__(kT, 1) chunk_bwd_kernel(BwdArgs a, Ws ws) {
     }
 }
 
-// grid (ceil(conv_dim / kCB), ntiles, batch), kT threads, 2 * 5 * kCB floats of dynamic shared memory:
-// thread (channel lc, sub-tile) takes tokens t0 .. t0 + kBST - 1 of the tile.  With v_t the pre-SiLU conv
-// output, dv_t = du_t silu'(v_t), and the pre-conv gradient of token s is
-// w0 dv_{s+3} + w1 dv_{s+2} + w2 dv_{s+1} + w3 dv_s; so the thread loads the pre-conv values of tokens
-// t0 - 3 .. t0 + kBST + 2 and du of t0 .. t0 + kBST + 2 (the 3 tokens after its sub-tile reach back into it)
-// before any arithmetic.  The tile's conv_w / conv_b partials are its two sub-tiles' sums, in that order.
-// As in post_conv_kernel: 32-bit token indices and offsets from per-thread row pointers; kBf16 = a.act_bf16.
-template <bool kBf16>
-__global__ void __launch_bounds__(kT, 3) conv_bwd_kernel(BwdArgs a, Ws ws) {
+// The pre-conv array holding channel c (x, B or C), offset to c's column, and its row stride.
+template <typename T>
+__device__ __forceinline__ const T* raw_col(const BwdArgs& a, int c, int HP, int GN, int& rs) {
+    rs = c < HP ? HP : GN;
+    if (c < HP) return static_cast<const T*>(a.x) + c;
+    if (c < HP + GN) return static_cast<const T*>(a.B) + (c - HP);
+    return static_cast<const T*>(a.C) + (c - HP - GN);
+}
+
+// grid (ceil(conv_dim / kCB), ntiles, batch), kT threads, kConvBwdSmem bytes of dynamic shared memory.
+// With v_t the pre-SiLU conv output, dv_t = du_t silu'(v_t), and the pre-conv gradient of token s is
+// w0 dv_{s+3} + w1 dv_{s+2} + w2 dv_{s+1} + w3 dv_s.  The CTA first stages the pre-conv values of tokens
+// tb - 3 .. tb + kCT + 2 (tb the tile's first token; the conv history, or zero, before token 0) and du (plus
+// the second half's dB | dC) of tokens tb .. tb + kCT + 2, zero past the sequence; then thread (channel lc,
+// sub-tile) computes dv for its kBST tokens and the 3 after, its kBST gradients and its share of the tile's
+// conv_w / conv_b partials (summed over the sub-tiles in their order).  HP = 64 H and GN = G N (N a multiple
+// of 16) are multiples of 8, so a 16-byte chunk of a row never straddles x / B / C or conv_dim, and every
+// chunk is 16-byte aligned (the entry point rejects unaligned arrays).  kBf16 = a.act_bf16, kHist =
+// (a.init_conv_state != null).
+template <bool kBf16, bool kHist>
+__global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
     using T = typename std::conditional<kBf16, unsigned short, float>::type;
-    float* part = reinterpret_cast<float*>(SSD_DYN_SMEM());  // [2 sub-tiles][5][kCB]
+    constexpr int kE = 16 / sizeof(T);  // elements per 16-byte chunk
+    unsigned char* smem = SSD_DYN_SMEM();
+    T* raw_s = reinterpret_cast<T*>(smem);                                   // [kRawRows][kCB]
+    float* du_s = reinterpret_cast<float*>(smem + (size_t)kRawRows * kCB * 4);  // [kDuRows][kCB]
+    float* du2_s = du_s + kDuRows * kCB;                                     // [kDuRows][kCB]
+    float* part = du2_s + kDuRows * kCB;                                     // [kBSUB][5][kCB]
     const int HP = a.H * a.P, GN = a.G * a.N, conv_dim = HP + 2 * GN, L = static_cast<int>(a.L);
-    const int lc = threadIdx.x % kCB, sub = threadIdx.x / kCB;
-    const int c = blockIdx.x * kCB + lc;
+    const int tid = threadIdx.x, c0 = blockIdx.x * kCB, b = blockIdx.z, tile = blockIdx.y, tb = tile * kCT;
+    const int64_t row0 = (int64_t)b * L;
+    const bool add2 = head_split(a.H, a.G) == 2 && c0 + kCB > HP;  // the second half's dB | dC apply here
+    for (int e = tid; e < kRawRows * (kCB / kE); e += kT) {
+        const int i = e / (kCB / kE), c = c0 + (e - i * (kCB / kE)) * kE, s = tb - 3 + i;
+        if (s < 0) continue;  // history rows: below
+        const bool ok = s < L && c < conv_dim;
+        int rs = 0;
+        const T* g = ok ? raw_col<T>(a, c, HP, GN, rs) : static_cast<const T*>(a.x);
+        cp_async16(raw_s + i * kCB + (c - c0), ok ? g + (row0 + s) * rs : g, ok ? 16 : 0);
+    }
+    for (int e = tid; e < kDuRows * (kCB / 4); e += kT) {
+        const int i = e / (kCB / 4), c = c0 + (e - i * (kCB / 4)) * 4, t = tb + i;
+        const bool ok = t < L && c < conv_dim;
+        cp_async16(du_s + i * kCB + (c - c0), ok ? ws.DU + (row0 + t) * conv_dim + c : ws.DU, ok ? 16 : 0);
+        if (add2) {
+            const bool ok2 = ok && c >= HP;
+            cp_async16(du2_s + i * kCB + (c - c0), ok2 ? ws.DU2 + (row0 + t) * 2 * GN + (c - HP) : ws.DU, ok2 ? 16 : 0);
+        }
+    }
+    if (tb == 0) {
+        // tokens -3 .. -1: the conv history (layout [batch][conv_dim][3]) or zero
+        for (int e = tid; e < 3 * kCB; e += kT) {
+            const int i = e / kCB, c = c0 + (e - i * kCB);
+            T v = 0;
+            if (kHist && c < conv_dim) v = static_cast<const T*>(a.init_conv_state)[((int64_t)b * conv_dim + c) * 3 + i];
+            raw_s[i * kCB + (c - c0)] = v;
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    const int lc = tid % kCB, sub = tid / kCB, c = c0 + lc, t0 = tb + sub * kBST;
     const bool live = c < conv_dim;  // threads past the last channel still meet the barrier
     const int cc = live ? c : 0;
-    const int b = blockIdx.z, tile = blockIdx.y, t0 = tile * kCT + sub * kBST;
     const float w0 = a.conv_w[cc * 4 + 0], w1 = a.conv_w[cc * 4 + 1], w2 = a.conv_w[cc * 4 + 2],
                 w3 = a.conv_w[cc * 4 + 3], bias = a.conv_b[cc];
-    // this channel's input array and gradient array (x / B / C and dx / dB / dC) and their row stride
-    const T* src;
-    float* out;
-    int rs;
-    if (cc < HP) {
-        src = static_cast<const T*>(a.x) + cc, out = a.dx + cc, rs = HP;
-    } else if (cc < HP + GN) {
-        src = static_cast<const T*>(a.B) + (cc - HP), out = a.dB + (cc - HP), rs = GN;
-    } else {
-        src = static_cast<const T*>(a.C) + (cc - HP - GN), out = a.dC + (cc - HP - GN), rs = GN;
-    }
-    const int64_t row = (int64_t)b * L + t0;  // this thread's first token, as a row of the [batch * L] arrays
-    src += row * rs;
-    out += row * rs;
-    const float* dp = ws.DU + row * conv_dim + cc;
-    // tokens of t0 .. t0 + kBST + 2 that exist (negative past the end: slot i reads token t0 - 3 + i only when
-    // i - 3 < n, so -3 turns every load of a thread past the last channel off)
+    // tokens of t0 .. t0 + kBST + 2 that exist (negative past the end; -3 for a thread past the last channel)
     const int n = live ? (L - t0 < kBST + 3 ? L - t0 : kBST + 3) : -3;
     float r[kBST + 6], d[kBST + 3];  // r[i]: pre-conv value of token t0 - 3 + i; d[i]: du, then dv, of t0 + i
 #pragma unroll
-    for (int i = 0; i < kBST + 6; ++i) {
-        r[i] = 0.f;
-        if (i - 3 < n) r[i] = i >= 3 || t0 - 3 + i >= 0 ? act_to_f(src[(i - 3) * rs]) : raw_at(a, b, t0 - 3 + i, cc);
-    }
+    for (int i = 0; i < kBST + 6; ++i) r[i] = act_to_f(raw_s[(sub * kBST + i) * kCB + lc]);
+    const bool second = add2 && c >= HP;
 #pragma unroll
-    for (int i = 0; i < kBST + 3; ++i) d[i] = i < n ? dp[i * conv_dim] : 0.f;
-    if (cc >= HP && head_split(a.H, a.G) == 2) {
-        const float* du2 = ws.DU2 + row * 2 * GN + (cc - HP);
-#pragma unroll
-        for (int i = 0; i < kBST + 3; ++i)
-            if (i < n) d[i] += du2[i * 2 * GN];
+    for (int i = 0; i < kBST + 3; ++i) {
+        d[i] = du_s[(sub * kBST + i) * kCB + lc];
+        if (second) d[i] += du2_s[(sub * kBST + i) * kCB + lc];
     }
     float gw0 = 0.f, gw1 = 0.f, gw2 = 0.f, gw3 = 0.f, gb = 0.f;
 #pragma unroll
@@ -1098,15 +1150,26 @@ __global__ void __launch_bounds__(kT, 3) conv_bwd_kernel(BwdArgs a, Ws ws) {
             gb += d[i];
         }
     }
+    if (live) {
+        float* out;
+        const int rs = cc < HP ? HP : GN;
+        if (cc < HP)
+            out = a.dx + cc;
+        else if (cc < HP + GN)
+            out = a.dB + (cc - HP);
+        else
+            out = a.dC + (cc - HP - GN);
+        out += (row0 + t0) * rs;
 #pragma unroll
-    for (int j = 0; j < kBST; ++j)
-        if (j < n) out[j * rs] = w0 * d[j + 3] + w1 * d[j + 2] + w2 * d[j + 1] + w3 * d[j];
-    if (live && t0 == 0 && a.d_init_conv_state) {
-        // the history tokens s = -3, -2, -1 (dv is zero before token 0)
-        float* dh = a.d_init_conv_state + ((int64_t)b * conv_dim + cc) * 3;
-        dh[0] = w0 * d[0];
-        dh[1] = w0 * d[1] + w1 * d[0];
-        dh[2] = w0 * d[2] + w1 * d[1] + w2 * d[0];
+        for (int j = 0; j < kBST; ++j)
+            if (j < n) out[j * rs] = w0 * d[j + 3] + w1 * d[j + 2] + w2 * d[j + 1] + w3 * d[j];
+        if (t0 == 0 && a.d_init_conv_state) {
+            // the history tokens s = -3, -2, -1 (dv is zero before token 0)
+            float* dh = a.d_init_conv_state + ((int64_t)b * conv_dim + cc) * 3;
+            dh[0] = w0 * d[0];
+            dh[1] = w0 * d[1] + w1 * d[0];
+            dh[2] = w0 * d[2] + w1 * d[1] + w2 * d[0];
+        }
     }
     float* mine = part + sub * 5 * kCB + lc;
     mine[0] = gw0;
@@ -1118,7 +1181,12 @@ __global__ void __launch_bounds__(kT, 3) conv_bwd_kernel(BwdArgs a, Ws ws) {
     if (sub == 0 && live) {
         float* pw = ws.PW + (((int64_t)b * ntiles(a.L) + tile) * conv_dim + c) * 5;
 #pragma unroll
-        for (int k = 0; k < 5; ++k) pw[k] = part[k * kCB + lc] + part[(5 + k) * kCB + lc];
+        for (int k = 0; k < 5; ++k) {
+            float v = part[k * kCB + lc];
+#pragma unroll
+            for (int q = 1; q < kBSUB; ++q) v += part[(5 * q + k) * kCB + lc];
+            pw[k] = v;
+        }
     }
 }
 
@@ -1188,10 +1256,10 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
         if ((err = SSD_SET_SMEM(chunk_state_kernel<N>, state_smem)) != cudaSuccess) return err;
         if ((err = SSD_SET_SMEM(chunk_bwd_kernel<N>, chunk_smem)) != cudaSuccess) return err;
         const dim3 tiles(cgrid, static_cast<unsigned>(ntiles(a.L)), static_cast<unsigned>(a.batch));
-        if (a.act_bf16)
-            SSD_LAUNCH(post_conv_kernel<true>, tiles, dim3(kT), 0, st, a, ws);
-        else
-            SSD_LAUNCH(post_conv_kernel<false>, tiles, dim3(kT), 0, st, a, ws);
+        const bool hist = a.init_conv_state != nullptr;
+        void (*post_conv)(BwdArgs, Ws) = a.act_bf16 ? (hist ? post_conv_kernel<true, true> : post_conv_kernel<true, false>)
+                                                    : (hist ? post_conv_kernel<false, true> : post_conv_kernel<false, false>);
+        SSD_LAUNCH(post_conv, tiles, dim3(kT), 0, st, a, ws);
         SSD_LAUNCH(dt_kernel,
                    dim3(static_cast<unsigned>(nc), static_cast<unsigned>((a.H + kT / 32 - 1) / (kT / 32)),
                         static_cast<unsigned>(a.batch)),
@@ -1244,11 +1312,11 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
     if (a.batch > 0) {
         const dim3 grid(static_cast<unsigned>((conv_dim + kCB - 1) / kCB), static_cast<unsigned>(nt),
                         static_cast<unsigned>(a.batch));
-        const size_t smem = 2 * 5 * kCB * sizeof(float);
-        if (a.act_bf16)
-            SSD_LAUNCH(conv_bwd_kernel<true>, grid, dim3(kT), smem, st, a, ws);
-        else
-            SSD_LAUNCH(conv_bwd_kernel<false>, grid, dim3(kT), smem, st, a, ws);
+        const size_t smem = kConvBwdSmem;
+        const bool hist = a.init_conv_state != nullptr;
+        void (*conv_bwd)(BwdArgs, Ws) = a.act_bf16 ? (hist ? conv_bwd_kernel<true, true> : conv_bwd_kernel<true, false>)
+                                                   : (hist ? conv_bwd_kernel<false, true> : conv_bwd_kernel<false, false>);
+        SSD_LAUNCH(conv_bwd, grid, dim3(kT), smem, st, a, ws);
     }
     SSD_LAUNCH(reduce_kernel, dim3(static_cast<unsigned>((conv_dim + 31) / 32 + (a.H + 31) / 32)), dim3(kT),
                5 * (size_t)kT * sizeof(float), st, a, ws);
