@@ -192,14 +192,20 @@ constexpr int kPC = 32;                // post_conv: channel pairs per CTA
 constexpr int kPST = kCT * kPC / kT;   // post_conv: tokens per thread (kT / kPC sub-tiles of the tile)
 static_assert(kPST * (kT / kPC) == kCT, "the sub-tiles cover the tile");
 // conv_bwd stages its tile in shared memory instead: kCB channels x (kCT + 6) pre-conv rows and (kCT + 3) du
-// rows arrive by cp.async, so the loads in flight hold no registers; then kT / kCB sub-tiles of kBST tokens
-// per channel compute from shared memory.
-constexpr int kCB = 64;                      // channels per CTA
-constexpr int kBSUB = kT / kCB;              // sub-tiles per tile (4)
-constexpr int kBST = kCT / kBSUB;            // tokens per thread (8)
+// rows arrive by cp.async, so the loads in flight hold no registers, and each row is read as one kCB-channel
+// run (DRAM serves long runs of a row better than many short ones); then each thread takes a channel pair
+// (packed fp32 arithmetic) and kBST tokens of the tile, in two passes through shared memory.
+constexpr int kCB = 128;                     // channels per CTA
+constexpr int kBPairs = kCB / 2;             // channel pairs per CTA
+constexpr int kBSUB = kT / kBPairs;          // sub-tiles per tile
+constexpr int kBST = kCT / kBSUB;            // tokens per thread
 constexpr int kRawRows = kCT + 6, kDuRows = kCT + 3;
-constexpr size_t kConvBwdSmem = (size_t)kRawRows * kCB * 4 + 2 * (size_t)kDuRows * kCB * 4 + (size_t)kBSUB * 5 * kCB * 4;
-static_assert(kBST * kBSUB == kCT && kCB % 8 == 0, "the sub-tiles cover the tile; whole 16-byte chunks per row");
+static_assert(kBST * kBSUB == kCT && kCB % 8 == 0 && kBPairs % 32 == 0,
+              "the sub-tiles cover the tile; whole 16-byte chunks per row; a warp within one sub-tile");
+// shared memory of conv_bwd_kernel: the staged pre-conv rows (element size esz), du and du2 rows, partials
+inline size_t conv_bwd_smem(size_t esz) {
+    return (size_t)kRawRows * kCB * esz + 2 * (size_t)kDuRows * kCB * 4 + (size_t)kBSUB * 5 * kCB * 4;
+}
 
 // Channels c, c + 1 of one token from its row: bf16 pairs as one 32-bit load, fp32 pairs as one 64-bit load.
 __device__ __forceinline__ float2 act_pair(const unsigned short* p) {
@@ -1069,25 +1075,31 @@ __device__ __forceinline__ const T* raw_col(const BwdArgs& a, int c, int HP, int
     return static_cast<const T*>(a.C) + (c - HP - GN);
 }
 
-// grid (ceil(conv_dim / kCB), ntiles, batch), kT threads, kConvBwdSmem bytes of dynamic shared memory.
+// Channels c, c + 1 of a staged row (c even): one 32-bit (bf16) or 64-bit (fp32) shared load.
+__device__ __forceinline__ float2 pair_at(const unsigned short* row, int c) { return act_pair(row + c); }
+__device__ __forceinline__ float2 pair_at(const float* row, int c) { return *reinterpret_cast<const float2*>(row + c); }
+__device__ __forceinline__ float2 dsilu_fast2(float2 v) { return make_float2(dsilu_fast(v.x), dsilu_fast(v.y)); }
+
+// grid (ceil(conv_dim / kCB), ntiles, batch), kT threads, conv_bwd_smem(sizeof(T)) bytes of dynamic shared memory.
 // With v_t the pre-SiLU conv output, dv_t = du_t silu'(v_t), and the pre-conv gradient of token s is
 // w0 dv_{s+3} + w1 dv_{s+2} + w2 dv_{s+1} + w3 dv_s.  The CTA first stages the pre-conv values of tokens
 // tb - 3 .. tb + kCT + 2 (tb the tile's first token; the conv history, or zero, before token 0) and du (plus
-// the second half's dB | dC) of tokens tb .. tb + kCT + 2, zero past the sequence; then thread (channel lc,
-// sub-tile) computes dv for its kBST tokens and the 3 after, its kBST gradients and its share of the tile's
-// conv_w / conv_b partials (summed over the sub-tiles in their order).  HP = 64 H and GN = G N (N a multiple
-// of 16) are multiples of 8, so a 16-byte chunk of a row never straddles x / B / C or conv_dim, and every
-// chunk is 16-byte aligned (the entry point rejects unaligned arrays).  kBf16 = a.act_bf16, kHist =
-// (a.init_conv_state != null).
+// the second half's dB | dC) of tokens tb .. tb + kCT + 2, zero past the sequence.  Then thread (pair pr,
+// sub-tile) computes dv of its kBST tokens once (the last sub-tile also the 3 tokens after the tile), in place
+// of du, with its share of the tile's conv_w / conv_b partials; and, after a barrier, the kBST gradients from
+// dv of its tokens and the 3 after.  The partials are summed over the sub-tiles in their order.
+// HP = 64 H and GN = G N (N a multiple of 16) are multiples of 8, so a 16-byte chunk of a row never straddles
+// x / B / C or conv_dim, every chunk is 16-byte aligned (the entry point rejects unaligned arrays), and a
+// channel pair never straddles an array.  kBf16 = a.act_bf16, kHist = (a.init_conv_state != null).
 template <bool kBf16, bool kHist>
 __global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
     using T = typename std::conditional<kBf16, unsigned short, float>::type;
     constexpr int kE = 16 / sizeof(T);  // elements per 16-byte chunk
     unsigned char* smem = SSD_DYN_SMEM();
-    T* raw_s = reinterpret_cast<T*>(smem);                                   // [kRawRows][kCB]
-    float* du_s = reinterpret_cast<float*>(smem + (size_t)kRawRows * kCB * 4);  // [kDuRows][kCB]
-    float* du2_s = du_s + kDuRows * kCB;                                     // [kDuRows][kCB]
-    float* part = du2_s + kDuRows * kCB;                                     // [kBSUB][5][kCB]
+    T* raw_s = reinterpret_cast<T*>(smem);                                               // [kRawRows][kCB]
+    float* du_s = reinterpret_cast<float*>(smem + (size_t)kRawRows * kCB * sizeof(T));  // [kDuRows][kCB]: du, then dv
+    float* du2_s = du_s + kDuRows * kCB;                                        // [kDuRows][kCB]
+    float* part = du2_s + kDuRows * kCB;                                        // [kBSUB][5][kCB]
     const int HP = a.H * a.P, GN = a.G * a.N, conv_dim = HP + 2 * GN, L = static_cast<int>(a.L);
     const int tid = threadIdx.x, c0 = blockIdx.x * kCB, b = blockIdx.z, tile = blockIdx.y, tb = tile * kCT;
     const int64_t row0 = (int64_t)b * L;
@@ -1121,70 +1133,97 @@ __global__ void __launch_bounds__(kT) conv_bwd_kernel(BwdArgs a, Ws ws) {
     cp_async_wait_all();
     __syncthreads();
 
-    const int lc = tid % kCB, sub = tid / kCB, c = c0 + lc, t0 = tb + sub * kBST;
-    const bool live = c < conv_dim;  // threads past the last channel still meet the barrier
+    const int pr = tid % kBPairs, sub = tid / kBPairs;  // sub is the warp: every branch on it is uniform
+    const int lcp = 2 * pr, c = c0 + lcp, i0 = sub * kBST;  // channels c, c + 1; rows i0 .. of the tile
+    const bool live = c < conv_dim;  // conv_dim is even: both channels of the pair or neither
     const int cc = live ? c : 0;
-    const float w0 = a.conv_w[cc * 4 + 0], w1 = a.conv_w[cc * 4 + 1], w2 = a.conv_w[cc * 4 + 2],
-                w3 = a.conv_w[cc * 4 + 3], bias = a.conv_b[cc];
-    // tokens of t0 .. t0 + kBST + 2 that exist (negative past the end; -3 for a thread past the last channel)
-    const int n = live ? (L - t0 < kBST + 3 ? L - t0 : kBST + 3) : -3;
-    float r[kBST + 6], d[kBST + 3];  // r[i]: pre-conv value of token t0 - 3 + i; d[i]: du, then dv, of t0 + i
-#pragma unroll
-    for (int i = 0; i < kBST + 6; ++i) r[i] = act_to_f(raw_s[(sub * kBST + i) * kCB + lc]);
+    float2 w[4], bias;
+    {
+        const float4 wa = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cc * 4);
+        const float4 wb = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cc * 4 + 4);
+        w[0] = make_float2(wa.x, wb.x), w[1] = make_float2(wa.y, wb.y);
+        w[2] = make_float2(wa.z, wb.z), w[3] = make_float2(wa.w, wb.w);
+        bias = make_float2(a.conv_b[cc], a.conv_b[cc + 1]);
+    }
+    // pass 1: dv of tokens tb + i0 .. (kBST of them; kBST + 3 for the last sub-tile), from the pre-conv rows
+    // i0 .. i0 + n1 + 2 (staged row k holds token tb - 3 + k)
+    constexpr int kN1 = kBST + 3;
+    const int n1 = sub == kBSUB - 1 ? kN1 : kBST;
     const bool second = add2 && c >= HP;
+    // a sliding window over the staged rows: r0..r2 the three before token tb + i0 + k, r3 its own
+    float2 r0 = pair_at(raw_s + i0 * kCB, lcp), r1 = pair_at(raw_s + (i0 + 1) * kCB, lcp),
+           r2 = pair_at(raw_s + (i0 + 2) * kCB, lcp);
+    float2 g[5];
 #pragma unroll
-    for (int i = 0; i < kBST + 3; ++i) {
-        d[i] = du_s[(sub * kBST + i) * kCB + lc];
-        if (second) d[i] += du2_s[(sub * kBST + i) * kCB + lc];
-    }
-    float gw0 = 0.f, gw1 = 0.f, gw2 = 0.f, gw3 = 0.f, gb = 0.f;
+    for (int k = 0; k < 5; ++k) g[k] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < kBST + 3; ++i) {
-        const float v = bias + w0 * r[i] + w1 * r[i + 1] + w2 * r[i + 2] + w3 * r[i + 3];
-        d[i] = i < n ? d[i] * dsilu_fast(v) : 0.f;
-        if (i < kBST) {
-            gw0 += d[i] * r[i];
-            gw1 += d[i] * r[i + 1];
-            gw2 += d[i] * r[i + 2];
-            gw3 += d[i] * r[i + 3];
-            gb += d[i];
+    for (int k = 0; k < kN1; ++k) {
+        if (k < n1) {
+            const int i = i0 + k, t = tb + i;
+            const float2 r3 = pair_at(raw_s + (i + 3) * kCB, lcp);
+            float2 v = __ffma2_rn(w[0], r0, bias);
+            v = __ffma2_rn(w[1], r1, v);
+            v = __ffma2_rn(w[2], r2, v);
+            v = __ffma2_rn(w[3], r3, v);
+            float2* dup = reinterpret_cast<float2*>(du_s + i * kCB + lcp);
+            float2 du = *dup;
+            if (second) du = __fadd2_rn(du, *reinterpret_cast<const float2*>(du2_s + i * kCB + lcp));
+            const float2 dv = t < L ? __fmul2_rn(du, dsilu_fast2(v)) : make_float2(0.f, 0.f);
+            *dup = dv;
+            if (i < kCT) {  // the tile's own tokens (dv is zero past the sequence)
+                g[0] = __ffma2_rn(dv, r0, g[0]);
+                g[1] = __ffma2_rn(dv, r1, g[1]);
+                g[2] = __ffma2_rn(dv, r2, g[2]);
+                g[3] = __ffma2_rn(dv, r3, g[3]);
+                g[4] = __fadd2_rn(dv, g[4]);
+            }
+            r0 = r1;
+            r1 = r2;
+            r2 = r3;
         }
     }
-    if (live) {
-        float* out;
-        const int rs = cc < HP ? HP : GN;
-        if (cc < HP)
-            out = a.dx + cc;
-        else if (cc < HP + GN)
-            out = a.dB + (cc - HP);
-        else
-            out = a.dC + (cc - HP - GN);
-        out += (row0 + t0) * rs;
 #pragma unroll
-        for (int j = 0; j < kBST; ++j)
-            if (j < n) out[j * rs] = w0 * d[j + 3] + w1 * d[j + 2] + w2 * d[j + 1] + w3 * d[j];
-        if (t0 == 0 && a.d_init_conv_state) {
-            // the history tokens s = -3, -2, -1 (dv is zero before token 0)
-            float* dh = a.d_init_conv_state + ((int64_t)b * conv_dim + cc) * 3;
-            dh[0] = w0 * d[0];
-            dh[1] = w0 * d[1] + w1 * d[0];
-            dh[2] = w0 * d[2] + w1 * d[1] + w2 * d[0];
-        }
-    }
-    float* mine = part + sub * 5 * kCB + lc;
-    mine[0] = gw0;
-    mine[kCB] = gw1;
-    mine[2 * kCB] = gw2;
-    mine[3 * kCB] = gw3;
-    mine[4 * kCB] = gb;
+    for (int k = 0; k < 5; ++k) *reinterpret_cast<float2*>(part + (sub * 5 + k) * kCB + lcp) = g[k];
     __syncthreads();
-    if (sub == 0 && live) {
-        float* pw = ws.PW + (((int64_t)b * ntiles(a.L) + tile) * conv_dim + c) * 5;
+    // pass 2: the gradients of tokens tb + i0 .. tb + i0 + kBST - 1 from dv of rows i0 .. i0 + kBST + 2
+    if (live) {
+        const auto dv_at = [&](int k) { return *reinterpret_cast<const float2*>(du_s + (i0 + k) * kCB + lcp); };
+        const int rs = cc < HP ? HP : GN;
+        float* out = cc < HP ? a.dx + cc : (cc < HP + GN ? a.dB + (cc - HP) : a.dC + (cc - HP - GN));
+        out += (row0 + tb + i0) * rs;
+        const int n = L - tb - i0;  // tokens of the sub-tile that exist (may be <= 0)
+        // a sliding window: d0..d3 = dv of tokens j .. j + 3 of the sub-tile
+        float2 d0 = dv_at(0), d1 = dv_at(1), d2 = dv_at(2);
+        const float2 e0 = d0, e1 = d1, e2 = d2;  // for the conv history below
+#pragma unroll
+        for (int j = 0; j < kBST; ++j) {
+            const float2 d3 = dv_at(j + 3);
+            float2 o = __fmul2_rn(w[0], d3);
+            o = __ffma2_rn(w[1], d2, o);
+            o = __ffma2_rn(w[2], d1, o);
+            o = __ffma2_rn(w[3], d0, o);
+            if (j < n) *reinterpret_cast<float2*>(out + j * rs) = o;
+            d0 = d1;
+            d1 = d2;
+            d2 = d3;
+        }
+        if (tb + i0 == 0 && a.d_init_conv_state) {
+            // the history tokens s = -3, -2, -1 of channels c, c + 1 (dv is zero before token 0)
+            float* dh = a.d_init_conv_state + ((int64_t)b * conv_dim + cc) * 3;
+            const float2 h0 = __fmul2_rn(w[0], e0);
+            const float2 h1 = __ffma2_rn(w[1], e0, __fmul2_rn(w[0], e1));
+            const float2 h2 = __ffma2_rn(w[2], e0, __ffma2_rn(w[1], e1, __fmul2_rn(w[0], e2)));
+            dh[0] = h0.x, dh[1] = h1.x, dh[2] = h2.x;
+            dh[3] = h0.y, dh[4] = h1.y, dh[5] = h2.y;
+        }
+    }
+    if (tid < kCB && c0 + tid < conv_dim) {
+        float* pw = ws.PW + (((int64_t)b * ntiles(a.L) + tile) * conv_dim + c0 + tid) * 5;
 #pragma unroll
         for (int k = 0; k < 5; ++k) {
-            float v = part[k * kCB + lc];
+            float v = part[k * kCB + tid];
 #pragma unroll
-            for (int q = 1; q < kBSUB; ++q) v += part[(5 * q + k) * kCB + lc];
+            for (int q = 1; q < kBSUB; ++q) v += part[(5 * q + k) * kCB + tid];
             pw[k] = v;
         }
     }
@@ -1312,10 +1351,11 @@ cudaError_t launch_n(const BwdArgs& a, const Ws& ws, cudaStream_t st) {
     if (a.batch > 0) {
         const dim3 grid(static_cast<unsigned>((conv_dim + kCB - 1) / kCB), static_cast<unsigned>(nt),
                         static_cast<unsigned>(a.batch));
-        const size_t smem = kConvBwdSmem;
+        const size_t smem = conv_bwd_smem(a.act_bf16 ? 2 : 4);
         const bool hist = a.init_conv_state != nullptr;
         void (*conv_bwd)(BwdArgs, Ws) = a.act_bf16 ? (hist ? conv_bwd_kernel<true, true> : conv_bwd_kernel<true, false>)
                                                    : (hist ? conv_bwd_kernel<false, true> : conv_bwd_kernel<false, false>);
+        if ((err = SSD_SET_SMEM(conv_bwd, smem)) != cudaSuccess) return err;
         SSD_LAUNCH(conv_bwd, grid, dim3(kT), smem, st, a, ws);
     }
     SSD_LAUNCH(reduce_kernel, dim3(static_cast<unsigned>((conv_dim + 31) / 32 + (a.H + 31) / 32)), dim3(kT),

@@ -152,6 +152,10 @@ inline float4 __ldcs(const float4* p) { return *p; }
 inline void __stcs(float4* p, float4 v) { *p = v; }
 inline float __expf(float v) { return expf(v); }
 inline float __fdividef(float a, float b) { return a / b; }
+// Blackwell's packed fp32 arithmetic, lane by lane
+inline float2 __ffma2_rn(float2 x, float2 y, float2 z) { return make_float2(fmaf(x.x, y.x, z.x), fmaf(x.y, y.y, z.y)); }
+inline float2 __fmul2_rn(float2 x, float2 y) { return make_float2(x.x * y.x, x.y * y.y); }
+inline float2 __fadd2_rn(float2 x, float2 y) { return make_float2(x.x + y.x, x.y + y.y); }
 
 // bf16 storage: round to nearest, ties to even, on the 16 dropped bits (NaN kept quiet)
 struct __nv_bfloat16 {

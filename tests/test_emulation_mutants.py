@@ -22,7 +22,8 @@ MUTANTS = {
     # reads x one token past the tile: beyond the array for the last tile of the last sequence
     "post-conv reads past its tile": ("r[i] = act_pair(src + (i - 3) * rs);", "r[i] = act_pair(src + (i - 2) * rs);"),
     # writes each pre-conv gradient one token late: beyond dx / dB / dC for the last token
-    "conv backward writes one row late": ("if (j < n) out[j * rs] =", "if (j < n) out[(j + 1) * rs] ="),
+    "conv backward writes one row late": ("if (j < n) *reinterpret_cast<float2*>(out + j * rs) = o;",
+                                          "if (j < n) *reinterpret_cast<float2*>(out + (j + 1) * rs) = o;"),
     # leaves the rows of a ragged chunk past its end as they were (NaN bytes for the first head)
     "ragged rows not cleared": ("            xs[j * kS + p] = xv;", "            if (j < Qv) xs[j * kS + p] = xv;"),
     # shared rows no longer 16-byte aligned: the emulation's alignment check must stop the vector loads
