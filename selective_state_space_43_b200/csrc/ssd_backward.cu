@@ -188,7 +188,7 @@ __device__ __forceinline__ float raw_at(const BwdArgs& a, int64_t b, int64_t s, 
 // The two conv kernels spread a kCT-token tile over several threads per channel: each thread takes a short
 // window, loads all of it, then computes, so that many loads are in flight without long per-thread chains
 // (measured: both the 2-token streaming loop and one thread per whole tile leave HBM well under half busy).
-constexpr int kPC = 32;                // post_conv: channel pairs per CTA
+constexpr int kPC = 64;                // post_conv: channel pairs per CTA
 constexpr int kPST = kCT * kPC / kT;   // post_conv: tokens per thread (kT / kPC sub-tiles of the tile)
 static_assert(kPST * (kT / kPC) == kCT, "the sub-tiles cover the tile");
 // conv_bwd stages its tile in shared memory instead: kCB channels x (kCT + 6) pre-conv rows and (kCT + 3) du
