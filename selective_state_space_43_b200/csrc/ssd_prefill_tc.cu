@@ -73,7 +73,11 @@ using namespace sm100;
 
 constexpr int kQ = 128, kP = 64, kN = 128;
 constexpr int kThreads = 640;
-constexpr int kWarpRaw = 0, kWarpMma = 1, kWarpCs = 2, kWarpBc = 3, kFirstCompute = 4;
+// Warp w issues from scheduler w % 4, which it shares with the compute warps of TMEM lane quadrant w % 4.
+// The causal mask gives quadrant q (rows 32q .. 32q + 31) about q + 1 times quadrant 0's work, so the
+// busiest single-warp role (the cumsum / tables warp, ~800 instructions per chunk) sits on scheduler 0 and
+// the light TMA producer on scheduler 2.
+constexpr int kWarpRaw = 2, kWarpMma = 1, kWarpCs = 0, kWarpBc = 3, kFirstCompute = 4;
 // The 16 compute warps form two groups of 8 (two warps per TMEM lane quadrant in each), specialised by
 // phase so that the phases of neighbouring chunks overlap: group A (warps 4-11) builds each chunk's decay
 // mask and runs its epilogue, group B (warps 12-19) runs the x conv and the state pass.
