@@ -99,29 +99,33 @@ constexpr uint32_t OFF_DTRAW = OFF_SMALL;              // 2 stages [128 tok][8 h
 constexpr uint32_t OFF_WT = OFF_DTRAW + 2 * 2048;      // conv taps of the head's x channels [4][64] float
 constexpr uint32_t OFF_CB = OFF_WT + 4 * 64 * 4;       // conv bias [64] float
 constexpr uint32_t OFF_HALO = OFF_CB + 64 * 4;         // [2][3][64] bf16 raw x history
-constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;  // cs [2][128] float (double-buffered by chunk parity)
-constexpr uint32_t OFF_COLF = OFF_CS + 2 * 128 * 4;    // exp(cs_end(g(j)) - cs_j) dt_j [2][128]
-constexpr uint32_t OFF_WX = OFF_COLF + 2 * 128 * 4;    // weight of x_j in the chunk state [2][128]
+// the cumsum warp's per-chunk vectors, three chunks deep (slot c % 3), so that it can run ahead of both
+// compute groups: a slot is rewritten once both groups are done with the chunk three back
+constexpr int kCsSlots = 3;
+constexpr uint32_t OFF_CS = OFF_HALO + 2 * 3 * 64 * 2;      // cs [3][128] float
+constexpr uint32_t OFF_COLF = OFF_CS + kCsSlots * 128 * 4;  // exp(cs_end(g(j)) - cs_j) dt_j [3][128]
+constexpr uint32_t OFF_WX = OFF_COLF + kCsSlots * 128 * 4;  // weight of x_j in the chunk state [3][128]
 // decay tables of one chunk (single buffer: rewritten once every thread's mask of the previous chunk is done);
 // g = 8-row group, cs_end(g) = cs at the group's last row
-constexpr uint32_t OFF_RFAC = OFF_WX + 2 * 128 * 4;    // exp(cs_i - cs_end(g(i)-1)) [128]
+constexpr uint32_t OFF_RFAC = OFF_WX + kCsSlots * 128 * 4;  // exp(cs_i - cs_end(g(i)-1)) [128]
 constexpr uint32_t OFF_PG = OFF_RFAC + 128 * 4;        // exp(cs_end(gi-1) - cs_end(g)), g < gi: [16 gi][4 q][4 kb]
 constexpr uint32_t OFF_DG = OFF_PG + 256 * 4;          // exp(cs_i - cs_j) dt_j inside a group, j <= i: [16][8][8]
 constexpr uint32_t OFF_BAR = OFF_DG + 1024 * 4;        // mbarriers (8 B each)
-constexpr int NBAR = 21;
+constexpr int NBAR = 23;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;  // TMEM base address
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// FULL_RAW / XREADY / EPI_DONE / CS_* come in pairs by chunk parity (a waiter of one group may be a whole
+// FULL_RAW / XREADY / EPI_DONE come in pairs by chunk parity, CS_* in threes by chunk mod 3 (a waiter of one group may be a whole
 // chunk behind the other group, and a barrier must never run two phases past a waiter); EPI_DONE = a
 // chunk's epilogue is complete (its Y / Y2 / z / conv output read, its y written); EMPTY_BC = the chunk's
 // last B / C reader (Y2) is complete; SREADY = the state entering the next chunk is in shared memory.
 enum Bar { FULL_RAW0 = 0, FULL_RAW1, XREADY0, XREADY1, FULL_Z, EPI_DONE0, EPI_DONE1, FULL_BC, EMPTY_BC, MREADY,
-           G_FULL, SC_FULL, Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1, TAB_READY, SREADY,
-           NEVER };  // NEVER: nothing arrives on it (the test stall of the timeout path waits on it)
+           G_FULL, SC_FULL, Y_FULL, MMA_DONE, CS_READY0, CS_READY1, CS_READY2, CS_FREE0, CS_FREE1, CS_FREE2,
+           TAB_READY, SREADY, NEVER };  // NEVER: nothing arrives on it (the test stall of the timeout path waits on it)
+static_assert(NEVER + 1 == NBAR, "barrier count");
 
 // TMEM columns (fp32, 128 lanes): G = C B^T, Y = M X, Y2 = C S^T, S_c, the running state, and the
 // post-conv x of two chunks (for the D skip)
@@ -213,7 +217,8 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
                                            int half) {
     const int buf = cc & 1;
     // this chunk's cumsum (its raw x tile arrived before it) and raw x
-    if (!warp_wait2(&bars[CS_READY0 + buf], (cc >> 1) & 1, &bars[FULL_RAW0 + buf], (cc >> 1) & 1, abort_flag))
+    if (!warp_wait2(&bars[CS_READY0 + cc % kCsSlots], (cc / kCsSlots) & 1, &bars[FULL_RAW0 + buf], (cc >> 1) & 1,
+                    abort_flag))
         return false;
     // the raw history rows were written by other threads in the previous chunk's conv; the X tile and the
     // conv output of this parity were last read by chunk cc-2's Y MMA and epilogue
@@ -231,7 +236,7 @@ __device__ __forceinline__ bool conv_chunk(const PrefillArgs& a, uint8_t* sm, ui
     const uint4* halo_in = reinterpret_cast<const uint4*>(sm + OFF_HALO + (cc & 1) * 384);
     const float4* wt = reinterpret_cast<const float4*>(sm + OFF_WT);   // [tap][64 channels]
     const float4* cb = reinterpret_cast<const float4*>(sm + OFF_CB);
-    const float wxr = s_wx_at(sm, buf, i);
+    const float wxr = s_wx_at(sm, cc % kCsSlots, i);
     uint8_t* sX = sm + OFF_X + buf * 16384;
     uint8_t* sXp = sm + OFF_XP;
 #pragma unroll 1
@@ -389,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
-    float* s_cs = reinterpret_cast<float*>(sm + OFF_CS);      // [2][128] per chunk parity
+    float* s_cs = reinterpret_cast<float*>(sm + OFF_CS);      // [3][128] by chunk mod 3
     float* s_colf = reinterpret_cast<float*>(sm + OFF_COLF);
     float* s_wx = reinterpret_cast<float*>(sm + OFF_WX);
     constexpr bool kTmaStoreY = sizeof(TY) == 2;  // bf16 y goes out through TMA from the stage it was written in
@@ -412,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             uint32_t cnt = 1;
             if (k == XREADY0 || k == XREADY1) cnt = kGroupThreads;                      // group B
             if (k == EPI_DONE0 || k == EPI_DONE1 || k == MREADY) cnt = kGroupThreads;   // group A
-            if (k == CS_FREE0 || k == CS_FREE1 || k == SREADY) cnt = 2 * kGroupThreads; // both
-            if (k == CS_READY0 || k == CS_READY1 || k == TAB_READY) cnt = 32;
+            if (k == CS_FREE0 || k == CS_FREE1 || k == CS_FREE2 || k == SREADY) cnt = 2 * kGroupThreads;  // both
+            if (k == CS_READY0 || k == CS_READY1 || k == CS_READY2 || k == TAB_READY) cnt = 32;
             mbar_init(&bars[k], cnt);
         }
         *abort_flag = 0;
@@ -532,10 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         const float A = a.A[h], dtb = a.dt_bias[h];
         for (int c = 0; c < nc; ++c) {
             // dt = softplus(dt_raw + bias) and the inclusive cumsum of dt*A over the chunk's 128 rows,
-            // into the buffer of this chunk's parity once every compute thread is done with it; the raw
-            // dt tile arrives with the chunk's raw x
-            const int buf = c & 1;
-            if (c >= 2 && !warp_wait(&bars[CS_FREE0 + buf], ((c >> 1) + 1) & 1, abort_flag)) {
+            // into slot c % 3 once every compute thread is done with chunk c - 3; the raw dt tile arrives
+            // with the chunk's raw x (stage c & 1)
+            const int buf = c & 1, cb = c % kCsSlots;
+            if (c >= kCsSlots && !warp_wait(&bars[CS_FREE0 + cb], ((c / kCsSlots) + 1) & 1, abort_flag)) {
                 raise_abort(abort_flag);
                 break;
             }
@@ -600,10 +605,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 cf[k] = sm_k * dtv[k];             // exp(cs_end(gi) - cs_j) dt_j
                 wx[k] = sm_k * later * dtv[k];     // exp(cs_last - cs_j) dt_j
             }
-            reinterpret_cast<float4*>(s_cs + buf * 128)[lane] = make_float4(csr[0], csr[1], csr[2], csr[3]);
-            reinterpret_cast<float4*>(s_colf + buf * 128)[lane] = make_float4(cf[0], cf[1], cf[2], cf[3]);
-            reinterpret_cast<float4*>(s_wx + buf * 128)[lane] = make_float4(wx[0], wx[1], wx[2], wx[3]);
-            mbar_arrive(&bars[CS_READY0 + buf]);
+            reinterpret_cast<float4*>(s_cs + cb * 128)[lane] = make_float4(csr[0], csr[1], csr[2], csr[3]);
+            reinterpret_cast<float4*>(s_colf + cb * 128)[lane] = make_float4(cf[0], cf[1], cf[2], cf[3]);
+            reinterpret_cast<float4*>(s_wx + cb * 128)[lane] = make_float4(wx[0], wx[1], wx[2], wx[3]);
+            mbar_arrive(&bars[CS_READY0 + cb]);
 
             // decay tables of this chunk, once every thread's mask of the previous chunk has read them
             if (c >= 1 && !warp_wait(&bars[MREADY], (c - 1) & 1, abort_flag)) { raise_abort(abort_flag); break; }
@@ -735,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 const float4 p4b = reinterpret_cast<const float4*>(sm + OFF_PG)[gi * 4 + 2 * half + 1];
                 const float pk[2][4] = {{p4a.x, p4a.y, p4a.z, p4a.w}, {p4b.x, p4b.y, p4b.z, p4b.w}};
                 const float4* drow = reinterpret_cast<const float4*>(sm + OFF_DG) + (gi * 8 + (i & 7)) * 2;
-                const float* colf_b = s_colf + buf * 128;
+                const float* colf_b = s_colf + (c % kCsSlots) * 128;
 #pragma unroll
                 for (int kb2 = 0; kb2 < 4; kb2 += 2) {
                     float gv[2][16];  // two 32-column blocks per TMEM round trip (warp-uniform: blocks right of
@@ -783,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             mbar_arrive(&bars[MREADY]);
 
             // (f) this thread's half of the state pass of chunk c
-            if (!state_half(sm, bars, abort_flag, tmem, lane_base, c, s_cs[buf * 128 + kQ - 1], i, 32 * half)) {
+            if (!state_half(sm, bars, abort_flag, tmem, lane_base, c, s_cs[(c % kCsSlots) * 128 + kQ - 1], i, 32 * half)) {
                 raise_abort(abort_flag);
                 break;
             }
@@ -799,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             tc_fence_after();
             {
                 uint8_t* rz = sm + OFF_Z;  // z in, y out (same positions, this thread's only)
-                const float ecs = __expf(s_cs[buf * 128 + i]);  // decay of S_prev up to row i
+                const float ecs = __expf(s_cs[(c % kCsSlots) * 128 + i]);  // decay of S_prev up to row i
                 const float2 e2 = make_float2(ecs, ecs), d2 = make_float2(Dh, Dh);
 #pragma unroll 1
                 for (int sub = 0; sub < 2; ++sub) {
@@ -853,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[EPI_DONE0 + buf]);
-            mbar_arrive(&bars[CS_FREE0 + buf]);  // group A's reads of this chunk's cumsum buffer are done
+            mbar_arrive(&bars[CS_FREE0 + c % kCsSlots]);  // group A's reads of this chunk's cumsum slot are done
         }
         // final state of this thread's columns (an empty sequence passes its initial state through)
         if (!*abort_flag) state_final(a, tmem, lane_base, b, h, i, 32 * half);
@@ -876,11 +881,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
                 break;
             }
             // (f) this thread's half of the state pass of chunk c
-            if (!state_half(sm, bars, abort_flag, tmem, lane_base, c, s_cs[buf * 128 + kQ - 1], i, 32 * half + 16)) {
+            if (!state_half(sm, bars, abort_flag, tmem, lane_base, c, s_cs[(c % kCsSlots) * 128 + kQ - 1], i,
+                            32 * half + 16)) {
                 raise_abort(abort_flag);
                 break;
             }
-            mbar_arrive(&bars[CS_FREE0 + buf]);  // group B's reads of this chunk's cumsum buffer are done
+            mbar_arrive(&bars[CS_FREE0 + c % kCsSlots]);  // group B's reads of this chunk's cumsum slot are done
         }
         if (!*abort_flag) state_final(a, tmem, lane_base, b, h, i, 32 * half + 16);
     }
