@@ -52,7 +52,7 @@ def test_single_rank_needs_no_process_group():
     assert ms == 0.5 and value == pytest.approx(4096 / 0.5e-3)
 
 
-def test_algorithmic_byte_and_flop_counts_match_the_survey_figures():
+def test_algorithmic_byte_and_flop_counts_per_token():
     from selective_state_space_43_b200.synth import WORKLOADS
     d = WORKLOADS["nemotron_h_8b"]["dims"]
     # 53,504 B per token of activations plus the 4.19 MB final state and the conv tail
