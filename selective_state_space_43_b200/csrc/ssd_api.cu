@@ -363,12 +363,13 @@ ssd_status ssd_mimo_decode_step(const ssd_dims* d, int32_t rank, ssd_dtype dtype
 ssd_status ssd_device_status(void* stream) {
     int flag = 0;
     if (ssd::read_and_clear_tc_error(&flag, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSD_ERR_CUDA;
-    int mimo_flag = 0, bwd_flag = 0, chunk_bwd_flag = 0;
+    int mimo_flag = 0, bwd_flag = 0, chunk_bwd_flag = 0, decode_flag = 0;
+    if (ssd::read_and_clear_decode_error(&decode_flag) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::mimo::read_and_clear_mimo_error(&mimo_flag) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::bwd::read_and_clear_bwd_tc_error(&bwd_flag) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::bwd::read_and_clear_chunk_bwd_tc_error(&chunk_bwd_flag) != cudaSuccess) return SSD_ERR_CUDA;
     // the backward kernels' words: bit 0 a bounded wait gave up, bit 1 an operand beyond fp16 range
-    if ((flag & ssd::kErrTimeout) || mimo_flag || ((bwd_flag | chunk_bwd_flag) & 1)) return SSD_ERR_TIMEOUT;
+    if ((flag & ssd::kErrTimeout) || mimo_flag || decode_flag || ((bwd_flag | chunk_bwd_flag) & 1)) return SSD_ERR_TIMEOUT;
     if ((bwd_flag | chunk_bwd_flag) & 2) return SSD_ERR_RANGE;
     return flag & ssd::kErrBadSeqlens ? SSD_ERR_SHAPE : SSD_OK;
 }

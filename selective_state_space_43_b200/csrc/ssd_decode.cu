@@ -9,26 +9,43 @@
 //     post-conv channels it needs (64 x channels of its head, 2N B/C channels
 //     of its group) from the 3-column conv window plus the new token, and
 //     rolls the window of its own x channels;
-//   * the P x N fp32 state is streamed with 16-byte vectors: a row of N floats
-//     is covered by N/4 lanes, every load of the CTA is issued before the first
-//     FMA (P*N*4/256 bytes in flight per thread), loads and stores use the
-//     streaming cache hint since nothing is re-read within the step;
+//   * the P x N fp32 state moves as one bulk copy (cp.async.bulk) into shared
+//     memory and one back out, so the bytes in flight per SM are set by the
+//     CTAs resident (6 per SM, ~34 KB of shared memory each at N = 128), not by
+//     registers; the CTA computes the conv channels while the load lands; a
+//     row of N floats is updated by N/4 lanes, a float4 each.  The wait for the
+//     load is bounded: a CTA whose load never lands sets the decode error word
+//     (reported by ssd_device_status as SSD_ERR_TIMEOUT) and writes no state;
 //   * y = S.C is a segmented warp reduction over the N/4 lanes of a row;
 //   * the shared B/C conv channels are rolled by a second, tiny kernel that
 //     runs after every head has read the old window.
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_sm100.cuh"
+
+extern __shared__ __align__(16) unsigned char ssd_decode_smem[];
 
 namespace ssd {
 
+__device__ int g_decode_error = 0;  // set when a CTA's state load never landed (bounded wait gave up)
+
+namespace {
+constexpr int kDecodeCtas = 6;  // resident CTAs per SM the register budget is sized for
+// shared memory of decode_state_kernel: the [P][N] state, the P + 2N post-conv channels, P read-outs, a barrier
+constexpr size_t decode_smem_bytes(int P, int N) { return ((size_t)P * N + P + 2 * N + P) * 4 + 8; }
+}  // namespace
+
 template <typename T, typename TY, int N>
-__global__ void __launch_bounds__(256) decode_state_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(256, kDecodeCtas) decode_state_kernel(DecodeArgs a) {
     constexpr int P = 64;
     constexpr int LPR = N / 4;           // lanes per state row (float4 each)
     constexpr int RPW = 32 / LPR;        // rows per warp per pass
     constexpr int ITER = P / (8 * RPW);  // passes over the P rows with 8 warps
-    __shared__ float s_u[P + 2 * N];     // post-conv x (P), B (N), C (N)
-    __shared__ float s_y[P];
+    constexpr uint32_t kStateBytes = P * N * 4;
+    float* s_st = reinterpret_cast<float*>(ssd_decode_smem);  // [P][N] the head's state
+    float* s_u = s_st + P * N;                                // post-conv x (P), B (N), C (N)
+    float* s_y = s_u + P + 2 * N;                             // [P]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(s_y + P);
 
     const int bh = blockIdx.x;
     const int b = bh / a.H, h = bh - b * a.H;
@@ -38,16 +55,14 @@ __global__ void __launch_bounds__(256) decode_state_kernel(DecodeArgs a) {
     const T* Bm = static_cast<const T*>(a.B);
     const T* Cm = static_cast<const T*>(a.C);
     T* conv_state = static_cast<T*>(a.conv_state);
+    float* gstate = a.ssm_state + (size_t)bh * P * N;
 
-    // Issue the state loads first: they are the step's traffic.
-    const int warp = tid >> 5, lane = tid & 31;
-    const int rsub = lane / LPR, n0 = (lane % LPR) * 4;
-    float4* S = reinterpret_cast<float4*>(a.ssm_state + (size_t)bh * P * N);
-    float4 v[ITER];
-#pragma unroll
-    for (int it = 0; it < ITER; ++it) {
-        const int p = (it * 8 + warp) * RPW + rsub;
-        v[it] = __ldcs(S + ((p * N + n0) >> 2));
+    // the state load first: it is the step's traffic
+    if (tid == 0) {
+        sm100::mbar_init(bar, 1);
+        sm100::fence_mbar_init();
+        sm100::mbar_arrive_expect_tx(bar, kStateBytes);
+        sm100::bulk_load(s_st, gstate, kStateBytes, bar);
     }
 
     for (int i = tid; i < P + 2 * N; i += 256) {
@@ -78,32 +93,48 @@ __global__ void __launch_bounds__(256) decode_state_kernel(DecodeArgs a) {
     }
     const float dtv = softplus_f(to_f32(static_cast<const T*>(a.dt)[(size_t)b * a.H + h]) + a.dt_bias[h]);
     const float decay = __expf(dtv * a.A[h]);
-    __syncthreads();
+    __syncthreads();  // the post-conv channels staged; the barrier's initialisation visible to every thread
 
+    const int warp = tid >> 5, lane = tid & 31;
+    const int rsub = lane / LPR, n0 = (lane % LPR) * 4;
     const float4 bq = make_float4(s_u[P + n0], s_u[P + n0 + 1], s_u[P + n0 + 2], s_u[P + n0 + 3]);
     const float4 cq = make_float4(s_u[P + N + n0], s_u[P + N + n0 + 1], s_u[P + N + n0 + 2], s_u[P + N + n0 + 3]);
+    // bounded wait for the state (about 2 s); a CTA whose load never lands flags it and writes no state
+    const bool landed = sm100::mbar_wait(bar, 0, nullptr);
+    if (__syncthreads_or(landed ? 0 : 1)) {
+        if (tid == 0) atomicOr(&g_decode_error, 1);
+        return;
+    }
 #pragma unroll
     for (int it = 0; it < ITER; ++it) {
         const int p = (it * 8 + warp) * RPW + rsub;
+        float4* srow = reinterpret_cast<float4*>(s_st + p * N + n0);
         const float xd = dtv * s_u[p];
-        float4 s = v[it];
+        float4 s = *srow;
         s.x = fmaf(decay, s.x, xd * bq.x);
         s.y = fmaf(decay, s.y, xd * bq.y);
         s.z = fmaf(decay, s.z, xd * bq.z);
         s.w = fmaf(decay, s.w, xd * bq.w);
-        __stcs(S + ((p * N + n0) >> 2), s);
+        *srow = s;
         float part = s.x * cq.x + s.y * cq.y + s.z * cq.z + s.w * cq.w;
 #pragma unroll
         for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if ((lane % LPR) == 0) s_y[p] = part;
     }
+    // the updated state goes back in one bulk store, once every thread's writes are visible to it
+    sm100::fence_async_smem();
     __syncthreads();
+    if (tid == 0) {
+        sm100::bulk_store(gstate, s_st, kStateBytes);
+        sm100::bulk_commit();
+    }
     if (tid < P) {
         const size_t off = (size_t)b * a.HP + (size_t)h * P + tid;
         const float yv = s_y[tid] + a.D[h] * s_u[tid];
         const float zv = to_f32(static_cast<const T*>(a.z)[off]);
         static_cast<TY*>(a.y)[off] = from_f32<TY>(yv * silu_f(zv));
     }
+    if (tid == 0) sm100::bulk_wait_read_all();  // shared memory must outlive the store's reads
 }
 
 // Roll the 2*G*N shared B/C conv channels by one token (after every head read them).
@@ -125,7 +156,7 @@ __global__ void __launch_bounds__(256) decode_roll_bc_kernel(DecodeArgs a, int64
 template <typename T, typename TY, int N>
 static cudaError_t launch_decode_t(const DecodeArgs& a, int64_t batch, cudaStream_t st, const TimingHook& hook) {
     hook.before(st);
-    decode_state_kernel<T, TY, N><<<(unsigned)(batch * a.H), 256, 0, st>>>(a);
+    decode_state_kernel<T, TY, N><<<(unsigned)(batch * a.H), 256, decode_smem_bytes(64, N), st>>>(a);
     hook.after(st);
     const int64_t total = batch * 2 * a.GN;
     if (total > 0) decode_roll_bc_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(a, total);
@@ -151,6 +182,13 @@ cudaError_t launch_decode(const DecodeArgs& a, int64_t batch, ActKind kind, cuda
         default:
             return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t read_and_clear_decode_error(int* flag) {
+    cudaError_t e = cudaMemcpyFromSymbol(flag, g_decode_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(int));
 }
 
 }  // namespace ssd

@@ -84,6 +84,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
 // Synchronises `st`, then reads and clears the tensor-core kernel's timeout flag.
 cudaError_t read_and_clear_tc_error(int* flag, cudaStream_t st);
 
+// Reads and clears the decode step's error word (nonzero: a state load never landed).  Does not
+// synchronise: call after the stream is idle.
+cudaError_t read_and_clear_decode_error(int* flag);
+
 namespace mimo {
 struct MimoArgs;
 // The MIMO decode step (ssd_mimo.cu); sizes and pointers validated by the caller.
