@@ -900,12 +900,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
 
 // SiLU(conv4) of the B and C channels into the workspace [row][2][G*N] (bf16),
 // and the conv_state output (pre-conv inputs of the last 3 tokens of every channel).
-// Blocks with blockIdx.x < ntok: 256 channel pairs (bf16x2) over kProTok rows each; a
-// thread issues all kProTok + 3 loads of its window before the first FMA.  Blocks with
+// Blocks with blockIdx.x < ntok: 256 channel pairs (bf16x2) over kProTok rows each; the
+// block stages its kProTok + 3 input rows in shared memory before the first FMA.  Blocks with
 // blockIdx.x >= ntok (and blockIdx.z == 0): the conv_state tail, one element per thread.
 // In a packed batch (a.cu) the window runs over all rows; taps that reach before the
 // start of a row's sequence take that sequence's initial conv state (or zero) instead.
-constexpr int kProTok = 16;
+constexpr int kProTok = 32;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
 
 // Pre-conv value of channel c at position t (< 3 tokens before the start) of sequence b's history.
 __device__ __forceinline__ __nv_bfloat16 conv_history(const PrefillArgs& a, int64_t b, int c, int64_t t) {
@@ -914,7 +924,7 @@ __device__ __forceinline__ __nv_bfloat16 conv_history(const PrefillArgs& a, int6
 }
 
 template <bool kVarlen>
-__global__ void __launch_bounds__(256, kVarlen ? 3 : 5) bc_prologue_kernel(PrefillArgs a, int ntok) {
+__global__ void __launch_bounds__(256, 5) bc_prologue_kernel(PrefillArgs a, int ntok, bool vec16) {
     // the chunk scan may start its launch now; it waits for this grid before reading the workspace
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if ((int)blockIdx.x >= ntok) {
@@ -942,7 +952,7 @@ __global__ void __launch_bounds__(256, kVarlen ? 3 : 5) bc_prologue_kernel(Prefi
     const int64_t t0 = (int64_t)blockIdx.x * kProTok;  // first row of the window within [0, L)
     // packed batch: the sequence of row t0 (the largest s with cu[s] <= t0; empty sequences are skipped),
     // searched once per block
-    __shared__ int64_t s_seq;
+    __shared__ int64_t s_seq[3];  // the sequence, its first row and the first row after it
     if constexpr (kVarlen) {
         if (threadIdx.x == 0) {
             int64_t lo = 0, hi = a.batch;
@@ -951,74 +961,117 @@ __global__ void __launch_bounds__(256, kVarlen ? 3 : 5) bc_prologue_kernel(Prefi
                 if (a.cu[mid] <= t0) lo = mid;
                 else hi = mid;
             }
-            s_seq = lo;
+            s_seq[0] = lo;
+            s_seq[1] = a.cu[lo];
+            s_seq[2] = a.cu[lo + 1];
         }
         __syncthreads();
     }
     const int half_gn = a.GN / 2;                    // channel pairs per array
     const int pair = blockIdx.z * 256 + threadIdx.x;  // 0 .. GN-1 over both arrays
-    if (pair >= a.GN) return;
     const int sel = pair >= half_gn;                // 0 = B, 1 = C
     const int cp = pair - sel * half_gn;            // pair index within the array
     const int cglob = a.HP + sel * a.GN + 2 * cp;   // conv channel of the pair's first element
     const int64_t rs = (sel ? a.rs_C : a.rs_B) / 2;  // row stride in channel pairs
     const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B) + (size_t)b * a.L * rs + cp;
     uint32_t* dst = static_cast<uint32_t*>(a.workspace) + ((size_t)b * a.L * 2 + sel) * half_gn + cp;
+    // The block's window (rows t0-3 .. t0+kProTok-1 of its 256 pairs, the rows inside [0, L)) lands in
+    // shared memory by cp.async, so the loads in flight hold no registers: 16-byte pieces (4 pairs) where
+    // B and C allow it, else 4-byte ones.
+    __shared__ __align__(16) uint32_t s_win[kProTok + 3][256];
+    if (vec16) {
+        const int64_t row0 = b * a.L + t0 - 3;
+        for (int q = threadIdx.x; q < (kProTok + 3) * 64; q += 256) {
+            const int k = q >> 6, c4 = (q & 63) * 4;
+            const int gp = blockIdx.z * 256 + c4;  // first pair of the piece; a piece never spans B and C
+            const int64_t t = t0 - 3 + k;
+            if (gp < a.GN && t >= 0 && t < a.L) {
+                const int gsel = gp >= half_gn;
+                const int64_t grs = (gsel ? a.rs_C : a.rs_B) / 2;
+                const uint32_t* g =
+                    static_cast<const uint32_t*>(gsel ? a.C : a.B) + (size_t)(row0 + k) * grs + (gp - gsel * half_gn);
+                cp_async16(&s_win[k][c4], g);
+            }
+        }
+    } else if (pair < a.GN) {
+#pragma unroll
+        for (int k = 0; k < kProTok + 3; ++k) {
+            const int64_t t = t0 - 3 + k;
+            if (t >= 0 && t < a.L) cp_async4(&s_win[k][threadIdx.x], src + (size_t)t * rs);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    if (pair >= a.GN) return;
     const float4 w0 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)cglob * 4);
     const float4 w1 = *reinterpret_cast<const float4*>(a.conv_w + (size_t)(cglob + 1) * 4);
     const float2 bias = make_float2(a.conv_b[cglob], a.conv_b[cglob + 1]);
-    float2 v[kProTok + 3];  // rows t0-3 .. t0+kProTok-1, channels (2cp, 2cp+1)
-    uint32_t raw[kProTok + 3];
+    // Interior windows (all rows inside [0, L) and, in a packed batch, inside one sequence): no per-row
+    // checks and no history taps; the last three rows slide along in registers.
+    bool interior = t0 >= 3 && t0 + kProTok <= a.L;
+    if constexpr (kVarlen) interior = interior && s_seq[1] <= t0 - 3 && t0 + kProTok <= s_seq[2];
+    if (interior) {
+        uint32_t* q = dst + (size_t)t0 * 2 * half_gn;
+        const int qs = 2 * half_gn;  // workspace row stride in channel pairs
+        uint32_t r = s_win[0][threadIdx.x];
+        float2 x0 = make_float2(bf_lo(r), bf_hi(r));
+        r = s_win[1][threadIdx.x];
+        float2 x1 = make_float2(bf_lo(r), bf_hi(r));
+        r = s_win[2][threadIdx.x];
+        float2 x2 = make_float2(bf_lo(r), bf_hi(r));
 #pragma unroll
-    for (int k = 0; k < kProTok + 3; ++k) {
-        const int64_t t = t0 - 3 + k;
-        raw[k] = (t >= 0 && t < a.L) ? src[(size_t)t * rs] : 0u;
+        for (int k = 0; k < kProTok; ++k) {
+            r = s_win[k + 3][threadIdx.x];
+            const float2 x3 = make_float2(bf_lo(r), bf_hi(r));
+            float2 acc = bias;
+            acc = __ffma2_rn(make_float2(w0.x, w1.x), x0, acc);
+            acc = __ffma2_rn(make_float2(w0.y, w1.y), x1, acc);
+            acc = __ffma2_rn(make_float2(w0.z, w1.z), x2, acc);
+            acc = __ffma2_rn(make_float2(w0.w, w1.w), x3, acc);
+            const float2 u = silu2(acc);
+            q[k * qs] = pack_bf2(u.x, u.y);
+            x0 = x1;
+            x1 = x2;
+            x2 = x3;
+        }
+        return;
     }
-    // packed batch: the sequence of row t0 and where the next one starts
-    int64_t seq = 0, start = 0, next = a.L;
+    // Edge windows (the first rows of a batch row or of a sequence, or a window past L): one row at a
+    // time; a tap before the start of the row's sequence reads that sequence's conv history.
+    int64_t seq = b, start = 0, next = a.L;
     if constexpr (kVarlen) {
-        seq = s_seq;
-        start = a.cu[seq];
-        next = a.cu[seq + 1];
+        seq = s_seq[0];
+        start = s_seq[1];
+        next = s_seq[2];
     }
-#pragma unroll
-    for (int k = 0; k < kProTok + 3; ++k) {
-        const int64_t t = t0 - 3 + k;
-        if (!kVarlen && t < 0)
-            v[k] = make_float2(__bfloat162float(conv_history(a, b, cglob, t)),
-                               __bfloat162float(conv_history(a, b, cglob + 1, t)));
-        else
-            v[k] = make_float2(bf_lo(raw[k]), bf_hi(raw[k]));
-    }
-#pragma unroll
+    const float wt0[4] = {w0.x, w0.y, w0.z, w0.w}, wt1[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll 1
     for (int k = 0; k < kProTok; ++k) {
         const int64_t t = t0 + k;
-        if (t < a.L) {
-            float2 x4[4] = {v[k], v[k + 1], v[k + 2], v[k + 3]};
-            if constexpr (kVarlen) {
-                while (t >= next && seq + 1 < a.batch) {  // row t opens a later sequence
-                    ++seq;
-                    start = next;
-                    next = a.cu[seq + 1];
-                }
-                if (start <= t && t - 3 < start) {  // within 3 rows of its sequence's start: taps before it are history
-#pragma unroll
-                    for (int j = 0; j < 3; ++j) {
-                        const int64_t tt = t - 3 + j;
-                        if (tt < start)
-                            x4[j] = make_float2(__bfloat162float(conv_history(a, seq, cglob, tt - start)),
-                                                __bfloat162float(conv_history(a, seq, cglob + 1, tt - start)));
-                    }
-                }
+        if (t >= a.L) break;
+        if constexpr (kVarlen) {
+            while (t >= next && seq + 1 < a.batch) {  // row t opens a later sequence
+                ++seq;
+                start = next;
+                next = a.cu[seq + 1];
             }
-            float2 p = bias;
-            p = __ffma2_rn(make_float2(w0.x, w1.x), x4[0], p);
-            p = __ffma2_rn(make_float2(w0.y, w1.y), x4[1], p);
-            p = __ffma2_rn(make_float2(w0.z, w1.z), x4[2], p);
-            p = __ffma2_rn(make_float2(w0.w, w1.w), x4[3], p);
-            const float2 u = silu2(p);
-            dst[(size_t)t * 2 * half_gn] = pack_bf2(u.x, u.y);
         }
+        float2 acc = bias;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t tt = t - 3 + j;  // window row k + j
+            float2 x;
+            if (tt >= start) {
+                const uint32_t r = s_win[k + j][threadIdx.x];
+                x = make_float2(bf_lo(r), bf_hi(r));
+            } else {
+                x = make_float2(__bfloat162float(conv_history(a, seq, cglob, tt - start)),
+                                __bfloat162float(conv_history(a, seq, cglob + 1, tt - start)));
+            }
+            acc = __ffma2_rn(make_float2(wt0[j], wt1[j]), x, acc);
+        }
+        const float2 u = silu2(acc);
+        dst[(size_t)t * 2 * half_gn] = pack_bf2(u.x, u.y);
     }
 }
 
@@ -1094,8 +1147,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     const int64_t tail = a.batch * (int64_t)a.conv_dim * 3;
     const int tail_blocks = (int)((tail + 256 * mbatch - 1) / (256 * mbatch));
     const dim3 pgrid((unsigned)(ntok + tail_blocks), (unsigned)mbatch, (unsigned)((a.GN + 255) / 256));
-    if (a.cu) bc_prologue_kernel<true><<<pgrid, 256, 0, st>>>(a, ntok);
-    else bc_prologue_kernel<false><<<pgrid, 256, 0, st>>>(a, ntok);
+    // 16-byte window pieces: B and C 16-byte aligned, rows a multiple of 8 elements apart, and every
+    // array a multiple of 4 channel pairs wide (a piece of 4 pairs then never spans B and C)
+    const bool vec16 = reinterpret_cast<uintptr_t>(a.B) % 16 == 0 && reinterpret_cast<uintptr_t>(a.C) % 16 == 0 &&
+                       a.rs_B % 8 == 0 && a.rs_C % 8 == 0 && (a.GN / 2) % 4 == 0;
+    if (a.cu) bc_prologue_kernel<true><<<pgrid, 256, 0, st>>>(a, ntok, vec16);
+    else bc_prologue_kernel<false><<<pgrid, 256, 0, st>>>(a, ntok, vec16);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     auto kern = kind == ActKind::BF16_YF32 ? (a.cu ? chunk_scan_kernel<float, true> : chunk_scan_kernel<float, false>)
