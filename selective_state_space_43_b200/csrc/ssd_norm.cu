@@ -16,14 +16,16 @@
 namespace ssd {
 namespace {
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void unpack8(const uint4 w, float (&v)[8]) {
     const uint32_t r[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         v[2 * k] = __uint_as_float(r[k] << 16);
         v[2 * k + 1] = __uint_as_float(r[k] & 0xFFFF0000u);
     }
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    unpack8(*reinterpret_cast<const uint4*>(p), v);
 }
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
     const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
@@ -43,8 +45,9 @@ __device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
     reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-// Groups of up to kCache * 256 channels are read once and kept in registers; larger groups are read
-// twice (the second time from L2).
+// Groups of up to kCache * 256 channels are read once and kept in registers (bf16 as the packed words
+// loaded, unpacked twice, so that a thread holds 16 registers of data and more warps fit an SM); larger
+// groups are read twice (the second time from L2).
 constexpr int kCache = 4;
 
 template <typename T>
@@ -58,21 +61,31 @@ __global__ void __launch_bounds__(256) group_rmsnorm_kernel(int64_t units, int c
     const int c0 = (int)(u % ngroups) * group;
     const T* src = in + (size_t)row * channels + c0;
     T* dst = out + (size_t)row * channels + c0;
+    constexpr bool kPacked = sizeof(T) == 2;
     const bool cached = group <= kCache * 256;
-    float v[kCache][8];
+    uint4 raw[kPacked ? kCache : 1];
+    float v[kPacked ? 1 : kCache][8];
     float ss = 0.f;
     if (cached) {
 #pragma unroll
         for (int it = 0; it < kCache; ++it) {
             const int c = lane * 8 + it * 256;
-            if (c < group) load8(src + c, v[it]);
+            if (c < group) {
+                if constexpr (kPacked) raw[it] = *reinterpret_cast<const uint4*>(src + c);
+                else load8(src + c, v[it]);
+            }
         }
 #pragma unroll
         for (int it = 0; it < kCache; ++it) {
             const int c = lane * 8 + it * 256;
             if (c < group) {
+                float t[8];
+                if constexpr (kPacked) unpack8(raw[it], t);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) ss = fmaf(v[it][k], v[it][k], ss);
+                for (int k = 0; k < 8; ++k) {
+                    const float x = kPacked ? t[k] : v[kPacked ? 0 : it][k];
+                    ss = fmaf(x, x, ss);
+                }
             }
         }
     } else {
@@ -98,7 +111,15 @@ __global__ void __launch_bounds__(256) group_rmsnorm_kernel(int64_t units, int c
 #pragma unroll
         for (int it = 0; it < kCache; ++it) {
             const int c = lane * 8 + it * 256;
-            if (c < group) scale_store(c, v[it]);
+            if (c < group) {
+                if constexpr (kPacked) {
+                    float t[8];
+                    unpack8(raw[it], t);
+                    scale_store(c, t);
+                } else {
+                    scale_store(c, v[kPacked ? 0 : it]);
+                }
+            }
         }
     } else {
         for (int c = lane * 8; c < group; c += 256) {
