@@ -757,22 +757,27 @@ def bench_decode(ops, dev, world: int, sampler, peaks, nsteps: int):
         dstep(steps[i % len(steps)])
     torch.cuda.synchronize(dev)
     KD = len(steps)
-    ds = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
-    de = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
-    dks = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
-    dke = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+    # the steps back to back between one pair of events (an event between two steps would keep the next
+    # step's state kernel from starting under the previous step's roll, as it does in a decode loop)
+    ds, de = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     sampler.load(True)
+    ds.record()
     for k in range(KD):
-        ops.set_timing_events(dks[k], dke[k])
-        ds[k].record()
         dstep(steps[k])
-        de[k].record()
+    de.record()
     torch.cuda.synchronize(dev)
     sampler.load(False)
     barrier(world)
+    dms = max_over_ranks(ds.elapsed_time(de) / KD, world, dev)
+    # the state kernel alone: a second pass with events around each of its launches
+    dks = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+    dke = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+    for k in range(KD):
+        ops.set_timing_events(dks[k], dke[k])
+        dstep(steps[k])
+    torch.cuda.synchronize(dev)
     ops.set_timing_events(None, None)
-    dms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(ds, de)) / KD, world, dev)
     dkms = sum(a.elapsed_time(b) for a, b in zip(dks, dke)) / KD
     tot_b, kern_b = decode_bytes(dd, 2 if wd["dtype"] == torch.bfloat16 else 4)
     gbs = tot_b * world / (dms * 1e-3) / 1e9

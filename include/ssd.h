@@ -171,7 +171,16 @@ SSD_API ssd_status ssd_prefill_strided(const ssd_dims* dims, ssd_dtype dtype, co
  *   ssm_state   [batch][H][P][N] fp32, in/out, updated in place
  *   y           [batch][H*P]   dtype, fp32 for SSD_BF16_YF32 (out)
  * Two launches: the state stream (all heads) and the roll of the shared B/C
- * conv channels, which must follow every head's read of them.
+ * conv channels, which must follow every head's read of them.  Both are
+ * programmatic dependent launches (CUDA's programmatic stream serialization):
+ * the state kernel issues its ssm_state load before it waits for the kernel
+ * ahead of it in the stream, and reads everything else after.  So a kernel
+ * that precedes this call on the stream and lets its dependents start early
+ * (griddepcontrol.launch_dependents) must not write ssm_state after doing so;
+ * kernels that do not, copies and events order the call as usual.  In this
+ * library only the two decode kernels and the prefill's first kernel (always
+ * followed by the prefill's own scan) let dependents start early.  Back-to-back
+ * decode steps overlap the next step's state load with the previous roll.
  */
 SSD_API ssd_status ssd_decode_step(const ssd_dims* dims, ssd_dtype dtype, const ssd_params* params,
                            const void* x, const void* dt, const void* B, const void* C, const void* z,

@@ -18,7 +18,13 @@
 //     (reported by ssd_device_status as SSD_ERR_TIMEOUT) and writes no state;
 //   * y = S.C is a segmented warp reduction over the N/4 lanes of a row;
 //   * the shared B/C conv channels are rolled by a second, tiny kernel that
-//     runs after every head has read the old window.
+//     runs after every head has read the old window;
+//   * both kernels are programmatic dependents of the kernel before them: the
+//     roll waits for the state kernel's grid before it touches the windows, and
+//     lets the next step's state kernel start, whose state load (written by the
+//     previous state kernel, complete once the roll has passed its wait) then
+//     overlaps the roll; that kernel waits for the roll before reading the B/C
+//     windows.
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
 #include "ssd_sm100.cuh"
@@ -64,6 +70,10 @@ __global__ void __launch_bounds__(256, kDecodeCtas) decode_state_kernel(DecodeAr
         sm100::mbar_arrive_expect_tx(bar, kStateBytes);
         sm100::bulk_load(s_st, gstate, kStateBytes, bar);
     }
+    // the roll of the previous step may launch now (it waits for this grid), and this grid reads the conv
+    // windows only once the kernel before it (that roll, when it is) has completed
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     for (int i = tid; i < P + 2 * N; i += 256) {
         int c;
@@ -140,6 +150,10 @@ __global__ void __launch_bounds__(256, kDecodeCtas) decode_state_kernel(DecodeAr
 // Roll the 2*G*N shared B/C conv channels by one token (after every head read them).
 template <typename T>
 __global__ void __launch_bounds__(256) decode_roll_bc_kernel(DecodeArgs a, int64_t total) {
+    // every head has read the old window once the state kernel's grid is complete; the next step's state
+    // kernel may then start (its state load no longer races the state kernel that wrote it)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= total) return;
     const int two_gn = 2 * a.GN;
@@ -153,13 +167,36 @@ __global__ void __launch_bounds__(256) decode_roll_bc_kernel(DecodeArgs a, int64
     cs[2] = xin;
 }
 
+// A launch that may start before the kernel ahead of it in the stream completes (that kernel allows it
+// with griddepcontrol.launch_dependents; this one waits for it with griddepcontrol.wait).
+template <typename... Params, typename... Args>
+static cudaError_t launch_dependent(void (*kern)(Params...), unsigned grid, size_t smem, cudaStream_t st,
+                                    Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <typename T, typename TY, int N>
 static cudaError_t launch_decode_t(const DecodeArgs& a, int64_t batch, cudaStream_t st, const TimingHook& hook) {
     hook.before(st);
-    decode_state_kernel<T, TY, N><<<(unsigned)(batch * a.H), 256, decode_smem_bytes(64, N), st>>>(a);
+    cudaError_t e = launch_dependent(decode_state_kernel<T, TY, N>, (unsigned)(batch * a.H), decode_smem_bytes(64, N),
+                                     st, a);
+    if (e != cudaSuccess) return e;
     hook.after(st);
     const int64_t total = batch * 2 * a.GN;
-    if (total > 0) decode_roll_bc_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(a, total);
+    if (total > 0) {
+        e = launch_dependent(decode_roll_bc_kernel<T>, (unsigned)((total + 255) / 256), 0, st, a, total);
+        if (e != cudaSuccess) return e;
+    }
     return cudaGetLastError();
 }
 
