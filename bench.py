@@ -229,18 +229,18 @@ def bench_mimo(ops, d: Dims, act, dev, world: int, sampler, peaks, nsteps: int):
     for i in range(3):
         mstep(i)
     torch.cuda.synchronize(dev)
-    ms_ = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
-    me = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+    # the steps back to back between one pair of events, as a decode loop runs them
+    ms_, me = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     sampler.load(True)
+    ms_.record()
     for k in range(nsteps):
-        ms_[k].record()
         mstep(k)
-        me[k].record()
+    me.record()
     torch.cuda.synchronize(dev)
     sampler.load(False)
     barrier(world)
-    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(ms_, me)) / nsteps, world, dev)
+    ms = max_over_ranks(ms_.elapsed_time(me) / nsteps, world, dev)
     nbytes = mimo_decode_bytes(d, MIMO_RANK, 2 if act == torch.bfloat16 else 4)
     gbs = nbytes / (ms * 1e-3) / 1e9
     flops = 4 * MIMO_RANK * d.batch * d.nheads * d.headdim * d.d_state

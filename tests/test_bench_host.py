@@ -149,7 +149,9 @@ def test_backward_and_mimo_bench_legs_on_a_fake_device(monkeypatch):
     assert abs(rf["achieved"] - bench.backward_chunk_bytes(d, 2) / 2e-3 / 1e9) < 1e-6
     m = bench.bench_mimo(fake, d, torch.bfloat16, torch.device("cpu"), 1, _FakeSampler(), peaks, 4)
     assert fake.calls["mimo"] == 3 + 4
-    assert abs(m["value"] - bench.mimo_decode_bytes(d, bench.MIMO_RANK, 2) / 2e-3 / 1e9) < 1e-6
+    # the 4 timed steps run back to back between one pair of events (2 ms on the fake clock)
+    assert m["ms_per_step"] == 2.0 / 4
+    assert abs(m["value"] - bench.mimo_decode_bytes(d, bench.MIMO_RANK, 2) / 0.5e-3 / 1e9) < 1e-6
     assert m["roofline"]["frac"] == m["roofline"]["achieved"] / 6554.6
 
 
