@@ -874,7 +874,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_scan_kernel(const __grid_co
         bool ok = nc == 0 || conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, 0, nc, Ls, i, half);
         if (!ok) raise_abort(abort_flag);
         for (int c = 0; c < nc && ok; ++c) {
-            const int buf = c & 1;
             // (c) the next chunk's x conv first: this chunk's S_c (needed below) completes meanwhile
             if (c + 1 < nc && !conv_chunk(a, sm, bars, abort_flag, tmem, lane_base, c + 1, nc, Ls, i, half)) {
                 raise_abort(abort_flag);
@@ -910,9 +909,6 @@ constexpr int kProTok = 32;
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
 }
@@ -924,7 +920,7 @@ __device__ __forceinline__ __nv_bfloat16 conv_history(const PrefillArgs& a, int6
 }
 
 template <bool kVarlen>
-__global__ void __launch_bounds__(256, 5) bc_prologue_kernel(PrefillArgs a, int ntok, bool vec16) {
+__global__ void __launch_bounds__(256, 5) bc_prologue_kernel(PrefillArgs a, int ntok) {
     // the chunk scan may start its launch now; it waits for this grid before reading the workspace
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if ((int)blockIdx.x >= ntok) {
@@ -972,18 +968,17 @@ __global__ void __launch_bounds__(256, 5) bc_prologue_kernel(PrefillArgs a, int 
     const int sel = pair >= half_gn;                // 0 = B, 1 = C
     const int cp = pair - sel * half_gn;            // pair index within the array
     const int cglob = a.HP + sel * a.GN + 2 * cp;   // conv channel of the pair's first element
-    const int64_t rs = (sel ? a.rs_C : a.rs_B) / 2;  // row stride in channel pairs
-    const uint32_t* src = static_cast<const uint32_t*>(sel ? a.C : a.B) + (size_t)b * a.L * rs + cp;
     uint32_t* dst = static_cast<uint32_t*>(a.workspace) + ((size_t)b * a.L * 2 + sel) * half_gn + cp;
     // The block's window (rows t0-3 .. t0+kProTok-1 of its 256 pairs, the rows inside [0, L)) lands in
-    // shared memory by cp.async, so the loads in flight hold no registers: 16-byte pieces (4 pairs) where
-    // B and C allow it, else 4-byte ones.
+    // shared memory by 16-byte cp.async pieces (4 pairs each), so the loads in flight hold no registers.
+    // The entry points guarantee the alignment: B and C 16-byte aligned, rows a multiple of 16 bytes apart,
+    // and every array a multiple of 4 channel pairs wide (so a piece never spans B and C).
     __shared__ __align__(16) uint32_t s_win[kProTok + 3][256];
-    if (vec16) {
+    {
         const int64_t row0 = b * a.L + t0 - 3;
         for (int q = threadIdx.x; q < (kProTok + 3) * 64; q += 256) {
             const int k = q >> 6, c4 = (q & 63) * 4;
-            const int gp = blockIdx.z * 256 + c4;  // first pair of the piece; a piece never spans B and C
+            const int gp = blockIdx.z * 256 + c4;  // first pair of the piece
             const int64_t t = t0 - 3 + k;
             if (gp < a.GN && t >= 0 && t < a.L) {
                 const int gsel = gp >= half_gn;
@@ -992,12 +987,6 @@ __global__ void __launch_bounds__(256, 5) bc_prologue_kernel(PrefillArgs a, int 
                     static_cast<const uint32_t*>(gsel ? a.C : a.B) + (size_t)(row0 + k) * grs + (gp - gsel * half_gn);
                 cp_async16(&s_win[k][c4], g);
             }
-        }
-    } else if (pair < a.GN) {
-#pragma unroll
-        for (int k = 0; k < kProTok + 3; ++k) {
-            const int64_t t = t0 - 3 + k;
-            if (t >= 0 && t < a.L) cp_async4(&s_win[k][threadIdx.x], src + (size_t)t * rs);
         }
     }
     cp_async_wait_all();
@@ -1147,12 +1136,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, ActKind kind, cudaStream_t s
     const int64_t tail = a.batch * (int64_t)a.conv_dim * 3;
     const int tail_blocks = (int)((tail + 256 * mbatch - 1) / (256 * mbatch));
     const dim3 pgrid((unsigned)(ntok + tail_blocks), (unsigned)mbatch, (unsigned)((a.GN + 255) / 256));
-    // 16-byte window pieces: B and C 16-byte aligned, rows a multiple of 8 elements apart, and every
-    // array a multiple of 4 channel pairs wide (a piece of 4 pairs then never spans B and C)
-    const bool vec16 = reinterpret_cast<uintptr_t>(a.B) % 16 == 0 && reinterpret_cast<uintptr_t>(a.C) % 16 == 0 &&
-                       a.rs_B % 8 == 0 && a.rs_C % 8 == 0 && (a.GN / 2) % 4 == 0;
-    if (a.cu) bc_prologue_kernel<true><<<pgrid, 256, 0, st>>>(a, ntok, vec16);
-    else bc_prologue_kernel<false><<<pgrid, 256, 0, st>>>(a, ntok, vec16);
+    // the prologue's 16-byte window pieces (the entry points check the pointers and strides already)
+    if (reinterpret_cast<uintptr_t>(a.B) % 16 != 0 || reinterpret_cast<uintptr_t>(a.C) % 16 != 0 || a.rs_B % 8 != 0 ||
+        a.rs_C % 8 != 0 || (a.GN / 2) % 4 != 0)
+        return cudaErrorInvalidValue;
+    if (a.cu) bc_prologue_kernel<true><<<pgrid, 256, 0, st>>>(a, ntok);
+    else bc_prologue_kernel<false><<<pgrid, 256, 0, st>>>(a, ntok);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     auto kern = kind == ActKind::BF16_YF32 ? (a.cu ? chunk_scan_kernel<float, true> : chunk_scan_kernel<float, false>)
